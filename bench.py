@@ -1,0 +1,405 @@
+"""Benchmark of the DeepSeekMoE layer forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl ours|reference]
+
+A step is one whole layer forward (routing, permutation, both grouped GEMMs,
+combine) over one batch of T synthetic tokens, through the C ABI
+(moe_forward), inputs resident in HBM.  Under torchrun each rank runs its own
+replica on its own GPU with its own batch (no collective on the data path:
+the layer is data-parallel over tokens), so scaling is weak and the value is
+the tokens of all ranks over the slowest rank's time.
+
+Prints one JSON line (rank 0).  `--impl reference` times the fp64 CPU oracle
+on the host cores instead, on a bounded token sample per step.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+DEFAULT_CONFIG = "v3_bf16"
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": p["hbm_gbs"], "bf16_tflops": p["bf16_tflops"],
+                "bf16_tflops_sustained": p.get("bf16_tflops_sustained", p["bf16_tflops"]),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+def workload_name(cfg):
+    gate = "sigmoid+bias" if cfg.bias_half_range is not None else cfg.gate
+    return (f"DeepSeekMoE layer forward ({cfg.name}): T={cfg.T} d={cfg.d} "
+            f"{cfg.n_shared} shared + {cfg.n_routed} routed SwiGLU experts of width {cfg.inter}, "
+            f"top-{cfg.top_k}, {gate}, groups {cfg.n_group}/{cfg.topk_group}, "
+            f"{'renorm x' + str(cfg.route_scale) if cfg.renorm else 'no renorm'}, {cfg.dtype}")
+
+
+def config_dict(cfg, n):
+    return {"workload": workload_name(cfg), "T": cfg.T, "d": cfg.d, "n_shared": cfg.n_shared,
+            "n_routed": cfg.n_routed, "top_k": cfg.top_k, "inter": cfg.inter, "gate": cfg.gate,
+            "n_group": cfg.n_group, "topk_group": cfg.topk_group, "renorm": cfg.renorm,
+            "route_scale": cfg.route_scale, "tokens_per_gpu": cfg.T,
+            "global_tokens": cfg.T * n,
+            "parallelism": f"token batches, one replica per GPU x{n}",
+            "l2": "inputs larger than L2 (expert weights and x exceed the 126 MB L2)"}
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples of this GPU's clocks while the timed region runs."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax = float(parts[1])
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- CPU oracle leg
+class OracleSample:
+    """The fp64 oracle on a bounded token sample of the workload (CPU baseline).
+
+    One step routes `S` sampled tokens and evaluates their layer output with
+    the oracle as it stands.  Expert weights are regenerated once (synthetic
+    input generation, not timed) and kept as stored bf16/fp32 values; the
+    oracle's widening to float64 is part of the timed work."""
+
+    def __init__(self, cfg, n_tokens: int, zipf_offsets=None):
+        import numpy as np
+
+        from synth import recipes
+        self.np = np
+        self.cfg = cfg
+        T = cfg.T
+        self.tokens = [int(i * T // n_tokens) for i in range(n_tokens)]
+        self.x = recipes.host_x(cfg, rows=self.tokens)
+        self.w_r = recipes.host_router(cfg, zipf_offsets)
+        self.bias = recipes.host_bias(cfg)
+        # experts the sample touches (by the oracle's own routing), bits kept resident
+        from oracle import moe_oracle as mo
+        r = mo.route(self.x, self.w_r, self.bias, gate=cfg.gate, top_k=cfg.top_k,
+                     n_group=cfg.n_group, topk_group=cfg.topk_group, renorm=cfg.renorm,
+                     route_scale=cfg.route_scale)
+        need = set(range(cfg.n_shared)) | {cfg.n_shared + int(j) for j in np.unique(r["idx"])}
+        self.bits = {e: recipes.host_expert_bits(cfg, e) for e in sorted(need)}
+
+    def _expert(self, e):
+        np = self.np
+        gu, dn = self.bits[e]
+        I = self.cfg.inter
+        if gu.dtype == np.uint16:
+            from synth import bf16_bits_to_f64
+            gu64, dn64 = bf16_bits_to_f64(gu), bf16_bits_to_f64(dn)
+        else:
+            gu64, dn64 = gu.astype(np.float64), dn.astype(np.float64)
+        return gu64[:I], gu64[I:], dn64
+
+    def step(self):
+        from oracle import moe_oracle as mo
+        c = self.cfg
+        t0 = time.perf_counter()
+        mo.moe_forward(self.x, self.w_r, self.bias, self._expert, n_shared=c.n_shared,
+                       gate=c.gate, top_k=c.top_k, n_group=c.n_group, topk_group=c.topk_group,
+                       renorm=c.renorm, route_scale=c.route_scale)
+        return time.perf_counter() - t0
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def oracle_sample_size(cfg):
+    # keep one step to a few seconds of host work
+    work = cfg.d * cfg.inter * (cfg.top_k + cfg.n_shared)
+    return max(1, min(64, int(2e9 // max(work * 40, 1))))
+
+
+def run_reference(args, cfg):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    S = oracle_sample_size(cfg)
+    samp = OracleSample(cfg, S, load_zipf(cfg))
+    for _ in range(args.warmup):
+        samp.step()
+    times = [samp.step() for _ in range(args.steps)]
+    total = sum(times)
+    value = S * args.steps / total
+    cores = blas_threads()
+    line = {"impl": "reference", "metric": "MoE-layer tokens/s", "value": value,
+            "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": config_dict(cfg, 1),
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores,
+                             "kind": "oracle",
+                             "sample": f"{S} tokens per step (strided over T={cfg.T}), "
+                                       f"routing + all expert FFNs in fp64"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def load_zipf(cfg):
+    if not cfg.zipf:
+        return None
+    import numpy as np
+    path = os.path.join(ROOT, "tests", "golden", f"zipf_offsets_{cfg.name.split('@')[0]}.txt")
+    return np.loadtxt(path, dtype=np.float64)
+
+
+# ----------------------------------------------------------------------------- GPU leg
+def run_ours(args, cfg):
+    import torch
+    import torch.distributed as dist
+
+    import forward_moe_route_b200 as moe
+    from synth import recipes
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    desc = moe.desc_from_config(cfg)
+    inp = recipes.device_inputs(cfg, "cuda", load_zipf(cfg))
+    if cfg.dtype == "e4m3":
+        raise SystemExit("the FP8 layer is not wired into the bench yet")
+    ws = moe.workspace(desc)
+    h = torch.empty(cfg.T, cfg.d, dtype=inp["x"].dtype, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step(x=None):
+        moe.moe_forward(desc, inp["x"] if x is None else x, None, inp["w_r"], inp["bias"],
+                        inp["w_gu"], None, inp["w_down"], None, h, None, None, ws, stream)
+
+    for _ in range(args.warmup):
+        step()
+    st = moe.moe_last_device_status()
+    if st != moe.OK:
+        raise SystemExit(f"device status after warm-up: {moe.moe_status_string(st)}")
+
+    # ---- timed region: K steps, events on the launching stream
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    clocks = ClockSampler(int(os.environ.get("CUDA_VISIBLE_DEVICES", str(local)).split(",")[0])
+                          if os.environ.get("CUDA_VISIBLE_DEVICES", "").replace(",", "").isdigit()
+                          else local)
+    barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for i in range(args.steps):
+        moe.moe_trace_events(ev[i])
+        step()
+    moe.moe_trace_events(None)
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    st = moe.moe_last_device_status()
+    if st != moe.OK:
+        raise SystemExit(f"device status after the timed region: {moe.moe_status_string(st)}")
+    ms = t_start.elapsed_time(t_end)
+    stages = {"route": [], "permute": [], "gemm1_swiglu": [], "gemm2_scatter": [],
+              "combine": []}
+    for e in ev:
+        stages["route"].append(e[0].elapsed_time(e[1]))
+        stages["permute"].append(e[1].elapsed_time(e[2]))
+        stages["gemm1_swiglu"].append(e[2].elapsed_time(e[3]))
+        stages["gemm2_scatter"].append(e[3].elapsed_time(e[4]))
+        stages["combine"].append(e[4].elapsed_time(e[5]))
+    stage_ms = {k: sum(v) / len(v) for k, v in stages.items()}
+    if world > 1:
+        t = torch.tensor([ms], device="cuda", dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+
+    # ---- end to end through the public API: pinned host x in, h back out, every step
+    x_host = inp["x"].cpu().pin_memory()
+    h_host = torch.empty(h.shape, dtype=h.dtype).pin_memory()
+    x_dev = torch.empty_like(inp["x"])
+    for _ in range(2):
+        x_dev.copy_(x_host, non_blocking=True)
+        step(x_dev)
+        h_host.copy_(h, non_blocking=True)
+    barrier()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e2e_steps = max(3, min(args.steps, 10))
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        x_dev.copy_(x_host, non_blocking=True)
+        step(x_dev)
+        h_host.copy_(h, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    if world > 1:
+        t = torch.tensor([e2e_ms], device="cuda", dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+
+    ms_step = ms / args.steps
+    tokens_s = cfg.T * world / (ms_step * 1e-3)
+    pk = peaks()
+    gemm_flops = cfg.expert_gemm_flops()
+    g1 = stage_ms["gemm1_swiglu"] * 1e-3
+    g2 = stage_ms["gemm2_scatter"] * 1e-3
+    gemm_tflops = gemm_flops / (g1 + g2) / 1e12
+    g1_tflops = gemm_flops * 2 / 3 / g1 / 1e12
+    peak = pk["bf16_tflops_sustained"] if cfg.dtype != "f32" else pk["bf16_tflops_sustained"] / 2
+    out = None
+    if rank == 0:
+        route_bytes = (cfg.T * cfg.d * 2 + cfg.n_routed * cfg.d * 2 + cfg.T * cfg.n_routed * 4 * 2)
+        perm_bytes = cfg.T * cfg.d * 2 + cfg.rows_routed * cfg.d * 2
+        comb_bytes = cfg.T * (cfg.top_k + cfg.n_shared) * cfg.d * 2 + 2 * cfg.T * cfg.d * 2
+        rpc_ms = stage_ms["route"] + stage_ms["permute"] + stage_ms["combine"]
+        rpc_gbs = (route_bytes + perm_bytes + comb_bytes) / (rpc_ms * 1e-3) / 1e9
+        out = {
+            "metric": "MoE-layer tokens/s", "value": tokens_s, "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": cfg.dtype, "data": "synthetic",
+            "config": config_dict(cfg, world),
+            "grouped_gemm_tflops": gemm_tflops,
+            "grouped_gemm_frac_of_bf16_peak": {
+                "measured_sustained": gemm_tflops / pk["bf16_tflops_sustained"],
+                "measured_burst": gemm_tflops / pk["bf16_tflops"],
+                "spec_2250": gemm_tflops / 2250.0},
+            "stages_ms": stage_ms,
+            "route_permute_combine_gbs": rpc_gbs,
+            "route_permute_combine_frac_of_hbm": rpc_gbs / pk["hbm_gbs"],
+            "roofline": {"kernel": "grouped GEMM 1 (gate/up + SwiGLU epilogue)",
+                         "bound": "tensor", "achieved": g1_tflops, "peak": peak,
+                         "unit": "TFLOP/s", "frac": g1_tflops / peak, "traffic": None,
+                         "peak_source": f"{pk['source']} bf16 sustained"},
+            "roofline_gemm2": {"kernel": "grouped GEMM 2 (down + weighted scatter)",
+                               "bound": "tensor",
+                               "achieved": gemm_flops / 3 / g2 / 1e12, "peak": peak,
+                               "unit": "TFLOP/s", "frac": gemm_flops / 3 / g2 / 1e12 / peak},
+            "e2e": {"value": cfg.T * world / (e2e_ms * 1e-3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": x_host.numel() * x_host.element_size(),
+                    "d2h_bytes_per_step": h_host.numel() * h_host.element_size()},
+            "gpu_launches": moe.moe_forward_launch_count(desc) * args.steps,
+            "clocks": clk,
+        }
+    if world > 1:
+        dist.destroy_process_group()
+    return out
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default=DEFAULT_CONFIG)
+    ap.add_argument("--T", type=int, default=None, help="override the token count")
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    from synth import recipes
+    cfg = recipes.CONFIGS[args.config]
+    if args.T is not None:
+        cfg = cfg.with_T(args.T)
+    if args.impl == "reference":
+        return run_reference(args, cfg)
+    out = run_ours(args, cfg)
+    if out is not None:
+        if not args.no_cpu_baseline and args.gpus == 1:
+            S = oracle_sample_size(cfg)
+            samp = OracleSample(cfg, S, load_zipf(cfg))
+            samp.step()
+            t = [samp.step() for _ in range(2)]
+            v = S * len(t) / sum(t)
+            out["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": blas_threads(),
+                                   "kind": "oracle",
+                                   "sample": f"{S} tokens (strided over T={cfg.T}), routing + "
+                                             f"all expert FFNs in fp64, 2 timed steps"}
+        print(json.dumps(out), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

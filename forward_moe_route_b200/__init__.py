@@ -1,0 +1,201 @@
+"""Python binding of the B200 DeepSeekMoE layer-forward library (libmoe_b200.so).
+
+Argument marshalling only: every function here forwards torch tensors' device
+pointers and the current CUDA stream to the C ABI of the same name
+(include/moe.h) and turns a non-OK status into MoeError.  All computation runs
+in the library's CUDA kernels; there is no fallback.  Importing this package
+fails loudly if the compiled library is missing.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoe_b200.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with `python forward_moe_route_b200/build.py` "
+        "(nvcc, sm_100a). The layer has no CPU or Python fallback.")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+# status codes (moe_status)
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT, ERR_DEVICE_CHECK = \
+    range(7)
+GATE_SOFTMAX, GATE_SIGMOID = 0, 1
+DT_F32, DT_BF16, DT_E4M3 = 0, 1, 2
+
+
+class MoeLayerDesc(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int32), ("d", ctypes.c_int32), ("n_shared", ctypes.c_int32),
+                ("n_routed", ctypes.c_int32), ("top_k", ctypes.c_int32),
+                ("inter", ctypes.c_int32), ("gate", ctypes.c_int32), ("renorm", ctypes.c_int32),
+                ("route_scale", ctypes.c_float), ("n_group", ctypes.c_int32),
+                ("topk_group", ctypes.c_int32), ("act_dtype", ctypes.c_int32),
+                ("w_dtype", ctypes.c_int32)]
+
+
+class MoeError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {moe_status_string(status)} (status {status})")
+
+
+_P = ctypes.c_void_p
+_D = ctypes.POINTER(MoeLayerDesc)
+_SIGS = {
+    "moe_workspace_size": (ctypes.c_size_t, [_D]),
+    "moe_route": (ctypes.c_int, [_D, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "moe_permute": (ctypes.c_int, [_D, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "moe_grouped_swiglu": (ctypes.c_int, [_D, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
+                                          ctypes.c_size_t, _P]),
+    "moe_combine": (ctypes.c_int, [_D, _P, _P, _P, _P]),
+    "moe_forward": (ctypes.c_int, [_D, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
+                                   ctypes.c_size_t, _P]),
+    "moe_quantize_fp8_blockwise": (ctypes.c_int, [_P, ctypes.c_int32, ctypes.c_int32,
+                                                  ctypes.c_int32, _P, _P, _P]),
+    "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "moe_last_device_status": (ctypes.c_int, [_P]),
+    "moe_forward_launch_count": (ctypes.c_int32, [_D]),
+    "moe_trace_events": (ctypes.c_int, [ctypes.POINTER(ctypes.c_void_p), ctypes.c_int32]),
+    "moe_selftest_bounded_wait": (ctypes.c_int, [ctypes.c_uint32, _P]),
+}
+for _name, (_res, _args) in _SIGS.items():
+    _f = getattr(_lib, _name)
+    _f.restype = _res
+    _f.argtypes = _args
+
+EXPORTED = tuple(_SIGS)
+
+
+def lib() -> ctypes.CDLL:
+    return _lib
+
+
+def _ptr(t) -> Optional[int]:
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(rc: int, where: str) -> None:
+    if rc != OK:
+        raise MoeError(rc, where)
+
+
+def moe_status_string(status: int) -> str:
+    return _lib.moe_status_string(status).decode()
+
+
+def make_desc(T: int, d: int, n_shared: int, n_routed: int, top_k: int, inter: int, gate: str,
+              renorm: bool, route_scale: float, n_group: int = 1, topk_group: int = 1,
+              dtype: str = "bf16") -> MoeLayerDesc:
+    act, w = {"f32": (DT_F32, DT_F32), "bf16": (DT_BF16, DT_BF16),
+              "e4m3": (DT_BF16, DT_E4M3)}[dtype]
+    return MoeLayerDesc(T, d, n_shared, n_routed, top_k, inter,
+                        {"softmax": GATE_SOFTMAX, "sigmoid": GATE_SIGMOID}[gate], int(renorm),
+                        route_scale, n_group, topk_group, act, w)
+
+
+def desc_from_config(cfg) -> MoeLayerDesc:
+    """Descriptor of a synth.recipes.LayerConfig-like object."""
+    return make_desc(cfg.T, cfg.d, cfg.n_shared, cfg.n_routed, cfg.top_k, cfg.inter, cfg.gate,
+                     cfg.renorm, cfg.route_scale, cfg.n_group, cfg.topk_group, cfg.dtype)
+
+
+def moe_workspace_size(desc: MoeLayerDesc) -> int:
+    return int(_lib.moe_workspace_size(ctypes.byref(desc)))
+
+
+def workspace(desc: MoeLayerDesc, device="cuda"):
+    """A uint8 CUDA tensor of moe_workspace_size(desc) bytes."""
+    import torch
+    n = moe_workspace_size(desc)
+    if n == 0:
+        raise MoeError(ERR_INVALID_ARG, "moe_workspace_size")
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def moe_route(desc, x, w_router, bias, topk_idx, topk_w, counts, ws, stream=None) -> None:
+    _check(_lib.moe_route(ctypes.byref(desc), _ptr(x), _ptr(w_router), _ptr(bias), _ptr(topk_idx),
+                          _ptr(topk_w), _ptr(counts), _ptr(ws), ws.numel() if ws is not None
+                          else 0, _stream(stream)), "moe_route")
+
+
+def moe_permute(desc, x, topk_idx, counts, offsets, perm_src, slot_of, x_perm, x_perm_scale, ws,
+                stream=None) -> None:
+    _check(_lib.moe_permute(ctypes.byref(desc), _ptr(x), _ptr(topk_idx), _ptr(counts),
+                            _ptr(offsets), _ptr(perm_src), _ptr(slot_of), _ptr(x_perm),
+                            _ptr(x_perm_scale), _ptr(ws), ws.numel() if ws is not None else 0,
+                            _stream(stream)), "moe_permute")
+
+
+def moe_grouped_swiglu(desc, x, x_perm, x_perm_scale, offsets, perm_src, slot_of, topk_w, w_gu,
+                       w_gu_scale, w_down, w_down_scale, y_slots, ws, stream=None) -> None:
+    _check(_lib.moe_grouped_swiglu(ctypes.byref(desc), _ptr(x), _ptr(x_perm), _ptr(x_perm_scale),
+                                   _ptr(offsets), _ptr(perm_src), _ptr(slot_of), _ptr(topk_w),
+                                   _ptr(w_gu), _ptr(w_gu_scale), _ptr(w_down),
+                                   _ptr(w_down_scale), _ptr(y_slots), _ptr(ws),
+                                   ws.numel() if ws is not None else 0, _stream(stream)),
+           "moe_grouped_swiglu")
+
+
+def moe_combine(desc, x_residual, y_slots, h, stream=None) -> None:
+    _check(_lib.moe_combine(ctypes.byref(desc), _ptr(x_residual), _ptr(y_slots), _ptr(h),
+                            _stream(stream)), "moe_combine")
+
+
+def moe_forward(desc, x, x_residual, w_router, bias, w_gu, w_gu_scale, w_down, w_down_scale, h,
+                topk_idx, counts, ws, stream=None) -> None:
+    _check(_lib.moe_forward(ctypes.byref(desc), _ptr(x), _ptr(x_residual), _ptr(w_router),
+                            _ptr(bias), _ptr(w_gu), _ptr(w_gu_scale), _ptr(w_down),
+                            _ptr(w_down_scale), _ptr(h), _ptr(topk_idx), _ptr(counts), _ptr(ws),
+                            ws.numel() if ws is not None else 0, _stream(stream)), "moe_forward")
+
+
+def moe_quantize_fp8_blockwise(w_bf16, rows: int, cols: int, batch: int, w_e4m3, scale,
+                               stream=None) -> None:
+    _check(_lib.moe_quantize_fp8_blockwise(_ptr(w_bf16), rows, cols, batch, _ptr(w_e4m3),
+                                           _ptr(scale), _stream(stream)),
+           "moe_quantize_fp8_blockwise")
+
+
+def moe_last_device_status(stream=None) -> int:
+    return int(_lib.moe_last_device_status(_stream(stream)))
+
+
+def moe_forward_launch_count(desc) -> int:
+    return int(_lib.moe_forward_launch_count(ctypes.byref(desc)))
+
+
+def moe_trace_events(events) -> None:
+    """Record stage-boundary events (a list of 6 torch.cuda.Event, or None to stop)."""
+    global _trace_keep
+    if events is None:
+        _trace_keep = None
+        _check(_lib.moe_trace_events(None, 0), "moe_trace_events")
+        return
+    arr = (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events])
+    _trace_keep = arr
+    _check(_lib.moe_trace_events(arr, len(events)), "moe_trace_events")
+
+
+_trace_keep = None
+
+
+def moe_selftest_bounded_wait(limit_us: int, stream=None) -> None:
+    _check(_lib.moe_selftest_bounded_wait(limit_us, _stream(stream)), "moe_selftest_bounded_wait")

@@ -1,0 +1,627 @@
+// C ABI of the DeepSeekMoE layer forward (declared in include/moe.h): argument
+// validation, workspace layout, tensor-map encoding and kernel launches.
+//
+// All kernels live in this one translation unit, so the per-device status
+// word is a single __device__ variable that every kernel names directly.
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstring>
+#include <mutex>
+
+#include "common.cuh"
+#include "gemm.cuh"
+#include "permute.cuh"
+#include "route.cuh"
+
+using namespace moe;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr size_t kAlign = 256;
+constexpr int kMaxShared = 64;     // shared experts accepted
+constexpr int kMaxRouted = 512;
+constexpr int kMaxSmem = 232448;   // dynamic shared memory per block on sm_100
+
+inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+struct Dims {
+  int64_t T, d, Ks, N, K, I, E, R;
+  int act, w;
+  bool fp8, f32;
+  size_t x_esz;   // bytes per element of x, w_router and x_residual
+  size_t op_esz;  // bytes per element of the GEMM operands x_perm and H
+  size_t y_esz;   // bytes per element of y_slots and h
+  int n_chunks;
+};
+
+moe_status fill_dims(const moe_layer_desc* desc, Dims* D) {
+  if (!desc) return MOE_ERR_INVALID_ARG;
+  const moe_layer_desc& s = *desc;
+  if (s.T < 0 || s.d < 1 || s.n_shared < 0 || s.n_shared > kMaxShared || s.n_routed < 1 ||
+      s.n_routed > kMaxRouted || s.top_k < 1 || s.top_k > route::MAXK || s.top_k > s.n_routed ||
+      s.inter < 16 || s.d > 65536 || s.inter > 65536)
+    return MOE_ERR_INVALID_ARG;
+  if (s.gate != MOE_GATE_SOFTMAX && s.gate != MOE_GATE_SIGMOID) return MOE_ERR_INVALID_ARG;
+  if (s.renorm != 0 && s.renorm != 1) return MOE_ERR_INVALID_ARG;
+  if (!std::isfinite(s.route_scale) || !(s.route_scale > 0.f)) return MOE_ERR_INVALID_ARG;
+  if (s.n_group < 1 || s.n_group > 32 || s.topk_group < 1 || s.topk_group > s.n_group ||
+      s.n_routed % s.n_group != 0)
+    return MOE_ERR_INVALID_ARG;
+  if (s.n_group > 1 && (s.n_routed / s.n_group < 2 ||
+                        (int64_t)s.topk_group * (s.n_routed / s.n_group) < s.top_k))
+    return MOE_ERR_INVALID_ARG;
+  int align;
+  if (s.act_dtype == MOE_DT_F32 && s.w_dtype == MOE_DT_F32) {
+    D->x_esz = 4; D->op_esz = 4; D->y_esz = 4; align = 32; D->fp8 = false; D->f32 = true;
+  } else if (s.act_dtype == MOE_DT_BF16 && s.w_dtype == MOE_DT_BF16) {
+    D->x_esz = 2; D->op_esz = 2; D->y_esz = 2; align = 64; D->fp8 = false; D->f32 = false;
+  } else if (s.act_dtype == MOE_DT_BF16 && s.w_dtype == MOE_DT_E4M3) {
+    D->x_esz = 2; D->op_esz = 1; D->y_esz = 2; align = 128; D->fp8 = true; D->f32 = false;
+  } else {
+    return MOE_ERR_INVALID_ARG;
+  }
+  if (s.d % align || s.inter % align) return MOE_ERR_INVALID_ARG;
+  D->T = s.T; D->d = s.d; D->Ks = s.n_shared; D->N = s.n_routed; D->K = s.top_k; D->I = s.inter;
+  D->E = D->Ks + D->N;
+  D->R = D->T * D->K;
+  D->act = s.act_dtype; D->w = s.w_dtype;
+  if (D->R + D->Ks * D->T + D->T >= ((int64_t)1 << 31)) return MOE_ERR_INVALID_ARG;
+  D->n_chunks = (int)((D->T + perm::CHUNK - 1) / perm::CHUNK);
+  return MOE_OK;
+}
+
+struct Layout {
+  size_t logits, topk_idx, topk_w, counts, hist, offsets, perm_src, slot_of, pair_of, gtab;
+  size_t x_perm, x_perm_scale, hbuf, hscale, y_slots, total;
+};
+
+Layout layout(const Dims& D) {
+  Layout L;
+  size_t o = 0;
+  auto take = [&](size_t bytes) { size_t at = o; o = align_up(o + bytes, kAlign); return at; };
+  L.logits = take(D.f32 ? 0 : (size_t)D.T * D.N * 4);
+  L.topk_idx = take((size_t)D.R * 4);
+  L.topk_w = take((size_t)D.R * 4);
+  L.counts = take((size_t)D.N * 4);
+  L.hist = take((size_t)(D.n_chunks > 0 ? D.n_chunks : 1) * D.N * 4);
+  L.offsets = take((size_t)(D.N + 1) * 4);
+  L.perm_src = take((size_t)D.R * 4);
+  L.slot_of = take((size_t)D.R * 4);
+  L.pair_of = take((size_t)D.R * 4);
+  L.gtab = take((size_t)gemm::group_tab_ints((int)D.E) * 4);
+  const size_t xrows = (size_t)D.R + (D.fp8 ? (size_t)D.T : 0);
+  L.x_perm = take(xrows * D.d * D.op_esz);
+  L.x_perm_scale = take(D.fp8 ? xrows * (D.d / 128) * 4 : 0);
+  const size_t hrows = (size_t)D.R + (size_t)D.Ks * D.T;
+  L.hbuf = take(hrows * D.I * D.op_esz);
+  L.hscale = take(D.fp8 ? hrows * (D.I / 128) * 4 : 0);
+  L.y_slots = take((size_t)D.T * (D.K + D.Ks) * D.d * D.y_esz);
+  L.total = o;
+  return L;
+}
+
+inline bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+// ----------------------------------------------------------------------------- device setup
+struct DeviceInfo {
+  int sms = 0;
+  bool attrs_done = false;
+};
+std::mutex g_mu;
+DeviceInfo g_dev[kMaxDevices];
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+template <int KIND, int EPI>
+cudaError_t set_gemm_attr() {
+  return cudaFuncSetAttribute(gemm::k_grouped_gemm<KIND, EPI>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
+}
+
+moe_status device_setup(int* sms) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MOE_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_mu);
+  DeviceInfo& di = g_dev[dev];
+  if (!di.attrs_done) {
+    if (cudaDeviceGetAttribute(&di.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    cudaError_t e = cudaSuccess;
+    if (e == cudaSuccess) e = set_gemm_attr<0, gemm::EPI_F32_STORE>();
+    if (e == cudaSuccess) e = set_gemm_attr<0, gemm::EPI_SWIGLU>();
+    if (e == cudaSuccess) e = set_gemm_attr<0, gemm::EPI_SCATTER>();
+    if (e == cudaSuccess) e = set_gemm_attr<1, gemm::EPI_SWIGLU>();
+    if (e == cudaSuccess) e = set_gemm_attr<1, gemm::EPI_SCATTER>();
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    if (!g_encode) {
+      void* fn = nullptr;
+      cudaDriverEntryPointQueryResult q;
+      if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
+              cudaSuccess ||
+          q != cudaDriverEntryPointSuccess || !fn)
+        return MOE_ERR_CUDA;
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+    di.attrs_done = true;
+  }
+  *sms = di.sms;
+  return MOE_OK;
+}
+
+// 2-D K-major tensor map with 128-byte swizzle: rows of `inner` elements,
+// box = (128 bytes of K) x box_rows.
+moe_status make_tmap(CUtensorMap* m, const void* base, size_t esz, uint64_t inner, uint64_t rows,
+                     uint32_t box_rows) {
+  CUtensorMapDataType dt = esz == 4   ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                           : esz == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                      : CU_TENSOR_MAP_DATA_TYPE_UINT8;
+  cuuint64_t dims[2] = {inner, rows > 0 ? rows : 1};
+  cuuint64_t strides[1] = {inner * esz};
+  cuuint32_t box[2] = {(cuuint32_t)(gemm::KB / esz), box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? MOE_OK : MOE_ERR_CUDA;
+}
+
+int pick_stages(int bn, int n_groups) {
+  for (int s = 8; s >= 2; --s)
+    if (gemm::smem_bytes(bn, s, n_groups) <= (size_t)kMaxSmem) return s;
+  return 0;
+}
+
+uint32_t tmem_cols_for(int bn) {
+  uint32_t c = 32;
+  while (c < (uint32_t)(2 * bn)) c <<= 1;
+  return c;
+}
+
+template <int KIND, int EPI>
+moe_status launch_gemm(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b,
+                       gemm::Args args, int grid, cudaStream_t st) {
+  const int ng = args.gt.base ? args.gt.n : 1;
+  args.stages = pick_stages(args.bn, ng);
+  if (!args.stages) return MOE_ERR_UNSUPPORTED;
+  args.tmem_cols = tmem_cols_for(args.bn);
+  if (args.tmem_cols > 512) return MOE_ERR_UNSUPPORTED;
+  const size_t smem = gemm::smem_bytes(args.bn, args.stages, ng);
+  gemm::k_grouped_gemm<KIND, EPI><<<grid, gemm::NUM_THREADS, smem, st>>>(a0, a1, b, args);
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+inline moe_status launched() { return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+// Stage-timing events of the calling host thread (moe_trace_events).
+thread_local cudaEvent_t* t_events = nullptr;
+inline void trace(int i, cudaStream_t st) {
+  if (t_events) cudaEventRecord(t_events[i], st);
+}
+
+route::Params route_params(const moe_layer_desc& s) {
+  route::Params p;
+  p.T = s.T; p.N = s.n_routed; p.K = s.top_k; p.gate = s.gate; p.renorm = s.renorm;
+  p.n_group = s.n_group; p.topk_group = s.topk_group; p.scale = s.route_scale;
+  return p;
+}
+
+template <int VPL>
+void launch_topk(const float* logits, const float* bias, const route::Params& p, int32_t* idx,
+                 float* w, int32_t* counts, cudaStream_t st) {
+  route::k_topk<VPL><<<(p.T + 7) / 8, 256, 0, st>>>(logits, bias, p, idx, w, counts);
+}
+template <int VPL>
+void launch_route_f32(const float* x, const float* wr, int d, const float* bias,
+                      const route::Params& p, int32_t* idx, float* w, int32_t* counts,
+                      cudaStream_t st) {
+  route::k_route_f32<VPL><<<(p.T + 7) / 8, 256, 0, st>>>(x, wr, d, bias, p, idx, w, counts);
+}
+
+// ----------------------------------------------------------------------------- stages
+moe_status do_route(const moe_layer_desc& s, const Dims& D, const Layout& L, const void* x,
+                    const void* w_router, const float* bias, int32_t* topk_idx, float* topk_w,
+                    int32_t* counts, uint8_t* ws, int sms, cudaStream_t st) {
+  const route::Params p = route_params(s);
+  const int N = (int)D.N;
+  if (D.T == 0) {
+    route::k_zero_i32<<<1, 256, 0, st>>>(counts, N);
+    return launched();
+  }
+  if (D.f32) {
+    route::k_zero_i32<<<1, 256, 0, st>>>(counts, N);
+    const float* xf = static_cast<const float*>(x);
+    const float* wf = static_cast<const float*>(w_router);
+    const int dd = (int)D.d;
+    if (N <= 32) launch_route_f32<1>(xf, wf, dd, bias, p, topk_idx, topk_w, counts, st);
+    else if (N <= 64) launch_route_f32<2>(xf, wf, dd, bias, p, topk_idx, topk_w, counts, st);
+    else if (N <= 128) launch_route_f32<4>(xf, wf, dd, bias, p, topk_idx, topk_w, counts, st);
+    else if (N <= 256) launch_route_f32<8>(xf, wf, dd, bias, p, topk_idx, topk_w, counts, st);
+    else launch_route_f32<16>(xf, wf, dd, bias, p, topk_idx, topk_w, counts, st);
+    return launched();
+  }
+  // bf16 router GEMM on tensor cores: logits [T, N] fp32 (counts zeroed in its prologue)
+  float* logits = reinterpret_cast<float*>(ws + L.logits);
+  const int bn_full = (N + 15) / 16 * 16;
+  const int bn = bn_full <= 256 ? bn_full : 256;
+  CUtensorMap ta, tb;
+  moe_status rc = make_tmap(&ta, x, 2, D.d, D.T, gemm::BM);
+  if (rc == MOE_OK) rc = make_tmap(&tb, w_router, 2, D.d, D.N, bn);
+  if (rc != MOE_OK) return rc;
+  gemm::Args a;
+  memset(&a, 0, sizeof(a));
+  a.gt.base = nullptr;
+  a.gt.n = 1;
+  a.gt.single_rows = (int)D.T;
+  a.n_tiles_n = (N + bn - 1) / bn;
+  a.num_kb = (int)(D.d * 2 / gemm::KB);
+  a.kb_elems = gemm::KB / 2;
+  a.bn = bn;
+  a.b_rows_per_expert = 0;
+  a.idesc = umma_idesc(1, gemm::BM, bn);
+  a.out = logits;
+  a.out_ld = N;
+  a.out_cols = N;
+  a.out_bf16 = 0;
+  a.zero_ptr = counts;
+  a.zero_n = N;
+  const int tiles = (int)((D.T + 127) / 128) * a.n_tiles_n;
+  rc = launch_gemm<0, gemm::EPI_F32_STORE>(ta, ta, tb, a, tiles < sms ? tiles : sms, st);
+  if (rc != MOE_OK) return rc;
+  if (N <= 32) launch_topk<1>(logits, bias, p, topk_idx, topk_w, counts, st);
+  else if (N <= 64) launch_topk<2>(logits, bias, p, topk_idx, topk_w, counts, st);
+  else if (N <= 128) launch_topk<4>(logits, bias, p, topk_idx, topk_w, counts, st);
+  else if (N <= 256) launch_topk<8>(logits, bias, p, topk_idx, topk_w, counts, st);
+  else launch_topk<16>(logits, bias, p, topk_idx, topk_w, counts, st);
+  return launched();
+}
+
+moe_status do_permute(const Dims& D, const Layout& L, const void* x, const int32_t* topk_idx,
+                      const int32_t* counts, int32_t* offsets, int32_t* perm_src,
+                      int32_t* slot_of, void* x_perm, float* x_perm_scale, uint8_t* ws,
+                      cudaStream_t st) {
+  const int T = (int)D.T, K = (int)D.K, N = (int)D.N;
+  int32_t* hist = reinterpret_cast<int32_t*>(ws + L.hist);
+  if (T == 0) {
+    route::k_zero_i32<<<1, 256, 0, st>>>(offsets, N + 1);
+    return launched();
+  }
+  perm::k_hist<<<D.n_chunks, 256, N * 4, st>>>(topk_idx, T, K, N, hist);
+  perm::k_scan<<<1, 1024, 0, st>>>(hist, D.n_chunks, N, counts, offsets);
+  perm::k_slots<<<D.n_chunks, 32, N * 4, st>>>(topk_idx, T, K, N, hist, slot_of, perm_src);
+  if (D.fp8) {
+    perm::k_gather_quant<<<(T + 7) / 8, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(x), T, K,
+                                                      (int)D.d, (int)D.R, slot_of,
+                                                      static_cast<uint8_t*>(x_perm), x_perm_scale);
+  } else {
+    perm::k_gather<<<(T + 7) / 8, 256, 0, st>>>(static_cast<const uint8_t*>(x), T, K,
+                                                (int)(D.d * D.x_esz), slot_of,
+                                                static_cast<uint8_t*>(x_perm));
+  }
+  return launched();
+}
+
+moe_status do_grouped(const Dims& D, const Layout& L, const void* x, const void* x_perm,
+                      const int32_t* offsets, const int32_t* slot_of, const float* topk_w,
+                      const void* w_gu, const void* w_down, void* y_slots, uint8_t* ws, int sms,
+                      cudaStream_t st) {
+  if (D.T == 0) return MOE_OK;
+  if (D.fp8) return MOE_ERR_UNSUPPORTED;
+  const int E = (int)D.E;
+  int32_t* gtab = reinterpret_cast<int32_t*>(ws + L.gtab);
+  int32_t* pair_of = reinterpret_cast<int32_t*>(ws + L.pair_of);
+  void* hbuf = ws + L.hbuf;
+  const int prep_blocks = 1 + (int)((D.R + 1023) / 1024 < 4 * sms ? (D.R + 1023) / 1024 : 4 * sms);
+  trace(2, st);
+  perm::k_prep_groups<<<prep_blocks, 1024, 0, st>>>(offsets, (int)D.T, (int)D.K, (int)D.Ks,
+                                                    (int)D.N, 0, gtab, slot_of, pair_of);
+  moe_status rc = launched();
+  if (rc != MOE_OK) return rc;
+
+  const size_t esz = D.op_esz;
+  const int kind = D.f32 ? 1 : 0;
+  const uint32_t fmt = D.f32 ? 2u : 1u;
+  const int kbe = (int)(gemm::KB / esz);
+  const int64_t hrows = D.R + D.Ks * D.T;
+  // upper bound on m-tiles over all groups
+  const int64_t mt_bound = (D.R + (int64_t)D.N * 127) / 128 + D.Ks * ((D.T + 127) / 128);
+
+  // GEMM1: H = SiLU(A Wg^T) * (A Wu^T)
+  {
+    int hn = 128;
+    while (hn > 16 && D.I % hn) hn >>= 1;
+    if (D.I % hn) return MOE_ERR_UNSUPPORTED;
+    CUtensorMap ta0, ta1, tb;
+    rc = make_tmap(&ta0, x, esz, D.d, D.T, gemm::BM);
+    if (rc == MOE_OK) rc = make_tmap(&ta1, x_perm, esz, D.d, D.R, gemm::BM);
+    if (rc == MOE_OK) rc = make_tmap(&tb, w_gu, esz, D.d, (uint64_t)E * 2 * D.I, hn);
+    if (rc != MOE_OK) return rc;
+    gemm::Args a;
+    memset(&a, 0, sizeof(a));
+    a.gt.base = gtab;
+    a.gt.n = E;
+    a.n_tiles_n = (int)(D.I / hn);
+    a.num_kb = (int)(D.d * esz / gemm::KB);
+    a.kb_elems = kbe;
+    a.bn = 2 * hn;
+    a.b_half = hn;
+    a.b_up_off = (int)D.I;
+    a.b_rows_per_expert = (int)(2 * D.I);
+    a.idesc = umma_idesc(fmt, gemm::BM, 2 * hn);
+    a.out = hbuf;
+    a.out_ld = D.I;
+    a.out_bf16 = D.f32 ? 0 : 1;
+    const int64_t tiles = mt_bound * a.n_tiles_n;
+    const int grid = (int)(tiles < sms ? tiles : sms);
+    rc = kind == 0 ? launch_gemm<0, gemm::EPI_SWIGLU>(ta0, ta1, tb, a, grid, st)
+                   : launch_gemm<1, gemm::EPI_SWIGLU>(ta0, ta1, tb, a, grid, st);
+    if (rc != MOE_OK) return rc;
+    trace(3, st);
+  }
+  // GEMM2: Y = H Wd^T, times g, scattered to the token-major slots
+  {
+    int bn = 256;
+    while (bn > 16 && D.d % bn) bn >>= 1;
+    if (D.d % bn) return MOE_ERR_UNSUPPORTED;
+    CUtensorMap ta, tb;
+    rc = make_tmap(&ta, hbuf, esz, D.I, hrows, gemm::BM);
+    if (rc == MOE_OK) rc = make_tmap(&tb, w_down, esz, D.I, (uint64_t)E * D.d, bn);
+    if (rc != MOE_OK) return rc;
+    gemm::Args a;
+    memset(&a, 0, sizeof(a));
+    a.gt.base = gtab;
+    a.gt.n = E;
+    a.n_tiles_n = (int)(D.d / bn);
+    a.num_kb = (int)(D.I * esz / gemm::KB);
+    a.kb_elems = kbe;
+    a.bn = bn;
+    a.b_rows_per_expert = (int)D.d;
+    a.a_from_crow = 1;
+    a.idesc = umma_idesc(fmt, gemm::BM, bn);
+    a.out = y_slots;
+    a.out_ld = D.d;
+    a.out_bf16 = D.f32 ? 0 : 1;
+    a.pair_of = pair_of;
+    a.topk_w = topk_w;
+    a.K = (int)D.K;
+    a.Ks = (int)D.Ks;
+    const int64_t tiles = mt_bound * a.n_tiles_n;
+    const int grid = (int)(tiles < sms ? tiles : sms);
+    rc = kind == 0 ? launch_gemm<0, gemm::EPI_SCATTER>(ta, ta, tb, a, grid, st)
+                   : launch_gemm<1, gemm::EPI_SCATTER>(ta, ta, tb, a, grid, st);
+    if (rc == MOE_OK) trace(4, st);
+  }
+  return rc;
+}
+
+moe_status do_combine(const Dims& D, const void* x_res, const void* y, void* h, cudaStream_t st) {
+  if (D.T == 0) return MOE_OK;
+  const int vec = D.f32 ? 4 : 8;
+  const int64_t threads = D.T * (D.d / vec);
+  const int blocks = (int)((threads + 255) / 256);
+  if (D.f32)
+    perm::k_combine<false><<<blocks, 256, 0, st>>>(x_res, y, h, (int)D.T, (int)D.d, (int)D.K,
+                                                   (int)D.Ks);
+  else
+    perm::k_combine<true><<<blocks, 256, 0, st>>>(x_res, y, h, (int)D.T, (int)D.d, (int)D.K,
+                                                  (int)D.Ks);
+  return launched();
+}
+
+__global__ void k_selftest_wait(uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    // Nothing arrives on `bar`: the wait must give up after limit_ns.
+    const uint64_t t0 = globaltimer_ns();
+    bool done = false;
+    while (!done) {
+      if (mbar_try_wait(&bar, 0)) break;
+      if (globaltimer_ns() - t0 > limit_ns) {
+        set_status(MOE_ERR_TIMEOUT);
+        done = true;
+      }
+    }
+  }
+  __syncthreads();
+}
+
+}  // namespace
+
+// ============================================================================= C ABI
+extern "C" {
+
+size_t moe_workspace_size(const moe_layer_desc* desc) {
+  Dims D;
+  if (fill_dims(desc, &D) != MOE_OK) return 0;
+  return layout(D).total;
+}
+
+moe_status moe_route(const moe_layer_desc* desc, const void* x, const void* w_router,
+                     const float* bias, int32_t* topk_idx, float* topk_w, int32_t* counts,
+                     void* ws, size_t ws_bytes, cudaStream_t stream) {
+  Dims D;
+  moe_status rc = fill_dims(desc, &D);
+  if (rc != MOE_OK) return rc;
+  if (bias && desc->gate != MOE_GATE_SIGMOID) return MOE_ERR_INVALID_ARG;
+  if (!counts || !aligned16(counts)) return MOE_ERR_INVALID_ARG;
+  if (D.T > 0) {
+    if (!x || !w_router || !topk_idx || !topk_w || !aligned16(x) || !aligned16(w_router) ||
+        !aligned16(topk_idx) || !aligned16(topk_w) || (bias && !aligned16(bias)))
+      return MOE_ERR_INVALID_ARG;
+  }
+  const Layout L = layout(D);
+  if (!ws || ws_bytes < L.total || !aligned16(ws)) return MOE_ERR_WORKSPACE;
+  int sms;
+  if ((rc = device_setup(&sms)) != MOE_OK) return rc;
+  return do_route(*desc, D, L, x, w_router, bias, topk_idx, topk_w, counts,
+                  static_cast<uint8_t*>(ws), sms, stream);
+}
+
+moe_status moe_permute(const moe_layer_desc* desc, const void* x, const int32_t* topk_idx,
+                       const int32_t* counts, int32_t* offsets, int32_t* perm_src,
+                       int32_t* slot_of, void* x_perm, float* x_perm_scale, void* ws,
+                       size_t ws_bytes, cudaStream_t stream) {
+  Dims D;
+  moe_status rc = fill_dims(desc, &D);
+  if (rc != MOE_OK) return rc;
+  if (!offsets || !aligned16(offsets)) return MOE_ERR_INVALID_ARG;
+  if (D.T > 0) {
+    if (!x || !topk_idx || !counts || !perm_src || !slot_of || !x_perm || !aligned16(x) ||
+        !aligned16(topk_idx) || !aligned16(perm_src) || !aligned16(slot_of) ||
+        !aligned16(x_perm))
+      return MOE_ERR_INVALID_ARG;
+    if (D.fp8 != (x_perm_scale != nullptr)) return MOE_ERR_INVALID_ARG;
+    if (x_perm_scale && !aligned16(x_perm_scale)) return MOE_ERR_INVALID_ARG;
+  }
+  const Layout L = layout(D);
+  if (!ws || ws_bytes < L.total || !aligned16(ws)) return MOE_ERR_WORKSPACE;
+  int sms;
+  if ((rc = device_setup(&sms)) != MOE_OK) return rc;
+  return do_permute(D, L, x, topk_idx, counts, offsets, perm_src, slot_of, x_perm, x_perm_scale,
+                    static_cast<uint8_t*>(ws), stream);
+}
+
+moe_status moe_grouped_swiglu(const moe_layer_desc* desc, const void* x, const void* x_perm,
+                              const float* x_perm_scale, const int32_t* offsets,
+                              const int32_t* perm_src, const int32_t* slot_of,
+                              const float* topk_w, const void* w_gu, const float* w_gu_scale,
+                              const void* w_down, const float* w_down_scale, void* y_slots,
+                              void* ws, size_t ws_bytes, cudaStream_t stream) {
+  (void)perm_src;
+  Dims D;
+  moe_status rc = fill_dims(desc, &D);
+  if (rc != MOE_OK) return rc;
+  if (D.T > 0) {
+    if (!x_perm || !offsets || !slot_of || !topk_w || !w_gu || !w_down || !y_slots ||
+        !aligned16(x_perm) || !aligned16(w_gu) || !aligned16(w_down) || !aligned16(y_slots))
+      return MOE_ERR_INVALID_ARG;
+    if (!D.fp8 && (!x || !aligned16(x))) return MOE_ERR_INVALID_ARG;
+    if (D.fp8 && (!x_perm_scale || !w_gu_scale || !w_down_scale)) return MOE_ERR_INVALID_ARG;
+  }
+  const Layout L = layout(D);
+  if (!ws || ws_bytes < L.total || !aligned16(ws)) return MOE_ERR_WORKSPACE;
+  int sms;
+  if ((rc = device_setup(&sms)) != MOE_OK) return rc;
+  return do_grouped(D, L, x, x_perm, offsets, slot_of, topk_w, w_gu, w_down, y_slots,
+                    static_cast<uint8_t*>(ws), sms, stream);
+}
+
+moe_status moe_combine(const moe_layer_desc* desc, const void* x_residual, const void* y_slots,
+                       void* h, cudaStream_t stream) {
+  Dims D;
+  moe_status rc = fill_dims(desc, &D);
+  if (rc != MOE_OK) return rc;
+  if (D.T > 0 && (!x_residual || !y_slots || !h || !aligned16(x_residual) ||
+                  !aligned16(y_slots) || !aligned16(h)))
+    return MOE_ERR_INVALID_ARG;
+  return do_combine(D, x_residual, y_slots, h, stream);
+}
+
+moe_status moe_forward(const moe_layer_desc* desc, const void* x, const void* x_residual,
+                       const void* w_router, const float* bias, const void* w_gu,
+                       const float* w_gu_scale, const void* w_down, const float* w_down_scale,
+                       void* h, int32_t* topk_idx, int32_t* counts, void* ws, size_t ws_bytes,
+                       cudaStream_t stream) {
+  Dims D;
+  moe_status rc = fill_dims(desc, &D);
+  if (rc != MOE_OK) return rc;
+  if (bias && desc->gate != MOE_GATE_SIGMOID) return MOE_ERR_INVALID_ARG;
+  if (D.T > 0) {
+    if (!x || !w_router || !w_gu || !w_down || !h || !aligned16(x) || !aligned16(w_router) ||
+        !aligned16(w_gu) || !aligned16(w_down) || !aligned16(h) || (bias && !aligned16(bias)) ||
+        (x_residual && !aligned16(x_residual)) || (topk_idx && !aligned16(topk_idx)))
+      return MOE_ERR_INVALID_ARG;
+    if (D.fp8 && (!w_gu_scale || !w_down_scale)) return MOE_ERR_INVALID_ARG;
+  }
+  if (counts && !aligned16(counts)) return MOE_ERR_INVALID_ARG;
+  const Layout L = layout(D);
+  if (!ws || ws_bytes < L.total || !aligned16(ws)) return MOE_ERR_WORKSPACE;
+  int sms;
+  if ((rc = device_setup(&sms)) != MOE_OK) return rc;
+  uint8_t* w8 = static_cast<uint8_t*>(ws);
+  int32_t* idx = topk_idx ? topk_idx : reinterpret_cast<int32_t*>(w8 + L.topk_idx);
+  float* tw = reinterpret_cast<float*>(w8 + L.topk_w);
+  int32_t* cnt = counts ? counts : reinterpret_cast<int32_t*>(w8 + L.counts);
+  int32_t* offsets = reinterpret_cast<int32_t*>(w8 + L.offsets);
+  int32_t* perm_src = reinterpret_cast<int32_t*>(w8 + L.perm_src);
+  int32_t* slot_of = reinterpret_cast<int32_t*>(w8 + L.slot_of);
+  void* x_perm = w8 + L.x_perm;
+  float* x_perm_scale = D.fp8 ? reinterpret_cast<float*>(w8 + L.x_perm_scale) : nullptr;
+  void* y = w8 + L.y_slots;
+  trace(0, stream);
+  if ((rc = do_route(*desc, D, L, x, w_router, bias, idx, tw, cnt, w8, sms, stream)) != MOE_OK)
+    return rc;
+  trace(1, stream);
+  if ((rc = do_permute(D, L, x, idx, cnt, offsets, perm_src, slot_of, x_perm, x_perm_scale, w8,
+                       stream)) != MOE_OK)
+    return rc;
+  if ((rc = do_grouped(D, L, x, x_perm, offsets, slot_of, tw, w_gu, w_down, y, w8, sms,
+                       stream)) != MOE_OK)
+    return rc;
+  rc = do_combine(D, x_residual ? x_residual : x, y, h, stream);
+  if (rc == MOE_OK) trace(5, stream);
+  return rc;
+}
+
+moe_status moe_quantize_fp8_blockwise(const void* w_bf16, int32_t rows, int32_t cols,
+                                      int32_t batch, void* w_e4m3, float* scale,
+                                      cudaStream_t stream) {
+  if (rows <= 0 || cols <= 0 || batch <= 0 || rows % 128 || cols % 128) return MOE_ERR_INVALID_ARG;
+  if (!w_bf16 || !w_e4m3 || !scale || !aligned16(w_bf16) || !aligned16(w_e4m3))
+    return MOE_ERR_INVALID_ARG;
+  const int64_t blocks = (int64_t)batch * (rows / 128) * (cols / 128);
+  if (blocks >= ((int64_t)1 << 31)) return MOE_ERR_INVALID_ARG;
+  perm::k_quant_w<<<(unsigned)blocks, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(w_bf16),
+                                                         rows, cols,
+                                                         static_cast<uint8_t*>(w_e4m3), scale);
+  return launched();
+}
+
+const char* moe_status_string(moe_status status) {
+  switch (status) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED: return "unsupported shape";
+    case MOE_ERR_WORKSPACE: return "workspace too small";
+    case MOE_ERR_CUDA: return "CUDA error";
+    case MOE_ERR_TIMEOUT: return "device wait timed out";
+    case MOE_ERR_DEVICE_CHECK: return "device consistency check failed";
+  }
+  return "unknown status";
+}
+
+moe_status moe_last_device_status(cudaStream_t stream) {
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return MOE_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_status, sizeof(int)) != cudaSuccess) return MOE_ERR_CUDA;
+  const int zero = 0;
+  if (cudaMemcpyToSymbol(g_status, &zero, sizeof(int)) != cudaSuccess) return MOE_ERR_CUDA;
+  return static_cast<moe_status>(v);
+}
+
+moe_status moe_trace_events(cudaEvent_t* events, int32_t n) {
+  if (events && n != 6) return MOE_ERR_INVALID_ARG;
+  t_events = events;
+  return MOE_OK;
+}
+
+int32_t moe_forward_launch_count(const moe_layer_desc* desc) {
+  Dims D;
+  if (fill_dims(desc, &D) != MOE_OK) return 0;
+  if (D.T == 0) return 2;
+  // route (2) + permute (4) + grouped (3) + combine (1)
+  return 10;
+}
+
+moe_status moe_selftest_bounded_wait(uint32_t limit_us, cudaStream_t stream) {
+  if (limit_us < 1 || limit_us > 1000000) return MOE_ERR_INVALID_ARG;
+  k_selftest_wait<<<1, 32, 0, stream>>>((uint64_t)limit_us * 1000ull);
+  return launched();
+}
+
+}  // extern "C"

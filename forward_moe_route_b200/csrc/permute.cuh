@@ -1,0 +1,399 @@
+// Token -> expert permutation, expert-contiguous gather (with fused 1x128 E4M3
+// quantisation), group-table preparation for the grouped GEMMs, and the
+// weighted combine.
+//
+// Permutation: the pair (t, k) with expert e = idx[t,k] goes to row
+// offsets[e] + #{t' < t : e in idx[t']}.  It is built deterministically from
+// per-chunk histograms (chunks of CHUNK tokens), a scan over chunks and
+// experts, and an in-order walk of each chunk, so it is stable by token and
+// identical from run to run.
+#pragma once
+
+#include "common.cuh"
+#include "gemm.cuh"
+
+namespace moe {
+namespace perm {
+
+constexpr int CHUNK = 128;  // tokens per histogram chunk
+
+// hist[c * N + e] = number of pairs of chunk c routed to expert e.
+__global__ void __launch_bounds__(256) k_hist(const int32_t* __restrict__ idx, int T, int K, int N,
+                                              int32_t* __restrict__ hist) {
+  extern __shared__ int32_t sh[];
+  for (int e = threadIdx.x; e < N; e += blockDim.x) sh[e] = 0;
+  __syncthreads();
+  const int t0 = blockIdx.x * CHUNK;
+  const int t1 = min(T, t0 + CHUNK);
+  for (int i = t0 * K + threadIdx.x; i < t1 * K; i += blockDim.x) {
+    const int e = idx[i];
+    if ((unsigned)e < (unsigned)N) atomicAdd(&sh[e], 1);
+    else set_status(MOE_ERR_DEVICE_CHECK);
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < N; e += blockDim.x) hist[(size_t)blockIdx.x * N + e] = sh[e];
+}
+
+// One block of 1024 threads.  Turns hist into each chunk's first row per
+// expert (offsets[e] + pairs of expert e in earlier chunks), writes offsets
+// [N+1], and checks the totals against `counts`.
+__global__ void __launch_bounds__(1024) k_scan(int32_t* __restrict__ hist, int n_chunks, int N,
+                                               const int32_t* __restrict__ counts,
+                                               int32_t* __restrict__ offsets) {
+  __shared__ int32_t part_sum[1024];
+  __shared__ int32_t tot[1024];
+  __shared__ int32_t warp_tot[32];
+  const int P = max(1, (int)(blockDim.x / N));  // parts per expert
+  const int tid = threadIdx.x;
+  const int e = tid % N, part = tid / N;
+  const bool active = part < P && tid < N * P;
+  const int per = (n_chunks + P - 1) / P;
+  const int c0 = part * per, c1 = min(n_chunks, c0 + per);
+  int sum = 0;
+  if (active) {
+#pragma unroll 8
+    for (int c = c0; c < c1; ++c) sum += hist[(size_t)c * N + e];
+    part_sum[tid] = sum;
+  }
+  __syncthreads();
+  // exclusive prefix over parts, and expert totals
+  int before = 0;
+  if (active) {
+    for (int q = 0; q < part; ++q) before += part_sum[q * N + e];
+    if (part == 0) {
+      int total = 0;
+      for (int q = 0; q < P; ++q) total += part_sum[q * N + e];
+      tot[e] = total;
+      if (counts && counts[e] != total) set_status(MOE_ERR_DEVICE_CHECK);
+    }
+  }
+  __syncthreads();
+  // exclusive scan of tot[0..N) -> offsets (warp scans + scan of warp totals)
+  int v = (tid < N) ? tot[tid] : 0;
+  int incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane_id() >= o) incl += y;
+  }
+  if (lane_id() == 31) warp_tot[warp_id()] = incl;
+  __syncthreads();
+  if (warp_id() == 0) {
+    int wv = warp_tot[lane_id()];
+    int wi = wv;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, wi, o);
+      if (lane_id() >= o) wi += y;
+    }
+    warp_tot[lane_id()] = wi - wv;
+  }
+  __syncthreads();
+  const int excl = incl - v + warp_tot[warp_id()];
+  __syncthreads();
+  if (tid < N) {
+    offsets[tid] = excl;
+    part_sum[tid] = excl;  // reuse as expert base
+    if (tid == N - 1) offsets[N] = excl + v;
+  }
+  __syncthreads();
+  if (active) {
+    int run = part_sum[e] + before;
+    // note: part_sum[e] now holds offsets[e] for e < N (all parts read it)
+#pragma unroll 8
+    for (int c = c0; c < c1; ++c) {
+      const int h = hist[(size_t)c * N + e];
+      hist[(size_t)c * N + e] = run;
+      run += h;
+    }
+  }
+}
+
+// One warp per chunk: walks the chunk's tokens in order and hands out rows.
+__global__ void __launch_bounds__(32) k_slots(const int32_t* __restrict__ idx, int T, int K, int N,
+                                              const int32_t* __restrict__ base,
+                                              int32_t* __restrict__ slot_of,
+                                              int32_t* __restrict__ perm_src) {
+  extern __shared__ int32_t next[];
+  const int lane = lane_id();
+  for (int e = lane; e < N; e += 32) next[e] = base[(size_t)blockIdx.x * N + e];
+  __syncwarp();
+  const int t0 = blockIdx.x * CHUNK;
+  const int t1 = min(T, t0 + CHUNK);
+  for (int t = t0; t < t1; ++t) {
+    if (lane < K) {
+      const int e = idx[(size_t)t * K + lane];
+      if ((unsigned)e < (unsigned)N) {
+        const int row = next[e];
+        next[e] = row + 1;
+        slot_of[(size_t)t * K + lane] = row;
+        perm_src[row] = t;
+      } else {
+        slot_of[(size_t)t * K + lane] = -1;
+      }
+    }
+    __syncwarp();
+  }
+}
+
+// Row gather x -> x_perm (fp32 / bf16): one warp per token reads the row once
+// and writes it to its K rows with 16-byte vectors.
+__global__ void __launch_bounds__(256) k_gather(const uint8_t* __restrict__ x, int T, int K,
+                                                int row_bytes, const int32_t* __restrict__ slot_of,
+                                                uint8_t* __restrict__ x_perm) {
+  const int R = T * K;
+  const int t = blockIdx.x * 8 + warp_id();
+  if (t >= T) return;
+  const int lane = lane_id();
+  int my_slot = lane < K ? slot_of[(size_t)t * K + lane] : 0;
+  const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * row_bytes);
+  const int nvec = row_bytes / 16;
+  for (int c0 = 0; c0 < nvec; c0 += 32 * 4) {
+    uint4 v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int c = c0 + u * 32 + lane;
+      if (c < nvec) v[u] = __ldg(src + c);
+    }
+    for (int k = 0; k < K; ++k) {
+      const int row = __shfl_sync(0xffffffffu, my_slot, k);
+      if ((unsigned)row >= (unsigned)R) continue;  // invalid pair (already reported)
+      uint4* dst = reinterpret_cast<uint4*>(x_perm + (size_t)row * row_bytes);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int c = c0 + u * 32 + lane;
+        if (c < nvec) dst[c] = v[u];
+      }
+    }
+  }
+}
+
+// bf16 row -> E4M3 codes per 1x128 tile, written to the token's K permuted rows
+// and to row R + t (the shared experts' input), with the fp32 tile scales.
+// Scale rule: amax = max|v|, scale = amax / 448, code = E4M3(v * (448 / amax))
+// rounded to nearest even with saturation; amax = 0 gives scale 0, codes 0.
+__global__ void __launch_bounds__(256) k_gather_quant(const __nv_bfloat16* __restrict__ x, int T,
+                                                      int K, int d, int R,
+                                                      const int32_t* __restrict__ slot_of,
+                                                      uint8_t* __restrict__ xq,
+                                                      float* __restrict__ xs) {
+  const int t = blockIdx.x * 8 + warp_id();
+  if (t >= T) return;
+  const int lane = lane_id();
+  const int ng = d / 128;
+  int my_slot = lane < K ? slot_of[(size_t)t * K + lane] : 0;
+  const __nv_bfloat16* xr = x + (size_t)t * d;
+  for (int g = 0; g < ng; ++g) {
+    const uint2 raw = *reinterpret_cast<const uint2*>(xr + g * 128 + lane * 4);
+    const __nv_bfloat162 p0 = *reinterpret_cast<const __nv_bfloat162*>(&raw.x);
+    const __nv_bfloat162 p1 = *reinterpret_cast<const __nv_bfloat162*>(&raw.y);
+    const float v0 = __low2float(p0), v1 = __high2float(p0), v2 = __low2float(p1),
+                v3 = __high2float(p1);
+    const float amax = warp_max(fmaxf(fmaxf(fabsf(v0), fabsf(v1)), fmaxf(fabsf(v2), fabsf(v3))));
+    const float scale = amax > 0.f ? __fdiv_rn(amax, 448.0f) : 0.f;
+    const float inv = amax > 0.f ? __fdiv_rn(448.0f, amax) : 0.f;
+    const uint32_t code = (uint32_t)f32_to_e4m3(__fmul_rn(v0, inv)) |
+                          ((uint32_t)f32_to_e4m3(__fmul_rn(v1, inv)) << 8) |
+                          ((uint32_t)f32_to_e4m3(__fmul_rn(v2, inv)) << 16) |
+                          ((uint32_t)f32_to_e4m3(__fmul_rn(v3, inv)) << 24);
+    for (int k = 0; k <= K; ++k) {
+      const int row = k < K ? __shfl_sync(0xffffffffu, my_slot, k) : R + t;
+      if (k < K && (unsigned)row >= (unsigned)R) continue;  // invalid pair (already reported)
+      *reinterpret_cast<uint32_t*>(xq + (size_t)row * d + g * 128 + lane * 4) = code;
+      if (lane == 0) xs[(size_t)row * ng + g] = scale;
+    }
+  }
+}
+
+// Group table for the grouped GEMMs (block 0) and the permuted-row -> pair map
+// (all blocks).  Groups: shared experts 0..Ks-1 then routed experts 0..N-1.
+__global__ void __launch_bounds__(1024) k_prep_groups(const int32_t* __restrict__ offsets, int T,
+                                                      int K, int Ks, int N, int fp8,
+                                                      int32_t* __restrict__ gtab,
+                                                      const int32_t* __restrict__ slot_of,
+                                                      int32_t* __restrict__ pair_of) {
+  const int R = T * K;
+  if (blockIdx.x > 0) {
+    for (int i = (blockIdx.x - 1) * blockDim.x + threadIdx.x; i < R;
+         i += (gridDim.x - 1) * blockDim.x) {
+      const int row = slot_of[i];
+      if ((unsigned)row < (unsigned)R) pair_of[row] = i;
+      else set_status(MOE_ERR_DEVICE_CHECK);
+    }
+    return;
+  }
+  __shared__ int32_t warp_tot[32];
+  const int n = Ks + N;
+  int32_t* prefix = gtab;
+  int32_t* rows = gtab + n + 1;
+  int32_t* a_row = rows + n;
+  int32_t* a_map = a_row + n;
+  int32_t* expert = a_map + n;
+  int32_t* c_row = expert + n;
+  int32_t* aux = c_row + n;
+  // n <= blockDim.x (checked on the host): one thread per group.
+  const int g = threadIdx.x;
+  int mtiles = 0;
+  if (g < n) {
+    int rws, ar, am, cr, ax;
+    if (g < Ks) {
+      rws = T;
+      am = fp8 ? 1 : 0;
+      ar = fp8 ? R : 0;
+      cr = R + g * T;
+      ax = g;
+    } else {
+      const int j = g - Ks;
+      const int o0 = offsets[j], o1 = offsets[j + 1];
+      rws = o1 - o0;
+      if (rws < 0 || o0 < 0 || o1 > R) { set_status(MOE_ERR_DEVICE_CHECK); rws = 0; }
+      am = 1;
+      ar = o0;
+      cr = o0;
+      ax = -1;
+    }
+    rows[g] = rws;
+    a_row[g] = ar;
+    a_map[g] = am;
+    expert[g] = g;
+    c_row[g] = cr;
+    aux[g] = ax;
+    mtiles = (rws + gemm::BM - 1) / gemm::BM;
+  }
+  int incl = mtiles;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane_id() >= o) incl += y;
+  }
+  if (lane_id() == 31) warp_tot[warp_id()] = incl;
+  __syncthreads();
+  if (warp_id() == 0) {
+    const int nw = blockDim.x / 32;
+    const int wv = lane_id() < nw ? warp_tot[lane_id()] : 0;
+    int wi = wv;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, wi, o);
+      if (lane_id() >= o) wi += y;
+    }
+    if (lane_id() < nw) warp_tot[lane_id()] = wi - wv;
+  }
+  __syncthreads();
+  const int excl = incl - mtiles + warp_tot[warp_id()];
+  if (g < n) prefix[g] = excl;
+  if (g == n - 1) prefix[n] = excl + mtiles;
+}
+
+// h[t] = x_res[t] + sum_{s<Ks} y[t, K+s] + sum_{k<K} y[t, k], fp32, in that order.
+// Each thread owns 8 consecutive elements (bf16) or 4 (fp32) of one token.
+template <bool BF16>
+__global__ void __launch_bounds__(256) k_combine(const void* __restrict__ x_res,
+                                                 const void* __restrict__ y, void* __restrict__ h,
+                                                 int T, int d, int K, int Ks) {
+  constexpr int VEC = BF16 ? 8 : 4;
+  const int per_tok = d / VEC;
+  const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (gid >= (long long)T * per_tok) return;
+  const int t = (int)(gid / per_tok);
+  const int c = (int)(gid - (long long)t * per_tok) * VEC;
+  const int S = K + Ks;
+  float acc[VEC];
+  auto load = [&](const void* base, long long elem_off, float (&v)[VEC]) {
+    if (BF16) {
+      const uint4 raw = __ldg(reinterpret_cast<const uint4*>(
+          reinterpret_cast<const __nv_bfloat16*>(base) + elem_off));
+      const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+      for (int i = 0; i < VEC / 2; ++i) {
+        v[2 * i] = __low2float(p[i]);
+        v[2 * i + 1] = __high2float(p[i]);
+      }
+    } else {
+      const float4 raw = __ldg(reinterpret_cast<const float4*>(
+          reinterpret_cast<const float*>(base) + elem_off));
+      v[0] = raw.x; v[1] = raw.y; v[2] = raw.z; v[3] = raw.w;
+    }
+  };
+  load(x_res, (long long)t * d + c, acc);
+  const long long ybase = (long long)t * S * d + c;
+  for (int s = 0; s < Ks; ++s) {
+    float v[VEC];
+    load(y, ybase + (long long)(K + s) * d, v);
+#pragma unroll
+    for (int i = 0; i < VEC; ++i) acc[i] += v[i];
+  }
+  for (int k = 0; k < K; ++k) {
+    float v[VEC];
+    load(y, ybase + (long long)k * d, v);
+#pragma unroll
+    for (int i = 0; i < VEC; ++i) acc[i] += v[i];
+  }
+  if (BF16) {
+    uint4 out;
+    uint32_t* o = reinterpret_cast<uint32_t*>(&out);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) o[i] = gemm::pack_bf16x2(acc[2 * i], acc[2 * i + 1]);
+    *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(h) + (long long)t * d + c) = out;
+  } else {
+    *reinterpret_cast<float4*>(reinterpret_cast<float*>(h) + (long long)t * d + c) =
+        make_float4(acc[0], acc[1], acc[2], acc[3]);
+  }
+}
+
+// 128x128 block quantisation of bf16 weights to E4M3 (same rule as the
+// activation tiles).  One block of 256 threads per weight block.
+__global__ void __launch_bounds__(256) k_quant_w(const __nv_bfloat16* __restrict__ w, int rows,
+                                                 int cols, uint8_t* __restrict__ q,
+                                                 float* __restrict__ scale) {
+  __shared__ float red[8];
+  const int bc = cols / 128, br = rows / 128;
+  const int b = blockIdx.x;  // over batch * br * bc
+  const int mat = b / (br * bc), rem = b - mat * br * bc;
+  const int bi = rem / bc, bj = rem - bi * bc;
+  const __nv_bfloat16* src = w + (size_t)mat * rows * cols + (size_t)bi * 128 * cols + bj * 128;
+  uint8_t* dst = q + (size_t)mat * rows * cols + (size_t)bi * 128 * cols + bj * 128;
+  // each thread: rows r = tid/2 (128 rows, 2 threads per row), 64 columns
+  const int r = threadIdx.x >> 1, half = threadIdx.x & 1;
+  const __nv_bfloat16* rp = src + (size_t)r * cols + half * 64;
+  float v[64];
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const uint4 raw = *reinterpret_cast<const uint4*>(rp + i * 8);
+    const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      v[i * 8 + 2 * j] = __low2float(p[j]);
+      v[i * 8 + 2 * j + 1] = __high2float(p[j]);
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 64; ++i) amax = fmaxf(amax, fabsf(v[i]));
+  amax = warp_max(amax);
+  if (lane_id() == 0) red[warp_id()] = amax;
+  __syncthreads();
+  amax = red[0];
+#pragma unroll
+  for (int i = 1; i < 8; ++i) amax = fmaxf(amax, red[i]);
+  const float sc = amax > 0.f ? __fdiv_rn(amax, 448.0f) : 0.f;
+  const float inv = amax > 0.f ? __fdiv_rn(448.0f, amax) : 0.f;
+  uint8_t* dp = dst + (size_t)r * cols + half * 64;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    uint32_t wds[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int o = i * 16 + j * 4;
+      wds[j] = (uint32_t)f32_to_e4m3(__fmul_rn(v[o], inv)) |
+               ((uint32_t)f32_to_e4m3(__fmul_rn(v[o + 1], inv)) << 8) |
+               ((uint32_t)f32_to_e4m3(__fmul_rn(v[o + 2], inv)) << 16) |
+               ((uint32_t)f32_to_e4m3(__fmul_rn(v[o + 3], inv)) << 24);
+    }
+    *reinterpret_cast<uint4*>(dp + i * 16) = make_uint4(wds[0], wds[1], wds[2], wds[3]);
+  }
+  if (threadIdx.x == 0) scale[(size_t)mat * br * bc + bi * bc + bj] = sc;
+}
+
+}  // namespace perm
+}  // namespace moe

@@ -1,0 +1,201 @@
+/*
+ * moe.h -- C ABI of the B200 (sm_100a) DeepSeekMoE layer forward.
+ *
+ * One MoE layer computes, for every token t,
+ *
+ *   h_t = x_res_t + sum_{i<Ks} FFN_i(u_t) + sum_{k<K} g_{t,k} FFN_{Ks+idx_{t,k}}(u_t)
+ *
+ * with SwiGLU experts FFN(v) = W_down (SiLU(W_gate v) * (W_up v)).
+ *   - output equation: "DeepSeek Technical Report: MoE Architecture", §1.1(2)
+ *     (DeepSeekMoE equation with Ks shared experts), equation [1] of §5.3;
+ *   - SwiGLU experts: "DeepSeek-V3 아키텍처 둘러보기", the invariant-core
+ *     section (the MLP is SwiGLU);
+ *   - gating: §2.3 (softmax gate, DeepSeekMoE / V2) and §3.3 with equations
+ *     [3], [4] of §5.3 (sigmoid affinity, bias used for selection only) of
+ *     the MoE Architecture report;
+ *   - FP8: §3.6 of the same report (E4M3, 1x128 activation tiles, 128x128
+ *     weight blocks, fp32 accumulation with promotion every 128 elements).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  T tokens, d hidden, Ks = n_shared, N = n_routed, K = top_k, I = inter,
+ *  E = Ks + N experts, R = T*K routed rows.
+ *  - All pointers are DEVICE pointers (except `desc`, a host pointer) to
+ *    row-major contiguous arrays, 16-byte aligned.  The caller allocates and
+ *    owns every buffer, including the workspace; the library allocates
+ *    nothing on these paths.
+ *  - Shared experts are experts 0..Ks-1 of w_gu / w_down; routed expert j
+ *    (0 <= j < N) is expert Ks+j.  topk_idx holds routed indices j.
+ *  - w_gu [E, 2I, d]: rows 0..I-1 of an expert are W_gate, rows I..2I-1 W_up.
+ *    w_down [E, d, I].
+ *  - Every call validates its arguments synchronously and returns a status;
+ *    nothing is thrown across the ABI.  Work is enqueued asynchronously on
+ *    `stream`.  Problems detected on the device (an index out of range, a
+ *    counts array that disagrees with topk_idx, a bounded wait that ran out)
+ *    are recorded in a per-device status word read by moe_last_device_status.
+ *  - Results are bit-identical from run to run (no floating-point atomics).
+ *  - Concurrent calls that share a workspace race; give each stream its own.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,   /* a size, pointer, alignment or mode is not accepted */
+  MOE_ERR_UNSUPPORTED = 2,   /* valid layer, but a shape this build does not handle */
+  MOE_ERR_WORKSPACE = 3,     /* ws_bytes below moe_workspace_size(desc) */
+  MOE_ERR_CUDA = 4,          /* a CUDA runtime/driver call or a launch failed */
+  MOE_ERR_TIMEOUT = 5,       /* a device-side bounded wait expired (device status) */
+  MOE_ERR_DEVICE_CHECK = 6   /* a device-side consistency check failed (device status) */
+} moe_status;
+
+typedef enum { MOE_GATE_SOFTMAX = 0, MOE_GATE_SIGMOID = 1 } moe_gate;
+
+typedef enum { MOE_DT_F32 = 0, MOE_DT_BF16 = 1, MOE_DT_E4M3 = 2 } moe_dtype;
+
+/* The layer's problem statement.  Accepted dtype pairs (act_dtype, w_dtype):
+ *   (F32, F32)   fp32 activations and weights; GEMMs on tf32 tensor cores,
+ *                router in fp32; H, expert outputs and h in fp32.
+ *   (BF16, BF16) bf16 activations and weights, fp32 accumulation; H, expert
+ *                outputs and h in bf16.
+ *   (BF16, E4M3) bf16 x and router (gating stays BF16), E4M3 expert weights
+ *                with fp32 128x128 block scales; x and H quantised to E4M3 per
+ *                1x128 tile; expert outputs and h in bf16. */
+typedef struct moe_layer_desc {
+  int32_t T;           /* tokens, >= 0 */
+  int32_t d;           /* hidden size */
+  int32_t n_shared;    /* Ks >= 0 */
+  int32_t n_routed;    /* N, 1..512 */
+  int32_t top_k;       /* K, 1..min(N, 16) */
+  int32_t inter;       /* I, expert width */
+  int32_t gate;        /* moe_gate */
+  int32_t renorm;      /* 1: g = s / sum_selected(s); 0: g = s */
+  float route_scale;   /* multiplies g after normalisation (1.0; 2.5 for V3) */
+  int32_t n_group;     /* expert groups for group-limited routing (1 = none) */
+  int32_t topk_group;  /* groups kept; a group's score is the sum of its two largest keys */
+  int32_t act_dtype;   /* moe_dtype */
+  int32_t w_dtype;     /* moe_dtype */
+} moe_layer_desc;
+
+/* Shape rules (MOE_ERR_INVALID_ARG otherwise):
+ *   d, I multiples of 64 (bf16), 32 (f32) or 128 (E4M3); I >= 16; d <= 65536;
+ *   N % n_group == 0, 1 <= topk_group <= n_group <= 32, N/n_group >= 2 when
+ *   n_group > 1, topk_group*(N/n_group) >= K; bias only with sigmoid gating;
+ *   R + Ks*T < 2^31. */
+
+/* Bytes of workspace moe_forward needs for `desc` (the other entry points need
+ * no more than this).  0 if desc is invalid. */
+size_t moe_workspace_size(const moe_layer_desc* desc);
+
+/* (a) Gating.  Router logits l = x W_r^T (fp32 accumulate), affinities s
+ * (softmax over the N routed experts, or sigmoid), selection keys s + bias,
+ * group limit, top-K with ties to the lower expert index, and gate weights
+ * g = route_scale * s (/ sum of the selected s when renorm).  The bias
+ * changes the selection only, never g.
+ *   x [T, d] act_dtype;  w_router [N, d] act_dtype;  bias [N] fp32 or NULL
+ *   topk_idx [T, K] int32 out (ordered by key desc, index asc)
+ *   topk_w   [T, K] fp32 out
+ *   counts   [N] int32 out (tokens per routed expert) */
+moe_status moe_route(const moe_layer_desc* desc, const void* x, const void* w_router,
+                     const float* bias, int32_t* topk_idx, float* topk_w, int32_t* counts,
+                     void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/* (b) Token -> expert permutation.  offsets = exclusive scan of the counts;
+ * the pair (t, k) with expert e = topk_idx[t,k] goes to permuted row
+ * slot_of[t*K+k] = offsets[e] + #{t' < t : e in topk_idx[t']} (stable by
+ * token), perm_src[row] = t, and x_perm[row] = x[t] (E4M3: the 1x128
+ * quantised row and its scales).
+ *   counts [N] int32 in: must equal the histogram of topk_idx (checked on the
+ *     device; a mismatch or an index outside [0, N) sets MOE_ERR_DEVICE_CHECK)
+ *   offsets [N+1], perm_src [R], slot_of [R] int32 out
+ *   x_perm  [R, d] act_dtype (F32/BF16), or [R + T, d] E4M3 bytes whose rows
+ *     R..R+T-1 hold the quantised x in token order (the shared experts' input)
+ *   x_perm_scale [R + T, d/128] fp32 out for E4M3, NULL otherwise */
+moe_status moe_permute(const moe_layer_desc* desc, const void* x, const int32_t* topk_idx,
+                       const int32_t* counts, int32_t* offsets, int32_t* perm_src,
+                       int32_t* slot_of, void* x_perm, float* x_perm_scale, void* ws,
+                       size_t ws_bytes, cudaStream_t stream);
+
+/* (c) Shared and routed experts.  One persistent tcgen05 grouped GEMM computes
+ * H = SiLU(A W_gate^T) * (A W_up^T) for every expert (A = x for the shared
+ * experts, the expert's x_perm rows for routed ones); a second computes
+ * Y = H W_down^T and scatters each row, times g_{t,k} (1 for shared experts),
+ * to y_slots[t, k] (routed) or y_slots[t, K+s] (shared expert s).
+ *   x [T, d] (F32/BF16 shared-expert input; unused for E4M3)
+ *   x_perm, x_perm_scale, offsets, slot_of: as written by moe_permute
+ *   perm_src: as written by moe_permute (accepted for symmetry; unused)
+ *   topk_w [T, K] fp32
+ *   w_gu [E, 2I, d], w_down [E, d, I] in w_dtype; for E4M3 their fp32 block
+ *     scales w_gu_scale [E, 2I/128, d/128], w_down_scale [E, d/128, I/128]
+ *   y_slots [T, K+Ks, d] out: fp32 for F32, bf16 otherwise */
+moe_status moe_grouped_swiglu(const moe_layer_desc* desc, const void* x, const void* x_perm,
+                              const float* x_perm_scale, const int32_t* offsets,
+                              const int32_t* perm_src, const int32_t* slot_of,
+                              const float* topk_w, const void* w_gu, const float* w_gu_scale,
+                              const void* w_down, const float* w_down_scale, void* y_slots,
+                              void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/* (d) Weighted combine and residual: h[t] = x_res[t] + sum_{s<Ks} y[t, K+s]
+ * + sum_{k<K} y[t, k], accumulated in fp32 in that order.
+ *   x_residual [T, d] act_dtype; y_slots as above; h [T, d] out (fp32 for F32,
+ *   bf16 otherwise). */
+moe_status moe_combine(const moe_layer_desc* desc, const void* x_residual, const void* y_slots,
+                       void* h, cudaStream_t stream);
+
+/* The whole layer: moe_route, moe_permute, moe_grouped_swiglu, moe_combine,
+ * with every intermediate in the workspace.
+ *   x_residual: NULL means x (pass RMSNorm(u) as x and u as x_residual to
+ *     keep the residual outside the normalisation).
+ *   topk_idx [T,K], counts [N]: optional int32 copies of the routing result. */
+moe_status moe_forward(const moe_layer_desc* desc, const void* x, const void* x_residual,
+                       const void* w_router, const float* bias, const void* w_gu,
+                       const float* w_gu_scale, const void* w_down, const float* w_down_scale,
+                       void* h, int32_t* topk_idx, int32_t* counts, void* ws, size_t ws_bytes,
+                       cudaStream_t stream);
+
+/* Offline FP8 quantisation of weights in 128x128 blocks (not on the hot path).
+ * w_bf16 [batch, rows, cols] bf16 in; w_e4m3 [batch, rows, cols] bytes out;
+ * scale [batch, rows/128, cols/128] fp32 out.  rows, cols multiples of 128.
+ * Rule per block: amax = max|w|, scale = amax/448, code = E4M3_rn_satfinite(
+ * w * (448/amax)) in fp32; an all-zero block gets scale 0 and zero codes. */
+moe_status moe_quantize_fp8_blockwise(const void* w_bf16, int32_t rows, int32_t cols,
+                                      int32_t batch, void* w_e4m3, float* scale,
+                                      cudaStream_t stream);
+
+/* Human-readable name of a status. */
+const char* moe_status_string(moe_status status);
+
+/* Synchronises `stream`, then returns and clears the current device's status
+ * word (MOE_OK if no device-side check fired since the last call). */
+moe_status moe_last_device_status(cudaStream_t stream);
+
+/* Stage timing.  While set on the calling host thread, moe_forward records
+ * events[0] before routing, [1] after routing, [2] after the permutation,
+ * [3] after the gate/up GEMM, [4] after the down GEMM and [5] after the
+ * combine, on the call's stream; moe_grouped_swiglu records [2], [3] and [4]
+ * around its own launches.  n must be 6 (events owned by the caller); pass
+ * NULL, 0 to stop. */
+moe_status moe_trace_events(cudaEvent_t* events, int32_t n);
+
+/* Number of kernels moe_forward launches for `desc` (0 if invalid). */
+int32_t moe_forward_launch_count(const moe_layer_desc* desc);
+
+/* Self-test of the device-side bounded wait: launches one block that waits on
+ * a shared-memory barrier nothing ever completes, gives up after limit_us
+ * microseconds (1..1000000), records MOE_ERR_TIMEOUT in the status word and
+ * returns.  The context stays usable. */
+moe_status moe_selftest_bounded_wait(uint32_t limit_us, cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

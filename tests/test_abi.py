@@ -1,0 +1,129 @@
+"""The C ABI library: it loads, exports every symbol include/moe.h declares,
+and its host-side validation rejects bad problem statements (no GPU needed:
+these calls return before touching CUDA)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import forward_moe_route_b200 as moe
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    with open(os.path.join(ROOT, "include", "moe.h")) as f:
+        text = f.read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[a-z_0-9]+\s*\*?\s+(moe_[a-z_0-9]+)\s*\(", text, re.M)
+    return sorted(set(names))
+
+
+def test_every_declared_symbol_is_exported():
+    names = declared_functions()
+    assert len(names) >= 11
+    for n in names:
+        assert hasattr(moe.lib(), n), f"{n} declared but not exported"
+    assert set(names) == set(moe.EXPORTED)
+
+
+def test_desc_struct_matches_header_layout():
+    # 13 four-byte fields, no padding
+    assert ctypes.sizeof(moe.MoeLayerDesc) == 13 * 4
+
+
+def v3(**kw):
+    base = dict(T=16384, d=7168, n_shared=1, n_routed=256, top_k=8, inter=2048, gate="sigmoid",
+                renorm=True, route_scale=2.5, n_group=8, topk_group=4, dtype="bf16")
+    base.update(kw)
+    return moe.make_desc(**base)
+
+
+def test_workspace_size_valid_configs():
+    assert moe.moe_workspace_size(v3()) > 4e9
+    assert moe.moe_workspace_size(v3(dtype="e4m3")) > 0
+    tiny = moe.make_desc(64, 256, 1, 16, 4, 64, "softmax", True, 1.0, 1, 1, "f32")
+    assert moe.moe_workspace_size(tiny) > 0
+    assert moe.moe_workspace_size(v3(T=0)) > 0
+
+
+@pytest.mark.parametrize("kw", [
+    dict(top_k=300),                      # K > N
+    dict(top_k=17),                       # K above the supported maximum
+    dict(n_group=8, topk_group=1),        # 1 group of 32 experts < K? (32 >= 8: valid) -> see below
+    dict(n_group=7),                      # N not divisible by n_group
+    dict(n_group=8, topk_group=9),        # topk_group > n_group
+    dict(n_routed=16, n_group=16, topk_group=3, top_k=8),  # groups of 1 expert
+    dict(d=7100),                         # d not a multiple of 64 (bf16)
+    dict(inter=8),
+    dict(dtype="e4m3", d=7168 + 64),      # FP8 needs multiples of 128
+    dict(T=-1),
+    dict(route_scale=0.0),
+    dict(route_scale=float("nan")),
+    dict(n_routed=0),
+    dict(n_routed=1024, n_group=1, topk_group=1),
+    dict(n_shared=65),
+])
+def test_invalid_descriptors(kw):
+    d = v3(**kw)
+    if kw == dict(n_group=8, topk_group=1):
+        assert moe.moe_workspace_size(d) > 0   # 1 group of 32 experts holds K=8: valid
+        return
+    assert moe.moe_workspace_size(d) == 0
+
+
+def test_group_capacity_rule():
+    # topk_group * (N / n_group) must be >= K
+    assert moe.moe_workspace_size(v3(n_routed=32, n_group=8, topk_group=1, top_k=8)) == 0
+    assert moe.moe_workspace_size(v3(n_routed=32, n_group=8, topk_group=2, top_k=8)) > 0
+
+
+def test_bad_dtype_pair():
+    d = v3()
+    d.act_dtype, d.w_dtype = moe.DT_E4M3, moe.DT_E4M3
+    assert moe.moe_workspace_size(d) == 0
+    d.act_dtype, d.w_dtype = moe.DT_F32, moe.DT_BF16
+    assert moe.moe_workspace_size(d) == 0
+
+
+def test_entry_points_reject_before_touching_cuda():
+    L = moe.lib()
+    bad = v3(top_k=300)
+    assert L.moe_route(ctypes.byref(bad), None, None, None, None, None, None, None, 0,
+                       None) == moe.ERR_INVALID_ARG
+    good = v3()
+    # bias with softmax gating is not part of the method
+    sm = v3(gate="softmax", n_group=1, topk_group=1)
+    assert L.moe_route(ctypes.byref(sm), 16, 16, 16, 16, 16, 16, 16, 1 << 40,
+                       None) == moe.ERR_INVALID_ARG
+    # null / misaligned pointers
+    assert L.moe_route(ctypes.byref(good), None, 16, None, 16, 16, 16, 16, 1 << 40,
+                       None) == moe.ERR_INVALID_ARG
+    assert L.moe_route(ctypes.byref(good), 17, 16, None, 16, 16, 16, 16, 1 << 40,
+                       None) == moe.ERR_INVALID_ARG
+    # workspace too small
+    assert L.moe_route(ctypes.byref(good), 16, 16, None, 16, 16, 16, 16, 1024,
+                       None) == moe.ERR_WORKSPACE
+    assert L.moe_forward(ctypes.byref(good), 16, None, 16, None, 16, None, 16, None, 16, None,
+                         None, 16, 1024, None) == moe.ERR_WORKSPACE
+    # FP8 forward needs the weight scales
+    f8 = v3(dtype="e4m3")
+    assert L.moe_forward(ctypes.byref(f8), 16, None, 16, None, 16, None, 16, None, 16, None,
+                         None, 16, 1 << 40, None) == moe.ERR_INVALID_ARG
+    # permute: E4M3 needs the scale output, bf16 must not get one
+    assert L.moe_permute(ctypes.byref(good), 16, 16, 16, 16, 16, 16, 16, 16, 16, 1 << 40,
+                         None) == moe.ERR_INVALID_ARG
+    assert L.moe_quantize_fp8_blockwise(16, 100, 128, 1, 16, 16, None) == moe.ERR_INVALID_ARG
+    assert L.moe_selftest_bounded_wait(0, None) == moe.ERR_INVALID_ARG
+
+
+def test_status_strings():
+    for s in range(7):
+        assert moe.moe_status_string(s)
+    assert moe.moe_status_string(99) == "unknown status"
+
+
+def test_launch_count():
+    assert moe.moe_forward_launch_count(v3()) == 10
+    assert moe.moe_forward_launch_count(v3(top_k=300)) == 0

@@ -256,6 +256,9 @@ def run_ours(args, cfg):
 
     # ---- timed region: K steps, events on the launching stream
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    for row in ev:            # torch creates its events lazily, at the first record
+        for e in row:
+            e.record(stream)
     clocks = ClockSampler(int(os.environ.get("CUDA_VISIBLE_DEVICES", str(local)).split(",")[0])
                           if os.environ.get("CUDA_VISIBLE_DEVICES", "").replace(",", "").isdigit()
                           else local)

@@ -60,6 +60,7 @@ _SIGS = {
     "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "moe_last_device_status": (ctypes.c_int, [_P]),
     "moe_forward_launch_count": (ctypes.c_int32, [_D]),
+    "moe_last_error_message": (ctypes.c_char_p, []),
     "moe_trace_events": (ctypes.c_int, [ctypes.POINTER(ctypes.c_void_p), ctypes.c_int32]),
     "moe_selftest_bounded_wait": (ctypes.c_int, [ctypes.c_uint32, _P]),
 }
@@ -94,6 +95,8 @@ def _stream(stream) -> Optional[int]:
 
 def _check(rc: int, where: str) -> None:
     if rc != OK:
+        if rc == ERR_CUDA:
+            where = f"{where} [{_lib.moe_last_error_message().decode()}]"
         raise MoeError(rc, where)
 
 
@@ -189,7 +192,10 @@ def moe_trace_events(events) -> None:
         _trace_keep = None
         _check(_lib.moe_trace_events(None, 0), "moe_trace_events")
         return
-    arr = (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events])
+    handles = [e.cuda_event for e in events]
+    if not all(handles):
+        raise ValueError("trace events must exist: record each torch.cuda.Event once first")
+    arr = (ctypes.c_void_p * len(events))(*handles)
     _trace_keep = arr
     _check(_lib.moe_trace_events(arr, len(events)), "moe_trace_events")
 

@@ -6,6 +6,7 @@
 #include <cudaTypedefs.h>
 
 #include <cmath>
+#include <cstdio>
 #include <cstring>
 #include <mutex>
 
@@ -149,6 +150,20 @@ moe_status device_setup(int* sms) {
   return MOE_OK;
 }
 
+// Text of the last CUDA failure on this host thread (moe_last_error_message).
+thread_local char t_errmsg[256] = "";
+
+moe_status cuda_fail(cudaError_t e, const char* where) {
+  snprintf(t_errmsg, sizeof(t_errmsg), "%s: %s (%s)", where, cudaGetErrorName(e),
+           cudaGetErrorString(e));
+  return MOE_ERR_CUDA;
+}
+
+inline moe_status launched(const char* where) {
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, where);
+}
+
 // 2-D K-major tensor map with 128-byte swizzle: rows of `inner` elements,
 // box = (128 bytes of K) x box_rows.
 moe_status make_tmap(CUtensorMap* m, const void* base, size_t esz, uint64_t inner, uint64_t rows,
@@ -163,7 +178,23 @@ moe_status make_tmap(CUtensorMap* m, const void* base, size_t esz, uint64_t inne
   CUresult r = g_encode(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? MOE_OK : MOE_ERR_CUDA;
+  if (r != CUDA_SUCCESS) {
+    snprintf(t_errmsg, sizeof(t_errmsg), "cuTensorMapEncodeTiled: CUresult %d (rows %llu, "
+             "inner %llu, box rows %u)", (int)r, (unsigned long long)rows,
+             (unsigned long long)inner, box_rows);
+    return MOE_ERR_CUDA;
+  }
+  return MOE_OK;
+}
+
+
+
+// Stage-timing events of the calling host thread (moe_trace_events).
+thread_local cudaEvent_t* t_events = nullptr;
+inline moe_status trace(int i, cudaStream_t st) {
+  if (!t_events) return MOE_OK;
+  const cudaError_t e = cudaEventRecord(t_events[i], st);
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "cudaEventRecord (stage trace)");
 }
 
 int pick_stages(int bn, int n_groups) {
@@ -188,16 +219,12 @@ moe_status launch_gemm(const CUtensorMap& a0, const CUtensorMap& a1, const CUten
   if (args.tmem_cols > 512) return MOE_ERR_UNSUPPORTED;
   const size_t smem = gemm::smem_bytes(args.bn, args.stages, ng);
   gemm::k_grouped_gemm<KIND, EPI><<<grid, gemm::NUM_THREADS, smem, st>>>(a0, a1, b, args);
-  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+  return launched("grouped GEMM launch");
 }
 
-inline moe_status launched() { return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
-// Stage-timing events of the calling host thread (moe_trace_events).
-thread_local cudaEvent_t* t_events = nullptr;
-inline void trace(int i, cudaStream_t st) {
-  if (t_events) cudaEventRecord(t_events[i], st);
-}
+
+
 
 route::Params route_params(const moe_layer_desc& s) {
   route::Params p;
@@ -226,7 +253,7 @@ moe_status do_route(const moe_layer_desc& s, const Dims& D, const Layout& L, con
   const int N = (int)D.N;
   if (D.T == 0) {
     route::k_zero_i32<<<1, 256, 0, st>>>(counts, N);
-    return launched();
+    return launched("k_zero_i32");
   }
   if (D.f32) {
     route::k_zero_i32<<<1, 256, 0, st>>>(counts, N);
@@ -238,7 +265,7 @@ moe_status do_route(const moe_layer_desc& s, const Dims& D, const Layout& L, con
     else if (N <= 128) launch_route_f32<4>(xf, wf, dd, bias, p, topk_idx, topk_w, counts, st);
     else if (N <= 256) launch_route_f32<8>(xf, wf, dd, bias, p, topk_idx, topk_w, counts, st);
     else launch_route_f32<16>(xf, wf, dd, bias, p, topk_idx, topk_w, counts, st);
-    return launched();
+    return launched("k_route_f32");
   }
   // bf16 router GEMM on tensor cores: logits [T, N] fp32 (counts zeroed in its prologue)
   float* logits = reinterpret_cast<float*>(ws + L.logits);
@@ -273,7 +300,7 @@ moe_status do_route(const moe_layer_desc& s, const Dims& D, const Layout& L, con
   else if (N <= 128) launch_topk<4>(logits, bias, p, topk_idx, topk_w, counts, st);
   else if (N <= 256) launch_topk<8>(logits, bias, p, topk_idx, topk_w, counts, st);
   else launch_topk<16>(logits, bias, p, topk_idx, topk_w, counts, st);
-  return launched();
+  return launched("k_topk");
 }
 
 moe_status do_permute(const Dims& D, const Layout& L, const void* x, const int32_t* topk_idx,
@@ -284,7 +311,7 @@ moe_status do_permute(const Dims& D, const Layout& L, const void* x, const int32
   int32_t* hist = reinterpret_cast<int32_t*>(ws + L.hist);
   if (T == 0) {
     route::k_zero_i32<<<1, 256, 0, st>>>(offsets, N + 1);
-    return launched();
+    return launched("k_zero_i32");
   }
   perm::k_hist<<<D.n_chunks, 256, N * 4, st>>>(topk_idx, T, K, N, hist);
   perm::k_scan<<<1, 1024, 0, st>>>(hist, D.n_chunks, N, counts, offsets);
@@ -298,7 +325,7 @@ moe_status do_permute(const Dims& D, const Layout& L, const void* x, const int32
                                                 (int)(D.d * D.x_esz), slot_of,
                                                 static_cast<uint8_t*>(x_perm));
   }
-  return launched();
+  return launched("permutation kernels");
 }
 
 moe_status do_grouped(const Dims& D, const Layout& L, const void* x, const void* x_perm,
@@ -312,10 +339,11 @@ moe_status do_grouped(const Dims& D, const Layout& L, const void* x, const void*
   int32_t* pair_of = reinterpret_cast<int32_t*>(ws + L.pair_of);
   void* hbuf = ws + L.hbuf;
   const int prep_blocks = 1 + (int)((D.R + 1023) / 1024 < 4 * sms ? (D.R + 1023) / 1024 : 4 * sms);
-  trace(2, st);
+  moe_status rc = trace(2, st);
+  if (rc != MOE_OK) return rc;
   perm::k_prep_groups<<<prep_blocks, 1024, 0, st>>>(offsets, (int)D.T, (int)D.K, (int)D.Ks,
                                                     (int)D.N, 0, gtab, slot_of, pair_of);
-  moe_status rc = launched();
+  rc = launched("k_prep_groups");
   if (rc != MOE_OK) return rc;
 
   const size_t esz = D.op_esz;
@@ -356,7 +384,7 @@ moe_status do_grouped(const Dims& D, const Layout& L, const void* x, const void*
     rc = kind == 0 ? launch_gemm<0, gemm::EPI_SWIGLU>(ta0, ta1, tb, a, grid, st)
                    : launch_gemm<1, gemm::EPI_SWIGLU>(ta0, ta1, tb, a, grid, st);
     if (rc != MOE_OK) return rc;
-    trace(3, st);
+    if ((rc = trace(3, st)) != MOE_OK) return rc;
   }
   // GEMM2: Y = H Wd^T, times g, scattered to the token-major slots
   {
@@ -389,7 +417,7 @@ moe_status do_grouped(const Dims& D, const Layout& L, const void* x, const void*
     const int grid = (int)(tiles < sms ? tiles : sms);
     rc = kind == 0 ? launch_gemm<0, gemm::EPI_SCATTER>(ta, ta, tb, a, grid, st)
                    : launch_gemm<1, gemm::EPI_SCATTER>(ta, ta, tb, a, grid, st);
-    if (rc == MOE_OK) trace(4, st);
+    if (rc == MOE_OK) rc = trace(4, st);
   }
   return rc;
 }
@@ -405,7 +433,7 @@ moe_status do_combine(const Dims& D, const void* x_res, const void* y, void* h, 
   else
     perm::k_combine<true><<<blocks, 256, 0, st>>>(x_res, y, h, (int)D.T, (int)D.d, (int)D.K,
                                                   (int)D.Ks);
-  return launched();
+  return launched("k_combine<true>");
 }
 
 __global__ void k_selftest_wait(uint64_t limit_ns) {
@@ -553,10 +581,10 @@ moe_status moe_forward(const moe_layer_desc* desc, const void* x, const void* x_
   void* x_perm = w8 + L.x_perm;
   float* x_perm_scale = D.fp8 ? reinterpret_cast<float*>(w8 + L.x_perm_scale) : nullptr;
   void* y = w8 + L.y_slots;
-  trace(0, stream);
+  if ((rc = trace(0, stream)) != MOE_OK) return rc;
   if ((rc = do_route(*desc, D, L, x, w_router, bias, idx, tw, cnt, w8, sms, stream)) != MOE_OK)
     return rc;
-  trace(1, stream);
+  if ((rc = trace(1, stream)) != MOE_OK) return rc;
   if ((rc = do_permute(D, L, x, idx, cnt, offsets, perm_src, slot_of, x_perm, x_perm_scale, w8,
                        stream)) != MOE_OK)
     return rc;
@@ -564,7 +592,7 @@ moe_status moe_forward(const moe_layer_desc* desc, const void* x, const void* x_
                        stream)) != MOE_OK)
     return rc;
   rc = do_combine(D, x_residual ? x_residual : x, y, h, stream);
-  if (rc == MOE_OK) trace(5, stream);
+  if (rc == MOE_OK) rc = trace(5, stream);
   return rc;
 }
 
@@ -579,7 +607,7 @@ moe_status moe_quantize_fp8_blockwise(const void* w_bf16, int32_t rows, int32_t 
   perm::k_quant_w<<<(unsigned)blocks, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(w_bf16),
                                                          rows, cols,
                                                          static_cast<uint8_t*>(w_e4m3), scale);
-  return launched();
+  return launched("k_quant_w");
 }
 
 const char* moe_status_string(moe_status status) {
@@ -610,6 +638,8 @@ moe_status moe_trace_events(cudaEvent_t* events, int32_t n) {
   return MOE_OK;
 }
 
+const char* moe_last_error_message(void) { return t_errmsg; }
+
 int32_t moe_forward_launch_count(const moe_layer_desc* desc) {
   Dims D;
   if (fill_dims(desc, &D) != MOE_OK) return 0;
@@ -621,7 +651,7 @@ int32_t moe_forward_launch_count(const moe_layer_desc* desc) {
 moe_status moe_selftest_bounded_wait(uint32_t limit_us, cudaStream_t stream) {
   if (limit_us < 1 || limit_us > 1000000) return MOE_ERR_INVALID_ARG;
   k_selftest_wait<<<1, 32, 0, stream>>>((uint64_t)limit_us * 1000ull);
-  return launched();
+  return launched("k_selftest_wait");
 }
 
 }  // extern "C"

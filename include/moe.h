@@ -185,6 +185,11 @@ moe_status moe_last_device_status(cudaStream_t stream);
  * NULL, 0 to stop. */
 moe_status moe_trace_events(cudaEvent_t* events, int32_t n);
 
+/* Text describing the last MOE_ERR_CUDA returned on the calling host thread
+ * (the failing call and the CUDA error name); "" if none.  Owned by the
+ * library, valid until the next call on this thread. */
+const char* moe_last_error_message(void);
+
 /* Number of kernels moe_forward launches for `desc` (0 if invalid). */
 int32_t moe_forward_launch_count(const moe_layer_desc* desc);
 

@@ -50,6 +50,7 @@ _SIGS = {
     "moe_workspace_size": (ctypes.c_size_t, [_D]),
     "moe_route": (ctypes.c_int, [_D, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "moe_permute": (ctypes.c_int, [_D, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "moe_permute_noalloc": (ctypes.c_int, [_D, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "moe_grouped_swiglu": (ctypes.c_int, [_D, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                                           ctypes.c_size_t, _P]),
     "moe_combine": (ctypes.c_int, [_D, _P, _P, _P, _P]),
@@ -145,6 +146,14 @@ def moe_permute(desc, x, topk_idx, counts, offsets, perm_src, slot_of, x_perm, x
                             _ptr(offsets), _ptr(perm_src), _ptr(slot_of), _ptr(x_perm),
                             _ptr(x_perm_scale), _ptr(ws), ws.numel() if ws is not None else 0,
                             _stream(stream)), "moe_permute")
+
+
+def moe_permute_noalloc(desc, x, topk_idx, counts, offsets, perm_src, slot_of, x_perm,
+                        x_perm_scale, stream=None) -> None:
+    """moe_permute without a workspace (fixed 1 MiB device scratch; see include/moe.h)."""
+    _check(_lib.moe_permute_noalloc(ctypes.byref(desc), _ptr(x), _ptr(topk_idx), _ptr(counts),
+                                    _ptr(offsets), _ptr(perm_src), _ptr(slot_of), _ptr(x_perm),
+                                    _ptr(x_perm_scale), _stream(stream)), "moe_permute_noalloc")
 
 
 def moe_grouped_swiglu(desc, x, x_perm, x_perm_scale, offsets, perm_src, slot_of, topk_w, w_gu,

@@ -458,6 +458,33 @@ __global__ void k_selftest_wait(uint64_t limit_ns) {
   __syncthreads();
 }
 
+
+// ----------------------------------------------------------------------------- no-allocation permute
+// Scratch of moe_permute_noalloc: the per-chunk histogram, in a fixed device
+// array that every device loading this library holds until the process exits.
+static __device__ __align__(256) int32_t g_noalloc_hist[MOE_NOALLOC_HIST_INTS];
+
+// Device address of g_noalloc_hist, looked up once per device (host code
+// cannot use the symbol itself: on the host it names a stand-in, not device
+// memory).
+int32_t* g_noalloc_ptr[kMaxDevices] = {};
+
+moe_status noalloc_scratch(int32_t** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return MOE_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_hist);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(no-alloc scratch)");
+    g_noalloc_ptr[dev] = static_cast<int32_t*>(p);
+  }
+  *out = g_noalloc_ptr[dev];
+  return MOE_OK;
+}
+
 }  // namespace
 
 // ============================================================================= C ABI
@@ -652,6 +679,56 @@ moe_status moe_selftest_bounded_wait(uint32_t limit_us, cudaStream_t stream) {
   if (limit_us < 1 || limit_us > 1000000) return MOE_ERR_INVALID_ARG;
   k_selftest_wait<<<1, 32, 0, stream>>>((uint64_t)limit_us * 1000ull);
   return launched("k_selftest_wait");
+}
+
+moe_status moe_permute_noalloc(const moe_layer_desc* desc, const void* x,
+                               const int32_t* topk_idx, const int32_t* counts, int32_t* offsets,
+                               int32_t* perm_src, int32_t* slot_of, void* x_perm,
+                               float* x_perm_scale, cudaStream_t stream) {
+  Dims D;
+  moe_status rc = fill_dims(desc, &D);
+  if (rc != MOE_OK) return rc;
+  if (!offsets || !aligned16(offsets)) return MOE_ERR_INVALID_ARG;
+  if (D.T > 0) {
+    if (!x || !topk_idx || !counts || !perm_src || !slot_of || !x_perm || !aligned16(x) ||
+        !aligned16(topk_idx) || !aligned16(perm_src) || !aligned16(slot_of) ||
+        !aligned16(x_perm))
+      return MOE_ERR_INVALID_ARG;
+    if (D.fp8 != (x_perm_scale != nullptr)) return MOE_ERR_INVALID_ARG;
+    if (x_perm_scale && !aligned16(x_perm_scale)) return MOE_ERR_INVALID_ARG;
+  }
+  const int64_t need = (int64_t)D.n_chunks * D.N;
+  if (need > MOE_NOALLOC_HIST_INTS) {
+    snprintf(t_errmsg, sizeof(t_errmsg),
+             "moe_permute_noalloc: ceil(T/128)*N = %lld histogram entries exceed the fixed "
+             "scratch of %d; use moe_permute with a workspace",
+             (long long)need, (int)MOE_NOALLOC_HIST_INTS);
+    return MOE_ERR_UNSUPPORTED;
+  }
+  int sms;
+  if ((rc = device_setup(&sms)) != MOE_OK) return rc;
+  int32_t* hist = nullptr;
+  if ((rc = noalloc_scratch(&hist)) != MOE_OK) return rc;
+  const int T = (int)D.T, K = (int)D.K, N = (int)D.N;
+  if (T == 0) {
+    route::k_zero_i32<<<1, 256, 0, stream>>>(offsets, N + 1);
+    return launched("k_zero_i32");
+  }
+  // Every histogram entry the scan reads is written first by k_hist, so the
+  // previous call's contents never leak into this one.
+  perm::k_hist<<<D.n_chunks, 256, N * 4, stream>>>(topk_idx, T, K, N, hist);
+  perm::k_scan<<<1, 1024, 0, stream>>>(hist, D.n_chunks, N, counts, offsets);
+  perm::k_slots<<<D.n_chunks, 32, N * 4, stream>>>(topk_idx, T, K, N, hist, slot_of, perm_src);
+  if (D.fp8) {
+    perm::k_gather_quant<<<(T + 7) / 8, 256, 0, stream>>>(
+        static_cast<const __nv_bfloat16*>(x), T, K, (int)D.d, (int)D.R, slot_of,
+        static_cast<uint8_t*>(x_perm), x_perm_scale);
+  } else {
+    perm::k_gather<<<(T + 7) / 8, 256, 0, stream>>>(static_cast<const uint8_t*>(x), T, K,
+                                                    (int)(D.d * D.x_esz), slot_of,
+                                                    static_cast<uint8_t*>(x_perm));
+  }
+  return launched("permutation kernels (no-alloc)");
 }
 
 }  // extern "C"

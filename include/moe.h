@@ -124,6 +124,29 @@ moe_status moe_permute(const moe_layer_desc* desc, const void* x, const int32_t*
                        int32_t* slot_of, void* x_perm, float* x_perm_scale, void* ws,
                        size_t ws_bytes, cudaStream_t stream);
 
+/* moe_permute without a workspace, for callers that cannot allocate device
+ * memory: code that runs inside a host framework which owns all device
+ * memory and gives an operator no allocator or scratch buffer, or a C caller
+ * that only holds the layer's input and output buffers.  The pages have no
+ * counterpart; it is a packaging of moe_permute (same arguments minus the
+ * workspace, same results bit for bit).
+ *   Scratch: a fixed device array of MOE_NOALLOC_HIST_INTS int32 (1 MiB) that
+ *   each device that loads this library holds until the process exits.  It
+ *   bounds the shape: ceil(T/128) * N <= MOE_NOALLOC_HIST_INTS (T <= 131072
+ *   tokens for N = 256); larger shapes return MOE_ERR_UNSUPPORTED with the
+ *   reason in moe_last_error_message.  No device memory is allocated or freed.
+ *   The first call on a device looks up the array's device address (with that
+ *   device current); make that first call before any stream capture.
+ *   Every call uses the same array: calls whose work overlaps on the GPU (two
+ *   streams, or two host threads) race and must be serialised by the caller.
+ *   The array keeps the last call's contents; each call writes every entry it
+ *   reads before reading it, so nothing needs clearing. */
+#define MOE_NOALLOC_HIST_INTS 262144
+moe_status moe_permute_noalloc(const moe_layer_desc* desc, const void* x,
+                               const int32_t* topk_idx, const int32_t* counts, int32_t* offsets,
+                               int32_t* perm_src, int32_t* slot_of, void* x_perm,
+                               float* x_perm_scale, cudaStream_t stream);
+
 /* (c) Shared and routed experts.  One persistent tcgen05 grouped GEMM computes
  * H = SiLU(A W_gate^T) * (A W_up^T) for every expert (A = x for the shared
  * experts, the expert's x_perm rows for routed ones); a second computes

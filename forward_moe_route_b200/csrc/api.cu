@@ -12,6 +12,7 @@
 
 #include "common.cuh"
 #include "gemm.cuh"
+#include "gemm_fp8.cuh"
 #include "permute.cuh"
 #include "route.cuh"
 
@@ -134,6 +135,12 @@ moe_status device_setup(int* sms) {
     if (e == cudaSuccess) e = set_gemm_attr<0, gemm::EPI_SCATTER>();
     if (e == cudaSuccess) e = set_gemm_attr<1, gemm::EPI_SWIGLU>();
     if (e == cudaSuccess) e = set_gemm_attr<1, gemm::EPI_SCATTER>();
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(gemm8::k_grouped_gemm_fp8<gemm8::EPI_SWIGLU_Q>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(gemm8::k_grouped_gemm_fp8<gemm8::EPI_SCATTER>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     if (!g_encode) {
       void* fn = nullptr;
@@ -328,12 +335,93 @@ moe_status do_permute(const Dims& D, const Layout& L, const void* x, const int32
   return launched("permutation kernels");
 }
 
+// FP8 experts: E4M3 x_perm / H with fp32 1x128 scales, E4M3 weights with fp32
+// 128x128 block scales, promotion to fp32 every 128 elements of K.
+moe_status do_grouped_fp8(const Dims& D, const Layout& L, const void* x_perm,
+                          const float* x_perm_scale, const int32_t* gtab, const int32_t* pair_of,
+                          const float* topk_w, const void* w_gu, const float* w_gu_scale,
+                          const void* w_down, const float* w_down_scale, void* y_slots,
+                          uint8_t* ws, int sms, cudaStream_t st) {
+  const int E = (int)D.E;
+  if (D.d % gemm8::BN) return MOE_ERR_UNSUPPORTED;
+  uint8_t* hq = ws + L.hbuf;
+  float* hs = reinterpret_cast<float*>(ws + L.hscale);
+  const int64_t hrows = D.R + D.Ks * D.T;
+  const int64_t mt_bound = (D.R + (int64_t)D.N * 127) / 128 + D.Ks * ((D.T + 127) / 128);
+  int stages = 0;
+  for (int s = 6; s >= 2 && !stages; --s)
+    if (gemm8::smem_bytes(s, E) <= (size_t)kMaxSmem) stages = s;
+  if (!stages) return MOE_ERR_UNSUPPORTED;
+  const size_t smem = gemm8::smem_bytes(stages, E);
+  moe_status rc;
+  {
+    CUtensorMap ta, tb;
+    rc = make_tmap(&ta, x_perm, 1, D.d, D.R + D.T, gemm8::BM);
+    if (rc == MOE_OK) rc = make_tmap(&tb, w_gu, 1, D.d, (uint64_t)E * 2 * D.I, 32);
+    if (rc != MOE_OK) return rc;
+    gemm8::Args a;
+    memset(&a, 0, sizeof(a));
+    a.gt.base = gtab;
+    a.gt.n = E;
+    a.n_tiles_n = (int)(D.I / 128);
+    a.num_kb = (int)(D.d / 128);
+    a.b_rows_per_expert = (int)(2 * D.I);
+    a.b_up_off = (int)D.I;
+    a.stages = stages;
+    a.idesc = umma_idesc(0, gemm8::BM, gemm8::BN);
+    a.a_scale = x_perm_scale;
+    a.a_rows = (int)(D.R + D.T);
+    a.b_scale = w_gu_scale;
+    a.hq = hq;
+    a.hs = hs;
+    a.inter = (int)D.I;
+    const int64_t tiles = mt_bound * a.n_tiles_n;
+    const int grid = (int)(tiles < sms ? tiles : sms);
+    gemm8::k_grouped_gemm_fp8<gemm8::EPI_SWIGLU_Q><<<grid, gemm8::NUM_THREADS, smem, st>>>(ta, tb,
+                                                                                          a);
+    if ((rc = launched("FP8 grouped GEMM 1")) != MOE_OK) return rc;
+    if ((rc = trace(3, st)) != MOE_OK) return rc;
+  }
+  {
+    CUtensorMap ta, tb;
+    rc = make_tmap(&ta, hq, 1, D.I, hrows, gemm8::BM);
+    if (rc == MOE_OK) rc = make_tmap(&tb, w_down, 1, D.I, (uint64_t)E * D.d, gemm8::BN);
+    if (rc != MOE_OK) return rc;
+    gemm8::Args a;
+    memset(&a, 0, sizeof(a));
+    a.gt.base = gtab;
+    a.gt.n = E;
+    a.n_tiles_n = (int)(D.d / gemm8::BN);
+    a.num_kb = (int)(D.I / 128);
+    a.b_rows_per_expert = (int)D.d;
+    a.a_from_crow = 1;
+    a.stages = stages;
+    a.idesc = umma_idesc(0, gemm8::BM, gemm8::BN);
+    a.a_scale = hs;
+    a.a_rows = (int)hrows;
+    a.b_scale = w_down_scale;
+    a.y = static_cast<__nv_bfloat16*>(y_slots);
+    a.d = (int)D.d;
+    a.pair_of = pair_of;
+    a.topk_w = topk_w;
+    a.K = (int)D.K;
+    a.Ks = (int)D.Ks;
+    const int64_t tiles = mt_bound * a.n_tiles_n;
+    const int grid = (int)(tiles < sms ? tiles : sms);
+    gemm8::k_grouped_gemm_fp8<gemm8::EPI_SCATTER><<<grid, gemm8::NUM_THREADS, smem, st>>>(ta, tb,
+                                                                                         a);
+    if ((rc = launched("FP8 grouped GEMM 2")) != MOE_OK) return rc;
+    rc = trace(4, st);
+  }
+  return rc;
+}
+
 moe_status do_grouped(const Dims& D, const Layout& L, const void* x, const void* x_perm,
-                      const int32_t* offsets, const int32_t* slot_of, const float* topk_w,
-                      const void* w_gu, const void* w_down, void* y_slots, uint8_t* ws, int sms,
-                      cudaStream_t st) {
+                      const float* x_perm_scale, const int32_t* offsets, const int32_t* slot_of,
+                      const float* topk_w, const void* w_gu, const float* w_gu_scale,
+                      const void* w_down, const float* w_down_scale, void* y_slots, uint8_t* ws,
+                      int sms, cudaStream_t st) {
   if (D.T == 0) return MOE_OK;
-  if (D.fp8) return MOE_ERR_UNSUPPORTED;
   const int E = (int)D.E;
   int32_t* gtab = reinterpret_cast<int32_t*>(ws + L.gtab);
   int32_t* pair_of = reinterpret_cast<int32_t*>(ws + L.pair_of);
@@ -342,9 +430,13 @@ moe_status do_grouped(const Dims& D, const Layout& L, const void* x, const void*
   moe_status rc = trace(2, st);
   if (rc != MOE_OK) return rc;
   perm::k_prep_groups<<<prep_blocks, 1024, 0, st>>>(offsets, (int)D.T, (int)D.K, (int)D.Ks,
-                                                    (int)D.N, 0, gtab, slot_of, pair_of);
+                                                    (int)D.N, D.fp8 ? 1 : 0, gtab, slot_of,
+                                                    pair_of);
   rc = launched("k_prep_groups");
   if (rc != MOE_OK) return rc;
+  if (D.fp8)
+    return do_grouped_fp8(D, L, x_perm, x_perm_scale, gtab, pair_of, topk_w, w_gu, w_gu_scale,
+                          w_down, w_down_scale, y_slots, ws, sms, st);
 
   const size_t esz = D.op_esz;
   const int kind = D.f32 ? 1 : 0;
@@ -562,7 +654,8 @@ moe_status moe_grouped_swiglu(const moe_layer_desc* desc, const void* x, const v
   if (!ws || ws_bytes < L.total || !aligned16(ws)) return MOE_ERR_WORKSPACE;
   int sms;
   if ((rc = device_setup(&sms)) != MOE_OK) return rc;
-  return do_grouped(D, L, x, x_perm, offsets, slot_of, topk_w, w_gu, w_down, y_slots,
+  return do_grouped(D, L, x, x_perm, x_perm_scale, offsets, slot_of, topk_w, w_gu, w_gu_scale,
+                    w_down, w_down_scale, y_slots,
                     static_cast<uint8_t*>(ws), sms, stream);
 }
 
@@ -615,7 +708,8 @@ moe_status moe_forward(const moe_layer_desc* desc, const void* x, const void* x_
   if ((rc = do_permute(D, L, x, idx, cnt, offsets, perm_src, slot_of, x_perm, x_perm_scale, w8,
                        stream)) != MOE_OK)
     return rc;
-  if ((rc = do_grouped(D, L, x, x_perm, offsets, slot_of, tw, w_gu, w_down, y, w8, sms,
+  if ((rc = do_grouped(D, L, x, x_perm, x_perm_scale, offsets, slot_of, tw, w_gu, w_gu_scale,
+                       w_down, w_down_scale, y, w8, sms,
                        stream)) != MOE_OK)
     return rc;
   rc = do_combine(D, x_residual ? x_residual : x, y, h, stream);

@@ -1,0 +1,321 @@
+// Grouped GEMM with FP8 E4M3 operands and fine-grained fp32 scales.
+//
+// Follows "DeepSeek Technical Report: MoE Architecture", §3.6 (FP8 mixed
+// precision): E4M3 operands, activations scaled per 1x128 tile, weights per
+// 128x128 block, fp32 accumulation with promotion every 128 elements of K.
+//
+// Each 128-element block of K (one 128-byte k-block) is multiplied on the
+// tensor cores into a fresh TMEM partial P_kb (tcgen05.mma kind::f8f6f4, fp32
+// accumulation).  The epilogue warps promote it on the CUDA cores:
+//   acc += (sa[row, kb] * sb[col block, kb]) * P_kb
+// so every k-block carries its own activation and weight scale.  Two TMEM
+// partials (2 x 256 columns) let the MMA of k-block kb+1 overlap the promotion
+// of kb.
+//
+// Warp roles (576 threads, one CTA per SM):
+//   warp 0      TMA producer (and TMEM allocator)
+//   warp 1      MMA issuer
+//   warps 2..17 16 promotion/epilogue warps: warp w owns TMEM lane quadrant
+//               w % 4 (32 rows) and the 64-column slice (w - 2) / 4 of the tile.
+// Tile: 128 rows x 256 accumulator columns.
+//   GEMM1 (SWIGLU): the B tile holds W_gate and W_up rows interleaved in
+//     chunks of 32 (gate 0-31, up 0-31, gate 32-63, up 32-63, ...), so each
+//     64-column slice holds matching gate and up columns; the epilogue forms
+//     H = SiLU(gate) * up for 128 H columns (one 1x128 quantisation tile per
+//     row), exchanges the per-slice amax through shared memory, and writes E4M3
+//     codes plus the fp32 tile scale.
+//   GEMM2 (SCATTER): 256 output columns, times the gate weight, bf16 rows
+//     scattered to the token-major slots.
+#pragma once
+
+#include "common.cuh"
+#include "gemm.cuh"
+
+namespace moe {
+namespace gemm8 {
+
+constexpr int BM = 128;
+constexpr int BN = 256;
+constexpr int KB = 128;              // bytes = elements of K per k-block
+constexpr int NUM_THREADS = 576;
+constexpr int EPI_WARP0 = 2;
+constexpr int NUM_EPI = NUM_THREADS - EPI_WARP0 * 32;   // 512
+constexpr int TMEM_COLS = 512;       // two 256-column partials
+
+enum Epi { EPI_SWIGLU_Q = 1, EPI_SCATTER = 2 };
+
+struct Args {
+  gemm::GroupTab gt;
+  int n_tiles_n;
+  int num_kb;
+  int b_rows_per_expert;     // rows of B per expert (2I for GEMM1, d for GEMM2)
+  int b_up_off;              // GEMM1: row offset of W_up inside an expert (I)
+  int a_from_crow;           // GEMM2 reads A (H) rows from c_row
+  int stages;
+  uint32_t idesc;
+  // scales
+  const float* a_scale;      // [A rows, num_kb]
+  int a_rows;                // rows of the A tensor (scales beyond it read as 0)
+  const float* b_scale;      // [E, b_rows_per_expert/128, num_kb]
+  // GEMM1 outputs
+  uint8_t* hq;               // [H rows, I] E4M3
+  float* hs;                 // [H rows, I/128]
+  int inter;                 // I
+  // GEMM2 outputs
+  __nv_bfloat16* y;          // [T*(K+Ks), d]
+  int d;
+  const int* pair_of;
+  const float* topk_w;
+  int K, Ks;
+};
+
+__host__ inline size_t smem_bytes(int stages, int n_groups) {
+  return 1024 + (size_t)stages * (BM * KB + BN * KB) + (size_t)(2 * stages + 6) * 8 + 16 +
+         2 * 4 * BM * sizeof(float) + (size_t)(n_groups + 1) * 4 + 64;
+}
+
+template <int EPI>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    k_grouped_gemm_fp8(const __grid_constant__ CUtensorMap tmA,
+                       const __grid_constant__ CUtensorMap tmB, const Args a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  constexpr uint32_t a_bytes = BM * KB;
+  constexpr uint32_t b_bytes = BN * KB;
+  constexpr uint32_t stage_bytes = a_bytes + b_bytes;
+  const int S = a.stages;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)S * stage_bytes);
+  uint64_t* empty = full + S;
+  uint64_t* pfull = empty + S;
+  uint64_t* pempty = pfull + 2;
+  uint64_t* xbar = pempty + 2;       // amax exchange between the epilogue warps
+  uint64_t* drain = xbar + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* amax_buf = reinterpret_cast<float*>(tmem_slot + 4);   // [2][4][128]
+  int* s_prefix = reinterpret_cast<int*>(amax_buf + 2 * 4 * BM);
+
+  const int warp = warp_id(), lane = lane_id();
+  const int n_groups = a.gt.count();
+  for (int i = threadIdx.x; i <= n_groups; i += NUM_THREADS) s_prefix[i] = a.gt.prefix(i);
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int j = 0; j < 2; ++j) {
+      mbar_init(&pfull[j], 1);
+      mbar_init(&pempty[j], NUM_EPI / 32);
+    }
+    mbar_init(xbar, NUM_EPI);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    fence_proxy_async_smem();
+  }
+  if (warp == 0) {
+    if (lane == 0) {
+      tma_prefetch_desc(&tmA);
+      tma_prefetch_desc(&tmB);
+    }
+    __syncwarp();
+    tmem_alloc(tmem_slot, TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int total_tiles = s_prefix[n_groups] * a.n_tiles_n;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ TMA producer
+    if (elect_one()) {
+      int it = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
+        const int mt = tile / a.n_tiles_n, nt = tile - mt * a.n_tiles_n;
+        const int g = gemm::find_group(s_prefix, n_groups, mt);
+        const int lm = mt - s_prefix[g];
+        const int arow = (a.a_from_crow ? a.gt.c_row(g) : a.gt.a_row(g)) + lm * BM;
+        const int ebase = a.gt.expert(g) * a.b_rows_per_expert;
+        for (int kb = 0; kb < a.num_kb; ++kb, ++it) {
+          const int s = it % S;
+          const uint32_t ph = (uint32_t)(it / S) & 1u;
+          if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag)) { ok = false; break; }
+          uint8_t* sa = smem + (size_t)s * stage_bytes;
+          uint8_t* sb = sa + a_bytes;
+          mbar_arrive_expect_tx(&full[s], stage_bytes);
+          const int kx = kb * KB;
+          tma_load_2d(&tmA, &full[s], sa, kx, arow);
+          if (EPI == EPI_SWIGLU_Q) {
+            const int gr = ebase + nt * 128, ur = ebase + a.b_up_off + nt * 128;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              tma_load_2d(&tmB, &full[s], sb + (size_t)(2 * c) * 32 * KB, kx, gr + 32 * c);
+              tma_load_2d(&tmB, &full[s], sb + (size_t)(2 * c + 1) * 32 * KB, kx, ur + 32 * c);
+            }
+          } else {
+            tma_load_2d(&tmB, &full[s], sb, kx, ebase + nt * BN);
+          }
+        }
+      }
+      if (!ok) {
+        volatile int no_abort = 0;
+        for (int j = (it - S > 0 ? it - S : 0); j < it; ++j)
+          mbar_wait(&full[j % S], (uint32_t)(j / S) & 1u, &no_abort);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (elect_one()) {
+      int it = 0, pu = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
+        for (int kb = 0; kb < a.num_kb; ++kb, ++it, ++pu) {
+          const int s = it % S;
+          const uint32_t ph = (uint32_t)(it / S) & 1u;
+          const int p = pu & 1;
+          const uint32_t pph = (uint32_t)(pu >> 1) & 1u;
+          if (!mbar_wait(&full[s], ph, abort_flag)) { ok = false; break; }
+          if (!mbar_wait(&pempty[p], pph ^ 1u, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + (size_t)s * stage_bytes);
+          const uint64_t ad = umma_desc_sw128(sa);
+          const uint64_t bd = umma_desc_sw128(sa + a_bytes);
+          const uint32_t d_tmem = tmem_base + (uint32_t)(p * BN);
+#pragma unroll
+          for (int k = 0; k < KB / 32; ++k)
+            umma<2>(d_tmem, ad + (uint64_t)(k * 2), bd + (uint64_t)(k * 2), a.idesc,
+                    k != 0 ? 1u : 0u);
+          umma_commit(&empty[s]);
+          umma_commit(&pfull[p]);
+        }
+      }
+      // every MMA issued above completes before the block may free TMEM
+      umma_commit(drain);
+      volatile int no_abort = 0;
+      mbar_wait(drain, 0, &no_abort);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------------ promotion + epilogue
+    const int ew = warp - EPI_WARP0;
+    const int q = warp & 3;
+    const int cs = ew >> 2;                 // 64-column slice 0..3
+    const int r = q * 32 + lane;
+    const int col0 = cs * 64;
+    const int kb_blocks_b = a.b_rows_per_expert / 128;
+    int pu = 0, tcount = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x, ++tcount) {
+      const int mt = tile / a.n_tiles_n, nt = tile - mt * a.n_tiles_n;
+      const int g = gemm::find_group(s_prefix, n_groups, mt);
+      const int lm = mt - s_prefix[g];
+      const int grow = lm * BM + r;
+      const bool valid = grow < a.gt.rows(g);
+      const int arow = (a.a_from_crow ? a.gt.c_row(g) : a.gt.a_row(g)) + grow;
+      const float* sa_row = arow < a.a_rows ? a.a_scale + (size_t)arow * a.num_kb : nullptr;
+      const size_t eb = (size_t)a.gt.expert(g) * kb_blocks_b;
+      const float* sb0;
+      const float* sb1;
+      if (EPI == EPI_SWIGLU_Q) {
+        sb0 = a.b_scale + (eb + nt) * a.num_kb;                          // gate block
+        sb1 = a.b_scale + (eb + a.b_up_off / 128 + nt) * a.num_kb;       // up block
+      } else {
+        sb0 = a.b_scale + (eb + 2 * nt + cs / 2) * a.num_kb;
+        sb1 = sb0;
+      }
+      float acc[64];
+#pragma unroll
+      for (int i = 0; i < 64; ++i) acc[i] = 0.f;
+      float na = sa_row ? sa_row[0] : 0.f, nb0 = sb0[0], nb1 = sb1[0];
+      for (int kb = 0; kb < a.num_kb; ++kb, ++pu) {
+        const float m0 = na * nb0, m1 = na * nb1;
+        if (kb + 1 < a.num_kb) {
+          na = sa_row ? sa_row[kb + 1] : 0.f;
+          nb0 = sb0[kb + 1];
+          nb1 = sb1[kb + 1];
+        }
+        const int p = pu & 1;
+        if (!mbar_wait(&pfull[p], (uint32_t)(pu >> 1) & 1u, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(p * BN + col0);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          float v[16];
+          tmem_ld16(tb + (uint32_t)(16 * c), v);
+          const float m = c < 2 ? m0 : m1;
+#pragma unroll
+          for (int i = 0; i < 16; ++i) acc[16 * c + i] = fmaf(m, v[i], acc[16 * c + i]);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&pempty[p]);
+      }
+      if (!ok) break;
+      if (EPI == EPI_SWIGLU_Q) {
+        // columns 0..31 of the slice are gate, 32..63 the matching up
+        float pam = 0.f;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          acc[i] = gemm::silu_f(acc[i]) * acc[32 + i];
+          pam = fmaxf(pam, fabsf(acc[i]));
+        }
+        float* ab = amax_buf + (tcount & 1) * 4 * BM;
+        ab[cs * BM + r] = pam;
+        mbar_arrive(xbar);
+        if (!mbar_wait(xbar, (uint32_t)tcount & 1u, abort_flag)) { ok = false; break; }
+        const float amax = fmaxf(fmaxf(ab[r], ab[BM + r]), fmaxf(ab[2 * BM + r], ab[3 * BM + r]));
+        const float scale = amax > 0.f ? __fdiv_rn(amax, 448.0f) : 0.f;
+        const float inv = amax > 0.f ? __fdiv_rn(448.0f, amax) : 0.f;
+        if (valid) {
+          const size_t hrow = (size_t)(a.gt.c_row(g) + grow);
+          uint32_t w[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            w[j] = (uint32_t)f32_to_e4m3(__fmul_rn(acc[4 * j], inv)) |
+                   ((uint32_t)f32_to_e4m3(__fmul_rn(acc[4 * j + 1], inv)) << 8) |
+                   ((uint32_t)f32_to_e4m3(__fmul_rn(acc[4 * j + 2], inv)) << 16) |
+                   ((uint32_t)f32_to_e4m3(__fmul_rn(acc[4 * j + 3], inv)) << 24);
+          uint4* dst = reinterpret_cast<uint4*>(a.hq + hrow * a.inter + nt * 128 + cs * 32);
+          dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+          dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+          if (cs == 0) a.hs[hrow * (a.inter / 128) + nt] = scale;
+        }
+      } else {
+        if (valid) {
+          long long dst;
+          float wgt = 1.0f;
+          const int s_idx = a.gt.aux(g);
+          if (s_idx < 0) {
+            const int pair = a.pair_of[a.gt.c_row(g) + grow];
+            const int t = pair / a.K, k = pair - t * a.K;
+            dst = (long long)t * (a.K + a.Ks) + k;
+            wgt = a.topk_w[pair];
+          } else {
+            dst = (long long)grow * (a.K + a.Ks) + a.K + s_idx;
+          }
+          uint4* o = reinterpret_cast<uint4*>(a.y + dst * a.d + nt * BN + col0);
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            o[j] = make_uint4(gemm::pack_bf16x2(acc[8 * j] * wgt, acc[8 * j + 1] * wgt),
+                              gemm::pack_bf16x2(acc[8 * j + 2] * wgt, acc[8 * j + 3] * wgt),
+                              gemm::pack_bf16x2(acc[8 * j + 4] * wgt, acc[8 * j + 5] * wgt),
+                              gemm::pack_bf16x2(acc[8 * j + 6] * wgt, acc[8 * j + 7] * wgt));
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+}  // namespace gemm8
+}  // namespace moe

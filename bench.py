@@ -59,6 +59,25 @@ def config_dict(cfg, n):
             "l2": "inputs larger than L2 (expert weights and x exceed the 126 MB L2)"}
 
 
+# ----------------------------------------------------------------------------- ranks
+def token_shard(T: int, rank: int, world: int):
+    """[lo, hi) of the tokens rank `rank` owns when a batch of T is split over `world`."""
+    base, extra = divmod(T, world)
+    lo = rank * base + min(rank, extra)
+    return lo, lo + base + (1 if rank < extra else 0)
+
+
+def max_over_ranks(value: float, device) -> float:
+    """The maximum of `value` over all ranks (the value itself without a process group)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([value], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 # ----------------------------------------------------------------------------- clocks
 class ClockSampler:
     """nvidia-smi samples of this GPU's clocks while the timed region runs."""
@@ -302,10 +321,7 @@ def run_ours(args, cfg):
         stages["gemm2_scatter"].append(e[3].elapsed_time(e[4]))
         stages["combine"].append(e[4].elapsed_time(e[5]))
     stage_ms = {k: sum(v) / len(v) for k, v in stages.items()}
-    if world > 1:
-        t = torch.tensor([ms], device="cuda", dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, "cuda")
 
     # ---- end to end through the public API: pinned host x in, h back out, every step
     x_host = inp["x"].cpu().pin_memory()
@@ -329,10 +345,7 @@ def run_ours(args, cfg):
     torch.cuda.synchronize()
     barrier()
     e2e_ms = e0.elapsed_time(e1) / e2e_steps
-    if world > 1:
-        t = torch.tensor([e2e_ms], device="cuda", dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e2e_ms, "cuda")
 
     ms_step = ms / args.steps
     tokens_s = cfg.T * world / (ms_step * 1e-3)
@@ -395,6 +408,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--config", default=DEFAULT_CONFIG)
     ap.add_argument("--T", type=int, default=None, help="override the token count")
+    ap.add_argument("--n-routed", type=int, default=None,
+                    help="override the routed expert count (smaller profiling cases)")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
@@ -404,6 +419,10 @@ def main():
     cfg = recipes.CONFIGS[args.config]
     if args.T is not None:
         cfg = cfg.with_T(args.T)
+    if args.n_routed is not None:
+        import dataclasses
+        cfg = dataclasses.replace(cfg, n_routed=args.n_routed,
+                                  name=f"{cfg.name}@N{args.n_routed}")
     if args.impl == "reference":
         return run_reference(args, cfg)
     out = run_ours(args, cfg)

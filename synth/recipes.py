@@ -46,7 +46,7 @@ class LayerConfig:
     wgu_sigma: float = 0.02
     wd_sigma: float = 0.02
     bias_half_range: Optional[float] = None   # bias ~ U(-a, a)
-    zipf: bool = False                        # skewed load: common-mode x[:,0] += 1, w_r[:,0] += c_i
+    zipf: bool = False                        # skewed load: constant feature x[:,0] = 1, w_r[:,0] += c_i
     seed: int = 0
 
     @property
@@ -124,7 +124,7 @@ def host_x(cfg: LayerConfig, rows: Optional[Sequence[int]] = None) -> np.ndarray
                       for t in rows]) if len(rows) else np.zeros((0, cfg.d), np.float32)
     if cfg.zipf:
         v = v.copy()
-        v[:, 0] = v[:, 0] + np.float32(1.0)
+        v[:, 0] = np.float32(1.0)
     return _round_like(cfg, v)
 
 
@@ -186,7 +186,7 @@ def device_inputs(cfg: LayerConfig, device="cuda", zipf_offsets: Optional[np.nda
     if cfg.zipf:
         if zipf_offsets is None:
             raise ValueError("skewed-load recipe needs its per-expert logit offsets")
-        x32[:, 0] += 1.0
+        x32[:, 0] = 1.0
         wr32[:, 0] += torch.as_tensor(np.asarray(zipf_offsets, np.float32), device=device)
     x = x32.to(dt)
     del x32

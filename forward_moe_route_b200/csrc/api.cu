@@ -136,10 +136,13 @@ moe_status device_setup(int* sms) {
     if (e == cudaSuccess) e = set_gemm_attr<1, gemm::EPI_SWIGLU>();
     if (e == cudaSuccess) e = set_gemm_attr<1, gemm::EPI_SCATTER>();
     if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(gemm8::k_grouped_gemm_fp8<gemm8::EPI_SWIGLU_Q>,
+      e = cudaFuncSetAttribute(gemm8::k_gemm_promoted<0, gemm8::EPI_F32_STORE>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
     if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(gemm8::k_grouped_gemm_fp8<gemm8::EPI_SCATTER>,
+      e = cudaFuncSetAttribute(gemm8::k_gemm_promoted<2, gemm8::EPI_SWIGLU_Q>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(gemm8::k_gemm_promoted<2, gemm8::EPI_SCATTER>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     if (!g_encode) {
@@ -274,34 +277,39 @@ moe_status do_route(const moe_layer_desc& s, const Dims& D, const Layout& L, con
     else launch_route_f32<16>(xf, wf, dd, bias, p, topk_idx, topk_w, counts, st);
     return launched("k_route_f32");
   }
-  // bf16 router GEMM on tensor cores: logits [T, N] fp32 (counts zeroed in its prologue)
+  // bf16 router GEMM on tensor cores: logits [T, N] fp32.  Each 64-element K
+  // block is a separate tensor-core product added into fp32 registers with
+  // round-to-nearest, so the logits keep fp32 accuracy over the whole of d
+  // (the selection is decided on them).  Its prologue zeroes the counts.
   float* logits = reinterpret_cast<float*>(ws + L.logits);
-  const int bn_full = (N + 15) / 16 * 16;
-  const int bn = bn_full <= 256 ? bn_full : 256;
   CUtensorMap ta, tb;
-  moe_status rc = make_tmap(&ta, x, 2, D.d, D.T, gemm::BM);
-  if (rc == MOE_OK) rc = make_tmap(&tb, w_router, 2, D.d, D.N, bn);
+  moe_status rc = make_tmap(&ta, x, 2, D.d, D.T, gemm8::BM);
+  if (rc == MOE_OK) rc = make_tmap(&tb, w_router, 2, D.d, D.N, gemm8::BN);
   if (rc != MOE_OK) return rc;
-  gemm::Args a;
+  gemm8::Args a;
   memset(&a, 0, sizeof(a));
   a.gt.base = nullptr;
   a.gt.n = 1;
   a.gt.single_rows = (int)D.T;
-  a.n_tiles_n = (N + bn - 1) / bn;
-  a.num_kb = (int)(D.d * 2 / gemm::KB);
-  a.kb_elems = gemm::KB / 2;
-  a.bn = bn;
+  a.n_tiles_n = (N + gemm8::BN - 1) / gemm8::BN;
+  a.num_kb = (int)(D.d * 2 / gemm8::KB);
+  a.kb_elems = gemm8::KB / 2;
   a.b_rows_per_expert = 0;
-  a.idesc = umma_idesc(1, gemm::BM, bn);
+  a.idesc = umma_idesc(1, gemm8::BM, gemm8::BN);
   a.out = logits;
   a.out_ld = N;
   a.out_cols = N;
-  a.out_bf16 = 0;
   a.zero_ptr = counts;
   a.zero_n = N;
+  int stages = 0;
+  for (int s = 6; s >= 2 && !stages; --s)
+    if (gemm8::smem_bytes(s, 1) <= (size_t)kMaxSmem) stages = s;
+  a.stages = stages;
   const int tiles = (int)((D.T + 127) / 128) * a.n_tiles_n;
-  rc = launch_gemm<0, gemm::EPI_F32_STORE>(ta, ta, tb, a, tiles < sms ? tiles : sms, st);
-  if (rc != MOE_OK) return rc;
+  gemm8::k_gemm_promoted<0, gemm8::EPI_F32_STORE>
+      <<<tiles < sms ? tiles : sms, gemm8::NUM_THREADS, gemm8::smem_bytes(stages, 1), st>>>(ta, tb,
+                                                                                          a);
+  if ((rc = launched("router GEMM")) != MOE_OK) return rc;
   if (N <= 32) launch_topk<1>(logits, bias, p, topk_idx, topk_w, counts, st);
   else if (N <= 64) launch_topk<2>(logits, bias, p, topk_idx, topk_w, counts, st);
   else if (N <= 128) launch_topk<4>(logits, bias, p, topk_idx, topk_w, counts, st);
@@ -365,6 +373,7 @@ moe_status do_grouped_fp8(const Dims& D, const Layout& L, const void* x_perm,
     a.gt.n = E;
     a.n_tiles_n = (int)(D.I / 128);
     a.num_kb = (int)(D.d / 128);
+    a.kb_elems = 128;
     a.b_rows_per_expert = (int)(2 * D.I);
     a.b_up_off = (int)D.I;
     a.stages = stages;
@@ -377,7 +386,7 @@ moe_status do_grouped_fp8(const Dims& D, const Layout& L, const void* x_perm,
     a.inter = (int)D.I;
     const int64_t tiles = mt_bound * a.n_tiles_n;
     const int grid = (int)(tiles < sms ? tiles : sms);
-    gemm8::k_grouped_gemm_fp8<gemm8::EPI_SWIGLU_Q><<<grid, gemm8::NUM_THREADS, smem, st>>>(ta, tb,
+    gemm8::k_gemm_promoted<2, gemm8::EPI_SWIGLU_Q><<<grid, gemm8::NUM_THREADS, smem, st>>>(ta, tb,
                                                                                           a);
     if ((rc = launched("FP8 grouped GEMM 1")) != MOE_OK) return rc;
     if ((rc = trace(3, st)) != MOE_OK) return rc;
@@ -393,6 +402,7 @@ moe_status do_grouped_fp8(const Dims& D, const Layout& L, const void* x_perm,
     a.gt.n = E;
     a.n_tiles_n = (int)(D.d / gemm8::BN);
     a.num_kb = (int)(D.I / 128);
+    a.kb_elems = 128;
     a.b_rows_per_expert = (int)D.d;
     a.a_from_crow = 1;
     a.stages = stages;
@@ -408,7 +418,7 @@ moe_status do_grouped_fp8(const Dims& D, const Layout& L, const void* x_perm,
     a.Ks = (int)D.Ks;
     const int64_t tiles = mt_bound * a.n_tiles_n;
     const int grid = (int)(tiles < sms ? tiles : sms);
-    gemm8::k_grouped_gemm_fp8<gemm8::EPI_SCATTER><<<grid, gemm8::NUM_THREADS, smem, st>>>(ta, tb,
+    gemm8::k_gemm_promoted<2, gemm8::EPI_SCATTER><<<grid, gemm8::NUM_THREADS, smem, st>>>(ta, tb,
                                                                                          a);
     if ((rc = launched("FP8 grouped GEMM 2")) != MOE_OK) return rc;
     rc = trace(4, st);

@@ -42,12 +42,13 @@ constexpr int EPI_WARP0 = 2;
 constexpr int NUM_EPI = NUM_THREADS - EPI_WARP0 * 32;   // 512
 constexpr int TMEM_COLS = 512;       // two 256-column partials
 
-enum Epi { EPI_SWIGLU_Q = 1, EPI_SCATTER = 2 };
+enum Epi { EPI_F32_STORE = 0, EPI_SWIGLU_Q = 1, EPI_SCATTER = 2 };
 
 struct Args {
   gemm::GroupTab gt;
   int n_tiles_n;
   int num_kb;
+  int kb_elems;              // elements of K per k-block (128 E4M3, 64 bf16)
   int b_rows_per_expert;     // rows of B per expert (2I for GEMM1, d for GEMM2)
   int b_up_off;              // GEMM1: row offset of W_up inside an expert (I)
   int a_from_crow;           // GEMM2 reads A (H) rows from c_row
@@ -67,6 +68,11 @@ struct Args {
   const int* pair_of;
   const float* topk_w;
   int K, Ks;
+  // F32_STORE (router logits): out [rows, out_ld] fp32, columns < out_cols
+  float* out;
+  int out_ld, out_cols;
+  int* zero_ptr;             // prologue: zero an int array (the expert counts)
+  int zero_n;
 };
 
 __host__ inline size_t smem_bytes(int stages, int n_groups) {
@@ -74,9 +80,9 @@ __host__ inline size_t smem_bytes(int stages, int n_groups) {
          2 * 4 * BM * sizeof(float) + (size_t)(n_groups + 1) * 4 + 64;
 }
 
-template <int EPI>
+template <int KIND, int EPI>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
-    k_grouped_gemm_fp8(const __grid_constant__ CUtensorMap tmA,
+    k_gemm_promoted(const __grid_constant__ CUtensorMap tmA,
                        const __grid_constant__ CUtensorMap tmB, const Args a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -98,6 +104,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   const int warp = warp_id(), lane = lane_id();
   const int n_groups = a.gt.count();
+  if (a.zero_ptr) {
+    for (int i = blockIdx.x * NUM_THREADS + threadIdx.x; i < a.zero_n; i += gridDim.x * NUM_THREADS)
+      a.zero_ptr[i] = 0;
+  }
   for (int i = threadIdx.x; i <= n_groups; i += NUM_THREADS) s_prefix[i] = a.gt.prefix(i);
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -147,7 +157,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           uint8_t* sa = smem + (size_t)s * stage_bytes;
           uint8_t* sb = sa + a_bytes;
           mbar_arrive_expect_tx(&full[s], stage_bytes);
-          const int kx = kb * KB;
+          const int kx = kb * a.kb_elems;
           tma_load_2d(&tmA, &full[s], sa, kx, arow);
           if (EPI == EPI_SWIGLU_Q) {
             const int gr = ebase + nt * 128, ur = ebase + a.b_up_off + nt * 128;
@@ -188,7 +198,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const uint32_t d_tmem = tmem_base + (uint32_t)(p * BN);
 #pragma unroll
           for (int k = 0; k < KB / 32; ++k)
-            umma<2>(d_tmem, ad + (uint64_t)(k * 2), bd + (uint64_t)(k * 2), a.idesc,
+            umma<KIND>(d_tmem, ad + (uint64_t)(k * 2), bd + (uint64_t)(k * 2), a.idesc,
                     k != 0 ? 1u : 0u);
           umma_commit(&empty[s]);
           umma_commit(&pfull[p]);
@@ -217,24 +227,30 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const int grow = lm * BM + r;
       const bool valid = grow < a.gt.rows(g);
       const int arow = (a.a_from_crow ? a.gt.c_row(g) : a.gt.a_row(g)) + grow;
-      const float* sa_row = arow < a.a_rows ? a.a_scale + (size_t)arow * a.num_kb : nullptr;
       const size_t eb = (size_t)a.gt.expert(g) * kb_blocks_b;
-      const float* sb0;
-      const float* sb1;
-      if (EPI == EPI_SWIGLU_Q) {
+      const float* sa_row = nullptr;
+      const float* sb0 = nullptr;
+      const float* sb1 = nullptr;
+      if (EPI == EPI_F32_STORE) {
+        // unscaled: plain fp32 accumulation of the k-block partials
+      } else if (EPI == EPI_SWIGLU_Q) {
+        sa_row = arow < a.a_rows ? a.a_scale + (size_t)arow * a.num_kb : nullptr;
         sb0 = a.b_scale + (eb + nt) * a.num_kb;                          // gate block
         sb1 = a.b_scale + (eb + a.b_up_off / 128 + nt) * a.num_kb;       // up block
       } else {
+        sa_row = arow < a.a_rows ? a.a_scale + (size_t)arow * a.num_kb : nullptr;
         sb0 = a.b_scale + (eb + 2 * nt + cs / 2) * a.num_kb;
         sb1 = sb0;
       }
       float acc[64];
 #pragma unroll
       for (int i = 0; i < 64; ++i) acc[i] = 0.f;
-      float na = sa_row ? sa_row[0] : 0.f, nb0 = sb0[0], nb1 = sb1[0];
+      const bool scaled = EPI != EPI_F32_STORE;
+      float na = scaled ? (sa_row ? sa_row[0] : 0.f) : 1.f;
+      float nb0 = scaled ? sb0[0] : 1.f, nb1 = scaled ? sb1[0] : 1.f;
       for (int kb = 0; kb < a.num_kb; ++kb, ++pu) {
         const float m0 = na * nb0, m1 = na * nb1;
-        if (kb + 1 < a.num_kb) {
+        if (scaled && kb + 1 < a.num_kb) {
           na = sa_row ? sa_row[kb + 1] : 0.f;
           nb0 = sb0[kb + 1];
           nb1 = sb1[kb + 1];
@@ -247,16 +263,36 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int c = 0; c < 4; ++c) {
           float v[16];
           tmem_ld16(tb + (uint32_t)(16 * c), v);
-          const float m = c < 2 ? m0 : m1;
+          if (EPI == EPI_F32_STORE) {
 #pragma unroll
-          for (int i = 0; i < 16; ++i) acc[16 * c + i] = fmaf(m, v[i], acc[16 * c + i]);
+            for (int i = 0; i < 16; ++i) acc[16 * c + i] += v[i];
+          } else {
+            const float m = c < 2 ? m0 : m1;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) acc[16 * c + i] = fmaf(m, v[i], acc[16 * c + i]);
+          }
         }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&pempty[p]);
       }
       if (!ok) break;
-      if (EPI == EPI_SWIGLU_Q) {
+      if (EPI == EPI_F32_STORE) {
+        if (valid) {
+          float* orow = a.out + (size_t)(a.gt.c_row(g) + grow) * a.out_ld + nt * BN + col0;
+          const int c0 = nt * BN + col0;
+          if (c0 + 64 <= a.out_cols) {
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+              reinterpret_cast<float4*>(orow)[j] =
+                  make_float4(acc[4 * j], acc[4 * j + 1], acc[4 * j + 2], acc[4 * j + 3]);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 64; ++j)
+              if (c0 + j < a.out_cols) orow[j] = acc[j];
+          }
+        }
+      } else if (EPI == EPI_SWIGLU_Q) {
         // columns 0..31 of the slice are gate, 32..63 the matching up
         float pam = 0.f;
 #pragma unroll

@@ -68,7 +68,8 @@ def sample_tokens(cfg, g_idx, counts, n_strided, n_extra=16):
     return np.array(sorted(toks))
 
 
-def check_layer(cfg, n_strided, fp8=False):
+def check_layer(cfg, n_strided):
+    fp8 = cfg.dtype == "e4m3"
     offs = zipf_offsets(cfg)
     inp = recipes.device_inputs(cfg, "cuda", offs)
     if fp8:
@@ -96,6 +97,13 @@ def check_layer(cfg, n_strided, fp8=False):
     c2 = torch.empty_like(counts)
     moe.moe_route(desc, inp["x"], inp["w_r"], inp["bias"], idx2, w2, c2, ws)
     assert torch.equal(idx2, idx) and torch.equal(c2, counts)
+    # the router logits sit at the start of the workspace: report their error
+    lg = ws[:cfg.T * cfg.n_routed * 4].view(torch.float32).view(cfg.T, cfg.n_routed)
+    lerr = np.abs(lg.double().cpu().numpy() - ref["logits"])
+    bad = np.nonzero(np.any(g_idx != ref["idx"], axis=1))[0]
+    print(f"{cfg.name}: router logits max abs err {lerr.max():.3e} (max |l| "
+          f"{np.abs(ref['logits']).max():.2f}); tokens selecting differently {len(bad)}: "
+          f"kgap {ref['kgap'][bad][:8]}, ggap {ref['ggap'][bad][:8]}")
     del ws
     ties = check_routing(cfg, ref, g_idx, w2.cpu().numpy().astype(np.float64), g_counts)
     _, offsets, perm_src, slot_of = mo.permutation(g_idx, cfg.n_routed)

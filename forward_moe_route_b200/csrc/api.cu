@@ -13,6 +13,7 @@
 #include "common.cuh"
 #include "gemm.cuh"
 #include "gemm_fp8.cuh"
+#include "gemm_t.cuh"
 #include "permute.cuh"
 #include "route.cuh"
 
@@ -121,6 +122,12 @@ cudaError_t set_gemm_attr() {
                               cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
 }
 
+template <int KIND>
+cudaError_t set_down_attr() {
+  return cudaFuncSetAttribute(gemmt::k_down_gemm<KIND>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
+}
+
 moe_status device_setup(int* sms) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MOE_ERR_CUDA;
@@ -130,11 +137,10 @@ moe_status device_setup(int* sms) {
     if (cudaDeviceGetAttribute(&di.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
       return MOE_ERR_CUDA;
     cudaError_t e = cudaSuccess;
-    if (e == cudaSuccess) e = set_gemm_attr<0, gemm::EPI_F32_STORE>();
     if (e == cudaSuccess) e = set_gemm_attr<0, gemm::EPI_SWIGLU>();
-    if (e == cudaSuccess) e = set_gemm_attr<0, gemm::EPI_SCATTER>();
     if (e == cudaSuccess) e = set_gemm_attr<1, gemm::EPI_SWIGLU>();
-    if (e == cudaSuccess) e = set_gemm_attr<1, gemm::EPI_SCATTER>();
+    if (e == cudaSuccess) e = set_down_attr<0>();
+    if (e == cudaSuccess) e = set_down_attr<1>();
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(gemm8::k_gemm_promoted<0, gemm8::EPI_F32_STORE>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
@@ -453,10 +459,11 @@ moe_status do_grouped(const Dims& D, const Layout& L, const void* x, const void*
   const uint32_t fmt = D.f32 ? 2u : 1u;
   const int kbe = (int)(gemm::KB / esz);
   const int64_t hrows = D.R + D.Ks * D.T;
-  // upper bound on m-tiles over all groups
+  // upper bound on 128-row m-tiles over all groups
   const int64_t mt_bound = (D.R + (int64_t)D.N * 127) / 128 + D.Ks * ((D.T + 127) / 128);
 
-  // GEMM1: H = SiLU(A Wg^T) * (A Wu^T)
+  // GEMM1: H = SiLU(A Wg^T) * (A Wu^T); token rows on the UMMA M side, 128 gate
+  // and 128 up columns per tile
   {
     int hn = 128;
     while (hn > 16 && D.I % hn) hn >>= 1;
@@ -488,38 +495,47 @@ moe_status do_grouped(const Dims& D, const Layout& L, const void* x, const void*
     if (rc != MOE_OK) return rc;
     if ((rc = trace(3, st)) != MOE_OK) return rc;
   }
-  // GEMM2: Y = H Wd^T, times g, scattered to the token-major slots
+  // GEMM2: Y = H Wd^T, times g, scattered to the token-major slots; W_down rows
+  // on the UMMA M side and up to 256 tokens per tile, so an expert's token
+  // tail costs at most 15 padded rows
   {
-    int bn = 256;
-    while (bn > 16 && D.d % bn) bn >>= 1;
-    if (D.d % bn) return MOE_ERR_UNSUPPORTED;
-    CUtensorMap ta, tb;
-    rc = make_tmap(&ta, hbuf, esz, D.I, hrows, gemm::BM);
-    if (rc == MOE_OK) rc = make_tmap(&tb, w_down, esz, D.I, (uint64_t)E * D.d, bn);
+    CUtensorMap tw, th;
+    rc = make_tmap(&tw, w_down, esz, D.I, (uint64_t)E * D.d, gemmt::WM);
+    if (rc == MOE_OK) rc = make_tmap(&th, hbuf, esz, D.I, hrows, 256);
     if (rc != MOE_OK) return rc;
-    gemm::Args a;
+    gemmt::Args a;
     memset(&a, 0, sizeof(a));
     a.gt.base = gtab;
     a.gt.n = E;
-    a.n_tiles_n = (int)(D.d / bn);
+    a.TN = 256;
+    a.n_wt = (int)((D.d + gemmt::WM - 1) / gemmt::WM);
     a.num_kb = (int)(D.I * esz / gemm::KB);
     a.kb_elems = kbe;
-    a.bn = bn;
-    a.b_rows_per_expert = (int)D.d;
-    a.a_from_crow = 1;
-    a.idesc = umma_idesc(fmt, gemm::BM, bn);
-    a.out = y_slots;
-    a.out_ld = D.d;
+    a.w_rows_per_expert = (int)D.d;
+    a.fmt = fmt;
     a.out_bf16 = D.f32 ? 0 : 1;
+    a.y = y_slots;
+    a.d = (int)D.d;
     a.pair_of = pair_of;
     a.topk_w = topk_w;
     a.K = (int)D.K;
     a.Ks = (int)D.Ks;
-    const int64_t tiles = mt_bound * a.n_tiles_n;
+    const int a_bytes = gemmt::WM * gemmt::KB, b_bytes = a.TN * gemmt::KB;
+    int stages = 0;
+    for (int s = 8; s >= 2 && !stages; --s)
+      if (gemmt::smem_bytes(a_bytes, b_bytes, s, E) <= (size_t)kMaxSmem) stages = s;
+    if (!stages) return MOE_ERR_UNSUPPORTED;
+    a.stages = stages;
+    const size_t smem = gemmt::smem_bytes(a_bytes, b_bytes, stages, E);
+    const int64_t tiles =
+        ((D.R + (int64_t)D.N * 255) / 256 + D.Ks * ((D.T + 255) / 256)) * a.n_wt;
     const int grid = (int)(tiles < sms ? tiles : sms);
-    rc = kind == 0 ? launch_gemm<0, gemm::EPI_SCATTER>(ta, ta, tb, a, grid, st)
-                   : launch_gemm<1, gemm::EPI_SCATTER>(ta, ta, tb, a, grid, st);
-    if (rc == MOE_OK) rc = trace(4, st);
+    if (kind == 0)
+      gemmt::k_down_gemm<0><<<grid, gemmt::NUM_THREADS, smem, st>>>(tw, th, a);
+    else
+      gemmt::k_down_gemm<1><<<grid, gemmt::NUM_THREADS, smem, st>>>(tw, th, a);
+    if ((rc = launched("down-projection GEMM")) != MOE_OK) return rc;
+    rc = trace(4, st);
   }
   return rc;
 }

@@ -1,8 +1,9 @@
-// Persistent grouped GEMM on tcgen05 / TMEM, fed by TMA.
+// Persistent grouped GEMM on tcgen05 / TMEM, fed by TMA: the gate/up
+// projection with the SwiGLU epilogue (GEMM1).
 //
 // One launch computes C_g = A_g * B_g^T for a list of row groups g (one per
-// expert, or one for the router), each A_g a block of rows of an activation
-// matrix and B_g one expert's weight matrix, both K-major.  The output tile is
+// expert), each A_g a block of token rows and B_g one expert's W_gate / W_up
+// rows, both K-major.  The output tile is
 // 128 rows x bn accumulator columns; tiles are numbered n-fastest across all
 // groups and strided over the persistent CTAs.
 //
@@ -26,7 +27,7 @@ constexpr int KB = 128;            // bytes of K per stage = one 128-byte swizzl
 constexpr int NUM_THREADS = 256;
 constexpr int EPI_WARP0 = 4;
 
-enum Epi { EPI_F32_STORE = 0, EPI_SWIGLU = 1, EPI_SCATTER = 2 };
+enum Epi { EPI_SWIGLU = 1 };
 
 // Group table (device, int32), struct of arrays for n groups:
 //   [0, n]           m-tile prefix (exclusive scan of ceil(rows/128)), n+1 entries
@@ -71,14 +72,7 @@ struct Args {
   // epilogue
   void* out;
   long long out_ld;    // elements per output row
-  int out_cols;        // valid output columns (EPI_F32_STORE)
   int out_bf16;        // 1: bf16 output, 0: fp32
-  const int* pair_of;  // SCATTER: permuted row -> t*K + k
-  const float* topk_w; // SCATTER: [T*K]
-  int K, Ks;
-  // prologue: zero an int array (counts) before anything else runs
-  int* zero_ptr;
-  int zero_n;
 };
 
 __device__ __forceinline__ int find_group(const int* prefix, int n, int mt) {
@@ -135,10 +129,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int warp = warp_id(), lane = lane_id();
   const int n_groups = a.gt.count();
 
-  if (a.zero_ptr) {
-    for (int i = blockIdx.x * NUM_THREADS + threadIdx.x; i < a.zero_n; i += gridDim.x * NUM_THREADS)
-      a.zero_ptr[i] = 0;
-  }
   for (int i = threadIdx.x; i <= n_groups; i += NUM_THREADS) s_prefix[i] = a.gt.prefix(i);
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -257,23 +247,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)acc * (a.tmem_cols / 2);
       const int grow = lm * BM + r;                 // row inside the group
       const bool valid = grow < a.gt.rows(g);
-      if (EPI == EPI_F32_STORE) {
-        float* orow = reinterpret_cast<float*>(a.out) +
-                      (long long)(a.gt.c_row(g) + grow) * a.out_ld + (long long)nt * a.bn;
-        for (int c = 0; c < a.bn; c += 16) {
-          float v[16];
-          tmem_ld16(tb + (uint32_t)c, v);
-          const int col0 = nt * a.bn + c;
-          if (valid) {
-            if (col0 + 16 <= a.out_cols) {
-              store16(orow + c, v, 0);
-            } else {
-              for (int i = 0; i < 16; ++i)
-                if (col0 + i < a.out_cols) orow[c + i] = v[i];
-            }
-          }
-        }
-      } else if (EPI == EPI_SWIGLU) {
+      {
         const int hn = a.b_half;
         const size_t esz = a.out_bf16 ? 2 : 4;
         uint8_t* orow = reinterpret_cast<uint8_t*>(a.out) +
@@ -285,30 +259,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
           for (int i = 0; i < 16; ++i) gv[i] = silu_f(gv[i]) * uv[i];
           if (valid) store16(orow + (size_t)c * esz, gv, a.out_bf16);
-        }
-      } else {  // EPI_SCATTER
-        long long dst = 0;
-        float w = 1.0f;
-        if (valid) {
-          const int s_idx = a.gt.aux(g);
-          if (s_idx < 0) {
-            const int pair = a.pair_of[a.gt.c_row(g) + grow];
-            const int t = pair / a.K, k = pair - t * a.K;
-            dst = (long long)t * (a.K + a.Ks) + k;
-            w = a.topk_w[pair];
-          } else {
-            dst = (long long)grow * (a.K + a.Ks) + a.K + s_idx;
-          }
-        }
-        const size_t esz = a.out_bf16 ? 2 : 4;
-        uint8_t* orow = reinterpret_cast<uint8_t*>(a.out) +
-                        ((size_t)dst * (size_t)a.out_ld + (size_t)nt * a.bn) * esz;
-        for (int c = 0; c < a.bn; c += 16) {
-          float v[16];
-          tmem_ld16(tb + (uint32_t)c, v);
-#pragma unroll
-          for (int i = 0; i < 16; ++i) v[i] *= w;
-          if (valid) store16(orow + (size_t)c * esz, v, a.out_bf16);
         }
       }
       tc_fence_before();

@@ -75,18 +75,17 @@ __device__ __forceinline__ void route_token(const float (&l)[VPL], const float* 
     const int gsz = p.N / p.n_group;
     // lane g (< n_group) ends up holding the score of group g
     float my_gscore = -INFINITY;
-    for (int g = 0; g < p.n_group; ++g) {
-      float b1 = -INFINITY, b2 = -INFINITY;   // two largest keys of this lane in group g
+    const int lpg = gsz / VPL;  // lanes per group when groups are whole lanes
+    if (gsz % VPL == 0 && lpg <= 32 && (lpg & (lpg - 1)) == 0) {
+      // every lane's VPL experts lie in one group: per-lane top-2, then a
+      // butterfly merge over the group's lpg lanes
+      float b1 = -INFINITY, b2 = -INFINITY;
 #pragma unroll
       for (int j = 0; j < VPL; ++j) {
-        const int e = lane * VPL + j;
-        if (e < p.N && e / gsz == g) {
-          const float v = key[j];
-          if (v > b1) { b2 = b1; b1 = v; } else if (v > b2) { b2 = v; }
-        }
+        const float v = key[j];
+        if (v > b1) { b2 = b1; b1 = v; } else if (v > b2) { b2 = v; }
       }
-#pragma unroll
-      for (int o = 16; o; o >>= 1) {
+      for (int o = 1; o < lpg; o <<= 1) {
         const float o1 = __shfl_xor_sync(0xffffffffu, b1, o);
         const float o2 = __shfl_xor_sync(0xffffffffu, b2, o);
         const float hi = fmaxf(b1, o1);
@@ -94,7 +93,33 @@ __device__ __forceinline__ void route_token(const float (&l)[VPL], const float* 
         b1 = hi;
         b2 = lo;
       }
-      if (lane == g) my_gscore = b1 + b2;
+      const float gs = b1 + b2;  // the group score, held by each of its lanes
+      // move group g's score to lane g
+      const int src = lane * lpg;
+      const float moved = __shfl_sync(0xffffffffu, gs, src < 32 ? src : 0);
+      if (lane < p.n_group) my_gscore = moved;
+    } else {
+      for (int g = 0; g < p.n_group; ++g) {
+        float b1 = -INFINITY, b2 = -INFINITY;   // two largest keys of this lane in group g
+#pragma unroll
+        for (int j = 0; j < VPL; ++j) {
+          const int e = lane * VPL + j;
+          if (e < p.N && e / gsz == g) {
+            const float v = key[j];
+            if (v > b1) { b2 = b1; b1 = v; } else if (v > b2) { b2 = v; }
+          }
+        }
+#pragma unroll
+        for (int o = 16; o; o >>= 1) {
+          const float o1 = __shfl_xor_sync(0xffffffffu, b1, o);
+          const float o2 = __shfl_xor_sync(0xffffffffu, b2, o);
+          const float hi = fmaxf(b1, o1);
+          const float lo = fmaxf(fminf(b1, o1), fmaxf(b2, o2));
+          b1 = hi;
+          b2 = lo;
+        }
+        if (lane == g) my_gscore = b1 + b2;
+      }
     }
     // keep the topk_group best groups (score desc, group asc)
     uint32_t keep = 0;

@@ -221,3 +221,47 @@ def max_abs_rel(got: np.ndarray, ref: np.ndarray) -> float:
     if den == 0.0:
         return float(np.max(np.abs(np.asarray(got, np.float64)))) if ref.size else 0.0
     return float(np.max(np.abs(np.asarray(got, np.float64) - ref)) / den)
+
+
+# ----------------------------------------------------------------------------- load balance
+def bias_update(bias: np.ndarray, counts: np.ndarray, gamma: float) -> np.ndarray:
+    """One step of the auxiliary-loss-free balancing rule.
+
+    b_i <- b_i - gamma when expert i is overloaded (its load above the mean
+    load T*K/N), b_i + gamma when underloaded (below it), unchanged at the mean
+    (DeepSeek Technical Report: MoE Architecture, §3.3 bias update rule,
+    gamma = 0.001).  The bias is stored in fp32, so the step is one fp32
+    subtraction or addition."""
+    b = np.asarray(bias, np.float32)
+    c = np.asarray(counts, np.int64)
+    total, n = int(c.sum()), len(c)
+    over = c * n > total            # load above the mean, compared exactly in integers
+    under = c * n < total
+    g = np.float32(gamma)
+    out = b.copy()
+    out[over] = (b[over] - g).astype(np.float32)
+    out[under] = (b[under] + g).astype(np.float32)
+    return out
+
+
+def balance_stats(s: np.ndarray, idx: np.ndarray, seq_len: int):
+    """Routing statistics per sequence of seq_len consecutive tokens.
+
+    f[q, i] = fraction of the sequence's tokens that selected expert i and
+    P[q, i] = mean affinity s_i over the sequence's tokens (DeepSeek Technical
+    Report: MoE Architecture, §1.2: f_i, P_i of L_ExpBal = alpha_1 sum_i f_i P_i;
+    with seq_len = T they are the batch-level statistics, with a shorter
+    seq_len the per-sequence ones of the sequence-wise balance loss of §3.3)."""
+    s = np.asarray(s, np.float64)
+    idx = np.asarray(idx, np.int64)
+    T, N = s.shape
+    if seq_len <= 0 or T % seq_len:
+        raise ValueError("seq_len must divide T")
+    S = T // seq_len
+    f = np.zeros((S, N))
+    P = np.zeros((S, N))
+    for q in range(S):
+        rows = slice(q * seq_len, (q + 1) * seq_len)
+        f[q] = np.bincount(idx[rows].reshape(-1), minlength=N) / seq_len
+        P[q] = s[rows].mean(axis=0)
+    return f, P

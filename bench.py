@@ -28,6 +28,30 @@ sys.path.insert(0, ROOT)
 
 DEFAULT_CONFIG = "v3_bf16"
 
+# DRAM traffic per launch of the GEMM1 kernel (dram__bytes_read.sum +
+# dram__bytes_write.sum from one ncu capture at full size, see profiles/
+# traffic_v3_bf16_T16384.md), with the sha256 of the kernel's sources at the
+# time of the capture: once the kernel changes, the number no longer applies.
+GEMM1_TRAFFIC = {"v3_bf16": {"bytes": 22257246464,
+                             "sources": "d210f10575955179d6b51e3d27cd89bf096124a9e180fd55a22873533d1034a3"}}
+GEMM1_SOURCES = ("forward_moe_route_b200/csrc/gemm.cuh", "forward_moe_route_b200/csrc/common.cuh")
+
+
+def sources_sha() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for rel in GEMM1_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def gemm1_traffic(cfg):
+    rec = GEMM1_TRAFFIC.get(cfg.name)
+    if not rec or rec["sources"] != sources_sha():
+        return None
+    return rec["bytes"]
+
 
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -383,7 +407,8 @@ def run_ours(args, cfg):
             "route_permute_combine_frac_of_hbm": rpc_gbs / pk["hbm_gbs"],
             "roofline": {"kernel": "grouped GEMM 1 (gate/up + SwiGLU epilogue)",
                          "bound": "tensor", "achieved": g1_tflops, "peak": peak,
-                         "unit": "TFLOP/s", "frac": g1_tflops / peak, "traffic": None,
+                         "unit": "TFLOP/s", "frac": g1_tflops / peak,
+                         "traffic": gemm1_traffic(cfg),
                          "peak_source": f"{pk['source']} bf16 sustained x {ratio} "
                                         f"(nominal {cfg.dtype}/bf16 ratio)"},
             "roofline_gemm2": {"kernel": "grouped GEMM 2 (down + weighted scatter)",

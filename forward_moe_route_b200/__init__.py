@@ -56,6 +56,9 @@ _SIGS = {
     "moe_combine": (ctypes.c_int, [_D, _P, _P, _P, _P]),
     "moe_forward": (ctypes.c_int, [_D, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                                    ctypes.c_size_t, _P]),
+    "moe_route_affinities": (ctypes.c_int, [_D, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "moe_balance_stats": (ctypes.c_int, [_D, _P, _P, ctypes.c_int32, _P, _P, _P]),
+    "moe_bias_update": (ctypes.c_int, [_D, _P, _P, ctypes.c_float, _P]),
     "moe_quantize_fp8_blockwise": (ctypes.c_int, [_P, ctypes.c_int32, ctypes.c_int32,
                                                   ctypes.c_int32, _P, _P, _P]),
     "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
@@ -177,6 +180,22 @@ def moe_forward(desc, x, x_residual, w_router, bias, w_gu, w_gu_scale, w_down, w
                             _ptr(bias), _ptr(w_gu), _ptr(w_gu_scale), _ptr(w_down),
                             _ptr(w_down_scale), _ptr(h), _ptr(topk_idx), _ptr(counts), _ptr(ws),
                             ws.numel() if ws is not None else 0, _stream(stream)), "moe_forward")
+
+
+def moe_route_affinities(desc, x, w_router, s_out, ws, stream=None) -> None:
+    _check(_lib.moe_route_affinities(ctypes.byref(desc), _ptr(x), _ptr(w_router), _ptr(s_out),
+                                     _ptr(ws), ws.numel() if ws is not None else 0,
+                                     _stream(stream)), "moe_route_affinities")
+
+
+def moe_balance_stats(desc, s, topk_idx, seq_len: int, f_out, p_out, stream=None) -> None:
+    _check(_lib.moe_balance_stats(ctypes.byref(desc), _ptr(s), _ptr(topk_idx), seq_len,
+                                  _ptr(f_out), _ptr(p_out), _stream(stream)), "moe_balance_stats")
+
+
+def moe_bias_update(desc, counts, bias, gamma: float, stream=None) -> None:
+    _check(_lib.moe_bias_update(ctypes.byref(desc), _ptr(counts), _ptr(bias), gamma,
+                                _stream(stream)), "moe_bias_update")
 
 
 def moe_quantize_fp8_blockwise(w_bf16, rows: int, cols: int, batch: int, w_e4m3, scale,

@@ -262,6 +262,43 @@ void launch_route_f32(const float* x, const float* wr, int d, const float* bias,
 }
 
 // ----------------------------------------------------------------------------- stages
+// bf16 router GEMM on tensor cores: logits [T, N] fp32.  Each 64-element K
+// block is a separate tensor-core product added into fp32 registers with
+// round-to-nearest, so the logits keep fp32 accuracy over the whole of d (the
+// selection is decided on them).  Its prologue zeroes `zero_counts` (if any).
+moe_status launch_router(const Dims& D, const void* x, const void* w_router, float* logits,
+                         int32_t* zero_counts, int sms, cudaStream_t st) {
+  const int N = (int)D.N;
+  CUtensorMap ta, tb;
+  moe_status rc = make_tmap(&ta, x, 2, D.d, D.T, gemm8::BM);
+  if (rc == MOE_OK) rc = make_tmap(&tb, w_router, 2, D.d, D.N, gemm8::BN);
+  if (rc != MOE_OK) return rc;
+  gemm8::Args a;
+  memset(&a, 0, sizeof(a));
+  a.gt.base = nullptr;
+  a.gt.n = 1;
+  a.gt.single_rows = (int)D.T;
+  a.n_tiles_n = (N + gemm8::BN - 1) / gemm8::BN;
+  a.num_kb = (int)(D.d * 2 / gemm8::KB);
+  a.kb_elems = gemm8::KB / 2;
+  a.b_rows_per_expert = 0;
+  a.idesc = umma_idesc(1, gemm8::BM, gemm8::BN);
+  a.out = logits;
+  a.out_ld = N;
+  a.out_cols = N;
+  a.zero_ptr = zero_counts;
+  a.zero_n = zero_counts ? N : 0;
+  int stages = 0;
+  for (int s = 6; s >= 2 && !stages; --s)
+    if (gemm8::smem_bytes(s, 1) <= (size_t)kMaxSmem) stages = s;
+  a.stages = stages;
+  const int tiles = (int)((D.T + 127) / 128) * a.n_tiles_n;
+  gemm8::k_gemm_promoted<0, gemm8::EPI_F32_STORE>
+      <<<tiles < sms ? tiles : sms, gemm8::NUM_THREADS, gemm8::smem_bytes(stages, 1), st>>>(ta, tb,
+                                                                                          a);
+  return launched("router GEMM");
+}
+
 moe_status do_route(const moe_layer_desc& s, const Dims& D, const Layout& L, const void* x,
                     const void* w_router, const float* bias, int32_t* topk_idx, float* topk_w,
                     int32_t* counts, uint8_t* ws, int sms, cudaStream_t st) {
@@ -283,39 +320,9 @@ moe_status do_route(const moe_layer_desc& s, const Dims& D, const Layout& L, con
     else launch_route_f32<16>(xf, wf, dd, bias, p, topk_idx, topk_w, counts, st);
     return launched("k_route_f32");
   }
-  // bf16 router GEMM on tensor cores: logits [T, N] fp32.  Each 64-element K
-  // block is a separate tensor-core product added into fp32 registers with
-  // round-to-nearest, so the logits keep fp32 accuracy over the whole of d
-  // (the selection is decided on them).  Its prologue zeroes the counts.
   float* logits = reinterpret_cast<float*>(ws + L.logits);
-  CUtensorMap ta, tb;
-  moe_status rc = make_tmap(&ta, x, 2, D.d, D.T, gemm8::BM);
-  if (rc == MOE_OK) rc = make_tmap(&tb, w_router, 2, D.d, D.N, gemm8::BN);
+  moe_status rc = launch_router(D, x, w_router, logits, counts, sms, st);
   if (rc != MOE_OK) return rc;
-  gemm8::Args a;
-  memset(&a, 0, sizeof(a));
-  a.gt.base = nullptr;
-  a.gt.n = 1;
-  a.gt.single_rows = (int)D.T;
-  a.n_tiles_n = (N + gemm8::BN - 1) / gemm8::BN;
-  a.num_kb = (int)(D.d * 2 / gemm8::KB);
-  a.kb_elems = gemm8::KB / 2;
-  a.b_rows_per_expert = 0;
-  a.idesc = umma_idesc(1, gemm8::BM, gemm8::BN);
-  a.out = logits;
-  a.out_ld = N;
-  a.out_cols = N;
-  a.zero_ptr = counts;
-  a.zero_n = N;
-  int stages = 0;
-  for (int s = 6; s >= 2 && !stages; --s)
-    if (gemm8::smem_bytes(s, 1) <= (size_t)kMaxSmem) stages = s;
-  a.stages = stages;
-  const int tiles = (int)((D.T + 127) / 128) * a.n_tiles_n;
-  gemm8::k_gemm_promoted<0, gemm8::EPI_F32_STORE>
-      <<<tiles < sms ? tiles : sms, gemm8::NUM_THREADS, gemm8::smem_bytes(stages, 1), st>>>(ta, tb,
-                                                                                          a);
-  if ((rc = launched("router GEMM")) != MOE_OK) return rc;
   if (N <= 32) launch_topk<1>(logits, bias, p, topk_idx, topk_w, counts, st);
   else if (N <= 64) launch_topk<2>(logits, bias, p, topk_idx, topk_w, counts, st);
   else if (N <= 128) launch_topk<4>(logits, bias, p, topk_idx, topk_w, counts, st);
@@ -336,7 +343,7 @@ moe_status do_permute(const Dims& D, const Layout& L, const void* x, const int32
   }
   perm::k_hist<<<D.n_chunks, 256, N * 4, st>>>(topk_idx, T, K, N, hist);
   perm::k_scan<<<1, 1024, 0, st>>>(hist, D.n_chunks, N, counts, offsets);
-  perm::k_slots<<<D.n_chunks, 32, N * 4, st>>>(topk_idx, T, K, N, hist, slot_of, perm_src);
+  perm::k_slots<<<D.n_chunks, perm::SLOT_WARPS * 32, perm::SLOT_WARPS * N * 4, st>>>(topk_idx, T, K, N, hist, slot_of, perm_src);
   if (D.fp8) {
     perm::k_gather_quant<<<(T + 7) / 8, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(x), T, K,
                                                       (int)D.d, (int)D.R, slot_of,
@@ -743,6 +750,67 @@ moe_status moe_forward(const moe_layer_desc* desc, const void* x, const void* x_
   return rc;
 }
 
+moe_status moe_route_affinities(const moe_layer_desc* desc, const void* x, const void* w_router,
+                                float* s_out, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  Dims D;
+  moe_status rc = fill_dims(desc, &D);
+  if (rc != MOE_OK) return rc;
+  if (D.T > 0 && (!x || !w_router || !s_out || !aligned16(x) || !aligned16(w_router) ||
+                  !aligned16(s_out)))
+    return MOE_ERR_INVALID_ARG;
+  const Layout L = layout(D);
+  if (!ws || ws_bytes < L.total || !aligned16(ws)) return MOE_ERR_WORKSPACE;
+  if (D.T == 0) return MOE_OK;
+  int sms;
+  if ((rc = device_setup(&sms)) != MOE_OK) return rc;
+  const route::Params p = route_params(*desc);
+  const int N = (int)D.N, blocks = (int)((D.T + 7) / 8);
+  if (D.f32) {
+    const float* xf = static_cast<const float*>(x);
+    const float* wf = static_cast<const float*>(w_router);
+    const int dd = (int)D.d;
+    if (N <= 32) route::k_affinity_f32<1><<<blocks, 256, 0, stream>>>(xf, wf, dd, p, s_out);
+    else if (N <= 64) route::k_affinity_f32<2><<<blocks, 256, 0, stream>>>(xf, wf, dd, p, s_out);
+    else if (N <= 128) route::k_affinity_f32<4><<<blocks, 256, 0, stream>>>(xf, wf, dd, p, s_out);
+    else if (N <= 256) route::k_affinity_f32<8><<<blocks, 256, 0, stream>>>(xf, wf, dd, p, s_out);
+    else route::k_affinity_f32<16><<<blocks, 256, 0, stream>>>(xf, wf, dd, p, s_out);
+    return launched("k_affinity_f32");
+  }
+  float* logits = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + L.logits);
+  if ((rc = launch_router(D, x, w_router, logits, nullptr, sms, stream)) != MOE_OK) return rc;
+  if (N <= 32) route::k_affinity<1><<<blocks, 256, 0, stream>>>(logits, p, s_out);
+  else if (N <= 64) route::k_affinity<2><<<blocks, 256, 0, stream>>>(logits, p, s_out);
+  else if (N <= 128) route::k_affinity<4><<<blocks, 256, 0, stream>>>(logits, p, s_out);
+  else if (N <= 256) route::k_affinity<8><<<blocks, 256, 0, stream>>>(logits, p, s_out);
+  else route::k_affinity<16><<<blocks, 256, 0, stream>>>(logits, p, s_out);
+  return launched("k_affinity");
+}
+
+moe_status moe_balance_stats(const moe_layer_desc* desc, const float* s, const int32_t* topk_idx,
+                             int32_t seq_len, float* f_out, float* p_out, cudaStream_t stream) {
+  Dims D;
+  moe_status rc = fill_dims(desc, &D);
+  if (rc != MOE_OK) return rc;
+  if (D.T == 0) return MOE_OK;
+  if (seq_len <= 0 || D.T % seq_len) return MOE_ERR_INVALID_ARG;
+  if (!s || !topk_idx || !f_out || !p_out || !aligned16(s) || !aligned16(topk_idx))
+    return MOE_ERR_INVALID_ARG;
+  const dim3 grid((unsigned)(D.T / seq_len), (unsigned)((D.N + 31) / 32));
+  route::k_balance_stats<<<grid, 256, 0, stream>>>(s, topk_idx, (int)D.T, (int)D.N, (int)D.K,
+                                                   seq_len, f_out, p_out);
+  return launched("k_balance_stats");
+}
+
+moe_status moe_bias_update(const moe_layer_desc* desc, const int32_t* counts, float* bias,
+                           float gamma, cudaStream_t stream) {
+  Dims D;
+  moe_status rc = fill_dims(desc, &D);
+  if (rc != MOE_OK) return rc;
+  if (!counts || !bias || !std::isfinite(gamma) || gamma < 0.f) return MOE_ERR_INVALID_ARG;
+  route::k_bias_update<<<1, 512, 0, stream>>>(counts, bias, (int)D.N, (long long)D.T * D.K, gamma);
+  return launched("k_bias_update");
+}
+
 moe_status moe_quantize_fp8_blockwise(const void* w_bf16, int32_t rows, int32_t cols,
                                       int32_t batch, void* w_e4m3, float* scale,
                                       cudaStream_t stream) {
@@ -838,7 +906,7 @@ moe_status moe_permute_noalloc(const moe_layer_desc* desc, const void* x,
   // previous call's contents never leak into this one.
   perm::k_hist<<<D.n_chunks, 256, N * 4, stream>>>(topk_idx, T, K, N, hist);
   perm::k_scan<<<1, 1024, 0, stream>>>(hist, D.n_chunks, N, counts, offsets);
-  perm::k_slots<<<D.n_chunks, 32, N * 4, stream>>>(topk_idx, T, K, N, hist, slot_of, perm_src);
+  perm::k_slots<<<D.n_chunks, perm::SLOT_WARPS * 32, perm::SLOT_WARPS * N * 4, stream>>>(topk_idx, T, K, N, hist, slot_of, perm_src);
   if (D.fp8) {
     perm::k_gather_quant<<<(T + 7) / 8, 256, 0, stream>>>(
         static_cast<const __nv_bfloat16*>(x), T, K, (int)D.d, (int)D.R, slot_of,

@@ -109,17 +109,42 @@ __global__ void __launch_bounds__(1024) k_scan(int32_t* __restrict__ hist, int n
   }
 }
 
-// One warp per chunk: walks the chunk's tokens in order and hands out rows.
-__global__ void __launch_bounds__(32) k_slots(const int32_t* __restrict__ idx, int T, int K, int N,
-                                              const int32_t* __restrict__ base,
-                                              int32_t* __restrict__ slot_of,
-                                              int32_t* __restrict__ perm_src) {
-  extern __shared__ int32_t next[];
-  const int lane = lane_id();
-  for (int e = lane; e < N; e += 32) next[e] = base[(size_t)blockIdx.x * N + e];
-  __syncwarp();
-  const int t0 = blockIdx.x * CHUNK;
-  const int t1 = min(T, t0 + CHUNK);
+// One block of SLOT_WARPS warps per chunk.  Warp w owns tokens
+// [16w, 16w+16) of the chunk: it first counts its pairs per expert, a prefix
+// over the warps gives each warp its first row per expert, and then each warp
+// walks its tokens in order handing out rows (distinct experts within a token
+// never collide), so the result is the same stable order as a single walk.
+constexpr int SLOT_WARPS = 8;
+constexpr int SLOT_TOKENS = CHUNK / SLOT_WARPS;   // 16
+
+__global__ void __launch_bounds__(SLOT_WARPS * 32) k_slots(const int32_t* __restrict__ idx, int T,
+                                                           int K, int N,
+                                                           const int32_t* __restrict__ base,
+                                                           int32_t* __restrict__ slot_of,
+                                                           int32_t* __restrict__ perm_src) {
+  extern __shared__ int32_t sub[];            // [SLOT_WARPS][N] counts, then first rows
+  const int lane = lane_id(), w = warp_id();
+  for (int i = threadIdx.x; i < SLOT_WARPS * N; i += blockDim.x) sub[i] = 0;
+  __syncthreads();
+  const int t0 = blockIdx.x * CHUNK + w * SLOT_TOKENS;
+  const int t1 = min(T, t0 + SLOT_TOKENS);
+  for (int i = t0 * K + lane; i < t1 * K; i += 32) {
+    const int e = idx[i];
+    if ((unsigned)e < (unsigned)N) atomicAdd(&sub[w * N + e], 1);
+  }
+  __syncthreads();
+  // exclusive prefix over the warps, seeded with the chunk's first row per expert
+  for (int e = threadIdx.x; e < N; e += blockDim.x) {
+    int run = base[(size_t)blockIdx.x * N + e];
+#pragma unroll
+    for (int j = 0; j < SLOT_WARPS; ++j) {
+      const int c = sub[j * N + e];
+      sub[j * N + e] = run;
+      run += c;
+    }
+  }
+  __syncthreads();
+  int32_t* next = sub + w * N;
   for (int t = t0; t < t1; ++t) {
     if (lane < K) {
       const int e = idx[(size_t)t * K + lane];

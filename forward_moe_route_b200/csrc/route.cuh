@@ -37,15 +37,13 @@ __device__ __forceinline__ void warp_argmax(float& v, int& i, float& s) {
   }
 }
 
-// Route one token given its N logits spread over the warp: lane l holds the
-// logits of experts l*VPL .. l*VPL+VPL-1 (entries with index >= N are ignored).
+// Affinities of one token in fp32: lane l holds experts l*VPL .. +VPL-1.
+// softmax over the N routed experts (max-subtracted, butterfly sums) or the
+// element-wise sigmoid; entries with index >= N get 0.
 template <int VPL>
-__device__ __forceinline__ void route_token(const float (&l)[VPL], const float* __restrict__ bias,
-                                            const Params& p, int t, int32_t* __restrict__ topk_idx,
-                                            float* __restrict__ topk_w,
-                                            int32_t* __restrict__ counts) {
+__device__ __forceinline__ void affinity_lane(const float (&l)[VPL], const Params& p,
+                                              float (&s)[VPL]) {
   const int lane = lane_id();
-  float s[VPL], key[VPL];
   if (p.gate == MOE_GATE_SOFTMAX) {
     float m = -INFINITY;
 #pragma unroll
@@ -63,8 +61,21 @@ __device__ __forceinline__ void route_token(const float (&l)[VPL], const float* 
     for (int j = 0; j < VPL; ++j) s[j] = s[j] / z;
   } else {
 #pragma unroll
-    for (int j = 0; j < VPL; ++j) s[j] = 1.0f / (1.0f + expf(-l[j]));
+    for (int j = 0; j < VPL; ++j)
+      s[j] = (lane * VPL + j < p.N) ? 1.0f / (1.0f + expf(-l[j])) : 0.f;
   }
+}
+
+// Route one token given its N logits spread over the warp: lane l holds the
+// logits of experts l*VPL .. l*VPL+VPL-1 (entries with index >= N are ignored).
+template <int VPL>
+__device__ __forceinline__ void route_token(const float (&l)[VPL], const float* __restrict__ bias,
+                                            const Params& p, int t, int32_t* __restrict__ topk_idx,
+                                            float* __restrict__ topk_w,
+                                            int32_t* __restrict__ counts) {
+  const int lane = lane_id();
+  float s[VPL], key[VPL];
+  affinity_lane<VPL>(l, p, s);
 #pragma unroll
   for (int j = 0; j < VPL; ++j) {
     const int e = lane * VPL + j;
@@ -229,6 +240,105 @@ __global__ void __launch_bounds__(256) k_route_f32(const float* __restrict__ x,
       if (lane * VPL + j == e) l[j] = acc;
   }
   route_token<VPL>(l, bias, p, t, topk_idx, topk_w, counts);
+}
+
+// Affinities of every token for every routed expert (for balance statistics):
+// s_out [T, N] fp32 from precomputed logits [T, N].
+template <int VPL>
+__global__ void __launch_bounds__(256) k_affinity(const float* __restrict__ logits, const Params p,
+                                                  float* __restrict__ s_out) {
+  const int t = blockIdx.x * 8 + warp_id();
+  if (t >= p.T) return;
+  float l[VPL], s[VPL];
+#pragma unroll
+  for (int j = 0; j < VPL; ++j) {
+    const int e = lane_id() * VPL + j;
+    l[j] = e < p.N ? logits[(size_t)t * p.N + e] : -INFINITY;
+  }
+  affinity_lane<VPL>(l, p, s);
+#pragma unroll
+  for (int j = 0; j < VPL; ++j) {
+    const int e = lane_id() * VPL + j;
+    if (e < p.N) s_out[(size_t)t * p.N + e] = s[j];
+  }
+}
+
+// The same for the fp32 layer, with the logits computed in fp32 on CUDA cores.
+template <int VPL>
+__global__ void __launch_bounds__(256) k_affinity_f32(const float* __restrict__ x,
+                                                      const float* __restrict__ w_r, int d,
+                                                      const Params p, float* __restrict__ s_out) {
+  const int t = blockIdx.x * 8 + warp_id();
+  if (t >= p.T) return;
+  const int lane = lane_id();
+  const float* xr = x + (size_t)t * d;
+  float l[VPL], s[VPL];
+#pragma unroll
+  for (int j = 0; j < VPL; ++j) l[j] = -INFINITY;
+  for (int e = 0; e < p.N; ++e) {
+    const float* wr = w_r + (size_t)e * d;
+    float acc = 0.f;
+    for (int c = lane; c < d; c += 32) acc = fmaf(xr[c], wr[c], acc);
+    acc = warp_sum(acc);
+#pragma unroll
+    for (int j = 0; j < VPL; ++j)
+      if (lane * VPL + j == e) l[j] = acc;
+  }
+  affinity_lane<VPL>(l, p, s);
+#pragma unroll
+  for (int j = 0; j < VPL; ++j) {
+    const int e = lane * VPL + j;
+    if (e < p.N) s_out[(size_t)t * p.N + e] = s[j];
+  }
+}
+
+// Per sequence q of L consecutive tokens and routed expert i:
+//   f[q, i] = (tokens of q that selected i) / L,  P[q, i] = (sum of s[t, i] over q) / L.
+// Block (q, 32-expert slice): lane = expert, the 8 warps split the sequence's
+// tokens into contiguous ranges; the partial sums are combined in warp order,
+// so the result is the same on every run.
+__global__ void __launch_bounds__(256) k_balance_stats(const float* __restrict__ s,
+                                                       const int32_t* __restrict__ idx, int T,
+                                                       int N, int K, int L,
+                                                       float* __restrict__ f_out,
+                                                       float* __restrict__ p_out) {
+  __shared__ float psum[8][32];
+  __shared__ int cnt[32];
+  const int q = blockIdx.x, e0 = blockIdx.y * 32;
+  const int lane = lane_id(), w = warp_id();
+  if (threadIdx.x < 32) cnt[threadIdx.x] = 0;
+  __syncthreads();
+  const int per = (L + 7) / 8;
+  const int ta = q * L + w * per, tb = min(q * L + L, ta + per);
+  const int e = e0 + lane;
+  float acc = 0.f;
+  for (int t = ta; t < tb; ++t) {
+    if (e < N) acc += s[(size_t)t * N + e];
+    if (lane < K) {
+      const int j = idx[(size_t)t * K + lane] - e0;
+      if ((unsigned)j < 32u) atomicAdd(&cnt[j], 1);
+    }
+  }
+  psum[w][lane] = acc;
+  __syncthreads();
+  if (w == 0 && e < N) {
+    float tot = 0.f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) tot += psum[j][lane];
+    p_out[(size_t)q * N + e] = tot / (float)L;
+    f_out[(size_t)q * N + e] = (float)cnt[lane] / (float)L;
+  }
+}
+
+// One step of the auxiliary-loss-free rule: b_i -= gamma above the mean load
+// T*K/N, += gamma below it (compared exactly in integers), in fp32.
+__global__ void k_bias_update(const int32_t* __restrict__ counts, float* __restrict__ bias, int N,
+                              long long total, float gamma) {
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < N; i += gridDim.x * blockDim.x) {
+    const long long c = (long long)counts[i] * N;
+    if (c > total) bias[i] = __fsub_rn(bias[i], gamma);
+    else if (c < total) bias[i] = __fadd_rn(bias[i], gamma);
+  }
 }
 
 __global__ void k_zero_i32(int32_t* p, int n) {

@@ -184,6 +184,31 @@ moe_status moe_forward(const moe_layer_desc* desc, const void* x, const void* x_
                        void* h, int32_t* topk_idx, int32_t* counts, void* ws, size_t ws_bytes,
                        cudaStream_t stream);
 
+/* ---- Load balancing (training-time statistics and the bias update) -------
+ * "DeepSeek Technical Report: MoE Architecture", §1.2 (L_ExpBal = alpha_1
+ * sum_i f_i P_i with f_i the fraction of tokens that chose expert i and P_i
+ * the mean routing probability) and §3.3 (auxiliary-loss-free bias update,
+ * gamma = 0.001; complementary sequence-wise balance loss). */
+
+/* Affinities s [T, N] fp32 of every token for every routed expert, computed
+ * exactly as moe_route computes them (same router GEMM and fp32 softmax or
+ * sigmoid; no bias).  ws as for moe_route. */
+moe_status moe_route_affinities(const moe_layer_desc* desc, const void* x, const void* w_router,
+                                float* s_out, void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/* Per sequence q of seq_len consecutive tokens (seq_len divides T; seq_len = T
+ * gives the batch statistics): f_out[q, i] = fraction of the sequence's tokens
+ * whose topk_idx holds i, p_out[q, i] = mean of s[t, i] over the sequence.
+ * f_out, p_out [T/seq_len, N] fp32.  Deterministic (fixed summation order). */
+moe_status moe_balance_stats(const moe_layer_desc* desc, const float* s, const int32_t* topk_idx,
+                             int32_t seq_len, float* f_out, float* p_out, cudaStream_t stream);
+
+/* One step of the auxiliary-loss-free rule on the fp32 bias [N], in place:
+ * b_i -= gamma when counts[i] is above the mean load T*K/N, b_i += gamma when
+ * below, unchanged when equal (the comparison is exact, in integers). */
+moe_status moe_bias_update(const moe_layer_desc* desc, const int32_t* counts, float* bias,
+                           float gamma, cudaStream_t stream);
+
 /* Offline FP8 quantisation of weights in 128x128 blocks (not on the hot path).
  * w_bf16 [batch, rows, cols] bf16 in; w_e4m3 [batch, rows, cols] bytes out;
  * scale [batch, rows/128, cols/128] fp32 out.  rows, cols multiples of 128.

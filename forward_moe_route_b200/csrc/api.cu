@@ -111,6 +111,8 @@ inline bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 struct DeviceInfo {
   int sms = 0;
   bool attrs_done = false;
+  size_t pair_smem = 0;     // dynamic shared memory the pair count below was taken for
+  int pair_clusters = 0;    // co-resident 2-CTA clusters of the pair down GEMM
 };
 std::mutex g_mu;
 DeviceInfo g_dev[kMaxDevices];
@@ -439,6 +441,61 @@ moe_status do_grouped_fp8(const Dims& D, const Layout& L, const void* x_perm,
   return rc;
 }
 
+// Down projection on 2-CTA clusters: each pair covers 256 W_down rows x up to
+// 256 tokens; the grid is the number of clusters that fit at once, times two.
+moe_status launch_down(int kind, const void* w_down, const void* hbuf, size_t esz,
+                       int64_t hrows, int64_t tok_tiles, gemmt::Args a, cudaStream_t st) {
+  CUtensorMap tw, th;
+  moe_status rc = make_tmap(&tw, w_down, esz, a.num_kb * (uint64_t)a.kb_elems,
+                            (uint64_t)a.gt.n * a.w_rows_per_expert, gemmt::WM);
+  if (rc == MOE_OK)
+    rc = make_tmap(&th, hbuf, esz, a.num_kb * (uint64_t)a.kb_elems, hrows, gemmt::TN / 2);
+  if (rc != MOE_OK) return rc;
+  int stages = 0;
+  for (int s = 8; s >= 2 && !stages; --s)
+    if (gemmt::smem_bytes(s, a.gt.n) <= (size_t)kMaxSmem) stages = s;
+  if (!stages) return MOE_ERR_UNSUPPORTED;
+  a.stages = stages;
+  const size_t smem = gemmt::smem_bytes(stages, a.gt.n);
+  cudaLaunchConfig_t cfg;
+  memset(&cfg, 0, sizeof(cfg));
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.blockDim = dim3(gemmt::NUM_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  int clusters = 0;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    DeviceInfo& di = g_dev[dev];
+    if (di.pair_smem != smem) {
+      cfg.gridDim = dim3(2 * di.sms, 1, 1);
+      e = kind == 0 ? cudaOccupancyMaxActiveClusters(&clusters, gemmt::k_down_gemm<0>, &cfg)
+                    : cudaOccupancyMaxActiveClusters(&clusters, gemmt::k_down_gemm<1>, &cfg);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaOccupancyMaxActiveClusters");
+      di.pair_smem = smem;
+      di.pair_clusters = clusters;
+    }
+    clusters = di.pair_clusters;
+  }
+  if (clusters < 1) return MOE_ERR_UNSUPPORTED;
+  const int64_t tiles = tok_tiles * a.n_wt;
+  if (tiles < clusters) clusters = (int)tiles;
+  cfg.gridDim = dim3(2 * clusters, 1, 1);
+  e = kind == 0 ? cudaLaunchKernelEx(&cfg, gemmt::k_down_gemm<0>, tw, th, a)
+                : cudaLaunchKernelEx(&cfg, gemmt::k_down_gemm<1>, tw, th, a);
+  if (e != cudaSuccess) return cuda_fail(e, "down-projection GEMM (CTA pairs)");
+  return launched("down-projection GEMM (CTA pairs)");
+}
+
 moe_status do_grouped(const Dims& D, const Layout& L, const void* x, const void* x_perm,
                       const float* x_perm_scale, const int32_t* offsets, const int32_t* slot_of,
                       const float* topk_w, const void* w_gu, const float* w_gu_scale,
@@ -503,19 +560,14 @@ moe_status do_grouped(const Dims& D, const Layout& L, const void* x, const void*
     if ((rc = trace(3, st)) != MOE_OK) return rc;
   }
   // GEMM2: Y = H Wd^T, times g, scattered to the token-major slots; W_down rows
-  // on the UMMA M side and up to 256 tokens per tile, so an expert's token
-  // tail costs at most 15 padded rows
+  // on the UMMA M side (256 per CTA pair) and up to 256 tokens per tile, so an
+  // expert's token tail costs at most 31 padded columns
   {
-    CUtensorMap tw, th;
-    rc = make_tmap(&tw, w_down, esz, D.I, (uint64_t)E * D.d, gemmt::WM);
-    if (rc == MOE_OK) rc = make_tmap(&th, hbuf, esz, D.I, hrows, 256);
-    if (rc != MOE_OK) return rc;
     gemmt::Args a;
     memset(&a, 0, sizeof(a));
     a.gt.base = gtab;
     a.gt.n = E;
-    a.TN = 256;
-    a.n_wt = (int)((D.d + gemmt::WM - 1) / gemmt::WM);
+    a.n_wt = (int)((D.d + 2 * gemmt::WM - 1) / (2 * gemmt::WM));
     a.num_kb = (int)(D.I * esz / gemm::KB);
     a.kb_elems = kbe;
     a.w_rows_per_expert = (int)D.d;
@@ -527,21 +579,9 @@ moe_status do_grouped(const Dims& D, const Layout& L, const void* x, const void*
     a.topk_w = topk_w;
     a.K = (int)D.K;
     a.Ks = (int)D.Ks;
-    const int a_bytes = gemmt::WM * gemmt::KB, b_bytes = a.TN * gemmt::KB;
-    int stages = 0;
-    for (int s = 8; s >= 2 && !stages; --s)
-      if (gemmt::smem_bytes(a_bytes, b_bytes, s, E) <= (size_t)kMaxSmem) stages = s;
-    if (!stages) return MOE_ERR_UNSUPPORTED;
-    a.stages = stages;
-    const size_t smem = gemmt::smem_bytes(a_bytes, b_bytes, stages, E);
-    const int64_t tiles =
-        ((D.R + (int64_t)D.N * 255) / 256 + D.Ks * ((D.T + 255) / 256)) * a.n_wt;
-    const int grid = (int)(tiles < sms ? tiles : sms);
-    if (kind == 0)
-      gemmt::k_down_gemm<0><<<grid, gemmt::NUM_THREADS, smem, st>>>(tw, th, a);
-    else
-      gemmt::k_down_gemm<1><<<grid, gemmt::NUM_THREADS, smem, st>>>(tw, th, a);
-    if ((rc = launched("down-projection GEMM")) != MOE_OK) return rc;
+    rc = launch_down(kind, w_down, hbuf, esz, hrows,
+                     (D.R + (int64_t)D.N * 255) / 256 + D.Ks * ((D.T + 255) / 256), a, st);
+    if (rc != MOE_OK) return rc;
     rc = trace(4, st);
   }
   return rc;

@@ -263,13 +263,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int c = 0; c < 4; ++c) {
           float v[16];
           tmem_ld16(tb + (uint32_t)(16 * c), v);
-          if (EPI == EPI_F32_STORE) {
+          // paired fp32 FMA (two lanes of the accumulator per instruction);
+          // the router's unscaled promotion is an FMA with multiplier 1
+          const float m = EPI == EPI_F32_STORE ? 1.0f : (c < 2 ? m0 : m1);
+          const float2 mm = make_float2(m, m);
 #pragma unroll
-            for (int i = 0; i < 16; ++i) acc[16 * c + i] += v[i];
-          } else {
-            const float m = c < 2 ? m0 : m1;
-#pragma unroll
-            for (int i = 0; i < 16; ++i) acc[16 * c + i] = fmaf(m, v[i], acc[16 * c + i]);
+          for (int i = 0; i < 8; ++i) {
+            const float2 r = __ffma2_rn(mm, make_float2(v[2 * i], v[2 * i + 1]),
+                                        make_float2(acc[16 * c + 2 * i], acc[16 * c + 2 * i + 1]));
+            acc[16 * c + 2 * i] = r.x;
+            acc[16 * c + 2 * i + 1] = r.y;
           }
         }
         tc_fence_before();

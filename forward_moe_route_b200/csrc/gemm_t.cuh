@@ -1,23 +1,38 @@
 // Persistent grouped expert GEMM with weights on the UMMA M side and tokens
-// on the N side (D^T = W X^T), on tcgen05 / TMEM, fed by TMA.
+// on the N side (D^T = W X^T), on tcgen05 / TMEM, fed by TMA, run on CTA
+// pairs (tcgen05.mma.cta_group::2).
 //
-// Used for the down projection (GEMM2): a tile is 128 W_down rows (output
-// features) x up to TN = 256 tokens of one expert.  The tile's UMMA takes the
-// tile's own token count rounded up to 16, so an expert's last token tile
-// wastes at most 15 rows of tensor-core work (a 128-row token tile would
-// waste up to 127).  The epilogue scales by each token's gate weight (1 for
-// shared experts) and writes the features into the token's slot row.
-// The per-group token-tile prefix is computed by each CTA from the group table.
-// Weight tiles run fastest inside an expert, so the CTAs of one wave share the
-// expert's token tiles in L2 and each weight tile is reused across the
-// expert's token tiles.
+// Used for the down projection (GEMM2).  A cluster of two CTAs (two SMs)
+// computes a tile of 256 W_down rows (output features) x up to TN = 256
+// tokens of one expert.  Each CTA loads its own 128 weight rows and half of
+// the token tile into its shared memory; the UMMA issued by the even CTA (the
+// leader) reads both CTAs' operands and writes each CTA's 128 rows x all
+// tokens into that CTA's TMEM.  Per SM this moves 32 KB per 128-byte K step
+// instead of 48 KB for a 1-SM 128 x 256 tile, for the same tensor-core work.
+// The tile's UMMA takes the tile's own token count rounded up to 32, so an
+// expert's last token tile wastes at most 31 columns of tensor-core work.
+// The epilogue scales by each token's gate weight (1 for shared experts) and
+// writes the features into the token's slot row.  Weight tiles run fastest
+// inside an expert, so the clusters of one wave share the expert's token
+// tiles in L2.
 //
-// Warp roles (384 threads, one CTA per SM): warp 0 TMA producer, warp 1 MMA
-// issuer, warp 2 TMEM allocator, warps 4..11 epilogue.  Epilogue warp w owns
-// TMEM lanes 32*(w%4) .. +31 (32 features) and every other 16-token chunk
-// ((w-4)/4 selects the parity).  A chunk goes TMEM -> registers -> a per-warp
-// shared-memory transpose -> 16-byte stores along the token's slot row.  Two
-// accumulator buffers of 256 TMEM columns each.
+// Warp roles (384 threads, one CTA per SM, in both CTAs): warp 0 TMA
+// producer, warp 1 MMA issuer (leader only), warp 2 TMEM allocator, warps
+// 4..11 epilogue.  Epilogue warp w owns TMEM lanes 32*(w%4) .. +31 (32
+// features) and every other 16-token chunk ((w-4)/4 selects the parity).  A
+// chunk goes TMEM -> registers -> a per-warp shared-memory transpose ->
+// 16-byte stores along the token's slot row.  Two accumulator buffers of 256
+// TMEM columns each.
+//
+// Synchronisation:
+//   full[s]   leader only: the leader's producer expects both CTAs' bytes; both
+//             CTAs' TMA loads complete on it (cta_group::2 form, leader address)
+//   empty[s]  both CTAs: the leader's MMA commits to its own and the peer's
+//   tfull[a]  both CTAs: the leader's MMA commits to both after a tile
+//   tempty[a] leader only: the epilogue threads of both CTAs arrive (the peer's
+//             through its cluster address)
+// Every wait is bounded; both CTAs finish with a cluster barrier before TMEM
+// is freed, so no CTA leaves while its peer may still touch its barriers.
 #pragma once
 
 #include "common.cuh"
@@ -26,20 +41,19 @@
 namespace moe {
 namespace gemmt {
 
-constexpr int WM = 128;              // weight rows per tile (UMMA M)
-constexpr int KB = 128;              // bytes of K per k-block
+constexpr int WM = 128;            // weight rows per CTA (the pair covers 256)
+constexpr int KB = 128;
+constexpr int TN = 256;            // tokens per pair tile (128 per CTA)
 constexpr int NUM_THREADS = 384;
 constexpr int EPI_WARP0 = 4;
 constexpr int NUM_EPI_WARPS = 8;
-constexpr int XPOSE_BYTES = 16 * 32 * 4;    // per-warp transpose buffer (16 tokens x 32 fp32)
-constexpr int ACC_COLS = 256;        // TMEM columns per accumulator buffer
+constexpr int XPOSE_BYTES = 16 * 32 * 4;
+constexpr int ACC_COLS = 256;
 constexpr int TMEM_COLS = 512;
-
 
 struct Args {
   gemm::GroupTab gt;
-  int TN;                  // tokens per tile (256)
-  int n_wt;                // weight tiles per expert (ceil(d/128))
+  int n_wt;                // weight tiles of 256 rows per expert
   int num_kb;
   int kb_elems;
   int w_rows_per_expert;   // d
@@ -53,23 +67,75 @@ struct Args {
   int K, Ks;
 };
 
-__host__ inline size_t smem_bytes(int a_bytes, int b_bytes, int stages, int n_groups) {
-  return 1024 + (size_t)stages * (a_bytes + b_bytes) + (size_t)NUM_EPI_WARPS * XPOSE_BYTES +
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// shared::cluster address of the same shared variable in CTA `rank` of the cluster
+__device__ __forceinline__ uint32_t mapa(uint32_t smem_addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_addr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;"
+               ::: "memory");
+}
+__device__ __forceinline__ void tma_load_2d_pair(const CUtensorMap* map, uint32_t bar_cluster,
+                                                 void* smem_dst, int32_t x, int32_t y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(smem_dst)),
+      "l"((uint64_t)map), "r"(bar_cluster), "r"(x), "r"(y)
+      : "memory");
+}
+template <int KIND>
+__device__ __forceinline__ void umma_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  if constexpr (KIND == 0) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+  } else {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+  }
+}
+// Arrive once on the barrier at `bar_cluster` (either CTA of the pair) when
+// all tcgen05 operations issued so far have completed.
+__device__ __forceinline__ void umma_commit_pair(uint32_t bar_cluster) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   bar_cluster)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster)
+               : "memory");
+}
+
+__host__ inline size_t smem_bytes(int stages, int n_groups) {
+  return 1024 + (size_t)stages * (WM * KB + (TN / 2) * KB) + (size_t)NUM_EPI_WARPS * XPOSE_BYTES +
          (size_t)(2 * stages + 5) * 8 + 16 + (size_t)(n_groups + 1) * 4 + 64;
 }
 
 template <int KIND>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     k_down_gemm(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmH,
-                const Args a) {
+                     const Args a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  const uint32_t a_bytes = WM * KB;
-  const uint32_t b_bytes = (uint32_t)a.TN * KB;
-  const uint32_t stage_bytes = a_bytes + b_bytes;
+  constexpr uint32_t a_bytes = WM * KB;
+  constexpr uint32_t b_bytes = (TN / 2) * KB;
+  constexpr uint32_t stage_bytes = a_bytes + b_bytes;
   const int S = a.stages;
-  uint8_t* xpose = smem + (size_t)S * stage_bytes;   // NUM_EPI_WARPS x XPOSE_BYTES
+  uint8_t* xpose = smem + (size_t)S * stage_bytes;
   uint64_t* full = reinterpret_cast<uint64_t*>(xpose + NUM_EPI_WARPS * XPOSE_BYTES);
   uint64_t* empty = full + S;
   uint64_t* tfull = empty + S;
@@ -80,13 +146,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   int* s_prefix = reinterpret_cast<int*>(tmem_slot + 4);
 
   const int warp = warp_id(), lane = lane_id();
+  const uint32_t rank = cluster_rank();
+  const bool leader = rank == 0;
   const int n_groups = a.gt.count();
-  // token-tile prefix over the groups: warp 0 scans ceil(rows / TN) 32 at a time
   if (warp == 0) {
     int carry = 0;
     for (int base = 0; base < n_groups; base += 32) {
       const int g = base + lane;
-      const int v = g < n_groups ? (a.gt.rows(g) + a.TN - 1) / a.TN : 0;
+      const int v = g < n_groups ? (a.gt.rows(g) + TN - 1) / TN : 0;
       int incl = v;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
@@ -105,7 +172,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     for (int j = 0; j < 2; ++j) {
       mbar_init(&tfull[j], 1);
-      mbar_init(&tempty[j], NUM_THREADS - EPI_WARP0 * 32);
+      mbar_init(&tempty[j], 2 * NUM_EPI_WARPS * 32);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -115,56 +182,64 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     tma_prefetch_desc(&tmH);
   }
   if (warp == 2) {
-    tmem_alloc(tmem_slot, TMEM_COLS);
-    tmem_relinquish();
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_slot)),
+                 "r"(TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
   }
   tc_fence_before();
   __syncthreads();
+  cluster_sync();      // barrier initialisation is visible to the peer from here on
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const int total_tiles = s_prefix[n_groups] * a.n_wt;
+  const int n_wt = a.n_wt;
+  const int total_tiles = s_prefix[n_groups] * n_wt;
+  const int pair = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;
 
   if (warp == 0) {
-    // ------------------------------------------------------------------ TMA producer
+    // ------------------------------------------------------------------ TMA producer (both CTAs)
     if (elect_one()) {
       int it = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
-        const int tt = tile / a.n_wt, wt = tile - tt * a.n_wt;
+      for (int tile = pair; tile < total_tiles && ok; tile += n_pairs) {
+        const int tt = tile / n_wt, wt = tile - tt * n_wt;
         const int g = gemm::find_group(s_prefix, n_groups, tt);
-        const int tok0 = (tt - s_prefix[g]) * a.TN;
-        const int trow = a.gt.c_row(g) + tok0;     // H rows of the group's tokens
-        const int wrow = a.gt.expert(g) * a.w_rows_per_expert + wt * WM;
+        const int tok0 = (tt - s_prefix[g]) * TN;
+        const int ntok = min(TN, a.gt.rows(g) - tok0);
+        const int nmma = (ntok + 31) & ~31;
+        const int trow = a.gt.c_row(g) + tok0 + (int)rank * (nmma / 2);
+        const int wrow = a.gt.expert(g) * a.w_rows_per_expert + wt * 2 * WM + (int)rank * WM;
         for (int kb = 0; kb < a.num_kb; ++kb, ++it) {
           const int s = it % S;
           const uint32_t ph = (uint32_t)(it / S) & 1u;
           if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag)) { ok = false; break; }
           uint8_t* sa = smem + (size_t)s * stage_bytes;
-          mbar_arrive_expect_tx(&full[s], stage_bytes);
+          const uint32_t full_leader = mapa(smem_u32(&full[s]), 0);
+          if (leader) mbar_arrive_expect_tx(&full[s], 2 * stage_bytes);
           const int kx = kb * a.kb_elems;
-          tma_load_2d(&tmW, &full[s], sa, kx, wrow);
-          tma_load_2d(&tmH, &full[s], sa + a_bytes, kx, trow);
+          tma_load_2d_pair(&tmW, full_leader, sa, kx, wrow);
+          tma_load_2d_pair(&tmH, full_leader, sa + a_bytes, kx, trow);
         }
       }
-      if (!ok) {
-        volatile int no_abort = 0;
-        for (int j = (it - S > 0 ? it - S : 0); j < it; ++j)
-          mbar_wait(&full[j % S], (uint32_t)(j / S) & 1u, &no_abort);
-      }
+      // the copies this CTA issued land before the block may leave (bounded)
+      volatile int no_abort = 0;
+      for (int j = (it - S > 0 ? it - S : 0); j < it; ++j)
+        mbar_wait(&empty[j % S], (uint32_t)(j / S) & 1u, &no_abort);
     }
     __syncwarp();
   } else if (warp == 1) {
-    // ------------------------------------------------------------------ MMA issuer
-    if (elect_one()) {
+    // ------------------------------------------------------------------ MMA issuer (leader)
+    if (leader && elect_one()) {
       int it = 0, tcount = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x, ++tcount) {
-        const int tt = tile / a.n_wt;
+      for (int tile = pair; tile < total_tiles && ok; tile += n_pairs, ++tcount) {
+        const int tt = tile / n_wt;
         const int g = gemm::find_group(s_prefix, n_groups, tt);
-        const int tok0 = (tt - s_prefix[g]) * a.TN;
-        const int ntok = min(a.TN, a.gt.rows(g) - tok0);
-        const int nmma = (ntok + 15) & ~15;
-        const uint32_t idesc = umma_idesc(a.fmt, WM, nmma);
+        const int tok0 = (tt - s_prefix[g]) * TN;
+        const int ntok = min(TN, a.gt.rows(g) - tok0);
+        const int nmma = (ntok + 31) & ~31;
+        const uint32_t idesc = umma_idesc(a.fmt, 2 * WM, nmma);
         const int acc = tcount & 1;
         const uint32_t use = (uint32_t)(tcount >> 1);
         if (!mbar_wait(&tempty[acc], (use & 1u) ^ 1u, abort_flag)) { ok = false; break; }
@@ -180,42 +255,48 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const uint64_t bd = umma_desc_sw128(sa + a_bytes);
 #pragma unroll
           for (int k = 0; k < KB / 32; ++k)
-            umma<KIND>(d_tmem, wd + (uint64_t)(k * 2), bd + (uint64_t)(k * 2), idesc,
-                       (kb | k) != 0 ? 1u : 0u);
-          umma_commit(&empty[s]);
+            umma_pair<KIND>(d_tmem, wd + (uint64_t)(k * 2), bd + (uint64_t)(k * 2), idesc,
+                            (kb | k) != 0 ? 1u : 0u);
+          const uint32_t e_local = smem_u32(&empty[s]);
+          umma_commit_pair(mapa(e_local, 0));
+          umma_commit_pair(mapa(e_local, 1));
         }
-        if (ok) umma_commit(&tfull[acc]);
+        if (ok) {
+          const uint32_t t_local = smem_u32(&tfull[acc]);
+          umma_commit_pair(mapa(t_local, 0));
+          umma_commit_pair(mapa(t_local, 1));
+        }
       }
-      umma_commit(drain);
+      umma_commit_pair(mapa(smem_u32(drain), 0));
       volatile int no_abort = 0;
       mbar_wait(drain, 0, &no_abort);
     }
     __syncwarp();
   } else if (warp >= EPI_WARP0) {
-    // ------------------------------------------------------------------ epilogue
-    const int ew = warp - EPI_WARP0;         // 0..7
-    const int q = warp & 3;                  // TMEM lane quadrant: features q*32 .. +31
-    const int par = ew >> 2;                 // this warp takes chunks c with c % 2 == par
+    // ------------------------------------------------------------------ epilogue (both CTAs)
+    const int ew = warp - EPI_WARP0;
+    const int q = warp & 3;
+    const int par = ew >> 2;
     uint8_t* xb = xpose + (size_t)ew * XPOSE_BYTES;
     const bool bf = a.out_bf16 != 0;
+    const uint32_t tempty_leader0 = mapa(smem_u32(&tempty[0]), 0);
+    const uint32_t tempty_leader1 = mapa(smem_u32(&tempty[1]), 0);
     int tcount = 0;
-    for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x, ++tcount) {
-      const int tt = tile / a.n_wt, wt = tile - tt * a.n_wt;
+    for (int tile = pair; tile < total_tiles; tile += n_pairs, ++tcount) {
+      const int tt = tile / n_wt, wt = tile - tt * n_wt;
       const int g = gemm::find_group(s_prefix, n_groups, tt);
-      const int tok0 = (tt - s_prefix[g]) * a.TN;
+      const int tok0 = (tt - s_prefix[g]) * TN;
       const int rows = a.gt.rows(g);
-      const int ntok = min(a.TN, rows - tok0);
+      const int ntok = min(TN, rows - tok0);
       const int acc = tcount & 1;
       const uint32_t use = (uint32_t)(tcount >> 1);
       if (!mbar_wait(&tfull[acc], use & 1u, abort_flag)) break;
       tc_fence_after();
       const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * ACC_COLS);
-      const int fw0 = wt * WM + q * 32;     // first feature of this warp
+      const int fw0 = wt * 2 * WM + (int)rank * WM + q * 32;
       const int crow = a.gt.c_row(g);
       const int s_idx = a.gt.aux(g);
       const int nch = (ntok + 15) >> 4;
-      // slot row and gate weight of the tile's tokens: lane l holds those of
-      // tokens l, l+32, ..., l+224; broadcast by shuffles
       long long dreg[8];
       float wreg[8];
 #pragma unroll
@@ -225,10 +306,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         wreg[i] = 0.f;
         if (32 * i < ntok && tok < rows) {
           if (s_idx < 0) {
-            const int pair = a.pair_of[crow + tok];
-            const int t = pair / a.K, k = pair - t * a.K;
+            const int pr = a.pair_of[crow + tok];
+            const int t = pr / a.K, k = pr - t * a.K;
             dreg[i] = (long long)t * (a.K + a.Ks) + k;
-            wreg[i] = a.topk_w[pair];
+            wreg[i] = a.topk_w[pr];
           } else {
             dreg[i] = (long long)tok * (a.K + a.Ks) + a.K + s_idx;
             wreg[i] = 1.0f;
@@ -240,7 +321,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if ((c & 1) == par && c < nch) {
           float v[16];
           tmem_ld16(tb + (uint32_t)(16 * c), v);
-          // scale by each token's gate weight and transpose: xb[j][lane]
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
             const float w = __shfl_sync(0xffffffffu, wreg[(16 * c + j) >> 5], (16 * c + j) & 31);
@@ -250,7 +330,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               reinterpret_cast<float*>(xb)[j * 32 + lane] = v[j] * w;
           }
           __syncwarp();
-          // each token's 32 features leave as 16-byte pieces along its slot row
           if (bf) {
 #pragma unroll
             for (int m = 0; m < 2; ++m) {
@@ -280,14 +359,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
       }
       tc_fence_before();
-      mbar_arrive(&tempty[acc]);
+      if (leader) mbar_arrive(&tempty[acc]);
+      else mbar_arrive_cluster(acc ? tempty_leader1 : tempty_leader0);
     }
   }
   tc_fence_before();
   __syncthreads();
+  cluster_sync();      // the peer no longer touches this CTA's barriers or TMEM
   if (warp == 2) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, TMEM_COLS);
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                 "r"(TMEM_COLS)
+                 : "memory");
   }
 }
 

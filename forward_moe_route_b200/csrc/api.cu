@@ -130,6 +130,9 @@ cudaError_t set_down_attr() {
                               cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
 }
 
+// Text of the last CUDA failure on this host thread (moe_last_error_message).
+thread_local char t_errmsg[256] = "";
+
 moe_status device_setup(int* sms) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MOE_ERR_CUDA;
@@ -153,6 +156,25 @@ moe_status device_setup(int* sms) {
       e = cudaFuncSetAttribute(gemm8::k_gemm_promoted<2, gemm8::EPI_SCATTER>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
+    // the promoted GEMMs re-split their registers with setmaxnreg; the split
+    // adds up only if a thread starts with exactly LAUNCH_REGS registers
+    {
+      cudaFuncAttributes fa[3];
+      if (cudaFuncGetAttributes(&fa[0], gemm8::k_gemm_promoted<0, gemm8::EPI_F32_STORE>) !=
+              cudaSuccess ||
+          cudaFuncGetAttributes(&fa[1], gemm8::k_gemm_promoted<2, gemm8::EPI_SWIGLU_Q>) !=
+              cudaSuccess ||
+          cudaFuncGetAttributes(&fa[2], gemm8::k_gemm_promoted<2, gemm8::EPI_SCATTER>) !=
+              cudaSuccess)
+        return MOE_ERR_CUDA;
+      for (const auto& f : fa)
+        if (f.numRegs != gemm8::LAUNCH_REGS) {
+          snprintf(t_errmsg, sizeof(t_errmsg),
+                   "promoted GEMM compiled with %d registers a thread, expected %d", f.numRegs,
+                   gemm8::LAUNCH_REGS);
+          return MOE_ERR_UNSUPPORTED;
+        }
+    }
     if (!g_encode) {
       void* fn = nullptr;
       cudaDriverEntryPointQueryResult q;
@@ -168,8 +190,6 @@ moe_status device_setup(int* sms) {
   return MOE_OK;
 }
 
-// Text of the last CUDA failure on this host thread (moe_last_error_message).
-thread_local char t_errmsg[256] = "";
 
 moe_status cuda_fail(cudaError_t e, const char* where) {
   snprintf(t_errmsg, sizeof(t_errmsg), "%s: %s (%s)", where, cudaGetErrorName(e),

@@ -12,11 +12,20 @@
 // partials (2 x 256 columns) let the MMA of k-block kb+1 overlap the promotion
 // of kb.
 //
-// Warp roles (576 threads, one CTA per SM):
+// Warp roles (640 threads, one CTA per SM):
 //   warp 0      TMA producer (and TMEM allocator)
 //   warp 1      MMA issuer
-//   warps 2..17 16 promotion/epilogue warps: warp w owns TMEM lane quadrant
-//               w % 4 (32 rows) and the 64-column slice (w - 2) / 4 of the tile.
+//   warps 2, 3  idle
+//   warps 4..19 16 promotion/epilogue warps: warp w owns TMEM lane quadrant
+//               w % 4 (32 rows) and the 64-column slice (w - 4) / 4 of the tile.
+// Registers: the register file is split evenly over the SM's four
+// sub-partitions and warp w lives on sub-partition w % 4, so with 20 warps
+// each sub-partition holds 5 and the launch gets 96 registers a thread.  The
+// first warpgroup then drops to 32 (setmaxnreg.dec) and the four epilogue
+// warpgroups rise to 112 (setmaxnreg.inc): 128 x 32 + 512 x 112 = 640 x 96.
+// The extra registers hold two TMEM loads in flight per warp during the
+// promotion (64 accumulators + 32 staging), which halves the number of
+// TMEM round trips per k-block.
 // Tile: 128 rows x 256 accumulator columns.
 //   GEMM1 (SWIGLU): the B tile holds W_gate and W_up rows interleaved in
 //     chunks of 32 (gate 0-31, up 0-31, gate 32-63, up 32-63, ...), so each
@@ -37,8 +46,13 @@ namespace gemm8 {
 constexpr int BM = 128;
 constexpr int BN = 256;
 constexpr int KB = 128;              // bytes = elements of K per k-block
-constexpr int NUM_THREADS = 576;
-constexpr int EPI_WARP0 = 2;
+constexpr int NUM_THREADS = 640;
+constexpr int EPI_WARP0 = 4;
+constexpr int LAUNCH_REGS = 96;      // registers a thread at launch (host checks)
+constexpr int CTRL_REGS = 32;        // first warpgroup after setmaxnreg.dec
+constexpr int EPI_REGS = 112;        // epilogue warpgroups after setmaxnreg.inc
+static_assert(128 * CTRL_REGS + (NUM_THREADS - 128) * EPI_REGS == NUM_THREADS * LAUNCH_REGS,
+              "register split must add up to the launch allocation");
 constexpr int NUM_EPI = NUM_THREADS - EPI_WARP0 * 32;   // 512
 constexpr int TMEM_COLS = 512;       // two 256-column partials
 
@@ -138,79 +152,82 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const int total_tiles = s_prefix[n_groups] * a.n_tiles_n;
-
-  if (warp == 0) {
-    // ------------------------------------------------------------------ TMA producer
-    if (elect_one()) {
-      int it = 0;
-      bool ok = true;
-      for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
-        const int mt = tile / a.n_tiles_n, nt = tile - mt * a.n_tiles_n;
-        const int g = gemm::find_group(s_prefix, n_groups, mt);
-        const int lm = mt - s_prefix[g];
-        const int arow = (a.a_from_crow ? a.gt.c_row(g) : a.gt.a_row(g)) + lm * BM;
-        const int ebase = a.gt.expert(g) * a.b_rows_per_expert;
-        for (int kb = 0; kb < a.num_kb; ++kb, ++it) {
-          const int s = it % S;
-          const uint32_t ph = (uint32_t)(it / S) & 1u;
-          if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag)) { ok = false; break; }
-          uint8_t* sa = smem + (size_t)s * stage_bytes;
-          uint8_t* sb = sa + a_bytes;
-          mbar_arrive_expect_tx(&full[s], stage_bytes);
-          const int kx = kb * a.kb_elems;
-          tma_load_2d(&tmA, &full[s], sa, kx, arow);
-          if (EPI == EPI_SWIGLU_Q) {
-            const int gr = ebase + nt * 128, ur = ebase + a.b_up_off + nt * 128;
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-              tma_load_2d(&tmB, &full[s], sb + (size_t)(2 * c) * 32 * KB, kx, gr + 32 * c);
-              tma_load_2d(&tmB, &full[s], sb + (size_t)(2 * c + 1) * 32 * KB, kx, ur + 32 * c);
+  if (warp < EPI_WARP0) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(CTRL_REGS));
+    if (warp == 0) {
+      // ------------------------------------------------------------------ TMA producer
+      if (elect_one()) {
+        int it = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
+          const int mt = tile / a.n_tiles_n, nt = tile - mt * a.n_tiles_n;
+          const int g = gemm::find_group(s_prefix, n_groups, mt);
+          const int lm = mt - s_prefix[g];
+          const int arow = (a.a_from_crow ? a.gt.c_row(g) : a.gt.a_row(g)) + lm * BM;
+          const int ebase = a.gt.expert(g) * a.b_rows_per_expert;
+          for (int kb = 0; kb < a.num_kb; ++kb, ++it) {
+            const int s = it % S;
+            const uint32_t ph = (uint32_t)(it / S) & 1u;
+            if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag)) { ok = false; break; }
+            uint8_t* sa = smem + (size_t)s * stage_bytes;
+            uint8_t* sb = sa + a_bytes;
+            mbar_arrive_expect_tx(&full[s], stage_bytes);
+            const int kx = kb * a.kb_elems;
+            tma_load_2d(&tmA, &full[s], sa, kx, arow);
+            if (EPI == EPI_SWIGLU_Q) {
+              const int gr = ebase + nt * 128, ur = ebase + a.b_up_off + nt * 128;
+  #pragma unroll
+              for (int c = 0; c < 4; ++c) {
+                tma_load_2d(&tmB, &full[s], sb + (size_t)(2 * c) * 32 * KB, kx, gr + 32 * c);
+                tma_load_2d(&tmB, &full[s], sb + (size_t)(2 * c + 1) * 32 * KB, kx, ur + 32 * c);
+              }
+            } else {
+              tma_load_2d(&tmB, &full[s], sb, kx, ebase + nt * BN);
             }
-          } else {
-            tma_load_2d(&tmB, &full[s], sb, kx, ebase + nt * BN);
           }
         }
-      }
-      if (!ok) {
-        volatile int no_abort = 0;
-        for (int j = (it - S > 0 ? it - S : 0); j < it; ++j)
-          mbar_wait(&full[j % S], (uint32_t)(j / S) & 1u, &no_abort);
-      }
-    }
-    __syncwarp();
-  } else if (warp == 1) {
-    // ------------------------------------------------------------------ MMA issuer
-    if (elect_one()) {
-      int it = 0, pu = 0;
-      bool ok = true;
-      for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
-        for (int kb = 0; kb < a.num_kb; ++kb, ++it, ++pu) {
-          const int s = it % S;
-          const uint32_t ph = (uint32_t)(it / S) & 1u;
-          const int p = pu & 1;
-          const uint32_t pph = (uint32_t)(pu >> 1) & 1u;
-          if (!mbar_wait(&full[s], ph, abort_flag)) { ok = false; break; }
-          if (!mbar_wait(&pempty[p], pph ^ 1u, abort_flag)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t sa = smem_u32(smem + (size_t)s * stage_bytes);
-          const uint64_t ad = umma_desc_sw128(sa);
-          const uint64_t bd = umma_desc_sw128(sa + a_bytes);
-          const uint32_t d_tmem = tmem_base + (uint32_t)(p * BN);
-#pragma unroll
-          for (int k = 0; k < KB / 32; ++k)
-            umma<KIND>(d_tmem, ad + (uint64_t)(k * 2), bd + (uint64_t)(k * 2), a.idesc,
-                    k != 0 ? 1u : 0u);
-          umma_commit(&empty[s]);
-          umma_commit(&pfull[p]);
+        if (!ok) {
+          volatile int no_abort = 0;
+          for (int j = (it - S > 0 ? it - S : 0); j < it; ++j)
+            mbar_wait(&full[j % S], (uint32_t)(j / S) & 1u, &no_abort);
         }
       }
-      // every MMA issued above completes before the block may free TMEM
-      umma_commit(drain);
-      volatile int no_abort = 0;
-      mbar_wait(drain, 0, &no_abort);
+      __syncwarp();
+    } else if (warp == 1) {
+      // ------------------------------------------------------------------ MMA issuer
+      if (elect_one()) {
+        int it = 0, pu = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
+          for (int kb = 0; kb < a.num_kb; ++kb, ++it, ++pu) {
+            const int s = it % S;
+            const uint32_t ph = (uint32_t)(it / S) & 1u;
+            const int p = pu & 1;
+            const uint32_t pph = (uint32_t)(pu >> 1) & 1u;
+            if (!mbar_wait(&full[s], ph, abort_flag)) { ok = false; break; }
+            if (!mbar_wait(&pempty[p], pph ^ 1u, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t sa = smem_u32(smem + (size_t)s * stage_bytes);
+            const uint64_t ad = umma_desc_sw128(sa);
+            const uint64_t bd = umma_desc_sw128(sa + a_bytes);
+            const uint32_t d_tmem = tmem_base + (uint32_t)(p * BN);
+  #pragma unroll
+            for (int k = 0; k < KB / 32; ++k)
+              umma<KIND>(d_tmem, ad + (uint64_t)(k * 2), bd + (uint64_t)(k * 2), a.idesc,
+                      k != 0 ? 1u : 0u);
+            umma_commit(&empty[s]);
+            umma_commit(&pfull[p]);
+          }
+        }
+        // every MMA issued above completes before the block may free TMEM
+        umma_commit(drain);
+        volatile int no_abort = 0;
+        mbar_wait(drain, 0, &no_abort);
+      }
+      __syncwarp();
     }
-    __syncwarp();
   } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(EPI_REGS));
     // ------------------------------------------------------------------ promotion + epilogue
     const int ew = warp - EPI_WARP0;
     const int q = warp & 3;
@@ -259,20 +276,33 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (!mbar_wait(&pfull[p], (uint32_t)(pu >> 1) & 1u, abort_flag)) { ok = false; break; }
         tc_fence_after();
         const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(p * BN + col0);
+        // two batches of two 16-column loads; the router's unscaled promotion
+        // is a paired FMA with multiplier 1
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          float v[16];
-          tmem_ld16(tb + (uint32_t)(16 * c), v);
-          // paired fp32 FMA (two lanes of the accumulator per instruction);
-          // the router's unscaled promotion is an FMA with multiplier 1
-          const float m = EPI == EPI_F32_STORE ? 1.0f : (c < 2 ? m0 : m1);
+        for (int h = 0; h < 2; ++h) {
+          uint32_t va[16], vb[16];
+          tmem_ld16_nowait(tb + (uint32_t)(32 * h), va);
+          tmem_ld16_nowait(tb + (uint32_t)(32 * h + 16), vb);
+          tmem_wait_ld2(va, vb);
+          const float m = EPI == EPI_F32_STORE ? 1.0f : (h == 0 ? m0 : m1);
           const float2 mm = make_float2(m, m);
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
-            const float2 r = __ffma2_rn(mm, make_float2(v[2 * i], v[2 * i + 1]),
-                                        make_float2(acc[16 * c + 2 * i], acc[16 * c + 2 * i + 1]));
-            acc[16 * c + 2 * i] = r.x;
-            acc[16 * c + 2 * i + 1] = r.y;
+            const int o = 32 * h + 2 * i;
+            const float2 r = __ffma2_rn(mm, make_float2(__uint_as_float(va[2 * i]),
+                                                        __uint_as_float(va[2 * i + 1])),
+                                        make_float2(acc[o], acc[o + 1]));
+            acc[o] = r.x;
+            acc[o + 1] = r.y;
+          }
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int o = 32 * h + 16 + 2 * i;
+            const float2 r = __ffma2_rn(mm, make_float2(__uint_as_float(vb[2 * i]),
+                                                        __uint_as_float(vb[2 * i + 1])),
+                                        make_float2(acc[o], acc[o + 1]));
+            acc[o] = r.x;
+            acc[o + 1] = r.y;
           }
         }
         tc_fence_before();

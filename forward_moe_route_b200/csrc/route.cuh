@@ -14,27 +14,18 @@
 namespace moe {
 namespace route {
 
-constexpr int MAXK = 16;
+constexpr int MAXK = 16;   // largest top-K accepted
 
 struct Params {
   int T, N, K, gate, renorm, n_group, topk_group;
   float scale;
 };
 
-// (key desc, index asc) ordering of candidates
-__device__ __forceinline__ bool better(float v, int i, float ov, int oi) {
-  return ov > v || (ov == v && oi < i);
-}
-
-// Warp arg-max over (key, index) carrying the affinity along.
-__device__ __forceinline__ void warp_argmax(float& v, int& i, float& s) {
-#pragma unroll
-  for (int o = 16; o; o >>= 1) {
-    const float ov = __shfl_xor_sync(0xffffffffu, v, o);
-    const int oi = __shfl_xor_sync(0xffffffffu, i, o);
-    const float os = __shfl_xor_sync(0xffffffffu, s, o);
-    if (better(v, i, ov, oi)) { v = ov; i = oi; s = os; }
-  }
+// Unsigned image of a float that orders like the float (-0 folded into +0),
+// so a warp arg-max is one redux.sync max plus a ballot for the lowest lane.
+__device__ __forceinline__ uint32_t ord_key(float v) {
+  const uint32_t u = __float_as_uint(v + 0.0f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
 // Affinities of one token in fp32: lane l holds experts l*VPL .. +VPL-1.
@@ -132,15 +123,15 @@ __device__ __forceinline__ void route_token(const float (&l)[VPL], const float* 
         if (lane == g) my_gscore = b1 + b2;
       }
     }
-    // keep the topk_group best groups (score desc, group asc)
+    // keep the topk_group best groups (score desc, group asc): the largest
+    // orderable score over the candidate lanes, the lowest such lane
     uint32_t keep = 0;
     for (int r = 0; r < p.topk_group; ++r) {
       const bool cand = lane < p.n_group && !((keep >> lane) & 1u);
-      float v = cand ? my_gscore : -INFINITY;
-      int gi = cand ? lane : (1 << 20);
-      float unused = 0.f;
-      warp_argmax(v, gi, unused);
-      if (gi < 32) keep |= 1u << gi;
+      const uint32_t o = cand ? ord_key(my_gscore) : 0u;
+      const uint32_t mx = __reduce_max_sync(0xffffffffu, o);
+      const uint32_t who = __ballot_sync(0xffffffffu, cand && o == mx);
+      if (who) keep |= 1u << (__ffs(who) - 1);
     }
 #pragma unroll
     for (int j = 0; j < VPL; ++j) {
@@ -149,44 +140,38 @@ __device__ __forceinline__ void route_token(const float (&l)[VPL], const float* 
     }
   }
 
-  // top-K by (key desc, index asc)
-  int sel_i[MAXK];
-  float sel_s[MAXK];
+  // top-K by (key desc, index asc), one pick per round: each lane offers its
+  // best untaken expert (lowest index among equal keys), the warp takes the
+  // largest key and, among equal keys, the lowest lane (experts are
+  // lane-major, so that is the lowest index).  Lane k keeps pick k; the
+  // weight denominator is summed in pick order.
   uint32_t taken = 0;
-#pragma unroll
-  for (int k = 0; k < MAXK; ++k) {
-    sel_i[k] = 0;
-    sel_s[k] = 0.f;
-    if (k < p.K) {
-      float v = -INFINITY, sv = 0.f;
-      int bi = 1 << 20;
-#pragma unroll
-      for (int j = 0; j < VPL; ++j) {
-        const int e = lane * VPL + j;
-        if (e < p.N && !((taken >> j) & 1u) && better(v, bi, key[j], e)) {
-          v = key[j];
-          bi = e;
-          sv = s[j];
-        }
-      }
-      warp_argmax(v, bi, sv);
-      sel_i[k] = bi;
-      sel_s[k] = sv;
-      if (bi / VPL == lane) taken |= 1u << (bi - lane * VPL);
-    }
-  }
-  float denom = 1.0f;
-  if (p.renorm) {
-    denom = 0.f;
-#pragma unroll
-    for (int k = 0; k < MAXK; ++k)
-      if (k < p.K) denom += sel_s[k];
-  }
   int my_i = 0;
-  float my_s = 0.f;
+  float my_s = 0.f, denom = 0.f;
+#pragma unroll 1
+  for (int k = 0; k < p.K; ++k) {
+    float v = -INFINITY, bs = 0.f;
+    int bj = -1;
 #pragma unroll
-  for (int k = 0; k < MAXK; ++k)
-    if (lane == k) { my_i = sel_i[k]; my_s = sel_s[k]; }
+    for (int j = 0; j < VPL; ++j) {
+      const int e = lane * VPL + j;
+      if (e < p.N && !((taken >> j) & 1u) && (bj < 0 || key[j] > v)) {
+        v = key[j];
+        bs = s[j];
+        bj = j;
+      }
+    }
+    const uint32_t o = bj >= 0 ? ord_key(v) : 0u;
+    const uint32_t mx = __reduce_max_sync(0xffffffffu, o);
+    const uint32_t who = __ballot_sync(0xffffffffu, bj >= 0 && o == mx);
+    const int wl = __ffs(who) - 1;
+    const int bi = __shfl_sync(0xffffffffu, lane * VPL + bj, wl);
+    const float sv = __shfl_sync(0xffffffffu, bs, wl);
+    if (lane == wl) taken |= 1u << bj;
+    if (lane == k) { my_i = bi; my_s = sv; }
+    denom += sv;
+  }
+  if (!p.renorm) denom = 1.0f;
   if (lane < p.K) {
     const float g = p.renorm ? my_s / denom * p.scale : my_s * p.scale;
     topk_idx[(size_t)t * p.K + lane] = my_i;
@@ -206,10 +191,17 @@ __global__ void __launch_bounds__(256) k_topk(const float* __restrict__ logits,
   if (t >= p.T) return;
   const float* row = logits + (size_t)t * p.N;
   float l[VPL];
+  const int e0 = lane_id() * VPL;
+  if (VPL % 4 == 0 && (p.N & 3) == 0 && e0 + VPL <= p.N) {
+    // rows start 16-byte aligned when N is a multiple of 4
 #pragma unroll
-  for (int j = 0; j < VPL; ++j) {
-    const int e = lane_id() * VPL + j;
-    l[j] = e < p.N ? row[e] : -INFINITY;
+    for (int j = 0; j < VPL; j += 4) {
+      const float4 q = *reinterpret_cast<const float4*>(row + e0 + j);
+      l[j] = q.x; l[j + 1] = q.y; l[j + 2] = q.z; l[j + 3] = q.w;
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < VPL; ++j) l[j] = e0 + j < p.N ? row[e0 + j] : -INFINITY;
   }
   route_token<VPL>(l, bias, p, t, topk_idx, topk_w, counts);
 }

@@ -32,9 +32,9 @@ DEFAULT_CONFIG = "v3_bf16"
 # dram__bytes_write.sum from one ncu capture at full size, see profiles/
 # traffic_v3_bf16_T16384.md), with the sha256 of the kernel's sources at the
 # time of the capture: once the kernel changes, the number no longer applies.
-GEMM1_TRAFFIC = {"v3_bf16": {"bytes": 22257246464,
-                             "sources": "d210f10575955179d6b51e3d27cd89bf096124a9e180fd55a22873533d1034a3"}}
-GEMM1_SOURCES = ("forward_moe_route_b200/csrc/gemm.cuh", "forward_moe_route_b200/csrc/common.cuh")
+GEMM1_TRAFFIC = {}
+GEMM1_SOURCES = ("forward_moe_route_b200/csrc/gemm_gu.cuh", "forward_moe_route_b200/csrc/gemm_t.cuh",
+                 "forward_moe_route_b200/csrc/gemm.cuh", "forward_moe_route_b200/csrc/common.cuh")
 
 
 def sources_sha() -> str:

@@ -14,6 +14,7 @@
 #include "gemm.cuh"
 #include "gemm_fp8.cuh"
 #include "gemm_t.cuh"
+#include "gemm_gu.cuh"
 #include "permute.cuh"
 #include "route.cuh"
 
@@ -111,23 +112,24 @@ inline bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 struct DeviceInfo {
   int sms = 0;
   bool attrs_done = false;
-  size_t pair_smem = 0;     // dynamic shared memory the pair count below was taken for
-  int pair_clusters = 0;    // co-resident 2-CTA clusters of the pair down GEMM
+  // co-resident 2-CTA clusters of the pair GEMMs (0: gate/up, 1: down), and
+  // the dynamic shared memory each count was taken for
+  size_t pair_smem[2] = {0, 0};
+  int pair_clusters[2] = {0, 0};
 };
 std::mutex g_mu;
 DeviceInfo g_dev[kMaxDevices];
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
-template <int KIND, int EPI>
-cudaError_t set_gemm_attr() {
-  return cudaFuncSetAttribute(gemm::k_grouped_gemm<KIND, EPI>,
-                              cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
-}
 
 template <int KIND>
 cudaError_t set_down_attr() {
-  return cudaFuncSetAttribute(gemmt::k_down_gemm<KIND>,
-                              cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
+  cudaError_t e = cudaFuncSetAttribute(gemmt::k_down_gemm<KIND>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(gemmgu::k_gate_up_gemm<KIND>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
+  return e;
 }
 
 // Text of the last CUDA failure on this host thread (moe_last_error_message).
@@ -142,8 +144,6 @@ moe_status device_setup(int* sms) {
     if (cudaDeviceGetAttribute(&di.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
       return MOE_ERR_CUDA;
     cudaError_t e = cudaSuccess;
-    if (e == cudaSuccess) e = set_gemm_attr<0, gemm::EPI_SWIGLU>();
-    if (e == cudaSuccess) e = set_gemm_attr<1, gemm::EPI_SWIGLU>();
     if (e == cudaSuccess) e = set_down_attr<0>();
     if (e == cudaSuccess) e = set_down_attr<1>();
     if (e == cudaSuccess)
@@ -235,30 +235,6 @@ inline moe_status trace(int i, cudaStream_t st) {
   return e == cudaSuccess ? MOE_OK : cuda_fail(e, "cudaEventRecord (stage trace)");
 }
 
-int pick_stages(int bn, int n_groups) {
-  for (int s = 8; s >= 2; --s)
-    if (gemm::smem_bytes(bn, s, n_groups) <= (size_t)kMaxSmem) return s;
-  return 0;
-}
-
-uint32_t tmem_cols_for(int bn) {
-  uint32_t c = 32;
-  while (c < (uint32_t)(2 * bn)) c <<= 1;
-  return c;
-}
-
-template <int KIND, int EPI>
-moe_status launch_gemm(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b,
-                       gemm::Args args, int grid, cudaStream_t st) {
-  const int ng = args.gt.base ? args.gt.n : 1;
-  args.stages = pick_stages(args.bn, ng);
-  if (!args.stages) return MOE_ERR_UNSUPPORTED;
-  args.tmem_cols = tmem_cols_for(args.bn);
-  if (args.tmem_cols > 512) return MOE_ERR_UNSUPPORTED;
-  const size_t smem = gemm::smem_bytes(args.bn, args.stages, ng);
-  gemm::k_grouped_gemm<KIND, EPI><<<grid, gemm::NUM_THREADS, smem, st>>>(a0, a1, b, args);
-  return launched("grouped GEMM launch");
-}
 
 
 
@@ -463,6 +439,45 @@ moe_status do_grouped_fp8(const Dims& D, const Layout& L, const void* x_perm,
 
 // Down projection on 2-CTA clusters: each pair covers 256 W_down rows x up to
 // 256 tokens; the grid is the number of clusters that fit at once, times two.
+// Launch configuration of a 2-CTA cluster kernel: the grid is the number of
+// clusters that fit at once (queried once per kernel and shared-memory size),
+// capped by the tile count, times two.
+template <typename F>
+moe_status pair_config(int slot, F* func, int threads, size_t smem, int64_t tiles,
+                       cudaStream_t st, cudaLaunchConfig_t* cfg, cudaLaunchAttribute* attr) {
+  memset(cfg, 0, sizeof(*cfg));
+  attr->id = cudaLaunchAttributeClusterDimension;
+  attr->val.clusterDim.x = 2;
+  attr->val.clusterDim.y = 1;
+  attr->val.clusterDim.z = 1;
+  cfg->blockDim = dim3(threads, 1, 1);
+  cfg->dynamicSmemBytes = smem;
+  cfg->stream = st;
+  cfg->attrs = attr;
+  cfg->numAttrs = 1;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  int clusters = 0;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    DeviceInfo& di = g_dev[dev];
+    if (di.pair_smem[slot] != smem) {
+      cfg->gridDim = dim3(2 * di.sms, 1, 1);
+      e = cudaOccupancyMaxActiveClusters(&clusters, func, cfg);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaOccupancyMaxActiveClusters");
+      di.pair_smem[slot] = smem;
+      di.pair_clusters[slot] = clusters;
+    }
+    clusters = di.pair_clusters[slot];
+  }
+  if (clusters < 1) return MOE_ERR_UNSUPPORTED;
+  if (tiles < clusters) clusters = (int)tiles;
+  if (clusters < 1) clusters = 1;
+  cfg->gridDim = dim3(2 * clusters, 1, 1);
+  return MOE_OK;
+}
+
 moe_status launch_down(int kind, const void* w_down, const void* hbuf, size_t esz,
                        int64_t hrows, int64_t tok_tiles, gemmt::Args a, cudaStream_t st) {
   CUtensorMap tw, th;
@@ -478,42 +493,48 @@ moe_status launch_down(int kind, const void* w_down, const void* hbuf, size_t es
   a.stages = stages;
   const size_t smem = gemmt::smem_bytes(stages, a.gt.n);
   cudaLaunchConfig_t cfg;
-  memset(&cfg, 0, sizeof(cfg));
   cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.blockDim = dim3(gemmt::NUM_THREADS, 1, 1);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = st;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
-  int clusters = 0;
-  {
-    std::lock_guard<std::mutex> lk(g_mu);
-    DeviceInfo& di = g_dev[dev];
-    if (di.pair_smem != smem) {
-      cfg.gridDim = dim3(2 * di.sms, 1, 1);
-      e = kind == 0 ? cudaOccupancyMaxActiveClusters(&clusters, gemmt::k_down_gemm<0>, &cfg)
-                    : cudaOccupancyMaxActiveClusters(&clusters, gemmt::k_down_gemm<1>, &cfg);
-      if (e != cudaSuccess) return cuda_fail(e, "cudaOccupancyMaxActiveClusters");
-      di.pair_smem = smem;
-      di.pair_clusters = clusters;
-    }
-    clusters = di.pair_clusters;
-  }
-  if (clusters < 1) return MOE_ERR_UNSUPPORTED;
-  const int64_t tiles = tok_tiles * a.n_wt;
-  if (tiles < clusters) clusters = (int)tiles;
-  cfg.gridDim = dim3(2 * clusters, 1, 1);
-  e = kind == 0 ? cudaLaunchKernelEx(&cfg, gemmt::k_down_gemm<0>, tw, th, a)
-                : cudaLaunchKernelEx(&cfg, gemmt::k_down_gemm<1>, tw, th, a);
+  rc = kind == 0 ? pair_config(1, gemmt::k_down_gemm<0>, gemmt::NUM_THREADS, smem,
+                               tok_tiles * a.n_wt, st, &cfg, attr)
+                 : pair_config(1, gemmt::k_down_gemm<1>, gemmt::NUM_THREADS, smem,
+                               tok_tiles * a.n_wt, st, &cfg, attr);
+  if (rc != MOE_OK) return rc;
+  const cudaError_t e = kind == 0 ? cudaLaunchKernelEx(&cfg, gemmt::k_down_gemm<0>, tw, th, a)
+                                  : cudaLaunchKernelEx(&cfg, gemmt::k_down_gemm<1>, tw, th, a);
   if (e != cudaSuccess) return cuda_fail(e, "down-projection GEMM (CTA pairs)");
   return launched("down-projection GEMM (CTA pairs)");
+}
+
+// Gate/up GEMM with the SwiGLU epilogue on CTA pairs: 128 features x up to
+// 256 tokens per cluster tile; shared experts read x, routed experts x_perm.
+moe_status launch_gate_up(int kind, const void* w_gu, const void* x, const void* x_perm,
+                          size_t esz, int64_t T, int64_t R, int64_t tok_tiles, gemmgu::Args a,
+                          cudaStream_t st) {
+  const uint64_t inner = a.num_kb * (uint64_t)a.kb_elems;
+  CUtensorMap tw, tx, txp;
+  moe_status rc = make_tmap(&tw, w_gu, esz, inner, (uint64_t)a.gt.n * a.w_rows_per_expert,
+                            gemmgu::FM);
+  if (rc == MOE_OK) rc = make_tmap(&tx, x, esz, inner, T, gemmgu::TN / 2);
+  if (rc == MOE_OK) rc = make_tmap(&txp, x_perm, esz, inner, R, gemmgu::TN / 2);
+  if (rc != MOE_OK) return rc;
+  int stages = 0;
+  for (int s = 8; s >= 2 && !stages; --s)
+    if (gemmgu::smem_bytes(s, a.gt.n) <= (size_t)kMaxSmem) stages = s;
+  if (!stages) return MOE_ERR_UNSUPPORTED;
+  a.stages = stages;
+  const size_t smem = gemmgu::smem_bytes(stages, a.gt.n);
+  cudaLaunchConfig_t cfg;
+  cudaLaunchAttribute attr[1];
+  rc = kind == 0 ? pair_config(0, gemmgu::k_gate_up_gemm<0>, gemmgu::NUM_THREADS, smem,
+                               tok_tiles * a.n_ft, st, &cfg, attr)
+                 : pair_config(0, gemmgu::k_gate_up_gemm<1>, gemmgu::NUM_THREADS, smem,
+                               tok_tiles * a.n_ft, st, &cfg, attr);
+  if (rc != MOE_OK) return rc;
+  const cudaError_t e =
+      kind == 0 ? cudaLaunchKernelEx(&cfg, gemmgu::k_gate_up_gemm<0>, tw, tx, txp, a)
+                : cudaLaunchKernelEx(&cfg, gemmgu::k_gate_up_gemm<1>, tw, tx, txp, a);
+  if (e != cudaSuccess) return cuda_fail(e, "gate/up GEMM (CTA pairs)");
+  return launched("gate/up GEMM (CTA pairs)");
 }
 
 moe_status do_grouped(const Dims& D, const Layout& L, const void* x, const void* x_perm,
@@ -543,39 +564,26 @@ moe_status do_grouped(const Dims& D, const Layout& L, const void* x, const void*
   const uint32_t fmt = D.f32 ? 2u : 1u;
   const int kbe = (int)(gemm::KB / esz);
   const int64_t hrows = D.R + D.Ks * D.T;
-  // upper bound on 128-row m-tiles over all groups
-  const int64_t mt_bound = (D.R + (int64_t)D.N * 127) / 128 + D.Ks * ((D.T + 127) / 128);
+  // upper bound on 256-token tiles over all groups
+  const int64_t tok_tiles = (D.R + (int64_t)D.N * 255) / 256 + D.Ks * ((D.T + 255) / 256);
 
-  // GEMM1: H = SiLU(A Wg^T) * (A Wu^T); token rows on the UMMA M side, 128 gate
-  // and 128 up columns per tile
+  // GEMM1: H = SiLU(X Wg^T) * (X Wu^T) on CTA pairs: W_gate / W_up rows on the
+  // UMMA M side (64 features of each per CTA), up to 256 tokens per tile, so an
+  // expert's token tail costs at most 31 padded columns
   {
-    int hn = 128;
-    while (hn > 16 && D.I % hn) hn >>= 1;
-    if (D.I % hn) return MOE_ERR_UNSUPPORTED;
-    CUtensorMap ta0, ta1, tb;
-    rc = make_tmap(&ta0, x, esz, D.d, D.T, gemm::BM);
-    if (rc == MOE_OK) rc = make_tmap(&ta1, x_perm, esz, D.d, D.R, gemm::BM);
-    if (rc == MOE_OK) rc = make_tmap(&tb, w_gu, esz, D.d, (uint64_t)E * 2 * D.I, hn);
-    if (rc != MOE_OK) return rc;
-    gemm::Args a;
+    gemmgu::Args a;
     memset(&a, 0, sizeof(a));
     a.gt.base = gtab;
     a.gt.n = E;
-    a.n_tiles_n = (int)(D.I / hn);
+    a.n_ft = (int)((D.I + 2 * gemmgu::FM - 1) / (2 * gemmgu::FM));
     a.num_kb = (int)(D.d * esz / gemm::KB);
     a.kb_elems = kbe;
-    a.bn = 2 * hn;
-    a.b_half = hn;
-    a.b_up_off = (int)D.I;
-    a.b_rows_per_expert = (int)(2 * D.I);
-    a.idesc = umma_idesc(fmt, gemm::BM, 2 * hn);
-    a.out = hbuf;
-    a.out_ld = D.I;
+    a.inter = (int)D.I;
+    a.w_rows_per_expert = (int)(2 * D.I);
+    a.fmt = fmt;
     a.out_bf16 = D.f32 ? 0 : 1;
-    const int64_t tiles = mt_bound * a.n_tiles_n;
-    const int grid = (int)(tiles < sms ? tiles : sms);
-    rc = kind == 0 ? launch_gemm<0, gemm::EPI_SWIGLU>(ta0, ta1, tb, a, grid, st)
-                   : launch_gemm<1, gemm::EPI_SWIGLU>(ta0, ta1, tb, a, grid, st);
+    a.h = hbuf;
+    rc = launch_gate_up(kind, w_gu, x, x_perm, esz, D.T, D.R, tok_tiles, a, st);
     if (rc != MOE_OK) return rc;
     if ((rc = trace(3, st)) != MOE_OK) return rc;
   }
@@ -599,8 +607,7 @@ moe_status do_grouped(const Dims& D, const Layout& L, const void* x, const void*
     a.topk_w = topk_w;
     a.K = (int)D.K;
     a.Ks = (int)D.Ks;
-    rc = launch_down(kind, w_down, hbuf, esz, hrows,
-                     (D.R + (int64_t)D.N * 255) / 256 + D.Ks * ((D.T + 255) / 256), a, st);
+    rc = launch_down(kind, w_down, hbuf, esz, hrows, tok_tiles, a, st);
     if (rc != MOE_OK) return rc;
     rc = trace(4, st);
   }

@@ -21,7 +21,8 @@
 // Synchronisation as in the pair down projection (full / empty / tfull /
 // tempty, every wait bounded, a cluster barrier before TMEM is freed), plus
 // xfull (the up warps' values are in the exchange buffer) and xempty (the
-// gate warps have read them) once per tile.
+// gate warps have read them) twice per tile: the buffer holds 128 tokens, so
+// a tile's 256 tokens go through it in two rounds.
 #pragma once
 
 #include "common.cuh"
@@ -38,7 +39,8 @@ constexpr int NUM_THREADS = 384;
 constexpr int EPI_WARP0 = 4;
 constexpr int NUM_EPI_WARPS = 8;
 constexpr int XPOSE_BYTES = 16 * 32 * 4;   // per gate warp: 16 tokens x 32 features (fp32)
-constexpr int XCHG_BYTES = 2 * TN * 32 * 4; // up values: 2 quadrants x 256 tokens x 32 lanes
+constexpr int XTOK = TN / 2;                  // tokens per exchange round (two rounds a tile)
+constexpr int XCHG_BYTES = 2 * XTOK * 32 * 4; // up values: 2 quadrants x 128 tokens x 32 lanes
 constexpr int ACC_COLS = 256;
 constexpr int TMEM_COLS = 512;
 
@@ -227,7 +229,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int par = (warp - EPI_WARP0) >> 2;  // 16-token chunks of this parity
     const bool up_warp = q >= 2;
     const bool bf = a.out_bf16 != 0;
-    float* xq = xchg + (size_t)(q & 1) * TN * 32;     // this quadrant pair's exchange rows
+    float* xq = xchg + (size_t)(q & 1) * XTOK * 32;   // this quadrant pair's exchange rows
     uint8_t* xb = xpose + (size_t)((q & 1) * 2 + par) * XPOSE_BYTES;
     const uint32_t tempty_leader0 = mapa(smem_u32(&tempty[0]), 0);
     const uint32_t tempty_leader1 = mapa(smem_u32(&tempty[1]), 0);
@@ -243,62 +245,70 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (!mbar_wait(&tfull[acc], use & 1u, abort_flag)) break;
       tc_fence_after();
       const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * ACC_COLS);
-      if (up_warp) {
-        // the gate warps have read the previous tile's values
-        if (!mbar_wait(xempty, ((uint32_t)tcount & 1u) ^ 1u, abort_flag)) break;
+      bool ok = true;
+      const int f_warp = ft * 2 * FM + (int)rank * FM + q * 32;   // first feature (gate warps)
+      const size_t hrow0 = (size_t)a.gt.c_row(g) + tok0;
+      // two exchange rounds of 8 chunks (128 tokens); xu counts rounds
 #pragma unroll 1
-        for (int c = par; c < nch; c += 2) {
-          float v[16];
-          tmem_ld16(tb + (uint32_t)(16 * c), v);
-#pragma unroll
-          for (int j = 0; j < 16; ++j) xq[(16 * c + j) * 32 + lane] = v[j];
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(xfull);
-      } else {
-        if (!mbar_wait(xfull, (uint32_t)tcount & 1u, abort_flag)) break;
-        const int f_warp = ft * 2 * FM + (int)rank * FM + q * 32;   // first feature of the warp
-        const size_t hrow0 = (size_t)a.gt.c_row(g) + tok0;
+      for (int h = 0; h < 2 && ok; ++h) {
+        const uint32_t xu = (uint32_t)(2 * tcount + h);
+        const int c_end = min(nch, 8 * h + 8);
+        if (up_warp) {
+          // the gate warps have read the previous round's values
+          if (!mbar_wait(xempty, (xu & 1u) ^ 1u, abort_flag)) { ok = false; break; }
 #pragma unroll 1
-        for (int c = par; c < nch; c += 2) {
-          float v[16];
-          tmem_ld16(tb + (uint32_t)(16 * c), v);
+          for (int c = 8 * h + par; c < c_end; c += 2) {
+            float v[16];
+            tmem_ld16(tb + (uint32_t)(16 * c), v);
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const float h = gemm::silu_f(v[j]) * xq[(16 * c + j) * 32 + lane];
-            if (bf)
-              reinterpret_cast<__nv_bfloat16*>(xb)[j * 32 + lane] = __float2bfloat16_rn(h);
-            else
-              reinterpret_cast<float*>(xb)[j * 32 + lane] = h;
+            for (int j = 0; j < 16; ++j) xq[(16 * (c - 8 * h) + j) * 32 + lane] = v[j];
           }
           __syncwarp();
-          if (bf) {
-            // token j: 32 features = 64 bytes = 4 pieces; 64 pieces, 2 per lane
+          if (lane == 0) mbar_arrive(xfull);
+        } else {
+          if (!mbar_wait(xfull, xu & 1u, abort_flag)) { ok = false; break; }
+#pragma unroll 1
+          for (int c = 8 * h + par; c < c_end; c += 2) {
+            float v[16];
+            tmem_ld16(tb + (uint32_t)(16 * c), v);
 #pragma unroll
-            for (int m = 0; m < 2; ++m) {
-              const int pi = lane + 32 * m, j = pi >> 2, pc = pi & 3;
-              const int f = f_warp + pc * 8;
-              if (16 * c + j < ntok && f < a.inter)
-                *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.h) +
-                                          (hrow0 + 16 * c + j) * a.inter + f) =
-                    *reinterpret_cast<const uint4*>(xb + j * 64 + pc * 16);
+            for (int j = 0; j < 16; ++j) {
+              const float hv = gemm::silu_f(v[j]) * xq[(16 * (c - 8 * h) + j) * 32 + lane];
+              if (bf)
+                reinterpret_cast<__nv_bfloat16*>(xb)[j * 32 + lane] = __float2bfloat16_rn(hv);
+              else
+                reinterpret_cast<float*>(xb)[j * 32 + lane] = hv;
             }
-          } else {
-            // token j: 32 features = 128 bytes = 8 pieces; 128 pieces, 4 per lane
+            __syncwarp();
+            if (bf) {
+              // token j: 32 features = 64 bytes = 4 pieces; 64 pieces, 2 per lane
 #pragma unroll
-            for (int m = 0; m < 4; ++m) {
-              const int pi = lane + 32 * m, j = pi >> 3, pc = pi & 7;
-              const int f = f_warp + pc * 4;
-              if (16 * c + j < ntok && f < a.inter)
-                *reinterpret_cast<uint4*>(reinterpret_cast<float*>(a.h) +
-                                          (hrow0 + 16 * c + j) * a.inter + f) =
-                    *reinterpret_cast<const uint4*>(xb + j * 128 + pc * 16);
+              for (int m = 0; m < 2; ++m) {
+                const int pi = lane + 32 * m, j = pi >> 2, pc = pi & 3;
+                const int f = f_warp + pc * 8;
+                if (16 * c + j < ntok && f < a.inter)
+                  *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.h) +
+                                            (hrow0 + 16 * c + j) * a.inter + f) =
+                      *reinterpret_cast<const uint4*>(xb + j * 64 + pc * 16);
+              }
+            } else {
+              // token j: 32 features = 128 bytes = 8 pieces; 128 pieces, 4 per lane
+#pragma unroll
+              for (int m = 0; m < 4; ++m) {
+                const int pi = lane + 32 * m, j = pi >> 3, pc = pi & 7;
+                const int f = f_warp + pc * 4;
+                if (16 * c + j < ntok && f < a.inter)
+                  *reinterpret_cast<uint4*>(reinterpret_cast<float*>(a.h) +
+                                            (hrow0 + 16 * c + j) * a.inter + f) =
+                      *reinterpret_cast<const uint4*>(xb + j * 128 + pc * 16);
+              }
             }
+            __syncwarp();
           }
-          __syncwarp();
+          if (lane == 0) mbar_arrive(xempty);
         }
-        if (lane == 0) mbar_arrive(xempty);
       }
+      if (!ok) break;
       tc_fence_before();
       if (leader) mbar_arrive(&tempty[acc]);
       else mbar_arrive_cluster(acc ? tempty_leader1 : tempty_leader0);

@@ -21,8 +21,10 @@
 // Synchronisation as in the pair down projection (full / empty / tfull /
 // tempty, every wait bounded, a cluster barrier before TMEM is freed), plus
 // xfull (the up warps' values are in the exchange buffer) and xempty (the
-// gate warps have read them) twice per tile: the buffer holds 128 tokens, so
-// a tile's 256 tokens go through it in two rounds.
+// gate warps have read them) once per exchange round: the buffer holds a
+// whole tile (256 tokens) or half of one, chosen by the host (the smaller
+// buffer leaves room for another operand stage, which pays when the K loop
+// is long; with a short one the extra round costs more than it saves).
 #pragma once
 
 #include "common.cuh"
@@ -39,8 +41,9 @@ constexpr int NUM_THREADS = 384;
 constexpr int EPI_WARP0 = 4;
 constexpr int NUM_EPI_WARPS = 8;
 constexpr int XPOSE_BYTES = 16 * 32 * 4;   // per gate warp: 16 tokens x 32 features (fp32)
-constexpr int XTOK = TN / 2;                  // tokens per exchange round (two rounds a tile)
-constexpr int XCHG_BYTES = 2 * XTOK * 32 * 4; // up values: 2 quadrants x 128 tokens x 32 lanes
+// up-value exchange buffer: 2 quadrants x xtok tokens x 32 lanes of fp32,
+// xtok = 256 (one round a tile) or 128 (two rounds, one more operand stage)
+__host__ __device__ constexpr int xchg_bytes(int xtok) { return 2 * xtok * 32 * 4; }
 constexpr int ACC_COLS = 256;
 constexpr int TMEM_COLS = 512;
 
@@ -55,10 +58,11 @@ struct Args {
   uint32_t fmt;            // UMMA operand format: 1 bf16, 2 tf32
   int out_bf16;
   void* h;                 // [rows, I]
+  int xtok;                // tokens per exchange round: 256 or 128
 };
 
-__host__ inline size_t smem_bytes(int stages, int n_groups) {
-  return 1024 + (size_t)stages * (2 * FM * KB + (TN / 2) * KB) + XCHG_BYTES +
+__host__ inline size_t smem_bytes(int stages, int n_groups, int xtok) {
+  return 1024 + (size_t)stages * (2 * FM * KB + (TN / 2) * KB) + xchg_bytes(xtok) +
          (size_t)4 * XPOSE_BYTES + (size_t)(2 * stages + 7) * 8 + 16 +
          (size_t)(n_groups + 1) * 4 + 64;
 }
@@ -77,7 +81,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   constexpr uint32_t stage_bytes = a_bytes + b_bytes;
   const int S = a.stages;
   float* xchg = reinterpret_cast<float*>(smem + (size_t)S * stage_bytes);
-  uint8_t* xpose = reinterpret_cast<uint8_t*>(xchg) + XCHG_BYTES;
+  uint8_t* xpose = reinterpret_cast<uint8_t*>(xchg) + xchg_bytes(a.xtok);
   uint64_t* full = reinterpret_cast<uint64_t*>(xpose + 4 * XPOSE_BYTES);
   uint64_t* empty = full + S;
   uint64_t* tfull = empty + S;
@@ -229,7 +233,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int par = (warp - EPI_WARP0) >> 2;  // 16-token chunks of this parity
     const bool up_warp = q >= 2;
     const bool bf = a.out_bf16 != 0;
-    float* xq = xchg + (size_t)(q & 1) * XTOK * 32;   // this quadrant pair's exchange rows
+    float* xq = xchg + (size_t)(q & 1) * a.xtok * 32;  // this quadrant pair's exchange rows
+    const int rch = a.xtok / 16;                        // chunks per round
+    const int rounds = TN / a.xtok;
     uint8_t* xb = xpose + (size_t)((q & 1) * 2 + par) * XPOSE_BYTES;
     const uint32_t tempty_leader0 = mapa(smem_u32(&tempty[0]), 0);
     const uint32_t tempty_leader1 = mapa(smem_u32(&tempty[1]), 0);
@@ -248,32 +254,33 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       bool ok = true;
       const int f_warp = ft * 2 * FM + (int)rank * FM + q * 32;   // first feature (gate warps)
       const size_t hrow0 = (size_t)a.gt.c_row(g) + tok0;
-      // two exchange rounds of 8 chunks (128 tokens); xu counts rounds
+      // exchange rounds of rch chunks; xu counts rounds
 #pragma unroll 1
-      for (int h = 0; h < 2 && ok; ++h) {
-        const uint32_t xu = (uint32_t)(2 * tcount + h);
-        const int c_end = min(nch, 8 * h + 8);
+      for (int h = 0; h < rounds && ok; ++h) {
+        const uint32_t xu = (uint32_t)(rounds * tcount + h);
+        const int c0 = rch * h;
+        const int c_end = min(nch, c0 + rch);
         if (up_warp) {
           // the gate warps have read the previous round's values
           if (!mbar_wait(xempty, (xu & 1u) ^ 1u, abort_flag)) { ok = false; break; }
 #pragma unroll 1
-          for (int c = 8 * h + par; c < c_end; c += 2) {
+          for (int c = c0 + par; c < c_end; c += 2) {
             float v[16];
             tmem_ld16(tb + (uint32_t)(16 * c), v);
 #pragma unroll
-            for (int j = 0; j < 16; ++j) xq[(16 * (c - 8 * h) + j) * 32 + lane] = v[j];
+            for (int j = 0; j < 16; ++j) xq[(16 * (c - c0) + j) * 32 + lane] = v[j];
           }
           __syncwarp();
           if (lane == 0) mbar_arrive(xfull);
         } else {
           if (!mbar_wait(xfull, xu & 1u, abort_flag)) { ok = false; break; }
 #pragma unroll 1
-          for (int c = 8 * h + par; c < c_end; c += 2) {
+          for (int c = c0 + par; c < c_end; c += 2) {
             float v[16];
             tmem_ld16(tb + (uint32_t)(16 * c), v);
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
-              const float hv = gemm::silu_f(v[j]) * xq[(16 * (c - 8 * h) + j) * 32 + lane];
+              const float hv = gemm::silu_f(v[j]) * xq[(16 * (c - c0) + j) * 32 + lane];
               if (bf)
                 reinterpret_cast<__nv_bfloat16*>(xb)[j * 32 + lane] = __float2bfloat16_rn(hv);
               else

@@ -517,15 +517,12 @@ moe_status launch_gate_up(int kind, const void* w_gu, const void* x, const void*
   if (rc == MOE_OK) rc = make_tmap(&tx, x, esz, inner, T, gemmgu::TN / 2);
   if (rc == MOE_OK) rc = make_tmap(&txp, x_perm, esz, inner, R, gemmgu::TN / 2);
   if (rc != MOE_OK) return rc;
-  // a long K loop gains from a fifth operand stage (half-tile exchange rounds);
-  // a short one loses more to the second round than the stage gives back
-  a.xtok = a.num_kb >= 64 ? gemmgu::TN / 2 : gemmgu::TN;
   int stages = 0;
   for (int s = 8; s >= 2 && !stages; --s)
-    if (gemmgu::smem_bytes(s, a.gt.n, a.xtok) <= (size_t)kMaxSmem) stages = s;
+    if (gemmgu::smem_bytes(s, a.gt.n) <= (size_t)kMaxSmem) stages = s;
   if (!stages) return MOE_ERR_UNSUPPORTED;
   a.stages = stages;
-  const size_t smem = gemmgu::smem_bytes(stages, a.gt.n, a.xtok);
+  const size_t smem = gemmgu::smem_bytes(stages, a.gt.n);
   cudaLaunchConfig_t cfg;
   cudaLaunchAttribute attr[1];
   rc = kind == 0 ? pair_config(0, gemmgu::k_gate_up_gemm<0>, gemmgu::NUM_THREADS, smem,

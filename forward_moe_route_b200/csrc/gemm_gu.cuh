@@ -21,10 +21,7 @@
 // Synchronisation as in the pair down projection (full / empty / tfull /
 // tempty, every wait bounded, a cluster barrier before TMEM is freed), plus
 // xfull (the up warps' values are in the exchange buffer) and xempty (the
-// gate warps have read them) once per exchange round: the buffer holds a
-// whole tile (256 tokens) or half of one, chosen by the host (the smaller
-// buffer leaves room for another operand stage, which pays when the K loop
-// is long; with a short one the extra round costs more than it saves).
+// gate warps have read them) once per tile.
 #pragma once
 
 #include "common.cuh"
@@ -41,9 +38,7 @@ constexpr int NUM_THREADS = 384;
 constexpr int EPI_WARP0 = 4;
 constexpr int NUM_EPI_WARPS = 8;
 constexpr int XPOSE_BYTES = 16 * 32 * 4;   // per gate warp: 16 tokens x 32 features (fp32)
-// up-value exchange buffer: 2 quadrants x xtok tokens x 32 lanes of fp32,
-// xtok = 256 (one round a tile) or 128 (two rounds, one more operand stage)
-__host__ __device__ constexpr int xchg_bytes(int xtok) { return 2 * xtok * 32 * 4; }
+constexpr int XCHG_BYTES = 2 * TN * 32 * 4; // up values: 2 quadrants x 256 tokens x 32 lanes
 constexpr int ACC_COLS = 256;
 constexpr int TMEM_COLS = 512;
 
@@ -58,11 +53,10 @@ struct Args {
   uint32_t fmt;            // UMMA operand format: 1 bf16, 2 tf32
   int out_bf16;
   void* h;                 // [rows, I]
-  int xtok;                // tokens per exchange round: 256 or 128
 };
 
-__host__ inline size_t smem_bytes(int stages, int n_groups, int xtok) {
-  return 1024 + (size_t)stages * (2 * FM * KB + (TN / 2) * KB) + xchg_bytes(xtok) +
+__host__ inline size_t smem_bytes(int stages, int n_groups) {
+  return 1024 + (size_t)stages * (2 * FM * KB + (TN / 2) * KB) + XCHG_BYTES +
          (size_t)4 * XPOSE_BYTES + (size_t)(2 * stages + 7) * 8 + 16 +
          (size_t)(n_groups + 1) * 4 + 64;
 }
@@ -81,7 +75,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   constexpr uint32_t stage_bytes = a_bytes + b_bytes;
   const int S = a.stages;
   float* xchg = reinterpret_cast<float*>(smem + (size_t)S * stage_bytes);
-  uint8_t* xpose = reinterpret_cast<uint8_t*>(xchg) + xchg_bytes(a.xtok);
+  uint8_t* xpose = reinterpret_cast<uint8_t*>(xchg) + XCHG_BYTES;
   uint64_t* full = reinterpret_cast<uint64_t*>(xpose + 4 * XPOSE_BYTES);
   uint64_t* empty = full + S;
   uint64_t* tfull = empty + S;
@@ -233,9 +227,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int par = (warp - EPI_WARP0) >> 2;  // 16-token chunks of this parity
     const bool up_warp = q >= 2;
     const bool bf = a.out_bf16 != 0;
-    float* xq = xchg + (size_t)(q & 1) * a.xtok * 32;  // this quadrant pair's exchange rows
-    const int rch = a.xtok / 16;                        // chunks per round
-    const int rounds = TN / a.xtok;
+    float* xq = xchg + (size_t)(q & 1) * TN * 32;     // this quadrant pair's exchange rows
     uint8_t* xb = xpose + (size_t)((q & 1) * 2 + par) * XPOSE_BYTES;
     const uint32_t tempty_leader0 = mapa(smem_u32(&tempty[0]), 0);
     const uint32_t tempty_leader1 = mapa(smem_u32(&tempty[1]), 0);
@@ -251,71 +243,62 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (!mbar_wait(&tfull[acc], use & 1u, abort_flag)) break;
       tc_fence_after();
       const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * ACC_COLS);
-      bool ok = true;
-      const int f_warp = ft * 2 * FM + (int)rank * FM + q * 32;   // first feature (gate warps)
-      const size_t hrow0 = (size_t)a.gt.c_row(g) + tok0;
-      // exchange rounds of rch chunks; xu counts rounds
+      if (up_warp) {
+        // the gate warps have read the previous tile's values
+        if (!mbar_wait(xempty, ((uint32_t)tcount & 1u) ^ 1u, abort_flag)) break;
 #pragma unroll 1
-      for (int h = 0; h < rounds && ok; ++h) {
-        const uint32_t xu = (uint32_t)(rounds * tcount + h);
-        const int c0 = rch * h;
-        const int c_end = min(nch, c0 + rch);
-        if (up_warp) {
-          // the gate warps have read the previous round's values
-          if (!mbar_wait(xempty, (xu & 1u) ^ 1u, abort_flag)) { ok = false; break; }
-#pragma unroll 1
-          for (int c = c0 + par; c < c_end; c += 2) {
-            float v[16];
-            tmem_ld16(tb + (uint32_t)(16 * c), v);
+        for (int c = par; c < nch; c += 2) {
+          float v[16];
+          tmem_ld16(tb + (uint32_t)(16 * c), v);
 #pragma unroll
-            for (int j = 0; j < 16; ++j) xq[(16 * (c - c0) + j) * 32 + lane] = v[j];
+          for (int j = 0; j < 16; ++j) xq[(16 * c + j) * 32 + lane] = v[j];
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(xfull);
+      } else {
+        if (!mbar_wait(xfull, (uint32_t)tcount & 1u, abort_flag)) break;
+        const int f_warp = ft * 2 * FM + (int)rank * FM + q * 32;   // first feature of the warp
+        const size_t hrow0 = (size_t)a.gt.c_row(g) + tok0;
+#pragma unroll 1
+        for (int c = par; c < nch; c += 2) {
+          float v[16];
+          tmem_ld16(tb + (uint32_t)(16 * c), v);
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const float h = gemm::silu_f(v[j]) * xq[(16 * c + j) * 32 + lane];
+            if (bf)
+              reinterpret_cast<__nv_bfloat16*>(xb)[j * 32 + lane] = __float2bfloat16_rn(h);
+            else
+              reinterpret_cast<float*>(xb)[j * 32 + lane] = h;
           }
           __syncwarp();
-          if (lane == 0) mbar_arrive(xfull);
-        } else {
-          if (!mbar_wait(xfull, xu & 1u, abort_flag)) { ok = false; break; }
-#pragma unroll 1
-          for (int c = c0 + par; c < c_end; c += 2) {
-            float v[16];
-            tmem_ld16(tb + (uint32_t)(16 * c), v);
+          if (bf) {
+            // token j: 32 features = 64 bytes = 4 pieces; 64 pieces, 2 per lane
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              const float hv = gemm::silu_f(v[j]) * xq[(16 * (c - c0) + j) * 32 + lane];
-              if (bf)
-                reinterpret_cast<__nv_bfloat16*>(xb)[j * 32 + lane] = __float2bfloat16_rn(hv);
-              else
-                reinterpret_cast<float*>(xb)[j * 32 + lane] = hv;
+            for (int m = 0; m < 2; ++m) {
+              const int pi = lane + 32 * m, j = pi >> 2, pc = pi & 3;
+              const int f = f_warp + pc * 8;
+              if (16 * c + j < ntok && f < a.inter)
+                *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.h) +
+                                          (hrow0 + 16 * c + j) * a.inter + f) =
+                    *reinterpret_cast<const uint4*>(xb + j * 64 + pc * 16);
             }
-            __syncwarp();
-            if (bf) {
-              // token j: 32 features = 64 bytes = 4 pieces; 64 pieces, 2 per lane
+          } else {
+            // token j: 32 features = 128 bytes = 8 pieces; 128 pieces, 4 per lane
 #pragma unroll
-              for (int m = 0; m < 2; ++m) {
-                const int pi = lane + 32 * m, j = pi >> 2, pc = pi & 3;
-                const int f = f_warp + pc * 8;
-                if (16 * c + j < ntok && f < a.inter)
-                  *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.h) +
-                                            (hrow0 + 16 * c + j) * a.inter + f) =
-                      *reinterpret_cast<const uint4*>(xb + j * 64 + pc * 16);
-              }
-            } else {
-              // token j: 32 features = 128 bytes = 8 pieces; 128 pieces, 4 per lane
-#pragma unroll
-              for (int m = 0; m < 4; ++m) {
-                const int pi = lane + 32 * m, j = pi >> 3, pc = pi & 7;
-                const int f = f_warp + pc * 4;
-                if (16 * c + j < ntok && f < a.inter)
-                  *reinterpret_cast<uint4*>(reinterpret_cast<float*>(a.h) +
-                                            (hrow0 + 16 * c + j) * a.inter + f) =
-                      *reinterpret_cast<const uint4*>(xb + j * 128 + pc * 16);
-              }
+            for (int m = 0; m < 4; ++m) {
+              const int pi = lane + 32 * m, j = pi >> 3, pc = pi & 7;
+              const int f = f_warp + pc * 4;
+              if (16 * c + j < ntok && f < a.inter)
+                *reinterpret_cast<uint4*>(reinterpret_cast<float*>(a.h) +
+                                          (hrow0 + 16 * c + j) * a.inter + f) =
+                    *reinterpret_cast<const uint4*>(xb + j * 128 + pc * 16);
             }
-            __syncwarp();
           }
-          if (lane == 0) mbar_arrive(xempty);
+          __syncwarp();
         }
+        if (lane == 0) mbar_arrive(xempty);
       }
-      if (!ok) break;
       tc_fence_before();
       if (leader) mbar_arrive(&tempty[acc]);
       else mbar_arrive_cluster(acc ? tempty_leader1 : tempty_leader0);

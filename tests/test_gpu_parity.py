@@ -44,7 +44,7 @@ def small_cases():
         "v3_small": recipes.small_variant(C["v3_bf16"], T=900, d=512, inter=256),
         "v3_T1": recipes.small_variant(C["v3_bf16"], T=1, d=256, inter=128),
         "v3_T129": recipes.small_variant(C["v3_bf16"], T=129, d=256, inter=128),
-        # long K (64+ k-blocks): the gate/up GEMM exchanges in half-tile rounds
+        # long K: 64 k-blocks per tile
         "v3_d4096": recipes.small_variant(C["v3_bf16"], T=300, d=4096, inter=128),
     }
 

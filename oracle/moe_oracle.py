@@ -125,7 +125,9 @@ def route(x, w_r, bias, *, gate: str, top_k: int, n_group: int = 1, topk_group: 
     s = affinity(logits, gate)
     idx, kgap, ggap = select_experts(s, bias, top_k, n_group, topk_group)
     g = gate_weights(s, idx, renorm, route_scale)
-    return {"logits": logits, "s": s, "idx": idx, "w": g, "kgap": kgap, "ggap": ggap}
+    key = s + np.asarray(bias, np.float64)[None, :] if bias is not None else s
+    return {"logits": logits, "s": s, "key": key, "idx": idx, "w": g, "kgap": kgap,
+            "ggap": ggap}
 
 
 def near_tie_tokens(kgap: np.ndarray, ggap: np.ndarray, thr: float = NEAR_TIE) -> np.ndarray:

@@ -152,6 +152,6 @@ def test_v3_bf16_full():
     check_layer(C["v3_bf16"], 48)
 
 
-@pytest.mark.parametrize("T", [2048, 16384])
+@pytest.mark.parametrize("T", [256, 2048, 16384, 65536])
 def test_v3_fp8_full(T):
     check_layer(C["v3_fp8"].with_T(T), 12)

@@ -202,6 +202,27 @@ inline moe_status launched(const char* where) {
   return e == cudaSuccess ? MOE_OK : cuda_fail(e, where);
 }
 
+// Launch one kernel of the layer's chain with programmatic stream
+// serialisation: its launch may overlap the end of the previous kernel on the
+// stream; the kernel itself waits for that kernel's results (grid_dep_sync).
+template <typename... KArgs, typename... Args>
+moe_status launch_chain(const char* what, void (*kernel)(KArgs...), dim3 grid, dim3 block,
+                        size_t smem, cudaStream_t st, Args... args) {
+  cudaLaunchConfig_t cfg;
+  memset(&cfg, 0, sizeof(cfg));
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, args...);
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, what);
+}
+
 // 2-D K-major tensor map with 128-byte swizzle: rows of `inner` elements,
 // box = (128 bytes of K) x box_rows.
 moe_status make_tmap(CUtensorMap* m, const void* base, size_t esz, uint64_t inner, uint64_t rows,
@@ -248,15 +269,17 @@ route::Params route_params(const moe_layer_desc& s) {
 }
 
 template <int VPL>
-void launch_topk(const float* logits, const float* bias, const route::Params& p, int32_t* idx,
-                 float* w, int32_t* counts, cudaStream_t st) {
-  route::k_topk<VPL><<<(p.T + 7) / 8, 256, 0, st>>>(logits, bias, p, idx, w, counts);
+moe_status launch_topk(const float* logits, const float* bias, const route::Params& p,
+                       int32_t* idx, float* w, int32_t* counts, cudaStream_t st) {
+  return launch_chain("k_topk", route::k_topk<VPL>, dim3((p.T + 7) / 8), dim3(256), 0, st,
+                      logits, bias, p, idx, w, counts);
 }
 template <int VPL>
-void launch_route_f32(const float* x, const float* wr, int d, const float* bias,
-                      const route::Params& p, int32_t* idx, float* w, int32_t* counts,
-                      cudaStream_t st) {
-  route::k_route_f32<VPL><<<(p.T + 7) / 8, 256, 0, st>>>(x, wr, d, bias, p, idx, w, counts);
+moe_status launch_route_f32(const float* x, const float* wr, int d, const float* bias,
+                            const route::Params& p, int32_t* idx, float* w, int32_t* counts,
+                            cudaStream_t st) {
+  return launch_chain("k_route_f32", route::k_route_f32<VPL>, dim3((p.T + 7) / 8), dim3(256), 0,
+                      st, x, wr, d, bias, p, idx, w, counts);
 }
 
 // ----------------------------------------------------------------------------- stages
@@ -291,10 +314,9 @@ moe_status launch_router(const Dims& D, const void* x, const void* w_router, flo
     if (gemm8::smem_bytes(s, 1) <= (size_t)kMaxSmem) stages = s;
   a.stages = stages;
   const int tiles = (int)((D.T + 127) / 128) * a.n_tiles_n;
-  gemm8::k_gemm_promoted<0, gemm8::EPI_F32_STORE>
-      <<<tiles < sms ? tiles : sms, gemm8::NUM_THREADS, gemm8::smem_bytes(stages, 1), st>>>(ta, tb,
-                                                                                          a);
-  return launched("router GEMM");
+  return launch_chain("router GEMM", gemm8::k_gemm_promoted<0, gemm8::EPI_F32_STORE>,
+                      dim3(tiles < sms ? tiles : sms), dim3(gemm8::NUM_THREADS),
+                      gemm8::smem_bytes(stages, 1), st, ta, tb, a);
 }
 
 moe_status do_route(const moe_layer_desc& s, const Dims& D, const Layout& L, const void* x,
@@ -302,31 +324,29 @@ moe_status do_route(const moe_layer_desc& s, const Dims& D, const Layout& L, con
                     int32_t* counts, uint8_t* ws, int sms, cudaStream_t st) {
   const route::Params p = route_params(s);
   const int N = (int)D.N;
-  if (D.T == 0) {
-    route::k_zero_i32<<<1, 256, 0, st>>>(counts, N);
-    return launched("k_zero_i32");
-  }
+  if (D.T == 0)
+    return launch_chain("k_zero_i32", route::k_zero_i32, dim3(1), dim3(256), 0, st, counts, N);
   if (D.f32) {
-    route::k_zero_i32<<<1, 256, 0, st>>>(counts, N);
+    moe_status rc =
+        launch_chain("k_zero_i32", route::k_zero_i32, dim3(1), dim3(256), 0, st, counts, N);
+    if (rc != MOE_OK) return rc;
     const float* xf = static_cast<const float*>(x);
     const float* wf = static_cast<const float*>(w_router);
     const int dd = (int)D.d;
-    if (N <= 32) launch_route_f32<1>(xf, wf, dd, bias, p, topk_idx, topk_w, counts, st);
-    else if (N <= 64) launch_route_f32<2>(xf, wf, dd, bias, p, topk_idx, topk_w, counts, st);
-    else if (N <= 128) launch_route_f32<4>(xf, wf, dd, bias, p, topk_idx, topk_w, counts, st);
-    else if (N <= 256) launch_route_f32<8>(xf, wf, dd, bias, p, topk_idx, topk_w, counts, st);
-    else launch_route_f32<16>(xf, wf, dd, bias, p, topk_idx, topk_w, counts, st);
-    return launched("k_route_f32");
+    if (N <= 32) return launch_route_f32<1>(xf, wf, dd, bias, p, topk_idx, topk_w, counts, st);
+    if (N <= 64) return launch_route_f32<2>(xf, wf, dd, bias, p, topk_idx, topk_w, counts, st);
+    if (N <= 128) return launch_route_f32<4>(xf, wf, dd, bias, p, topk_idx, topk_w, counts, st);
+    if (N <= 256) return launch_route_f32<8>(xf, wf, dd, bias, p, topk_idx, topk_w, counts, st);
+    return launch_route_f32<16>(xf, wf, dd, bias, p, topk_idx, topk_w, counts, st);
   }
   float* logits = reinterpret_cast<float*>(ws + L.logits);
   moe_status rc = launch_router(D, x, w_router, logits, counts, sms, st);
   if (rc != MOE_OK) return rc;
-  if (N <= 32) launch_topk<1>(logits, bias, p, topk_idx, topk_w, counts, st);
-  else if (N <= 64) launch_topk<2>(logits, bias, p, topk_idx, topk_w, counts, st);
-  else if (N <= 128) launch_topk<4>(logits, bias, p, topk_idx, topk_w, counts, st);
-  else if (N <= 256) launch_topk<8>(logits, bias, p, topk_idx, topk_w, counts, st);
-  else launch_topk<16>(logits, bias, p, topk_idx, topk_w, counts, st);
-  return launched("k_topk");
+  if (N <= 32) return launch_topk<1>(logits, bias, p, topk_idx, topk_w, counts, st);
+  if (N <= 64) return launch_topk<2>(logits, bias, p, topk_idx, topk_w, counts, st);
+  if (N <= 128) return launch_topk<4>(logits, bias, p, topk_idx, topk_w, counts, st);
+  if (N <= 256) return launch_topk<8>(logits, bias, p, topk_idx, topk_w, counts, st);
+  return launch_topk<16>(logits, bias, p, topk_idx, topk_w, counts, st);
 }
 
 moe_status do_permute(const Dims& D, const Layout& L, const void* x, const int32_t* topk_idx,
@@ -335,23 +355,27 @@ moe_status do_permute(const Dims& D, const Layout& L, const void* x, const int32
                       cudaStream_t st) {
   const int T = (int)D.T, K = (int)D.K, N = (int)D.N;
   int32_t* hist = reinterpret_cast<int32_t*>(ws + L.hist);
-  if (T == 0) {
-    route::k_zero_i32<<<1, 256, 0, st>>>(offsets, N + 1);
-    return launched("k_zero_i32");
-  }
-  perm::k_hist<<<D.n_chunks, 256, N * 4, st>>>(topk_idx, T, K, N, hist);
-  perm::k_scan<<<1, 1024, 0, st>>>(hist, D.n_chunks, N, counts, offsets);
-  perm::k_slots<<<D.n_chunks, perm::SLOT_WARPS * 32, perm::SLOT_WARPS * N * 4, st>>>(topk_idx, T, K, N, hist, slot_of, perm_src);
-  if (D.fp8) {
-    perm::k_gather_quant<<<(T + 7) / 8, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(x), T, K,
-                                                      (int)D.d, (int)D.R, slot_of,
-                                                      static_cast<uint8_t*>(x_perm), x_perm_scale);
-  } else {
-    perm::k_gather<<<(T + 7) / 8, 256, 0, st>>>(static_cast<const uint8_t*>(x), T, K,
-                                                (int)(D.d * D.x_esz), slot_of,
-                                                static_cast<uint8_t*>(x_perm));
-  }
-  return launched("permutation kernels");
+  if (T == 0)
+    return launch_chain("k_zero_i32", route::k_zero_i32, dim3(1), dim3(256), 0, st, offsets,
+                        N + 1);
+  moe_status rc = launch_chain("k_hist", perm::k_hist, dim3(D.n_chunks), dim3(256), N * 4, st,
+                               topk_idx, T, K, N, hist);
+  if (rc == MOE_OK)
+    rc = launch_chain("k_scan", perm::k_scan, dim3(1), dim3(1024), 0, st, hist, (int)D.n_chunks,
+                      N, counts, offsets);
+  if (rc == MOE_OK)
+    rc = launch_chain("k_slots", perm::k_slots, dim3(D.n_chunks), dim3(perm::SLOT_WARPS * 32),
+                      perm::SLOT_WARPS * N * 4, st, topk_idx, T, K, N,
+                      static_cast<const int32_t*>(hist), slot_of, perm_src);
+  if (rc != MOE_OK) return rc;
+  if (D.fp8)
+    return launch_chain("k_gather_quant", perm::k_gather_quant, dim3((T + 7) / 8), dim3(256), 0,
+                        st, static_cast<const __nv_bfloat16*>(x), T, K, (int)D.d, (int)D.R,
+                        static_cast<const int32_t*>(slot_of), static_cast<uint8_t*>(x_perm),
+                        x_perm_scale);
+  return launch_chain("k_gather", perm::k_gather, dim3((T + 7) / 8), dim3(256), 0, st,
+                      static_cast<const uint8_t*>(x), T, K, (int)(D.d * D.x_esz),
+                      static_cast<const int32_t*>(slot_of), static_cast<uint8_t*>(x_perm));
 }
 
 // FP8 experts: E4M3 x_perm / H with fp32 1x128 scales, E4M3 weights with fp32
@@ -397,9 +421,9 @@ moe_status do_grouped_fp8(const Dims& D, const Layout& L, const void* x_perm,
     a.inter = (int)D.I;
     const int64_t tiles = mt_bound * a.n_tiles_n;
     const int grid = (int)(tiles < sms ? tiles : sms);
-    gemm8::k_gemm_promoted<2, gemm8::EPI_SWIGLU_Q><<<grid, gemm8::NUM_THREADS, smem, st>>>(ta, tb,
-                                                                                          a);
-    if ((rc = launched("FP8 grouped GEMM 1")) != MOE_OK) return rc;
+    rc = launch_chain("FP8 grouped GEMM 1", gemm8::k_gemm_promoted<2, gemm8::EPI_SWIGLU_Q>,
+                      dim3(grid), dim3(gemm8::NUM_THREADS), smem, st, ta, tb, a);
+    if (rc != MOE_OK) return rc;
     if ((rc = trace(3, st)) != MOE_OK) return rc;
   }
   {
@@ -429,9 +453,9 @@ moe_status do_grouped_fp8(const Dims& D, const Layout& L, const void* x_perm,
     a.Ks = (int)D.Ks;
     const int64_t tiles = mt_bound * a.n_tiles_n;
     const int grid = (int)(tiles < sms ? tiles : sms);
-    gemm8::k_gemm_promoted<2, gemm8::EPI_SCATTER><<<grid, gemm8::NUM_THREADS, smem, st>>>(ta, tb,
-                                                                                         a);
-    if ((rc = launched("FP8 grouped GEMM 2")) != MOE_OK) return rc;
+    rc = launch_chain("FP8 grouped GEMM 2", gemm8::k_gemm_promoted<2, gemm8::EPI_SCATTER>,
+                      dim3(grid), dim3(gemm8::NUM_THREADS), smem, st, ta, tb, a);
+    if (rc != MOE_OK) return rc;
     rc = trace(4, st);
   }
   return rc;
@@ -446,15 +470,17 @@ template <typename F>
 moe_status pair_config(int slot, F* func, int threads, size_t smem, int64_t tiles,
                        cudaStream_t st, cudaLaunchConfig_t* cfg, cudaLaunchAttribute* attr) {
   memset(cfg, 0, sizeof(*cfg));
-  attr->id = cudaLaunchAttributeClusterDimension;
-  attr->val.clusterDim.x = 2;
-  attr->val.clusterDim.y = 1;
-  attr->val.clusterDim.z = 1;
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg->blockDim = dim3(threads, 1, 1);
   cfg->dynamicSmemBytes = smem;
   cfg->stream = st;
   cfg->attrs = attr;
-  cfg->numAttrs = 1;
+  cfg->numAttrs = 1;   // the occupancy query takes the cluster shape only
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
@@ -475,6 +501,7 @@ moe_status pair_config(int slot, F* func, int threads, size_t smem, int64_t tile
   if (tiles < clusters) clusters = (int)tiles;
   if (clusters < 1) clusters = 1;
   cfg->gridDim = dim3(2 * clusters, 1, 1);
+  cfg->numAttrs = 2;
   return MOE_OK;
 }
 
@@ -493,7 +520,7 @@ moe_status launch_down(int kind, const void* w_down, const void* hbuf, size_t es
   a.stages = stages;
   const size_t smem = gemmt::smem_bytes(stages, a.gt.n);
   cudaLaunchConfig_t cfg;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   rc = kind == 0 ? pair_config(1, gemmt::k_down_gemm<0>, gemmt::NUM_THREADS, smem,
                                tok_tiles * a.n_wt, st, &cfg, attr)
                  : pair_config(1, gemmt::k_down_gemm<1>, gemmt::NUM_THREADS, smem,
@@ -524,7 +551,7 @@ moe_status launch_gate_up(int kind, const void* w_gu, const void* x, const void*
   a.stages = stages;
   const size_t smem = gemmgu::smem_bytes(stages, a.gt.n);
   cudaLaunchConfig_t cfg;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   rc = kind == 0 ? pair_config(0, gemmgu::k_gate_up_gemm<0>, gemmgu::NUM_THREADS, smem,
                                tok_tiles * a.n_ft, st, &cfg, attr)
                  : pair_config(0, gemmgu::k_gate_up_gemm<1>, gemmgu::NUM_THREADS, smem,
@@ -550,10 +577,9 @@ moe_status do_grouped(const Dims& D, const Layout& L, const void* x, const void*
   const int prep_blocks = 1 + (int)((D.R + 1023) / 1024 < 4 * sms ? (D.R + 1023) / 1024 : 4 * sms);
   moe_status rc = trace(2, st);
   if (rc != MOE_OK) return rc;
-  perm::k_prep_groups<<<prep_blocks, 1024, 0, st>>>(offsets, (int)D.T, (int)D.K, (int)D.Ks,
-                                                    (int)D.N, D.fp8 ? 1 : 0, gtab, slot_of,
-                                                    pair_of);
-  rc = launched("k_prep_groups");
+  rc = launch_chain("k_prep_groups", perm::k_prep_groups, dim3(prep_blocks), dim3(1024), 0, st,
+                    offsets, (int)D.T, (int)D.K, (int)D.Ks, (int)D.N, D.fp8 ? 1 : 0, gtab,
+                    slot_of, pair_of);
   if (rc != MOE_OK) return rc;
   if (D.fp8)
     return do_grouped_fp8(D, L, x_perm, x_perm_scale, gtab, pair_of, topk_w, w_gu, w_gu_scale,
@@ -620,12 +646,10 @@ moe_status do_combine(const Dims& D, const void* x_res, const void* y, void* h, 
   const int64_t threads = D.T * (D.d / vec);
   const int blocks = (int)((threads + 255) / 256);
   if (D.f32)
-    perm::k_combine<false><<<blocks, 256, 0, st>>>(x_res, y, h, (int)D.T, (int)D.d, (int)D.K,
-                                                   (int)D.Ks);
-  else
-    perm::k_combine<true><<<blocks, 256, 0, st>>>(x_res, y, h, (int)D.T, (int)D.d, (int)D.K,
-                                                  (int)D.Ks);
-  return launched("k_combine<true>");
+    return launch_chain("k_combine", perm::k_combine<false>, dim3(blocks), dim3(256), 0, st, x_res,
+                        y, h, (int)D.T, (int)D.d, (int)D.K, (int)D.Ks);
+  return launch_chain("k_combine", perm::k_combine<true>, dim3(blocks), dim3(256), 0, st, x_res,
+                      y, h, (int)D.T, (int)D.d, (int)D.K, (int)D.Ks);
 }
 
 __global__ void k_selftest_wait(uint64_t limit_ns) {

@@ -17,6 +17,17 @@ namespace moe {
 // One per device (a __device__ variable exists once per device context).
 // Kernels record the first problem they see; the host reads and clears it.
 __device__ int g_status = 0;
+// Programmatic dependent launch: the kernels of the layer's chain are launched
+// with programmatic stream serialisation, so a kernel's launch and prologue
+// may overlap the end of the one before it.  Each of them waits here, before
+// its first global memory access, until the previous grid has completed and
+// its writes are visible (a no-op when launched without the attribute), and
+// then lets the next kernel of the stream start launching.
+__device__ __forceinline__ void grid_dep_sync() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // Limit of every device-side wait, in nanoseconds of %globaltimer.
 __device__ unsigned long long g_wait_limit_ns = 1000000000ull;
 

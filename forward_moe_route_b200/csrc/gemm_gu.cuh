@@ -65,6 +65,7 @@ template <int KIND>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     k_gate_up_gemm(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                    const __grid_constant__ CUtensorMap tmXP, const Args a) {
+  grid_dep_sync();
   using namespace gemmt;   // cluster helpers of the pair down projection
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &

@@ -128,6 +128,7 @@ template <int KIND>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     k_down_gemm(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmH,
                      const Args a) {
+  grid_dep_sync();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));

@@ -20,6 +20,7 @@ constexpr int CHUNK = 128;  // tokens per histogram chunk
 // hist[c * N + e] = number of pairs of chunk c routed to expert e.
 __global__ void __launch_bounds__(256) k_hist(const int32_t* __restrict__ idx, int T, int K, int N,
                                               int32_t* __restrict__ hist) {
+  grid_dep_sync();
   extern __shared__ int32_t sh[];
   for (int e = threadIdx.x; e < N; e += blockDim.x) sh[e] = 0;
   __syncthreads();
@@ -40,6 +41,7 @@ __global__ void __launch_bounds__(256) k_hist(const int32_t* __restrict__ idx, i
 __global__ void __launch_bounds__(1024) k_scan(int32_t* __restrict__ hist, int n_chunks, int N,
                                                const int32_t* __restrict__ counts,
                                                int32_t* __restrict__ offsets) {
+  grid_dep_sync();
   __shared__ int32_t part_sum[1024];
   __shared__ int32_t tot[1024];
   __shared__ int32_t warp_tot[32];
@@ -122,6 +124,7 @@ __global__ void __launch_bounds__(SLOT_WARPS * 32) k_slots(const int32_t* __rest
                                                            const int32_t* __restrict__ base,
                                                            int32_t* __restrict__ slot_of,
                                                            int32_t* __restrict__ perm_src) {
+  grid_dep_sync();
   extern __shared__ int32_t sub[];            // [SLOT_WARPS][N] counts, then first rows
   const int lane = lane_id(), w = warp_id();
   for (int i = threadIdx.x; i < SLOT_WARPS * N; i += blockDim.x) sub[i] = 0;
@@ -166,6 +169,7 @@ __global__ void __launch_bounds__(SLOT_WARPS * 32) k_slots(const int32_t* __rest
 __global__ void __launch_bounds__(256) k_gather(const uint8_t* __restrict__ x, int T, int K,
                                                 int row_bytes, const int32_t* __restrict__ slot_of,
                                                 uint8_t* __restrict__ x_perm) {
+  grid_dep_sync();
   const int R = T * K;
   const int t = blockIdx.x * 8 + warp_id();
   if (t >= T) return;
@@ -202,6 +206,7 @@ __global__ void __launch_bounds__(256) k_gather_quant(const __nv_bfloat16* __res
                                                       const int32_t* __restrict__ slot_of,
                                                       uint8_t* __restrict__ xq,
                                                       float* __restrict__ xs) {
+  grid_dep_sync();
   const int t = blockIdx.x * 8 + warp_id();
   if (t >= T) return;
   const int lane = lane_id();
@@ -237,6 +242,7 @@ __global__ void __launch_bounds__(1024) k_prep_groups(const int32_t* __restrict_
                                                       int32_t* __restrict__ gtab,
                                                       const int32_t* __restrict__ slot_of,
                                                       int32_t* __restrict__ pair_of) {
+  grid_dep_sync();
   const int R = T * K;
   if (blockIdx.x > 0) {
     for (int i = (blockIdx.x - 1) * blockDim.x + threadIdx.x; i < R;
@@ -316,6 +322,7 @@ template <bool BF16>
 __global__ void __launch_bounds__(256) k_combine(const void* __restrict__ x_res,
                                                  const void* __restrict__ y, void* __restrict__ h,
                                                  int T, int d, int K, int Ks) {
+  grid_dep_sync();
   constexpr int VEC = BF16 ? 8 : 4;
   const int per_tok = d / VEC;
   const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;

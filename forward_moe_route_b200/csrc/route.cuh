@@ -187,6 +187,7 @@ __global__ void __launch_bounds__(256) k_topk(const float* __restrict__ logits,
                                               int32_t* __restrict__ topk_idx,
                                               float* __restrict__ topk_w,
                                               int32_t* __restrict__ counts) {
+  grid_dep_sync();
   const int t = blockIdx.x * 8 + warp_id();
   if (t >= p.T) return;
   const float* row = logits + (size_t)t * p.N;
@@ -215,6 +216,7 @@ __global__ void __launch_bounds__(256) k_route_f32(const float* __restrict__ x,
                                                    int32_t* __restrict__ topk_idx,
                                                    float* __restrict__ topk_w,
                                                    int32_t* __restrict__ counts) {
+  grid_dep_sync();
   const int t = blockIdx.x * 8 + warp_id();
   if (t >= p.T) return;
   const int lane = lane_id();
@@ -334,6 +336,7 @@ __global__ void k_bias_update(const int32_t* __restrict__ counts, float* __restr
 }
 
 __global__ void k_zero_i32(int32_t* p, int n) {
+  grid_dep_sync();
   for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) p[i] = 0;
 }
 

@@ -2,9 +2,12 @@
 
 Argument marshalling only: every function here forwards torch tensors' device
 pointers and the current CUDA stream to the C ABI of the same name
-(include/moe.h) and turns a non-OK status into MoeError.  All computation runs
-in the library's CUDA kernels; there is no fallback.  Importing this package
-fails loudly if the compiled library is missing.
+(include/moe.h) and turns a non-OK status into MoeError.  Because the ABI
+takes plain pointers, the binding first checks that each tensor argument is
+contiguous and holds at least the bytes the descriptor implies, and refuses a
+short or strided buffer instead of letting a kernel overrun it.  All
+computation runs in the library's CUDA kernels; there is no fallback.
+Importing this package fails loudly if the compiled library is missing.
 """
 from __future__ import annotations
 
@@ -104,6 +107,42 @@ def _check(rc: int, where: str) -> None:
         raise MoeError(rc, where)
 
 
+def _sizes(desc) -> dict:
+    """Bytes each buffer of the ABI needs for this descriptor."""
+    T, d, Ks, N = desc.T, desc.d, desc.n_shared, desc.n_routed
+    K, I = desc.top_k, desc.inter
+    E, R = Ks + N, desc.T * desc.top_k
+    a = 4 if desc.act_dtype == DT_F32 else 2
+    w = {DT_F32: 4, DT_BF16: 2, DT_E4M3: 1}[desc.w_dtype]
+    fp8 = desc.w_dtype == DT_E4M3
+    xp_rows = R + (T if fp8 else 0)
+    return {
+        "x": T * d * a, "h": T * d * a, "x_residual": T * d * a, "w_router": N * d * a,
+        "bias": N * 4, "topk_idx": R * 4, "topk_w": R * 4, "counts": N * 4,
+        "offsets": (N + 1) * 4, "perm_src": R * 4, "slot_of": R * 4,
+        "x_perm": xp_rows * d * (1 if fp8 else a),
+        "x_perm_scale": xp_rows * (d // 128) * 4 if fp8 else 0,
+        "w_gu": E * 2 * I * d * w, "w_down": E * d * I * w,
+        "w_gu_scale": E * (2 * I // 128) * (d // 128) * 4 if fp8 else 0,
+        "w_down_scale": E * (d // 128) * (I // 128) * 4 if fp8 else 0,
+        "y_slots": T * (K + Ks) * d * a, "s_out": T * N * 4,
+    }
+
+
+def _need(where: str, desc, **tensors) -> None:
+    """Refuse a tensor argument that is strided or smaller than the descriptor needs."""
+    sizes = _sizes(desc)
+    for name, t in tensors.items():
+        if t is None or isinstance(t, int) or not hasattr(t, "element_size"):
+            continue
+        if not t.is_contiguous():
+            raise MoeError(ERR_INVALID_ARG, f"{where}: {name} is not contiguous")
+        have = t.numel() * t.element_size()
+        if have < sizes[name]:
+            raise MoeError(ERR_INVALID_ARG,
+                           f"{where}: {name} holds {have} bytes, the layer needs {sizes[name]}")
+
+
 def moe_status_string(status: int) -> str:
     return _lib.moe_status_string(status).decode()
 
@@ -138,6 +177,8 @@ def workspace(desc: MoeLayerDesc, device="cuda"):
 
 
 def moe_route(desc, x, w_router, bias, topk_idx, topk_w, counts, ws, stream=None) -> None:
+    _need("moe_route", desc, x=x, w_router=w_router, bias=bias, topk_idx=topk_idx,
+          topk_w=topk_w, counts=counts)
     _check(_lib.moe_route(ctypes.byref(desc), _ptr(x), _ptr(w_router), _ptr(bias), _ptr(topk_idx),
                           _ptr(topk_w), _ptr(counts), _ptr(ws), ws.numel() if ws is not None
                           else 0, _stream(stream)), "moe_route")
@@ -145,6 +186,8 @@ def moe_route(desc, x, w_router, bias, topk_idx, topk_w, counts, ws, stream=None
 
 def moe_permute(desc, x, topk_idx, counts, offsets, perm_src, slot_of, x_perm, x_perm_scale, ws,
                 stream=None) -> None:
+    _need("moe_permute", desc, x=x, topk_idx=topk_idx, counts=counts, offsets=offsets,
+          perm_src=perm_src, slot_of=slot_of, x_perm=x_perm, x_perm_scale=x_perm_scale)
     _check(_lib.moe_permute(ctypes.byref(desc), _ptr(x), _ptr(topk_idx), _ptr(counts),
                             _ptr(offsets), _ptr(perm_src), _ptr(slot_of), _ptr(x_perm),
                             _ptr(x_perm_scale), _ptr(ws), ws.numel() if ws is not None else 0,
@@ -154,6 +197,9 @@ def moe_permute(desc, x, topk_idx, counts, offsets, perm_src, slot_of, x_perm, x
 def moe_permute_noalloc(desc, x, topk_idx, counts, offsets, perm_src, slot_of, x_perm,
                         x_perm_scale, stream=None) -> None:
     """moe_permute without a workspace (fixed 1 MiB device scratch; see include/moe.h)."""
+    _need("moe_permute_noalloc", desc, x=x, topk_idx=topk_idx, counts=counts,
+          offsets=offsets, perm_src=perm_src, slot_of=slot_of, x_perm=x_perm,
+          x_perm_scale=x_perm_scale)
     _check(_lib.moe_permute_noalloc(ctypes.byref(desc), _ptr(x), _ptr(topk_idx), _ptr(counts),
                                     _ptr(offsets), _ptr(perm_src), _ptr(slot_of), _ptr(x_perm),
                                     _ptr(x_perm_scale), _stream(stream)), "moe_permute_noalloc")
@@ -161,6 +207,9 @@ def moe_permute_noalloc(desc, x, topk_idx, counts, offsets, perm_src, slot_of, x
 
 def moe_grouped_swiglu(desc, x, x_perm, x_perm_scale, offsets, perm_src, slot_of, topk_w, w_gu,
                        w_gu_scale, w_down, w_down_scale, y_slots, ws, stream=None) -> None:
+    _need("moe_grouped_swiglu", desc, x=x, x_perm=x_perm, x_perm_scale=x_perm_scale,
+          offsets=offsets, perm_src=perm_src, slot_of=slot_of, topk_w=topk_w, w_gu=w_gu,
+          w_gu_scale=w_gu_scale, w_down=w_down, w_down_scale=w_down_scale, y_slots=y_slots)
     _check(_lib.moe_grouped_swiglu(ctypes.byref(desc), _ptr(x), _ptr(x_perm), _ptr(x_perm_scale),
                                    _ptr(offsets), _ptr(perm_src), _ptr(slot_of), _ptr(topk_w),
                                    _ptr(w_gu), _ptr(w_gu_scale), _ptr(w_down),
@@ -170,12 +219,16 @@ def moe_grouped_swiglu(desc, x, x_perm, x_perm_scale, offsets, perm_src, slot_of
 
 
 def moe_combine(desc, x_residual, y_slots, h, stream=None) -> None:
+    _need("moe_combine", desc, x_residual=x_residual, y_slots=y_slots, h=h)
     _check(_lib.moe_combine(ctypes.byref(desc), _ptr(x_residual), _ptr(y_slots), _ptr(h),
                             _stream(stream)), "moe_combine")
 
 
 def moe_forward(desc, x, x_residual, w_router, bias, w_gu, w_gu_scale, w_down, w_down_scale, h,
                 topk_idx, counts, ws, stream=None) -> None:
+    _need("moe_forward", desc, x=x, x_residual=x_residual, w_router=w_router, bias=bias,
+          w_gu=w_gu, w_gu_scale=w_gu_scale, w_down=w_down, w_down_scale=w_down_scale, h=h,
+          topk_idx=topk_idx, counts=counts)
     _check(_lib.moe_forward(ctypes.byref(desc), _ptr(x), _ptr(x_residual), _ptr(w_router),
                             _ptr(bias), _ptr(w_gu), _ptr(w_gu_scale), _ptr(w_down),
                             _ptr(w_down_scale), _ptr(h), _ptr(topk_idx), _ptr(counts), _ptr(ws),
@@ -183,6 +236,7 @@ def moe_forward(desc, x, x_residual, w_router, bias, w_gu, w_gu_scale, w_down, w
 
 
 def moe_route_affinities(desc, x, w_router, s_out, ws, stream=None) -> None:
+    _need("moe_route_affinities", desc, x=x, w_router=w_router, s_out=s_out)
     _check(_lib.moe_route_affinities(ctypes.byref(desc), _ptr(x), _ptr(w_router), _ptr(s_out),
                                      _ptr(ws), ws.numel() if ws is not None else 0,
                                      _stream(stream)), "moe_route_affinities")

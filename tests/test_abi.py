@@ -127,3 +127,36 @@ def test_status_strings():
 def test_launch_count():
     assert moe.moe_forward_launch_count(v3()) == 10
     assert moe.moe_forward_launch_count(v3(top_k=300)) == 0
+
+
+def test_binding_refuses_short_or_strided_buffers():
+    # the ABI takes plain pointers, so the binding checks every tensor against
+    # the descriptor before calling in; CPU tensors suffice for the check
+    import torch
+
+    desc = moe.make_desc(T=64, d=256, n_shared=1, n_routed=16, top_k=4, inter=64,
+                         gate="softmax", renorm=True, route_scale=1.0, dtype="bf16")
+    E = 17
+    x = torch.zeros(64, 256, dtype=torch.bfloat16)
+    w_r = torch.zeros(16, 256, dtype=torch.bfloat16)
+    w_gu = torch.zeros(E, 128, 256, dtype=torch.bfloat16)
+    w_d = torch.zeros(E, 256, 64, dtype=torch.bfloat16)
+    short_h = torch.zeros(63, 256, dtype=torch.bfloat16)
+    with pytest.raises(moe.MoeError, match="h holds"):
+        moe.moe_forward(desc, x, None, w_r, None, w_gu, None, w_d, None, short_h, None, None,
+                        None)
+    strided = torch.zeros(256, 64, dtype=torch.bfloat16).t()
+    with pytest.raises(moe.MoeError, match="not contiguous"):
+        moe.moe_forward(desc, strided, None, w_r, None, w_gu, None, w_d, None, x, None, None,
+                        None)
+    short_w = torch.zeros(E - 1, 128, 256, dtype=torch.bfloat16)
+    x_perm = torch.zeros(64 * 4, 256, dtype=torch.bfloat16)
+    with pytest.raises(moe.MoeError, match="w_gu holds"):
+        moe.moe_grouped_swiglu(desc, x, x_perm, None, None, None, None, None, short_w, None, w_d,
+                               None, None, None)
+    fp8 = moe.make_desc(T=64, d=256, n_shared=1, n_routed=16, top_k=4, inter=128,
+                        gate="softmax", renorm=True, route_scale=1.0, dtype="e4m3")
+    xp = torch.zeros(64 * 4 + 64, 256, dtype=torch.uint8)
+    short_scale = torch.zeros(64 * 4, 2, dtype=torch.float32)      # the T shared rows missing
+    with pytest.raises(moe.MoeError, match="x_perm_scale holds"):
+        moe.moe_permute(fp8, x, None, None, None, None, None, xp, short_scale, None)

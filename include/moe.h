@@ -35,6 +35,11 @@
  *    are recorded in a per-device status word read by moe_last_device_status.
  *  - Results are bit-identical from run to run (no floating-point atomics).
  *  - Concurrent calls that share a workspace race; give each stream its own.
+ *  - The library cannot see buffer sizes: each buffer must hold at least the
+ *    elements its comment states, or a kernel overruns it.
+ *  - The kernels of one call are launched with programmatic stream
+ *    serialisation and each waits for its predecessor's results before it
+ *    touches memory, so stream order is kept as for plain launches.
  */
 #ifndef MOE_B200_H
 #define MOE_B200_H

@@ -138,6 +138,13 @@ def max_over_ranks(value: float, device) -> float:
 
 
 # ----------------------------------------------------------------------------- clocks
+def visible_gpu(local: int) -> str:
+    """nvidia-smi's id of this rank's GPU: entry `local` of CUDA_VISIBLE_DEVICES
+    (an index or a UUID, both of which nvidia-smi -i accepts), else `local`."""
+    vis = [v.strip() for v in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if v.strip()]
+    return vis[local] if local < len(vis) else str(local)
+
+
 class ClockSampler:
     """nvidia-smi samples of this GPU's clocks while the timed region runs."""
 
@@ -145,8 +152,8 @@ class ClockSampler:
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
+    def __init__(self, gpu: str):
+        self.gpu = gpu
         self.proc = None
         self.lines = []
 
@@ -351,9 +358,7 @@ def run_ours(args, cfg):
     for row in ev:            # torch creates its events lazily, at the first record
         for e in row:
             e.record(stream)
-    clocks = ClockSampler(int(os.environ.get("CUDA_VISIBLE_DEVICES", str(local)).split(",")[0])
-                          if os.environ.get("CUDA_VISIBLE_DEVICES", "").replace(",", "").isdigit()
-                          else local)
+    clocks = ClockSampler(visible_gpu(local))
     barrier()
     torch.cuda.synchronize()
     clocks.start()

@@ -50,3 +50,14 @@ def test_measured_arm_fails_loudly_without_a_gpu():
     r = run_bench("--config", "tiny_f32", "--steps", "1", "--warmup", "3", "--no-cpu-baseline")
     assert r.returncode != 0
     assert not [l for l in r.stdout.splitlines() if l.strip().startswith("{")]
+
+
+def test_clock_sampler_follows_the_ranks_visible_gpu(monkeypatch):
+    sys.path.insert(0, ROOT)
+    import bench
+
+    monkeypatch.setenv("CUDA_VISIBLE_DEVICES", "3,5,GPU-0f1e2d")
+    assert [bench.visible_gpu(r) for r in range(3)] == ["3", "5", "GPU-0f1e2d"]
+    assert bench.visible_gpu(4) == "4"
+    monkeypatch.delenv("CUDA_VISIBLE_DEVICES")
+    assert bench.visible_gpu(2) == "2"

@@ -5,6 +5,7 @@ or a value the pages print, chosen so that a plausible mistake (a dropped
 term, a swapped operand, a wrong tie rule, a bias leaking into the weights)
 fails at least one of them.
 """
+import dataclasses
 import itertools
 import math
 import os
@@ -439,3 +440,23 @@ def test_max_abs_rel():
     ref = np.array([[1.0, -4.0], [2.0, 0.5]])
     got = ref + np.array([[0.0, 0.1], [-0.2, 0.0]])
     assert mo.max_abs_rel(got, ref) == pytest.approx(0.05)
+
+
+def test_three_matrix_experts_reproduce_the_v2_parameter_total():
+    # Reading C-9, pinned to printed totals: the oracle's SwiGLU expert holds
+    # W_gate, W_up [I, d] and W_down [d, I].  DeepSeek-V2 ("DeepSeek Technical
+    # Report: MoE Architecture", §2.1 and §2.3): 60 layers, hidden 5,120, MoE in
+    # every layer but the first, 2 shared + 160 routed experts of width 1,536,
+    # 236B parameters in all.  Three matrices put 95.5 % of the total in the
+    # experts (attention and embeddings take the rest); two would leave 36 %.
+    from synth import recipes
+
+    small = dataclasses.replace(recipes.CONFIGS["tiny_f32"], d=96, inter=32)
+    per_expert = sum(w.size for w in recipes.host_expert(small, 0))
+    assert per_expert == 3 * small.d * small.inter
+    d, I, layers, experts = 5120, 1536, 60 - 1, 2 + 160
+    total = 236e9
+    moe3 = layers * experts * (per_expert // (small.d * small.inter)) * d * I
+    moe2 = layers * experts * 2 * d * I
+    assert 0.9 * total <= moe3 <= total
+    assert moe2 < 0.7 * total

@@ -128,3 +128,96 @@ def test_fp8_ffn_exact_on_representable_inputs():
     exact = mo.swiglu_ffn(v, wg, wu, wd)
     got = fp8.fp8_swiglu_ffn(v, wg, wu, wd)
     assert mo.max_abs_rel(got, exact) < 2.0 ** -4
+
+
+# ----------------------------------------------------------------------------- H requantisation
+# The FP8 FFN requantises its intermediate H = SiLU(v W_gate^T) * (v W_up^T)
+# per 1x128 tile along I before the down projection ("DeepSeek Technical
+# Report: MoE Architecture", §3.6: activations are grouped per 1x128 tile and
+# every linear forward GEMM takes E4M3 inputs).  This construction makes H
+# known in closed form: v[:, 0] = 1 and every W_gate row is 64 e_0, so each
+# gate pre-activation is 64 and SiLU(64) = 64 / (1 + e^-64) = 64 exactly in
+# float64 (e^-64 < 2^-53); W_up row i is e_{1+i}, so H[t, i] = 64 * v[t, 1+i];
+# W_down is the identity, so the FFN returns the dequantised H itself.  The
+# expected codes below are worked out by hand from the E4M3 format (3 fraction
+# bits, subnormal spacing 2^-9, ties to even) and the tile rule
+# scale = amax / 448.
+I_H = 256
+
+
+def _h_design():
+    H = np.zeros((2, I_H))
+    want = np.zeros((2, I_H))
+    # row 0, tile 0 (columns 0..127): amax 448 at column 100 -> scale 1, codes = values
+    H[0, 100], want[0, 100] = 448.0, 448.0
+    H[0, 1], want[0, 1] = 1.0, 1.0                   # representable
+    H[0, 2], want[0, 2] = 1.0625, 1.0                # midpoint of 1 and 1.125: even mantissa -> 1
+    H[0, 3], want[0, 3] = 2.0 ** -10, 0.0            # midpoint of 0 and 2^-9 -> 0
+    H[0, 4], want[0, 4] = 3 * 2.0 ** -10, 2.0 ** -8  # midpoint of 1 and 2 x 2^-9 -> 2 x 2^-9
+    H[0, 5], want[0, 5] = 300.0, 288.0               # spacing 32 in [256, 512): nearest is 288
+    H[0, 7], want[0, 7] = 5 * 2.0 ** -11, 2.0 ** -9  # 1.25 x 2^-9 -> 1 x 2^-9
+    # row 0, tile 1 (columns 128..255): amax 28 -> scale 2^-4 (28 * 16 = 448)
+    H[0, 200], want[0, 200] = 28.0, 28.0
+    H[0, 129], want[0, 129] = 0.53125, 0.5           # 8.5 after scaling: tie between 8 and 9 -> 8
+    H[0, 130], want[0, 130] = 2.0 ** -14, 0.0        # 2^-10 after scaling: tie at zero -> 0
+    # row 1, tile 0: amax 1344 -> scale 3 (fp32 448/1344 is inexact but 1344 and 3 land exactly)
+    H[1, 100], want[1, 100] = 1344.0, 1344.0
+    H[1, 1], want[1, 1] = 3.0, 3.0
+    # row 1, tile 1 stays all zero: amax 0 -> scale 0, codes 0
+    return H, want
+
+
+def _h_layer(H):
+    d = 1 + I_H
+    v = np.zeros((2, d))
+    v[:, 0] = 1.0
+    v[:, 1:] = H / 64.0                              # exact: the chosen H are dyadic
+    wg = np.zeros((I_H, d))
+    wg[:, 0] = 64.0
+    wu = np.zeros((I_H, d))
+    wu[np.arange(I_H), 1 + np.arange(I_H)] = 1.0
+    return v, wg, wu, np.eye(I_H)
+
+
+def test_fp8_ffn_requantises_h_per_1x128_tile():
+    H, want = _h_design()
+    v, wg, wu, wd = _h_layer(H)
+    from oracle import moe_oracle as mo
+    # the construction really gives H: the unquantised FFN returns it exactly
+    np.testing.assert_array_equal(mo.swiglu_ffn(v, wg, wu, wd), H)
+    got = fp8.fp8_swiglu_ffn(v, wg, wu, wd)
+    np.testing.assert_array_equal(got, want)
+
+
+def _mutant_requant(kind):
+    """Wrong readings of the H requantisation, planted in the oracle on the CPU."""
+    def quant(h):
+        h = np.asarray(h, np.float32)
+        rows, cols = h.shape
+        if kind == "none":
+            return h.astype(np.float64), None
+        if kind == "1x64":
+            q, s = fp8._quantize_groups(h.reshape(rows, cols // 64, 64))
+            return (q * s.astype(np.float64)[..., None]).reshape(rows, cols), None
+        if kind == "128x128":   # one block over both rows and 128 columns
+            blk = h.reshape(rows, cols // 128, 128).transpose(1, 0, 2).reshape(cols // 128, -1)
+            q, s = fp8._quantize_groups(blk)
+            deq = (q * s.astype(np.float64)[..., None]).reshape(cols // 128, rows, 128)
+            return deq.transpose(1, 0, 2).reshape(rows, cols), None
+        if kind == "column":    # tiles along the token axis instead of along I
+            q, s = fp8._quantize_groups(h.T.copy())
+            return (q * s.astype(np.float64)[..., None]).T, None
+        raise ValueError(kind)
+    return quant
+
+
+def test_h_requantisation_pin_catches_wrong_readings(monkeypatch):
+    H, want = _h_design()
+    v, wg, wu, wd = _h_layer(H)
+    for kind in ("none", "1x64", "128x128", "column"):
+        mutant = _mutant_requant(kind)
+        monkeypatch.setattr(fp8, "quantize_act_1x128", mutant)
+        monkeypatch.setattr(fp8, "dequant_act", lambda deq, _s: deq)
+        got = fp8.fp8_swiglu_ffn(v, wg, wu, wd)
+        monkeypatch.undo()
+        assert not np.array_equal(got, want), f"the pin does not tell apart the {kind!r} reading"

@@ -258,9 +258,15 @@ def blas_threads():
 
 
 def oracle_sample_size(cfg):
-    # keep one step to a few seconds of host work
-    work = cfg.d * cfg.inter * (cfg.top_k + cfg.n_shared)
-    return max(1, min(64, int(2e9 // max(work * 40, 1))))
+    """Tokens per oracle step, sized so a step widens about 1.2e9 stored weight
+    elements to float64 (the oracle's dominant cost: every expert a sampled
+    token reaches is read whole) -- about 10 s on 16 host cores at the V3
+    shape (3 tokens), all 64 experts for the 16B shape (64 tokens)."""
+    per_expert = 3 * cfg.d * cfg.inter
+    experts = max(1, int(1.2e9 // per_expert))
+    if experts >= cfg.n_routed + cfg.n_shared:
+        return 64
+    return max(1, min(64, (experts - cfg.n_shared) // cfg.top_k))
 
 
 def run_reference(args, cfg):
@@ -498,6 +504,85 @@ def run_ours(args, cfg):
     return out
 
 
+# ----------------------------------------------------------------------------- backward leg
+def backward_flops(cfg):
+    """FLOPs of the backward's expert GEMMs per step, split into the algorithmic
+    part (dz, du, dW_down, dW_gu: 12 d I per active row) and the recomputation
+    of the pre-activations a, b (4 d I per active row), plus the router (4 T N d)."""
+    rows = cfg.T * (cfg.top_k + cfg.n_shared)
+    return {"algorithmic": 12.0 * cfg.d * cfg.inter * rows,
+            "recompute": 4.0 * cfg.d * cfg.inter * rows,
+            "router": 4.0 * cfg.T * cfg.n_routed * cfg.d}
+
+
+def run_backward(args, cfg):
+    """One layer backward per step (moe_backward: routing, permutation, the
+    recomputed pre-activations, dz with the SwiGLU backward, du, the gate and
+    affinity backward, dW_down, dW_gu, dW_r), inputs resident in HBM."""
+    import torch
+
+    import forward_moe_route_b200 as moe
+    import synth
+    from synth import recipes
+    torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+    if cfg.dtype != "bf16":
+        raise SystemExit("the backward is built for bf16 layers")
+    desc = moe.desc_from_config(cfg)
+    inp = recipes.device_inputs(cfg, "cuda", load_zipf(cfg))
+    dh32 = torch.empty(cfg.T, cfg.d, dtype=torch.float32, device="cuda")
+    synth.dev_fill_normal(dh32, 1.0, cfg.seed, 6)
+    dh = dh32.to(torch.bfloat16)
+    del dh32
+    E, I, d, N = cfg.n_experts, cfg.inter, cfg.d, cfg.n_routed
+    dx = torch.empty(cfg.T, d, dtype=torch.bfloat16, device="cuda")
+    dwr = torch.empty(N, d, dtype=torch.float32, device="cuda")
+    dwgu = torch.empty(E, 2 * I, d, dtype=torch.float32, device="cuda")
+    dwd = torch.empty(E, d, I, dtype=torch.float32, device="cuda")
+    ws = moe.backward_workspace(desc)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        moe.moe_backward(desc, inp["x"], inp["w_r"], inp["bias"], inp["w_gu"], inp["w_down"], dh,
+                         dx, dwr, dwgu, dwd, ws, stream)
+
+    for _ in range(args.warmup):
+        step()
+    st = moe.moe_last_device_status()
+    if st != moe.OK:
+        raise SystemExit(f"device status after warm-up: {moe.moe_status_string(st)}")
+    clocks = ClockSampler(visible_gpu(int(os.environ.get("LOCAL_RANK", "0"))))
+    torch.cuda.synchronize()
+    clocks.start()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    st = moe.moe_last_device_status()
+    if st != moe.OK:
+        raise SystemExit(f"device status after the timed region: {moe.moe_status_string(st)}")
+    ms = e0.elapsed_time(e1) / args.steps
+    fl = backward_flops(cfg)
+    pk = peaks()
+    done = fl["algorithmic"] + fl["recompute"] + fl["router"]
+    tflops = done / (ms * 1e-3) / 1e12
+    return {"metric": "MoE-layer backward tokens/s", "value": cfg.T / (ms * 1e-3),
+            "unit": "tokens/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": cfg.dtype, "data": "synthetic", "config": config_dict(cfg, 1),
+            "backward_gemm_tflops": tflops,
+            "backward_gemm_frac_of_peak": {
+                "measured_sustained": tflops / pk["bf16_tflops_sustained"],
+                "spec_dense": tflops / 2250.0},
+            "backward_flops": fl,
+            "algorithmic_tflops": (fl["algorithmic"] + fl["router"]) / (ms * 1e-3) / 1e12,
+            "gpu_launches": moe.moe_backward_launch_count(desc) * args.steps,
+            "clocks": clk}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -509,6 +594,8 @@ def main():
                     help="override the routed expert count (smaller profiling cases)")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--backward", action="store_true",
+                    help="time the layer backward (moe_backward) instead of the forward")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
@@ -522,6 +609,9 @@ def main():
                                   name=f"{cfg.name}@N{args.n_routed}")
     if args.impl == "reference":
         return run_reference(args, cfg)
+    if args.backward:
+        print(json.dumps(run_backward(args, cfg)), flush=True)
+        return 0
     out = run_ours(args, cfg)
     if out is not None:
         if not args.no_cpu_baseline and args.gpus == 1:

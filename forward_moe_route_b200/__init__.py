@@ -70,6 +70,16 @@ _SIGS = {
     "moe_last_error_message": (ctypes.c_char_p, []),
     "moe_trace_events": (ctypes.c_int, [ctypes.POINTER(ctypes.c_void_p), ctypes.c_int32]),
     "moe_selftest_bounded_wait": (ctypes.c_int, [ctypes.c_uint32, _P]),
+    "moe_backward_workspace_size": (ctypes.c_size_t, [_D]),
+    "moe_backward": (ctypes.c_int, [_D, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
+                                    ctypes.c_size_t, _P]),
+    "moe_backward_launch_count": (ctypes.c_int32, [_D]),
+    "moe_expert_ffn_workspace_size": (ctypes.c_size_t, [_D, ctypes.c_int32, ctypes.c_int32]),
+    "moe_expert_ffn": (ctypes.c_int, [_D, ctypes.c_int32, ctypes.c_int32, _P, ctypes.c_int32,
+                                      ctypes.c_int32, _P, _P, _P, _P, _P, _P, ctypes.c_size_t,
+                                      _P]),
+    "moe_combine_rows": (ctypes.c_int, [_D, _P, _P, _P, _P, ctypes.c_int32, _P, _P]),
+    "moe_dispatch_rows": (ctypes.c_int, [_D, _P, _P, _P, ctypes.c_int32, _P, _P, _P]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _f = getattr(_lib, _name)
@@ -126,6 +136,8 @@ def _sizes(desc) -> dict:
         "w_gu_scale": E * (2 * I // 128) * (d // 128) * 4 if fp8 else 0,
         "w_down_scale": E * (d // 128) * (I // 128) * 4 if fp8 else 0,
         "y_slots": T * (K + Ks) * d * a, "s_out": T * N * 4,
+        "dh": T * d * a, "dx": T * d * a, "dw_router": N * d * 4, "dw_gu": E * 2 * I * d * 4,
+        "dw_down": E * d * I * 4,
     }
 
 
@@ -287,3 +299,84 @@ _trace_keep = None
 
 def moe_selftest_bounded_wait(limit_us: int, stream=None) -> None:
     _check(_lib.moe_selftest_bounded_wait(limit_us, _stream(stream)), "moe_selftest_bounded_wait")
+
+
+def moe_backward_workspace_size(desc: MoeLayerDesc) -> int:
+    return int(_lib.moe_backward_workspace_size(ctypes.byref(desc)))
+
+
+def backward_workspace(desc: MoeLayerDesc, device="cuda"):
+    """A uint8 CUDA tensor of moe_backward_workspace_size(desc) bytes."""
+    import torch
+    n = moe_backward_workspace_size(desc)
+    if n == 0:
+        raise MoeError(ERR_UNSUPPORTED, "moe_backward_workspace_size")
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def moe_backward(desc, x, w_router, bias, w_gu, w_down, dh, dx, dw_router, dw_gu, dw_down, ws,
+                 stream=None) -> None:
+    _need("moe_backward", desc, x=x, w_router=w_router, bias=bias, w_gu=w_gu, w_down=w_down,
+          dh=dh, dx=dx, dw_router=dw_router, dw_gu=dw_gu, dw_down=dw_down)
+    _check(_lib.moe_backward(ctypes.byref(desc), _ptr(x), _ptr(w_router), _ptr(bias), _ptr(w_gu),
+                             _ptr(w_down), _ptr(dh), _ptr(dx), _ptr(dw_router), _ptr(dw_gu),
+                             _ptr(dw_down), _ptr(ws), ws.numel() if ws is not None else 0,
+                             _stream(stream)), "moe_backward")
+
+
+def moe_backward_launch_count(desc) -> int:
+    return int(_lib.moe_backward_launch_count(ctypes.byref(desc)))
+
+
+def moe_expert_ffn_workspace_size(desc: MoeLayerDesc, n_groups: int, n_rows_out: int) -> int:
+    return int(_lib.moe_expert_ffn_workspace_size(ctypes.byref(desc), n_groups, n_rows_out))
+
+
+def moe_expert_ffn(desc, n_experts: int, groups, x_rows, row_w, w_gu, w_down, y_rows, ws,
+                   stream=None) -> None:
+    """y_rows[out0 + r] = row_w[out0 + r] * FFN_expert(x_rows[row0 + r]) for each group
+    (row0, rows, expert, out0) of the int32 [n_groups, 4] device tensor `groups`."""
+    for name, t, rows_needed in (("x_rows", x_rows, x_rows.shape[0]),
+                                 ("y_rows", y_rows, y_rows.shape[0])):
+        if not t.is_contiguous() or t.shape[-1] != desc.d:
+            raise MoeError(ERR_INVALID_ARG, f"moe_expert_ffn: {name} must be contiguous [rows, d]")
+    if not groups.is_contiguous() or groups.dtype.itemsize != 4 or groups.shape[-1] != 4:
+        raise MoeError(ERR_INVALID_ARG, "moe_expert_ffn: groups must be contiguous int32 [n, 4]")
+    if row_w is not None and row_w.numel() < y_rows.shape[0]:
+        raise MoeError(ERR_INVALID_ARG, "moe_expert_ffn: row_w shorter than y_rows")
+    w = {DT_F32: 4, DT_BF16: 2, DT_E4M3: 1}[desc.w_dtype]
+    if w_gu.numel() * w_gu.element_size() < n_experts * 2 * desc.inter * desc.d * w or \
+            w_down.numel() * w_down.element_size() < n_experts * desc.d * desc.inter * w:
+        raise MoeError(ERR_INVALID_ARG, "moe_expert_ffn: expert weights shorter than n_experts")
+    _check(_lib.moe_expert_ffn(ctypes.byref(desc), n_experts, groups.shape[0], _ptr(groups),
+                               x_rows.shape[0], y_rows.shape[0], _ptr(x_rows), _ptr(row_w),
+                               _ptr(w_gu), _ptr(w_down), _ptr(y_rows), _ptr(ws),
+                               ws.numel() if ws is not None else 0, _stream(stream)),
+           "moe_expert_ffn")
+
+
+def moe_combine_rows(desc, x_residual, y_shared, y_rows, row_of, h, stream=None) -> None:
+    """h[t] = x_res[t] + sum_s y_shared[s*T + t] + sum_k y_rows[row_of[t*K + k]]."""
+    _need("moe_combine_rows", desc, x_residual=x_residual, h=h)
+    if row_of.numel() < desc.T * desc.top_k or not row_of.is_contiguous():
+        raise MoeError(ERR_INVALID_ARG, "moe_combine_rows: row_of must hold T*K int32")
+    if y_shared is not None and y_shared.numel() < desc.n_shared * desc.T * desc.d:
+        raise MoeError(ERR_INVALID_ARG, "moe_combine_rows: y_shared shorter than Ks*T rows")
+    _check(_lib.moe_combine_rows(ctypes.byref(desc), _ptr(x_residual), _ptr(y_shared),
+                                 _ptr(y_rows), _ptr(row_of),
+                                 y_rows.shape[0] if y_rows is not None else 0, _ptr(h),
+                                 _stream(stream)), "moe_combine_rows")
+
+
+def moe_dispatch_rows(desc, x, topk_w, row_of, x_rows, w_rows, stream=None) -> None:
+    """x_rows[row_of[t*K + k]] = x[t], w_rows[row_of[t*K + k]] = topk_w[t, k]."""
+    _need("moe_dispatch_rows", desc, x=x, topk_w=topk_w)
+    if row_of.numel() < desc.T * desc.top_k or not row_of.is_contiguous():
+        raise MoeError(ERR_INVALID_ARG, "moe_dispatch_rows: row_of must hold T*K int32")
+    if not x_rows.is_contiguous() or x_rows.shape[-1] != desc.d:
+        raise MoeError(ERR_INVALID_ARG, "moe_dispatch_rows: x_rows must be contiguous [rows, d]")
+    if w_rows is not None and w_rows.numel() < x_rows.shape[0]:
+        raise MoeError(ERR_INVALID_ARG, "moe_dispatch_rows: w_rows shorter than x_rows")
+    _check(_lib.moe_dispatch_rows(ctypes.byref(desc), _ptr(x), _ptr(topk_w), _ptr(row_of),
+                                  x_rows.shape[0], _ptr(x_rows), _ptr(w_rows), _stream(stream)),
+           "moe_dispatch_rows")

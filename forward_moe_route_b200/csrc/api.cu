@@ -17,6 +17,8 @@
 #include "gemm_gu.cuh"
 #include "permute.cuh"
 #include "route.cuh"
+#include "bwd.cuh"
+#include "gemm_bwd.cuh"
 
 using namespace moe;
 
@@ -78,7 +80,7 @@ moe_status fill_dims(const moe_layer_desc* desc, Dims* D) {
 
 struct Layout {
   size_t logits, topk_idx, topk_w, counts, hist, offsets, perm_src, slot_of, pair_of, gtab;
-  size_t x_perm, x_perm_scale, hbuf, hscale, y_slots, total;
+  size_t x_perm, x_perm_scale, hbuf, hscale, y_slots, cnt, total;
 };
 
 Layout layout(const Dims& D) {
@@ -102,6 +104,8 @@ Layout layout(const Dims& D) {
   L.hbuf = take(hrows * D.I * D.op_esz);
   L.hscale = take(D.fp8 ? hrows * (D.I / 128) * 4 : 0);
   L.y_slots = take((size_t)D.T * (D.K + D.Ks) * D.d * D.y_esz);
+  // arrival counters of the fused residual (bf16 layers): [T, d/32]
+  L.cnt = take((!D.f32 && !D.fp8) ? (size_t)D.T * (D.d / 32) * 4 : 0);
   L.total = o;
   return L;
 }
@@ -270,16 +274,15 @@ route::Params route_params(const moe_layer_desc& s) {
 
 template <int VPL>
 moe_status launch_topk(const float* logits, const float* bias, const route::Params& p,
-                       int32_t* idx, float* w, int32_t* counts, cudaStream_t st) {
+                       int32_t* idx, float* w, cudaStream_t st) {
   return launch_chain("k_topk", route::k_topk<VPL>, dim3((p.T + 7) / 8), dim3(256), 0, st,
-                      logits, bias, p, idx, w, counts);
+                      logits, bias, p, idx, w);
 }
 template <int VPL>
 moe_status launch_route_f32(const float* x, const float* wr, int d, const float* bias,
-                            const route::Params& p, int32_t* idx, float* w, int32_t* counts,
-                            cudaStream_t st) {
+                            const route::Params& p, int32_t* idx, float* w, cudaStream_t st) {
   return launch_chain("k_route_f32", route::k_route_f32<VPL>, dim3((p.T + 7) / 8), dim3(256), 0,
-                      st, x, wr, d, bias, p, idx, w, counts);
+                      st, x, wr, d, bias, p, idx, w);
 }
 
 // ----------------------------------------------------------------------------- stages
@@ -319,55 +322,79 @@ moe_status launch_router(const Dims& D, const void* x, const void* w_router, flo
                       gemm8::smem_bytes(stages, 1), st, ta, tb, a);
 }
 
+// Selection and gate weights.  With counts != nullptr the tokens per expert
+// are counted too: the per-chunk histogram and its totals (k_hist, k_scan),
+// which the layer forward instead takes from its permutation step.
 moe_status do_route(const moe_layer_desc& s, const Dims& D, const Layout& L, const void* x,
                     const void* w_router, const float* bias, int32_t* topk_idx, float* topk_w,
                     int32_t* counts, uint8_t* ws, int sms, cudaStream_t st) {
   const route::Params p = route_params(s);
   const int N = (int)D.N;
   if (D.T == 0)
-    return launch_chain("k_zero_i32", route::k_zero_i32, dim3(1), dim3(256), 0, st, counts, N);
+    return counts ? launch_chain("k_zero_i32", route::k_zero_i32, dim3(1), dim3(256), 0, st,
+                                 counts, N)
+                  : MOE_OK;
+  moe_status rc;
   if (D.f32) {
-    moe_status rc =
-        launch_chain("k_zero_i32", route::k_zero_i32, dim3(1), dim3(256), 0, st, counts, N);
-    if (rc != MOE_OK) return rc;
     const float* xf = static_cast<const float*>(x);
     const float* wf = static_cast<const float*>(w_router);
     const int dd = (int)D.d;
-    if (N <= 32) return launch_route_f32<1>(xf, wf, dd, bias, p, topk_idx, topk_w, counts, st);
-    if (N <= 64) return launch_route_f32<2>(xf, wf, dd, bias, p, topk_idx, topk_w, counts, st);
-    if (N <= 128) return launch_route_f32<4>(xf, wf, dd, bias, p, topk_idx, topk_w, counts, st);
-    if (N <= 256) return launch_route_f32<8>(xf, wf, dd, bias, p, topk_idx, topk_w, counts, st);
-    return launch_route_f32<16>(xf, wf, dd, bias, p, topk_idx, topk_w, counts, st);
+    if (N <= 32) rc = launch_route_f32<1>(xf, wf, dd, bias, p, topk_idx, topk_w, st);
+    else if (N <= 64) rc = launch_route_f32<2>(xf, wf, dd, bias, p, topk_idx, topk_w, st);
+    else if (N <= 128) rc = launch_route_f32<4>(xf, wf, dd, bias, p, topk_idx, topk_w, st);
+    else if (N <= 256) rc = launch_route_f32<8>(xf, wf, dd, bias, p, topk_idx, topk_w, st);
+    else rc = launch_route_f32<16>(xf, wf, dd, bias, p, topk_idx, topk_w, st);
+  } else {
+    float* logits = reinterpret_cast<float*>(ws + L.logits);
+    rc = launch_router(D, x, w_router, logits, nullptr, sms, st);
+    if (rc != MOE_OK) return rc;
+    if (N <= 32) rc = launch_topk<1>(logits, bias, p, topk_idx, topk_w, st);
+    else if (N <= 64) rc = launch_topk<2>(logits, bias, p, topk_idx, topk_w, st);
+    else if (N <= 128) rc = launch_topk<4>(logits, bias, p, topk_idx, topk_w, st);
+    else if (N <= 256) rc = launch_topk<8>(logits, bias, p, topk_idx, topk_w, st);
+    else rc = launch_topk<16>(logits, bias, p, topk_idx, topk_w, st);
   }
-  float* logits = reinterpret_cast<float*>(ws + L.logits);
-  moe_status rc = launch_router(D, x, w_router, logits, counts, sms, st);
-  if (rc != MOE_OK) return rc;
-  if (N <= 32) return launch_topk<1>(logits, bias, p, topk_idx, topk_w, counts, st);
-  if (N <= 64) return launch_topk<2>(logits, bias, p, topk_idx, topk_w, counts, st);
-  if (N <= 128) return launch_topk<4>(logits, bias, p, topk_idx, topk_w, counts, st);
-  if (N <= 256) return launch_topk<8>(logits, bias, p, topk_idx, topk_w, counts, st);
-  return launch_topk<16>(logits, bias, p, topk_idx, topk_w, counts, st);
+  if (rc != MOE_OK || !counts) return rc;
+  int32_t* hist = reinterpret_cast<int32_t*>(ws + L.hist);
+  int32_t* offsets = reinterpret_cast<int32_t*>(ws + L.offsets);
+  const int T = (int)D.T, K = (int)D.K;
+  rc = launch_chain("k_hist", perm::k_hist, dim3(D.n_chunks), dim3(256), N * 4, st,
+                    static_cast<const int32_t*>(topk_idx), T, K, N, hist);
+  if (rc == MOE_OK)
+    rc = launch_chain("k_scan", perm::k_scan, dim3(1), dim3(1024), 0, st, hist, (int)D.n_chunks,
+                      N, static_cast<const int32_t*>(nullptr), counts, offsets);
+  return rc;
 }
 
-moe_status do_permute(const Dims& D, const Layout& L, const void* x, const int32_t* topk_idx,
+// hist: the per-chunk histogram scratch, ceil(T/128) x N int32 (the
+// workspace's, or the fixed array of moe_permute_noalloc).
+// counts: checked against the histogram's totals when given; counts_out:
+// receives them when given (the layer forward's routing does not count).
+moe_status do_permute(const Dims& D, int32_t* hist, const void* x, const int32_t* topk_idx,
                       const int32_t* counts, int32_t* offsets, int32_t* perm_src,
-                      int32_t* slot_of, void* x_perm, float* x_perm_scale, uint8_t* ws,
-                      cudaStream_t st) {
+                      int32_t* slot_of, void* x_perm, float* x_perm_scale, cudaStream_t st,
+                      int32_t* counts_out = nullptr) {
   const int T = (int)D.T, K = (int)D.K, N = (int)D.N;
-  int32_t* hist = reinterpret_cast<int32_t*>(ws + L.hist);
-  if (T == 0)
+  if (T == 0) {
+    if (counts_out) {
+      const moe_status rc0 = launch_chain("k_zero_i32", route::k_zero_i32, dim3(1), dim3(256), 0,
+                                          st, counts_out, N);
+      if (rc0 != MOE_OK) return rc0;
+    }
     return launch_chain("k_zero_i32", route::k_zero_i32, dim3(1), dim3(256), 0, st, offsets,
                         N + 1);
+  }
   moe_status rc = launch_chain("k_hist", perm::k_hist, dim3(D.n_chunks), dim3(256), N * 4, st,
                                topk_idx, T, K, N, hist);
   if (rc == MOE_OK)
     rc = launch_chain("k_scan", perm::k_scan, dim3(1), dim3(1024), 0, st, hist, (int)D.n_chunks,
-                      N, counts, offsets);
+                      N, counts, counts_out, offsets);
   if (rc == MOE_OK)
     rc = launch_chain("k_slots", perm::k_slots, dim3(D.n_chunks), dim3(perm::SLOT_WARPS * 32),
                       perm::SLOT_WARPS * N * 4, st, topk_idx, T, K, N,
                       static_cast<const int32_t*>(hist), slot_of, perm_src);
   if (rc != MOE_OK) return rc;
+  if (!x_perm) return MOE_OK;   // maps only (moe_permute with x_perm = NULL)
   if (D.fp8)
     return launch_chain("k_gather_quant", perm::k_gather_quant, dim3((T + 7) / 8), dim3(256), 0,
                         st, static_cast<const __nv_bfloat16*>(x), T, K, (int)D.d, (int)D.R,
@@ -505,11 +532,14 @@ moe_status pair_config(int slot, F* func, int threads, size_t smem, int64_t tile
   return MOE_OK;
 }
 
-moe_status launch_down(int kind, const void* w_down, const void* hbuf, size_t esz,
-                       int64_t hrows, int64_t tok_tiles, gemmt::Args a, cudaStream_t st) {
+// n_experts: experts held in w_down (the weight map's extent; the group count
+// can be larger or smaller than it).
+moe_status launch_down(int kind, const void* w_down, int64_t n_experts, const void* hbuf,
+                       size_t esz, int64_t hrows, int64_t tok_tiles, gemmt::Args a,
+                       cudaStream_t st) {
   CUtensorMap tw, th;
   moe_status rc = make_tmap(&tw, w_down, esz, a.num_kb * (uint64_t)a.kb_elems,
-                            (uint64_t)a.gt.n * a.w_rows_per_expert, gemmt::WM);
+                            (uint64_t)n_experts * a.w_rows_per_expert, gemmt::WM);
   if (rc == MOE_OK)
     rc = make_tmap(&th, hbuf, esz, a.num_kb * (uint64_t)a.kb_elems, hrows, gemmt::TN / 2);
   if (rc != MOE_OK) return rc;
@@ -534,12 +564,12 @@ moe_status launch_down(int kind, const void* w_down, const void* hbuf, size_t es
 
 // Gate/up GEMM with the SwiGLU epilogue on CTA pairs: 128 features x up to
 // 256 tokens per cluster tile; shared experts read x, routed experts x_perm.
-moe_status launch_gate_up(int kind, const void* w_gu, const void* x, const void* x_perm,
-                          size_t esz, int64_t T, int64_t R, int64_t tok_tiles, gemmgu::Args a,
-                          cudaStream_t st) {
+moe_status launch_gate_up(int kind, const void* w_gu, int64_t n_experts, const void* x,
+                          const void* x_perm, size_t esz, int64_t T, int64_t R,
+                          int64_t tok_tiles, gemmgu::Args a, cudaStream_t st) {
   const uint64_t inner = a.num_kb * (uint64_t)a.kb_elems;
   CUtensorMap tw, tx, txp;
-  moe_status rc = make_tmap(&tw, w_gu, esz, inner, (uint64_t)a.gt.n * a.w_rows_per_expert,
+  moe_status rc = make_tmap(&tw, w_gu, esz, inner, (uint64_t)n_experts * a.w_rows_per_expert,
                             gemmgu::FM);
   if (rc == MOE_OK) rc = make_tmap(&tx, x, esz, inner, T, gemmgu::TN / 2);
   if (rc == MOE_OK) rc = make_tmap(&txp, x_perm, esz, inner, R, gemmgu::TN / 2);
@@ -564,22 +594,32 @@ moe_status launch_gate_up(int kind, const void* w_gu, const void* x, const void*
   return launched("gate/up GEMM (CTA pairs)");
 }
 
+// fuse_res / fuse_h (bf16 layers only): the down projection also adds the
+// residual and writes h (see gemm_t.cuh); nullptr keeps the slots-only path.
+bool fusable(const Dims& D) { (void)D; return false; }
+
 moe_status do_grouped(const Dims& D, const Layout& L, const void* x, const void* x_perm,
                       const float* x_perm_scale, const int32_t* offsets, const int32_t* slot_of,
                       const float* topk_w, const void* w_gu, const float* w_gu_scale,
                       const void* w_down, const float* w_down_scale, void* y_slots, uint8_t* ws,
-                      int sms, cudaStream_t st) {
+                      int sms, cudaStream_t st, const void* fuse_res = nullptr,
+                      void* fuse_h = nullptr) {
   if (D.T == 0) return MOE_OK;
   const int E = (int)D.E;
   int32_t* gtab = reinterpret_cast<int32_t*>(ws + L.gtab);
   int32_t* pair_of = reinterpret_cast<int32_t*>(ws + L.pair_of);
   void* hbuf = ws + L.hbuf;
-  const int prep_blocks = 1 + (int)((D.R + 1023) / 1024 < 4 * sms ? (D.R + 1023) / 1024 : 4 * sms);
+  const bool fuse = fuse_h && fusable(D);
+  int32_t* cnt = fuse ? reinterpret_cast<int32_t*>(ws + L.cnt) : nullptr;
+  const int n_cnt = fuse ? (int)(D.T * (D.d / 32)) : 0;
+  const int64_t prep_items = D.R > n_cnt ? D.R : n_cnt;
+  const int prep_blocks =
+      1 + (int)((prep_items + 1023) / 1024 < 4 * sms ? (prep_items + 1023) / 1024 : 4 * sms);
   moe_status rc = trace(2, st);
   if (rc != MOE_OK) return rc;
   rc = launch_chain("k_prep_groups", perm::k_prep_groups, dim3(prep_blocks), dim3(1024), 0, st,
                     offsets, (int)D.T, (int)D.K, (int)D.Ks, (int)D.N, D.fp8 ? 1 : 0, gtab,
-                    slot_of, pair_of);
+                    slot_of, pair_of, cnt, n_cnt);
   if (rc != MOE_OK) return rc;
   if (D.fp8)
     return do_grouped_fp8(D, L, x_perm, x_perm_scale, gtab, pair_of, topk_w, w_gu, w_gu_scale,
@@ -609,7 +649,7 @@ moe_status do_grouped(const Dims& D, const Layout& L, const void* x, const void*
     a.fmt = fmt;
     a.out_bf16 = D.f32 ? 0 : 1;
     a.h = hbuf;
-    rc = launch_gate_up(kind, w_gu, x, x_perm, esz, D.T, D.R, tok_tiles, a, st);
+    rc = launch_gate_up(kind, w_gu, D.E, x, x_perm, esz, D.T, D.R, tok_tiles, a, st);
     if (rc != MOE_OK) return rc;
     if ((rc = trace(3, st)) != MOE_OK) return rc;
   }
@@ -633,7 +673,12 @@ moe_status do_grouped(const Dims& D, const Layout& L, const void* x, const void*
     a.topk_w = topk_w;
     a.K = (int)D.K;
     a.Ks = (int)D.Ks;
-    rc = launch_down(kind, w_down, hbuf, esz, hrows, tok_tiles, a, st);
+    if (fuse) {
+      a.cnt = cnt;
+      a.x_res = static_cast<const __nv_bfloat16*>(fuse_res);
+      a.h = static_cast<__nv_bfloat16*>(fuse_h);
+    }
+    rc = launch_down(kind, w_down, D.E, hbuf, esz, hrows, tok_tiles, a, st);
     if (rc != MOE_OK) return rc;
     rc = trace(4, st);
   }
@@ -650,6 +695,331 @@ moe_status do_combine(const Dims& D, const void* x_res, const void* y, void* h, 
                         y, h, (int)D.T, (int)D.d, (int)D.K, (int)D.Ks);
   return launch_chain("k_combine", perm::k_combine<true>, dim3(blocks), dim3(256), 0, st, x_res,
                       y, h, (int)D.T, (int)D.d, (int)D.K, (int)D.Ks);
+}
+
+// ----------------------------------------------------------------------------- expert parallelism
+// Workspace of moe_expert_ffn: the group table, then H [n_rows_out, I].
+struct FfnLayout {
+  size_t gtab, hbuf, total;
+};
+FfnLayout ffn_layout(const Dims& D, int n_groups, int64_t n_rows_out) {
+  FfnLayout F;
+  size_t o = 0;
+  auto take = [&](size_t bytes) { size_t at = o; o = align_up(o + bytes, kAlign); return at; };
+  F.gtab = take((size_t)gemm::group_tab_ints(n_groups) * 4);
+  F.hbuf = take((size_t)(n_rows_out > 0 ? n_rows_out : 1) * D.I * D.op_esz);
+  F.total = o;
+  return F;
+}
+
+moe_status do_expert_ffn(const Dims& D, int n_experts, int n_groups, const int32_t* groups,
+                         int64_t n_in, int64_t n_out, const void* x_rows, const float* row_w,
+                         const void* w_gu, const void* w_down, void* y_rows, uint8_t* ws,
+                         int sms, cudaStream_t st) {
+  const FfnLayout F = ffn_layout(D, n_groups, n_out);
+  int32_t* gtab = reinterpret_cast<int32_t*>(ws + F.gtab);
+  void* hbuf = ws + F.hbuf;
+  moe_status rc = launch_chain("k_prep_user_groups", perm::k_prep_user_groups, dim3(1),
+                               dim3(1024), 0, st, groups, n_groups, n_experts, (int)n_in,
+                               (int)n_out, gtab);
+  if (rc != MOE_OK) return rc;
+  const size_t esz = D.op_esz;
+  const int kind = D.f32 ? 1 : 0;
+  const uint32_t fmt = D.f32 ? 2u : 1u;
+  const int kbe = (int)(gemm::KB / esz);
+  // upper bound on 256-token tiles over all groups
+  const int64_t tok_tiles = (n_out + (int64_t)n_groups * 255) / 256;
+  {
+    gemmgu::Args a;
+    memset(&a, 0, sizeof(a));
+    a.gt.base = gtab;
+    a.gt.n = n_groups;
+    a.n_ft = (int)((D.I + 2 * gemmgu::FM - 1) / (2 * gemmgu::FM));
+    a.num_kb = (int)(D.d * esz / gemm::KB);
+    a.kb_elems = kbe;
+    a.inter = (int)D.I;
+    a.w_rows_per_expert = (int)(2 * D.I);
+    a.fmt = fmt;
+    a.out_bf16 = D.f32 ? 0 : 1;
+    a.h = hbuf;
+    rc = launch_gate_up(kind, w_gu, n_experts, x_rows, x_rows, esz, n_in, n_in, tok_tiles, a,
+                        st);
+    if (rc != MOE_OK) return rc;
+  }
+  {
+    gemmt::Args a;
+    memset(&a, 0, sizeof(a));
+    a.gt.base = gtab;
+    a.gt.n = n_groups;
+    a.n_wt = (int)((D.d + 2 * gemmt::WM - 1) / (2 * gemmt::WM));
+    a.num_kb = (int)(D.I * esz / gemm::KB);
+    a.kb_elems = kbe;
+    a.w_rows_per_expert = (int)D.d;
+    a.fmt = fmt;
+    a.out_bf16 = D.f32 ? 0 : 1;
+    a.y = y_rows;
+    a.d = (int)D.d;
+    a.plain = 1;
+    a.row_w = row_w;
+    rc = launch_down(kind, w_down, n_experts, hbuf, esz, n_out, tok_tiles, a, st);
+  }
+  return rc;
+}
+
+// ----------------------------------------------------------------------------- backward
+// Workspace of moe_backward: the forward's routing buffers (same offsets as
+// the forward layout), then the padded row buffers of the backward.
+struct BwdLayout {
+  size_t poff, tabs, row_pair, row_w, x_pad, dh_pad, ab, dab, zg, dgp, dl, dxr, dslots, total;
+  int64_t rows_routed;   // rows of x_pad / dh_pad (routed segments, padded)
+  int64_t rows;          // rows of ab / dab / zg / dgp (routed and shared segments)
+  int n_it;              // feature tiles of 256 over I (partials per row)
+};
+
+constexpr int kBwdTables = 7;
+
+BwdLayout bwd_layout(const Dims& D, const Layout& L) {
+  BwdLayout B;
+  size_t o = align_up(L.gtab + (size_t)gemm::group_tab_ints((int)D.E) * 4, kAlign);
+  auto take = [&](size_t bytes) { size_t at = o; o = align_up(o + bytes, kAlign); return at; };
+  B.rows_routed = D.R + (int64_t)bwd::PAD * D.N;
+  B.rows = B.rows_routed + D.Ks * (int64_t)bwd::pad64((int)D.T);
+  B.n_it = (int)((D.I + gbwd::BN - 1) / gbwd::BN);
+  B.poff = take((size_t)(D.E + 1) * 4);
+  B.tabs = take((size_t)kBwdTables * D.E * gbwd::GB_FIELDS * 4);
+  B.row_pair = take((size_t)B.rows * 4);
+  B.row_w = take((size_t)B.rows * 4);
+  B.x_pad = take((size_t)B.rows_routed * D.d * 2);
+  B.dh_pad = take((size_t)B.rows_routed * D.d * 2);
+  B.ab = take((size_t)B.rows * 2 * D.I * 2);
+  B.dab = take((size_t)B.rows * 2 * D.I * 2);
+  B.zg = take((size_t)B.rows * D.I * 2);
+  B.dgp = take((size_t)B.rows * B.n_it * 4);
+  B.dl = take((size_t)D.T * D.N * 2);
+  B.dxr = take((size_t)D.T * D.d * 2);
+  B.dslots = take((size_t)D.T * (D.K + D.Ks) * D.d * 2);
+  B.total = o;
+  return B;
+}
+
+// 2-D tensor map for an operand read MN-major: rows of `inner` bf16 elements
+// (the M or N extent), `rows` rows (the K extent); box = 64 elements x 64 rows.
+moe_status make_tmap_mn(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows) {
+  cuuint64_t dims[2] = {inner, rows > 0 ? rows : 1};
+  cuuint64_t strides[1] = {inner * 2};
+  cuuint32_t box[2] = {64, 64};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    snprintf(t_errmsg, sizeof(t_errmsg), "cuTensorMapEncodeTiled (MN-major): CUresult %d "
+             "(rows %llu, inner %llu)", (int)r, (unsigned long long)rows,
+             (unsigned long long)inner);
+    return MOE_ERR_CUDA;
+  }
+  return MOE_OK;
+}
+
+// One operand of a backward GEMM: base, row length and row count, and whether
+// it is read MN-major (its rows are the K index).
+struct Operand {
+  const void* base;
+  uint64_t inner, rows;
+};
+
+template <bool A_MN, bool B_MN, int EPI>
+moe_status launch_gemm_bwd(const char* what, Operand a0, Operand a1, Operand b0, Operand b1,
+                           gbwd::Args args, int64_t tiles_bound, int sms, cudaStream_t st) {
+  CUtensorMap ta0, ta1, tb0, tb1;
+  auto mk = [&](CUtensorMap* m, const Operand& o, bool mn, uint32_t box_rows) {
+    return mn ? make_tmap_mn(m, o.base, o.inner, o.rows) : make_tmap(m, o.base, 2, o.inner, o.rows,
+                                                                     box_rows);
+  };
+  moe_status rc = mk(&ta0, a0, A_MN, gbwd::BM);
+  if (rc == MOE_OK) rc = mk(&ta1, a1, A_MN, gbwd::BM);
+  if (rc == MOE_OK) rc = mk(&tb0, b0, B_MN, gbwd::BN);
+  if (rc == MOE_OK) rc = mk(&tb1, b1, B_MN, gbwd::BN);
+  if (rc != MOE_OK) return rc;
+  int stages = 0;
+  for (int s = 4; s >= 2 && !stages; --s)
+    if (gbwd::smem_bytes(s, args.n_probs) <= (size_t)kMaxSmem) stages = s;
+  if (!stages) return MOE_ERR_UNSUPPORTED;
+  args.stages = stages;
+  const size_t smem = gbwd::smem_bytes(stages, args.n_probs);
+  cudaError_t e = cudaFuncSetAttribute(gbwd::k_gemm_bwd<A_MN, B_MN, EPI>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
+  if (e != cudaSuccess) return cuda_fail(e, what);
+  const int grid = (int)(tiles_bound < sms ? (tiles_bound > 0 ? tiles_bound : 1) : sms);
+  return launch_chain(what, gbwd::k_gemm_bwd<A_MN, B_MN, EPI>, dim3(grid),
+                      dim3(gbwd::NUM_THREADS), smem, st, ta0, ta1, tb0, tb1, args);
+}
+
+template <int VPL>
+moe_status launch_gate_bwd(const float* logits, const route::Params& p, const int32_t* idx,
+                           const int32_t* slot_of, const int32_t* offsets, const int32_t* poff,
+                           const float* dgp, int n_it, __nv_bfloat16* dl, cudaStream_t st) {
+  return launch_chain("k_gate_bwd", bwd::k_gate_bwd<VPL>, dim3((p.T + 7) / 8), dim3(256), 0, st,
+                      logits, p, idx, slot_of, offsets, poff, dgp, n_it, dl);
+}
+
+moe_status do_backward(const moe_layer_desc& s, const Dims& D, const Layout& L,
+                       const BwdLayout& B, const void* x, const void* w_router,
+                       const float* bias, const void* w_gu, const void* w_down, const void* dh,
+                       void* dx, float* dw_router, float* dw_gu, float* dw_down, uint8_t* ws,
+                       int sms, cudaStream_t st) {
+  const int T = (int)D.T, d = (int)D.d, I = (int)D.I, N = (int)D.N, K = (int)D.K;
+  const int Ks = (int)D.Ks, E = (int)D.E;
+  int32_t* idx = reinterpret_cast<int32_t*>(ws + L.topk_idx);
+  float* tw = reinterpret_cast<float*>(ws + L.topk_w);
+  int32_t* counts = reinterpret_cast<int32_t*>(ws + L.counts);
+  int32_t* hist = reinterpret_cast<int32_t*>(ws + L.hist);
+  int32_t* offsets = reinterpret_cast<int32_t*>(ws + L.offsets);
+  int32_t* perm_src = reinterpret_cast<int32_t*>(ws + L.perm_src);
+  int32_t* slot_of = reinterpret_cast<int32_t*>(ws + L.slot_of);
+  const float* logits = reinterpret_cast<const float*>(ws + L.logits);
+  int32_t* poff = reinterpret_cast<int32_t*>(ws + B.poff);
+  int32_t* tabs = reinterpret_cast<int32_t*>(ws + B.tabs);
+  const size_t tab_ints = (size_t)E * gbwd::GB_FIELDS;
+  int32_t* tab[kBwdTables];
+  for (int i = 0; i < kBwdTables; ++i) tab[i] = tabs + i * tab_ints;
+  int32_t* row_pair = reinterpret_cast<int32_t*>(ws + B.row_pair);
+  float* row_w = reinterpret_cast<float*>(ws + B.row_w);
+  auto* x_pad = reinterpret_cast<__nv_bfloat16*>(ws + B.x_pad);
+  auto* dh_pad = reinterpret_cast<__nv_bfloat16*>(ws + B.dh_pad);
+  auto* ab = reinterpret_cast<__nv_bfloat16*>(ws + B.ab);
+  auto* dab = reinterpret_cast<__nv_bfloat16*>(ws + B.dab);
+  auto* zg = reinterpret_cast<__nv_bfloat16*>(ws + B.zg);
+  float* dgp = reinterpret_cast<float*>(ws + B.dgp);
+  auto* dl = reinterpret_cast<__nv_bfloat16*>(ws + B.dl);
+  auto* dxr = reinterpret_cast<__nv_bfloat16*>(ws + B.dxr);
+  auto* dslots = reinterpret_cast<__nv_bfloat16*>(ws + B.dslots);
+
+  // routing and the permutation maps, as in the forward
+  moe_status rc = do_route(s, D, L, x, w_router, bias, idx, tw, nullptr, ws, sms, st);
+  if (rc != MOE_OK) return rc;
+  rc = launch_chain("k_hist", perm::k_hist, dim3(D.n_chunks), dim3(256), N * 4, st,
+                    static_cast<const int32_t*>(idx), T, K, N, hist);
+  if (rc == MOE_OK)
+    rc = launch_chain("k_scan", perm::k_scan, dim3(1), dim3(1024), 0, st, hist, (int)D.n_chunks,
+                      N, static_cast<const int32_t*>(nullptr), counts, offsets);
+  if (rc == MOE_OK)
+    rc = launch_chain("k_slots", perm::k_slots, dim3(D.n_chunks), dim3(perm::SLOT_WARPS * 32),
+                      perm::SLOT_WARPS * N * 4, st, static_cast<const int32_t*>(idx), T, K, N,
+                      static_cast<const int32_t*>(hist), slot_of, perm_src);
+  if (rc != MOE_OK) return rc;
+  bwd::PrepArgs pa;
+  pa.offsets = offsets;
+  pa.T = T; pa.d = d; pa.I = I; pa.Ks = Ks; pa.N = N;
+  pa.poff = poff;
+  pa.tab_ab = tab[0]; pa.tab_dz = tab[1]; pa.tab_du = tab[2]; pa.tab_dwd = tab[3];
+  pa.tab_dwgu = tab[4]; pa.tab_dxr = tab[5]; pa.tab_dwr = tab[6];
+  rc = launch_chain("k_bwd_prep", bwd::k_bwd_prep, dim3(1), dim3(1024), 0, st, pa);
+  if (rc == MOE_OK)
+    rc = launch_chain("k_bwd_gather", bwd::k_bwd_gather, dim3((T + 7) / 8), dim3(256), 0, st,
+                      static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(dh),
+                      T, K, d, static_cast<const int32_t*>(idx), static_cast<const float*>(tw),
+                      static_cast<const int32_t*>(slot_of), static_cast<const int32_t*>(offsets),
+                      static_cast<const int32_t*>(poff), N, x_pad, dh_pad, row_pair, row_w);
+  if (rc == MOE_OK)
+    rc = launch_chain("k_bwd_zero_pads", bwd::k_bwd_zero_pads, dim3(N), dim3(256), 0, st,
+                      static_cast<const int32_t*>(offsets), static_cast<const int32_t*>(poff), d,
+                      x_pad, dh_pad, row_pair, row_w);
+  if (rc != MOE_OK) return rc;
+
+  // tile bounds for the grid size (the exact counts are known on the device only)
+  const int64_t mt_rows = (B.rows + gbwd::BM - 1) / gbwd::BM + E;
+  auto nt = [](int64_t n) { return (n + gbwd::BN - 1) / gbwd::BN; };
+  const uint64_t W_gu_rows = (uint64_t)E * 2 * I, W_d_rows = (uint64_t)E * d;
+  const Operand X{x, (uint64_t)d, (uint64_t)T}, DH{dh, (uint64_t)d, (uint64_t)T};
+  const Operand XP{x_pad, (uint64_t)d, (uint64_t)B.rows_routed};
+  const Operand DHP{dh_pad, (uint64_t)d, (uint64_t)B.rows_routed};
+  const Operand WGU{w_gu, (uint64_t)d, W_gu_rows}, WD{w_down, (uint64_t)I, W_d_rows};
+  const Operand AB{ab, (uint64_t)(2 * I), (uint64_t)B.rows};
+  const Operand DAB{dab, (uint64_t)(2 * I), (uint64_t)B.rows};
+  const Operand ZG{zg, (uint64_t)I, (uint64_t)B.rows};
+  const Operand DL{dl, (uint64_t)N, (uint64_t)T}, WR{w_router, (uint64_t)d, (uint64_t)N};
+  (void)AB;
+  gbwd::Args ga;
+  memset(&ga, 0, sizeof(ga));
+  ga.n_probs = E;
+  ga.K = K;
+  ga.Ks = Ks;
+  ga.inter = I;
+  // G1: a | b pre-activations of every (row, expert)
+  ga.tab = tab[0];
+  ga.c = ab;
+  ga.ldc = 2 * I;
+  rc = launch_gemm_bwd<false, false, gbwd::EPI_BF16>("backward GEMM ab = X W_gu^T", X, XP, WGU,
+                                                      WGU, ga, mt_rows * nt(2 * I), sms, st);
+  if (rc != MOE_OK) return rc;
+  // G2: dz' = dY W_down with the SwiGLU backward in the epilogue
+  ga.tab = tab[1];
+  ga.c = nullptr;
+  ga.ab = ab;
+  ga.zg = zg;
+  ga.dab = dab;
+  ga.dgp = dgp;
+  ga.row_w = row_w;
+  rc = launch_gemm_bwd<false, true, gbwd::EPI_SWIGLU_BWD>("backward GEMM dz = dY W_down", DH, DHP,
+                                                           WD, WD, ga, mt_rows * nt(I), sms, st);
+  if (rc != MOE_OK) return rc;
+  // G3: du pieces = [da | db] W_gu, scattered to the token-major slots
+  ga.tab = tab[2];
+  ga.c = dslots;
+  ga.ldc = d;
+  ga.row_pair = row_pair;
+  rc = launch_gemm_bwd<false, true, gbwd::EPI_SCATTER>("backward GEMM du = dAB W_gu", DAB, DAB,
+                                                        WGU, WGU, ga, mt_rows * nt(d), sms, st);
+  if (rc != MOE_OK) return rc;
+  // gate-weight and affinity backward -> dl [T, N]
+  {
+    const route::Params p = route_params(s);
+    if (N <= 32) rc = launch_gate_bwd<1>(logits, p, idx, slot_of, offsets, poff, dgp, B.n_it, dl, st);
+    else if (N <= 64) rc = launch_gate_bwd<2>(logits, p, idx, slot_of, offsets, poff, dgp, B.n_it, dl, st);
+    else if (N <= 128) rc = launch_gate_bwd<4>(logits, p, idx, slot_of, offsets, poff, dgp, B.n_it, dl, st);
+    else if (N <= 256) rc = launch_gate_bwd<8>(logits, p, idx, slot_of, offsets, poff, dgp, B.n_it, dl, st);
+    else rc = launch_gate_bwd<16>(logits, p, idx, slot_of, offsets, poff, dgp, B.n_it, dl, st);
+    if (rc != MOE_OK) return rc;
+  }
+  // G6a: the router's part of dx, dx_router = dl W_r
+  ga.n_probs = 1;
+  ga.tab = tab[5];
+  ga.c = dxr;
+  ga.ldc = d;
+  rc = launch_gemm_bwd<false, true, gbwd::EPI_BF16>("backward GEMM dx_router = dL W_r", DL, DL,
+                                                     WR, WR, ga, nt(d) * ((T + 127) / 128), sms,
+                                                     st);
+  if (rc != MOE_OK) return rc;
+  // dx = dx_router + sum over the token's expert slots, fp32, fixed order
+  rc = do_combine(D, dxr, dslots, dx, st);
+  if (rc != MOE_OK) return rc;
+  // G4: dW_down = dY^T (g z) over each expert's rows
+  ga.n_probs = E;
+  ga.tab = tab[3];
+  ga.c = dw_down;
+  ga.ldc = I;
+  rc = launch_gemm_bwd<true, true, gbwd::EPI_F32>("backward GEMM dW_down = dY^T Z", DH, DHP, ZG,
+                                                   ZG, ga, (int64_t)E * ((d + 127) / 128) * nt(I),
+                                                   sms, st);
+  if (rc != MOE_OK) return rc;
+  // G5: dW_gu = [da | db]^T X over each expert's rows
+  ga.tab = tab[4];
+  ga.c = dw_gu;
+  ga.ldc = d;
+  rc = launch_gemm_bwd<true, true, gbwd::EPI_F32>("backward GEMM dW_gu = dAB^T X", DAB, DAB, X,
+                                                   XP, ga,
+                                                   (int64_t)E * ((2 * I + 127) / 128) * nt(d),
+                                                   sms, st);
+  if (rc != MOE_OK) return rc;
+  // G6b: dW_r = dl^T X over all tokens
+  ga.n_probs = 1;
+  ga.tab = tab[6];
+  ga.c = dw_router;
+  ga.ldc = d;
+  return launch_gemm_bwd<true, true, gbwd::EPI_F32>("backward GEMM dW_r = dL^T X", DL, DL, X, X,
+                                                     ga, ((N + 127) / 128) * nt(d), sms, st);
 }
 
 __global__ void k_selftest_wait(uint64_t limit_ns) {
@@ -742,19 +1112,26 @@ moe_status moe_permute(const moe_layer_desc* desc, const void* x, const int32_t*
   if (rc != MOE_OK) return rc;
   if (!offsets || !aligned16(offsets)) return MOE_ERR_INVALID_ARG;
   if (D.T > 0) {
-    if (!x || !topk_idx || !counts || !perm_src || !slot_of || !x_perm || !aligned16(x) ||
-        !aligned16(topk_idx) || !aligned16(perm_src) || !aligned16(slot_of) ||
-        !aligned16(x_perm))
-      return MOE_ERR_INVALID_ARG;
-    if (D.fp8 != (x_perm_scale != nullptr)) return MOE_ERR_INVALID_ARG;
-    if (x_perm_scale && !aligned16(x_perm_scale)) return MOE_ERR_INVALID_ARG;
+    if (!x_perm && !x_perm_scale) {
+      // maps only: x is not read
+      if (!topk_idx || !counts || !perm_src || !slot_of || !aligned16(topk_idx) ||
+          !aligned16(perm_src) || !aligned16(slot_of))
+        return MOE_ERR_INVALID_ARG;
+    } else {
+      if (!x || !topk_idx || !counts || !perm_src || !slot_of || !x_perm || !aligned16(x) ||
+          !aligned16(topk_idx) || !aligned16(perm_src) || !aligned16(slot_of) ||
+          !aligned16(x_perm))
+        return MOE_ERR_INVALID_ARG;
+      if (D.fp8 != (x_perm_scale != nullptr)) return MOE_ERR_INVALID_ARG;
+      if (x_perm_scale && !aligned16(x_perm_scale)) return MOE_ERR_INVALID_ARG;
+    }
   }
   const Layout L = layout(D);
   if (!ws || ws_bytes < L.total || !aligned16(ws)) return MOE_ERR_WORKSPACE;
   int sms;
   if ((rc = device_setup(&sms)) != MOE_OK) return rc;
-  return do_permute(D, L, x, topk_idx, counts, offsets, perm_src, slot_of, x_perm, x_perm_scale,
-                    static_cast<uint8_t*>(ws), stream);
+  return do_permute(D, reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + L.hist), x,
+                    topk_idx, counts, offsets, perm_src, slot_of, x_perm, x_perm_scale, stream);
 }
 
 moe_status moe_grouped_swiglu(const moe_layer_desc* desc, const void* x, const void* x_perm,
@@ -826,17 +1203,22 @@ moe_status moe_forward(const moe_layer_desc* desc, const void* x, const void* x_
   float* x_perm_scale = D.fp8 ? reinterpret_cast<float*>(w8 + L.x_perm_scale) : nullptr;
   void* y = w8 + L.y_slots;
   if ((rc = trace(0, stream)) != MOE_OK) return rc;
-  if ((rc = do_route(*desc, D, L, x, w_router, bias, idx, tw, cnt, w8, sms, stream)) != MOE_OK)
+  if ((rc = do_route(*desc, D, L, x, w_router, bias, idx, tw, nullptr, w8, sms, stream)) !=
+      MOE_OK)
     return rc;
   if ((rc = trace(1, stream)) != MOE_OK) return rc;
-  if ((rc = do_permute(D, L, x, idx, cnt, offsets, perm_src, slot_of, x_perm, x_perm_scale, w8,
-                       stream)) != MOE_OK)
+  // the permutation's histogram totals are the expert counts
+  if ((rc = do_permute(D, reinterpret_cast<int32_t*>(w8 + L.hist), x, idx, nullptr, offsets,
+                       perm_src, slot_of, x_perm, x_perm_scale, stream, cnt)) != MOE_OK)
     return rc;
+  const void* x_res = x_residual ? x_residual : x;
+  const bool fuse = fusable(D);
   if ((rc = do_grouped(D, L, x, x_perm, x_perm_scale, offsets, slot_of, tw, w_gu, w_gu_scale,
-                       w_down, w_down_scale, y, w8, sms,
-                       stream)) != MOE_OK)
+                       w_down, w_down_scale, y, w8, sms, stream, fuse ? x_res : nullptr,
+                       fuse ? h : nullptr)) != MOE_OK)
     return rc;
-  rc = do_combine(D, x_residual ? x_residual : x, y, h, stream);
+  // bf16: the down projection has added the residual and written h
+  if (!fuse || D.T == 0) rc = do_combine(D, x_res, y, h, stream);
   if (rc == MOE_OK) rc = trace(5, stream);
   return rc;
 }
@@ -950,8 +1332,10 @@ int32_t moe_forward_launch_count(const moe_layer_desc* desc) {
   Dims D;
   if (fill_dims(desc, &D) != MOE_OK) return 0;
   if (D.T == 0) return 2;
-  // route (2) + permute (4) + grouped (3) + combine (1)
-  return 10;
+  // route (router GEMM + top-K; fp32: one kernel) + permute (4) + grouped (3)
+  // + combine (1); bf16 layers add the residual in the down projection and
+  // launch no combine
+  return (D.f32 ? 1 : 2) + 4 + 3 + (fusable(D) ? 0 : 1);
 }
 
 moe_status moe_selftest_bounded_wait(uint32_t limit_us, cudaStream_t stream) {
@@ -988,26 +1372,130 @@ moe_status moe_permute_noalloc(const moe_layer_desc* desc, const void* x,
   if ((rc = device_setup(&sms)) != MOE_OK) return rc;
   int32_t* hist = nullptr;
   if ((rc = noalloc_scratch(&hist)) != MOE_OK) return rc;
-  const int T = (int)D.T, K = (int)D.K, N = (int)D.N;
-  if (T == 0) {
-    route::k_zero_i32<<<1, 256, 0, stream>>>(offsets, N + 1);
-    return launched("k_zero_i32");
+  // The same launch chain as moe_permute.  Every histogram entry the scan
+  // reads is written first by k_hist, so the previous call's contents never
+  // leak into this one.
+  return do_permute(D, hist, x, topk_idx, counts, offsets, perm_src, slot_of, x_perm,
+                    x_perm_scale, stream);
+}
+
+size_t moe_backward_workspace_size(const moe_layer_desc* desc) {
+  Dims D;
+  if (fill_dims(desc, &D) != MOE_OK) return 0;
+  if (D.act != MOE_DT_BF16 || D.w != MOE_DT_BF16) return 0;
+  const Layout L = layout(D);
+  return bwd_layout(D, L).total;
+}
+
+moe_status moe_backward(const moe_layer_desc* desc, const void* x, const void* w_router,
+                        const float* bias, const void* w_gu, const void* w_down, const void* dh,
+                        void* dx, float* dw_router, float* dw_gu, float* dw_down, void* ws,
+                        size_t ws_bytes, cudaStream_t stream) {
+  Dims D;
+  moe_status rc = fill_dims(desc, &D);
+  if (rc != MOE_OK) return rc;
+  if (D.act != MOE_DT_BF16 || D.w != MOE_DT_BF16) return MOE_ERR_UNSUPPORTED;
+  if (bias && desc->gate != MOE_GATE_SIGMOID) return MOE_ERR_INVALID_ARG;
+  if (D.E > 1024) return MOE_ERR_UNSUPPORTED;
+  if (D.T > 0) {
+    if (!x || !w_router || !w_gu || !w_down || !dh || !dx || !dw_router || !dw_gu || !dw_down ||
+        !aligned16(x) || !aligned16(w_router) || !aligned16(w_gu) || !aligned16(w_down) ||
+        !aligned16(dh) || !aligned16(dx) || !aligned16(dw_router) || !aligned16(dw_gu) ||
+        !aligned16(dw_down) || (bias && !aligned16(bias)))
+      return MOE_ERR_INVALID_ARG;
+    if ((D.N * 2) % 16) return MOE_ERR_UNSUPPORTED;   // rows of dl must be 16-byte aligned
   }
-  // Every histogram entry the scan reads is written first by k_hist, so the
-  // previous call's contents never leak into this one.
-  perm::k_hist<<<D.n_chunks, 256, N * 4, stream>>>(topk_idx, T, K, N, hist);
-  perm::k_scan<<<1, 1024, 0, stream>>>(hist, D.n_chunks, N, counts, offsets);
-  perm::k_slots<<<D.n_chunks, perm::SLOT_WARPS * 32, perm::SLOT_WARPS * N * 4, stream>>>(topk_idx, T, K, N, hist, slot_of, perm_src);
-  if (D.fp8) {
-    perm::k_gather_quant<<<(T + 7) / 8, 256, 0, stream>>>(
-        static_cast<const __nv_bfloat16*>(x), T, K, (int)D.d, (int)D.R, slot_of,
-        static_cast<uint8_t*>(x_perm), x_perm_scale);
-  } else {
-    perm::k_gather<<<(T + 7) / 8, 256, 0, stream>>>(static_cast<const uint8_t*>(x), T, K,
-                                                    (int)(D.d * D.x_esz), slot_of,
-                                                    static_cast<uint8_t*>(x_perm));
-  }
-  return launched("permutation kernels (no-alloc)");
+  const Layout L = layout(D);
+  const BwdLayout B = bwd_layout(D, L);
+  if (!ws || ws_bytes < B.total || !aligned16(ws)) return MOE_ERR_WORKSPACE;
+  if (B.rows >= ((int64_t)1 << 31)) return MOE_ERR_INVALID_ARG;
+  if (D.T == 0) return MOE_OK;
+  int sms;
+  if ((rc = device_setup(&sms)) != MOE_OK) return rc;
+  return do_backward(*desc, D, L, B, x, w_router, bias, w_gu, w_down, dh, dx, dw_router, dw_gu,
+                     dw_down, static_cast<uint8_t*>(ws), sms, stream);
+}
+
+int32_t moe_backward_launch_count(const moe_layer_desc* desc) {
+  Dims D;
+  if (fill_dims(desc, &D) != MOE_OK) return 0;
+  if (D.T == 0) return 0;
+  // route (2) + hist, scan, slots (3) + prep, gather, zero pads (3) + six GEMMs on the
+  // rows and experts + gate backward + combine + the router-weight GEMM
+  return 2 + 3 + 3 + 5 + 1 + 1 + 1;
+}
+
+size_t moe_expert_ffn_workspace_size(const moe_layer_desc* desc, int32_t n_groups,
+                                     int32_t n_rows_out) {
+  Dims D;
+  if (fill_dims(desc, &D) != MOE_OK || D.fp8 || n_groups < 1 || n_rows_out < 0) return 0;
+  return ffn_layout(D, n_groups, n_rows_out).total;
+}
+
+moe_status moe_expert_ffn(const moe_layer_desc* desc, int32_t n_experts, int32_t n_groups,
+                          const int32_t* groups, int32_t n_rows_in, int32_t n_rows_out,
+                          const void* x_rows, const float* row_w, const void* w_gu,
+                          const void* w_down, void* y_rows, void* ws, size_t ws_bytes,
+                          cudaStream_t stream) {
+  Dims D;
+  moe_status rc = fill_dims(desc, &D);
+  if (rc != MOE_OK) return rc;
+  if (D.fp8) return MOE_ERR_UNSUPPORTED;
+  if (n_experts < 1 || n_groups < 1 || n_groups > 1024 || n_rows_in < 0 || n_rows_out < 0)
+    return MOE_ERR_INVALID_ARG;
+  if (!groups || !aligned16(groups) || !w_gu || !w_down || !aligned16(w_gu) ||
+      !aligned16(w_down))
+    return MOE_ERR_INVALID_ARG;
+  if (n_rows_out > 0 && (!y_rows || !aligned16(y_rows))) return MOE_ERR_INVALID_ARG;
+  if (n_rows_in > 0 && (!x_rows || !aligned16(x_rows))) return MOE_ERR_INVALID_ARG;
+  const FfnLayout F = ffn_layout(D, n_groups, n_rows_out);
+  if (!ws || ws_bytes < F.total || !aligned16(ws)) return MOE_ERR_WORKSPACE;
+  if (n_rows_out == 0 || n_rows_in == 0) return MOE_OK;
+  int sms;
+  if ((rc = device_setup(&sms)) != MOE_OK) return rc;
+  return do_expert_ffn(D, n_experts, n_groups, groups, n_rows_in, n_rows_out, x_rows, row_w, w_gu,
+                       w_down, y_rows, static_cast<uint8_t*>(ws), sms, stream);
+}
+
+moe_status moe_combine_rows(const moe_layer_desc* desc, const void* x_residual,
+                            const void* y_shared, const void* y_rows, const int32_t* row_of,
+                            int32_t n_rows, void* h, cudaStream_t stream) {
+  Dims D;
+  moe_status rc = fill_dims(desc, &D);
+  if (rc != MOE_OK) return rc;
+  if (n_rows < 0) return MOE_ERR_INVALID_ARG;
+  if (D.T == 0) return MOE_OK;
+  if (!x_residual || !h || !row_of || !aligned16(x_residual) || !aligned16(h) ||
+      (D.Ks > 0 && (!y_shared || !aligned16(y_shared))) ||
+      (n_rows > 0 && (!y_rows || !aligned16(y_rows))))
+    return MOE_ERR_INVALID_ARG;
+  const int vec = D.f32 ? 4 : 8;
+  const int64_t threads = D.T * (D.d / vec);
+  const int blocks = (int)((threads + 255) / 256);
+  if (D.f32)
+    return launch_chain("k_combine_rows", perm::k_combine_rows<false>, dim3(blocks), dim3(256), 0,
+                        stream, x_residual, y_shared, y_rows, row_of, (int)n_rows, h, (int)D.T,
+                        (int)D.d, (int)D.K, (int)D.Ks);
+  return launch_chain("k_combine_rows", perm::k_combine_rows<true>, dim3(blocks), dim3(256), 0,
+                      stream, x_residual, y_shared, y_rows, row_of, (int)n_rows, h, (int)D.T,
+                      (int)D.d, (int)D.K, (int)D.Ks);
+}
+
+moe_status moe_dispatch_rows(const moe_layer_desc* desc, const void* x, const float* topk_w,
+                             const int32_t* row_of, int32_t n_rows, void* x_rows, float* w_rows,
+                             cudaStream_t stream) {
+  Dims D;
+  moe_status rc = fill_dims(desc, &D);
+  if (rc != MOE_OK) return rc;
+  if (D.fp8) return MOE_ERR_UNSUPPORTED;
+  if (n_rows < 0) return MOE_ERR_INVALID_ARG;
+  if (D.T == 0) return MOE_OK;
+  if (!x || !row_of || !x_rows || !aligned16(x) || !aligned16(x_rows) || (w_rows && !topk_w))
+    return MOE_ERR_INVALID_ARG;
+  return launch_chain("k_dispatch_rows", perm::k_dispatch_rows, dim3((unsigned)((D.T + 7) / 8)),
+                      dim3(256), 0, stream, static_cast<const uint8_t*>(x), (int)D.T, (int)D.K,
+                      (int)(D.d * D.x_esz), topk_w, row_of, (int)n_rows,
+                      static_cast<uint8_t*>(x_rows), w_rows);
 }
 
 }  // extern "C"

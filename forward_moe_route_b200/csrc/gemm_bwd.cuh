@@ -1,0 +1,417 @@
+// Grouped GEMM of the layer backward: C_g = A_g B_g^T for a device-built list
+// of problems, on tcgen05 / TMEM (one CTA per SM, 128 x 256 tiles, the fp32
+// accumulator kept in TMEM over the whole K loop), fed by TMA.
+//
+// Every backward GEMM contracts over an index that is the row index of one of
+// its operands in memory: the hidden size d of W_down [d, I] (dz = dY W_down),
+// the 2I rows of W_gu [2I, d] (du = [da | db] W_gu), and the expert's token
+// rows for the weight gradients (dW_down = dY^T Z, dW_gu = [dA | dB]^T X).
+// Instead of transposing those tensors in memory, an operand can be read
+// "MN-major": the tile is loaded as 64-element (128-byte) slices of its M (or
+// N) extent, one K row per 128-byte line with the 128-byte swizzle, and the
+// UMMA instruction descriptor marks the operand as MN-major.  In the
+// descriptor of such a tile, 8 K rows form a 1 KB core group (stride byte
+// offset 1024) and consecutive 64-element slices are one TMA box apart
+// (leading byte offset 64 rows x 128 bytes = 8 KB); one UMMA of K = 16 then
+// starts 16 rows (2 KB) further on.  K-major operands use the same layout as
+// the forward GEMMs.
+//
+// Problem table (int32, GB_FIELDS per problem), built on the device:
+//   m, n, k            sizes (k may be 0: the tile is written as zeros)
+//   a_map, a_m0, a_k0  which A tensor map and the problem's origin in it
+//   b_map, b_n0, b_k0  the same for B
+//   c_row0             first output row of the problem
+//   m_pad              rows in [m, m_pad) of the output are written as zeros
+//                      (row-store epilogues; the zero rows are the K padding
+//                      of the weight-gradient GEMMs that read them later)
+//   aux                epilogue-specific (shared-expert index or -1)
+// Tiles: ceil(m/128) x ceil(n/256) per problem, N fastest, problems in order,
+// strided over the persistent CTAs.
+//
+// Warp roles (256 threads): warp 0 TMA producer, warp 1 MMA issuer, warp 2
+// TMEM allocator, warps 4..7 epilogue (warp w reads TMEM lanes 32(w-4)..+31,
+// one output row per thread).  Two accumulators of 256 columns.  Every wait
+// is bounded (see common.cuh).
+#pragma once
+
+#include "common.cuh"
+#include "gemm.cuh"
+
+namespace moe {
+namespace gbwd {
+
+constexpr int BM = 128;
+constexpr int BN = 256;
+constexpr int BK = 64;                 // bf16 elements per k-block (128 bytes)
+constexpr int NUM_THREADS = 256;
+constexpr int EPI_WARP0 = 4;
+constexpr int ACC_COLS = 256;
+constexpr int TMEM_COLS = 512;
+constexpr int GB_FIELDS = 13;
+constexpr uint32_t A_BYTES = BM * 128;
+constexpr uint32_t B_BYTES = BN * 128;
+constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr uint32_t MN_BOX_BYTES = 64 * 128;   // one MN-major box: 64 K rows x 128 bytes
+
+enum Epi {
+  EPI_F32 = 0,          // C fp32 row-major (weight gradients)
+  EPI_BF16 = 1,         // C bf16 row-major, rows [m, m_pad) zeroed
+  EPI_SWIGLU_BWD = 2,   // dz' tile -> zg, [da | db], per-row <dz', z> partials
+  EPI_SCATTER = 3       // bf16 rows to the token-major slots [T, K+Ks, d]
+};
+
+enum Field { F_M = 0, F_N, F_K, F_AMAP, F_AM0, F_AK0, F_BMAP, F_BN0, F_BK0, F_CROW, F_MPAD, F_AUX,
+             F_SPARE };
+
+struct Args {
+  const int* tab;          // [n_probs][GB_FIELDS]
+  int n_probs;
+  int stages;
+  void* c;                 // EPI_F32 / EPI_BF16 / EPI_SCATTER output
+  long long ldc;           // elements per output row
+  // EPI_SWIGLU_BWD
+  const __nv_bfloat16* ab; // [rows, 2I] pre-activations a | b
+  __nv_bfloat16* zg;       // [rows, I]  g * SiLU(a) * b
+  __nv_bfloat16* dab;      // [rows, 2I] da | db
+  float* dgp;              // [rows, I / 256] partial <dz', z>
+  const float* row_w;      // [rows] gate weight of each padded row (routed problems)
+  int inter;
+  // EPI_SCATTER
+  const int* row_pair;     // [rows] pair index t*K + k of each padded routed row (-1: pad)
+  int K, Ks;
+};
+
+__host__ inline size_t smem_bytes(int stages, int n_probs) {
+  return 1024 + (size_t)stages * STAGE_BYTES + (size_t)(2 * stages + 5) * 8 + 16 +
+         (size_t)(n_probs + 1) * 4 + 64;
+}
+
+// UMMA descriptor of an MN-major operand tile loaded as 64-element boxes of
+// 64 K rows each, 128-byte swizzle: core groups of 8 K rows (1 KB), boxes
+// 8 KB apart along M / N.
+__device__ __forceinline__ uint64_t umma_desc_sw128_mn(uint32_t smem_addr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((smem_addr & 0x3FFFF) >> 4);
+  d |= (uint64_t)(MN_BOX_BYTES >> 4) << 16;            // leading byte offset: next 64-element slice
+  d |= (uint64_t)(1024 >> 4) << 32;                    // stride byte offset: next 8 K rows
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)2 << 61;
+  return d;
+}
+
+template <bool A_MN, bool B_MN, int EPI>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    k_gemm_bwd(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
+               const __grid_constant__ CUtensorMap tmB0, const __grid_constant__ CUtensorMap tmB1,
+               const Args a) {
+  grid_dep_sync();
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const int S = a.stages;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)S * STAGE_BYTES);
+  uint64_t* empty = full + S;
+  uint64_t* tfull = empty + S;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* s_prefix = reinterpret_cast<int*>(tmem_slot + 4);
+
+  const int warp = warp_id(), lane = lane_id();
+  const int np = a.n_probs;
+  if (warp == 0) {
+    int carry = 0;
+    for (int base = 0; base < np; base += 32) {
+      const int g = base + lane;
+      int v = 0;
+      if (g < np) {
+        const int* p = a.tab + (size_t)g * GB_FIELDS;
+        v = ((p[F_M] + BM - 1) / BM) * ((p[F_N] + BN - 1) / BN);
+      }
+      int incl = v;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      if (g < np) s_prefix[g] = carry + incl - v;
+      carry += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) s_prefix[np] = carry;
+  }
+  if (threadIdx.x == 32) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int j = 0; j < 2; ++j) {
+      mbar_init(&tfull[j], 1);
+      mbar_init(&tempty[j], 4 * 32);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    fence_proxy_async_smem();
+    tma_prefetch_desc(&tmA0);
+    tma_prefetch_desc(&tmA1);
+    tma_prefetch_desc(&tmB0);
+    tma_prefetch_desc(&tmB1);
+  }
+  if (warp == 2) {
+    tmem_alloc(tmem_slot, TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int total = s_prefix[np];
+
+  // tile -> (problem, m tile, n tile)
+  auto locate = [&](int tile, int& g, int& mt, int& nt, const int*& p) {
+    g = gemm::find_group(s_prefix, np, tile);
+    p = a.tab + (size_t)g * GB_FIELDS;
+    const int ntn = (p[F_N] + BN - 1) / BN;
+    const int lt = tile - s_prefix[g];
+    mt = lt / ntn;
+    nt = lt - mt * ntn;
+  };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ TMA producer
+    if (elect_one()) {
+      int it = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+        int g, mt, nt;
+        const int* p;
+        locate(tile, g, mt, nt, p);
+        const int nkb = (p[F_K] + BK - 1) / BK;
+        const CUtensorMap* tA = p[F_AMAP] ? &tmA1 : &tmA0;
+        const CUtensorMap* tB = p[F_BMAP] ? &tmB1 : &tmB0;
+        const int am = p[F_AM0] + mt * BM, ak = p[F_AK0];
+        const int bn = p[F_BN0] + nt * BN, bk = p[F_BK0];
+        for (int kb = 0; kb < nkb; ++kb, ++it) {
+          const int s = it % S;
+          const uint32_t ph = (uint32_t)(it / S) & 1u;
+          if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag)) { ok = false; break; }
+          uint8_t* sa = smem + (size_t)s * STAGE_BYTES;
+          uint8_t* sb = sa + A_BYTES;
+          mbar_arrive_expect_tx(&full[s], STAGE_BYTES);
+          const int k0 = kb * BK;
+          if (A_MN) {
+            tma_load_2d(tA, &full[s], sa, am, ak + k0);
+            tma_load_2d(tA, &full[s], sa + MN_BOX_BYTES, am + 64, ak + k0);
+          } else {
+            tma_load_2d(tA, &full[s], sa, ak + k0, am);
+          }
+          if (B_MN) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              tma_load_2d(tB, &full[s], sb + j * MN_BOX_BYTES, bn + 64 * j, bk + k0);
+          } else {
+            tma_load_2d(tB, &full[s], sb, bk + k0, bn);
+          }
+        }
+      }
+      // the copies this CTA issued land before the block may leave (bounded)
+      volatile int no_abort = 0;
+      for (int j = (it - S > 0 ? it - S : 0); j < it; ++j)
+        mbar_wait(&full[j % S], (uint32_t)(j / S) & 1u, &no_abort);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (elect_one()) {
+      int it = 0, tcount = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x, ++tcount) {
+        int g, mt, nt;
+        const int* p;
+        locate(tile, g, mt, nt, p);
+        const int nkb = (p[F_K] + BK - 1) / BK;
+        int ncols = min(BN, p[F_N] - nt * BN);
+        ncols = (ncols + 15) & ~15;
+        const uint32_t idesc = umma_idesc(1, BM, ncols) | (A_MN ? (1u << 15) : 0u) |
+                               (B_MN ? (1u << 16) : 0u);
+        const int acc = tcount & 1;
+        const uint32_t use = (uint32_t)(tcount >> 1);
+        if (!mbar_wait(&tempty[acc], (use & 1u) ^ 1u, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * ACC_COLS);
+        for (int kb = 0; kb < nkb; ++kb, ++it) {
+          const int s = it % S;
+          const uint32_t ph = (uint32_t)(it / S) & 1u;
+          if (!mbar_wait(&full[s], ph, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + (size_t)s * STAGE_BYTES);
+          const uint64_t ad = A_MN ? umma_desc_sw128_mn(sa) : umma_desc_sw128(sa);
+          const uint64_t bd = B_MN ? umma_desc_sw128_mn(sa + A_BYTES) : umma_desc_sw128(sa + A_BYTES);
+          // one UMMA per 16 elements of K: 32 bytes further along a K-major
+          // line, 16 rows (2 KB) further down an MN-major tile
+          constexpr uint64_t a_step = A_MN ? (2048 >> 4) : (32 >> 4);
+          constexpr uint64_t b_step = B_MN ? (2048 >> 4) : (32 >> 4);
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k)
+            umma<0>(d_tmem, ad + a_step * k, bd + b_step * k, idesc, (kb | k) != 0 ? 1u : 0u);
+          umma_commit(&empty[s]);
+        }
+        if (ok) umma_commit(&tfull[acc]);
+      }
+      umma_commit(drain);
+      volatile int no_abort = 0;
+      mbar_wait(drain, 0, &no_abort);
+    }
+    __syncwarp();
+  } else if (warp >= EPI_WARP0) {
+    // ------------------------------------------------------------------ epilogue
+    const int q = warp - EPI_WARP0;            // TMEM lane quadrant
+    const int r_local = q * 32 + lane;         // this thread's row of the tile
+    int tcount = 0;
+    for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++tcount) {
+      int g, mt, nt;
+      const int* p;
+      locate(tile, g, mt, nt, p);
+      const int acc = tcount & 1;
+      const uint32_t use = (uint32_t)(tcount >> 1);
+      if (!mbar_wait(&tfull[acc], use & 1u, abort_flag)) break;
+      tc_fence_after();
+      const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * ACC_COLS);
+      const int m = p[F_M], n = p[F_N], mpad = p[F_MPAD];
+      const int row = mt * BM + r_local;                  // row within the problem
+      const bool has_k = p[F_K] > 0;
+      const long long crow = (long long)p[F_CROW] + row;
+      const int col0 = nt * BN;
+      const int ncol = min(BN, n - col0);
+      const bool valid = row < m;
+      const bool zero_row = !valid && row < mpad;
+      if (EPI == EPI_F32) {
+        float* out = reinterpret_cast<float*>(a.c) + crow * a.ldc + col0;
+#pragma unroll 1
+        for (int c = 0; c < BN / 16; ++c) {
+          float v[16];
+          tmem_ld16(tb + (uint32_t)(16 * c), v);
+          if (valid && 16 * c < ncol) {
+            if (!has_k) {
+#pragma unroll
+              for (int j = 0; j < 16; ++j) v[j] = 0.f;
+            }
+            if (16 * c + 16 <= ncol) {
+#pragma unroll
+              for (int j = 0; j < 4; ++j)
+                reinterpret_cast<float4*>(out + 16 * c)[j] =
+                    make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+            } else {
+#pragma unroll
+              for (int j = 0; j < 16; ++j)
+                if (16 * c + j < ncol) out[16 * c + j] = v[j];
+            }
+          }
+        }
+      } else if (EPI == EPI_BF16 || EPI == EPI_SCATTER) {
+        long long dst_row = crow;
+        if (EPI == EPI_SCATTER && valid) {
+          const int s_idx = p[F_AUX];
+          if (s_idx < 0) {
+            const int pr = a.row_pair[crow];
+            dst_row = pr < 0 ? -1 : (long long)(pr / a.K) * (a.K + a.Ks) + pr % a.K;
+          } else {
+            dst_row = (long long)row * (a.K + a.Ks) + a.K + s_idx;
+          }
+        }
+        const bool write = EPI == EPI_SCATTER ? (valid && dst_row >= 0) : (valid || zero_row);
+        __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(a.c) + dst_row * a.ldc + col0;
+#pragma unroll 1
+        for (int c = 0; c < BN / 16; ++c) {
+          float v[16];
+          tmem_ld16(tb + (uint32_t)(16 * c), v);
+          if (write && 16 * c < ncol) {
+            const bool z = !valid || !has_k;
+            uint32_t w[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              w[j] = z ? 0u : gemm::pack_bf16x2(v[2 * j], v[2 * j + 1]);
+            if (16 * c + 16 <= ncol) {
+              reinterpret_cast<uint4*>(out + 16 * c)[0] = make_uint4(w[0], w[1], w[2], w[3]);
+              reinterpret_cast<uint4*>(out + 16 * c)[1] = make_uint4(w[4], w[5], w[6], w[7]);
+            } else {
+#pragma unroll
+              for (int j = 0; j < 16; ++j)
+                if (16 * c + j < ncol) out[16 * c + j] = __float2bfloat16_rn(z ? 0.f : v[j]);
+            }
+          }
+        }
+      } else {
+        // EPI_SWIGLU_BWD: the tile holds dz' = dY W_down (unscaled) for 256
+        // features of each row.  With a, b the forward pre-activations and g
+        // the row's gate weight (1 for shared experts):
+        //   z = SiLU(a) b,  zg = g z,  dz = g dz',
+        //   da = dz b SiLU'(a),  db = dz SiLU(a),  dg partial = sum dz' z.
+        const int I = a.inter;
+        const float gw = (p[F_AUX] < 0 && valid) ? a.row_w[crow] : 1.0f;
+        const __nv_bfloat16* abr = a.ab + crow * 2 * I + col0;
+        __nv_bfloat16* zr = a.zg + crow * I + col0;
+        __nv_bfloat16* dar = a.dab + crow * 2 * I + col0;
+        float dgs = 0.f;
+#pragma unroll 1
+        for (int c = 0; c < BN / 16; ++c) {
+          float v[16];
+          tmem_ld16(tb + (uint32_t)(16 * c), v);
+          if ((valid || zero_row) && 16 * c < ncol) {
+            uint32_t wz[8], wa[8], wb[8];
+            if (valid && has_k) {
+              const uint4* pa = reinterpret_cast<const uint4*>(abr + 16 * c);
+              const uint4* pb = reinterpret_cast<const uint4*>(abr + I + 16 * c);
+              uint4 ra[2] = {pa[0], pa[1]}, rb[2] = {pb[0], pb[1]};
+              const __nv_bfloat162* ha = reinterpret_cast<const __nv_bfloat162*>(ra);
+              const __nv_bfloat162* hb = reinterpret_cast<const __nv_bfloat162*>(rb);
+#pragma unroll
+              for (int j = 0; j < 8; ++j) {
+                float zz[2], da2[2], db2[2];
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                  const float av = h ? __high2float(ha[j]) : __low2float(ha[j]);
+                  const float bv = h ? __high2float(hb[j]) : __low2float(hb[j]);
+                  const float sg = 1.0f / (1.0f + __expf(-av));
+                  const float si = av * sg;
+                  const float z = si * bv;
+                  const float dzp = v[2 * j + h];
+                  const float dz = gw * dzp;
+                  dgs = fmaf(dzp, z, dgs);
+                  zz[h] = gw * z;
+                  da2[h] = dz * bv * (sg * (1.0f + av * (1.0f - sg)));
+                  db2[h] = dz * si;
+                }
+                wz[j] = gemm::pack_bf16x2(zz[0], zz[1]);
+                wa[j] = gemm::pack_bf16x2(da2[0], da2[1]);
+                wb[j] = gemm::pack_bf16x2(db2[0], db2[1]);
+              }
+            } else {
+#pragma unroll
+              for (int j = 0; j < 8; ++j) wz[j] = wa[j] = wb[j] = 0u;
+            }
+            reinterpret_cast<uint4*>(zr + 16 * c)[0] = make_uint4(wz[0], wz[1], wz[2], wz[3]);
+            reinterpret_cast<uint4*>(zr + 16 * c)[1] = make_uint4(wz[4], wz[5], wz[6], wz[7]);
+            reinterpret_cast<uint4*>(dar + 16 * c)[0] = make_uint4(wa[0], wa[1], wa[2], wa[3]);
+            reinterpret_cast<uint4*>(dar + 16 * c)[1] = make_uint4(wa[4], wa[5], wa[6], wa[7]);
+            reinterpret_cast<uint4*>(dar + I + 16 * c)[0] = make_uint4(wb[0], wb[1], wb[2], wb[3]);
+            reinterpret_cast<uint4*>(dar + I + 16 * c)[1] = make_uint4(wb[4], wb[5], wb[6], wb[7]);
+          }
+        }
+        if (valid || zero_row) a.dgp[crow * ((I + BN - 1) / BN) + nt] = valid ? dgs : 0.f;
+      }
+      tc_fence_before();
+      mbar_arrive(&tempty[acc]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+}  // namespace gbwd
+}  // namespace moe

@@ -37,9 +37,11 @@ __global__ void __launch_bounds__(256) k_hist(const int32_t* __restrict__ idx, i
 
 // One block of 1024 threads.  Turns hist into each chunk's first row per
 // expert (offsets[e] + pairs of expert e in earlier chunks), writes offsets
-// [N+1], and checks the totals against `counts`.
+// [N+1], and checks the per-expert totals against `counts` (when given) or
+// writes them to `counts_out` (when given).
 __global__ void __launch_bounds__(1024) k_scan(int32_t* __restrict__ hist, int n_chunks, int N,
                                                const int32_t* __restrict__ counts,
+                                               int32_t* __restrict__ counts_out,
                                                int32_t* __restrict__ offsets) {
   grid_dep_sync();
   __shared__ int32_t part_sum[1024];
@@ -67,6 +69,7 @@ __global__ void __launch_bounds__(1024) k_scan(int32_t* __restrict__ hist, int n
       for (int q = 0; q < P; ++q) total += part_sum[q * N + e];
       tot[e] = total;
       if (counts && counts[e] != total) set_status(MOE_ERR_DEVICE_CHECK);
+      if (counts_out) counts_out[e] = total;
     }
   }
   __syncthreads();
@@ -237,11 +240,14 @@ __global__ void __launch_bounds__(256) k_gather_quant(const __nv_bfloat16* __res
 
 // Group table for the grouped GEMMs (block 0) and the permuted-row -> pair map
 // (all blocks).  Groups: shared experts 0..Ks-1 then routed experts 0..N-1.
+// With cnt != nullptr the other blocks also zero the n_cnt arrival counters
+// of the down projection's fused residual.
 __global__ void __launch_bounds__(1024) k_prep_groups(const int32_t* __restrict__ offsets, int T,
                                                       int K, int Ks, int N, int fp8,
                                                       int32_t* __restrict__ gtab,
                                                       const int32_t* __restrict__ slot_of,
-                                                      int32_t* __restrict__ pair_of) {
+                                                      int32_t* __restrict__ pair_of,
+                                                      int32_t* __restrict__ cnt, int n_cnt) {
   grid_dep_sync();
   const int R = T * K;
   if (blockIdx.x > 0) {
@@ -251,6 +257,10 @@ __global__ void __launch_bounds__(1024) k_prep_groups(const int32_t* __restrict_
       if ((unsigned)row < (unsigned)R) pair_of[row] = i;
       else set_status(MOE_ERR_DEVICE_CHECK);
     }
+    if (cnt)
+      for (int i = (blockIdx.x - 1) * blockDim.x + threadIdx.x; i < n_cnt;
+           i += (gridDim.x - 1) * blockDim.x)
+        cnt[i] = 0;
     return;
   }
   __shared__ int32_t warp_tot[32];
@@ -358,6 +368,164 @@ __global__ void __launch_bounds__(256) k_combine(const void* __restrict__ x_res,
   for (int k = 0; k < K; ++k) {
     float v[VEC];
     load(y, ybase + (long long)k * d, v);
+#pragma unroll
+    for (int i = 0; i < VEC; ++i) acc[i] += v[i];
+  }
+  if (BF16) {
+    uint4 out;
+    uint32_t* o = reinterpret_cast<uint32_t*>(&out);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) o[i] = gemm::pack_bf16x2(acc[2 * i], acc[2 * i + 1]);
+    *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(h) + (long long)t * d + c) = out;
+  } else {
+    *reinterpret_cast<float4*>(reinterpret_cast<float*>(h) + (long long)t * d + c) =
+        make_float4(acc[0], acc[1], acc[2], acc[3]);
+  }
+}
+
+// Dispatch gather (expert parallelism): x_rows[row_of[t*K + k]] = x[t] and
+// w_rows[row_of[t*K + k]] = topk_w[t*K + k].  One warp per token reads its row
+// once and writes it to its K rows with 16-byte vectors.
+__global__ void __launch_bounds__(256) k_dispatch_rows(const uint8_t* __restrict__ x, int T,
+                                                       int K, int row_bytes,
+                                                       const float* __restrict__ topk_w,
+                                                       const int32_t* __restrict__ row_of,
+                                                       int n_rows, uint8_t* __restrict__ x_rows,
+                                                       float* __restrict__ w_rows) {
+  grid_dep_sync();
+  const int t = blockIdx.x * 8 + warp_id();
+  if (t >= T) return;
+  const int lane = lane_id();
+  int my_row = -1;
+  if (lane < K) {
+    my_row = row_of[(size_t)t * K + lane];
+    if ((unsigned)my_row >= (unsigned)n_rows) {
+      set_status(MOE_ERR_DEVICE_CHECK);
+      my_row = -1;
+    } else if (w_rows) {
+      w_rows[my_row] = topk_w[(size_t)t * K + lane];
+    }
+  }
+  const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * row_bytes);
+  const int nvec = row_bytes / 16;
+  for (int c0 = 0; c0 < nvec; c0 += 32) {
+    const int c = c0 + lane;
+    const bool in = c < nvec;
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (in) v = __ldg(src + c);
+    for (int k = 0; k < K; ++k) {
+      const int row = __shfl_sync(0xffffffffu, my_row, k);
+      if (in && row >= 0) reinterpret_cast<uint4*>(x_rows + (size_t)row * row_bytes)[c] = v;
+    }
+  }
+}
+
+// Group table of a caller-given list of row groups (expert parallelism): group
+// i reads rows [row0, row0 + rows) of x_rows with expert `expert` and writes
+// rows [out0, out0 + rows) of H and of the output.  One block; n <= 1024.
+__global__ void __launch_bounds__(1024) k_prep_user_groups(const int32_t* __restrict__ groups,
+                                                           int n, int n_experts, int n_in,
+                                                           int n_out, int32_t* __restrict__ gtab) {
+  grid_dep_sync();
+  __shared__ int32_t warp_tot[32];
+  int32_t* prefix = gtab;
+  int32_t* rows = gtab + n + 1;
+  int32_t* a_row = rows + n;
+  int32_t* a_map = a_row + n;
+  int32_t* expert = a_map + n;
+  int32_t* c_row = expert + n;
+  int32_t* aux = c_row + n;
+  const int g = threadIdx.x;
+  int mtiles = 0;
+  if (g < n) {
+    const int r0 = groups[4 * g], rw = groups[4 * g + 1], ex = groups[4 * g + 2],
+              o0 = groups[4 * g + 3];
+    const bool ok = rw >= 0 && r0 >= 0 && o0 >= 0 && (long long)r0 + rw <= n_in &&
+                    (long long)o0 + rw <= n_out && ex >= 0 && ex < n_experts;
+    if (!ok) set_status(MOE_ERR_DEVICE_CHECK);
+    rows[g] = ok ? rw : 0;
+    a_row[g] = ok ? r0 : 0;
+    a_map[g] = 1;
+    expert[g] = ok ? ex : 0;
+    c_row[g] = ok ? o0 : 0;
+    aux[g] = -1;
+    mtiles = ok ? (rw + gemm::BM - 1) / gemm::BM : 0;
+  }
+  int incl = mtiles;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane_id() >= o) incl += y;
+  }
+  if (lane_id() == 31) warp_tot[warp_id()] = incl;
+  __syncthreads();
+  if (warp_id() == 0) {
+    const int nw = blockDim.x / 32;
+    const int wv = lane_id() < nw ? warp_tot[lane_id()] : 0;
+    int wi = wv;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, wi, o);
+      if (lane_id() >= o) wi += y;
+    }
+    if (lane_id() < nw) warp_tot[lane_id()] = wi - wv;
+  }
+  __syncthreads();
+  const int excl = incl - mtiles + warp_tot[warp_id()];
+  if (g < n) prefix[g] = excl;
+  if (g == n - 1) prefix[n] = excl + mtiles;
+}
+
+// h[t] = x_res[t] + sum_{s<Ks} y_shared[s*T + t] + sum_{k<K} y_rows[row_of[t*K + k]],
+// fp32, in that order (the order of k_combine, so the two agree bit for bit
+// when the rows hold the same values).  A row index outside [0, n_rows) is
+// reported and skipped.
+template <bool BF16>
+__global__ void __launch_bounds__(256) k_combine_rows(const void* __restrict__ x_res,
+                                                      const void* __restrict__ y_shared,
+                                                      const void* __restrict__ y_rows,
+                                                      const int32_t* __restrict__ row_of,
+                                                      int n_rows, void* __restrict__ h, int T,
+                                                      int d, int K, int Ks) {
+  grid_dep_sync();
+  constexpr int VEC = BF16 ? 8 : 4;
+  const int per_tok = d / VEC;
+  const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (gid >= (long long)T * per_tok) return;
+  const int t = (int)(gid / per_tok);
+  const int c = (int)(gid - (long long)t * per_tok) * VEC;
+  float acc[VEC];
+  auto load = [&](const void* base, long long elem_off, float (&v)[VEC]) {
+    if (BF16) {
+      const uint4 raw = __ldg(reinterpret_cast<const uint4*>(
+          reinterpret_cast<const __nv_bfloat16*>(base) + elem_off));
+      const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+      for (int i = 0; i < VEC / 2; ++i) {
+        v[2 * i] = __low2float(p[i]);
+        v[2 * i + 1] = __high2float(p[i]);
+      }
+    } else {
+      const float4 raw = __ldg(reinterpret_cast<const float4*>(
+          reinterpret_cast<const float*>(base) + elem_off));
+      v[0] = raw.x; v[1] = raw.y; v[2] = raw.z; v[3] = raw.w;
+    }
+  };
+  load(x_res, (long long)t * d + c, acc);
+  for (int s = 0; s < Ks; ++s) {
+    float v[VEC];
+    load(y_shared, ((long long)s * T + t) * d + c, v);
+#pragma unroll
+    for (int i = 0; i < VEC; ++i) acc[i] += v[i];
+  }
+  for (int k = 0; k < K; ++k) {
+    const int r = row_of[(size_t)t * K + k];
+    if ((unsigned)r >= (unsigned)n_rows) {
+      if (c == 0) set_status(MOE_ERR_DEVICE_CHECK);
+      continue;
+    }
+    float v[VEC];
+    load(y_rows, (long long)r * d + c, v);
 #pragma unroll
     for (int i = 0; i < VEC; ++i) acc[i] += v[i];
   }

@@ -1,5 +1,7 @@
 // Gating: affinities, bias-for-selection keys, group limit, top-K and gate
-// weights, one warp per token with shuffle reductions.
+// weights, one warp per token with shuffle reductions.  The expert counts are
+// not taken here: they are the totals of the permutation's per-chunk
+// histogram (k_hist / k_scan), which costs no global atomics.
 //
 // Follows "DeepSeek Technical Report: MoE Architecture": §2.3 (softmax gate
 // over the routed experts, then TopK), §3.3 and equations [3]/[4] of §5.3
@@ -57,13 +59,38 @@ __device__ __forceinline__ void affinity_lane(const float (&l)[VPL], const Param
   }
 }
 
+// Put the better of list positions a < b first: the larger key image, and
+// among equal keys the lower expert (j ascending within a lane).
+template <int VPL>
+__device__ __forceinline__ void cas_pick(uint32_t (&ok)[VPL], int (&jj)[VPL], float (&ss)[VPL],
+                                         int a, int b) {
+  const bool sw = ok[b] > ok[a] || (ok[b] == ok[a] && jj[b] < jj[a]);
+  const uint32_t o0 = ok[a], o1 = ok[b];
+  const int j0 = jj[a], j1 = jj[b];
+  const float s0 = ss[a], s1 = ss[b];
+  ok[a] = sw ? o1 : o0; ok[b] = sw ? o0 : o1;
+  jj[a] = sw ? j1 : j0; jj[b] = sw ? j0 : j1;
+  ss[a] = sw ? s1 : s0; ss[b] = sw ? s0 : s1;
+}
+
 // Route one token given its N logits spread over the warp: lane l holds the
 // logits of experts l*VPL .. l*VPL+VPL-1 (entries with index >= N are ignored).
+//   1. affinities s (softmax or sigmoid) and selection keys s + b;
+//   2. group limit: each group's score is the sum of its two largest keys;
+//      a group is kept when fewer than topk_group groups rank above it
+//      (larger score, or equal score and lower index), and the experts of the
+//      other groups drop out;
+//   3. each lane sorts its eligible experts by (key desc, index asc) into a
+//      list; the K picks then each take the largest list head over the warp
+//      (one redux.sync max on the keys' order-preserving images) and, among
+//      equal keys, the lowest lane -- experts are lane-major, so that is the
+//      lowest index -- and that lane drops its head;
+//   4. weights in pick order: g_k = scale * s_k (/ sum of the picked s when
+//      renorm); lane k writes pick k.
 template <int VPL>
 __device__ __forceinline__ void route_token(const float (&l)[VPL], const float* __restrict__ bias,
                                             const Params& p, int t, int32_t* __restrict__ topk_idx,
-                                            float* __restrict__ topk_w,
-                                            int32_t* __restrict__ counts) {
+                                            float* __restrict__ topk_w) {
   const int lane = lane_id();
   float s[VPL], key[VPL];
   affinity_lane<VPL>(l, p, s);
@@ -72,6 +99,9 @@ __device__ __forceinline__ void route_token(const float (&l)[VPL], const float* 
     const int e = lane * VPL + j;
     key[j] = (e < p.N) ? (bias ? s[j] + bias[e] : s[j]) : -INFINITY;
   }
+  uint32_t ok[VPL];   // order-preserving key images; 0 = not eligible
+#pragma unroll
+  for (int j = 0; j < VPL; ++j) ok[j] = (lane * VPL + j < p.N) ? ord_key(key[j]) : 0u;
 
   if (p.n_group > 1) {
     const int gsz = p.N / p.n_group;
@@ -123,51 +153,44 @@ __device__ __forceinline__ void route_token(const float (&l)[VPL], const float* 
         if (lane == g) my_gscore = b1 + b2;
       }
     }
-    // keep the topk_group best groups (score desc, group asc): the largest
-    // orderable score over the candidate lanes, the lowest such lane
-    uint32_t keep = 0;
-    for (int r = 0; r < p.topk_group; ++r) {
-      const bool cand = lane < p.n_group && !((keep >> lane) & 1u);
-      const uint32_t o = cand ? ord_key(my_gscore) : 0u;
-      const uint32_t mx = __reduce_max_sync(0xffffffffu, o);
-      const uint32_t who = __ballot_sync(0xffffffffu, cand && o == mx);
-      if (who) keep |= 1u << (__ffs(who) - 1);
+    // rank of each group: groups with a larger score, or an equal score and a
+    // lower index, come first; the topk_group first groups are kept
+    int rank = 0;
+    for (int g = 0; g < p.n_group; ++g) {
+      const float o = __shfl_sync(0xffffffffu, my_gscore, g);
+      rank += (o > my_gscore || (o == my_gscore && g < lane)) ? 1 : 0;
     }
+    const uint32_t keep = __ballot_sync(0xffffffffu, lane < p.n_group && rank < p.topk_group);
 #pragma unroll
     for (int j = 0; j < VPL; ++j) {
       const int e = lane * VPL + j;
-      if (e < p.N && !((keep >> (e / gsz)) & 1u)) key[j] = -INFINITY;
+      if (e < p.N && !((keep >> (e / gsz)) & 1u)) ok[j] = 0u;
     }
   }
 
-  // top-K by (key desc, index asc), one pick per round: each lane offers its
-  // best untaken expert (lowest index among equal keys), the warp takes the
-  // largest key and, among equal keys, the lowest lane (experts are
-  // lane-major, so that is the lowest index).  Lane k keeps pick k; the
-  // weight denominator is summed in pick order.
-  uint32_t taken = 0;
+  // per-lane list, sorted by (key desc, index asc): odd-even transposition
+  int jj[VPL];
+#pragma unroll
+  for (int j = 0; j < VPL; ++j) jj[j] = j;
+#pragma unroll
+  for (int r = 0; r < VPL; ++r)
+#pragma unroll
+    for (int i = r & 1; i + 1 < VPL; i += 2) cas_pick<VPL>(ok, jj, s, i, i + 1);
+
   int my_i = 0;
   float my_s = 0.f, denom = 0.f;
 #pragma unroll 1
   for (int k = 0; k < p.K; ++k) {
-    float v = -INFINITY, bs = 0.f;
-    int bj = -1;
-#pragma unroll
-    for (int j = 0; j < VPL; ++j) {
-      const int e = lane * VPL + j;
-      if (e < p.N && !((taken >> j) & 1u) && (bj < 0 || key[j] > v)) {
-        v = key[j];
-        bs = s[j];
-        bj = j;
-      }
-    }
-    const uint32_t o = bj >= 0 ? ord_key(v) : 0u;
-    const uint32_t mx = __reduce_max_sync(0xffffffffu, o);
-    const uint32_t who = __ballot_sync(0xffffffffu, bj >= 0 && o == mx);
+    const uint32_t mx = __reduce_max_sync(0xffffffffu, ok[0]);
+    const uint32_t who = __ballot_sync(0xffffffffu, ok[0] == mx);
     const int wl = __ffs(who) - 1;
-    const int bi = __shfl_sync(0xffffffffu, lane * VPL + bj, wl);
-    const float sv = __shfl_sync(0xffffffffu, bs, wl);
-    if (lane == wl) taken |= 1u << bj;
+    const int bi = __shfl_sync(0xffffffffu, lane * VPL + jj[0], wl);
+    const float sv = __shfl_sync(0xffffffffu, s[0], wl);
+    if (lane == wl) {
+#pragma unroll
+      for (int j = 0; j + 1 < VPL; ++j) { ok[j] = ok[j + 1]; jj[j] = jj[j + 1]; s[j] = s[j + 1]; }
+      ok[VPL - 1] = 0u;
+    }
     if (lane == k) { my_i = bi; my_s = sv; }
     denom += sv;
   }
@@ -176,7 +199,6 @@ __device__ __forceinline__ void route_token(const float (&l)[VPL], const float* 
     const float g = p.renorm ? my_s / denom * p.scale : my_s * p.scale;
     topk_idx[(size_t)t * p.K + lane] = my_i;
     topk_w[(size_t)t * p.K + lane] = g;
-    atomicAdd(&counts[my_i], 1);
   }
 }
 
@@ -185,8 +207,7 @@ template <int VPL>
 __global__ void __launch_bounds__(256) k_topk(const float* __restrict__ logits,
                                               const float* __restrict__ bias, const Params p,
                                               int32_t* __restrict__ topk_idx,
-                                              float* __restrict__ topk_w,
-                                              int32_t* __restrict__ counts) {
+                                              float* __restrict__ topk_w) {
   grid_dep_sync();
   const int t = blockIdx.x * 8 + warp_id();
   if (t >= p.T) return;
@@ -204,7 +225,7 @@ __global__ void __launch_bounds__(256) k_topk(const float* __restrict__ logits,
 #pragma unroll
     for (int j = 0; j < VPL; ++j) l[j] = e0 + j < p.N ? row[e0 + j] : -INFINITY;
   }
-  route_token<VPL>(l, bias, p, t, topk_idx, topk_w, counts);
+  route_token<VPL>(l, bias, p, t, topk_idx, topk_w);
 }
 
 // fp32 gating: router logits on CUDA cores in fp32 (one warp per token, a
@@ -214,8 +235,7 @@ __global__ void __launch_bounds__(256) k_route_f32(const float* __restrict__ x,
                                                    const float* __restrict__ w_r, int d,
                                                    const float* __restrict__ bias, const Params p,
                                                    int32_t* __restrict__ topk_idx,
-                                                   float* __restrict__ topk_w,
-                                                   int32_t* __restrict__ counts) {
+                                                   float* __restrict__ topk_w) {
   grid_dep_sync();
   const int t = blockIdx.x * 8 + warp_id();
   if (t >= p.T) return;
@@ -233,7 +253,7 @@ __global__ void __launch_bounds__(256) k_route_f32(const float* __restrict__ x,
     for (int j = 0; j < VPL; ++j)
       if (lane * VPL + j == e) l[j] = acc;
   }
-  route_token<VPL>(l, bias, p, t, topk_idx, topk_w, counts);
+  route_token<VPL>(l, bias, p, t, topk_idx, topk_w);
 }
 
 // Affinities of every token for every routed expert (for balance statistics):

@@ -1,0 +1,340 @@
+"""Expert parallelism for the DeepSeekMoE layer: routed experts split over
+ranks, rows exchanged by all-to-all, redundant copies of hot experts.
+
+"DeepSeek Technical Report: MoE Architecture", §3.8 (expert parallelism: each
+GPU holds a contiguous share of the routed experts; tokens are dispatched to
+the GPUs holding their experts and the results combined back, with FP8
+dispatch and BF16 combine in §3.6's low-precision communication list) and
+§3.11 (inference deployment: redundant experts, extra copies of the most
+loaded experts placed on other GPUs so that each copy serves part of the
+expert's tokens).
+
+Layout of one rank's step (world W, this rank r, T_r own tokens):
+  1. moe_route + moe_permute (maps only) on the rank's own tokens: the rows
+     of the pairs expert by expert (global routed-expert order), offsets[N+1].
+  2. plan (this module, host integers): every routed expert j has holders
+     (its home rank, then its redundant copies); the rank's rows of j are cut
+     into one contiguous chunk per holder.  The send buffer lists, for each
+     destination rank q in order, the chunks of q's local expert slots in
+     slot order.
+  3. exchange: per-(destination, slot) row counts by all-to-all, then the rows
+     (bf16) and their gate weights by one uneven all-to-all each.
+  4. moe_expert_ffn on the received rows: one group per (source rank, local
+     slot), output in the received order, gate weight applied.
+  5. exchange back with the splits reversed; moe_combine_rows adds the
+     residual, the rank's own shared-expert outputs and the K returned rows of
+     each token, in the order of the single-GPU combine.
+
+Only the plan and the collectives live here; every other step runs in the
+library's CUDA kernels (moe_route, moe_permute, moe_dispatch_rows,
+moe_expert_ffn, moe_combine_rows).  The phases (ep_dispatch, ep_compute,
+ep_combine) are separate functions so that the exchange between them can be
+any transport; ep_forward chains them over torch.distributed.  The plan needs the rank's per-expert row counts on the
+host, so a step reads N integers back from the device before the exchange.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass, field
+from typing import Dict, List, Optional, Sequence
+
+import numpy as np
+
+
+# ----------------------------------------------------------------------------- placement
+@dataclass(frozen=True)
+class Placement:
+    """Which rank holds which routed expert.
+
+    home(j) = j // (N / W) (contiguous ranges, as in §3.8).  replicas[j] lists
+    the extra ranks holding a redundant copy of expert j (§3.11).  Rank r's
+    local slots are its home experts in index order, then its redundant
+    copies in expert order; slot s of rank r runs expert slots[r][s]."""
+    n_routed: int
+    world: int
+    replicas: Dict[int, tuple] = field(default_factory=dict)
+
+    def __post_init__(self):
+        if self.world < 1 or self.n_routed % self.world:
+            raise ValueError("the routed experts must split evenly over the ranks")
+        for j, ranks in self.replicas.items():
+            if not 0 <= j < self.n_routed:
+                raise ValueError(f"replica of unknown expert {j}")
+            if len(set(ranks)) != len(ranks) or self.home(j) in ranks or \
+                    any(not 0 <= q < self.world for q in ranks):
+                raise ValueError(f"bad replica ranks {ranks} for expert {j}")
+
+    @property
+    def per_rank(self) -> int:
+        return self.n_routed // self.world
+
+    def home(self, j: int) -> int:
+        return j // self.per_rank
+
+    def holders(self, j: int) -> List[int]:
+        return [self.home(j)] + list(self.replicas.get(j, ()))
+
+    def slots(self, r: int) -> List[int]:
+        own = list(range(r * self.per_rank, (r + 1) * self.per_rank))
+        return own + [j for j in sorted(self.replicas) if r in self.replicas[j]]
+
+    @property
+    def max_slots(self) -> int:
+        return max(len(self.slots(r)) for r in range(self.world))
+
+
+def choose_replicas(loads: Sequence[int], world: int, n_redundant: int) -> Dict[int, tuple]:
+    """Redundant copies for the n_redundant most loaded experts.
+
+    loads[j] = rows of expert j over all ranks.  Greedy: take the experts by
+    load (descending, ties to the lower index); each gets one copy on the rank
+    whose projected load is lowest (ties to the lower rank), not its home;
+    the expert's load is then shared equally between its holders."""
+    loads = np.asarray(loads, np.int64)
+    N = len(loads)
+    per = N // world
+    rank_load = np.zeros(world)
+    for j in range(N):
+        rank_load[j // per] += loads[j]
+    order = sorted(range(N), key=lambda j: (-int(loads[j]), j))
+    out: Dict[int, tuple] = {}
+    for j in order[:n_redundant]:
+        if loads[j] == 0:
+            break
+        home = j // per
+        cand = [q for q in range(world) if q != home]
+        if not cand:
+            break
+        q = min(cand, key=lambda q: (rank_load[q], q))
+        half = loads[j] / 2.0
+        rank_load[home] -= half
+        rank_load[q] += half
+        out[j] = (q,)
+    return out
+
+
+def chunk_bounds(rows: int, n: int) -> List[int]:
+    """Cut `rows` consecutive rows into n contiguous chunks: chunk c is
+    [b[c], b[c+1]) with b[c] = floor(c * rows / n)."""
+    return [(c * rows) // n for c in range(n + 1)]
+
+
+# ----------------------------------------------------------------------------- one rank's plan
+@dataclass
+class DispatchPlan:
+    """What rank r sends where, and how its returned rows map back.
+
+    send_perm[i]       x_perm row placed at send-buffer row i
+    send_splits[q]     rows sent to rank q
+    send_counts[q, s]  rows sent to rank q for q's local slot s
+    row_of[p]          send-buffer row holding pair p = t*K + k (the rows come
+                       back in the same order)"""
+    send_perm: np.ndarray
+    send_splits: List[int]
+    send_counts: np.ndarray
+    row_of: np.ndarray
+
+
+def dispatch_plan(pl: Placement, counts: Sequence[int], offsets: Sequence[int],
+                  slot_of: Sequence[int]) -> DispatchPlan:
+    """The plan of one rank from its own routing (counts [N], offsets [N+1] and
+    slot_of [T*K] as moe_permute writes them)."""
+    counts = np.asarray(counts, np.int64)
+    offsets = np.asarray(offsets, np.int64)
+    slot_of = np.asarray(slot_of, np.int64)
+    N, W = pl.n_routed, pl.world
+    if counts.shape != (N,) or offsets.shape != (N + 1,):
+        raise ValueError("counts / offsets do not match the placement's expert count")
+    if not np.array_equal(np.diff(offsets), counts) or offsets[0] != 0:
+        raise ValueError("offsets are not the exclusive scan of counts")
+    # chunk c of expert j goes to holder c
+    chunk_of = {}
+    for j in range(N):
+        h = pl.holders(j)
+        b = chunk_bounds(int(counts[j]), len(h))
+        for c, q in enumerate(h):
+            chunk_of[(j, q)] = (int(offsets[j]) + b[c], int(offsets[j]) + b[c + 1])
+    S = pl.max_slots
+    send_counts = np.zeros((W, S), np.int64)
+    pieces, splits = [], []
+    for q in range(W):
+        tot = 0
+        for s, j in enumerate(pl.slots(q)):
+            a, b = chunk_of[(j, q)]
+            pieces.append(np.arange(a, b, dtype=np.int64))
+            send_counts[q, s] = b - a
+            tot += b - a
+        splits.append(tot)
+    send_perm = np.concatenate(pieces) if pieces else np.zeros(0, np.int64)
+    if len(send_perm) != int(offsets[-1]) or \
+            not np.array_equal(np.sort(send_perm), np.arange(int(offsets[-1]))):
+        raise AssertionError("the plan does not send every row exactly once")
+    inv = np.empty(len(send_perm), np.int64)
+    inv[send_perm] = np.arange(len(send_perm))
+    row_of = inv[slot_of] if len(slot_of) else np.zeros(0, np.int64)
+    return DispatchPlan(send_perm, splits, send_counts, row_of)
+
+
+@dataclass
+class ReceivePlan:
+    """Rows rank r receives: from source s, for local slot l, in (s, l) order.
+
+    groups[i] = (row0, rows, slot, out0) for the expert FFN over the received
+    rows (the output keeps the received order, so out0 = row0)."""
+    recv_splits: List[int]
+    groups: np.ndarray
+    slot_rows: np.ndarray      # rows of each local slot over all sources
+
+
+def receive_plan(pl: Placement, rank: int, recv_counts: np.ndarray) -> ReceivePlan:
+    """recv_counts[s, l] = rows source s sent for this rank's local slot l."""
+    recv_counts = np.asarray(recv_counts, np.int64)
+    n_slots = len(pl.slots(rank))
+    groups, splits, run = [], [], 0
+    for s in range(pl.world):
+        tot = 0
+        for l in range(n_slots):
+            c = int(recv_counts[s, l])
+            if c:
+                groups.append((run, c, l, run))
+            run += c
+            tot += c
+        splits.append(tot)
+    g = np.array(groups, np.int64).reshape(-1, 4)
+    return ReceivePlan(splits, g, recv_counts[:, :n_slots].sum(axis=0))
+
+
+# ----------------------------------------------------------------------------- exchange
+class Transport:
+    """All-to-all of rows between ranks.  The default is torch.distributed
+    (NCCL for device tensors, gloo for host tensors)."""
+
+    def all_to_all(self, send, send_splits: List[int], recv_splits: List[int]):
+        import torch
+        import torch.distributed as dist
+        out = torch.empty((sum(recv_splits),) + tuple(send.shape[1:]), dtype=send.dtype,
+                          device=send.device)
+        dist.all_to_all_single(out, send.contiguous(), output_split_sizes=list(recv_splits),
+                               input_split_sizes=list(send_splits))
+        return out
+
+    def counts(self, send_counts: np.ndarray) -> np.ndarray:
+        """send_counts [W, S] -> recv_counts [W, S] (row q of the result came from rank q)."""
+        import torch
+        import torch.distributed as dist
+        backend = dist.get_backend()
+        dev = "cuda" if backend == "nccl" else "cpu"
+        t = torch.as_tensor(np.ascontiguousarray(send_counts), dtype=torch.int64, device=dev)
+        out = torch.empty_like(t)
+        dist.all_to_all_single(out, t)
+        return out.cpu().numpy()
+
+
+# ----------------------------------------------------------------------------- GPU step
+@dataclass
+class RankStep:
+    """One rank's state between the phases of an expert-parallel forward."""
+    rank: int
+    plan: DispatchPlan
+    x_send: object = None
+    w_send: object = None
+    recv: Optional[ReceivePlan] = None
+    y_recv: object = None
+
+
+def ep_dispatch(desc, pl: Placement, rank: int, x, w_router, bias, ws=None) -> RankStep:
+    """Phase 1 on the rank's GPU: routing, the permutation maps, the plan and
+    the send buffer (rows grouped by destination rank, with gate weights)."""
+    import torch
+
+    from . import moe_dispatch_rows, moe_permute, moe_route, workspace
+    T, K, N, d = desc.T, desc.top_k, desc.n_routed, desc.d
+    dev = x.device
+    ws = workspace(desc) if ws is None else ws
+    i32 = dict(dtype=torch.int32, device=dev)
+    idx = torch.empty(max(T, 1), K, **i32)
+    w = torch.empty(max(T, 1), K, dtype=torch.float32, device=dev)
+    counts = torch.empty(N, **i32)
+    moe_route(desc, x, w_router, bias, idx, w, counts, ws)
+    offsets = torch.empty(N + 1, **i32)
+    perm_src = torch.empty(max(T * K, 1), **i32)
+    slot_of = torch.empty(max(T * K, 1), **i32)
+    moe_permute(desc, x, idx, counts, offsets, perm_src, slot_of, None, None, ws)   # maps only
+    plan = dispatch_plan(pl, counts.cpu().numpy(), offsets.cpu().numpy(),
+                         slot_of[:T * K].cpu().numpy())
+    row_of = torch.as_tensor(plan.row_of, dtype=torch.int32, device=dev)
+    x_send = torch.empty(T * K, d, dtype=x.dtype, device=dev)
+    w_send = torch.empty(T * K, dtype=torch.float32, device=dev)
+    moe_dispatch_rows(desc, x, w, row_of, x_send, w_send)
+    return RankStep(rank, plan, x_send, w_send)
+
+
+def ep_compute(desc, pl: Placement, st: RankStep, recv_counts: np.ndarray, x_recv, w_recv,
+               w_gu_local, w_down_local):
+    """Phase 2 on the rank's GPU: the experts it holds on the rows it received
+    (one group per source rank and local slot), gate weights applied."""
+    import torch
+
+    from . import moe_expert_ffn, moe_expert_ffn_workspace_size
+    st.recv = receive_plan(pl, st.rank, recv_counts)
+    n_recv = int(sum(st.recv.recv_splits))
+    dev = x_recv.device
+    y = torch.empty(n_recv, desc.d, dtype=x_recv.dtype, device=dev)
+    if n_recv and len(st.recv.groups):
+        g = st.recv.groups.copy()
+        g[:, 2] += desc.n_shared            # local weight index of slot l
+        groups = torch.as_tensor(g, dtype=torch.int32, device=dev)
+        fws = torch.empty(moe_expert_ffn_workspace_size(desc, len(g), n_recv),
+                          dtype=torch.uint8, device=dev)
+        moe_expert_ffn(desc, w_gu_local.shape[0], groups, x_recv, w_recv, w_gu_local,
+                       w_down_local, y, fws)
+    st.y_recv = y
+    return y
+
+
+def ep_combine(desc, st: RankStep, x, x_residual, y_back, w_gu_local, w_down_local):
+    """Phase 3 on the rank's GPU: its shared experts on its own tokens and the
+    combine of the returned rows, in the single-GPU combine's order."""
+    import torch
+
+    from . import moe_combine_rows, moe_expert_ffn, moe_expert_ffn_workspace_size
+    T, d, Ks = desc.T, desc.d, desc.n_shared
+    dev = x.device
+    y_shared = None
+    if Ks and T:
+        sg = torch.as_tensor([[0, T, s, s * T] for s in range(Ks)], dtype=torch.int32, device=dev)
+        y_shared = torch.empty(Ks * T, d, dtype=x.dtype, device=dev)
+        sws = torch.empty(moe_expert_ffn_workspace_size(desc, Ks, Ks * T), dtype=torch.uint8,
+                          device=dev)
+        moe_expert_ffn(desc, w_gu_local.shape[0], sg, x, None, w_gu_local, w_down_local,
+                       y_shared, sws)
+    h = torch.empty(max(T, 1), d, dtype=x.dtype, device=dev)
+    row_of = torch.as_tensor(st.plan.row_of, dtype=torch.int32, device=dev)
+    y_rows = y_back if len(y_back) else torch.zeros(1, d, dtype=x.dtype, device=dev)
+    moe_combine_rows(desc, x if x_residual is None else x_residual, y_shared, y_rows, row_of, h)
+    return h[:T]
+
+
+def ep_forward(desc, pl: Placement, rank: int, x, x_residual, w_router, bias, w_gu_local,
+               w_down_local, transport: Optional[Transport] = None, ws=None):
+    """One expert-parallel layer forward of this rank's tokens (all ranks call
+    it together).  w_gu_local / w_down_local hold the rank's experts: the Ks
+    shared experts first, then local slot s at index Ks + s (pl.slots(rank)).
+    Returns h [T, d] and the number of rows this rank's experts processed."""
+    transport = transport or Transport()
+    st = ep_dispatch(desc, pl, rank, x, w_router, bias, ws)
+    recv_counts = transport.counts(st.plan.send_counts)
+    recv_splits = [int(v) for v in recv_counts[:, :len(pl.slots(rank))].sum(axis=1)]
+    x_recv = transport.all_to_all(st.x_send, st.plan.send_splits, recv_splits)
+    w_recv = transport.all_to_all(st.w_send, st.plan.send_splits, recv_splits)
+    y = ep_compute(desc, pl, st, recv_counts, x_recv, w_recv, w_gu_local, w_down_local)
+    y_back = transport.all_to_all(y, recv_splits, st.plan.send_splits)
+    return ep_combine(desc, st, x, x_residual, y_back, w_gu_local, w_down_local), len(y)
+
+
+def local_weights(pl: Placement, rank: int, n_shared: int, w_gu, w_down):
+    """The rank's expert weights (shared experts, then its local slots) taken
+    from full [Ks+N, ...] tensors: the placement a deployment would load."""
+    import torch
+    ids = list(range(n_shared)) + [n_shared + j for j in pl.slots(rank)]
+    sel = torch.as_tensor(ids, device=w_gu.device)
+    return w_gu.index_select(0, sel).contiguous(), w_down.index_select(0, sel).contiguous()

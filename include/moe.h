@@ -123,7 +123,9 @@ moe_status moe_route(const moe_layer_desc* desc, const void* x, const void* w_ro
  *   offsets [N+1], perm_src [R], slot_of [R] int32 out
  *   x_perm  [R, d] act_dtype (F32/BF16), or [R + T, d] E4M3 bytes whose rows
  *     R..R+T-1 hold the quantised x in token order (the shared experts' input)
- *   x_perm_scale [R + T, d/128] fp32 out for E4M3, NULL otherwise */
+ *   x_perm_scale [R + T, d/128] fp32 out for E4M3, NULL otherwise
+ *   x_perm and x_perm_scale both NULL: only offsets, perm_src and slot_of are
+ *     written (x is not read; used by the expert-parallel dispatch below) */
 moe_status moe_permute(const moe_layer_desc* desc, const void* x, const int32_t* topk_idx,
                        const int32_t* counts, int32_t* offsets, int32_t* perm_src,
                        int32_t* slot_of, void* x_perm, float* x_perm_scale, void* ws,
@@ -141,7 +143,11 @@ moe_status moe_permute(const moe_layer_desc* desc, const void* x, const int32_t*
  *   tokens for N = 256); larger shapes return MOE_ERR_UNSUPPORTED with the
  *   reason in moe_last_error_message.  No device memory is allocated or freed.
  *   The first call on a device looks up the array's device address (with that
- *   device current); make that first call before any stream capture.
+ *   device current); make that first call before any stream capture.  The
+ *   address is kept for the life of the process, so the library does not
+ *   support cudaDeviceReset (or another teardown of the primary context)
+ *   between calls; the same holds for the per-device set-up of every entry
+ *   point.
  *   Every call uses the same array: calls whose work overlaps on the GPU (two
  *   streams, or two host threads) race and must be serialised by the caller.
  *   The array keeps the last call's contents; each call writes every entry it
@@ -213,6 +219,87 @@ moe_status moe_balance_stats(const moe_layer_desc* desc, const float* s, const i
  * below, unchanged when equal (the comparison is exact, in integers). */
 moe_status moe_bias_update(const moe_layer_desc* desc, const int32_t* counts, float* bias,
                            float gamma, cudaStream_t stream);
+
+/* ---- Expert parallelism ---------------------------------------------------
+ * "DeepSeek Technical Report: MoE Architecture" §3.8: the routed experts are
+ * split over GPUs; each GPU routes its own tokens, dispatches the permuted rows
+ * of every expert to the GPU that holds it, runs the experts it holds on the
+ * rows it receives, and returns the results for the combine.  §3.11 adds
+ * redundant copies of heavily loaded experts on other GPUs, each copy taking a
+ * share of the expert's rows.  The exchange itself (all-to-all of rows) is the
+ * caller's collective; these two calls are the compute on either side of it.
+ *
+ * Expert FFN over caller-given groups of rows: group i (groups[4i..4i+3] =
+ * row0, rows, expert, out_row0, device int32) computes, for r < rows,
+ *   y_rows[out_row0 + r] = row_w[out_row0 + r] * FFN_expert(x_rows[row0 + r])
+ * (row_w NULL: weight 1) with the same GEMMs as moe_grouped_swiglu.  expert
+ * indexes w_gu [n_experts, 2I, d] / w_down [n_experts, d, I]; the output
+ * ranges of the groups must not overlap.  F32 and BF16 layers only.
+ *   n_groups 1..1024; x_rows [n_rows_in, d], y_rows [n_rows_out, d], row_w
+ *   [n_rows_out] fp32.  A group outside these bounds, or with an expert outside
+ *   [0, n_experts), is skipped and sets MOE_ERR_DEVICE_CHECK.
+ *   ws: moe_expert_ffn_workspace_size(desc, n_groups, n_rows_out) bytes. */
+size_t moe_expert_ffn_workspace_size(const moe_layer_desc* desc, int32_t n_groups,
+                                     int32_t n_rows_out);
+moe_status moe_expert_ffn(const moe_layer_desc* desc, int32_t n_experts, int32_t n_groups,
+                          const int32_t* groups, int32_t n_rows_in, int32_t n_rows_out,
+                          const void* x_rows, const float* row_w, const void* w_gu,
+                          const void* w_down, void* y_rows, void* ws, size_t ws_bytes,
+                          cudaStream_t stream);
+
+/* Dispatch gather: x_rows[row_of[t*K + k]] = x[t] and, when w_rows is not
+ * NULL, w_rows[row_of[t*K + k]] = topk_w[t*K + k] -- the send buffer of the
+ * exchange, in the row order the caller's plan chose.  x [T, d] act_dtype,
+ * topk_w [T, K] fp32, row_of [T*K] int32 (an index outside [0, n_rows) is
+ * skipped and sets MOE_ERR_DEVICE_CHECK), x_rows [n_rows, d], w_rows [n_rows]
+ * fp32.  F32 and BF16 layers only. */
+moe_status moe_dispatch_rows(const moe_layer_desc* desc, const void* x, const float* topk_w,
+                             const int32_t* row_of, int32_t n_rows, void* x_rows, float* w_rows,
+                             cudaStream_t stream);
+
+/* Combine of returned rows: h[t] = x_res[t] + sum_{s<Ks} y_shared[s*T + t]
+ * + sum_{k<K} y_rows[row_of[t*K + k]], in fp32, in that order (the order of
+ * moe_combine, so with the same row values the two agree bit for bit).
+ *   y_shared [Ks*T, d] (NULL when Ks = 0), y_rows [n_rows, d], row_of [T*K]
+ *   int32; an index outside [0, n_rows) is skipped and sets
+ *   MOE_ERR_DEVICE_CHECK.  Element types as for moe_combine. */
+moe_status moe_combine_rows(const moe_layer_desc* desc, const void* x_residual,
+                            const void* y_shared, const void* y_rows, const int32_t* row_of,
+                            int32_t n_rows, void* h, cudaStream_t stream);
+
+/* ---- Layer backward (bf16) ------------------------------------------------
+ * The gradients of the layer for an upstream gradient dh = dL/dh, by the
+ * chain rule of the output equation above through SwiGLU experts, the gate
+ * weights and the affinities ("DeepSeek Technical Report: MoE Architecture",
+ * §1.1(2) and equation [1] of §5.3 for the output, §2.3 and §3.3 with
+ * equations [3]/[4] of §5.3 for the gating; §3.6 lists the activation- and
+ * weight-backward GEMMs of every linear layer).  Per active (token, expert)
+ * row with gate weight g (1 for shared experts): a = W_gate u, b = W_up u,
+ * z = SiLU(a) b, dz = g W_down^T dh, da = dz b SiLU'(a), db = dz SiLU(a),
+ * du += W_gate^T da + W_up^T db, dW_down += g dh z^T, dW_gate += da u^T,
+ * dW_up += db u^T, dg = <dh, W_down z>; then the gate-weight backward
+ * (renorm: ds_k = c (dg_k - sum_k' dg_k' s_k' / S) / S), the affinity backward
+ * (sigmoid: dl = ds s (1 - s); softmax: dl = s (ds - <ds, s>)), and the
+ * router: du += W_r^T dl, dW_r = dl^T u.  No gradient flows through the
+ * selection, and the selection bias gets none.  The residual's gradient is dh
+ * itself and is not written.
+ * The call recomputes the routing, the permutation and the pre-activations
+ * a, b from x (nothing is kept from the forward).  bf16 layers only
+ * (MOE_ERR_UNSUPPORTED otherwise); N*2 bytes must be a multiple of 16.
+ *   x [T, d], w_router [N, d], w_gu [E, 2I, d], w_down [E, d, I], dh [T, d]: bf16 in
+ *   bias [N] fp32 or NULL (selection only, as in moe_route)
+ *   dx [T, d] bf16 out: gradient of x through the experts and the router
+ *   dw_router [N, d] fp32 out; dw_gu [E, 2I, d] fp32 out; dw_down [E, d, I]
+ *     fp32 out (overwritten, zeros for experts no token reaches)
+ *   ws: moe_backward_workspace_size(desc) bytes. */
+size_t moe_backward_workspace_size(const moe_layer_desc* desc);
+moe_status moe_backward(const moe_layer_desc* desc, const void* x, const void* w_router,
+                        const float* bias, const void* w_gu, const void* w_down, const void* dh,
+                        void* dx, float* dw_router, float* dw_gu, float* dw_down, void* ws,
+                        size_t ws_bytes, cudaStream_t stream);
+
+/* Number of kernels moe_backward launches for `desc` (0 if invalid or T = 0). */
+int32_t moe_backward_launch_count(const moe_layer_desc* desc);
 
 /* Offline FP8 quantisation of weights in 128x128 blocks (not on the hot path).
  * w_bf16 [batch, rows, cols] bf16 in; w_e4m3 [batch, rows, cols] bytes out;

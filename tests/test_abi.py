@@ -125,8 +125,15 @@ def test_status_strings():
 
 
 def test_launch_count():
+    # router GEMM, top-K, histogram, scan, slots, gather, group table, GEMM1,
+    # GEMM2, combine; fp32 routes in one kernel
     assert moe.moe_forward_launch_count(v3()) == 10
+    assert moe.moe_forward_launch_count(v3(dtype="e4m3")) == 10
+    assert moe.moe_forward_launch_count(v3(dtype="f32")) == 9
+    assert moe.moe_forward_launch_count(v3(T=0)) == 2
     assert moe.moe_forward_launch_count(v3(top_k=300)) == 0
+    assert moe.moe_backward_launch_count(v3()) == 16
+    assert moe.moe_backward_launch_count(v3(T=0)) == 0
 
 
 def test_binding_refuses_short_or_strided_buffers():

@@ -1,0 +1,123 @@
+"""GPU parity of the layer backward (moe_backward) against the fp64 backward
+oracle (oracle/moe_backward.py, itself pinned to central differences of the
+forward oracle in tests/test_oracle_backward.py).
+
+Every gradient is compared as a whole tensor with the max-abs-relative measure
+of the forward tests: dx (through the experts and the router), dW_r, and the
+three matrices of every expert (zeros for experts no token reaches).  The
+bound 2e-2 is the bf16 one of the forward: the operands x, dh, the weights and
+the backward's intermediates (a, b, g z, da, db, dl) are bf16, products
+accumulate in fp32.  Both sides use the GPU's selection (checked against the
+oracle's first, bit-exact outside near-ties), since no gradient flows through
+the choice of experts.
+"""
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+import forward_moe_route_b200 as moe
+import synth
+from oracle import moe_backward as mb
+from oracle import moe_oracle as mo
+from synth import recipes
+
+from gpu_layer import HostLayer, check_routing, f64
+
+pytestmark = pytest.mark.gpu
+
+TOL = 2e-2
+TID_DH = 6          # tensor id of the upstream gradient in the seeded generator
+
+C = recipes.CONFIGS
+CASES = {
+    # V3-like: sigmoid + selection bias, 4 groups / top-2 groups, renorm x 2.5;
+    # T spans several 128-row tiles with a ragged tail
+    "v3_small": dataclasses.replace(
+        recipes.small_variant(C["v3_bf16"], T=300, d=512, inter=256, n_routed=32),
+        n_group=4, topk_group=2),
+    # 16B-like: softmax without renorm, 2 shared experts, d and I not multiples of 256
+    "dsmoe16b_small": recipes.small_variant(C["dsmoe16b_bf16"], T=257, d=320, inter=192,
+                                            n_routed=16),
+    # a single token: most experts get no row, their weight gradients must be zero
+    "v3_T1": dataclasses.replace(
+        recipes.small_variant(C["v3_bf16"], T=1, d=256, inter=128, n_routed=32),
+        n_group=4, topk_group=2),
+}
+
+
+def upstream(cfg):
+    v = synth.host_normal(cfg.T * cfg.d, 1.0, cfg.seed, TID_DH).reshape(cfg.T, cfg.d)
+    dh = torch.from_numpy(v).to(torch.bfloat16)
+    return dh.cuda(), dh.double().numpy()
+
+
+def run_backward(cfg, inp, dh):
+    desc = moe.desc_from_config(cfg)
+    ws = moe.backward_workspace(desc)
+    E, I, d, N = cfg.n_experts, cfg.inter, cfg.d, cfg.n_routed
+    dx = torch.full((cfg.T, d), float("nan"), dtype=torch.bfloat16, device="cuda")
+    dwr = torch.full((N, d), float("nan"), dtype=torch.float32, device="cuda")
+    dwgu = torch.full((E, 2 * I, d), float("nan"), dtype=torch.float32, device="cuda")
+    dwd = torch.full((E, d, I), float("nan"), dtype=torch.float32, device="cuda")
+    moe.moe_backward(desc, inp["x"], inp["w_r"], inp["bias"], inp["w_gu"], inp["w_down"], dh, dx,
+                     dwr, dwgu, dwd, ws)
+    st = moe.moe_last_device_status()
+    return dx, dwr, dwgu, dwd, st
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_backward_parity(name):
+    cfg = CASES[name]
+    moe.moe_last_device_status()
+    inp = recipes.device_inputs(cfg)
+    dh, dh64 = upstream(cfg)
+    dx, dwr, dwgu, dwd, st = run_backward(cfg, inp, dh)
+    assert st == moe.OK, moe.moe_status_string(st)
+    # the selection the backward used: the forward's routing of the same inputs
+    desc = moe.desc_from_config(cfg)
+    ws = moe.workspace(desc)
+    idx = torch.empty(cfg.T, cfg.top_k, dtype=torch.int32, device="cuda")
+    w = torch.empty(cfg.T, cfg.top_k, dtype=torch.float32, device="cuda")
+    counts = torch.empty(cfg.n_routed, dtype=torch.int32, device="cuda")
+    moe.moe_route(desc, inp["x"], inp["w_r"], inp["bias"], idx, w, counts, ws)
+    host = HostLayer(cfg)
+    ref_route = host.route()
+    g_idx = idx.cpu().numpy().astype(np.int64)
+    check_routing(cfg, ref_route, g_idx, w.cpu().numpy().astype(np.float64),
+                  counts.cpu().numpy())
+    ref = mb.moe_backward(host.x, host.w_r, host.bias, host.expert, dh64, n_shared=cfg.n_shared,
+                          gate=cfg.gate, top_k=cfg.top_k, n_group=cfg.n_group,
+                          topk_group=cfg.topk_group, renorm=cfg.renorm,
+                          route_scale=cfg.route_scale, idx_override=g_idx)
+    E, I = cfg.n_experts, cfg.inter
+    gu_ref = np.zeros((E, 2 * I, cfg.d))
+    d_ref = np.zeros((E, cfg.d, I))
+    for e, (g_, u_, dd) in ref["experts"].items():
+        gu_ref[e, :I], gu_ref[e, I:], d_ref[e] = g_, u_, dd
+    errs = {
+        "dx": mo.max_abs_rel(f64(dx), ref["dx"]),
+        "dw_router": mo.max_abs_rel(f64(dwr), ref["dw_r"]),
+        "dw_gu": mo.max_abs_rel(f64(dwgu), gu_ref),
+        "dw_down": mo.max_abs_rel(f64(dwd), d_ref),
+    }
+    print(f"{name}: " + ", ".join(f"{k} {v:.2e}" for k, v in errs.items()))
+    # experts that no token reaches get exactly zero weight gradients
+    untouched = [cfg.n_shared + j for j in range(cfg.n_routed) if not np.any(g_idx == j)]
+    if untouched:
+        assert torch.count_nonzero(dwgu[untouched]) == 0
+        assert torch.count_nonzero(dwd[untouched]) == 0
+    for k, v in errs.items():
+        assert v <= TOL, f"{k}: max-abs-rel {v:.3e} above {TOL}"
+
+
+def test_backward_is_deterministic():
+    cfg = CASES["v3_small"]
+    inp = recipes.device_inputs(cfg)
+    dh, _ = upstream(cfg)
+    a = run_backward(cfg, inp, dh)
+    b = run_backward(cfg, inp, dh)
+    assert a[4] == moe.OK and b[4] == moe.OK
+    for x, y in zip(a[:4], b[:4]):
+        assert torch.equal(x, y)

@@ -55,6 +55,37 @@ def test_noalloc_permute_matches_workspace_permute_twice():
             assert torch.equal(a, b), f"call {call}: no-alloc result differs"
 
 
+@pytest.mark.gpu
+def test_noalloc_permute_e4m3_and_empty_batch():
+    # E4M3 layer: the quantising gather (codes and 1x128 scales, rows R..R+T-1
+    # holding x in token order) must match the workspace path byte for byte
+    cfg = recipes.small_variant(recipes.CONFIGS["v3_fp8"], T=300, d=512, inter=256)
+    inp = recipes.device_inputs(cfg)
+    desc, ws, idx, counts = _route(cfg, inp)
+    T, K, N, d = cfg.T, cfg.top_k, cfg.n_routed, cfg.d
+    rows = T * K + T
+
+    def outs():
+        i32 = dict(dtype=torch.int32, device="cuda")
+        return (torch.full((N + 1,), -1, **i32), torch.full((T * K,), -1, **i32),
+                torch.full((T * K,), -1, **i32),
+                torch.zeros(rows, d, dtype=torch.uint8, device="cuda"),
+                torch.zeros(rows, d // 128, dtype=torch.float32, device="cuda"))
+    ref, got = outs(), outs()
+    moe.moe_permute(desc, inp["x"], idx, counts, *ref, ws)
+    moe.moe_permute_noalloc(desc, inp["x"], idx, counts, *got)
+    assert moe.moe_last_device_status() == moe.OK
+    for a, b in zip(ref, got):
+        assert torch.equal(a, b), "no-alloc E4M3 result differs"
+    # T = 0: offsets are all zero, nothing else is touched
+    empty = moe.make_desc(0, 512, 1, 32, 8, 256, "sigmoid", True, 2.5, 4, 2, "bf16")
+    offsets = torch.full((33,), -1, dtype=torch.int32, device="cuda")
+    dummy = torch.zeros(64, dtype=torch.int32, device="cuda")   # >= N int32 for counts
+    moe.moe_permute_noalloc(empty, dummy, dummy, dummy, offsets, dummy, dummy, dummy, None)
+    assert moe.moe_last_device_status() == moe.OK
+    assert torch.count_nonzero(offsets) == 0
+
+
 def test_noalloc_rejects_shapes_beyond_the_fixed_scratch():
     # ceil(T/128) * N above MOE_NOALLOC_HIST_INTS is refused before any CUDA call
     big = moe.make_desc(131073, 7168, 1, 256, 8, 2048, "sigmoid", True, 2.5, 8, 4, "bf16")

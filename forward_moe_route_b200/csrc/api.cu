@@ -80,7 +80,7 @@ moe_status fill_dims(const moe_layer_desc* desc, Dims* D) {
 
 struct Layout {
   size_t logits, topk_idx, topk_w, counts, hist, offsets, perm_src, slot_of, pair_of, gtab;
-  size_t x_perm, x_perm_scale, hbuf, hscale, y_slots, cnt, total;
+  size_t x_perm, x_perm_scale, hbuf, hscale, y_slots, total;
 };
 
 Layout layout(const Dims& D) {
@@ -104,8 +104,6 @@ Layout layout(const Dims& D) {
   L.hbuf = take(hrows * D.I * D.op_esz);
   L.hscale = take(D.fp8 ? hrows * (D.I / 128) * 4 : 0);
   L.y_slots = take((size_t)D.T * (D.K + D.Ks) * D.d * D.y_esz);
-  // arrival counters of the fused residual (bf16 layers): [T, d/32]
-  L.cnt = take((!D.f32 && !D.fp8) ? (size_t)D.T * (D.d / 32) * 4 : 0);
   L.total = o;
   return L;
 }
@@ -594,32 +592,22 @@ moe_status launch_gate_up(int kind, const void* w_gu, int64_t n_experts, const v
   return launched("gate/up GEMM (CTA pairs)");
 }
 
-// fuse_res / fuse_h (bf16 layers only): the down projection also adds the
-// residual and writes h (see gemm_t.cuh); nullptr keeps the slots-only path.
-bool fusable(const Dims& D) { (void)D; return false; }
-
 moe_status do_grouped(const Dims& D, const Layout& L, const void* x, const void* x_perm,
                       const float* x_perm_scale, const int32_t* offsets, const int32_t* slot_of,
                       const float* topk_w, const void* w_gu, const float* w_gu_scale,
                       const void* w_down, const float* w_down_scale, void* y_slots, uint8_t* ws,
-                      int sms, cudaStream_t st, const void* fuse_res = nullptr,
-                      void* fuse_h = nullptr) {
+                      int sms, cudaStream_t st) {
   if (D.T == 0) return MOE_OK;
   const int E = (int)D.E;
   int32_t* gtab = reinterpret_cast<int32_t*>(ws + L.gtab);
   int32_t* pair_of = reinterpret_cast<int32_t*>(ws + L.pair_of);
   void* hbuf = ws + L.hbuf;
-  const bool fuse = fuse_h && fusable(D);
-  int32_t* cnt = fuse ? reinterpret_cast<int32_t*>(ws + L.cnt) : nullptr;
-  const int n_cnt = fuse ? (int)(D.T * (D.d / 32)) : 0;
-  const int64_t prep_items = D.R > n_cnt ? D.R : n_cnt;
-  const int prep_blocks =
-      1 + (int)((prep_items + 1023) / 1024 < 4 * sms ? (prep_items + 1023) / 1024 : 4 * sms);
+  const int prep_blocks = 1 + (int)((D.R + 1023) / 1024 < 4 * sms ? (D.R + 1023) / 1024 : 4 * sms);
   moe_status rc = trace(2, st);
   if (rc != MOE_OK) return rc;
   rc = launch_chain("k_prep_groups", perm::k_prep_groups, dim3(prep_blocks), dim3(1024), 0, st,
                     offsets, (int)D.T, (int)D.K, (int)D.Ks, (int)D.N, D.fp8 ? 1 : 0, gtab,
-                    slot_of, pair_of, cnt, n_cnt);
+                    slot_of, pair_of);
   if (rc != MOE_OK) return rc;
   if (D.fp8)
     return do_grouped_fp8(D, L, x_perm, x_perm_scale, gtab, pair_of, topk_w, w_gu, w_gu_scale,
@@ -673,11 +661,6 @@ moe_status do_grouped(const Dims& D, const Layout& L, const void* x, const void*
     a.topk_w = topk_w;
     a.K = (int)D.K;
     a.Ks = (int)D.Ks;
-    if (fuse) {
-      a.cnt = cnt;
-      a.x_res = static_cast<const __nv_bfloat16*>(fuse_res);
-      a.h = static_cast<__nv_bfloat16*>(fuse_h);
-    }
     rc = launch_down(kind, w_down, D.E, hbuf, esz, hrows, tok_tiles, a, st);
     if (rc != MOE_OK) return rc;
     rc = trace(4, st);
@@ -1211,14 +1194,10 @@ moe_status moe_forward(const moe_layer_desc* desc, const void* x, const void* x_
   if ((rc = do_permute(D, reinterpret_cast<int32_t*>(w8 + L.hist), x, idx, nullptr, offsets,
                        perm_src, slot_of, x_perm, x_perm_scale, stream, cnt)) != MOE_OK)
     return rc;
-  const void* x_res = x_residual ? x_residual : x;
-  const bool fuse = fusable(D);
   if ((rc = do_grouped(D, L, x, x_perm, x_perm_scale, offsets, slot_of, tw, w_gu, w_gu_scale,
-                       w_down, w_down_scale, y, w8, sms, stream, fuse ? x_res : nullptr,
-                       fuse ? h : nullptr)) != MOE_OK)
+                       w_down, w_down_scale, y, w8, sms, stream)) != MOE_OK)
     return rc;
-  // bf16: the down projection has added the residual and written h
-  if (!fuse || D.T == 0) rc = do_combine(D, x_res, y, h, stream);
+  rc = do_combine(D, x_residual ? x_residual : x, y, h, stream);
   if (rc == MOE_OK) rc = trace(5, stream);
   return rc;
 }
@@ -1333,9 +1312,8 @@ int32_t moe_forward_launch_count(const moe_layer_desc* desc) {
   if (fill_dims(desc, &D) != MOE_OK) return 0;
   if (D.T == 0) return 2;
   // route (router GEMM + top-K; fp32: one kernel) + permute (4) + grouped (3)
-  // + combine (1); bf16 layers add the residual in the down projection and
-  // launch no combine
-  return (D.f32 ? 1 : 2) + 4 + 3 + (fusable(D) ? 0 : 1);
+  // + combine (1)
+  return (D.f32 ? 1 : 2) + 4 + 3 + 1;
 }
 
 moe_status moe_selftest_bounded_wait(uint32_t limit_us, cudaStream_t stream) {

@@ -12,10 +12,7 @@
 // The tile's UMMA takes the tile's own token count rounded up to 32, so an
 // expert's last token tile wastes at most 31 columns of tensor-core work.
 // The epilogue scales by each token's gate weight (1 for shared experts) and
-// writes the features into the token's slot row; in the layer forward it also
-// adds the residual: the tile whose piece completes a token's K+Ks pieces of a
-// 32-feature slice (counted per slice with an atomic) sums them with x_res in
-// the combine's fixed order and writes h.  Weight tiles run fastest
+// writes the features into the token's slot row.  Weight tiles run fastest
 // inside an expert, so the clusters of one wave share the expert's token
 // tiles in L2.
 //
@@ -72,30 +69,7 @@ struct Args {
   // c_row + i, scaled by row_w[c_row + i] (1 without row_w)
   int plain;
   const float* row_w;
-  // fused residual (bf16 slot mode): cnt [T, d/32] arrival counters, zero on
-  // entry; the warp whose piece completes a (token, 32-feature slice) writes
-  // h = x_res + sum of the token's slot pieces there (see the epilogue)
-  int* cnt;
-  const __nv_bfloat16* x_res;
-  __nv_bfloat16* h;
 };
-
-// Atomic add with acquire-release semantics at GPU scope (returns the old value).
-__device__ __forceinline__ int atom_add_acq_rel(int* p, int v) {
-  int old;
-  asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v)
-               : "memory");
-  return old;
-}
-// 16-byte load cached in L2 only (the rows were written by other SMs).
-__device__ __forceinline__ uint4 ld_cg_v4(const void* p) {
-  uint4 v;
-  asm volatile("ld.global.cg.v4.u32 {%0,%1,%2,%3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(p)
-               : "memory");
-  return v;
-}
 
 __device__ __forceinline__ uint32_t cluster_rank() {
   uint32_t r;
@@ -375,60 +349,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               if (dst >= 0 && feat < a.d)
                 *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.y) +
                                           (size_t)dst * a.d + feat) = val;
-            }
-            if (a.cnt) {
-              // Fused residual.  The chunk's pieces (16 tokens x this warp's 32
-              // features) are in y; each token counts its arrival on its
-              // (token, slice) counter.  The K+Ks pieces of a token-slice come
-              // from K+Ks different tiles, and the arrival that completes the
-              // count sums them -- x_res + shared pieces + routed pieces, fp32,
-              // in the order of k_combine -- and writes h.  Release: every
-              // lane's stores are fenced before the warp barrier that precedes
-              // the atomic; acquire: the atomic is acq_rel and the readers
-              // fence again and read through L2.
-              __threadfence();
-              __syncwarp();
-              const int S = a.K + a.Ks;
-              const long long dj =
-                  __shfl_sync(0xffffffffu, dreg[(16 * c) >> 5], ((16 * c) & 31) + (lane & 15));
-              const long long tj = dj >= 0 ? dj / S : -1;
-              const bool mine = lane < 16 && 16 * c + lane < ntok && dj >= 0 && fw0 < a.d;
-              int old = 0;
-              if (mine) old = atom_add_acq_rel(a.cnt + (size_t)tj * (a.d / 32) + fw0 / 32, 1);
-              const uint32_t last = __ballot_sync(0xffffffffu, mine && old == S - 1);
-              if (last) {
-                __threadfence();
-#pragma unroll
-                for (int round = 0; round < 2; ++round) {
-                  const int jj = round * 8 + (lane >> 2);
-                  const long long t = __shfl_sync(0xffffffffu, tj, jj);
-                  if ((last >> jj) & 1u) {
-                    const int feat = fw0 + (lane & 3) * 8;
-                    float acc[8];
-                    auto add8 = [&](uint4 r, bool init) {
-                      const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&r);
-#pragma unroll
-                      for (int i = 0; i < 4; ++i) {
-                        const float lo = __low2float(p2[i]), hi = __high2float(p2[i]);
-                        acc[2 * i] = init ? lo : acc[2 * i] + lo;
-                        acc[2 * i + 1] = init ? hi : acc[2 * i + 1] + hi;
-                      }
-                    };
-                    add8(*reinterpret_cast<const uint4*>(a.x_res + (size_t)t * a.d + feat), true);
-                    const __nv_bfloat16* yb = reinterpret_cast<const __nv_bfloat16*>(a.y) +
-                                              (size_t)t * S * a.d + feat;
-                    for (int sh = 0; sh < a.Ks; ++sh)
-                      add8(ld_cg_v4(yb + (size_t)(a.K + sh) * a.d), false);
-                    for (int k = 0; k < a.K; ++k) add8(ld_cg_v4(yb + (size_t)k * a.d), false);
-                    uint4 o;
-                    o.x = gemm::pack_bf16x2(acc[0], acc[1]);
-                    o.y = gemm::pack_bf16x2(acc[2], acc[3]);
-                    o.z = gemm::pack_bf16x2(acc[4], acc[5]);
-                    o.w = gemm::pack_bf16x2(acc[6], acc[7]);
-                    *reinterpret_cast<uint4*>(a.h + (size_t)t * a.d + feat) = o;
-                  }
-                }
-              }
             }
           } else {
 #pragma unroll

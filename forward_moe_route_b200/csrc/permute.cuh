@@ -240,14 +240,11 @@ __global__ void __launch_bounds__(256) k_gather_quant(const __nv_bfloat16* __res
 
 // Group table for the grouped GEMMs (block 0) and the permuted-row -> pair map
 // (all blocks).  Groups: shared experts 0..Ks-1 then routed experts 0..N-1.
-// With cnt != nullptr the other blocks also zero the n_cnt arrival counters
-// of the down projection's fused residual.
 __global__ void __launch_bounds__(1024) k_prep_groups(const int32_t* __restrict__ offsets, int T,
                                                       int K, int Ks, int N, int fp8,
                                                       int32_t* __restrict__ gtab,
                                                       const int32_t* __restrict__ slot_of,
-                                                      int32_t* __restrict__ pair_of,
-                                                      int32_t* __restrict__ cnt, int n_cnt) {
+                                                      int32_t* __restrict__ pair_of) {
   grid_dep_sync();
   const int R = T * K;
   if (blockIdx.x > 0) {
@@ -257,10 +254,6 @@ __global__ void __launch_bounds__(1024) k_prep_groups(const int32_t* __restrict_
       if ((unsigned)row < (unsigned)R) pair_of[row] = i;
       else set_status(MOE_ERR_DEVICE_CHECK);
     }
-    if (cnt)
-      for (int i = (blockIdx.x - 1) * blockDim.x + threadIdx.x; i < n_cnt;
-           i += (gridDim.x - 1) * blockDim.x)
-        cnt[i] = 0;
     return;
   }
   __shared__ int32_t warp_tot[32];

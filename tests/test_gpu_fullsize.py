@@ -79,19 +79,8 @@ def sample_tokens(cfg, g_idx, counts, offsets, perm_src, n_strided, n_extra=64, 
 
 
 def check_layer(cfg, n_strided):
-    fp8 = cfg.dtype == "e4m3"
     offs = zipf_offsets(cfg)
     inp = recipes.device_inputs(cfg, "cuda", offs)
-    if fp8:
-        E, I, d = cfg.n_experts, cfg.inter, cfg.d
-        gq = torch.empty(E, 2 * I, d, dtype=torch.uint8, device="cuda")
-        gs = torch.empty(E, 2 * I // 128, d // 128, dtype=torch.float32, device="cuda")
-        dq = torch.empty(E, d, I, dtype=torch.uint8, device="cuda")
-        ds = torch.empty(E, d // 128, I // 128, dtype=torch.float32, device="cuda")
-        moe.moe_quantize_fp8_blockwise(inp["w_gu"], 2 * I, d, E, gq, gs)
-        moe.moe_quantize_fp8_blockwise(inp["w_down"], d, I, E, dq, ds)
-        inp.update(w_gu=gq, w_gu_scale=gs, w_down=dq, w_down_scale=ds)
-        torch.cuda.synchronize()
     h, idx, counts, perm = forward(cfg, inp, want_perm=True)
     h_moe, _, _, _ = forward(cfg, inp, x_res=torch.zeros_like(inp["x"]))
     host = HostLayer(cfg, offs)
@@ -122,36 +111,13 @@ def check_layer(cfg, n_strided):
     toks = sample_tokens(cfg, g_idx, g_counts, offsets, perm_src, n_strided)
     w_used = mo.gate_weights(ref["s"], g_idx, cfg.renorm, cfg.route_scale)
     xs = host.x[toks]
-    if fp8:
-        def expert(e):
-            # one expert at a time: layer_output asks for each expert once, and
-            # keeping all of them in float64 would need ~90 GB at the V3 shape
-            wg, wu, wd = recipes.host_expert(cfg, e)
-            qg, sg = of8.quantize_weight_128x128(np.concatenate([wg, wu]).astype(np.float32))
-            qd, sd = of8.quantize_weight_128x128(wd.astype(np.float32))
-            gu = of8.dequant_weight(qg, sg)
-            return gu[:cfg.inter], gu[cfg.inter:], of8.dequant_weight(qd, sd)
-
-        q, s = of8.quantize_act_1x128(xs.astype(np.float32))
-        h_ref, d_ref = mo.layer_output(of8.dequant_act(q, s), xs, g_idx[toks], w_used[toks],
-                                       cfg.n_shared, expert, ffn=of8.fp8_swiglu_ffn)
-        tol = TOL["e4m3"]
-        # the quantisation error itself: distance of the MoE part to the
-        # unquantised fp64 layer, gated separately at twice E4M3's step 2^-4
-        _, d_plain = mo.layer_output(xs, xs, g_idx[toks], w_used[toks], cfg.n_shared,
-                                     lambda e: recipes.host_expert(cfg, e))
-        err_plain = mo.max_abs_rel(f64(h_moe)[toks], d_plain)
-        print(f"{cfg.name}: MoE part vs the unquantised layer {err_plain:.3e}")
-        assert err_plain <= 2.0 ** -3
-    else:
-        h_ref, d_ref = mo.layer_output(xs, xs, g_idx[toks], w_used[toks], cfg.n_shared,
-                                       lambda e: recipes.host_expert(cfg, e))
-        tol = TOL["bf16"]
+    h_ref, d_ref = mo.layer_output(xs, xs, g_idx[toks], w_used[toks], cfg.n_shared,
+                                   lambda e: recipes.host_expert(cfg, e))
     err = mo.max_abs_rel(f64(h)[toks], h_ref)
     err_d = mo.max_abs_rel(f64(h_moe)[toks], d_ref)
     print(f"{cfg.name}: {len(toks)} sampled tokens, h {err:.3e}, MoE part {err_d:.3e}, "
           f"near-ties {len(ties)} of {cfg.T}, max/mean load {g_counts.max() / g_counts.mean():.2f}")
-    assert err <= tol and err_d <= tol
+    assert err <= TOL["bf16"] and err_d <= TOL["bf16"]
 
 
 def test_dsmoe16b_full():
@@ -167,6 +133,96 @@ def test_v3_bf16_full():
     check_layer(C["v3_bf16"], 256)
 
 
-@pytest.mark.parametrize("T", [256, 2048, 16384, 65536])
-def test_v3_fp8_full(T):
-    check_layer(C["v3_fp8"].with_T(T), 256)
+def fp8_expert(cfg, e):
+    """Expert e as the FP8 layer sees it: the oracle's 128x128 quantisation."""
+    wg, wu, wd = recipes.host_expert(cfg, e)
+    qg, sg = of8.quantize_weight_128x128(np.concatenate([wg, wu]).astype(np.float32))
+    qd, sd = of8.quantize_weight_128x128(wd.astype(np.float32))
+    gu = of8.dequant_weight(qg, sg)
+    return gu[:cfg.inter], gu[cfg.inter:], of8.dequant_weight(qd, sd)
+
+
+def test_v3_fp8_sweep_full():
+    """The FP8 layer at T = 256, 2048, 16384 and 65536.  The weights are the
+    same at every T, so the GPU layers run first and keep their sampled rows;
+    then one pass over the experts prepares each expert once (a thread pool,
+    the contributions summed in expert order) for all four samples."""
+    from concurrent.futures import ThreadPoolExecutor
+    samples = []
+    for T in recipes.FP8_SWEEP_T:
+        cfg = C["v3_fp8"].with_T(T)
+        inp = recipes.device_inputs(cfg, "cuda")
+        E, I, d = cfg.n_experts, cfg.inter, cfg.d
+        gq = torch.empty(E, 2 * I, d, dtype=torch.uint8, device="cuda")
+        gs = torch.empty(E, 2 * I // 128, d // 128, dtype=torch.float32, device="cuda")
+        dq = torch.empty(E, d, I, dtype=torch.uint8, device="cuda")
+        ds = torch.empty(E, d // 128, I // 128, dtype=torch.float32, device="cuda")
+        moe.moe_quantize_fp8_blockwise(inp["w_gu"], 2 * I, d, E, gq, gs)
+        moe.moe_quantize_fp8_blockwise(inp["w_down"], d, I, E, dq, ds)
+        inp.update(w_gu=gq, w_gu_scale=gs, w_down=dq, w_down_scale=ds)
+        torch.cuda.synchronize()
+        h, idx, counts, perm = forward(cfg, inp, want_perm=True)
+        h_moe, _, _, _ = forward(cfg, inp, x_res=torch.zeros_like(inp["x"]))
+        host = HostLayer(cfg)
+        ref = host.route()
+        g_idx = idx.cpu().numpy().astype(np.int64)
+        g_counts = counts.cpu().numpy()
+        desc = moe.desc_from_config(cfg)
+        ws = moe.workspace(desc)
+        w2 = torch.empty(cfg.T, cfg.top_k, dtype=torch.float32, device="cuda")
+        moe.moe_route(desc, inp["x"], inp["w_r"], inp["bias"], torch.empty_like(idx), w2,
+                      torch.empty_like(counts), ws)
+        ties = check_routing(cfg, ref, g_idx, w2.cpu().numpy().astype(np.float64), g_counts)
+        _, offsets, perm_src, slot_of = mo.permutation(g_idx, cfg.n_routed)
+        assert np.array_equal(perm[0], offsets)
+        assert np.array_equal(perm[1], perm_src) and np.array_equal(perm[2], slot_of)
+        toks = sample_tokens(cfg, g_idx, g_counts, offsets, perm_src, 256)
+        xs = host.x[toks]
+        q, sc = of8.quantize_act_1x128(xs.astype(np.float32))
+        samples.append(dict(cfg=cfg, toks=toks, xs=xs, xq=of8.dequant_act(q, sc),
+                            idx=g_idx[toks],
+                            w=mo.gate_weights(ref["s"], g_idx, cfg.renorm, cfg.route_scale)[toks],
+                            h=f64(h)[toks], h_moe=f64(h_moe)[toks], ties=len(ties)))
+        del inp, gq, dq, ws, h, h_moe
+        torch.cuda.empty_cache()
+    cfg0 = samples[0]["cfg"]
+    Ks = cfg0.n_shared
+    needed = sorted(set(range(Ks)) | {Ks + int(j) for sm in samples for j in np.unique(sm["idx"])})
+
+    def contributions(e):
+        """(FP8-emulated, unquantised) MoE-part contributions of expert e to each sample."""
+        wq = fp8_expert(cfg0, e)
+        wp = recipes.host_expert(cfg0, e)
+        out = []
+        for sm in samples:
+            if e < Ks:
+                rows, g = np.arange(len(sm["toks"])), np.ones(len(sm["toks"]))
+            else:
+                rows, ks = np.nonzero(sm["idx"] == e - Ks)
+                g = sm["w"][rows, ks]
+            if len(rows) == 0:
+                out.append(None)
+                continue
+            cq = g[:, None] * of8.fp8_swiglu_ffn(sm["xq"][rows], *wq)
+            cp = g[:, None] * mo.swiglu_ffn(sm["xs"][rows], *wp)
+            out.append((rows, cq, cp))
+        return e, out
+
+    acc_q = [np.zeros_like(sm["xs"]) for sm in samples]
+    acc_p = [np.zeros_like(sm["xs"]) for sm in samples]
+    with ThreadPoolExecutor(max_workers=6) as pool:
+        results = dict(pool.map(contributions, needed))
+    for e in needed:                          # fixed summation order
+        for i, r in enumerate(results[e]):
+            if r is not None:
+                rows, cq, cp = r
+                acc_q[i][rows] += cq
+                acc_p[i][rows] += cp
+    for i, sm in enumerate(samples):
+        err = mo.max_abs_rel(sm["h"], sm["xs"] + acc_q[i])
+        err_d = mo.max_abs_rel(sm["h_moe"], acc_q[i])
+        err_plain = mo.max_abs_rel(sm["h_moe"], acc_p[i])
+        print(f"{sm['cfg'].name}: {len(sm['toks'])} sampled tokens, h {err:.3e}, MoE part "
+              f"{err_d:.3e}, vs the unquantised layer {err_plain:.3e}, near-ties {sm['ties']}")
+        assert err <= TOL["e4m3"] and err_d <= TOL["e4m3"]
+        assert err_plain <= 2.0 ** -3

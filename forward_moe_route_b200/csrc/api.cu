@@ -320,6 +320,16 @@ moe_status launch_router(const Dims& D, const void* x, const void* w_router, flo
                       gemm8::smem_bytes(stages, 1), st, ta, tb, a);
 }
 
+// The per-chunk histogram scan, with 16-byte loads along the rows when N % 4 == 0.
+moe_status launch_scan(cudaStream_t st, int32_t* hist, int n_chunks, int N,
+                       const int32_t* counts, int32_t* counts_out, int32_t* offsets) {
+  if (N % 4 == 0)
+    return launch_chain("k_scan", perm::k_scan<4>, dim3(1), dim3(1024), 0, st, hist, n_chunks, N,
+                        counts, counts_out, offsets);
+  return launch_chain("k_scan", perm::k_scan<1>, dim3(1), dim3(1024), 0, st, hist, n_chunks, N,
+                      counts, counts_out, offsets);
+}
+
 // Selection and gate weights.  With counts != nullptr the tokens per expert
 // are counted too: the per-chunk histogram and its totals (k_hist, k_scan),
 // which the layer forward instead takes from its permutation step.
@@ -359,7 +369,7 @@ moe_status do_route(const moe_layer_desc& s, const Dims& D, const Layout& L, con
   rc = launch_chain("k_hist", perm::k_hist, dim3(D.n_chunks), dim3(256), N * 4, st,
                     static_cast<const int32_t*>(topk_idx), T, K, N, hist);
   if (rc == MOE_OK)
-    rc = launch_chain("k_scan", perm::k_scan, dim3(1), dim3(1024), 0, st, hist, (int)D.n_chunks,
+    rc = launch_scan(st, hist, (int)D.n_chunks,
                       N, static_cast<const int32_t*>(nullptr), counts, offsets);
   return rc;
 }
@@ -385,7 +395,7 @@ moe_status do_permute(const Dims& D, int32_t* hist, const void* x, const int32_t
   moe_status rc = launch_chain("k_hist", perm::k_hist, dim3(D.n_chunks), dim3(256), N * 4, st,
                                topk_idx, T, K, N, hist);
   if (rc == MOE_OK)
-    rc = launch_chain("k_scan", perm::k_scan, dim3(1), dim3(1024), 0, st, hist, (int)D.n_chunks,
+    rc = launch_scan(st, hist, (int)D.n_chunks,
                       N, counts, counts_out, offsets);
   if (rc == MOE_OK)
     rc = launch_chain("k_slots", perm::k_slots, dim3(D.n_chunks), dim3(perm::SLOT_WARPS * 32),
@@ -885,7 +895,7 @@ moe_status do_backward(const moe_layer_desc& s, const Dims& D, const Layout& L,
   rc = launch_chain("k_hist", perm::k_hist, dim3(D.n_chunks), dim3(256), N * 4, st,
                     static_cast<const int32_t*>(idx), T, K, N, hist);
   if (rc == MOE_OK)
-    rc = launch_chain("k_scan", perm::k_scan, dim3(1), dim3(1024), 0, st, hist, (int)D.n_chunks,
+    rc = launch_scan(st, hist, (int)D.n_chunks,
                       N, static_cast<const int32_t*>(nullptr), counts, offsets);
   if (rc == MOE_OK)
     rc = launch_chain("k_slots", perm::k_slots, dim3(D.n_chunks), dim3(perm::SLOT_WARPS * 32),

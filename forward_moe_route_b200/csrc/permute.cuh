@@ -9,6 +9,8 @@
 // identical from run to run.
 #pragma once
 
+#include <type_traits>
+
 #include "common.cuh"
 #include "gemm.cuh"
 
@@ -39,43 +41,76 @@ __global__ void __launch_bounds__(256) k_hist(const int32_t* __restrict__ idx, i
 // expert (offsets[e] + pairs of expert e in earlier chunks), writes offsets
 // [N+1], and checks the per-expert totals against `counts` (when given) or
 // writes them to `counts_out` (when given).
+//
+// Thread (q, part) owns experts 4q..4q+3 (16-byte loads along a histogram row;
+// N % 4 == 0, else one expert per thread) and a contiguous run of chunks; runs
+// of up to SCAN_REG chunks stay in registers, so the histogram is read once
+// and written once.
+constexpr int SCAN_REG = 8;
+
+template <int V>
 __global__ void __launch_bounds__(1024) k_scan(int32_t* __restrict__ hist, int n_chunks, int N,
                                                const int32_t* __restrict__ counts,
                                                int32_t* __restrict__ counts_out,
                                                int32_t* __restrict__ offsets) {
   grid_dep_sync();
-  __shared__ int32_t part_sum[1024];
-  __shared__ int32_t tot[1024];
+  __shared__ int32_t part_sum[1024 * V];   // [part][expert]
+  __shared__ int32_t tot[512];
   __shared__ int32_t warp_tot[32];
-  const int P = max(1, (int)(blockDim.x / N));  // parts per expert
+  using vec_t = typename std::conditional<V == 4, int4, int>::type;
+  const int groups = (N + V - 1) / V;                      // expert groups of V
+  const int P = max(1, (int)(blockDim.x / groups));        // parts per group
   const int tid = threadIdx.x;
-  const int e = tid % N, part = tid / N;
-  const bool active = part < P && tid < N * P;
+  const int q = tid % groups, part = tid / groups;
+  const bool active = part < P && tid < groups * P;
   const int per = (n_chunks + P - 1) / P;
   const int c0 = part * per, c1 = min(n_chunks, c0 + per);
-  int sum = 0;
+  auto load = [&](int c) -> vec_t { return *reinterpret_cast<const vec_t*>(hist + (size_t)c * N + q * V); };
+  auto store = [&](int c, vec_t v) { *reinterpret_cast<vec_t*>(hist + (size_t)c * N + q * V) = v; };
+  auto lane_of = [&](const vec_t& v, int i) -> int {
+    if constexpr (V == 4) return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
+    else return v;
+  };
+  vec_t reg[SCAN_REG];
+  const bool in_regs = c1 - c0 <= SCAN_REG;
+  int sum[V];
+#pragma unroll
+  for (int i = 0; i < V; ++i) sum[i] = 0;
   if (active) {
+    if (in_regs) {
+#pragma unroll
+      for (int j = 0; j < SCAN_REG; ++j)
+        if (c0 + j < c1) reg[j] = load(c0 + j);
+#pragma unroll
+      for (int j = 0; j < SCAN_REG; ++j)
+        if (c0 + j < c1) {
+#pragma unroll
+          for (int i = 0; i < V; ++i) sum[i] += lane_of(reg[j], i);
+        }
+    } else {
 #pragma unroll 8
-    for (int c = c0; c < c1; ++c) sum += hist[(size_t)c * N + e];
-    part_sum[tid] = sum;
-  }
-  __syncthreads();
-  // exclusive prefix over parts, and expert totals
-  int before = 0;
-  if (active) {
-    for (int q = 0; q < part; ++q) before += part_sum[q * N + e];
-    if (part == 0) {
-      int total = 0;
-      for (int q = 0; q < P; ++q) total += part_sum[q * N + e];
-      tot[e] = total;
-      if (counts && counts[e] != total) set_status(MOE_ERR_DEVICE_CHECK);
-      if (counts_out) counts_out[e] = total;
+      for (int c = c0; c < c1; ++c) {
+        const vec_t v = load(c);
+#pragma unroll
+        for (int i = 0; i < V; ++i) sum[i] += lane_of(v, i);
+      }
     }
+#pragma unroll
+    for (int i = 0; i < V; ++i) part_sum[part * groups * V + q * V + i] = sum[i];
   }
   __syncthreads();
-  // exclusive scan of tot[0..N) -> offsets (warp scans + scan of warp totals)
-  int v = (tid < N) ? tot[tid] : 0;
-  int incl = v;
+  // expert totals (parts in order) and the check against counts
+  for (int e = tid; e < N; e += blockDim.x) {
+    int total = 0;
+    for (int pp = 0; pp < P; ++pp) total += part_sum[pp * groups * V + e];
+    tot[e] = total;
+    if (counts && counts[e] != total) set_status(MOE_ERR_DEVICE_CHECK);
+    if (counts_out) counts_out[e] = total;
+  }
+  __syncthreads();
+  // exclusive scan of tot[0..N) -> offsets (N <= 512: two elements a thread at most)
+  const int v0 = tid < N ? tot[tid] : 0;
+  int incl = v0;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
     const int y = __shfl_up_sync(0xffffffffu, incl, o);
@@ -84,7 +119,7 @@ __global__ void __launch_bounds__(1024) k_scan(int32_t* __restrict__ hist, int n
   if (lane_id() == 31) warp_tot[warp_id()] = incl;
   __syncthreads();
   if (warp_id() == 0) {
-    int wv = warp_tot[lane_id()];
+    const int wv = warp_tot[lane_id()];
     int wi = wv;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -94,22 +129,42 @@ __global__ void __launch_bounds__(1024) k_scan(int32_t* __restrict__ hist, int n
     warp_tot[lane_id()] = wi - wv;
   }
   __syncthreads();
-  const int excl = incl - v + warp_tot[warp_id()];
+  const int excl = incl - v0 + warp_tot[warp_id()];
   __syncthreads();
   if (tid < N) {
     offsets[tid] = excl;
-    part_sum[tid] = excl;  // reuse as expert base
-    if (tid == N - 1) offsets[N] = excl + v;
+    if (tid == N - 1) offsets[N] = excl + v0;
+    tot[tid] = excl;                       // now the expert's first row
   }
   __syncthreads();
+  // each part's first row per expert: the expert base plus the earlier parts
   if (active) {
-    int run = part_sum[e] + before;
-    // note: part_sum[e] now holds offsets[e] for e < N (all parts read it)
+    int run[V];
+#pragma unroll
+    for (int i = 0; i < V; ++i) {
+      const int e = q * V + i;
+      int r = e < N ? tot[e] : 0;
+      for (int pp = 0; pp < part; ++pp) r += part_sum[pp * groups * V + e];
+      run[i] = r;
+    }
+    auto emit = [&](int c, const vec_t& h) {
+      vec_t o;
+      if constexpr (V == 4) {
+        o.x = run[0]; o.y = run[1]; o.z = run[2]; o.w = run[3];
+        run[0] += h.x; run[1] += h.y; run[2] += h.z; run[3] += h.w;
+      } else {
+        o = run[0];
+        run[0] += h;
+      }
+      store(c, o);
+    };
+    if (in_regs) {
+#pragma unroll
+      for (int j = 0; j < SCAN_REG; ++j)
+        if (c0 + j < c1) emit(c0 + j, reg[j]);
+    } else {
 #pragma unroll 8
-    for (int c = c0; c < c1; ++c) {
-      const int h = hist[(size_t)c * N + e];
-      hist[(size_t)c * N + e] = run;
-      run += h;
+      for (int c = c0; c < c1; ++c) emit(c, load(c));
     }
   }
 }

@@ -81,8 +81,13 @@ struct Args {
   int K, Ks;
 };
 
+// fp32 epilogue staging: per epilogue warp a 32 x 32 block with rows padded
+// to 33 floats (lane l writes row l column by column without bank conflicts)
+constexpr int XPOSE_FLOATS = 32 * 33;
+constexpr uint32_t XPOSE_BYTES = 4 * XPOSE_FLOATS * 4;
+
 __host__ inline size_t smem_bytes(int stages, int n_probs) {
-  return 1024 + (size_t)stages * STAGE_BYTES + (size_t)(2 * stages + 5) * 8 + 16 +
+  return 1024 + (size_t)stages * STAGE_BYTES + XPOSE_BYTES + (size_t)(2 * stages + 5) * 8 + 16 +
          (size_t)(n_probs + 1) * 4 + 64;
 }
 
@@ -109,7 +114,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   const int S = a.stages;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)S * STAGE_BYTES);
+  float* xpose = reinterpret_cast<float*>(smem + (size_t)S * STAGE_BYTES);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)S * STAGE_BYTES + XPOSE_BYTES);
   uint64_t* empty = full + S;
   uint64_t* tfull = empty + S;
   uint64_t* tempty = tfull + 2;
@@ -287,27 +293,47 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const bool valid = row < m;
       const bool zero_row = !valid && row < mpad;
       if (EPI == EPI_F32) {
-        float* out = reinterpret_cast<float*>(a.c) + crow * a.ldc + col0;
+        // Per 32-column chunk: the warp's 32 rows x 32 columns go through a
+        // padded shared block, then each store instruction writes 4 rows x
+        // 128 contiguous bytes (8 lanes a row), whole lines instead of one
+        // 16-byte piece per row.
+        float* xb = xpose + q * XPOSE_FLOATS;
+        const int rb = mt * BM + q * 32;                     // first row of the warp's block
+        const int sub_r = lane >> 3, sub_c = (lane & 7) * 4; // store phase: row in a group of 4, column
 #pragma unroll 1
-        for (int c = 0; c < BN / 16; ++c) {
-          float v[16];
-          tmem_ld16(tb + (uint32_t)(16 * c), v);
-          if (valid && 16 * c < ncol) {
-            if (!has_k) {
+        for (int c = 0; c < BN / 32; ++c) {
+          uint32_t va[16], vb[16];
+          tmem_ld16_nowait(tb + (uint32_t)(32 * c), va);
+          tmem_ld16_nowait(tb + (uint32_t)(32 * c + 16), vb);
+          tmem_wait_ld2(va, vb);
+          if (32 * c >= ncol) continue;                      // warp-uniform
 #pragma unroll
-              for (int j = 0; j < 16; ++j) v[j] = 0.f;
-            }
-            if (16 * c + 16 <= ncol) {
+          for (int j = 0; j < 16; ++j) {
+            xb[lane * 33 + j] = has_k ? __uint_as_float(va[j]) : 0.f;
+            xb[lane * 33 + 16 + j] = has_k ? __uint_as_float(vb[j]) : 0.f;
+          }
+          __syncwarp();
 #pragma unroll
-              for (int j = 0; j < 4; ++j)
-                reinterpret_cast<float4*>(out + 16 * c)[j] =
-                    make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
-            } else {
+          for (int g = 0; g < 8; ++g) {
+            const int rr = g * 4 + sub_r;                    // row within the warp's block
+            const int row_g = rb + rr;
+            const int colg = 32 * c + sub_c;
+            if (row_g < m && colg < ncol) {
+              float4 v4 = make_float4(xb[rr * 33 + sub_c], xb[rr * 33 + sub_c + 1],
+                                      xb[rr * 33 + sub_c + 2], xb[rr * 33 + sub_c + 3]);
+              float* dst = reinterpret_cast<float*>(a.c) +
+                           ((long long)p[F_CROW] + row_g) * a.ldc + col0 + colg;
+              if (colg + 4 <= ncol) {
+                *reinterpret_cast<float4*>(dst) = v4;
+              } else {
+                const float e4[4] = {v4.x, v4.y, v4.z, v4.w};
 #pragma unroll
-              for (int j = 0; j < 16; ++j)
-                if (16 * c + j < ncol) out[16 * c + j] = v[j];
+                for (int k = 0; k < 4; ++k)
+                  if (colg + k < ncol) dst[k] = e4[k];
+              }
             }
           }
+          __syncwarp();
         }
       } else if (EPI == EPI_BF16 || EPI == EPI_SCATTER) {
         long long dst_row = crow;

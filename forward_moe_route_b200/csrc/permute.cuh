@@ -59,7 +59,9 @@ __global__ void __launch_bounds__(1024) k_scan(int32_t* __restrict__ hist, int n
   __shared__ int32_t warp_tot[32];
   using vec_t = typename std::conditional<V == 4, int4, int>::type;
   const int groups = (N + V - 1) / V;                      // expert groups of V
-  const int P = max(1, (int)(blockDim.x / groups));        // parts per group
+  // parts per group: as many as the threads allow, but each part covers at
+  // least 4 chunks, since the totals and the part prefix walk the parts serially
+  const int P = max(1, min((int)(blockDim.x / groups), (n_chunks + 3) / 4));
   const int tid = threadIdx.x;
   const int q = tid % groups, part = tid / groups;
   const bool active = part < P && tid < groups * P;

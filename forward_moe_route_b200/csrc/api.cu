@@ -116,8 +116,8 @@ struct DeviceInfo {
   bool attrs_done = false;
   // co-resident 2-CTA clusters of the pair GEMMs (0: gate/up, 1: down), and
   // the dynamic shared memory each count was taken for
-  size_t pair_smem[2] = {0, 0};
-  int pair_clusters[2] = {0, 0};
+  size_t pair_smem[3] = {0, 0, 0};
+  int pair_clusters[3] = {0, 0, 0};
 };
 std::mutex g_mu;
 DeviceInfo g_dev[kMaxDevices];
@@ -849,6 +849,35 @@ moe_status launch_gemm_bwd(const char* what, Operand a0, Operand a1, Operand b0,
                       dim3(gbwd::NUM_THREADS), smem, st, ta0, ta1, tb0, tb1, args);
 }
 
+// The weight-gradient problems on CTA pairs (k_gemm_bwd_pair): 256 x 256 pair
+// tiles, grid = co-resident pairs (capped by the tile count) x 2.
+moe_status launch_gemm_bwd_pair(const char* what, Operand a0, Operand a1, Operand b0, Operand b1,
+                                gbwd::Args args, int64_t pair_tiles_bound, cudaStream_t st) {
+  CUtensorMap ta0, ta1, tb0, tb1;
+  moe_status rc = make_tmap_mn(&ta0, a0.base, a0.inner, a0.rows);
+  if (rc == MOE_OK) rc = make_tmap_mn(&ta1, a1.base, a1.inner, a1.rows);
+  if (rc == MOE_OK) rc = make_tmap_mn(&tb0, b0.base, b0.inner, b0.rows);
+  if (rc == MOE_OK) rc = make_tmap_mn(&tb1, b1.base, b1.inner, b1.rows);
+  if (rc != MOE_OK) return rc;
+  int stages = 0;
+  for (int s = 6; s >= 2 && !stages; --s)
+    if (gbwd::pair_smem_bytes(s, args.n_probs) <= (size_t)kMaxSmem) stages = s;
+  if (!stages) return MOE_ERR_UNSUPPORTED;
+  args.stages = stages;
+  const size_t smem = gbwd::pair_smem_bytes(stages, args.n_probs);
+  cudaError_t e = cudaFuncSetAttribute(gbwd::k_gemm_bwd_pair,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
+  if (e != cudaSuccess) return cuda_fail(e, what);
+  cudaLaunchConfig_t cfg;
+  cudaLaunchAttribute attr[2];
+  rc = pair_config(2, gbwd::k_gemm_bwd_pair, gbwd::NUM_THREADS, smem, pair_tiles_bound, st, &cfg,
+                   attr);
+  if (rc != MOE_OK) return rc;
+  e = cudaLaunchKernelEx(&cfg, gbwd::k_gemm_bwd_pair, ta0, ta1, tb0, tb1, args);
+  if (e != cudaSuccess) return cuda_fail(e, what);
+  return launched(what);
+}
+
 template <int VPL>
 moe_status launch_gate_bwd(const float* logits, const route::Params& p, const int32_t* idx,
                            const int32_t* slot_of, const int32_t* offsets, const int32_t* poff,
@@ -993,26 +1022,23 @@ moe_status do_backward(const moe_layer_desc& s, const Dims& D, const Layout& L,
   ga.tab = tab[3];
   ga.c = dw_down;
   ga.ldc = I;
-  rc = launch_gemm_bwd<true, true, gbwd::EPI_F32>("backward GEMM dW_down = dY^T Z", DH, DHP, ZG,
-                                                   ZG, ga, (int64_t)E * ((d + 127) / 128) * nt(I),
-                                                   sms, st);
+  rc = launch_gemm_bwd_pair("backward GEMM dW_down = dY^T Z (CTA pairs)", DH, DHP, ZG, ZG, ga,
+                            (int64_t)E * ((d + 255) / 256) * nt(I), st);
   if (rc != MOE_OK) return rc;
   // G5: dW_gu = [da | db]^T X over each expert's rows
   ga.tab = tab[4];
   ga.c = dw_gu;
   ga.ldc = d;
-  rc = launch_gemm_bwd<true, true, gbwd::EPI_F32>("backward GEMM dW_gu = dAB^T X", DAB, DAB, X,
-                                                   XP, ga,
-                                                   (int64_t)E * ((2 * I + 127) / 128) * nt(d),
-                                                   sms, st);
+  rc = launch_gemm_bwd_pair("backward GEMM dW_gu = dAB^T X (CTA pairs)", DAB, DAB, X, XP, ga,
+                            (int64_t)E * ((2 * I + 255) / 256) * nt(d), st);
   if (rc != MOE_OK) return rc;
   // G6b: dW_r = dl^T X over all tokens
   ga.n_probs = 1;
   ga.tab = tab[6];
   ga.c = dw_router;
   ga.ldc = d;
-  return launch_gemm_bwd<true, true, gbwd::EPI_F32>("backward GEMM dW_r = dL^T X", DL, DL, X, X,
-                                                     ga, ((N + 127) / 128) * nt(d), sms, st);
+  return launch_gemm_bwd_pair("backward GEMM dW_r = dL^T X (CTA pairs)", DL, DL, X, X, ga,
+                              ((N + 255) / 256) * nt(d), st);
 }
 
 __global__ void k_selftest_wait(uint64_t limit_ns) {

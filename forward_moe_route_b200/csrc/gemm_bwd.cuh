@@ -36,6 +36,7 @@
 
 #include "common.cuh"
 #include "gemm.cuh"
+#include "gemm_t.cuh"
 
 namespace moe {
 namespace gbwd {
@@ -436,6 +437,274 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (warp == 2) {
     tc_fence_after();
     tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+// ----------------------------------------------------------------------------- CTA pairs
+// The weight-gradient problems (both operands MN-major, fp32 output) on CTA
+// pairs: a cluster of two CTAs computes a 256 x 256 tile with one
+// tcgen05.mma.cta_group::2 per K step issued by the even CTA; CTA r loads the
+// A rows [256 mt + 128 r, +128) and the B columns of its half of the tile's N
+// range, and its TMEM receives its 128 rows x the whole N.  Per SM a 64-row K
+// step then moves 32 KB instead of 48 KB for the same tensor-core work: these
+// GEMMs contract over one expert's rows only (~576 at the V3 shape), so the
+// operand stream from L2, not the tensor pipe, sets their pace.
+// Synchronisation as in the forward pair kernels (gemm_t.cuh): full[s] on the
+// leader receives both CTAs' TMA bytes, the leader's MMA commits empty[s] and
+// tfull[a] to both CTAs, both CTAs' epilogue threads arrive on the leader's
+// tempty[a], every wait is bounded and a cluster barrier precedes the TMEM free.
+constexpr int PBM = 256;                 // rows per pair tile (128 per CTA)
+constexpr uint32_t PA_BYTES = 2 * MN_BOX_BYTES;   // a CTA's A: 128 rows of M (2 boxes of 64) x 64 K rows
+constexpr uint32_t PB_BYTES = 2 * MN_BOX_BYTES;   // its half of B: up to 128 columns of N
+constexpr uint32_t PSTAGE_BYTES = PA_BYTES + PB_BYTES;
+
+__host__ inline size_t pair_smem_bytes(int stages, int n_probs) {
+  return 1024 + (size_t)stages * PSTAGE_BYTES + XPOSE_BYTES + (size_t)(2 * stages + 5) * 8 + 16 +
+         (size_t)(n_probs + 1) * 4 + 64;
+}
+
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    k_gemm_bwd_pair(const __grid_constant__ CUtensorMap tmA0,
+                    const __grid_constant__ CUtensorMap tmA1,
+                    const __grid_constant__ CUtensorMap tmB0,
+                    const __grid_constant__ CUtensorMap tmB1, const Args a) {
+  using namespace gemmt;   // cluster helpers of the forward pair kernels
+  grid_dep_sync();
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const int S = a.stages;
+  float* xpose = reinterpret_cast<float*>(smem + (size_t)S * PSTAGE_BYTES);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)S * PSTAGE_BYTES + XPOSE_BYTES);
+  uint64_t* empty = full + S;
+  uint64_t* tfull = empty + S;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* s_prefix = reinterpret_cast<int*>(tmem_slot + 4);
+
+  const int warp = warp_id(), lane = lane_id();
+  const uint32_t rank = cluster_rank();
+  const bool leader = rank == 0;
+  const int np = a.n_probs;
+  if (warp == 0) {
+    int carry = 0;
+    for (int base = 0; base < np; base += 32) {
+      const int g = base + lane;
+      int v = 0;
+      if (g < np) {
+        const int* p = a.tab + (size_t)g * GB_FIELDS;
+        v = ((p[F_M] + PBM - 1) / PBM) * ((p[F_N] + BN - 1) / BN);
+      }
+      int incl = v;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      if (g < np) s_prefix[g] = carry + incl - v;
+      carry += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) s_prefix[np] = carry;
+  }
+  if (threadIdx.x == 32) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int j = 0; j < 2; ++j) {
+      mbar_init(&tfull[j], 1);
+      mbar_init(&tempty[j], 2 * 4 * 32);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    fence_proxy_async_smem();
+    tma_prefetch_desc(&tmA0);
+    tma_prefetch_desc(&tmA1);
+    tma_prefetch_desc(&tmB0);
+    tma_prefetch_desc(&tmB1);
+  }
+  if (warp == 2) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_slot)),
+                 "r"(TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();      // barrier initialisation is visible to the peer from here on
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int total = s_prefix[np];
+  const int pair = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;
+
+  auto locate = [&](int tile, int& mt, int& nt, const int*& p) {
+    const int g = gemm::find_group(s_prefix, np, tile);
+    p = a.tab + (size_t)g * GB_FIELDS;
+    const int ntn = (p[F_N] + BN - 1) / BN;
+    const int lt = tile - s_prefix[g];
+    mt = lt / ntn;
+    nt = lt - mt * ntn;
+  };
+  // the tile's UMMA N (its columns rounded up to 32, so each CTA's half is a
+  // multiple of 16 columns) and this CTA's first column
+  auto tile_cols = [&](const int* p, int nt) {
+    int nc = min(BN, p[F_N] - nt * BN);
+    return (nc + 31) & ~31;
+  };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ TMA producer (both CTAs)
+    if (elect_one()) {
+      int it = 0;
+      bool ok = true;
+      for (int tile = pair; tile < total && ok; tile += n_pairs) {
+        int mt, nt;
+        const int* p;
+        locate(tile, mt, nt, p);
+        const int nkb = (p[F_K] + BK - 1) / BK;
+        const CUtensorMap* tA = p[F_AMAP] ? &tmA1 : &tmA0;
+        const CUtensorMap* tB = p[F_BMAP] ? &tmB1 : &tmB0;
+        const int am = p[F_AM0] + mt * PBM + (int)rank * 128, ak = p[F_AK0];
+        const int bn = p[F_BN0] + nt * BN + (int)rank * (tile_cols(p, nt) / 2), bk = p[F_BK0];
+        for (int kb = 0; kb < nkb; ++kb, ++it) {
+          const int s = it % S;
+          const uint32_t ph = (uint32_t)(it / S) & 1u;
+          if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag)) { ok = false; break; }
+          uint8_t* sa = smem + (size_t)s * PSTAGE_BYTES;
+          uint8_t* sb = sa + PA_BYTES;
+          const uint32_t full_leader = mapa(smem_u32(&full[s]), 0);
+          if (leader) mbar_arrive_expect_tx(&full[s], 2 * PSTAGE_BYTES);
+          const int k0 = ak + kb * BK, kb0 = bk + kb * BK;
+          tma_load_2d_pair(tA, full_leader, sa, am, k0);
+          tma_load_2d_pair(tA, full_leader, sa + MN_BOX_BYTES, am + 64, k0);
+          tma_load_2d_pair(tB, full_leader, sb, bn, kb0);
+          tma_load_2d_pair(tB, full_leader, sb + MN_BOX_BYTES, bn + 64, kb0);
+        }
+      }
+      // the copies this CTA issued land before the block may leave (bounded)
+      volatile int no_abort = 0;
+      for (int j = (it - S > 0 ? it - S : 0); j < it; ++j)
+        mbar_wait(&empty[j % S], (uint32_t)(j / S) & 1u, &no_abort);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer (leader)
+    if (leader && elect_one()) {
+      int it = 0, tcount = 0;
+      bool ok = true;
+      for (int tile = pair; tile < total && ok; tile += n_pairs, ++tcount) {
+        int mt, nt;
+        const int* p;
+        locate(tile, mt, nt, p);
+        const int nkb = (p[F_K] + BK - 1) / BK;
+        const uint32_t idesc =
+            umma_idesc(1, PBM, tile_cols(p, nt)) | (1u << 15) | (1u << 16);   // A, B MN-major
+        const int acc = tcount & 1;
+        const uint32_t use = (uint32_t)(tcount >> 1);
+        if (!mbar_wait(&tempty[acc], (use & 1u) ^ 1u, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * ACC_COLS);
+        for (int kb = 0; kb < nkb; ++kb, ++it) {
+          const int s = it % S;
+          const uint32_t ph = (uint32_t)(it / S) & 1u;
+          if (!mbar_wait(&full[s], ph, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + (size_t)s * PSTAGE_BYTES);
+          const uint64_t ad = umma_desc_sw128_mn(sa);
+          const uint64_t bd = umma_desc_sw128_mn(sa + PA_BYTES);
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k)
+            umma_pair<0>(d_tmem, ad + (uint64_t)(128 * k), bd + (uint64_t)(128 * k), idesc,
+                         (kb | k) != 0 ? 1u : 0u);
+          const uint32_t e_local = smem_u32(&empty[s]);
+          umma_commit_pair(mapa(e_local, 0));
+          umma_commit_pair(mapa(e_local, 1));
+        }
+        if (ok) {
+          const uint32_t t_local = smem_u32(&tfull[acc]);
+          umma_commit_pair(mapa(t_local, 0));
+          umma_commit_pair(mapa(t_local, 1));
+        }
+      }
+      umma_commit_pair(mapa(smem_u32(drain), 0));
+      volatile int no_abort = 0;
+      mbar_wait(drain, 0, &no_abort);
+    }
+    __syncwarp();
+  } else if (warp >= EPI_WARP0) {
+    // ------------------------------------------------------------------ epilogue (both CTAs)
+    const int q = warp - EPI_WARP0;
+    float* xb = xpose + q * XPOSE_FLOATS;
+    const int sub_r = lane >> 3, sub_c = (lane & 7) * 4;
+    const uint32_t tempty_leader0 = mapa(smem_u32(&tempty[0]), 0);
+    const uint32_t tempty_leader1 = mapa(smem_u32(&tempty[1]), 0);
+    int tcount = 0;
+    for (int tile = pair; tile < total; tile += n_pairs, ++tcount) {
+      int mt, nt;
+      const int* p;
+      locate(tile, mt, nt, p);
+      const int acc = tcount & 1;
+      const uint32_t use = (uint32_t)(tcount >> 1);
+      if (!mbar_wait(&tfull[acc], use & 1u, abort_flag)) break;
+      tc_fence_after();
+      const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * ACC_COLS);
+      const int m = p[F_M];
+      const bool has_k = p[F_K] > 0;
+      const int col0 = nt * BN;
+      const int ncol = min(BN, p[F_N] - col0);
+      const int rb = mt * PBM + (int)rank * 128 + q * 32;   // first row of the warp's block
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t va[16], vb[16];
+        tmem_ld16_nowait(tb + (uint32_t)(32 * c), va);
+        tmem_ld16_nowait(tb + (uint32_t)(32 * c + 16), vb);
+        tmem_wait_ld2(va, vb);
+        if (32 * c >= ncol) continue;                      // warp-uniform
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          xb[lane * 33 + j] = has_k ? __uint_as_float(va[j]) : 0.f;
+          xb[lane * 33 + 16 + j] = has_k ? __uint_as_float(vb[j]) : 0.f;
+        }
+        __syncwarp();
+#pragma unroll
+        for (int g = 0; g < 8; ++g) {
+          const int rr = g * 4 + sub_r;
+          const int row_g = rb + rr;
+          const int colg = 32 * c + sub_c;
+          if (row_g < m && colg < ncol) {
+            const float4 v4 = make_float4(xb[rr * 33 + sub_c], xb[rr * 33 + sub_c + 1],
+                                          xb[rr * 33 + sub_c + 2], xb[rr * 33 + sub_c + 3]);
+            float* dst = reinterpret_cast<float*>(a.c) +
+                         ((long long)p[F_CROW] + row_g) * a.ldc + col0 + colg;
+            if (colg + 4 <= ncol) {
+              *reinterpret_cast<float4*>(dst) = v4;
+            } else {
+              const float e4[4] = {v4.x, v4.y, v4.z, v4.w};
+#pragma unroll
+              for (int k = 0; k < 4; ++k)
+                if (colg + k < ncol) dst[k] = e4[k];
+            }
+          }
+        }
+        __syncwarp();
+      }
+      tc_fence_before();
+      if (leader) mbar_arrive(&tempty[acc]);
+      else mbar_arrive_cluster(acc ? tempty_leader1 : tempty_leader0);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();      // the peer no longer touches this CTA's barriers or TMEM
+  if (warp == 2) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                 "r"(TMEM_COLS)
+                 : "memory");
   }
 }
 

@@ -849,15 +849,44 @@ moe_status launch_gemm_bwd(const char* what, Operand a0, Operand a1, Operand b0,
                       dim3(gbwd::NUM_THREADS), smem, st, ta0, ta1, tb0, tb1, args);
 }
 
+// Output map of the weight-gradient GEMMs: fp32 [nz][m][ldc], box 32 x 32 x 1,
+// 128-byte swizzle (the epilogue's staging layout).  Rows are one expert's,
+// so a TMA store clips at the expert's last row and at the row's end.
+moe_status make_tmap_out(CUtensorMap* mp, void* base, uint64_t ldc, uint64_t m, uint64_t nz) {
+  if (ldc % 4 != 0 || m == 0 || nz == 0) {
+    snprintf(t_errmsg, sizeof(t_errmsg), "weight-gradient output map: row length %llu must be a "
+             "multiple of 4", (unsigned long long)ldc);
+    return MOE_ERR_UNSUPPORTED;
+  }
+  cuuint64_t dims[3] = {ldc, m, nz};
+  cuuint64_t strides[2] = {ldc * 4, m * ldc * 4};
+  cuuint32_t box[3] = {32, 32, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = g_encode(mp, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    snprintf(t_errmsg, sizeof(t_errmsg), "cuTensorMapEncodeTiled (gradient output): CUresult %d "
+             "(row %llu, rows %llu, experts %llu)", (int)r, (unsigned long long)ldc,
+             (unsigned long long)m, (unsigned long long)nz);
+    return MOE_ERR_CUDA;
+  }
+  return MOE_OK;
+}
+
 // The weight-gradient problems on CTA pairs (k_gemm_bwd_pair): 256 x 256 pair
-// tiles, grid = co-resident pairs (capped by the tile count) x 2.
+// tiles, grid = co-resident pairs (capped by the tile count) x 2.  Every
+// problem's output is the expert's block crow = e * m_rows of args.c with N =
+// args.ldc columns; the epilogue stores through a [n_z][m_rows][ldc] map.
 moe_status launch_gemm_bwd_pair(const char* what, Operand a0, Operand a1, Operand b0, Operand b1,
-                                gbwd::Args args, int64_t pair_tiles_bound, cudaStream_t st) {
-  CUtensorMap ta0, ta1, tb0, tb1;
+                                gbwd::Args args, uint64_t m_rows, uint64_t n_z,
+                                int64_t pair_tiles_bound, cudaStream_t st) {
+  CUtensorMap ta0, ta1, tb0, tb1, tc;
   moe_status rc = make_tmap_mn(&ta0, a0.base, a0.inner, a0.rows);
   if (rc == MOE_OK) rc = make_tmap_mn(&ta1, a1.base, a1.inner, a1.rows);
   if (rc == MOE_OK) rc = make_tmap_mn(&tb0, b0.base, b0.inner, b0.rows);
   if (rc == MOE_OK) rc = make_tmap_mn(&tb1, b1.base, b1.inner, b1.rows);
+  if (rc == MOE_OK) rc = make_tmap_out(&tc, args.c, (uint64_t)args.ldc, m_rows, n_z);
   if (rc != MOE_OK) return rc;
   int stages = 0;
   for (int s = 6; s >= 2 && !stages; --s)
@@ -873,7 +902,7 @@ moe_status launch_gemm_bwd_pair(const char* what, Operand a0, Operand a1, Operan
   rc = pair_config(2, gbwd::k_gemm_bwd_pair, gbwd::NUM_THREADS, smem, pair_tiles_bound, st, &cfg,
                    attr);
   if (rc != MOE_OK) return rc;
-  e = cudaLaunchKernelEx(&cfg, gbwd::k_gemm_bwd_pair, ta0, ta1, tb0, tb1, args);
+  e = cudaLaunchKernelEx(&cfg, gbwd::k_gemm_bwd_pair, ta0, ta1, tb0, tb1, tc, args);
   if (e != cudaSuccess) return cuda_fail(e, what);
   return launched(what);
 }
@@ -1023,13 +1052,14 @@ moe_status do_backward(const moe_layer_desc& s, const Dims& D, const Layout& L,
   ga.c = dw_down;
   ga.ldc = I;
   rc = launch_gemm_bwd_pair("backward GEMM dW_down = dY^T Z (CTA pairs)", DH, DHP, ZG, ZG, ga,
-                            (int64_t)E * ((d + 255) / 256) * nt(I), st);
+                            (uint64_t)d, (uint64_t)E, (int64_t)E * ((d + 255) / 256) * nt(I), st);
   if (rc != MOE_OK) return rc;
   // G5: dW_gu = [da | db]^T X over each expert's rows
   ga.tab = tab[4];
   ga.c = dw_gu;
   ga.ldc = d;
   rc = launch_gemm_bwd_pair("backward GEMM dW_gu = dAB^T X (CTA pairs)", DAB, DAB, X, XP, ga,
+                            (uint64_t)(2 * I), (uint64_t)E,
                             (int64_t)E * ((2 * I + 255) / 256) * nt(d), st);
   if (rc != MOE_OK) return rc;
   // G6b: dW_r = dl^T X over all tokens
@@ -1038,7 +1068,7 @@ moe_status do_backward(const moe_layer_desc& s, const Dims& D, const Layout& L,
   ga.c = dw_router;
   ga.ldc = d;
   return launch_gemm_bwd_pair("backward GEMM dW_r = dL^T X (CTA pairs)", DL, DL, X, X, ga,
-                              ((N + 255) / 256) * nt(d), st);
+                              (uint64_t)N, 1, ((N + 255) / 256) * nt(d), st);
 }
 
 __global__ void k_selftest_wait(uint64_t limit_ns) {

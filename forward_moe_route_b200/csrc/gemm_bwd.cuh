@@ -457,25 +457,51 @@ constexpr int PBM = 256;                 // rows per pair tile (128 per CTA)
 constexpr uint32_t PA_BYTES = 2 * MN_BOX_BYTES;   // a CTA's A: 128 rows of M (2 boxes of 64) x 64 K rows
 constexpr uint32_t PB_BYTES = 2 * MN_BOX_BYTES;   // its half of B: up to 128 columns of N
 constexpr uint32_t PSTAGE_BYTES = PA_BYTES + PB_BYTES;
+// fp32 store staging: per epilogue warp two 32 x 32 blocks (4 KB each) in the
+// 128-byte-swizzled layout of the output tensor map, written out by TMA
+constexpr uint32_t PSTORE_BYTES = 4 * 2 * 4096;
 
 __host__ inline size_t pair_smem_bytes(int stages, int n_probs) {
-  return 1024 + (size_t)stages * PSTAGE_BYTES + XPOSE_BYTES + (size_t)(2 * stages + 5) * 8 + 16 +
+  return 1024 + (size_t)stages * PSTAGE_BYTES + PSTORE_BYTES + (size_t)(2 * stages + 5) * 8 + 16 +
          (size_t)(n_probs + 1) * 4 + 64;
+}
+
+// TMA store of one 32 x 32 fp32 block (the tensor map's box) from shared
+// memory, completion tracked by the thread's bulk async-group.
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void* smem_src, int32_t x,
+                                             int32_t y, int32_t z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+          (uint64_t)map),
+      "r"(smem_u32(smem_src)), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_commit_group() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// at most N of this thread's bulk groups still reading shared memory
+template <int N>
+__device__ __forceinline__ void bulk_wait_group_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ void bulk_wait_group_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     k_gemm_bwd_pair(const __grid_constant__ CUtensorMap tmA0,
                     const __grid_constant__ CUtensorMap tmA1,
                     const __grid_constant__ CUtensorMap tmB0,
-                    const __grid_constant__ CUtensorMap tmB1, const Args a) {
+                    const __grid_constant__ CUtensorMap tmB1,
+                    const __grid_constant__ CUtensorMap tmC, const Args a) {
   using namespace gemmt;   // cluster helpers of the forward pair kernels
   grid_dep_sync();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   const int S = a.stages;
-  float* xpose = reinterpret_cast<float*>(smem + (size_t)S * PSTAGE_BYTES);
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)S * PSTAGE_BYTES + XPOSE_BYTES);
+  uint8_t* store_buf = smem + (size_t)S * PSTAGE_BYTES;     // 1024-byte aligned
+  uint64_t* full = reinterpret_cast<uint64_t*>(store_buf + PSTORE_BYTES);
   uint64_t* empty = full + S;
   uint64_t* tfull = empty + S;
   uint64_t* tempty = tfull + 2;
@@ -525,6 +551,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     tma_prefetch_desc(&tmA1);
     tma_prefetch_desc(&tmB0);
     tma_prefetch_desc(&tmB1);
+    tma_prefetch_desc(&tmC);
   }
   if (warp == 2) {
     asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
@@ -637,12 +664,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     __syncwarp();
   } else if (warp >= EPI_WARP0) {
     // ------------------------------------------------------------------ epilogue (both CTAs)
+    // Warp q owns TMEM lanes 32q .. 32q+31 (output rows); per 32-column chunk
+    // it writes the block into one of its two swizzled staging buffers and
+    // one lane stores it with TMA.  The output map's rows are one expert's
+    // (m) and its columns the full row (N = ldc), so the store clips the
+    // tile's edges itself.
     const int q = warp - EPI_WARP0;
-    float* xb = xpose + q * XPOSE_FLOATS;
-    const int sub_r = lane >> 3, sub_c = (lane & 7) * 4;
+    uint8_t* stg = store_buf + (size_t)q * 2 * 4096;
     const uint32_t tempty_leader0 = mapa(smem_u32(&tempty[0]), 0);
     const uint32_t tempty_leader1 = mapa(smem_u32(&tempty[1]), 0);
-    int tcount = 0;
+    int tcount = 0, nst = 0;
     for (int tile = pair; tile < total; tile += n_pairs, ++tcount) {
       int mt, nt;
       const int* p;
@@ -655,47 +686,50 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const int m = p[F_M];
       const bool has_k = p[F_K] > 0;
       const int col0 = nt * BN;
-      const int ncol = min(BN, p[F_N] - col0);
-      const int rb = mt * PBM + (int)rank * 128 + q * 32;   // first row of the warp's block
+      const int nc = (min(BN, p[F_N] - col0) + 31) >> 5;    // 32-column chunks with data
+      const int row0 = mt * PBM + (int)rank * 128 + q * 32;  // first row (within m) of the warp
+      const int z = m > 0 ? p[F_CROW] / m : 0;
+      const int nchunks = row0 < m ? nc : 0;
+      if (nchunks == 0) {
+        tc_fence_before();
+        if (leader) mbar_arrive(&tempty[acc]);
+        else mbar_arrive_cluster(acc ? tempty_leader1 : tempty_leader0);
+        continue;
+      }
 #pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
+      for (int c = 0; c < nchunks; ++c, ++nst) {
         uint32_t va[16], vb[16];
         tmem_ld16_nowait(tb + (uint32_t)(32 * c), va);
         tmem_ld16_nowait(tb + (uint32_t)(32 * c + 16), vb);
         tmem_wait_ld2(va, vb);
-        if (32 * c >= ncol) continue;                      // warp-uniform
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          xb[lane * 33 + j] = has_k ? __uint_as_float(va[j]) : 0.f;
-          xb[lane * 33 + 16 + j] = has_k ? __uint_as_float(vb[j]) : 0.f;
+        if (c == nchunks - 1) {
+          // the warp's last TMEM read of the tile: hand the accumulator back
+          tc_fence_before();
+          if (leader) mbar_arrive(&tempty[acc]);
+          else mbar_arrive_cluster(acc ? tempty_leader1 : tempty_leader0);
         }
+        uint8_t* buf = stg + (size_t)(nst & 1) * 4096;
+        // the store issued from this buffer two chunks ago has read it
+        if (lane == 0) bulk_wait_group_read<1>();
         __syncwarp();
+        // row `lane`, 16-byte piece j at (j ^ (row % 8)) (128-byte swizzle)
 #pragma unroll
-        for (int g = 0; g < 8; ++g) {
-          const int rr = g * 4 + sub_r;
-          const int row_g = rb + rr;
-          const int colg = 32 * c + sub_c;
-          if (row_g < m && colg < ncol) {
-            const float4 v4 = make_float4(xb[rr * 33 + sub_c], xb[rr * 33 + sub_c + 1],
-                                          xb[rr * 33 + sub_c + 2], xb[rr * 33 + sub_c + 3]);
-            float* dst = reinterpret_cast<float*>(a.c) +
-                         ((long long)p[F_CROW] + row_g) * a.ldc + col0 + colg;
-            if (colg + 4 <= ncol) {
-              *reinterpret_cast<float4*>(dst) = v4;
-            } else {
-              const float e4[4] = {v4.x, v4.y, v4.z, v4.w};
-#pragma unroll
-              for (int k = 0; k < 4; ++k)
-                if (colg + k < ncol) dst[k] = e4[k];
-            }
-          }
+        for (int j = 0; j < 8; ++j) {
+          const uint32_t* src = j < 4 ? &va[4 * j] : &vb[4 * (j - 4)];
+          const uint4 v = has_k ? make_uint4(src[0], src[1], src[2], src[3])
+                                : make_uint4(0u, 0u, 0u, 0u);
+          *reinterpret_cast<uint4*>(buf + lane * 128 + ((j ^ (lane & 7)) << 4)) = v;
         }
+        fence_proxy_async_smem();
         __syncwarp();
+        if (lane == 0) {
+          tma_store_3d(&tmC, buf, col0 + 32 * c, row0, z);
+          bulk_commit_group();
+        }
       }
-      tc_fence_before();
-      if (leader) mbar_arrive(&tempty[acc]);
-      else mbar_arrive_cluster(acc ? tempty_leader1 : tempty_leader0);
     }
+    if (lane == 0) bulk_wait_group_all();
+    __syncwarp();
   }
   tc_fence_before();
   __syncthreads();

@@ -94,6 +94,100 @@ __host__ inline size_t smem_bytes(int stages, int n_groups) {
          2 * 4 * BM * sizeof(float) + (size_t)(n_groups + 1) * 4 + 64;
 }
 
+// ----------------------------------------------------------------------------- shared pieces
+// Promotion of one k-block partial into the warp's 64 accumulator columns:
+// acc[0..31] += m0 * P[col0 .. col0+31], acc[32..63] += m1 * P[col0+32 ..],
+// two batches of two 16-column TMEM loads (tb already points at col0).
+__device__ __forceinline__ void promote64(uint32_t tb, float (&acc)[64], float m0, float m1) {
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    uint32_t va[16], vb[16];
+    tmem_ld16_nowait(tb + (uint32_t)(32 * h), va);
+    tmem_ld16_nowait(tb + (uint32_t)(32 * h + 16), vb);
+    tmem_wait_ld2(va, vb);
+    const float m = h == 0 ? m0 : m1;
+    const float2 mm = make_float2(m, m);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int o = 32 * h + 2 * i;
+      const float2 r = __ffma2_rn(mm, make_float2(__uint_as_float(va[2 * i]),
+                                                  __uint_as_float(va[2 * i + 1])),
+                                  make_float2(acc[o], acc[o + 1]));
+      acc[o] = r.x;
+      acc[o + 1] = r.y;
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int o = 32 * h + 16 + 2 * i;
+      const float2 r = __ffma2_rn(mm, make_float2(__uint_as_float(vb[2 * i]),
+                                                  __uint_as_float(vb[2 * i + 1])),
+                                  make_float2(acc[o], acc[o + 1]));
+      acc[o] = r.x;
+      acc[o + 1] = r.y;
+    }
+  }
+}
+
+// GEMM1 epilogue of one row's 64-column slice cs (gate columns 0..31, the
+// matching up columns 32..63): H = SiLU(gate) * up, the row's 1x128 amax over
+// the four slices through shared memory (xbar, bounded), E4M3 codes and the
+// fp32 tile scale.  Returns false when the exchange wait gave up.
+__device__ __forceinline__ bool epi_swiglu_q(float (&acc)[64], const Args& a, float* amax_buf,
+                                             uint64_t* xbar, int tcount, int cs, int r, bool valid,
+                                             size_t hrow, int nt, volatile int* abort_flag) {
+  float pam = 0.f;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    acc[i] = gemm::silu_f(acc[i]) * acc[32 + i];
+    pam = fmaxf(pam, fabsf(acc[i]));
+  }
+  float* ab = amax_buf + (tcount & 1) * 4 * BM;
+  ab[cs * BM + r] = pam;
+  mbar_arrive(xbar);
+  if (!mbar_wait(xbar, (uint32_t)tcount & 1u, abort_flag)) return false;
+  const float amax = fmaxf(fmaxf(ab[r], ab[BM + r]), fmaxf(ab[2 * BM + r], ab[3 * BM + r]));
+  const float scale = amax > 0.f ? __fdiv_rn(amax, 448.0f) : 0.f;
+  const float inv = amax > 0.f ? __fdiv_rn(448.0f, amax) : 0.f;
+  if (valid) {
+    uint32_t w[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      w[j] = (uint32_t)f32_to_e4m3(__fmul_rn(acc[4 * j], inv)) |
+             ((uint32_t)f32_to_e4m3(__fmul_rn(acc[4 * j + 1], inv)) << 8) |
+             ((uint32_t)f32_to_e4m3(__fmul_rn(acc[4 * j + 2], inv)) << 16) |
+             ((uint32_t)f32_to_e4m3(__fmul_rn(acc[4 * j + 3], inv)) << 24);
+    uint4* dst = reinterpret_cast<uint4*>(a.hq + hrow * a.inter + nt * 128 + cs * 32);
+    dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+    dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+    if (cs == 0) a.hs[hrow * (a.inter / 128) + nt] = scale;
+  }
+  return true;
+}
+
+// GEMM2 epilogue of one row's 64 output columns (feature col): times the gate
+// weight (1 for a shared expert) and written as bf16 to the row's slot.
+__device__ __forceinline__ void epi_scatter(const float (&acc)[64], const Args& a, int g,
+                                            int grow, int col) {
+  long long dst;
+  float wgt = 1.0f;
+  const int s_idx = a.gt.aux(g);
+  if (s_idx < 0) {
+    const int pair = a.pair_of[a.gt.c_row(g) + grow];
+    const int t = pair / a.K, k = pair - t * a.K;
+    dst = (long long)t * (a.K + a.Ks) + k;
+    wgt = a.topk_w[pair];
+  } else {
+    dst = (long long)grow * (a.K + a.Ks) + a.K + s_idx;
+  }
+  uint4* o = reinterpret_cast<uint4*>(a.y + dst * a.d + col);
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+    o[j] = make_uint4(gemm::pack_bf16x2(acc[8 * j] * wgt, acc[8 * j + 1] * wgt),
+                      gemm::pack_bf16x2(acc[8 * j + 2] * wgt, acc[8 * j + 3] * wgt),
+                      gemm::pack_bf16x2(acc[8 * j + 4] * wgt, acc[8 * j + 5] * wgt),
+                      gemm::pack_bf16x2(acc[8 * j + 6] * wgt, acc[8 * j + 7] * wgt));
+}
+
 template <int KIND, int EPI>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     k_gemm_promoted(const __grid_constant__ CUtensorMap tmA,
@@ -277,35 +371,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (!mbar_wait(&pfull[p], (uint32_t)(pu >> 1) & 1u, abort_flag)) { ok = false; break; }
         tc_fence_after();
         const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(p * BN + col0);
-        // two batches of two 16-column loads; the router's unscaled promotion
-        // is a paired FMA with multiplier 1
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          uint32_t va[16], vb[16];
-          tmem_ld16_nowait(tb + (uint32_t)(32 * h), va);
-          tmem_ld16_nowait(tb + (uint32_t)(32 * h + 16), vb);
-          tmem_wait_ld2(va, vb);
-          const float m = EPI == EPI_F32_STORE ? 1.0f : (h == 0 ? m0 : m1);
-          const float2 mm = make_float2(m, m);
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const int o = 32 * h + 2 * i;
-            const float2 r = __ffma2_rn(mm, make_float2(__uint_as_float(va[2 * i]),
-                                                        __uint_as_float(va[2 * i + 1])),
-                                        make_float2(acc[o], acc[o + 1]));
-            acc[o] = r.x;
-            acc[o + 1] = r.y;
-          }
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const int o = 32 * h + 16 + 2 * i;
-            const float2 r = __ffma2_rn(mm, make_float2(__uint_as_float(vb[2 * i]),
-                                                        __uint_as_float(vb[2 * i + 1])),
-                                        make_float2(acc[o], acc[o + 1]));
-            acc[o] = r.x;
-            acc[o + 1] = r.y;
-          }
-        }
+        // the router's unscaled promotion is a paired FMA with multiplier 1
+        promote64(tb, acc, m0, m1);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&pempty[p]);
@@ -327,55 +394,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
         }
       } else if (EPI == EPI_SWIGLU_Q) {
-        // columns 0..31 of the slice are gate, 32..63 the matching up
-        float pam = 0.f;
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          acc[i] = gemm::silu_f(acc[i]) * acc[32 + i];
-          pam = fmaxf(pam, fabsf(acc[i]));
-        }
-        float* ab = amax_buf + (tcount & 1) * 4 * BM;
-        ab[cs * BM + r] = pam;
-        mbar_arrive(xbar);
-        if (!mbar_wait(xbar, (uint32_t)tcount & 1u, abort_flag)) { ok = false; break; }
-        const float amax = fmaxf(fmaxf(ab[r], ab[BM + r]), fmaxf(ab[2 * BM + r], ab[3 * BM + r]));
-        const float scale = amax > 0.f ? __fdiv_rn(amax, 448.0f) : 0.f;
-        const float inv = amax > 0.f ? __fdiv_rn(448.0f, amax) : 0.f;
-        if (valid) {
-          const size_t hrow = (size_t)(a.gt.c_row(g) + grow);
-          uint32_t w[8];
-#pragma unroll
-          for (int j = 0; j < 8; ++j)
-            w[j] = (uint32_t)f32_to_e4m3(__fmul_rn(acc[4 * j], inv)) |
-                   ((uint32_t)f32_to_e4m3(__fmul_rn(acc[4 * j + 1], inv)) << 8) |
-                   ((uint32_t)f32_to_e4m3(__fmul_rn(acc[4 * j + 2], inv)) << 16) |
-                   ((uint32_t)f32_to_e4m3(__fmul_rn(acc[4 * j + 3], inv)) << 24);
-          uint4* dst = reinterpret_cast<uint4*>(a.hq + hrow * a.inter + nt * 128 + cs * 32);
-          dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
-          dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
-          if (cs == 0) a.hs[hrow * (a.inter / 128) + nt] = scale;
+        if (!epi_swiglu_q(acc, a, amax_buf, xbar, tcount, cs, r, valid,
+                          (size_t)(a.gt.c_row(g) + grow), nt, abort_flag)) {
+          ok = false;
+          break;
         }
       } else {
-        if (valid) {
-          long long dst;
-          float wgt = 1.0f;
-          const int s_idx = a.gt.aux(g);
-          if (s_idx < 0) {
-            const int pair = a.pair_of[a.gt.c_row(g) + grow];
-            const int t = pair / a.K, k = pair - t * a.K;
-            dst = (long long)t * (a.K + a.Ks) + k;
-            wgt = a.topk_w[pair];
-          } else {
-            dst = (long long)grow * (a.K + a.Ks) + a.K + s_idx;
-          }
-          uint4* o = reinterpret_cast<uint4*>(a.y + dst * a.d + nt * BN + col0);
-#pragma unroll
-          for (int j = 0; j < 8; ++j)
-            o[j] = make_uint4(gemm::pack_bf16x2(acc[8 * j] * wgt, acc[8 * j + 1] * wgt),
-                              gemm::pack_bf16x2(acc[8 * j + 2] * wgt, acc[8 * j + 3] * wgt),
-                              gemm::pack_bf16x2(acc[8 * j + 4] * wgt, acc[8 * j + 5] * wgt),
-                              gemm::pack_bf16x2(acc[8 * j + 6] * wgt, acc[8 * j + 7] * wgt));
-        }
+        if (valid) epi_scatter(acc, a, g, grow, nt * BN + col0);
       }
     }
   }

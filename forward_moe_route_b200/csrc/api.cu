@@ -1466,7 +1466,7 @@ int32_t moe_backward_launch_count(const moe_layer_desc* desc) {
   if (D.T == 0) return 0;
   // route (2) + hist, scan, slots (3) + prep, gather, zero pads (3) + six GEMMs on the
   // rows and experts + gate backward + combine + the router-weight GEMM
-  return 2 + 3 + 3 + 5 + 1 + 1 + 1;
+  return 2 + 3 + 3 + 6 + 1 + 1 + 1;
 }
 
 size_t moe_expert_ffn_workspace_size(const moe_layer_desc* desc, int32_t n_groups,

@@ -114,10 +114,11 @@ inline bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 struct DeviceInfo {
   int sms = 0;
   bool attrs_done = false;
-  // co-resident 2-CTA clusters of the pair GEMMs (0: gate/up, 1: down), and
-  // the dynamic shared memory each count was taken for
-  size_t pair_smem[3] = {0, 0, 0};
-  int pair_clusters[3] = {0, 0, 0};
+  // co-resident 2-CTA clusters of the pair GEMMs (0: gate/up, 1: down,
+  // 2: backward weight gradients, 3: backward activation GEMMs), and the
+  // dynamic shared memory each count was taken for
+  size_t pair_smem[4] = {0, 0, 0, 0};
+  int pair_clusters[4] = {0, 0, 0, 0};
 };
 std::mutex g_mu;
 DeviceInfo g_dev[kMaxDevices];
@@ -822,31 +823,38 @@ struct Operand {
   uint64_t inner, rows;
 };
 
-template <bool A_MN, bool B_MN, int EPI>
+// The activation-side backward problems (A = token rows, K-major) on CTA
+// pairs: 256-row tiles, each CTA loading its 128 rows and half of the tile's
+// 256 B columns.
+template <bool B_MN, int EPI>
 moe_status launch_gemm_bwd(const char* what, Operand a0, Operand a1, Operand b0, Operand b1,
-                           gbwd::Args args, int64_t tiles_bound, int sms, cudaStream_t st) {
+                           gbwd::Args args, int64_t tiles_bound, cudaStream_t st) {
   CUtensorMap ta0, ta1, tb0, tb1;
   auto mk = [&](CUtensorMap* m, const Operand& o, bool mn, uint32_t box_rows) {
     return mn ? make_tmap_mn(m, o.base, o.inner, o.rows) : make_tmap(m, o.base, 2, o.inner, o.rows,
                                                                      box_rows);
   };
-  moe_status rc = mk(&ta0, a0, A_MN, gbwd::BM);
-  if (rc == MOE_OK) rc = mk(&ta1, a1, A_MN, gbwd::BM);
-  if (rc == MOE_OK) rc = mk(&tb0, b0, B_MN, gbwd::BN);
-  if (rc == MOE_OK) rc = mk(&tb1, b1, B_MN, gbwd::BN);
+  moe_status rc = mk(&ta0, a0, false, gbwd::BM);
+  if (rc == MOE_OK) rc = mk(&ta1, a1, false, gbwd::BM);
+  if (rc == MOE_OK) rc = mk(&tb0, b0, B_MN, gbwd::BN / 2);
+  if (rc == MOE_OK) rc = mk(&tb1, b1, B_MN, gbwd::BN / 2);
   if (rc != MOE_OK) return rc;
   int stages = 0;
-  for (int s = 4; s >= 2 && !stages; --s)
+  for (int s = 6; s >= 2 && !stages; --s)
     if (gbwd::smem_bytes(s, args.n_probs) <= (size_t)kMaxSmem) stages = s;
   if (!stages) return MOE_ERR_UNSUPPORTED;
   args.stages = stages;
   const size_t smem = gbwd::smem_bytes(stages, args.n_probs);
-  cudaError_t e = cudaFuncSetAttribute(gbwd::k_gemm_bwd<A_MN, B_MN, EPI>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
+  auto* k = gbwd::k_gemm_bwd<B_MN, EPI>;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
   if (e != cudaSuccess) return cuda_fail(e, what);
-  const int grid = (int)(tiles_bound < sms ? (tiles_bound > 0 ? tiles_bound : 1) : sms);
-  return launch_chain(what, gbwd::k_gemm_bwd<A_MN, B_MN, EPI>, dim3(grid),
-                      dim3(gbwd::NUM_THREADS), smem, st, ta0, ta1, tb0, tb1, args);
+  cudaLaunchConfig_t cfg;
+  cudaLaunchAttribute attr[2];
+  rc = pair_config(3, k, gbwd::NUM_THREADS, smem, tiles_bound, st, &cfg, attr);
+  if (rc != MOE_OK) return rc;
+  e = cudaLaunchKernelEx(&cfg, k, ta0, ta1, tb0, tb1, args);
+  if (e != cudaSuccess) return cuda_fail(e, what);
+  return launched(what);
 }
 
 // Output map of the weight-gradient GEMMs: fp32 [nz][m][ldc], box 32 x 32 x 1,
@@ -1002,8 +1010,8 @@ moe_status do_backward(const moe_layer_desc& s, const Dims& D, const Layout& L,
   ga.tab = tab[0];
   ga.c = ab;
   ga.ldc = 2 * I;
-  rc = launch_gemm_bwd<false, false, gbwd::EPI_BF16>("backward GEMM ab = X W_gu^T", X, XP, WGU,
-                                                      WGU, ga, mt_rows * nt(2 * I), sms, st);
+  rc = launch_gemm_bwd<false, gbwd::EPI_BF16>("backward GEMM ab = X W_gu^T", X, XP, WGU, WGU, ga,
+                                              mt_rows * nt(2 * I), st);
   if (rc != MOE_OK) return rc;
   // G2: dz' = dY W_down with the SwiGLU backward in the epilogue
   ga.tab = tab[1];
@@ -1013,16 +1021,16 @@ moe_status do_backward(const moe_layer_desc& s, const Dims& D, const Layout& L,
   ga.dab = dab;
   ga.dgp = dgp;
   ga.row_w = row_w;
-  rc = launch_gemm_bwd<false, true, gbwd::EPI_SWIGLU_BWD>("backward GEMM dz = dY W_down", DH, DHP,
-                                                           WD, WD, ga, mt_rows * nt(I), sms, st);
+  rc = launch_gemm_bwd<true, gbwd::EPI_SWIGLU_BWD>("backward GEMM dz = dY W_down", DH, DHP, WD,
+                                                   WD, ga, mt_rows * nt(I), st);
   if (rc != MOE_OK) return rc;
   // G3: du pieces = [da | db] W_gu, scattered to the token-major slots
   ga.tab = tab[2];
   ga.c = dslots;
   ga.ldc = d;
   ga.row_pair = row_pair;
-  rc = launch_gemm_bwd<false, true, gbwd::EPI_SCATTER>("backward GEMM du = dAB W_gu", DAB, DAB,
-                                                        WGU, WGU, ga, mt_rows * nt(d), sms, st);
+  rc = launch_gemm_bwd<true, gbwd::EPI_SCATTER>("backward GEMM du = dAB W_gu", DAB, DAB, WGU,
+                                                WGU, ga, mt_rows * nt(d), st);
   if (rc != MOE_OK) return rc;
   // gate-weight and affinity backward -> dl [T, N]
   {
@@ -1039,9 +1047,8 @@ moe_status do_backward(const moe_layer_desc& s, const Dims& D, const Layout& L,
   ga.tab = tab[5];
   ga.c = dxr;
   ga.ldc = d;
-  rc = launch_gemm_bwd<false, true, gbwd::EPI_BF16>("backward GEMM dx_router = dL W_r", DL, DL,
-                                                     WR, WR, ga, nt(d) * ((T + 127) / 128), sms,
-                                                     st);
+  rc = launch_gemm_bwd<true, gbwd::EPI_BF16>("backward GEMM dx_router = dL W_r", DL, DL, WR, WR,
+                                             ga, nt(d) * ((T + 127) / 128), st);
   if (rc != MOE_OK) return rc;
   // dx = dx_router + sum over the token's expert slots, fp32, fixed order
   rc = do_combine(D, dxr, dslots, dx, st);

@@ -1,6 +1,10 @@
 // Grouped GEMM of the layer backward: C_g = A_g B_g^T for a device-built list
-// of problems, on tcgen05 / TMEM (one CTA per SM, 128 x 256 tiles, the fp32
-// accumulator kept in TMEM over the whole K loop), fed by TMA.
+// of problems, on tcgen05 / TMEM (the fp32 accumulator kept in TMEM over the
+// whole K loop), fed by TMA, on clusters of two CTAs (tcgen05.mma.cta_group::2).
+// Two kernels: k_gemm_bwd for the activation-side problems (A = token rows,
+// K-major; 256-row tiles, each CTA loading its 128 rows and half of the
+// tile's 256 B columns), and k_gemm_bwd_pair for the weight gradients (both
+// operands MN-major, 256 x 256 tiles, fp32 output).
 //
 // Every backward GEMM contracts over an index that is the row index of one of
 // its operands in memory: the hidden size d of W_down [d, I] (dz = dY W_down),
@@ -25,13 +29,16 @@
 //                      (row-store epilogues; the zero rows are the K padding
 //                      of the weight-gradient GEMMs that read them later)
 //   aux                epilogue-specific (shared-expert index or -1)
-// Tiles: ceil(m/128) x ceil(n/256) per problem, N fastest, problems in order,
-// strided over the persistent CTAs.
+// Tiles: ceil(m/256) x ceil(n/256) per problem, N fastest, problems in
+// order, strided over the persistent pairs.
 //
-// Warp roles (256 threads): warp 0 TMA producer, warp 1 MMA issuer, warp 2
-// TMEM allocator, warps 4..7 epilogue (warp w reads TMEM lanes 32(w-4)..+31,
-// one output row per thread).  Two accumulators of 256 columns.  Every wait
-// is bounded (see common.cuh).
+// Warp roles (256 threads per CTA): warp 0 TMA producer, warp 1 MMA issuer
+// (the even CTA's), warp 2 TMEM allocator, warps 4..7 epilogue (warp w reads
+// TMEM lanes 32(w-4)..+31, one output row per thread).  Two accumulators of
+// 256 columns.  full[s] on the leader receives both CTAs' bytes; the leader's
+// MMA commits empty[s] and tfull[a] to both; both CTAs' epilogue threads
+// arrive on the leader's tempty[a].  Every wait is bounded (see common.cuh),
+// and a cluster barrier precedes the TMEM free.
 #pragma once
 
 #include "common.cuh"
@@ -51,7 +58,6 @@ constexpr int TMEM_COLS = 512;
 constexpr int GB_FIELDS = 13;
 constexpr uint32_t A_BYTES = BM * 128;
 constexpr uint32_t B_BYTES = BN * 128;
-constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr uint32_t MN_BOX_BYTES = 64 * 128;   // one MN-major box: 64 K rows x 128 bytes
 
 enum Epi {
@@ -82,13 +88,11 @@ struct Args {
   int K, Ks;
 };
 
-// fp32 epilogue staging: per epilogue warp a 32 x 32 block with rows padded
-// to 33 floats (lane l writes row l column by column without bank conflicts)
-constexpr int XPOSE_FLOATS = 32 * 33;
-constexpr uint32_t XPOSE_BYTES = 4 * XPOSE_FLOATS * 4;
-
+// Shared memory of k_gemm_bwd: a stage holds the CTA's 128 A rows and its
+// half of the tile's 256 B columns.
+constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES / 2;
 __host__ inline size_t smem_bytes(int stages, int n_probs) {
-  return 1024 + (size_t)stages * STAGE_BYTES + XPOSE_BYTES + (size_t)(2 * stages + 5) * 8 + 16 +
+  return 1024 + (size_t)stages * STAGE_BYTES + (size_t)(2 * stages + 5) * 8 + 16 +
          (size_t)(n_probs + 1) * 4 + 64;
 }
 
@@ -105,18 +109,21 @@ __device__ __forceinline__ uint64_t umma_desc_sw128_mn(uint32_t smem_addr) {
   return d;
 }
 
-template <bool A_MN, bool B_MN, int EPI>
+template <bool B_MN, int EPI>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     k_gemm_bwd(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
                const __grid_constant__ CUtensorMap tmB0, const __grid_constant__ CUtensorMap tmB1,
                const Args a) {
+  static_assert(EPI != EPI_F32, "fp32 weight gradients run in k_gemm_bwd_pair");
+  using namespace gemmt;   // cluster helpers of the forward pair kernels
   grid_dep_sync();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
+  constexpr int TM = 2 * BM;                          // rows per pair tile
+  constexpr uint32_t SB = STAGE_BYTES;
   const int S = a.stages;
-  float* xpose = reinterpret_cast<float*>(smem + (size_t)S * STAGE_BYTES);
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)S * STAGE_BYTES + XPOSE_BYTES);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)S * SB);
   uint64_t* empty = full + S;
   uint64_t* tfull = empty + S;
   uint64_t* tempty = tfull + 2;
@@ -126,6 +133,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   int* s_prefix = reinterpret_cast<int*>(tmem_slot + 4);
 
   const int warp = warp_id(), lane = lane_id();
+  const uint32_t rank = cluster_rank();
+  const bool leader = rank == 0;
   const int np = a.n_probs;
   if (warp == 0) {
     int carry = 0;
@@ -134,7 +143,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       int v = 0;
       if (g < np) {
         const int* p = a.tab + (size_t)g * GB_FIELDS;
-        v = ((p[F_M] + BM - 1) / BM) * ((p[F_N] + BN - 1) / BN);
+        v = ((p[F_M] + TM - 1) / TM) * ((p[F_N] + BN - 1) / BN);
       }
       int incl = v;
 #pragma unroll
@@ -154,7 +163,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     for (int j = 0; j < 2; ++j) {
       mbar_init(&tfull[j], 1);
-      mbar_init(&tempty[j], 4 * 32);
+      mbar_init(&tempty[j], 2 * 4 * 32);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -166,14 +175,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     tma_prefetch_desc(&tmB1);
   }
   if (warp == 2) {
-    tmem_alloc(tmem_slot, TMEM_COLS);
-    tmem_relinquish();
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_slot)),
+                 "r"(TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
   }
   tc_fence_before();
   __syncthreads();
+  cluster_sync();      // barrier initialisation is visible to the peer from here on
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const int total = s_prefix[np];
+  const int tile0 = (int)(blockIdx.x >> 1), tstep = (int)(gridDim.x >> 1);
 
   // tile -> (problem, m tile, n tile)
   auto locate = [&](int tile, int& g, int& mt, int& nt, const int*& p) {
@@ -184,64 +198,62 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     mt = lt / ntn;
     nt = lt - mt * ntn;
   };
+  // the tile's UMMA N: its columns rounded up to 32, so each CTA's half of B
+  // is a multiple of 16 columns
+  auto mma_cols = [&](const int* p, int nt) {
+    const int nc = min(BN, p[F_N] - nt * BN);
+    return (nc + 31) & ~31;
+  };
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
     if (elect_one()) {
       int it = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+      for (int tile = tile0; tile < total && ok; tile += tstep) {
         int g, mt, nt;
         const int* p;
         locate(tile, g, mt, nt, p);
         const int nkb = (p[F_K] + BK - 1) / BK;
         const CUtensorMap* tA = p[F_AMAP] ? &tmA1 : &tmA0;
         const CUtensorMap* tB = p[F_BMAP] ? &tmB1 : &tmB0;
-        const int am = p[F_AM0] + mt * BM, ak = p[F_AK0];
-        const int bn = p[F_BN0] + nt * BN, bk = p[F_BK0];
+        const int am = p[F_AM0] + mt * TM + (int)rank * BM, ak = p[F_AK0];
+        const int bn = p[F_BN0] + nt * BN + (int)rank * (mma_cols(p, nt) / 2), bk = p[F_BK0];
         for (int kb = 0; kb < nkb; ++kb, ++it) {
           const int s = it % S;
           const uint32_t ph = (uint32_t)(it / S) & 1u;
           if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag)) { ok = false; break; }
-          uint8_t* sa = smem + (size_t)s * STAGE_BYTES;
+          uint8_t* sa = smem + (size_t)s * SB;
           uint8_t* sb = sa + A_BYTES;
-          mbar_arrive_expect_tx(&full[s], STAGE_BYTES);
           const int k0 = kb * BK;
-          if (A_MN) {
-            tma_load_2d(tA, &full[s], sa, am, ak + k0);
-            tma_load_2d(tA, &full[s], sa + MN_BOX_BYTES, am + 64, ak + k0);
-          } else {
-            tma_load_2d(tA, &full[s], sa, ak + k0, am);
-          }
+          const uint32_t fl = mapa(smem_u32(&full[s]), 0);
+          if (leader) mbar_arrive_expect_tx(&full[s], 2 * SB);
+          tma_load_2d_pair(tA, fl, sa, ak + k0, am);
           if (B_MN) {
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-              tma_load_2d(tB, &full[s], sb + j * MN_BOX_BYTES, bn + 64 * j, bk + k0);
+            tma_load_2d_pair(tB, fl, sb, bn, bk + k0);
+            tma_load_2d_pair(tB, fl, sb + MN_BOX_BYTES, bn + 64, bk + k0);
           } else {
-            tma_load_2d(tB, &full[s], sb, bk + k0, bn);
+            tma_load_2d_pair(tB, fl, sb, bk + k0, bn);
           }
         }
       }
       // the copies this CTA issued land before the block may leave (bounded)
       volatile int no_abort = 0;
       for (int j = (it - S > 0 ? it - S : 0); j < it; ++j)
-        mbar_wait(&full[j % S], (uint32_t)(j / S) & 1u, &no_abort);
+        mbar_wait(&empty[j % S], (uint32_t)(j / S) & 1u, &no_abort);
     }
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
-    if (elect_one()) {
+    if (leader && elect_one()) {
       int it = 0, tcount = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x, ++tcount) {
+      for (int tile = tile0; tile < total && ok; tile += tstep, ++tcount) {
         int g, mt, nt;
         const int* p;
         locate(tile, g, mt, nt, p);
         const int nkb = (p[F_K] + BK - 1) / BK;
-        int ncols = min(BN, p[F_N] - nt * BN);
-        ncols = (ncols + 15) & ~15;
-        const uint32_t idesc = umma_idesc(1, BM, ncols) | (A_MN ? (1u << 15) : 0u) |
-                               (B_MN ? (1u << 16) : 0u);
+        const uint32_t idesc = umma_idesc(1, TM, mma_cols(p, nt)) | (B_MN ? (1u << 16) : 0u);
         const int acc = tcount & 1;
         const uint32_t use = (uint32_t)(tcount >> 1);
         if (!mbar_wait(&tempty[acc], (use & 1u) ^ 1u, abort_flag)) { ok = false; break; }
@@ -252,21 +264,28 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const uint32_t ph = (uint32_t)(it / S) & 1u;
           if (!mbar_wait(&full[s], ph, abort_flag)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t sa = smem_u32(smem + (size_t)s * STAGE_BYTES);
-          const uint64_t ad = A_MN ? umma_desc_sw128_mn(sa) : umma_desc_sw128(sa);
+          const uint32_t sa = smem_u32(smem + (size_t)s * SB);
+          const uint64_t ad = umma_desc_sw128(sa);
           const uint64_t bd = B_MN ? umma_desc_sw128_mn(sa + A_BYTES) : umma_desc_sw128(sa + A_BYTES);
           // one UMMA per 16 elements of K: 32 bytes further along a K-major
           // line, 16 rows (2 KB) further down an MN-major tile
-          constexpr uint64_t a_step = A_MN ? (2048 >> 4) : (32 >> 4);
           constexpr uint64_t b_step = B_MN ? (2048 >> 4) : (32 >> 4);
 #pragma unroll
-          for (int k = 0; k < BK / 16; ++k)
-            umma<0>(d_tmem, ad + a_step * k, bd + b_step * k, idesc, (kb | k) != 0 ? 1u : 0u);
-          umma_commit(&empty[s]);
+          for (int k = 0; k < BK / 16; ++k) {
+            const uint32_t accum = (kb | k) != 0 ? 1u : 0u;
+            umma_pair<0>(d_tmem, ad + (uint64_t)(2 * k), bd + b_step * k, idesc, accum);
+          }
+          const uint32_t e_local = smem_u32(&empty[s]);
+          umma_commit_pair(mapa(e_local, 0));
+          umma_commit_pair(mapa(e_local, 1));
         }
-        if (ok) umma_commit(&tfull[acc]);
+        if (ok) {
+          const uint32_t t_local = smem_u32(&tfull[acc]);
+          umma_commit_pair(mapa(t_local, 0));
+          umma_commit_pair(mapa(t_local, 1));
+        }
       }
-      umma_commit(drain);
+      umma_commit_pair(mapa(smem_u32(drain), 0));
       volatile int no_abort = 0;
       mbar_wait(drain, 0, &no_abort);
     }
@@ -274,9 +293,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   } else if (warp >= EPI_WARP0) {
     // ------------------------------------------------------------------ epilogue
     const int q = warp - EPI_WARP0;            // TMEM lane quadrant
-    const int r_local = q * 32 + lane;         // this thread's row of the tile
+    const int r_local = (int)rank * BM + q * 32 + lane;   // this thread's row of the tile
+    const uint32_t tempty_leader0 = mapa(smem_u32(&tempty[0]), 0);
+    const uint32_t tempty_leader1 = mapa(smem_u32(&tempty[1]), 0);
     int tcount = 0;
-    for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++tcount) {
+    for (int tile = tile0; tile < total; tile += tstep, ++tcount) {
       int g, mt, nt;
       const int* p;
       locate(tile, g, mt, nt, p);
@@ -286,57 +307,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tc_fence_after();
       const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * ACC_COLS);
       const int m = p[F_M], n = p[F_N], mpad = p[F_MPAD];
-      const int row = mt * BM + r_local;                  // row within the problem
+      const int row = mt * TM + r_local;                  // row within the problem
       const bool has_k = p[F_K] > 0;
       const long long crow = (long long)p[F_CROW] + row;
       const int col0 = nt * BN;
       const int ncol = min(BN, n - col0);
       const bool valid = row < m;
       const bool zero_row = !valid && row < mpad;
-      if (EPI == EPI_F32) {
-        // Per 32-column chunk: the warp's 32 rows x 32 columns go through a
-        // padded shared block, then each store instruction writes 4 rows x
-        // 128 contiguous bytes (8 lanes a row), whole lines instead of one
-        // 16-byte piece per row.
-        float* xb = xpose + q * XPOSE_FLOATS;
-        const int rb = mt * BM + q * 32;                     // first row of the warp's block
-        const int sub_r = lane >> 3, sub_c = (lane & 7) * 4; // store phase: row in a group of 4, column
-#pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
-          uint32_t va[16], vb[16];
-          tmem_ld16_nowait(tb + (uint32_t)(32 * c), va);
-          tmem_ld16_nowait(tb + (uint32_t)(32 * c + 16), vb);
-          tmem_wait_ld2(va, vb);
-          if (32 * c >= ncol) continue;                      // warp-uniform
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            xb[lane * 33 + j] = has_k ? __uint_as_float(va[j]) : 0.f;
-            xb[lane * 33 + 16 + j] = has_k ? __uint_as_float(vb[j]) : 0.f;
-          }
-          __syncwarp();
-#pragma unroll
-          for (int g = 0; g < 8; ++g) {
-            const int rr = g * 4 + sub_r;                    // row within the warp's block
-            const int row_g = rb + rr;
-            const int colg = 32 * c + sub_c;
-            if (row_g < m && colg < ncol) {
-              float4 v4 = make_float4(xb[rr * 33 + sub_c], xb[rr * 33 + sub_c + 1],
-                                      xb[rr * 33 + sub_c + 2], xb[rr * 33 + sub_c + 3]);
-              float* dst = reinterpret_cast<float*>(a.c) +
-                           ((long long)p[F_CROW] + row_g) * a.ldc + col0 + colg;
-              if (colg + 4 <= ncol) {
-                *reinterpret_cast<float4*>(dst) = v4;
-              } else {
-                const float e4[4] = {v4.x, v4.y, v4.z, v4.w};
-#pragma unroll
-                for (int k = 0; k < 4; ++k)
-                  if (colg + k < ncol) dst[k] = e4[k];
-              }
-            }
-          }
-          __syncwarp();
-        }
-      } else if (EPI == EPI_BF16 || EPI == EPI_SCATTER) {
+      if (EPI == EPI_BF16 || EPI == EPI_SCATTER) {
         long long dst_row = crow;
         if (EPI == EPI_SCATTER && valid) {
           const int s_idx = p[F_AUX];
@@ -429,14 +407,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (valid || zero_row) a.dgp[crow * ((I + BN - 1) / BN) + nt] = valid ? dgs : 0.f;
       }
       tc_fence_before();
-      mbar_arrive(&tempty[acc]);
+      if (leader) mbar_arrive(&tempty[acc]);
+      else mbar_arrive_cluster(acc ? tempty_leader1 : tempty_leader0);
     }
   }
   tc_fence_before();
   __syncthreads();
+  cluster_sync();      // the peer no longer touches this CTA's barriers or TMEM
   if (warp == 2) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, TMEM_COLS);
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                 "r"(TMEM_COLS)
+                 : "memory");
   }
 }
 

@@ -138,6 +138,12 @@ cudaError_t set_down_attr() {
 // Text of the last CUDA failure on this host thread (moe_last_error_message).
 thread_local char t_errmsg[256] = "";
 
+moe_status cuda_fail(cudaError_t e, const char* where) {
+  snprintf(t_errmsg, sizeof(t_errmsg), "%s: %s (%s)", where, cudaGetErrorName(e),
+           cudaGetErrorString(e));
+  return MOE_ERR_CUDA;
+}
+
 moe_status device_setup(int* sms) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MOE_ERR_CUDA;
@@ -150,6 +156,9 @@ moe_status device_setup(int* sms) {
     if (e == cudaSuccess) e = set_down_attr<0>();
     if (e == cudaSuccess) e = set_down_attr<1>();
     if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(perm::k_gather, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               kMaxSmem);
+    if (e == cudaSuccess)
       e = cudaFuncSetAttribute(gemm8::k_gemm_promoted<0, gemm8::EPI_F32_STORE>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
     if (e == cudaSuccess)
@@ -158,7 +167,7 @@ moe_status device_setup(int* sms) {
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(gemm8::k_gemm_promoted<2, gemm8::EPI_SCATTER>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
-    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute (dynamic shared memory)");
     // the promoted GEMMs re-split their registers with setmaxnreg; the split
     // adds up only if a thread starts with exactly LAUNCH_REGS registers
     {
@@ -193,12 +202,6 @@ moe_status device_setup(int* sms) {
   return MOE_OK;
 }
 
-
-moe_status cuda_fail(cudaError_t e, const char* where) {
-  snprintf(t_errmsg, sizeof(t_errmsg), "%s: %s (%s)", where, cudaGetErrorName(e),
-           cudaGetErrorString(e));
-  return MOE_ERR_CUDA;
-}
 
 inline moe_status launched(const char* where) {
   const cudaError_t e = cudaGetLastError();
@@ -409,8 +412,17 @@ moe_status do_permute(const Dims& D, int32_t* hist, const void* x, const int32_t
                         st, static_cast<const __nv_bfloat16*>(x), T, K, (int)D.d, (int)D.R,
                         static_cast<const int32_t*>(slot_of), static_cast<uint8_t*>(x_perm),
                         x_perm_scale);
-  return launch_chain("k_gather", perm::k_gather, dim3((T + 7) / 8), dim3(256), 0, st,
-                      static_cast<const uint8_t*>(x), T, K, (int)(D.d * D.x_esz),
+  // bulk-copy gather: a few CTAs per SM, each streaming its tokens' rows
+  const int row_bytes = (int)(D.d * D.x_esz);
+  const size_t gsmem = perm::gather_smem_bytes(row_bytes);
+  if (gsmem > (size_t)kMaxSmem) return MOE_ERR_UNSUPPORTED;
+  int sms = 0;
+  moe_status rc2 = device_setup(&sms);
+  if (rc2 != MOE_OK) return rc2;
+  const int per_sm = (int)(200 * 1024 / gsmem) > 0 ? (int)(200 * 1024 / gsmem) : 1;
+  const int grid = T < sms * per_sm ? T : sms * per_sm;
+  return launch_chain("k_gather", perm::k_gather, dim3(grid), dim3(32), gsmem, st,
+                      static_cast<const uint8_t*>(x), T, K, row_bytes,
                       static_cast<const int32_t*>(slot_of), static_cast<uint8_t*>(x_perm));
 }
 

@@ -224,37 +224,64 @@ __global__ void __launch_bounds__(SLOT_WARPS * 32) k_slots(const int32_t* __rest
   }
 }
 
-// Row gather x -> x_perm (fp32 / bf16): one warp per token reads the row once
-// and writes it to its K rows with 16-byte vectors.
-__global__ void __launch_bounds__(256) k_gather(const uint8_t* __restrict__ x, int T, int K,
-                                                int row_bytes, const int32_t* __restrict__ slot_of,
-                                                uint8_t* __restrict__ x_perm) {
+// Row gather x -> x_perm (fp32 / bf16) on the bulk-copy engine: one thread
+// per CTA streams its tokens (t = blockIdx.x, += gridDim.x) through a ring of
+// GATHER_BUFS row buffers in shared memory: one bulk load of the token's row,
+// then K bulk stores of it to the token's permuted rows (one bulk group per
+// token).  GATHER_BUFS - 1 loads are in flight ahead of the stores; a buffer is
+// reloaded once the stores of the token that used it have read it.  The SM
+// issues a handful of instructions per row, so the copy keeps its pace when
+// the SM clock drops under the power limit.
+constexpr int GATHER_BUFS = 4;
+
+__host__ __device__ inline size_t gather_smem_bytes(int row_bytes) {
+  return 128 + (size_t)GATHER_BUFS * row_bytes + 128;   // barriers, then the 128-aligned rows
+}
+
+__global__ void __launch_bounds__(32) k_gather(const uint8_t* __restrict__ x, int T, int K,
+                                               int row_bytes, const int32_t* __restrict__ slot_of,
+                                               uint8_t* __restrict__ x_perm) {
   grid_dep_sync();
+  extern __shared__ __align__(16) uint8_t gather_raw[];
+  if (threadIdx.x != 0) return;
+  uint64_t* bar = reinterpret_cast<uint64_t*>(gather_raw);
+  uint8_t* buf = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(gather_raw) + 128 + 127) &
+                                            ~static_cast<uintptr_t>(127));
+  for (int j = 0; j < GATHER_BUFS; ++j) mbar_init(&bar[j], 1);
+  fence_barrier_init();
   const int R = T * K;
-  const int t = blockIdx.x * 8 + warp_id();
-  if (t >= T) return;
-  const int lane = lane_id();
-  int my_slot = lane < K ? slot_of[(size_t)t * K + lane] : 0;
-  const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * row_bytes);
-  const int nvec = row_bytes / 16;
-  for (int c0 = 0; c0 < nvec; c0 += 32 * 4) {
-    uint4 v[4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int c = c0 + u * 32 + lane;
-      if (c < nvec) v[u] = __ldg(src + c);
+  const int first = blockIdx.x, step = gridDim.x;
+  const int n_my = first < T ? (T - 1 - first) / step + 1 : 0;
+  auto load = [&](int i) {
+    const int j = i % GATHER_BUFS;
+    mbar_arrive_expect_tx(&bar[j], (uint32_t)row_bytes);
+    bulk_load_1d(buf + (size_t)j * row_bytes, x + (size_t)(first + i * step) * row_bytes,
+                 (uint32_t)row_bytes, &bar[j]);
+  };
+  for (int i = 0; i < GATHER_BUFS - 1 && i < n_my; ++i) load(i);
+  volatile int no_abort = 0;
+  for (int i = 0; i < n_my; ++i) {
+    const int t = first + i * step, j = i % GATHER_BUFS;
+    if (!mbar_wait(&bar[j], (uint32_t)(i / GATHER_BUFS) & 1u, &no_abort)) {
+      // gave up (status set): let the loads already issued land before leaving
+      for (int i2 = i; i2 < i + GATHER_BUFS - 1 && i2 < n_my; ++i2)
+        mbar_wait(&bar[i2 % GATHER_BUFS], (uint32_t)(i2 / GATHER_BUFS) & 1u, &no_abort);
+      break;
     }
+    const uint8_t* src = buf + (size_t)j * row_bytes;
     for (int k = 0; k < K; ++k) {
-      const int row = __shfl_sync(0xffffffffu, my_slot, k);
+      const int row = slot_of[(size_t)t * K + k];
       if ((unsigned)row >= (unsigned)R) continue;  // invalid pair (already reported)
-      uint4* dst = reinterpret_cast<uint4*>(x_perm + (size_t)row * row_bytes);
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int c = c0 + u * 32 + lane;
-        if (c < nvec) dst[c] = v[u];
-      }
+      bulk_store_1d(x_perm + (size_t)row * row_bytes, src, (uint32_t)row_bytes);
+    }
+    bulk_commit_group();
+    if (i + GATHER_BUFS - 1 < n_my) {
+      // the buffer of token i - 1 is next: its stores have read it
+      bulk_wait_group_read<1>();
+      load(i + GATHER_BUFS - 1);
     }
   }
+  bulk_wait_group_all();
 }
 
 // bf16 row -> E4M3 codes per 1x128 tile, written to the token's K permuted rows

@@ -41,6 +41,7 @@
 // and a cluster barrier precedes the TMEM free.
 #pragma once
 
+#include "bulk.cuh"
 #include "common.cuh"
 #include "gemm.cuh"
 #include "gemm_t.cuh"

@@ -11,6 +11,7 @@
 
 #include <type_traits>
 
+#include "bulk.cuh"
 #include "common.cuh"
 #include "gemm.cuh"
 

@@ -41,6 +41,17 @@ class MoeLayerDesc(ctypes.Structure):
                 ("w_dtype", ctypes.c_int32)]
 
 
+MAX_PEERS = 16
+IPC_HANDLE_BYTES = 64
+
+
+class MoePeerRows(ctypes.Structure):
+    """moe_peer_rows: where the send-order rows of a peer dispatch land."""
+    _fields_ = [("x", ctypes.c_void_p * MAX_PEERS), ("w", ctypes.c_void_p * MAX_PEERS),
+                ("start", ctypes.c_int32 * (MAX_PEERS + 1)), ("base", ctypes.c_int32 * MAX_PEERS),
+                ("n_ranks", ctypes.c_int32)]
+
+
 class MoeError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
@@ -80,6 +91,13 @@ _SIGS = {
                                       _P]),
     "moe_combine_rows": (ctypes.c_int, [_D, _P, _P, _P, _P, ctypes.c_int32, _P, _P]),
     "moe_dispatch_rows": (ctypes.c_int, [_D, _P, _P, _P, ctypes.c_int32, _P, _P, _P]),
+    "moe_dispatch_rows_to": (ctypes.c_int, [_D, _P, _P, _P, ctypes.c_int32, _P, _P]),
+    "moe_expert_ffn_to": (ctypes.c_int, [_D, ctypes.c_int32, ctypes.c_int32, _P, ctypes.c_int32,
+                                         ctypes.c_int32, _P, _P, _P, _P, _P, _P, ctypes.c_size_t,
+                                         _P]),
+    "moe_ipc_get_handle": (ctypes.c_int, [_P, _P, ctypes.POINTER(ctypes.c_uint64)]),
+    "moe_ipc_open": (ctypes.c_int, [_P, ctypes.POINTER(ctypes.c_void_p)]),
+    "moe_ipc_close": (ctypes.c_int, [_P]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _f = getattr(_lib, _name)
@@ -380,3 +398,70 @@ def moe_dispatch_rows(desc, x, topk_w, row_of, x_rows, w_rows, stream=None) -> N
     _check(_lib.moe_dispatch_rows(ctypes.byref(desc), _ptr(x), _ptr(topk_w), _ptr(row_of),
                                   x_rows.shape[0], _ptr(x_rows), _ptr(w_rows), _stream(stream)),
            "moe_dispatch_rows")
+
+
+def moe_dispatch_rows_to(desc, x, topk_w, row_of, n_rows: int, x_addr, w_addr, start, base,
+                         stream=None) -> None:
+    """Peer dispatch: send-order row r (start[q] <= r < start[q+1]) lands at row
+    base[q] + r - start[q] of the buffers at device addresses x_addr[q] (rows)
+    and w_addr[q] (gate weights, or 0)."""
+    _need("moe_dispatch_rows_to", desc, x=x, topk_w=topk_w)
+    if row_of.numel() < desc.T * desc.top_k or not row_of.is_contiguous():
+        raise MoeError(ERR_INVALID_ARG, "moe_dispatch_rows_to: row_of must hold T*K int32")
+    n = len(x_addr)
+    if not 1 <= n <= MAX_PEERS or len(w_addr) != n or len(start) != n + 1 or len(base) != n:
+        raise MoeError(ERR_INVALID_ARG, "moe_dispatch_rows_to: one address, start and base a rank")
+    P = MoePeerRows()
+    P.n_ranks = n
+    for q in range(n):
+        P.x[q] = int(x_addr[q]) or None
+        P.w[q] = int(w_addr[q]) or None
+        P.start[q] = int(start[q])
+        P.base[q] = int(base[q])
+    P.start[n] = int(start[n])
+    _check(_lib.moe_dispatch_rows_to(ctypes.byref(desc), _ptr(x), _ptr(topk_w), _ptr(row_of),
+                                     int(n_rows), ctypes.byref(P), _stream(stream)),
+           "moe_dispatch_rows_to")
+
+
+def moe_expert_ffn_to(desc, n_experts: int, groups, n_rows_in: int, n_rows_out: int, x_rows,
+                      row_w, w_gu, w_down, group_out, ws, stream=None) -> None:
+    """As moe_expert_ffn, with group i's output rows stored at the device byte
+    address group_out[i] (a uint64/int64 device tensor [n_groups])."""
+    if not groups.is_contiguous() or groups.dtype.itemsize != 4 or groups.shape[-1] != 4:
+        raise MoeError(ERR_INVALID_ARG, "moe_expert_ffn_to: groups must be contiguous int32 [n, 4]")
+    if group_out.numel() < groups.shape[0] or group_out.dtype.itemsize != 8 or \
+            not group_out.is_contiguous():
+        raise MoeError(ERR_INVALID_ARG, "moe_expert_ffn_to: group_out must hold one uint64 a group")
+    if not x_rows.is_contiguous() or x_rows.shape[-1] != desc.d:
+        raise MoeError(ERR_INVALID_ARG, "moe_expert_ffn_to: x_rows must be contiguous [rows, d]")
+    _check(_lib.moe_expert_ffn_to(ctypes.byref(desc), int(n_experts), groups.shape[0],
+                                  _ptr(groups), int(n_rows_in), int(n_rows_out), _ptr(x_rows),
+                                  _ptr(row_w), _ptr(w_gu), _ptr(w_down), _ptr(group_out),
+                                  _ptr(ws), ws.numel() if ws is not None else 0,
+                                  _stream(stream)),
+           "moe_expert_ffn_to")
+
+
+def moe_ipc_get_handle(t):
+    """(handle, offset): the CUDA IPC handle of the allocation holding tensor
+    t's data and the data's byte offset in it."""
+    buf = ctypes.create_string_buffer(IPC_HANDLE_BYTES)
+    off = ctypes.c_uint64()
+    _check(_lib.moe_ipc_get_handle(_ptr(t), buf, ctypes.byref(off)), "moe_ipc_get_handle")
+    return buf.raw, int(off.value)
+
+
+def moe_ipc_open(handle: bytes) -> int:
+    """Device address, in this process, of another process's allocation (its
+    base: add the offset moe_ipc_get_handle returned with the handle)."""
+    if len(handle) != IPC_HANDLE_BYTES:
+        raise MoeError(ERR_INVALID_ARG, "moe_ipc_open: handle must be 64 bytes")
+    out = ctypes.c_void_p()
+    _check(_lib.moe_ipc_open(ctypes.create_string_buffer(handle, IPC_HANDLE_BYTES),
+                             ctypes.byref(out)), "moe_ipc_open")
+    return int(out.value)
+
+
+def moe_ipc_close(addr: int) -> None:
+    _check(_lib.moe_ipc_close(ctypes.c_void_p(addr)), "moe_ipc_close")

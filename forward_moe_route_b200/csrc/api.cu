@@ -720,8 +720,8 @@ FfnLayout ffn_layout(const Dims& D, int n_groups, int64_t n_rows_out) {
 
 moe_status do_expert_ffn(const Dims& D, int n_experts, int n_groups, const int32_t* groups,
                          int64_t n_in, int64_t n_out, const void* x_rows, const float* row_w,
-                         const void* w_gu, const void* w_down, void* y_rows, uint8_t* ws,
-                         int sms, cudaStream_t st) {
+                         const void* w_gu, const void* w_down, void* y_rows,
+                         const uint64_t* group_out, uint8_t* ws, int sms, cudaStream_t st) {
   const FfnLayout F = ffn_layout(D, n_groups, n_out);
   int32_t* gtab = reinterpret_cast<int32_t*>(ws + F.gtab);
   void* hbuf = ws + F.hbuf;
@@ -767,6 +767,7 @@ moe_status do_expert_ffn(const Dims& D, int n_experts, int n_groups, const int32
     a.d = (int)D.d;
     a.plain = 1;
     a.row_w = row_w;
+    a.group_base = reinterpret_cast<const unsigned long long*>(group_out);
     rc = launch_down(kind, w_down, n_experts, hbuf, esz, n_out, tok_tiles, a, st);
   }
   return rc;
@@ -1517,7 +1518,31 @@ moe_status moe_expert_ffn(const moe_layer_desc* desc, int32_t n_experts, int32_t
   int sms;
   if ((rc = device_setup(&sms)) != MOE_OK) return rc;
   return do_expert_ffn(D, n_experts, n_groups, groups, n_rows_in, n_rows_out, x_rows, row_w, w_gu,
-                       w_down, y_rows, static_cast<uint8_t*>(ws), sms, stream);
+                       w_down, y_rows, nullptr, static_cast<uint8_t*>(ws), sms, stream);
+}
+
+moe_status moe_expert_ffn_to(const moe_layer_desc* desc, int32_t n_experts, int32_t n_groups,
+                             const int32_t* groups, int32_t n_rows_in, int32_t n_rows_out,
+                             const void* x_rows, const float* row_w, const void* w_gu,
+                             const void* w_down, const uint64_t* group_out, void* ws,
+                             size_t ws_bytes, cudaStream_t stream) {
+  Dims D;
+  moe_status rc = fill_dims(desc, &D);
+  if (rc != MOE_OK) return rc;
+  if (D.fp8) return MOE_ERR_UNSUPPORTED;
+  if (n_experts < 1 || n_groups < 1 || n_groups > 1024 || n_rows_in < 0 || n_rows_out < 0)
+    return MOE_ERR_INVALID_ARG;
+  if (!groups || !aligned16(groups) || !w_gu || !w_down || !aligned16(w_gu) ||
+      !aligned16(w_down) || !group_out || (reinterpret_cast<uintptr_t>(group_out) & 7u))
+    return MOE_ERR_INVALID_ARG;
+  if (n_rows_in > 0 && (!x_rows || !aligned16(x_rows))) return MOE_ERR_INVALID_ARG;
+  const FfnLayout F = ffn_layout(D, n_groups, n_rows_out);
+  if (!ws || ws_bytes < F.total || !aligned16(ws)) return MOE_ERR_WORKSPACE;
+  if (n_rows_out == 0 || n_rows_in == 0) return MOE_OK;
+  int sms;
+  if ((rc = device_setup(&sms)) != MOE_OK) return rc;
+  return do_expert_ffn(D, n_experts, n_groups, groups, n_rows_in, n_rows_out, x_rows, row_w, w_gu,
+                       w_down, nullptr, group_out, static_cast<uint8_t*>(ws), sms, stream);
 }
 
 moe_status moe_combine_rows(const moe_layer_desc* desc, const void* x_residual,
@@ -1555,10 +1580,93 @@ moe_status moe_dispatch_rows(const moe_layer_desc* desc, const void* x, const fl
   if (D.T == 0) return MOE_OK;
   if (!x || !row_of || !x_rows || !aligned16(x) || !aligned16(x_rows) || (w_rows && !topk_w))
     return MOE_ERR_INVALID_ARG;
-  return launch_chain("k_dispatch_rows", perm::k_dispatch_rows, dim3((unsigned)((D.T + 7) / 8)),
-                      dim3(256), 0, stream, static_cast<const uint8_t*>(x), (int)D.T, (int)D.K,
-                      (int)(D.d * D.x_esz), topk_w, row_of, (int)n_rows,
-                      static_cast<uint8_t*>(x_rows), w_rows);
+  perm::PeerDest none;
+  memset(&none, 0, sizeof(none));
+  return launch_chain("k_dispatch_rows", perm::k_dispatch_rows<false>,
+                      dim3((unsigned)((D.T + 7) / 8)), dim3(256), 0, stream,
+                      static_cast<const uint8_t*>(x), (int)D.T, (int)D.K, (int)(D.d * D.x_esz),
+                      topk_w, row_of, (int)n_rows, static_cast<uint8_t*>(x_rows), w_rows, none);
+}
+
+moe_status moe_dispatch_rows_to(const moe_layer_desc* desc, const void* x, const float* topk_w,
+                                const int32_t* row_of, int32_t n_rows, const moe_peer_rows* dst,
+                                cudaStream_t stream) {
+  Dims D;
+  moe_status rc = fill_dims(desc, &D);
+  if (rc != MOE_OK) return rc;
+  if (D.fp8) return MOE_ERR_UNSUPPORTED;
+  if (n_rows < 0 || !dst || dst->n_ranks < 1 || dst->n_ranks > MOE_MAX_PEERS)
+    return MOE_ERR_INVALID_ARG;
+  if (D.T == 0) return MOE_OK;
+  if (!x || !row_of || !aligned16(x) || !topk_w) return MOE_ERR_INVALID_ARG;
+  perm::PeerDest P;
+  memset(&P, 0, sizeof(P));
+  P.n = dst->n_ranks;
+  if (dst->start[0] != 0 || dst->start[P.n] != n_rows) return MOE_ERR_INVALID_ARG;
+  for (int q = 0; q < P.n; ++q) {
+    if (dst->start[q + 1] < dst->start[q] || dst->base[q] < 0) return MOE_ERR_INVALID_ARG;
+    if (dst->start[q + 1] > dst->start[q] && (!dst->x[q] || !aligned16(dst->x[q])))
+      return MOE_ERR_INVALID_ARG;
+    P.x[q] = static_cast<uint8_t*>(dst->x[q]);
+    P.w[q] = dst->w[q];
+    P.start[q] = dst->start[q];
+    P.base[q] = dst->base[q];
+  }
+  P.start[P.n] = dst->start[P.n];
+  return launch_chain("k_dispatch_rows", perm::k_dispatch_rows<true>,
+                      dim3((unsigned)((D.T + 7) / 8)), dim3(256), 0, stream,
+                      static_cast<const uint8_t*>(x), (int)D.T, (int)D.K, (int)(D.d * D.x_esz),
+                      topk_w, row_of, (int)n_rows, static_cast<uint8_t*>(nullptr),
+                      static_cast<float*>(nullptr), P);
+}
+
+moe_status moe_ipc_get_handle(const void* dev_ptr, void* handle, uint64_t* offset) {
+  if (!dev_ptr || !handle || !offset) return MOE_ERR_INVALID_ARG;
+  static_assert(sizeof(cudaIpcMemHandle_t) == MOE_IPC_HANDLE_BYTES, "IPC handle size");
+  // the handle names the whole allocation (a caching allocator hands out
+  // pieces of larger ones): find the allocation's base for the offset
+  typedef CUresult (*RangeFn)(CUdeviceptr*, size_t*, CUdeviceptr);
+  static RangeFn range = nullptr;
+  if (!range) {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuMemGetAddressRange", &fn, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || !fn) {
+      snprintf(t_errmsg, sizeof(t_errmsg), "cuMemGetAddressRange entry point not found");
+      return MOE_ERR_CUDA;
+    }
+    range = reinterpret_cast<RangeFn>(fn);
+  }
+  CUdeviceptr base = 0;
+  size_t size = 0;
+  const CUresult r = range(&base, &size, reinterpret_cast<CUdeviceptr>(dev_ptr));
+  if (r != CUDA_SUCCESS) {
+    snprintf(t_errmsg, sizeof(t_errmsg), "cuMemGetAddressRange: CUresult %d", (int)r);
+    return MOE_ERR_CUDA;
+  }
+  cudaIpcMemHandle_t h;
+  const cudaError_t e = cudaIpcGetMemHandle(&h, reinterpret_cast<void*>(base));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaIpcGetMemHandle");
+  memcpy(handle, &h, sizeof(h));
+  *offset = (uint64_t)(reinterpret_cast<CUdeviceptr>(dev_ptr) - base);
+  return MOE_OK;
+}
+
+moe_status moe_ipc_open(const void* handle, void** dev_ptr) {
+  if (!handle || !dev_ptr) return MOE_ERR_INVALID_ARG;
+  cudaIpcMemHandle_t h;
+  memcpy(&h, handle, sizeof(h));
+  const cudaError_t e = cudaIpcOpenMemHandle(dev_ptr, h, cudaIpcMemLazyEnablePeerAccess);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaIpcOpenMemHandle");
+  return MOE_OK;
+}
+
+moe_status moe_ipc_close(void* dev_ptr) {
+  if (!dev_ptr) return MOE_ERR_INVALID_ARG;
+  const cudaError_t e = cudaIpcCloseMemHandle(dev_ptr);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaIpcCloseMemHandle");
+  return MOE_OK;
 }
 
 }  // extern "C"

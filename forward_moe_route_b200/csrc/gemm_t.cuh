@@ -66,9 +66,13 @@ struct Args {
   const float* topk_w;
   int K, Ks;
   // plain-row mode (expert parallelism): group row i goes to output row
-  // c_row + i, scaled by row_w[c_row + i] (1 without row_w)
+  // c_row + i, scaled by row_w[c_row + i] (1 without row_w); with group_base,
+  // group g's row i goes to row i of the buffer at byte address group_base[g]
+  // (which may be another GPU's memory: the expert outputs go straight back to
+  // the ranks that sent the rows)
   int plain;
   const float* row_w;
+  const unsigned long long* group_base;
 };
 
 __device__ __forceinline__ uint32_t cluster_rank() {
@@ -302,6 +306,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const int crow = a.gt.c_row(g);
       const int s_idx = a.gt.aux(g);
       const int nch = (ntok + 15) >> 4;
+      uint8_t* ybase = a.group_base ? reinterpret_cast<uint8_t*>(a.group_base[g])
+                                    : reinterpret_cast<uint8_t*>(a.y);
       long long dreg[8];
       float wreg[8];
 #pragma unroll
@@ -311,7 +317,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         wreg[i] = 0.f;
         if (32 * i < ntok && tok < rows) {
           if (a.plain) {
-            dreg[i] = (long long)crow + tok;
+            dreg[i] = (a.group_base ? 0LL : (long long)crow) + tok;
             wreg[i] = a.row_w ? a.row_w[crow + tok] : 1.0f;
           } else if (s_idx < 0) {
             const int pr = a.pair_of[crow + tok];
@@ -347,7 +353,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               const uint4 val = *reinterpret_cast<const uint4*>(xb + j * 64 + pc * 16);
               const int feat = fw0 + pc * 8;
               if (dst >= 0 && feat < a.d)
-                *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.y) +
+                *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(ybase) +
                                           (size_t)dst * a.d + feat) = val;
             }
           } else {
@@ -359,7 +365,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               const uint4 val = *reinterpret_cast<const uint4*>(xb + j * 128 + pc * 16);
               const int feat = fw0 + pc * 4;
               if (dst >= 0 && feat < a.d)
-                *reinterpret_cast<uint4*>(reinterpret_cast<float*>(a.y) + (size_t)dst * a.d +
+                *reinterpret_cast<uint4*>(reinterpret_cast<float*>(ybase) + (size_t)dst * a.d +
                                           feat) = val;
             }
           }

@@ -461,27 +461,50 @@ __global__ void __launch_bounds__(256) k_combine(const void* __restrict__ x_res,
   }
 }
 
-// Dispatch gather (expert parallelism): x_rows[row_of[t*K + k]] = x[t] and
-// w_rows[row_of[t*K + k]] = topk_w[t*K + k].  One warp per token reads its row
-// once and writes it to its K rows with 16-byte vectors.
+// Destinations of a dispatch straight into the ranks' receive buffers: the
+// send-order rows [start[q], start[q+1]) go to rows base[q] + (row - start[q])
+// of rank q's buffers x[q] (rows) and w[q] (gate weights).  The addresses may
+// be other GPUs' memory (CUDA IPC mappings); the kernel only stores to them.
+constexpr int MAX_PEERS = 16;
+struct PeerDest {
+  uint8_t* x[MAX_PEERS];
+  float* w[MAX_PEERS];
+  int start[MAX_PEERS + 1];
+  int base[MAX_PEERS];
+  int n;
+};
+
+// Dispatch gather (expert parallelism): the send-order row row_of[t*K + k]
+// receives x[t] and topk_w[t*K + k].  Local (PEER = false): row r of x_rows /
+// w_rows.  PEER: the row's rank and place from the PeerDest table.  One warp
+// per token reads its row once and writes it to its K rows with 16-byte
+// vectors.
+template <bool PEER>
 __global__ void __launch_bounds__(256) k_dispatch_rows(const uint8_t* __restrict__ x, int T,
                                                        int K, int row_bytes,
                                                        const float* __restrict__ topk_w,
                                                        const int32_t* __restrict__ row_of,
                                                        int n_rows, uint8_t* __restrict__ x_rows,
-                                                       float* __restrict__ w_rows) {
+                                                       float* __restrict__ w_rows,
+                                                       const PeerDest P) {
   grid_dep_sync();
   const int t = blockIdx.x * 8 + warp_id();
   if (t >= T) return;
   const int lane = lane_id();
-  int my_row = -1;
+  uint8_t* my_dst = nullptr;
   if (lane < K) {
-    my_row = row_of[(size_t)t * K + lane];
-    if ((unsigned)my_row >= (unsigned)n_rows) {
+    const int row = row_of[(size_t)t * K + lane];
+    if ((unsigned)row >= (unsigned)n_rows) {
       set_status(MOE_ERR_DEVICE_CHECK);
-      my_row = -1;
-    } else if (w_rows) {
-      w_rows[my_row] = topk_w[(size_t)t * K + lane];
+    } else if (!PEER) {
+      my_dst = x_rows + (size_t)row * row_bytes;
+      if (w_rows) w_rows[row] = topk_w[(size_t)t * K + lane];
+    } else {
+      int q = 0;
+      while (q + 1 < P.n && row >= P.start[q + 1]) ++q;
+      const size_t r = (size_t)P.base[q] + (size_t)(row - P.start[q]);
+      my_dst = P.x[q] + r * row_bytes;
+      if (P.w[q]) P.w[q][r] = topk_w[(size_t)t * K + lane];
     }
   }
   const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * row_bytes);
@@ -492,8 +515,9 @@ __global__ void __launch_bounds__(256) k_dispatch_rows(const uint8_t* __restrict
     uint4 v = make_uint4(0, 0, 0, 0);
     if (in) v = __ldg(src + c);
     for (int k = 0; k < K; ++k) {
-      const int row = __shfl_sync(0xffffffffu, my_row, k);
-      if (in && row >= 0) reinterpret_cast<uint4*>(x_rows + (size_t)row * row_bytes)[c] = v;
+      uint8_t* dst = reinterpret_cast<uint8_t*>(
+          __shfl_sync(0xffffffffu, reinterpret_cast<unsigned long long>(my_dst), k));
+      if (in && dst) reinterpret_cast<uint4*>(dst)[c] = v;
     }
   }
 }

@@ -239,11 +239,15 @@ class RankStep:
     w_send: object = None
     recv: Optional[ReceivePlan] = None
     y_recv: object = None
+    topk_w: object = None
 
 
-def ep_dispatch(desc, pl: Placement, rank: int, x, w_router, bias, ws=None) -> RankStep:
+def ep_dispatch(desc, pl: Placement, rank: int, x, w_router, bias, ws=None,
+                build_send: bool = True) -> RankStep:
     """Phase 1 on the rank's GPU: routing, the permutation maps, the plan and
-    the send buffer (rows grouped by destination rank, with gate weights)."""
+    the send buffer (rows grouped by destination rank, with gate weights).
+    With build_send=False the send buffer is skipped (the peer-memory exchange
+    writes the rows straight into the receiving ranks' buffers)."""
     import torch
 
     from . import moe_dispatch_rows, moe_permute, moe_route, workspace
@@ -261,6 +265,10 @@ def ep_dispatch(desc, pl: Placement, rank: int, x, w_router, bias, ws=None) -> R
     moe_permute(desc, x, idx, counts, offsets, perm_src, slot_of, None, None, ws)   # maps only
     plan = dispatch_plan(pl, counts.cpu().numpy(), offsets.cpu().numpy(),
                          slot_of[:T * K].cpu().numpy())
+    if not build_send:
+        st = RankStep(rank, plan)
+        st.topk_w = w
+        return st
     row_of = torch.as_tensor(plan.row_of, dtype=torch.int32, device=dev)
     x_send = torch.empty(T * K, d, dtype=x.dtype, device=dev)
     w_send = torch.empty(T * K, dtype=torch.float32, device=dev)
@@ -338,3 +346,178 @@ def local_weights(pl: Placement, rank: int, n_shared: int, w_gu, w_down):
     ids = list(range(n_shared)) + [n_shared + j for j in pl.slots(rank)]
     sel = torch.as_tensor(ids, device=w_gu.device)
     return w_gu.index_select(0, sel).contiguous(), w_down.index_select(0, sel).contiguous()
+
+
+# ----------------------------------------------------------------------------- peer-memory exchange
+def peer_offsets(M: np.ndarray, rank: int):
+    """Where this rank's send-order rows land, from the send matrix of all
+    ranks (M[s, q, l] = rows rank s sends to rank q for q's local slot l):
+    start[q] .. start[q+1] are the rows it sends to rank q (its send order is
+    destination-major), placed from row base[q] of q's receive buffer, after
+    the rows of every lower-numbered source (the order an all-to-all would
+    concatenate them in)."""
+    M = np.asarray(M, np.int64)
+    W = M.shape[0]
+    per_dest = M[rank].sum(axis=1)                       # rows to each rank
+    start = np.concatenate([[0], np.cumsum(per_dest)]).astype(np.int64)
+    base = M[:rank].sum(axis=(0, 2)) if rank else np.zeros(W, np.int64)
+    return [int(v) for v in start], [int(v) for v in base]
+
+
+def peer_return_rows(M: np.ndarray, rank: int, recv: ReceivePlan):
+    """For each received group (source s, slot l, row0, rows): the row of the
+    source's send order its outputs return to.  The source sent its rows for
+    this rank from send-order row start_s[rank] on, in slot order, which is
+    the order they arrived in."""
+    M = np.asarray(M, np.int64)
+    W = M.shape[0]
+    recv_start = np.concatenate([[0], np.cumsum(M[:, rank, :].sum(axis=1))])
+    out = []
+    for row0, rows, slot, _ in recv.groups:
+        # the source whose block [recv_start[s], recv_start[s+1]) holds row0
+        s = int(np.searchsorted(recv_start, row0, side="right") - 1)
+        start_s = int(M[s, :rank].sum())
+        out.append((s, start_s + int(row0 - recv_start[s])))
+    return out
+
+
+class PeerExchange:
+    """The buffers of one rank for the peer-memory exchange, and the device
+    addresses of every rank's buffers in this process.
+
+    recv_x [capacity, d] / recv_w [capacity] receive the rows other ranks
+    dispatch to this rank's experts; ret_y [T*K, d] receives the expert
+    outputs of this rank's own rows, in its send order.  Ranks in other
+    processes are reached through CUDA IPC (open_peers); ranks emulated in one
+    process share their local addresses (link)."""
+
+    def __init__(self, desc, pl: Placement, rank: int, capacity: int, device, dtype):
+        import torch
+        self.desc, self.pl, self.rank, self.capacity = desc, pl, rank, int(capacity)
+        d, TK = desc.d, max(desc.T * desc.top_k, 1)
+        self.recv_x = torch.empty(max(self.capacity, 1), d, dtype=dtype, device=device)
+        self.recv_w = torch.empty(max(self.capacity, 1), dtype=torch.float32, device=device)
+        self.ret_y = torch.empty(TK, d, dtype=dtype, device=device)
+        W = pl.world
+        self.x_addr = [0] * W
+        self.w_addr = [0] * W
+        self.ret_addr = [0] * W
+        self.x_addr[rank] = self.recv_x.data_ptr()
+        self.w_addr[rank] = self.recv_w.data_ptr()
+        self.ret_addr[rank] = self.ret_y.data_ptr()
+        self._opened: List[int] = []
+
+    @staticmethod
+    def link(exchanges: Sequence["PeerExchange"]) -> None:
+        """Ranks emulated in one process: every rank sees the others' buffers."""
+        for ex in exchanges:
+            for other in exchanges:
+                q = other.rank
+                ex.x_addr[q] = other.recv_x.data_ptr()
+                ex.w_addr[q] = other.recv_w.data_ptr()
+                ex.ret_addr[q] = other.ret_y.data_ptr()
+
+    def open_peers(self, group=None) -> None:
+        """Ranks in separate processes: exchange CUDA IPC handles over the
+        process group and map every other rank's buffers."""
+        import torch.distributed as dist
+
+        from . import moe_ipc_get_handle, moe_ipc_open
+        mine = (moe_ipc_get_handle(self.recv_x), moe_ipc_get_handle(self.recv_w),
+                moe_ipc_get_handle(self.ret_y))
+        allh = [None] * self.pl.world
+        dist.all_gather_object(allh, mine, group=group)
+        bases = {}        # an allocation is mapped once, however many buffers it holds
+        for q, handles in enumerate(allh):
+            if q == self.rank:
+                continue
+            addrs = []
+            for h, off in handles:
+                if h not in bases:
+                    bases[h] = moe_ipc_open(h)
+                    self._opened.append(bases[h])
+                addrs.append(bases[h] + off)
+            self.x_addr[q], self.w_addr[q], self.ret_addr[q] = addrs
+
+    def close(self) -> None:
+        from . import moe_ipc_close
+        for a in self._opened:
+            moe_ipc_close(a)
+        self._opened = []
+
+
+def peer_dispatch(desc, ex: PeerExchange, st: RankStep, x, M: np.ndarray) -> None:
+    """Dispatch phase: the rank's rows and gate weights go straight into the
+    holders' receive buffers (one kernel, peer stores)."""
+    import torch
+
+    from . import moe_dispatch_rows_to
+    T, K = desc.T, desc.top_k
+    if not T:
+        return
+    start, base = peer_offsets(M, st.rank)
+    for q in range(ex.pl.world):      # every rank's buffer holds ex.capacity rows
+        if base[q] + start[q + 1] - start[q] > ex.capacity:
+            raise ValueError(f"rank {q}'s receive buffer is too small")
+    row_of = torch.as_tensor(st.plan.row_of, dtype=torch.int32, device=x.device)
+    moe_dispatch_rows_to(desc, x, st.topk_w, row_of, T * K, ex.x_addr, ex.w_addr, start, base)
+
+
+def peer_compute(desc, ex: PeerExchange, st: RankStep, M: np.ndarray, w_gu_local,
+                 w_down_local) -> int:
+    """Expert phase: the rank's experts on the rows it received; the down
+    projection stores each output row straight into its source rank's return
+    buffer.  Returns the number of rows processed."""
+    import torch
+
+    from . import moe_expert_ffn_to, moe_expert_ffn_workspace_size
+    M = np.asarray(M, np.int64)
+    r = st.rank
+    st.recv = receive_plan(ex.pl, r, M[:, r, :])
+    n_recv = int(sum(st.recv.recv_splits))
+    if n_recv > ex.capacity:
+        raise ValueError("receive buffer too small")
+    if not n_recv or not len(st.recv.groups):
+        return 0
+    esz = ex.recv_x.element_size()
+    back = peer_return_rows(M, r, st.recv)
+    addrs = [ex.ret_addr[s] + row * desc.d * esz for s, row in back]
+    dev = ex.recv_x.device
+    g = st.recv.groups.copy()
+    g[:, 2] += desc.n_shared
+    groups = torch.as_tensor(g, dtype=torch.int32, device=dev)
+    group_out = torch.as_tensor(np.array(addrs, np.uint64).view(np.int64), device=dev)
+    fws = torch.empty(moe_expert_ffn_workspace_size(desc, len(g), n_recv), dtype=torch.uint8,
+                      device=dev)
+    moe_expert_ffn_to(desc, w_gu_local.shape[0], groups, n_recv, n_recv, ex.recv_x, ex.recv_w,
+                      w_gu_local, w_down_local, group_out, fws)
+    return n_recv
+
+
+def peer_combine(desc, ex: PeerExchange, st: RankStep, x, x_residual, w_gu_local, w_down_local):
+    """Combine phase: the returned rows are in the rank's send order already."""
+    T, K = desc.T, desc.top_k
+    return ep_combine(desc, st, x, x_residual, ex.ret_y[:max(T * K, 1)], w_gu_local,
+                      w_down_local)
+
+
+def ep_forward_peer(desc, pl: Placement, rank: int, x, x_residual, w_router, bias, w_gu_local,
+                    w_down_local, ex: PeerExchange, group=None, ws=None):
+    """One expert-parallel layer forward over peer memory (all ranks call it
+    together, each in its own process with ex.open_peers() done): the send
+    matrix by all-gather, then dispatch, expert and combine phases separated
+    by a device synchronise and a barrier over the ranks."""
+    import torch
+    import torch.distributed as dist
+    st = ep_dispatch(desc, pl, rank, x, w_router, bias, ws, build_send=False)
+    mine = np.ascontiguousarray(st.plan.send_counts)
+    allm = [None] * pl.world
+    dist.all_gather_object(allm, mine, group=group)
+    M = np.stack(allm)
+    peer_dispatch(desc, ex, st, x, M)
+    torch.cuda.synchronize()
+    dist.barrier(group=group)
+    n = peer_compute(desc, ex, st, M, w_gu_local, w_down_local)
+    torch.cuda.synchronize()
+    dist.barrier(group=group)
+    return peer_combine(desc, ex, st, x, x_residual, w_gu_local, w_down_local), n

@@ -257,6 +257,60 @@ moe_status moe_dispatch_rows(const moe_layer_desc* desc, const void* x, const fl
                              const int32_t* row_of, int32_t n_rows, void* x_rows, float* w_rows,
                              cudaStream_t stream);
 
+/* ---- Expert parallelism over peer memory --------------------------------
+ * The exchange of §3.8 written by the compute kernels themselves, with no
+ * collective in between: the dispatch gather stores each row straight into
+ * the receive buffer of the rank that holds its expert, and the expert FFN's
+ * down projection stores each output row straight back into the receive
+ * buffer of the rank that sent the row.  The addresses are device addresses
+ * of every rank's buffers in this process: other GPUs' memory opened through
+ * CUDA IPC (moe_ipc_get_handle on the owner, moe_ipc_open here; NVLink P2P
+ * stores), or local buffers.  No kernel waits on another rank: the caller
+ * orders the phases (finish the launches, then a barrier over the ranks)
+ * between dispatch, expert FFN and combine.
+ *
+ * moe_dispatch_rows_to: as moe_dispatch_rows, but the send-order row r lands
+ * in rank q's buffers, q being the rank with start[q] <= r < start[q+1], at
+ * row base[q] + (r - start[q]) of dst->x[q] (row of d act_dtype elements) and
+ * of dst->w[q] (the gate weight, fp32; w[q] may be NULL).  start[0] = 0,
+ * start[n_ranks] = n_rows, non-decreasing; 1 <= n_ranks <= MOE_MAX_PEERS;
+ * x[q] 16-byte aligned wherever rank q receives rows.  Host struct, read
+ * during the call. */
+#define MOE_MAX_PEERS 16
+typedef struct moe_peer_rows {
+  void* x[MOE_MAX_PEERS];
+  float* w[MOE_MAX_PEERS];
+  int32_t start[MOE_MAX_PEERS + 1];
+  int32_t base[MOE_MAX_PEERS];
+  int32_t n_ranks;
+} moe_peer_rows;
+moe_status moe_dispatch_rows_to(const moe_layer_desc* desc, const void* x, const float* topk_w,
+                                const int32_t* row_of, int32_t n_rows, const moe_peer_rows* dst,
+                                cudaStream_t stream);
+
+/* moe_expert_ffn_to: as moe_expert_ffn, but group i's output row r (times
+ * row_w[out0 + r], as there) is stored at row r of the buffer at device byte
+ * address group_out[i] (uint64 device array [n_groups], 8-byte aligned; each
+ * buffer 16-byte aligned and holding the group's rows of d act_dtype
+ * elements).  n_rows_out sizes the workspace (H) as in moe_expert_ffn. */
+moe_status moe_expert_ffn_to(const moe_layer_desc* desc, int32_t n_experts, int32_t n_groups,
+                             const int32_t* groups, int32_t n_rows_in, int32_t n_rows_out,
+                             const void* x_rows, const float* row_w, const void* w_gu,
+                             const void* w_down, const uint64_t* group_out, void* ws,
+                             size_t ws_bytes, cudaStream_t stream);
+
+/* CUDA IPC of device memory (thin wrappers; a handle is MOE_IPC_HANDLE_BYTES
+ * opaque bytes).  moe_ipc_get_handle: the handle of the allocation holding
+ * dev_ptr and *offset = dev_ptr minus that allocation's base (allocators hand
+ * out pieces of larger allocations).  moe_ipc_open: in another process, the
+ * device address of that allocation's base (peer access enabled lazily; add
+ * the offset); moe_ipc_close unmaps it (pass the base).  CUDA errors return
+ * MOE_ERR_CUDA with the message in moe_last_error_message. */
+#define MOE_IPC_HANDLE_BYTES 64
+moe_status moe_ipc_get_handle(const void* dev_ptr, void* handle, uint64_t* offset);
+moe_status moe_ipc_open(const void* handle, void** dev_ptr);
+moe_status moe_ipc_close(void* dev_ptr);
+
 /* Combine of returned rows: h[t] = x_res[t] + sum_{s<Ks} y_shared[s*T + t]
  * + sum_{k<K} y_rows[row_of[t*K + k]], in fp32, in that order (the order of
  * moe_combine, so with the same row values the two agree bit for bit).

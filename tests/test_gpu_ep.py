@@ -90,3 +90,48 @@ def test_emulated_expert_parallel_equals_single_gpu(world, n_redundant):
         f"max |diff| {float((h.float() - h_ref.float()).abs().max()):.3e}"
     assert sum(loads) == CFG.T * CFG.top_k
     print(f"W={world} redundant={n_redundant}: rows per rank {loads}")
+
+
+def emulate_peer(cfg, inp, pl):
+    """The peer-memory exchange with W ranks emulated on one GPU: each rank's
+    dispatch kernel stores straight into the other ranks' receive buffers and
+    each rank's down projection straight into the senders' return buffers
+    (local addresses here; CUDA IPC mappings of other GPUs' memory on a
+    node).  Phases run rank by rank, all dispatches before any expert phase."""
+    W = pl.world
+    shards = [bench.token_shard(cfg.T, r, W) for r in range(W)]
+    descs, steps, xs = [], [], []
+    for r, (lo, hi) in enumerate(shards):
+        c = dataclasses.replace(cfg, T=hi - lo)
+        d = moe.desc_from_config(c)
+        x = inp["x"][lo:hi].contiguous()
+        descs.append(d)
+        xs.append(x)
+        steps.append(ep.ep_dispatch(d, pl, r, x, inp["w_r"], inp["bias"], build_send=False))
+    M = np.stack([s.plan.send_counts for s in steps])                    # [src, dst, slot]
+    cap = int(M.sum(axis=(0, 2)).max())
+    exs = [ep.PeerExchange(descs[r], pl, r, cap, "cuda", torch.bfloat16) for r in range(W)]
+    ep.PeerExchange.link(exs)
+    for r in range(W):
+        ep.peer_dispatch(descs[r], exs[r], steps[r], xs[r], M)
+    weights = [ep.local_weights(pl, r, cfg.n_shared, inp["w_gu"], inp["w_down"])
+               for r in range(W)]
+    loads = [ep.peer_compute(descs[r], exs[r], steps[r], M, *weights[r]) for r in range(W)]
+    hs = [ep.peer_combine(descs[r], exs[r], steps[r], xs[r], None, *weights[r])
+          for r in range(W)]
+    return torch.cat(hs), loads
+
+
+@pytest.mark.parametrize("world,n_redundant", [(1, 0), (2, 0), (4, 0), (4, 4)])
+def test_emulated_peer_exchange_equals_single_gpu(world, n_redundant):
+    moe.moe_last_device_status()
+    inp = recipes.device_inputs(CFG)
+    h_ref, counts = reference(CFG, inp)
+    replicas = ep.choose_replicas(counts, world, n_redundant) if n_redundant else {}
+    pl = ep.Placement(CFG.n_routed, world, replicas)
+    h, loads = emulate_peer(CFG, inp, pl)
+    assert moe.moe_last_device_status() == moe.OK
+    assert torch.equal(h, h_ref), \
+        f"max |diff| {float((h.float() - h_ref.float()).abs().max()):.3e}"
+    assert sum(loads) == CFG.T * CFG.top_k
+    print(f"peer W={world} redundant={n_redundant}: rows per rank {loads}")

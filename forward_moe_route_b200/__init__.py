@@ -48,6 +48,7 @@ IPC_HANDLE_BYTES = 64
 class MoePeerRows(ctypes.Structure):
     """moe_peer_rows: where the send-order rows of a peer dispatch land."""
     _fields_ = [("x", ctypes.c_void_p * MAX_PEERS), ("w", ctypes.c_void_p * MAX_PEERS),
+                ("scale", ctypes.c_void_p * MAX_PEERS),
                 ("start", ctypes.c_int32 * (MAX_PEERS + 1)), ("base", ctypes.c_int32 * MAX_PEERS),
                 ("n_ranks", ctypes.c_int32)]
 
@@ -96,6 +97,11 @@ _SIGS = {
                                          ctypes.c_int32, _P, _P, _P, _P, _P, _P, ctypes.c_size_t,
                                          _P]),
     "moe_ipc_get_handle": (ctypes.c_int, [_P, _P, ctypes.POINTER(ctypes.c_uint64)]),
+    "moe_dispatch_rows_fp8": (ctypes.c_int, [_D, _P, _P, _P, ctypes.c_int32, _P, _P, _P, _P]),
+    "moe_quantize_rows_fp8": (ctypes.c_int, [_D, _P, ctypes.c_int32, _P, _P, _P]),
+    "moe_expert_ffn_fp8": (ctypes.c_int, [_D, ctypes.c_int32, ctypes.c_int32, _P, ctypes.c_int32,
+                                          ctypes.c_int32, _P, _P, _P, _P, _P, _P, _P, _P, _P,
+                                          _P, ctypes.c_size_t, _P]),
     "moe_ipc_open": (ctypes.c_int, [_P, ctypes.POINTER(ctypes.c_void_p)]),
     "moe_ipc_close": (ctypes.c_int, [_P]),
 }
@@ -401,10 +407,11 @@ def moe_dispatch_rows(desc, x, topk_w, row_of, x_rows, w_rows, stream=None) -> N
 
 
 def moe_dispatch_rows_to(desc, x, topk_w, row_of, n_rows: int, x_addr, w_addr, start, base,
-                         stream=None) -> None:
+                         stream=None, s_addr=None) -> None:
     """Peer dispatch: send-order row r (start[q] <= r < start[q+1]) lands at row
     base[q] + r - start[q] of the buffers at device addresses x_addr[q] (rows)
-    and w_addr[q] (gate weights, or 0)."""
+    and w_addr[q] (gate weights, or 0); for an E4M3 layer the rows are the
+    quantised codes and s_addr[q] receives their 1x128 scales."""
     _need("moe_dispatch_rows_to", desc, x=x, topk_w=topk_w)
     if row_of.numel() < desc.T * desc.top_k or not row_of.is_contiguous():
         raise MoeError(ERR_INVALID_ARG, "moe_dispatch_rows_to: row_of must hold T*K int32")
@@ -416,6 +423,7 @@ def moe_dispatch_rows_to(desc, x, topk_w, row_of, n_rows: int, x_addr, w_addr, s
     for q in range(n):
         P.x[q] = int(x_addr[q]) or None
         P.w[q] = int(w_addr[q]) or None
+        P.scale[q] = (int(s_addr[q]) or None) if s_addr is not None else None
         P.start[q] = int(start[q])
         P.base[q] = int(base[q])
     P.start[n] = int(start[n])
@@ -465,3 +473,47 @@ def moe_ipc_open(handle: bytes) -> int:
 
 def moe_ipc_close(addr: int) -> None:
     _check(_lib.moe_ipc_close(ctypes.c_void_p(addr)), "moe_ipc_close")
+
+
+def moe_dispatch_rows_fp8(desc, x, topk_w, row_of, x_rows, x_rows_scale, w_rows,
+                          stream=None) -> None:
+    """E4M3 dispatch: each token's row quantised per 1x128 tile once, codes to
+    x_rows[row_of[t*K + k]], scales to x_rows_scale, gate weights to w_rows."""
+    _need("moe_dispatch_rows_fp8", desc, x=x, topk_w=topk_w)
+    if row_of.numel() < desc.T * desc.top_k or not row_of.is_contiguous():
+        raise MoeError(ERR_INVALID_ARG, "moe_dispatch_rows_fp8: row_of must hold T*K int32")
+    n = x_rows.shape[0]
+    if not x_rows.is_contiguous() or x_rows.shape[-1] != desc.d or x_rows.element_size() != 1:
+        raise MoeError(ERR_INVALID_ARG, "moe_dispatch_rows_fp8: x_rows must be uint8 [rows, d]")
+    if x_rows_scale.numel() < n * (desc.d // 128) or (w_rows is not None and w_rows.numel() < n):
+        raise MoeError(ERR_INVALID_ARG, "moe_dispatch_rows_fp8: scale / weight rows too short")
+    _check(_lib.moe_dispatch_rows_fp8(ctypes.byref(desc), _ptr(x), _ptr(topk_w), _ptr(row_of), n,
+                                      _ptr(x_rows), _ptr(x_rows_scale), _ptr(w_rows),
+                                      _stream(stream)), "moe_dispatch_rows_fp8")
+
+
+def moe_quantize_rows_fp8(desc, x, codes, scales, stream=None) -> None:
+    """1x128 E4M3 quantisation of the bf16 rows of x [n, d]."""
+    n = x.shape[0]
+    if codes.numel() < n * desc.d or scales.numel() < n * (desc.d // 128):
+        raise MoeError(ERR_INVALID_ARG, "moe_quantize_rows_fp8: outputs too short")
+    _check(_lib.moe_quantize_rows_fp8(ctypes.byref(desc), _ptr(x), n, _ptr(codes), _ptr(scales),
+                                      _stream(stream)), "moe_quantize_rows_fp8")
+
+
+def moe_expert_ffn_fp8(desc, n_experts: int, groups, n_rows_in: int, n_rows_out: int, x_rows,
+                       x_rows_scale, row_w, w_gu, w_gu_scale, w_down, w_down_scale, ws,
+                       y_rows=None, group_out=None, stream=None) -> None:
+    """The FP8 expert GEMMs over caller-given row groups; outputs to y_rows or
+    to the per-group addresses of group_out."""
+    if not groups.is_contiguous() or groups.dtype.itemsize != 4 or groups.shape[-1] != 4:
+        raise MoeError(ERR_INVALID_ARG, "moe_expert_ffn_fp8: groups must be contiguous int32 [n, 4]")
+    if (y_rows is None) == (group_out is None):
+        raise MoeError(ERR_INVALID_ARG, "moe_expert_ffn_fp8: give y_rows or group_out")
+    _check(_lib.moe_expert_ffn_fp8(ctypes.byref(desc), int(n_experts), groups.shape[0],
+                                   _ptr(groups), int(n_rows_in), int(n_rows_out), _ptr(x_rows),
+                                   _ptr(x_rows_scale), _ptr(row_w), _ptr(w_gu), _ptr(w_gu_scale),
+                                   _ptr(w_down), _ptr(w_down_scale), _ptr(y_rows),
+                                   _ptr(group_out), _ptr(ws),
+                                   ws.numel() if ws is not None else 0, _stream(stream)),
+           "moe_expert_ffn_fp8")

@@ -706,16 +706,103 @@ moe_status do_combine(const Dims& D, const void* x_res, const void* y, void* h, 
 // ----------------------------------------------------------------------------- expert parallelism
 // Workspace of moe_expert_ffn: the group table, then H [n_rows_out, I].
 struct FfnLayout {
-  size_t gtab, hbuf, total;
+  size_t gtab, hbuf, hscale, total;
 };
 FfnLayout ffn_layout(const Dims& D, int n_groups, int64_t n_rows_out) {
   FfnLayout F;
   size_t o = 0;
   auto take = [&](size_t bytes) { size_t at = o; o = align_up(o + bytes, kAlign); return at; };
+  const size_t rows = (size_t)(n_rows_out > 0 ? n_rows_out : 1);
   F.gtab = take((size_t)gemm::group_tab_ints(n_groups) * 4);
-  F.hbuf = take((size_t)(n_rows_out > 0 ? n_rows_out : 1) * D.I * D.op_esz);
+  F.hbuf = take(rows * D.I * D.op_esz);
+  F.hscale = D.fp8 ? take(rows * (D.I / 128) * 4) : 0;   // E4M3 H: its 1x128 tile scales
   F.total = o;
   return F;
+}
+
+// moe_expert_ffn for E4M3 layers: the FP8 grouped GEMMs over caller-given row
+// groups (x_rows codes and 1x128 scales in, H requantised per 1x128 between
+// the GEMMs, bf16 rows out in plain-row mode).
+moe_status do_expert_ffn_fp8(const Dims& D, int n_experts, int n_groups, const int32_t* groups,
+                             int64_t n_in, int64_t n_out, const void* x_rows,
+                             const float* x_rows_scale, const float* row_w, const void* w_gu,
+                             const float* w_gu_scale, const void* w_down,
+                             const float* w_down_scale, void* y_rows, const uint64_t* group_out,
+                             uint8_t* ws, int sms, cudaStream_t st) {
+  if (D.d % gemm8::BN || D.I % 128) return MOE_ERR_UNSUPPORTED;
+  const FfnLayout F = ffn_layout(D, n_groups, n_out);
+  int32_t* gtab = reinterpret_cast<int32_t*>(ws + F.gtab);
+  uint8_t* hq = ws + F.hbuf;
+  float* hs = reinterpret_cast<float*>(ws + F.hscale);
+  moe_status rc = launch_chain("k_prep_user_groups", perm::k_prep_user_groups, dim3(1),
+                               dim3(1024), 0, st, groups, n_groups, n_experts, (int)n_in,
+                               (int)n_out, gtab);
+  if (rc != MOE_OK) return rc;
+  int stages = 0;
+  for (int s = 6; s >= 2 && !stages; --s)
+    if (gemm8::smem_bytes(s, n_groups) <= (size_t)kMaxSmem) stages = s;
+  if (!stages) return MOE_ERR_UNSUPPORTED;
+  const size_t smem = gemm8::smem_bytes(stages, n_groups);
+  // upper bound on 128-row tiles over all groups
+  const int64_t mt_bound = (n_out + (int64_t)n_groups * 127) / 128;
+  {
+    CUtensorMap ta, tb;
+    rc = make_tmap(&ta, x_rows, 1, D.d, (uint64_t)n_in, gemm8::BM);
+    if (rc == MOE_OK) rc = make_tmap(&tb, w_gu, 1, D.d, (uint64_t)n_experts * 2 * D.I, 32);
+    if (rc != MOE_OK) return rc;
+    gemm8::Args a;
+    memset(&a, 0, sizeof(a));
+    a.gt.base = gtab;
+    a.gt.n = n_groups;
+    a.n_tiles_n = (int)(D.I / 128);
+    a.num_kb = (int)(D.d / 128);
+    a.kb_elems = 128;
+    a.b_rows_per_expert = (int)(2 * D.I);
+    a.b_up_off = (int)D.I;
+    a.stages = stages;
+    a.idesc = umma_idesc(0, gemm8::BM, gemm8::BN);
+    a.a_scale = x_rows_scale;
+    a.a_rows = (int)n_in;
+    a.b_scale = w_gu_scale;
+    a.hq = hq;
+    a.hs = hs;
+    a.inter = (int)D.I;
+    const int64_t tiles = mt_bound * a.n_tiles_n;
+    const int grid = (int)(tiles < sms ? tiles : sms);
+    rc = launch_chain("FP8 expert GEMM 1", gemm8::k_gemm_promoted<2, gemm8::EPI_SWIGLU_Q>,
+                      dim3(grid), dim3(gemm8::NUM_THREADS), smem, st, ta, tb, a);
+    if (rc != MOE_OK) return rc;
+  }
+  {
+    CUtensorMap ta, tb;
+    rc = make_tmap(&ta, hq, 1, D.I, (uint64_t)n_out, gemm8::BM);
+    if (rc == MOE_OK) rc = make_tmap(&tb, w_down, 1, D.I, (uint64_t)n_experts * D.d, gemm8::BN);
+    if (rc != MOE_OK) return rc;
+    gemm8::Args a;
+    memset(&a, 0, sizeof(a));
+    a.gt.base = gtab;
+    a.gt.n = n_groups;
+    a.n_tiles_n = (int)(D.d / gemm8::BN);
+    a.num_kb = (int)(D.I / 128);
+    a.kb_elems = 128;
+    a.b_rows_per_expert = (int)D.d;
+    a.a_from_crow = 1;
+    a.stages = stages;
+    a.idesc = umma_idesc(0, gemm8::BM, gemm8::BN);
+    a.a_scale = hs;
+    a.a_rows = (int)n_out;
+    a.b_scale = w_down_scale;
+    a.y = static_cast<__nv_bfloat16*>(y_rows);
+    a.d = (int)D.d;
+    a.plain = 1;
+    a.row_w = row_w;
+    a.group_base = reinterpret_cast<const unsigned long long*>(group_out);
+    const int64_t tiles = mt_bound * a.n_tiles_n;
+    const int grid = (int)(tiles < sms ? tiles : sms);
+    rc = launch_chain("FP8 expert GEMM 2", gemm8::k_gemm_promoted<2, gemm8::EPI_SCATTER>,
+                      dim3(grid), dim3(gemm8::NUM_THREADS), smem, st, ta, tb, a);
+  }
+  return rc;
 }
 
 moe_status do_expert_ffn(const Dims& D, int n_experts, int n_groups, const int32_t* groups,
@@ -1492,7 +1579,7 @@ int32_t moe_backward_launch_count(const moe_layer_desc* desc) {
 size_t moe_expert_ffn_workspace_size(const moe_layer_desc* desc, int32_t n_groups,
                                      int32_t n_rows_out) {
   Dims D;
-  if (fill_dims(desc, &D) != MOE_OK || D.fp8 || n_groups < 1 || n_rows_out < 0) return 0;
+  if (fill_dims(desc, &D) != MOE_OK || n_groups < 1 || n_rows_out < 0) return 0;
   return ffn_layout(D, n_groups, n_rows_out).total;
 }
 
@@ -1519,6 +1606,36 @@ moe_status moe_expert_ffn(const moe_layer_desc* desc, int32_t n_experts, int32_t
   if ((rc = device_setup(&sms)) != MOE_OK) return rc;
   return do_expert_ffn(D, n_experts, n_groups, groups, n_rows_in, n_rows_out, x_rows, row_w, w_gu,
                        w_down, y_rows, nullptr, static_cast<uint8_t*>(ws), sms, stream);
+}
+
+moe_status moe_expert_ffn_fp8(const moe_layer_desc* desc, int32_t n_experts, int32_t n_groups,
+                              const int32_t* groups, int32_t n_rows_in, int32_t n_rows_out,
+                              const void* x_rows, const float* x_rows_scale, const float* row_w,
+                              const void* w_gu, const float* w_gu_scale, const void* w_down,
+                              const float* w_down_scale, void* y_rows, const uint64_t* group_out,
+                              void* ws, size_t ws_bytes, cudaStream_t stream) {
+  Dims D;
+  moe_status rc = fill_dims(desc, &D);
+  if (rc != MOE_OK) return rc;
+  if (!D.fp8) return MOE_ERR_INVALID_ARG;
+  if (n_experts < 1 || n_groups < 1 || n_groups > 1024 || n_rows_in < 0 || n_rows_out < 0)
+    return MOE_ERR_INVALID_ARG;
+  if (!groups || !aligned16(groups) || !w_gu || !w_down || !aligned16(w_gu) ||
+      !aligned16(w_down) || !w_gu_scale || !w_down_scale)
+    return MOE_ERR_INVALID_ARG;
+  if ((y_rows == nullptr) == (group_out == nullptr)) return MOE_ERR_INVALID_ARG;
+  if (y_rows && n_rows_out > 0 && !aligned16(y_rows)) return MOE_ERR_INVALID_ARG;
+  if (group_out && (reinterpret_cast<uintptr_t>(group_out) & 7u)) return MOE_ERR_INVALID_ARG;
+  if (n_rows_in > 0 && (!x_rows || !aligned16(x_rows) || !x_rows_scale))
+    return MOE_ERR_INVALID_ARG;
+  const FfnLayout F = ffn_layout(D, n_groups, n_rows_out);
+  if (!ws || ws_bytes < F.total || !aligned16(ws)) return MOE_ERR_WORKSPACE;
+  if (n_rows_out == 0 || n_rows_in == 0) return MOE_OK;
+  int sms;
+  if ((rc = device_setup(&sms)) != MOE_OK) return rc;
+  return do_expert_ffn_fp8(D, n_experts, n_groups, groups, n_rows_in, n_rows_out, x_rows,
+                           x_rows_scale, row_w, w_gu, w_gu_scale, w_down, w_down_scale, y_rows,
+                           group_out, static_cast<uint8_t*>(ws), sms, stream);
 }
 
 moe_status moe_expert_ffn_to(const moe_layer_desc* desc, int32_t n_experts, int32_t n_groups,
@@ -1582,10 +1699,45 @@ moe_status moe_dispatch_rows(const moe_layer_desc* desc, const void* x, const fl
     return MOE_ERR_INVALID_ARG;
   perm::PeerDest none;
   memset(&none, 0, sizeof(none));
-  return launch_chain("k_dispatch_rows", perm::k_dispatch_rows<false>,
+  return launch_chain("k_dispatch_rows", perm::k_dispatch_rows<false, false>,
                       dim3((unsigned)((D.T + 7) / 8)), dim3(256), 0, stream,
                       static_cast<const uint8_t*>(x), (int)D.T, (int)D.K, (int)(D.d * D.x_esz),
-                      topk_w, row_of, (int)n_rows, static_cast<uint8_t*>(x_rows), w_rows, none);
+                      topk_w, row_of, (int)n_rows, static_cast<uint8_t*>(x_rows), w_rows,
+                      static_cast<float*>(nullptr), none);
+}
+
+moe_status moe_dispatch_rows_fp8(const moe_layer_desc* desc, const void* x, const float* topk_w,
+                                 const int32_t* row_of, int32_t n_rows, void* x_rows,
+                                 float* x_rows_scale, float* w_rows, cudaStream_t stream) {
+  Dims D;
+  moe_status rc = fill_dims(desc, &D);
+  if (rc != MOE_OK) return rc;
+  if (!D.fp8) return MOE_ERR_INVALID_ARG;
+  if (n_rows < 0) return MOE_ERR_INVALID_ARG;
+  if (D.T == 0) return MOE_OK;
+  if (!x || !row_of || !x_rows || !x_rows_scale || !aligned16(x) || !aligned16(x_rows) ||
+      (w_rows && !topk_w))
+    return MOE_ERR_INVALID_ARG;
+  perm::PeerDest none;
+  memset(&none, 0, sizeof(none));
+  return launch_chain("k_dispatch_rows", perm::k_dispatch_rows<false, true>,
+                      dim3((unsigned)((D.T + 7) / 8)), dim3(256), 0, stream,
+                      static_cast<const uint8_t*>(x), (int)D.T, (int)D.K, (int)D.d, topk_w,
+                      row_of, (int)n_rows, static_cast<uint8_t*>(x_rows), w_rows, x_rows_scale,
+                      none);
+}
+
+moe_status moe_quantize_rows_fp8(const moe_layer_desc* desc, const void* x, int32_t n_rows,
+                                 void* codes, float* scales, cudaStream_t stream) {
+  Dims D;
+  moe_status rc = fill_dims(desc, &D);
+  if (rc != MOE_OK) return rc;
+  if (!D.fp8 || n_rows < 0) return MOE_ERR_INVALID_ARG;
+  if (n_rows == 0) return MOE_OK;
+  if (!x || !codes || !scales || !aligned16(x) || !aligned16(codes)) return MOE_ERR_INVALID_ARG;
+  return launch_chain("k_quant_rows", perm::k_quant_rows, dim3((unsigned)((n_rows + 7) / 8)),
+                      dim3(256), 0, stream, static_cast<const __nv_bfloat16*>(x), (int)n_rows,
+                      (int)D.d, static_cast<uint8_t*>(codes), scales);
 }
 
 moe_status moe_dispatch_rows_to(const moe_layer_desc* desc, const void* x, const float* topk_w,
@@ -1594,7 +1746,6 @@ moe_status moe_dispatch_rows_to(const moe_layer_desc* desc, const void* x, const
   Dims D;
   moe_status rc = fill_dims(desc, &D);
   if (rc != MOE_OK) return rc;
-  if (D.fp8) return MOE_ERR_UNSUPPORTED;
   if (n_rows < 0 || !dst || dst->n_ranks < 1 || dst->n_ranks > MOE_MAX_PEERS)
     return MOE_ERR_INVALID_ARG;
   if (D.T == 0) return MOE_OK;
@@ -1605,19 +1756,27 @@ moe_status moe_dispatch_rows_to(const moe_layer_desc* desc, const void* x, const
   if (dst->start[0] != 0 || dst->start[P.n] != n_rows) return MOE_ERR_INVALID_ARG;
   for (int q = 0; q < P.n; ++q) {
     if (dst->start[q + 1] < dst->start[q] || dst->base[q] < 0) return MOE_ERR_INVALID_ARG;
-    if (dst->start[q + 1] > dst->start[q] && (!dst->x[q] || !aligned16(dst->x[q])))
+    if (dst->start[q + 1] > dst->start[q] &&
+        (!dst->x[q] || !aligned16(dst->x[q]) || (D.fp8 && !dst->scale[q])))
       return MOE_ERR_INVALID_ARG;
     P.x[q] = static_cast<uint8_t*>(dst->x[q]);
     P.w[q] = dst->w[q];
+    P.s[q] = dst->scale[q];
     P.start[q] = dst->start[q];
     P.base[q] = dst->base[q];
   }
   P.start[P.n] = dst->start[P.n];
-  return launch_chain("k_dispatch_rows", perm::k_dispatch_rows<true>,
+  if (D.fp8)
+    return launch_chain("k_dispatch_rows", perm::k_dispatch_rows<true, true>,
+                        dim3((unsigned)((D.T + 7) / 8)), dim3(256), 0, stream,
+                        static_cast<const uint8_t*>(x), (int)D.T, (int)D.K, (int)D.d, topk_w,
+                        row_of, (int)n_rows, static_cast<uint8_t*>(nullptr),
+                        static_cast<float*>(nullptr), static_cast<float*>(nullptr), P);
+  return launch_chain("k_dispatch_rows", perm::k_dispatch_rows<true, false>,
                       dim3((unsigned)((D.T + 7) / 8)), dim3(256), 0, stream,
                       static_cast<const uint8_t*>(x), (int)D.T, (int)D.K, (int)(D.d * D.x_esz),
                       topk_w, row_of, (int)n_rows, static_cast<uint8_t*>(nullptr),
-                      static_cast<float*>(nullptr), P);
+                      static_cast<float*>(nullptr), static_cast<float*>(nullptr), P);
 }
 
 moe_status moe_ipc_get_handle(const void* dev_ptr, void* handle, uint64_t* offset) {

@@ -87,6 +87,12 @@ struct Args {
   int out_ld, out_cols;
   int* zero_ptr;             // prologue: zero an int array (the expert counts)
   int zero_n;
+  // GEMM2 plain-row mode (expert parallelism): group row i goes to output row
+  // c_row + i (or row i of the buffer at byte address group_base[g]), scaled
+  // by row_w[c_row + i] (1 without row_w)
+  int plain;
+  const float* row_w;
+  const unsigned long long* group_base;
 };
 
 __host__ inline size_t smem_bytes(int stages, int n_groups) {
@@ -165,13 +171,24 @@ __device__ __forceinline__ bool epi_swiglu_q(float (&acc)[64], const Args& a, fl
 }
 
 // GEMM2 epilogue of one row's 64 output columns (feature col): times the gate
-// weight (1 for a shared expert) and written as bf16 to the row's slot.
+// weight (1 for a shared expert) and written as bf16 to the row's slot, or in
+// plain-row mode to the group's output row.
 __device__ __forceinline__ void epi_scatter(const float (&acc)[64], const Args& a, int g,
                                             int grow, int col) {
   long long dst;
   float wgt = 1.0f;
+  __nv_bfloat16* base = a.y;
   const int s_idx = a.gt.aux(g);
-  if (s_idx < 0) {
+  if (a.plain) {
+    const int crow = a.gt.c_row(g);
+    if (a.group_base) {
+      base = reinterpret_cast<__nv_bfloat16*>(a.group_base[g]);
+      dst = grow;
+    } else {
+      dst = (long long)crow + grow;
+    }
+    wgt = a.row_w ? a.row_w[crow + grow] : 1.0f;
+  } else if (s_idx < 0) {
     const int pair = a.pair_of[a.gt.c_row(g) + grow];
     const int t = pair / a.K, k = pair - t * a.K;
     dst = (long long)t * (a.K + a.Ks) + k;
@@ -179,7 +196,7 @@ __device__ __forceinline__ void epi_scatter(const float (&acc)[64], const Args& 
   } else {
     dst = (long long)grow * (a.K + a.Ks) + a.K + s_idx;
   }
-  uint4* o = reinterpret_cast<uint4*>(a.y + dst * a.d + col);
+  uint4* o = reinterpret_cast<uint4*>(base + dst * a.d + col);
 #pragma unroll
   for (int j = 0; j < 8; ++j)
     o[j] = make_uint4(gemm::pack_bf16x2(acc[8 * j] * wgt, acc[8 * j + 1] * wgt),

@@ -289,6 +289,25 @@ __global__ void __launch_bounds__(32) k_gather(const uint8_t* __restrict__ x, in
 // and to row R + t (the shared experts' input), with the fp32 tile scales.
 // Scale rule: amax = max|v|, scale = amax / 448, code = E4M3(v * (448 / amax))
 // rounded to nearest even with saturation; amax = 0 gives scale 0, codes 0.
+// One warp quantises the 1x128 tile g of a bf16 row: lane l takes elements
+// 4l .. 4l+3 and returns their E4M3 codes packed little-endian, and every lane
+// the tile's fp32 scale (amax / 448; 0 for an all-zero tile).
+__device__ __forceinline__ void quant_tile_1x128(const __nv_bfloat16* __restrict__ xr, int g,
+                                                 int lane, uint32_t& code, float& scale) {
+  const uint2 raw = *reinterpret_cast<const uint2*>(xr + g * 128 + lane * 4);
+  const __nv_bfloat162 p0 = *reinterpret_cast<const __nv_bfloat162*>(&raw.x);
+  const __nv_bfloat162 p1 = *reinterpret_cast<const __nv_bfloat162*>(&raw.y);
+  const float v0 = __low2float(p0), v1 = __high2float(p0), v2 = __low2float(p1),
+              v3 = __high2float(p1);
+  const float amax = warp_max(fmaxf(fmaxf(fabsf(v0), fabsf(v1)), fmaxf(fabsf(v2), fabsf(v3))));
+  scale = amax > 0.f ? __fdiv_rn(amax, 448.0f) : 0.f;
+  const float inv = amax > 0.f ? __fdiv_rn(448.0f, amax) : 0.f;
+  code = (uint32_t)f32_to_e4m3(__fmul_rn(v0, inv)) |
+         ((uint32_t)f32_to_e4m3(__fmul_rn(v1, inv)) << 8) |
+         ((uint32_t)f32_to_e4m3(__fmul_rn(v2, inv)) << 16) |
+         ((uint32_t)f32_to_e4m3(__fmul_rn(v3, inv)) << 24);
+}
+
 __global__ void __launch_bounds__(256) k_gather_quant(const __nv_bfloat16* __restrict__ x, int T,
                                                       int K, int d, int R,
                                                       const int32_t* __restrict__ slot_of,
@@ -302,18 +321,9 @@ __global__ void __launch_bounds__(256) k_gather_quant(const __nv_bfloat16* __res
   int my_slot = lane < K ? slot_of[(size_t)t * K + lane] : 0;
   const __nv_bfloat16* xr = x + (size_t)t * d;
   for (int g = 0; g < ng; ++g) {
-    const uint2 raw = *reinterpret_cast<const uint2*>(xr + g * 128 + lane * 4);
-    const __nv_bfloat162 p0 = *reinterpret_cast<const __nv_bfloat162*>(&raw.x);
-    const __nv_bfloat162 p1 = *reinterpret_cast<const __nv_bfloat162*>(&raw.y);
-    const float v0 = __low2float(p0), v1 = __high2float(p0), v2 = __low2float(p1),
-                v3 = __high2float(p1);
-    const float amax = warp_max(fmaxf(fmaxf(fabsf(v0), fabsf(v1)), fmaxf(fabsf(v2), fabsf(v3))));
-    const float scale = amax > 0.f ? __fdiv_rn(amax, 448.0f) : 0.f;
-    const float inv = amax > 0.f ? __fdiv_rn(448.0f, amax) : 0.f;
-    const uint32_t code = (uint32_t)f32_to_e4m3(__fmul_rn(v0, inv)) |
-                          ((uint32_t)f32_to_e4m3(__fmul_rn(v1, inv)) << 8) |
-                          ((uint32_t)f32_to_e4m3(__fmul_rn(v2, inv)) << 16) |
-                          ((uint32_t)f32_to_e4m3(__fmul_rn(v3, inv)) << 24);
+    uint32_t code;
+    float scale;
+    quant_tile_1x128(xr, g, lane, code, scale);
     for (int k = 0; k <= K; ++k) {
       const int row = k < K ? __shfl_sync(0xffffffffu, my_slot, k) : R + t;
       if (k < K && (unsigned)row >= (unsigned)R) continue;  // invalid pair (already reported)
@@ -469,6 +479,7 @@ constexpr int MAX_PEERS = 16;
 struct PeerDest {
   uint8_t* x[MAX_PEERS];
   float* w[MAX_PEERS];
+  float* s[MAX_PEERS];     // E4M3 rows: the 1x128 tile scales of the rows
   int start[MAX_PEERS + 1];
   int base[MAX_PEERS];
   int n;
@@ -476,36 +487,62 @@ struct PeerDest {
 
 // Dispatch gather (expert parallelism): the send-order row row_of[t*K + k]
 // receives x[t] and topk_w[t*K + k].  Local (PEER = false): row r of x_rows /
-// w_rows.  PEER: the row's rank and place from the PeerDest table.  One warp
-// per token reads its row once and writes it to its K rows with 16-byte
-// vectors.
-template <bool PEER>
+// w_rows (and of the tile scales s_rows).  PEER: the row's rank and place from
+// the PeerDest table.  FP8: x is bf16 and each 1x128 tile is quantised to
+// E4M3 once (codes and fp32 scale, as the layer's gather does) before its K
+// copies are stored.  One warp per token reads its row once and writes it to
+// its K rows.
+template <bool PEER, bool FP8>
 __global__ void __launch_bounds__(256) k_dispatch_rows(const uint8_t* __restrict__ x, int T,
                                                        int K, int row_bytes,
                                                        const float* __restrict__ topk_w,
                                                        const int32_t* __restrict__ row_of,
                                                        int n_rows, uint8_t* __restrict__ x_rows,
                                                        float* __restrict__ w_rows,
+                                                       float* __restrict__ s_rows,
                                                        const PeerDest P) {
   grid_dep_sync();
   const int t = blockIdx.x * 8 + warp_id();
   if (t >= T) return;
   const int lane = lane_id();
+  const int ng = row_bytes / 128;      // FP8: row_bytes = d
   uint8_t* my_dst = nullptr;
+  float* my_sdst = nullptr;
   if (lane < K) {
     const int row = row_of[(size_t)t * K + lane];
     if ((unsigned)row >= (unsigned)n_rows) {
       set_status(MOE_ERR_DEVICE_CHECK);
     } else if (!PEER) {
       my_dst = x_rows + (size_t)row * row_bytes;
+      if (FP8) my_sdst = s_rows + (size_t)row * ng;
       if (w_rows) w_rows[row] = topk_w[(size_t)t * K + lane];
     } else {
       int q = 0;
       while (q + 1 < P.n && row >= P.start[q + 1]) ++q;
       const size_t r = (size_t)P.base[q] + (size_t)(row - P.start[q]);
       my_dst = P.x[q] + r * row_bytes;
+      if (FP8) my_sdst = P.s[q] + r * ng;
       if (P.w[q]) P.w[q][r] = topk_w[(size_t)t * K + lane];
     }
+  }
+  if (FP8) {
+    const __nv_bfloat16* xr = reinterpret_cast<const __nv_bfloat16*>(x) + (size_t)t * row_bytes;
+    for (int g = 0; g < ng; ++g) {
+      uint32_t code;
+      float scale;
+      quant_tile_1x128(xr, g, lane, code, scale);
+      for (int k = 0; k < K; ++k) {
+        uint8_t* dst = reinterpret_cast<uint8_t*>(
+            __shfl_sync(0xffffffffu, reinterpret_cast<unsigned long long>(my_dst), k));
+        float* sdst = reinterpret_cast<float*>(
+            __shfl_sync(0xffffffffu, reinterpret_cast<unsigned long long>(my_sdst), k));
+        if (dst) {
+          *reinterpret_cast<uint32_t*>(dst + g * 128 + lane * 4) = code;
+          if (lane == 0) sdst[g] = scale;
+        }
+      }
+    }
+    return;
   }
   const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * row_bytes);
   const int nvec = row_bytes / 16;
@@ -519,6 +556,25 @@ __global__ void __launch_bounds__(256) k_dispatch_rows(const uint8_t* __restrict
           __shfl_sync(0xffffffffu, reinterpret_cast<unsigned long long>(my_dst), k));
       if (in && dst) reinterpret_cast<uint4*>(dst)[c] = v;
     }
+  }
+}
+
+// 1x128 E4M3 quantisation of n bf16 rows of d elements (one warp a row):
+// codes [n, d], scales [n, d / 128].
+__global__ void __launch_bounds__(256) k_quant_rows(const __nv_bfloat16* __restrict__ x, int n,
+                                                    int d, uint8_t* __restrict__ codes,
+                                                    float* __restrict__ scales) {
+  grid_dep_sync();
+  const int t = blockIdx.x * 8 + warp_id();
+  if (t >= n) return;
+  const int lane = lane_id(), ng = d / 128;
+  const __nv_bfloat16* xr = x + (size_t)t * d;
+  for (int g = 0; g < ng; ++g) {
+    uint32_t code;
+    float scale;
+    quant_tile_1x128(xr, g, lane, code, scale);
+    *reinterpret_cast<uint32_t*>(codes + (size_t)t * d + g * 128 + lane * 4) = code;
+    if (lane == 0) scales[(size_t)t * ng + g] = scale;
   }
 }
 

@@ -230,6 +230,12 @@ class Transport:
 
 
 # ----------------------------------------------------------------------------- GPU step
+def is_fp8(desc) -> bool:
+    """E4M3 layer: rows travel as 1x128-quantised codes with their fp32 scales
+    (§3.6: FP8 dispatch), and come back as bf16 (BF16 combine)."""
+    from . import DT_E4M3
+    return desc.w_dtype == DT_E4M3
+
 @dataclass
 class RankStep:
     """One rank's state between the phases of an expert-parallel forward."""
@@ -240,6 +246,7 @@ class RankStep:
     recv: Optional[ReceivePlan] = None
     y_recv: object = None
     topk_w: object = None
+    s_send: object = None       # E4M3 layers: the 1x128 scales of the send rows
 
 
 def ep_dispatch(desc, pl: Placement, rank: int, x, w_router, bias, ws=None,
@@ -270,41 +277,60 @@ def ep_dispatch(desc, pl: Placement, rank: int, x, w_router, bias, ws=None,
         st.topk_w = w
         return st
     row_of = torch.as_tensor(plan.row_of, dtype=torch.int32, device=dev)
-    x_send = torch.empty(T * K, d, dtype=x.dtype, device=dev)
     w_send = torch.empty(T * K, dtype=torch.float32, device=dev)
+    if is_fp8(desc):
+        from . import moe_dispatch_rows_fp8
+        x_send = torch.empty(T * K, d, dtype=torch.uint8, device=dev)
+        s_send = torch.empty(T * K, d // 128, dtype=torch.float32, device=dev)
+        moe_dispatch_rows_fp8(desc, x, w, row_of, x_send, s_send, w_send)
+        st = RankStep(rank, plan, x_send, w_send)
+        st.s_send = s_send
+        return st
+    x_send = torch.empty(T * K, d, dtype=x.dtype, device=dev)
     moe_dispatch_rows(desc, x, w, row_of, x_send, w_send)
     return RankStep(rank, plan, x_send, w_send)
 
 
 def ep_compute(desc, pl: Placement, st: RankStep, recv_counts: np.ndarray, x_recv, w_recv,
-               w_gu_local, w_down_local):
+               w_gu_local, w_down_local, s_recv=None, w_gu_scale=None, w_down_scale=None):
     """Phase 2 on the rank's GPU: the experts it holds on the rows it received
-    (one group per source rank and local slot), gate weights applied."""
+    (one group per source rank and local slot), gate weights applied.  E4M3
+    layers take the received codes with their scales (s_recv) and the local
+    weights' block scales, and return bf16 rows."""
     import torch
 
-    from . import moe_expert_ffn, moe_expert_ffn_workspace_size
+    from . import moe_expert_ffn, moe_expert_ffn_fp8, moe_expert_ffn_workspace_size
     st.recv = receive_plan(pl, st.rank, recv_counts)
     n_recv = int(sum(st.recv.recv_splits))
     dev = x_recv.device
-    y = torch.empty(n_recv, desc.d, dtype=x_recv.dtype, device=dev)
+    fp8 = is_fp8(desc)
+    y = torch.empty(n_recv, desc.d, dtype=torch.bfloat16 if fp8 else x_recv.dtype, device=dev)
     if n_recv and len(st.recv.groups):
         g = st.recv.groups.copy()
         g[:, 2] += desc.n_shared            # local weight index of slot l
         groups = torch.as_tensor(g, dtype=torch.int32, device=dev)
         fws = torch.empty(moe_expert_ffn_workspace_size(desc, len(g), n_recv),
                           dtype=torch.uint8, device=dev)
-        moe_expert_ffn(desc, w_gu_local.shape[0], groups, x_recv, w_recv, w_gu_local,
-                       w_down_local, y, fws)
+        if fp8:
+            moe_expert_ffn_fp8(desc, w_gu_local.shape[0], groups, n_recv, n_recv, x_recv, s_recv,
+                               w_recv, w_gu_local, w_gu_scale, w_down_local, w_down_scale, fws,
+                               y_rows=y)
+        else:
+            moe_expert_ffn(desc, w_gu_local.shape[0], groups, x_recv, w_recv, w_gu_local,
+                           w_down_local, y, fws)
     st.y_recv = y
     return y
 
 
-def ep_combine(desc, st: RankStep, x, x_residual, y_back, w_gu_local, w_down_local):
+def ep_combine(desc, st: RankStep, x, x_residual, y_back, w_gu_local, w_down_local,
+               w_gu_scale=None, w_down_scale=None):
     """Phase 3 on the rank's GPU: its shared experts on its own tokens and the
-    combine of the returned rows, in the single-GPU combine's order."""
+    combine of the returned rows, in the single-GPU combine's order (bf16 for
+    E4M3 layers, whose shared experts read the tokens quantised per 1x128)."""
     import torch
 
-    from . import moe_combine_rows, moe_expert_ffn, moe_expert_ffn_workspace_size
+    from . import (moe_combine_rows, moe_expert_ffn, moe_expert_ffn_fp8,
+                   moe_expert_ffn_workspace_size, moe_quantize_rows_fp8)
     T, d, Ks = desc.T, desc.d, desc.n_shared
     dev = x.device
     y_shared = None
@@ -313,8 +339,16 @@ def ep_combine(desc, st: RankStep, x, x_residual, y_back, w_gu_local, w_down_loc
         y_shared = torch.empty(Ks * T, d, dtype=x.dtype, device=dev)
         sws = torch.empty(moe_expert_ffn_workspace_size(desc, Ks, Ks * T), dtype=torch.uint8,
                           device=dev)
-        moe_expert_ffn(desc, w_gu_local.shape[0], sg, x, None, w_gu_local, w_down_local,
-                       y_shared, sws)
+        if is_fp8(desc):
+            xq = torch.empty(T, d, dtype=torch.uint8, device=dev)
+            xs = torch.empty(T, d // 128, dtype=torch.float32, device=dev)
+            moe_quantize_rows_fp8(desc, x, xq, xs)
+            moe_expert_ffn_fp8(desc, w_gu_local.shape[0], sg, T, Ks * T, xq, xs, None,
+                               w_gu_local, w_gu_scale, w_down_local, w_down_scale, sws,
+                               y_rows=y_shared)
+        else:
+            moe_expert_ffn(desc, w_gu_local.shape[0], sg, x, None, w_gu_local, w_down_local,
+                           y_shared, sws)
     h = torch.empty(max(T, 1), d, dtype=x.dtype, device=dev)
     row_of = torch.as_tensor(st.plan.row_of, dtype=torch.int32, device=dev)
     y_rows = y_back if len(y_back) else torch.zeros(1, d, dtype=x.dtype, device=dev)
@@ -323,29 +357,37 @@ def ep_combine(desc, st: RankStep, x, x_residual, y_back, w_gu_local, w_down_loc
 
 
 def ep_forward(desc, pl: Placement, rank: int, x, x_residual, w_router, bias, w_gu_local,
-               w_down_local, transport: Optional[Transport] = None, ws=None):
+               w_down_local, transport: Optional[Transport] = None, ws=None, w_gu_scale=None,
+               w_down_scale=None):
     """One expert-parallel layer forward of this rank's tokens (all ranks call
     it together).  w_gu_local / w_down_local hold the rank's experts: the Ks
-    shared experts first, then local slot s at index Ks + s (pl.slots(rank)).
-    Returns h [T, d] and the number of rows this rank's experts processed."""
+    shared experts first, then local slot s at index Ks + s (pl.slots(rank));
+    for E4M3 layers also their 128x128 block scales.  Returns h [T, d] and the
+    number of rows this rank's experts processed."""
     transport = transport or Transport()
     st = ep_dispatch(desc, pl, rank, x, w_router, bias, ws)
     recv_counts = transport.counts(st.plan.send_counts)
     recv_splits = [int(v) for v in recv_counts[:, :len(pl.slots(rank))].sum(axis=1)]
     x_recv = transport.all_to_all(st.x_send, st.plan.send_splits, recv_splits)
     w_recv = transport.all_to_all(st.w_send, st.plan.send_splits, recv_splits)
-    y = ep_compute(desc, pl, st, recv_counts, x_recv, w_recv, w_gu_local, w_down_local)
+    s_recv = transport.all_to_all(st.s_send, st.plan.send_splits, recv_splits) \
+        if st.s_send is not None else None
+    y = ep_compute(desc, pl, st, recv_counts, x_recv, w_recv, w_gu_local, w_down_local, s_recv,
+                   w_gu_scale, w_down_scale)
     y_back = transport.all_to_all(y, recv_splits, st.plan.send_splits)
-    return ep_combine(desc, st, x, x_residual, y_back, w_gu_local, w_down_local), len(y)
+    h = ep_combine(desc, st, x, x_residual, y_back, w_gu_local, w_down_local, w_gu_scale,
+                   w_down_scale)
+    return h, len(y)
 
 
-def local_weights(pl: Placement, rank: int, n_shared: int, w_gu, w_down):
-    """The rank's expert weights (shared experts, then its local slots) taken
-    from full [Ks+N, ...] tensors: the placement a deployment would load."""
+def local_weights(pl: Placement, rank: int, n_shared: int, *full):
+    """The rank's expert tensors (shared experts, then its local slots) taken
+    from full [Ks+N, ...] tensors (weights, and for E4M3 layers their block
+    scales): the placement a deployment would load."""
     import torch
     ids = list(range(n_shared)) + [n_shared + j for j in pl.slots(rank)]
-    sel = torch.as_tensor(ids, device=w_gu.device)
-    return w_gu.index_select(0, sel).contiguous(), w_down.index_select(0, sel).contiguous()
+    sel = torch.as_tensor(ids, device=full[0].device)
+    return tuple(t.index_select(0, sel).contiguous() for t in full)
 
 
 # ----------------------------------------------------------------------------- peer-memory exchange
@@ -392,20 +434,32 @@ class PeerExchange:
     process share their local addresses (link)."""
 
     def __init__(self, desc, pl: Placement, rank: int, capacity: int, device, dtype):
+        """dtype: the layer's activation type (bf16 / fp32); an E4M3 layer's
+        rows arrive as uint8 codes with fp32 1x128 scales (recv_s) and return
+        as bf16."""
         import torch
         self.desc, self.pl, self.rank, self.capacity = desc, pl, rank, int(capacity)
-        d, TK = desc.d, max(desc.T * desc.top_k, 1)
-        self.recv_x = torch.empty(max(self.capacity, 1), d, dtype=dtype, device=device)
-        self.recv_w = torch.empty(max(self.capacity, 1), dtype=torch.float32, device=device)
-        self.ret_y = torch.empty(TK, d, dtype=dtype, device=device)
+        d, TK, cap = desc.d, max(desc.T * desc.top_k, 1), max(self.capacity, 1)
+        fp8 = is_fp8(desc)
+        self.recv_x = torch.empty(cap, d, dtype=torch.uint8 if fp8 else dtype, device=device)
+        self.recv_s = torch.empty(cap, d // 128, dtype=torch.float32, device=device) if fp8 \
+            else None
+        self.recv_w = torch.empty(cap, dtype=torch.float32, device=device)
+        self.ret_y = torch.empty(TK, d, dtype=torch.bfloat16 if fp8 else dtype, device=device)
         W = pl.world
         self.x_addr = [0] * W
         self.w_addr = [0] * W
+        self.s_addr = [0] * W
         self.ret_addr = [0] * W
         self.x_addr[rank] = self.recv_x.data_ptr()
         self.w_addr[rank] = self.recv_w.data_ptr()
+        self.s_addr[rank] = self.recv_s.data_ptr() if fp8 else 0
         self.ret_addr[rank] = self.ret_y.data_ptr()
         self._opened: List[int] = []
+
+    def _buffers(self):
+        return [self.recv_x, self.recv_w, self.ret_y] + \
+            ([self.recv_s] if self.recv_s is not None else [])
 
     @staticmethod
     def link(exchanges: Sequence["PeerExchange"]) -> None:
@@ -416,6 +470,7 @@ class PeerExchange:
                 ex.x_addr[q] = other.recv_x.data_ptr()
                 ex.w_addr[q] = other.recv_w.data_ptr()
                 ex.ret_addr[q] = other.ret_y.data_ptr()
+                ex.s_addr[q] = other.recv_s.data_ptr() if other.recv_s is not None else 0
 
     def open_peers(self, group=None) -> None:
         """Ranks in separate processes: exchange CUDA IPC handles over the
@@ -423,8 +478,7 @@ class PeerExchange:
         import torch.distributed as dist
 
         from . import moe_ipc_get_handle, moe_ipc_open
-        mine = (moe_ipc_get_handle(self.recv_x), moe_ipc_get_handle(self.recv_w),
-                moe_ipc_get_handle(self.ret_y))
+        mine = tuple(moe_ipc_get_handle(b) for b in self._buffers())
         allh = [None] * self.pl.world
         dist.all_gather_object(allh, mine, group=group)
         bases = {}        # an allocation is mapped once, however many buffers it holds
@@ -437,7 +491,9 @@ class PeerExchange:
                     bases[h] = moe_ipc_open(h)
                     self._opened.append(bases[h])
                 addrs.append(bases[h] + off)
-            self.x_addr[q], self.w_addr[q], self.ret_addr[q] = addrs
+            self.x_addr[q], self.w_addr[q], self.ret_addr[q] = addrs[:3]
+            if len(addrs) > 3:
+                self.s_addr[q] = addrs[3]
 
     def close(self) -> None:
         from . import moe_ipc_close
@@ -460,17 +516,18 @@ def peer_dispatch(desc, ex: PeerExchange, st: RankStep, x, M: np.ndarray) -> Non
         if base[q] + start[q + 1] - start[q] > ex.capacity:
             raise ValueError(f"rank {q}'s receive buffer is too small")
     row_of = torch.as_tensor(st.plan.row_of, dtype=torch.int32, device=x.device)
-    moe_dispatch_rows_to(desc, x, st.topk_w, row_of, T * K, ex.x_addr, ex.w_addr, start, base)
+    moe_dispatch_rows_to(desc, x, st.topk_w, row_of, T * K, ex.x_addr, ex.w_addr, start, base,
+                         s_addr=ex.s_addr if is_fp8(desc) else None)
 
 
 def peer_compute(desc, ex: PeerExchange, st: RankStep, M: np.ndarray, w_gu_local,
-                 w_down_local) -> int:
+                 w_down_local, w_gu_scale=None, w_down_scale=None) -> int:
     """Expert phase: the rank's experts on the rows it received; the down
     projection stores each output row straight into its source rank's return
-    buffer.  Returns the number of rows processed."""
+    buffer (bf16 for E4M3 layers).  Returns the number of rows processed."""
     import torch
 
-    from . import moe_expert_ffn_to, moe_expert_ffn_workspace_size
+    from . import moe_expert_ffn_fp8, moe_expert_ffn_to, moe_expert_ffn_workspace_size
     M = np.asarray(M, np.int64)
     r = st.rank
     st.recv = receive_plan(ex.pl, r, M[:, r, :])
@@ -479,7 +536,7 @@ def peer_compute(desc, ex: PeerExchange, st: RankStep, M: np.ndarray, w_gu_local
         raise ValueError("receive buffer too small")
     if not n_recv or not len(st.recv.groups):
         return 0
-    esz = ex.recv_x.element_size()
+    esz = ex.ret_y.element_size()
     back = peer_return_rows(M, r, st.recv)
     addrs = [ex.ret_addr[s] + row * desc.d * esz for s, row in back]
     dev = ex.recv_x.device
@@ -489,20 +546,27 @@ def peer_compute(desc, ex: PeerExchange, st: RankStep, M: np.ndarray, w_gu_local
     group_out = torch.as_tensor(np.array(addrs, np.uint64).view(np.int64), device=dev)
     fws = torch.empty(moe_expert_ffn_workspace_size(desc, len(g), n_recv), dtype=torch.uint8,
                       device=dev)
-    moe_expert_ffn_to(desc, w_gu_local.shape[0], groups, n_recv, n_recv, ex.recv_x, ex.recv_w,
-                      w_gu_local, w_down_local, group_out, fws)
+    if is_fp8(desc):
+        moe_expert_ffn_fp8(desc, w_gu_local.shape[0], groups, n_recv, n_recv, ex.recv_x,
+                           ex.recv_s, ex.recv_w, w_gu_local, w_gu_scale, w_down_local,
+                           w_down_scale, fws, group_out=group_out)
+    else:
+        moe_expert_ffn_to(desc, w_gu_local.shape[0], groups, n_recv, n_recv, ex.recv_x,
+                          ex.recv_w, w_gu_local, w_down_local, group_out, fws)
     return n_recv
 
 
-def peer_combine(desc, ex: PeerExchange, st: RankStep, x, x_residual, w_gu_local, w_down_local):
+def peer_combine(desc, ex: PeerExchange, st: RankStep, x, x_residual, w_gu_local, w_down_local,
+                 w_gu_scale=None, w_down_scale=None):
     """Combine phase: the returned rows are in the rank's send order already."""
     T, K = desc.T, desc.top_k
     return ep_combine(desc, st, x, x_residual, ex.ret_y[:max(T * K, 1)], w_gu_local,
-                      w_down_local)
+                      w_down_local, w_gu_scale, w_down_scale)
 
 
 def ep_forward_peer(desc, pl: Placement, rank: int, x, x_residual, w_router, bias, w_gu_local,
-                    w_down_local, ex: PeerExchange, group=None, ws=None):
+                    w_down_local, ex: PeerExchange, group=None, ws=None, w_gu_scale=None,
+                    w_down_scale=None):
     """One expert-parallel layer forward over peer memory (all ranks call it
     together, each in its own process with ex.open_peers() done): the send
     matrix by all-gather, then dispatch, expert and combine phases separated
@@ -517,7 +581,8 @@ def ep_forward_peer(desc, pl: Placement, rank: int, x, x_residual, w_router, bia
     peer_dispatch(desc, ex, st, x, M)
     torch.cuda.synchronize()
     dist.barrier(group=group)
-    n = peer_compute(desc, ex, st, M, w_gu_local, w_down_local)
+    n = peer_compute(desc, ex, st, M, w_gu_local, w_down_local, w_gu_scale, w_down_scale)
     torch.cuda.synchronize()
     dist.barrier(group=group)
-    return peer_combine(desc, ex, st, x, x_residual, w_gu_local, w_down_local), n
+    return peer_combine(desc, ex, st, x, x_residual, w_gu_local, w_down_local, w_gu_scale,
+                        w_down_scale), n

@@ -234,7 +234,8 @@ moe_status moe_bias_update(const moe_layer_desc* desc, const int32_t* counts, fl
  *   y_rows[out_row0 + r] = row_w[out_row0 + r] * FFN_expert(x_rows[row0 + r])
  * (row_w NULL: weight 1) with the same GEMMs as moe_grouped_swiglu.  expert
  * indexes w_gu [n_experts, 2I, d] / w_down [n_experts, d, I]; the output
- * ranges of the groups must not overlap.  F32 and BF16 layers only.
+ * ranges of the groups must not overlap.  F32 and BF16 layers
+ * (moe_expert_ffn_fp8 below for E4M3).
  *   n_groups 1..1024; x_rows [n_rows_in, d], y_rows [n_rows_out, d], row_w
  *   [n_rows_out] fp32.  A group outside these bounds, or with an expert outside
  *   [0, n_experts), is skipped and sets MOE_ERR_DEVICE_CHECK.
@@ -252,7 +253,7 @@ moe_status moe_expert_ffn(const moe_layer_desc* desc, int32_t n_experts, int32_t
  * exchange, in the row order the caller's plan chose.  x [T, d] act_dtype,
  * topk_w [T, K] fp32, row_of [T*K] int32 (an index outside [0, n_rows) is
  * skipped and sets MOE_ERR_DEVICE_CHECK), x_rows [n_rows, d], w_rows [n_rows]
- * fp32.  F32 and BF16 layers only. */
+ * fp32.  F32 and BF16 layers (moe_dispatch_rows_fp8 below for E4M3). */
 moe_status moe_dispatch_rows(const moe_layer_desc* desc, const void* x, const float* topk_w,
                              const int32_t* row_of, int32_t n_rows, void* x_rows, float* w_rows,
                              cudaStream_t stream);
@@ -274,12 +275,15 @@ moe_status moe_dispatch_rows(const moe_layer_desc* desc, const void* x, const fl
  * row base[q] + (r - start[q]) of dst->x[q] (row of d act_dtype elements) and
  * of dst->w[q] (the gate weight, fp32; w[q] may be NULL).  start[0] = 0,
  * start[n_ranks] = n_rows, non-decreasing; 1 <= n_ranks <= MOE_MAX_PEERS;
- * x[q] 16-byte aligned wherever rank q receives rows.  Host struct, read
- * during the call. */
+ * x[q] 16-byte aligned wherever rank q receives rows.  For an E4M3 layer the
+ * rows are the 1x128-quantised codes (d bytes) and scale[q] receives their
+ * tile scales (d/128 fp32 a row; see moe_dispatch_rows_fp8); scale is unused
+ * otherwise.  Host struct, read during the call. */
 #define MOE_MAX_PEERS 16
 typedef struct moe_peer_rows {
   void* x[MOE_MAX_PEERS];
   float* w[MOE_MAX_PEERS];
+  float* scale[MOE_MAX_PEERS];
   int32_t start[MOE_MAX_PEERS + 1];
   int32_t base[MOE_MAX_PEERS];
   int32_t n_ranks;
@@ -298,6 +302,37 @@ moe_status moe_expert_ffn_to(const moe_layer_desc* desc, int32_t n_experts, int3
                              const void* x_rows, const float* row_w, const void* w_gu,
                              const void* w_down, const uint64_t* group_out, void* ws,
                              size_t ws_bytes, cudaStream_t stream);
+
+/* ---- FP8 expert parallelism ("DeepSeek Technical Report: MoE Architecture"
+ * §3.6: dispatch in FP8, combine in BF16) -------------------------------------
+ * moe_dispatch_rows_fp8: as moe_dispatch_rows for an E4M3 layer: each token's
+ * bf16 row is quantised per 1x128 tile (scale = amax/448, codes = E4M3(v *
+ * 448/amax), round to nearest even, saturating; the layer's own gather rule)
+ * once, and the codes x_rows [n_rows, d] uint8 and tile scales x_rows_scale
+ * [n_rows, d/128] fp32 are written to the token's K send rows (with the gate
+ * weights to w_rows when not NULL).  moe_dispatch_rows_to does the same for
+ * an E4M3 layer, with dst->scale[q] receiving the scales.
+ * moe_quantize_rows_fp8: that quantisation of n_rows bf16 rows [n_rows, d]
+ * into codes [n_rows, d] and scales [n_rows, d/128] (the shared experts'
+ * input on the rank that owns the tokens).
+ * moe_expert_ffn_fp8: the layer's FP8 expert GEMMs over caller-given row
+ * groups (as moe_expert_ffn): x_rows codes + x_rows_scale in, the expert
+ * weights as E4M3 with 128x128 block scales (as moe_forward takes them), H
+ * requantised per 1x128 between the GEMMs, bf16 rows out, times row_w.
+ * Exactly one of y_rows [n_rows_out, d] bf16 and group_out (per-group output
+ * addresses, as moe_expert_ffn_to) is given.  ws:
+ * moe_expert_ffn_workspace_size(desc, ...) of the E4M3 layer. */
+moe_status moe_dispatch_rows_fp8(const moe_layer_desc* desc, const void* x, const float* topk_w,
+                                 const int32_t* row_of, int32_t n_rows, void* x_rows,
+                                 float* x_rows_scale, float* w_rows, cudaStream_t stream);
+moe_status moe_quantize_rows_fp8(const moe_layer_desc* desc, const void* x, int32_t n_rows,
+                                 void* codes, float* scales, cudaStream_t stream);
+moe_status moe_expert_ffn_fp8(const moe_layer_desc* desc, int32_t n_experts, int32_t n_groups,
+                              const int32_t* groups, int32_t n_rows_in, int32_t n_rows_out,
+                              const void* x_rows, const float* x_rows_scale, const float* row_w,
+                              const void* w_gu, const float* w_gu_scale, const void* w_down,
+                              const float* w_down_scale, void* y_rows, const uint64_t* group_out,
+                              void* ws, size_t ws_bytes, cudaStream_t stream);
 
 /* CUDA IPC of device memory (thin wrappers; a handle is MOE_IPC_HANDLE_BYTES
  * opaque bytes).  moe_ipc_get_handle: the handle of the allocation holding

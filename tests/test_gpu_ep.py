@@ -50,13 +50,16 @@ def emulate(cfg, inp, pl):
     send_splits = [s.plan.send_splits for s in steps]
     x_recv = a2a([s.x_send for s in steps], send_splits)
     w_recv = a2a([s.w_send for s in steps], send_splits)
-    weights = [ep.local_weights(pl, r, cfg.n_shared, inp["w_gu"], inp["w_down"])
-               for r in range(W)]
+    fp8 = cfg.dtype == "e4m3"
+    s_recv = a2a([s.s_send for s in steps], send_splits) if fp8 else [None] * W
+    full = (inp["w_gu"], inp["w_down"]) + ((inp["w_gu_scale"], inp["w_down_scale"]) if fp8 else ())
+    weights = [ep.local_weights(pl, r, cfg.n_shared, *full) for r in range(W)]
+    scales = [wt[2:] if fp8 else (None, None) for wt in weights]
     ys = [ep.ep_compute(descs[r], pl, steps[r], recv_counts[r], x_recv[r], w_recv[r],
-                        *weights[r]) for r in range(W)]
+                        *weights[r][:2], s_recv[r], *scales[r]) for r in range(W)]
     recv_splits = [s.recv.recv_splits for s in steps]
     y_back = a2a(ys, recv_splits)
-    hs = [ep.ep_combine(descs[r], steps[r], xs[r], None, y_back[r], *weights[r])
+    hs = [ep.ep_combine(descs[r], steps[r], xs[r], None, y_back[r], *weights[r][:2], *scales[r])
           for r in range(W)]
     loads = [int(sum(s.recv.recv_splits)) for s in steps]
     return torch.cat(hs), loads
@@ -67,9 +70,24 @@ def reference(cfg, inp):
     ws = moe.workspace(desc)
     h = torch.empty(cfg.T, cfg.d, dtype=torch.bfloat16, device="cuda")
     counts = torch.empty(cfg.n_routed, dtype=torch.int32, device="cuda")
-    moe.moe_forward(desc, inp["x"], None, inp["w_r"], inp["bias"], inp["w_gu"], None,
-                    inp["w_down"], None, h, None, counts, ws)
+    moe.moe_forward(desc, inp["x"], None, inp["w_r"], inp["bias"], inp["w_gu"],
+                    inp.get("w_gu_scale"), inp["w_down"], inp.get("w_down_scale"), h, None,
+                    counts, ws)
     return h, counts.cpu().numpy()
+
+
+def fp8_inputs(cfg):
+    """The layer's inputs with the expert weights quantised 128x128 to E4M3."""
+    inp = recipes.device_inputs(cfg)
+    E, I, d = cfg.n_experts, cfg.inter, cfg.d
+    gq = torch.empty(E, 2 * I, d, dtype=torch.uint8, device="cuda")
+    gs = torch.empty(E, 2 * I // 128, d // 128, dtype=torch.float32, device="cuda")
+    dq = torch.empty(E, d, I, dtype=torch.uint8, device="cuda")
+    ds = torch.empty(E, d // 128, I // 128, dtype=torch.float32, device="cuda")
+    moe.moe_quantize_fp8_blockwise(inp["w_gu"], 2 * I, d, E, gq, gs)
+    moe.moe_quantize_fp8_blockwise(inp["w_down"], d, I, E, dq, ds)
+    inp.update(w_gu=gq, w_gu_scale=gs, w_down=dq, w_down_scale=ds)
+    return inp
 
 
 CFG = dataclasses.replace(
@@ -114,8 +132,9 @@ def emulate_peer(cfg, inp, pl):
     ep.PeerExchange.link(exs)
     for r in range(W):
         ep.peer_dispatch(descs[r], exs[r], steps[r], xs[r], M)
-    weights = [ep.local_weights(pl, r, cfg.n_shared, inp["w_gu"], inp["w_down"])
-               for r in range(W)]
+    fp8 = cfg.dtype == "e4m3"
+    full = (inp["w_gu"], inp["w_down"]) + ((inp["w_gu_scale"], inp["w_down_scale"]) if fp8 else ())
+    weights = [ep.local_weights(pl, r, cfg.n_shared, *full) for r in range(W)]
     loads = [ep.peer_compute(descs[r], exs[r], steps[r], M, *weights[r]) for r in range(W)]
     hs = [ep.peer_combine(descs[r], exs[r], steps[r], xs[r], None, *weights[r])
           for r in range(W)]
@@ -135,3 +154,23 @@ def test_emulated_peer_exchange_equals_single_gpu(world, n_redundant):
         f"max |diff| {float((h.float() - h_ref.float()).abs().max()):.3e}"
     assert sum(loads) == CFG.T * CFG.top_k
     print(f"peer W={world} redundant={n_redundant}: rows per rank {loads}")
+
+
+CFG_FP8 = dataclasses.replace(CFG, dtype="e4m3", name="v3_fp8-ep")
+
+
+@pytest.mark.parametrize("world,n_redundant,peer", [(1, 0, False), (4, 0, False), (4, 4, False),
+                                                    (2, 0, True), (4, 4, True)])
+def test_emulated_fp8_expert_parallel_equals_single_gpu(world, n_redundant, peer):
+    """§3.6's FP8 dispatch: rows travel as 1x128 E4M3 codes with their scales,
+    expert outputs come back in bf16; equal to the FP8 moe_forward bit for bit."""
+    moe.moe_last_device_status()
+    inp = fp8_inputs(CFG_FP8)
+    h_ref, counts = reference(CFG_FP8, inp)
+    replicas = ep.choose_replicas(counts, world, n_redundant) if n_redundant else {}
+    pl = ep.Placement(CFG_FP8.n_routed, world, replicas)
+    h, loads = (emulate_peer if peer else emulate)(CFG_FP8, inp, pl)
+    assert moe.moe_last_device_status() == moe.OK
+    assert torch.equal(h, h_ref), \
+        f"max |diff| {float((h.float() - h_ref.float()).abs().max()):.3e}"
+    assert sum(loads) == CFG_FP8.T * CFG_FP8.top_k

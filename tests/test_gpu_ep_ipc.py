@@ -5,7 +5,9 @@ the dispatch kernel of each rank stores into the other process's receive
 buffer, the down projection of each rank into the other's return buffer.
 The phases are ordered on the host (device synchronise, then a gloo barrier);
 no kernel waits on the other process.  Each rank's output must equal
-moe_forward over the whole batch, bit for bit, on its token shard."""
+moe_forward over the whole batch, bit for bit, on its token shard, for a
+bf16 layer and for an E4M3 one (rows exchanged as 1x128 codes with their
+scales, outputs returned in bf16)."""
 import dataclasses
 import os
 import socket
@@ -25,7 +27,7 @@ def _free_port():
         return s.getsockname()[1]
 
 
-def _rank_main(rank, world, port, n_redundant, out):
+def _rank_main(rank, world, port, n_redundant, fp8, out):
     sys.path.insert(0, ROOT)
     import datetime
 
@@ -43,14 +45,25 @@ def _rank_main(rank, world, port, n_redundant, out):
                                 timeout=datetime.timedelta(seconds=60))
         cfg = dataclasses.replace(
             recipes.small_variant(recipes.CONFIGS["v3_bf16"], T=777, d=512, inter=256,
-                                  n_routed=32), n_group=4, topk_group=2)
+                                  n_routed=32), n_group=4, topk_group=2,
+            dtype="e4m3" if fp8 else "bf16")
         inp = recipes.device_inputs(cfg)
+        if fp8:                                  # 128x128 E4M3 expert weights
+            E, I, d = cfg.n_experts, cfg.inter, cfg.d
+            gq = torch.empty(E, 2 * I, d, dtype=torch.uint8, device="cuda")
+            gs = torch.empty(E, 2 * I // 128, d // 128, dtype=torch.float32, device="cuda")
+            dq = torch.empty(E, d, I, dtype=torch.uint8, device="cuda")
+            ds = torch.empty(E, d // 128, I // 128, dtype=torch.float32, device="cuda")
+            moe.moe_quantize_fp8_blockwise(inp["w_gu"], 2 * I, d, E, gq, gs)
+            moe.moe_quantize_fp8_blockwise(inp["w_down"], d, I, E, dq, ds)
+            inp.update(w_gu=gq, w_gu_scale=gs, w_down=dq, w_down_scale=ds)
         desc_all = moe.desc_from_config(cfg)
         ws_all = moe.workspace(desc_all)
         h_ref = torch.empty(cfg.T, cfg.d, dtype=torch.bfloat16, device="cuda")
         counts = torch.empty(cfg.n_routed, dtype=torch.int32, device="cuda")
-        moe.moe_forward(desc_all, inp["x"], None, inp["w_r"], inp["bias"], inp["w_gu"], None,
-                        inp["w_down"], None, h_ref, None, counts, ws_all)
+        moe.moe_forward(desc_all, inp["x"], None, inp["w_r"], inp["bias"], inp["w_gu"],
+                        inp.get("w_gu_scale"), inp["w_down"], inp.get("w_down_scale"), h_ref,
+                        None, counts, ws_all)
         replicas = ep.choose_replicas(counts.cpu().numpy(), world, n_redundant) \
             if n_redundant else {}
         pl = ep.Placement(cfg.n_routed, world, replicas)
@@ -58,13 +71,17 @@ def _rank_main(rank, world, port, n_redundant, out):
         c = dataclasses.replace(cfg, T=hi - lo)
         desc = moe.desc_from_config(c)
         x = inp["x"][lo:hi].contiguous()
-        w_gu, w_down = ep.local_weights(pl, rank, cfg.n_shared, inp["w_gu"], inp["w_down"])
+        full = (inp["w_gu"], inp["w_down"]) + \
+            ((inp["w_gu_scale"], inp["w_down_scale"]) if fp8 else ())
+        wl = ep.local_weights(pl, rank, cfg.n_shared, *full)
+        w_gu, w_down = wl[:2]
+        scales = wl[2:] if fp8 else (None, None)
         ex = ep.PeerExchange(desc, pl, rank, cfg.T * cfg.top_k, "cuda", torch.bfloat16)
         ex.open_peers()
         outs = []
         for _ in range(2):                      # twice: the buffers are reused
             h, n = ep.ep_forward_peer(desc, pl, rank, x, None, inp["w_r"], inp["bias"], w_gu,
-                                      w_down, ex)
+                                      w_down, ex, w_gu_scale=scales[0], w_down_scale=scales[1])
             torch.cuda.synchronize()
             outs.append((bool(torch.equal(h, h_ref[lo:hi])), int(n)))
         st = moe.moe_last_device_status()
@@ -76,12 +93,12 @@ def _rank_main(rank, world, port, n_redundant, out):
         out.put((rank, None, None, repr(e)))
 
 
-@pytest.mark.parametrize("n_redundant", [0, 4])
-def test_ipc_peer_exchange_two_processes(n_redundant):
+@pytest.mark.parametrize("n_redundant,fp8", [(0, False), (4, False), (4, True)])
+def test_ipc_peer_exchange_two_processes(n_redundant, fp8):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_rank_main, args=(r, 2, port, n_redundant, q)) for r in range(2)]
+    procs = [ctx.Process(target=_rank_main, args=(r, 2, port, n_redundant, fp8, q)) for r in range(2)]
     for p in procs:
         p.start()
     results = {}

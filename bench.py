@@ -556,15 +556,17 @@ def run_backward(args, cfg):
     del dh32
     E, I, d, N = cfg.n_experts, cfg.inter, cfg.d, cfg.n_routed
     dx = torch.empty(cfg.T, d, dtype=torch.bfloat16, device="cuda")
-    dwr = torch.empty(N, d, dtype=torch.float32, device="cuda")
-    dwgu = torch.empty(E, 2 * I, d, dtype=torch.float32, device="cuda")
-    dwd = torch.empty(E, d, I, dtype=torch.float32, device="cuda")
+    gdt = torch.bfloat16 if args.bf16_grads else torch.float32
+    dwr = torch.empty(N, d, dtype=gdt, device="cuda")
+    dwgu = torch.empty(E, 2 * I, d, dtype=gdt, device="cuda")
+    dwd = torch.empty(E, d, I, dtype=gdt, device="cuda")
     ws = moe.backward_workspace(desc)
     stream = torch.cuda.current_stream()
+    call = moe.moe_backward_bf16_grads if args.bf16_grads else moe.moe_backward
 
     def step():
-        moe.moe_backward(desc, inp["x"], inp["w_r"], inp["bias"], inp["w_gu"], inp["w_down"], dh,
-                         dx, dwr, dwgu, dwd, ws, stream)
+        call(desc, inp["x"], inp["w_r"], inp["bias"], inp["w_gu"], inp["w_down"], dh, dx, dwr,
+             dwgu, dwd, ws, stream)
 
     for _ in range(args.warmup):
         step()
@@ -594,6 +596,7 @@ def run_backward(args, cfg):
             "unit": "tokens/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": cfg.dtype, "data": "synthetic", "config": config_dict(cfg, 1),
+            "weight_gradients": "bf16" if args.bf16_grads else "fp32",
             "backward_gemm_tflops": tflops,
             "backward_gemm_frac_of_peak": {
                 "measured_sustained": tflops / pk["bf16_tflops_sustained"],
@@ -617,6 +620,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--backward", action="store_true",
                     help="time the layer backward (moe_backward) instead of the forward")
+    ap.add_argument("--bf16-grads", action="store_true",
+                    help="with --backward: weight gradients in bf16 (moe_backward_bf16_grads)")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")

@@ -86,6 +86,8 @@ _SIGS = {
     "moe_backward": (ctypes.c_int, [_D, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                                     ctypes.c_size_t, _P]),
     "moe_backward_launch_count": (ctypes.c_int32, [_D]),
+    "moe_backward_bf16_grads": (ctypes.c_int, [_D, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
+                                               ctypes.c_size_t, _P]),
     "moe_expert_ffn_workspace_size": (ctypes.c_size_t, [_D, ctypes.c_int32, ctypes.c_int32]),
     "moe_expert_ffn": (ctypes.c_int, [_D, ctypes.c_int32, ctypes.c_int32, _P, ctypes.c_int32,
                                       ctypes.c_int32, _P, _P, _P, _P, _P, _P, ctypes.c_size_t,
@@ -346,6 +348,23 @@ def moe_backward(desc, x, w_router, bias, w_gu, w_down, dh, dx, dw_router, dw_gu
                              _ptr(w_down), _ptr(dh), _ptr(dx), _ptr(dw_router), _ptr(dw_gu),
                              _ptr(dw_down), _ptr(ws), ws.numel() if ws is not None else 0,
                              _stream(stream)), "moe_backward")
+
+
+def moe_backward_bf16_grads(desc, x, w_router, bias, w_gu, w_down, dh, dx, dw_router, dw_gu,
+                            dw_down, ws, stream=None) -> None:
+    """moe_backward with the weight gradients written as bf16 tensors."""
+    _need("moe_backward_bf16_grads", desc, x=x, w_router=w_router, bias=bias, w_gu=w_gu,
+          w_down=w_down, dh=dh, dx=dx)
+    sz = _sizes(desc)
+    for name, t in (("dw_router", dw_router), ("dw_gu", dw_gu), ("dw_down", dw_down)):
+        if not t.is_contiguous() or t.element_size() != 2 or 2 * t.numel() * 2 < sz[name]:
+            raise MoeError(ERR_INVALID_ARG, f"moe_backward_bf16_grads: {name} must be a "
+                           "contiguous bf16 tensor of the gradient's shape")
+    _check(_lib.moe_backward_bf16_grads(ctypes.byref(desc), _ptr(x), _ptr(w_router), _ptr(bias),
+                                        _ptr(w_gu), _ptr(w_down), _ptr(dh), _ptr(dx),
+                                        _ptr(dw_router), _ptr(dw_gu), _ptr(dw_down), _ptr(ws),
+                                        ws.numel() if ws is not None else 0, _stream(stream)),
+           "moe_backward_bf16_grads")
 
 
 def moe_backward_launch_count(desc) -> int:

@@ -957,21 +957,25 @@ moe_status launch_gemm_bwd(const char* what, Operand a0, Operand a1, Operand b0,
   return launched(what);
 }
 
-// Output map of the weight-gradient GEMMs: fp32 [nz][m][ldc], box 32 x 32 x 1,
-// 128-byte swizzle (the epilogue's staging layout).  Rows are one expert's,
+// Output map of the weight-gradient GEMMs: fp32 or bf16 [nz][m][ldc], box
+// 32 x 32 x 1; fp32 with the 128-byte swizzle, bf16 unswizzled (the
+// epilogue's staging layouts).  Rows are one expert's,
 // so a TMA store clips at the expert's last row and at the row's end.
-moe_status make_tmap_out(CUtensorMap* mp, void* base, uint64_t ldc, uint64_t m, uint64_t nz) {
-  if (ldc % 4 != 0 || m == 0 || nz == 0) {
-    snprintf(t_errmsg, sizeof(t_errmsg), "weight-gradient output map: row length %llu must be a "
-             "multiple of 4", (unsigned long long)ldc);
+moe_status make_tmap_out(CUtensorMap* mp, void* base, uint64_t ldc, uint64_t m, uint64_t nz,
+                         bool bf16) {
+  const uint64_t esz = bf16 ? 2 : 4;
+  if ((ldc * esz) % 16 != 0 || m == 0 || nz == 0) {
+    snprintf(t_errmsg, sizeof(t_errmsg), "weight-gradient output map: rows of %llu elements "
+             "are not a multiple of 16 bytes", (unsigned long long)ldc);
     return MOE_ERR_UNSUPPORTED;
   }
   cuuint64_t dims[3] = {ldc, m, nz};
-  cuuint64_t strides[2] = {ldc * 4, m * ldc * 4};
+  cuuint64_t strides[2] = {ldc * esz, m * ldc * esz};
   cuuint32_t box[3] = {32, 32, 1};
   cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = g_encode(mp, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, estr,
-                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+  CUresult r = g_encode(mp, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                        3, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        bf16 ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B,
                         CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) {
     snprintf(t_errmsg, sizeof(t_errmsg), "cuTensorMapEncodeTiled (gradient output): CUresult %d "
@@ -988,13 +992,13 @@ moe_status make_tmap_out(CUtensorMap* mp, void* base, uint64_t ldc, uint64_t m, 
 // args.ldc columns; the epilogue stores through a [n_z][m_rows][ldc] map.
 moe_status launch_gemm_bwd_pair(const char* what, Operand a0, Operand a1, Operand b0, Operand b1,
                                 gbwd::Args args, uint64_t m_rows, uint64_t n_z,
-                                int64_t pair_tiles_bound, cudaStream_t st) {
+                                int64_t pair_tiles_bound, bool bf16_out, cudaStream_t st) {
   CUtensorMap ta0, ta1, tb0, tb1, tc;
   moe_status rc = make_tmap_mn(&ta0, a0.base, a0.inner, a0.rows);
   if (rc == MOE_OK) rc = make_tmap_mn(&ta1, a1.base, a1.inner, a1.rows);
   if (rc == MOE_OK) rc = make_tmap_mn(&tb0, b0.base, b0.inner, b0.rows);
   if (rc == MOE_OK) rc = make_tmap_mn(&tb1, b1.base, b1.inner, b1.rows);
-  if (rc == MOE_OK) rc = make_tmap_out(&tc, args.c, (uint64_t)args.ldc, m_rows, n_z);
+  if (rc == MOE_OK) rc = make_tmap_out(&tc, args.c, (uint64_t)args.ldc, m_rows, n_z, bf16_out);
   if (rc != MOE_OK) return rc;
   int stages = 0;
   for (int s = 6; s >= 2 && !stages; --s)
@@ -1002,15 +1006,14 @@ moe_status launch_gemm_bwd_pair(const char* what, Operand a0, Operand a1, Operan
   if (!stages) return MOE_ERR_UNSUPPORTED;
   args.stages = stages;
   const size_t smem = gbwd::pair_smem_bytes(stages, args.n_probs);
-  cudaError_t e = cudaFuncSetAttribute(gbwd::k_gemm_bwd_pair,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
+  auto* k = bf16_out ? gbwd::k_gemm_bwd_pair<true> : gbwd::k_gemm_bwd_pair<false>;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
   if (e != cudaSuccess) return cuda_fail(e, what);
   cudaLaunchConfig_t cfg;
   cudaLaunchAttribute attr[2];
-  rc = pair_config(2, gbwd::k_gemm_bwd_pair, gbwd::NUM_THREADS, smem, pair_tiles_bound, st, &cfg,
-                   attr);
+  rc = pair_config(2, k, gbwd::NUM_THREADS, smem, pair_tiles_bound, st, &cfg, attr);
   if (rc != MOE_OK) return rc;
-  e = cudaLaunchKernelEx(&cfg, gbwd::k_gemm_bwd_pair, ta0, ta1, tb0, tb1, tc, args);
+  e = cudaLaunchKernelEx(&cfg, k, ta0, ta1, tb0, tb1, tc, args);
   if (e != cudaSuccess) return cuda_fail(e, what);
   return launched(what);
 }
@@ -1026,8 +1029,8 @@ moe_status launch_gate_bwd(const float* logits, const route::Params& p, const in
 moe_status do_backward(const moe_layer_desc& s, const Dims& D, const Layout& L,
                        const BwdLayout& B, const void* x, const void* w_router,
                        const float* bias, const void* w_gu, const void* w_down, const void* dh,
-                       void* dx, float* dw_router, float* dw_gu, float* dw_down, uint8_t* ws,
-                       int sms, cudaStream_t st) {
+                       void* dx, void* dw_router, void* dw_gu, void* dw_down, bool bf16_grads,
+                       uint8_t* ws, int sms, cudaStream_t st) {
   const int T = (int)D.T, d = (int)D.d, I = (int)D.I, N = (int)D.N, K = (int)D.K;
   const int Ks = (int)D.Ks, E = (int)D.E;
   int32_t* idx = reinterpret_cast<int32_t*>(ws + L.topk_idx);
@@ -1159,7 +1162,8 @@ moe_status do_backward(const moe_layer_desc& s, const Dims& D, const Layout& L,
   ga.c = dw_down;
   ga.ldc = I;
   rc = launch_gemm_bwd_pair("backward GEMM dW_down = dY^T Z (CTA pairs)", DH, DHP, ZG, ZG, ga,
-                            (uint64_t)d, (uint64_t)E, (int64_t)E * ((d + 255) / 256) * nt(I), st);
+                            (uint64_t)d, (uint64_t)E, (int64_t)E * ((d + 255) / 256) * nt(I),
+                            bf16_grads, st);
   if (rc != MOE_OK) return rc;
   // G5: dW_gu = [da | db]^T X over each expert's rows
   ga.tab = tab[4];
@@ -1167,7 +1171,7 @@ moe_status do_backward(const moe_layer_desc& s, const Dims& D, const Layout& L,
   ga.ldc = d;
   rc = launch_gemm_bwd_pair("backward GEMM dW_gu = dAB^T X (CTA pairs)", DAB, DAB, X, XP, ga,
                             (uint64_t)(2 * I), (uint64_t)E,
-                            (int64_t)E * ((2 * I + 255) / 256) * nt(d), st);
+                            (int64_t)E * ((2 * I + 255) / 256) * nt(d), bf16_grads, st);
   if (rc != MOE_OK) return rc;
   // G6b: dW_r = dl^T X over all tokens
   ga.n_probs = 1;
@@ -1175,7 +1179,7 @@ moe_status do_backward(const moe_layer_desc& s, const Dims& D, const Layout& L,
   ga.c = dw_router;
   ga.ldc = d;
   return launch_gemm_bwd_pair("backward GEMM dW_r = dL^T X (CTA pairs)", DL, DL, X, X, ga,
-                              (uint64_t)N, 1, ((N + 255) / 256) * nt(d), st);
+                              (uint64_t)N, 1, ((N + 255) / 256) * nt(d), bf16_grads, st);
 }
 
 __global__ void k_selftest_wait(uint64_t limit_ns) {
@@ -1538,10 +1542,11 @@ size_t moe_backward_workspace_size(const moe_layer_desc* desc) {
   return bwd_layout(D, L).total;
 }
 
-moe_status moe_backward(const moe_layer_desc* desc, const void* x, const void* w_router,
-                        const float* bias, const void* w_gu, const void* w_down, const void* dh,
-                        void* dx, float* dw_router, float* dw_gu, float* dw_down, void* ws,
-                        size_t ws_bytes, cudaStream_t stream) {
+static moe_status backward_entry(const moe_layer_desc* desc, const void* x,
+                                 const void* w_router, const float* bias, const void* w_gu,
+                                 const void* w_down, const void* dh, void* dx, void* dw_router,
+                                 void* dw_gu, void* dw_down, bool bf16_grads, void* ws,
+                                 size_t ws_bytes, cudaStream_t stream) {
   Dims D;
   moe_status rc = fill_dims(desc, &D);
   if (rc != MOE_OK) return rc;
@@ -1564,7 +1569,24 @@ moe_status moe_backward(const moe_layer_desc* desc, const void* x, const void* w
   int sms;
   if ((rc = device_setup(&sms)) != MOE_OK) return rc;
   return do_backward(*desc, D, L, B, x, w_router, bias, w_gu, w_down, dh, dx, dw_router, dw_gu,
-                     dw_down, static_cast<uint8_t*>(ws), sms, stream);
+                     dw_down, bf16_grads, static_cast<uint8_t*>(ws), sms, stream);
+}
+
+moe_status moe_backward(const moe_layer_desc* desc, const void* x, const void* w_router,
+                        const float* bias, const void* w_gu, const void* w_down, const void* dh,
+                        void* dx, float* dw_router, float* dw_gu, float* dw_down, void* ws,
+                        size_t ws_bytes, cudaStream_t stream) {
+  return backward_entry(desc, x, w_router, bias, w_gu, w_down, dh, dx, dw_router, dw_gu, dw_down,
+                        false, ws, ws_bytes, stream);
+}
+
+moe_status moe_backward_bf16_grads(const moe_layer_desc* desc, const void* x,
+                                   const void* w_router, const float* bias, const void* w_gu,
+                                   const void* w_down, const void* dh, void* dx, void* dw_router,
+                                   void* dw_gu, void* dw_down, void* ws, size_t ws_bytes,
+                                   cudaStream_t stream) {
+  return backward_entry(desc, x, w_router, bias, w_gu, w_down, dh, dx, dw_router, dw_gu, dw_down,
+                        true, ws, ws_bytes, stream);
 }
 
 int32_t moe_backward_launch_count(const moe_layer_desc* desc) {

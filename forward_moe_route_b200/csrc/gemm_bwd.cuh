@@ -440,8 +440,9 @@ constexpr int PBM = 256;                 // rows per pair tile (128 per CTA)
 constexpr uint32_t PA_BYTES = 2 * MN_BOX_BYTES;   // a CTA's A: 128 rows of M (2 boxes of 64) x 64 K rows
 constexpr uint32_t PB_BYTES = 2 * MN_BOX_BYTES;   // its half of B: up to 128 columns of N
 constexpr uint32_t PSTAGE_BYTES = PA_BYTES + PB_BYTES;
-// fp32 store staging: per epilogue warp two 32 x 32 blocks (4 KB each) in the
-// 128-byte-swizzled layout of the output tensor map, written out by TMA
+// store staging: per epilogue warp two 32 x 32 blocks (4 KB each), written out
+// by TMA: fp32 in the 128-byte-swizzled layout of the output tensor map, or
+// bf16 (2 KB used) row-major for an unswizzled map
 constexpr uint32_t PSTORE_BYTES = 4 * 2 * 4096;
 
 __host__ inline size_t pair_smem_bytes(int stages, int n_probs) {
@@ -460,6 +461,7 @@ __device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void*
       : "memory");
 }
 
+template <bool OUT_BF16>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     k_gemm_bwd_pair(const __grid_constant__ CUtensorMap tmA0,
                     const __grid_constant__ CUtensorMap tmA1,
@@ -684,13 +686,29 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         // the store issued from this buffer two chunks ago has read it
         if (lane == 0) bulk_wait_group_read<1>();
         __syncwarp();
-        // row `lane`, 16-byte piece j at (j ^ (row % 8)) (128-byte swizzle)
+        if (OUT_BF16) {
+          // row `lane`: 32 bf16 = 64 bytes, plain row-major (the map has no swizzle)
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const uint32_t* src = j < 4 ? &va[4 * j] : &vb[4 * (j - 4)];
-          const uint4 v = has_k ? make_uint4(src[0], src[1], src[2], src[3])
-                                : make_uint4(0u, 0u, 0u, 0u);
-          *reinterpret_cast<uint4*>(buf + lane * 128 + ((j ^ (lane & 7)) << 4)) = v;
+          for (int j = 0; j < 4; ++j) {
+            const uint32_t* src = j < 2 ? &va[8 * j] : &vb[8 * (j - 2)];
+            uint32_t w4[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              w4[i] = has_k ? gemm::pack_bf16x2(__uint_as_float(src[2 * i]),
+                                                __uint_as_float(src[2 * i + 1]))
+                            : 0u;
+            *reinterpret_cast<uint4*>(buf + lane * 64 + j * 16) =
+                make_uint4(w4[0], w4[1], w4[2], w4[3]);
+          }
+        } else {
+          // row `lane`, 16-byte piece j at (j ^ (row % 8)) (128-byte swizzle)
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const uint32_t* src = j < 4 ? &va[4 * j] : &vb[4 * (j - 4)];
+            const uint4 v = has_k ? make_uint4(src[0], src[1], src[2], src[3])
+                                  : make_uint4(0u, 0u, 0u, 0u);
+            *reinterpret_cast<uint4*>(buf + lane * 128 + ((j ^ (lane & 7)) << 4)) = v;
+          }
         }
         fence_proxy_async_smem();
         __syncwarp();

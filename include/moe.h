@@ -387,6 +387,17 @@ moe_status moe_backward(const moe_layer_desc* desc, const void* x, const void* w
                         void* dx, float* dw_router, float* dw_gu, float* dw_down, void* ws,
                         size_t ws_bytes, cudaStream_t stream);
 
+/* moe_backward with the three weight gradients written as bf16 (rounded to
+ * nearest even from the fp32 accumulators) instead of fp32: §3.6 of the same
+ * report keeps weight gradients in BF16 (master weights and optimizer maths in
+ * FP32).  dw_router [N, d], dw_gu [E, 2I, d], dw_down [E, d, I] bf16 out;
+ * everything else as moe_backward. */
+moe_status moe_backward_bf16_grads(const moe_layer_desc* desc, const void* x,
+                                   const void* w_router, const float* bias, const void* w_gu,
+                                   const void* w_down, const void* dh, void* dx, void* dw_router,
+                                   void* dw_gu, void* dw_down, void* ws, size_t ws_bytes,
+                                   cudaStream_t stream);
+
 /* Number of kernels moe_backward launches for `desc` (0 if invalid or T = 0). */
 int32_t moe_backward_launch_count(const moe_layer_desc* desc);
 

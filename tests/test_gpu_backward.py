@@ -134,3 +134,31 @@ def test_backward_is_deterministic():
     assert a[4] == moe.OK and b[4] == moe.OK
     for x, y in zip(a[:4], b[:4]):
         assert torch.equal(x, y)
+
+
+@pytest.mark.parametrize("name", ["v3_small", "dsmoe16b_small", "v3_T1"])
+def test_backward_bf16_weight_gradients(name):
+    """moe_backward_bf16_grads (weight gradients kept in BF16, as §3.6 keeps
+    them): the same fp32 accumulators rounded to nearest even, so each bf16
+    gradient equals the fp32 call's gradient cast to bf16 bit for bit, and dx
+    is unchanged."""
+    cfg = CASES[name]
+    moe.moe_last_device_status()
+    inp = recipes.device_inputs(cfg)
+    dh, _ = upstream(cfg)
+    dx, dwr, dwgu, dwd, st = run_backward(cfg, inp, dh)
+    assert st == moe.OK
+    desc = moe.desc_from_config(cfg)
+    ws = moe.backward_workspace(desc)
+    E, I, d, N = cfg.n_experts, cfg.inter, cfg.d, cfg.n_routed
+    bf = dict(dtype=torch.bfloat16, device="cuda")
+    dx2 = torch.full((cfg.T, d), float("nan"), **bf)
+    dwr2 = torch.full((N, d), float("nan"), **bf)
+    dwgu2 = torch.full((E, 2 * I, d), float("nan"), **bf)
+    dwd2 = torch.full((E, d, I), float("nan"), **bf)
+    moe.moe_backward_bf16_grads(desc, inp["x"], inp["w_r"], inp["bias"], inp["w_gu"],
+                                inp["w_down"], dh, dx2, dwr2, dwgu2, dwd2, ws)
+    assert moe.moe_last_device_status() == moe.OK
+    assert torch.equal(dx2, dx)
+    for got, ref in ((dwr2, dwr), (dwgu2, dwgu), (dwd2, dwd)):
+        assert torch.equal(got, ref.to(torch.bfloat16))

@@ -13,6 +13,11 @@ whole run ends in minutes:
   fp8       the same layer with E4M3 experts
   tiny      the tiny fp32 layer (tf32 GEMMs, fp32 router)
   backward  the V3-shaped layer with 8 routed experts, T = 2048
+  ep        the v3 case's layer (bf16, then E4M3) over two expert-parallel
+            ranks emulated on one GPU, exchanging over peer memory (local
+            addresses): peer dispatch, expert GEMMs with per-group output
+            addresses, the FP8 dispatch and row quantisation
+  backward_bf16  the backward case with bf16 weight gradients
 Inputs come from the seeded synthetic generator (synth/).
 """
 import argparse
@@ -131,8 +136,79 @@ def case_backward():
     torch.cuda.synchronize()
 
 
+def _quantised_weights(cfg, inp):
+    E, I, d = cfg.n_experts, cfg.inter, cfg.d
+    gq = torch.empty(E, 2 * I, d, dtype=torch.uint8, device="cuda")
+    gs = torch.empty(E, 2 * I // 128, d // 128, dtype=torch.float32, device="cuda")
+    dq = torch.empty(E, d, I, dtype=torch.uint8, device="cuda")
+    ds = torch.empty(E, d // 128, I // 128, dtype=torch.float32, device="cuda")
+    moe.moe_quantize_fp8_blockwise(inp["w_gu"], 2 * I, d, E, gq, gs)
+    moe.moe_quantize_fp8_blockwise(inp["w_down"], d, I, E, dq, ds)
+    inp.update(w_gu=gq, w_gu_scale=gs, w_down=dq, w_down_scale=ds)
+
+
+def case_ep():
+    import numpy as np
+    for dtype in ("bf16", "e4m3"):
+        cfg = dataclasses.replace(
+            recipes.small_variant(C["v3_bf16"], T=4096, d=7168, inter=2048, n_routed=32),
+            n_group=8, topk_group=4, dtype=dtype)
+        inp = recipes.device_inputs(cfg)
+        fp8 = dtype == "e4m3"
+        if fp8:
+            _quantised_weights(cfg, inp)
+        W = 2
+        pl = ep.Placement(cfg.n_routed, W)
+        full = (inp["w_gu"], inp["w_down"]) + \
+            ((inp["w_gu_scale"], inp["w_down_scale"]) if fp8 else ())
+        weights = [ep.local_weights(pl, r, cfg.n_shared, *full) for r in range(W)]
+        half = cfg.T // W
+        descs = [moe.desc_from_config(dataclasses.replace(cfg, T=half)) for _ in range(W)]
+        xs = [inp["x"][r * half:(r + 1) * half].contiguous() for r in range(W)]
+        for _ in range(2):
+            steps = [ep.ep_dispatch(descs[r], pl, r, xs[r], inp["w_r"], inp["bias"],
+                                    build_send=False) for r in range(W)]
+            M = np.stack([st.plan.send_counts for st in steps])
+            cap = int(M.sum(axis=(0, 2)).max())
+            exs = [ep.PeerExchange(descs[r], pl, r, cap, "cuda", torch.bfloat16)
+                   for r in range(W)]
+            ep.PeerExchange.link(exs)
+            for r in range(W):
+                ep.peer_dispatch(descs[r], exs[r], steps[r], xs[r], M)
+            for r in range(W):
+                ep.peer_compute(descs[r], exs[r], steps[r], M, *weights[r])
+            for r in range(W):
+                ep.peer_combine(descs[r], exs[r], steps[r], xs[r], None, *weights[r])
+        torch.cuda.synchronize()
+        del inp, weights, exs
+        torch.cuda.empty_cache()
+
+
+def case_backward_bf16():
+    import synth
+    cfg = dataclasses.replace(
+        recipes.small_variant(C["v3_bf16"], T=2048, d=7168, inter=2048, n_routed=8),
+        n_group=4, topk_group=2, top_k=4)
+    inp = recipes.device_inputs(cfg)
+    desc = moe.desc_from_config(cfg)
+    ws = moe.backward_workspace(desc)
+    dh32 = torch.empty(cfg.T, cfg.d, dtype=torch.float32, device="cuda")
+    synth.dev_fill_normal(dh32, 1.0, cfg.seed, 6)
+    dh = dh32.to(torch.bfloat16)
+    dx = torch.empty_like(dh)
+    E, I, d, N = cfg.n_experts, cfg.inter, cfg.d, cfg.n_routed
+    bf = dict(dtype=torch.bfloat16, device="cuda")
+    dwr = torch.empty(N, d, **bf)
+    dwgu = torch.empty(E, 2 * I, d, **bf)
+    dwd = torch.empty(E, d, I, **bf)
+    for _ in range(2):
+        moe.moe_backward_bf16_grads(desc, inp["x"], inp["w_r"], inp["bias"], inp["w_gu"],
+                                    inp["w_down"], dh, dx, dwr, dwgu, dwd, ws)
+    torch.cuda.synchronize()
+
+
 CASES = {"route": case_route, "v3": case_v3, "fp8": case_fp8, "tiny": case_tiny,
-         "backward": case_backward}
+         "backward": case_backward, "ep": case_ep, "backward_bf16": case_backward_bf16}
 
 
 def main():

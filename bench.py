@@ -499,6 +499,7 @@ def run_ours(args, cfg):
                             "stage_pass_ms_per_step",
             "route_permute_combine_gbs": rpc_gbs,
             "route_permute_combine_frac_of_hbm": rpc_gbs / pk["hbm_gbs"],
+            "route_permute_combine_frac_of_8tbs": rpc_gbs / 8000.0,
             "roofline": {"kernel": "grouped GEMM 1 (gate/up + SwiGLU epilogue)",
                          "bound": "tensor", "achieved": g1_tflops, "peak": peak,
                          "unit": "TFLOP/s", "frac": g1_tflops / peak,

@@ -55,7 +55,7 @@ extern "C" {
 typedef enum {
   MOE_OK = 0,
   MOE_ERR_INVALID_ARG = 1,   /* a size, pointer, alignment or mode is not accepted */
-  MOE_ERR_UNSUPPORTED = 2,   /* valid layer, but a shape this build does not handle */
+  MOE_ERR_UNSUPPORTED = 2,   /* valid layer, but a shape the library does not handle */
   MOE_ERR_WORKSPACE = 3,     /* ws_bytes below moe_workspace_size(desc) */
   MOE_ERR_CUDA = 4,          /* a CUDA runtime/driver call or a launch failed */
   MOE_ERR_TIMEOUT = 5,       /* a device-side bounded wait expired (device status) */

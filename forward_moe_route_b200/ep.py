@@ -29,8 +29,21 @@ Only the plan and the collectives live here; every other step runs in the
 library's CUDA kernels (moe_route, moe_permute, moe_dispatch_rows,
 moe_expert_ffn, moe_combine_rows).  The phases (ep_dispatch, ep_compute,
 ep_combine) are separate functions so that the exchange between them can be
-any transport; ep_forward chains them over torch.distributed.  The plan needs the rank's per-expert row counts on the
-host, so a step reads N integers back from the device before the exchange.
+any transport; ep_forward chains them over torch.distributed.  The plan needs
+the rank's per-expert row counts on the host, so a step reads N integers back
+from the device before the exchange.
+
+Exchange over peer memory (PeerExchange, ep_forward_peer): instead of a
+collective, the dispatch kernel stores each row straight into the receive
+buffer of the rank holding its expert, and the down projection of the
+expert GEMMs stores each output row straight into the return buffer of the
+rank that sent it (other processes' buffers mapped through CUDA IPC).  The
+ranks only all-gather their send matrices and order the phases with
+barriers.
+
+E4M3 layers (§3.6: FP8 dispatch, BF16 combine): the rows travel as 1x128
+E4M3 codes with their fp32 scales and the expert outputs come back in bf16,
+on either exchange.
 """
 from __future__ import annotations
 

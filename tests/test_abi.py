@@ -170,3 +170,53 @@ def test_binding_refuses_short_or_strided_buffers():
     short_scale = torch.zeros(64 * 4, 2, dtype=torch.float32)      # the T shared rows missing
     with pytest.raises(moe.MoeError, match="x_perm_scale holds"):
         moe.moe_permute(fp8, x, None, None, None, None, None, xp, short_scale, None)
+
+
+def test_expert_parallel_entry_points_reject_bad_arguments():
+    """The peer-memory, FP8 and IPC entry points refuse bad arguments on the
+    host, before any CUDA call."""
+    L = moe.lib()
+    bf, f8 = v3(T=64), v3(T=64, dtype="e4m3")
+    # peer dispatch: n_ranks out of range, start[] not ending at n_rows
+    P = moe.MoePeerRows()
+    P.n_ranks = 0
+    assert L.moe_dispatch_rows_to(ctypes.byref(bf), 16, 16, 16, 64, ctypes.byref(P),
+                                  None) == moe.ERR_INVALID_ARG
+    P.n_ranks = moe.MAX_PEERS + 1
+    assert L.moe_dispatch_rows_to(ctypes.byref(bf), 16, 16, 16, 64, ctypes.byref(P),
+                                  None) == moe.ERR_INVALID_ARG
+    P.n_ranks = 2
+    P.start[0], P.start[1], P.start[2] = 0, 10, 20          # does not end at n_rows = 64
+    P.x[0] = P.x[1] = 16
+    assert L.moe_dispatch_rows_to(ctypes.byref(bf), 16, 16, 16, 64, ctypes.byref(P),
+                                  None) == moe.ERR_INVALID_ARG
+    P.start[2] = 64
+    P.x[1] = 17                                              # misaligned destination
+    assert L.moe_dispatch_rows_to(ctypes.byref(bf), 16, 16, 16, 64, ctypes.byref(P),
+                                  None) == moe.ERR_INVALID_ARG
+    P.x[1] = 16                                              # E4M3 rows need scale buffers
+    assert L.moe_dispatch_rows_to(ctypes.byref(f8), 16, 16, 16, 64, ctypes.byref(P),
+                                  None) == moe.ERR_INVALID_ARG
+    # FP8 dispatch / quantisation only for E4M3 layers, with a scale output
+    assert L.moe_dispatch_rows_fp8(ctypes.byref(bf), 16, 16, 16, 64, 16, 16, 16,
+                                   None) == moe.ERR_INVALID_ARG
+    assert L.moe_dispatch_rows_fp8(ctypes.byref(f8), 16, 16, 16, 64, 16, None, 16,
+                                   None) == moe.ERR_INVALID_ARG
+    assert L.moe_quantize_rows_fp8(ctypes.byref(bf), 16, 4, 16, 16, None) == moe.ERR_INVALID_ARG
+    # FP8 expert FFN: exactly one of y_rows / group_out; bf16 layers go to moe_expert_ffn
+    args = (1, 1, 16, 64, 64, 16, 16, 16, 16, 16, 16, 16)
+    assert L.moe_expert_ffn_fp8(ctypes.byref(f8), *args, None, None, 16, 1 << 30,
+                                None) == moe.ERR_INVALID_ARG
+    assert L.moe_expert_ffn_fp8(ctypes.byref(f8), *args, 16, 16, 16, 1 << 30,
+                                None) == moe.ERR_INVALID_ARG
+    assert L.moe_expert_ffn_fp8(ctypes.byref(bf), *args, 16, None, 16, 1 << 30,
+                                None) == moe.ERR_INVALID_ARG
+    # per-group output addresses must be 8-byte aligned
+    assert L.moe_expert_ffn_to(ctypes.byref(bf), 1, 1, 16, 64, 64, 16, 16, 16, 16, 12, 16,
+                               1 << 30, None) == moe.ERR_INVALID_ARG
+    # IPC: null pointers
+    off = ctypes.c_uint64()
+    assert L.moe_ipc_get_handle(None, ctypes.create_string_buffer(64),
+                                ctypes.byref(off)) == moe.ERR_INVALID_ARG
+    assert L.moe_ipc_open(None, None) == moe.ERR_INVALID_ARG
+    assert L.moe_ipc_close(None) == moe.ERR_INVALID_ARG

@@ -540,7 +540,9 @@ def backward_flops(cfg):
 def run_backward(args, cfg):
     """One layer backward per step (moe_backward: routing, permutation, the
     recomputed pre-activations, dz with the SwiGLU backward, du, the gate and
-    affinity backward, dW_down, dW_gu, dW_r), inputs resident in HBM."""
+    affinity backward, dW_down, dW_gu, dW_r), inputs resident in HBM.  With
+    --saved the step is moe_backward_saved, which reads the pre-activations
+    moe_forward_save kept instead of recomputing them."""
     import torch
 
     import forward_moe_route_b200 as moe
@@ -563,11 +565,47 @@ def run_backward(args, cfg):
     dwd = torch.empty(E, d, I, dtype=gdt, device="cuda")
     ws = moe.backward_workspace(desc)
     stream = torch.cuda.current_stream()
-    call = moe.moe_backward_bf16_grads if args.bf16_grads else moe.moe_backward
+    fwd_cost = None
+    if args.saved:
+        # the forward keeps a | b (moe_forward_save, outside the timed region);
+        # its cost over the plain forward is timed alongside
+        ab = torch.empty(moe.moe_saved_ab_bytes(desc) // 2, dtype=torch.bfloat16, device="cuda")
+        fws = moe.workspace(desc)
+        h = torch.empty(cfg.T, d, dtype=torch.bfloat16, device="cuda")
 
-    def step():
-        call(desc, inp["x"], inp["w_r"], inp["bias"], inp["w_gu"], inp["w_down"], dh, dx, dwr,
-             dwgu, dwd, ws, stream)
+        def fwd(save):
+            if save:
+                moe.moe_forward_save(desc, inp["x"], None, inp["w_r"], inp["bias"], inp["w_gu"],
+                                     inp["w_down"], h, None, None, ab, fws, stream)
+            else:
+                moe.moe_forward(desc, inp["x"], None, inp["w_r"], inp["bias"], inp["w_gu"], None,
+                                inp["w_down"], None, h, None, None, fws, stream)
+
+        fwd_cost = {}
+        for save in (False, True, False, True):
+            for _ in range(3):
+                fwd(save)
+            f0 = torch.cuda.Event(enable_timing=True)
+            f1 = torch.cuda.Event(enable_timing=True)
+            f0.record(stream)
+            for _ in range(5):
+                fwd(save)
+            f1.record(stream)
+            torch.cuda.synchronize()
+            key = "forward_save_ms" if save else "forward_ms"
+            fwd_cost[key] = min(fwd_cost.get(key, 1e30), f0.elapsed_time(f1) / 5)
+        del fws
+
+        def step():
+            moe.moe_backward_saved(desc, inp["x"], inp["w_r"], inp["bias"], inp["w_gu"],
+                                   inp["w_down"], dh, ab, dx, dwr, dwgu, dwd, ws,
+                                   bf16_grads=args.bf16_grads, stream=stream)
+    else:
+        call = moe.moe_backward_bf16_grads if args.bf16_grads else moe.moe_backward
+
+        def step():
+            call(desc, inp["x"], inp["w_r"], inp["bias"], inp["w_gu"], inp["w_down"], dh, dx,
+                 dwr, dwgu, dwd, ws, stream)
 
     for _ in range(args.warmup):
         step()
@@ -591,20 +629,23 @@ def run_backward(args, cfg):
     ms = e0.elapsed_time(e1) / args.steps
     fl = backward_flops(cfg)
     pk = peaks()
-    done = fl["algorithmic"] + fl["recompute"] + fl["router"]
+    done = fl["algorithmic"] + (0.0 if args.saved else fl["recompute"]) + fl["router"]
     tflops = done / (ms * 1e-3) / 1e12
     return {"metric": "MoE-layer backward tokens/s", "value": cfg.T / (ms * 1e-3),
             "unit": "tokens/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": cfg.dtype, "data": "synthetic", "config": config_dict(cfg, 1),
             "weight_gradients": "bf16" if args.bf16_grads else "fp32",
+            "pre_activations": "saved by the forward" if args.saved else "recomputed",
+            "forward_cost": fwd_cost,
             "backward_gemm_tflops": tflops,
             "backward_gemm_frac_of_peak": {
                 "measured_sustained": tflops / pk["bf16_tflops_sustained"],
                 "spec_dense": tflops / 2250.0},
             "backward_flops": fl,
             "algorithmic_tflops": (fl["algorithmic"] + fl["router"]) / (ms * 1e-3) / 1e12,
-            "gpu_launches": moe.moe_backward_launch_count(desc) * args.steps,
+            "gpu_launches": (moe.moe_backward_launch_count(desc) - (1 if args.saved else 0))
+            * args.steps,
             "clocks": clk}
 
 
@@ -623,6 +664,9 @@ def main():
                     help="time the layer backward (moe_backward) instead of the forward")
     ap.add_argument("--bf16-grads", action="store_true",
                     help="with --backward: weight gradients in bf16 (moe_backward_bf16_grads)")
+    ap.add_argument("--saved", action="store_true",
+                    help="with --backward: the pre-activations kept by moe_forward_save "
+                    "(moe_backward_saved) instead of recomputed")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")

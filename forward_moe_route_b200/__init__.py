@@ -106,6 +106,11 @@ _SIGS = {
                                           _P, ctypes.c_size_t, _P]),
     "moe_ipc_open": (ctypes.c_int, [_P, ctypes.POINTER(ctypes.c_void_p)]),
     "moe_ipc_close": (ctypes.c_int, [_P]),
+    "moe_saved_ab_bytes": (ctypes.c_size_t, [_D]),
+    "moe_forward_save": (ctypes.c_int, [_D, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
+                                        ctypes.c_size_t, _P]),
+    "moe_backward_saved": (ctypes.c_int, [_D, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
+                                          ctypes.c_int32, _P, ctypes.c_size_t, _P]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _f = getattr(_lib, _name)
@@ -163,7 +168,7 @@ def _sizes(desc) -> dict:
         "w_down_scale": E * (d // 128) * (I // 128) * 4 if fp8 else 0,
         "y_slots": T * (K + Ks) * d * a, "s_out": T * N * 4,
         "dh": T * d * a, "dx": T * d * a, "dw_router": N * d * 4, "dw_gu": E * 2 * I * d * 4,
-        "dw_down": E * d * I * 4,
+        "dw_down": E * d * I * 4, "ab_saved": (R + Ks * T) * 2 * I * 2,
     }
 
 
@@ -273,6 +278,22 @@ def moe_forward(desc, x, x_residual, w_router, bias, w_gu, w_gu_scale, w_down, w
                             ws.numel() if ws is not None else 0, _stream(stream)), "moe_forward")
 
 
+def moe_saved_ab_bytes(desc: MoeLayerDesc) -> int:
+    return int(_lib.moe_saved_ab_bytes(ctypes.byref(desc)))
+
+
+def moe_forward_save(desc, x, x_residual, w_router, bias, w_gu, w_down, h, topk_idx, counts,
+                     ab_saved, ws, stream=None) -> None:
+    """moe_forward that also writes the expert pre-activations a | b to ab_saved."""
+    _need("moe_forward_save", desc, x=x, x_residual=x_residual, w_router=w_router, bias=bias,
+          w_gu=w_gu, w_down=w_down, h=h, topk_idx=topk_idx, counts=counts, ab_saved=ab_saved)
+    _check(_lib.moe_forward_save(ctypes.byref(desc), _ptr(x), _ptr(x_residual), _ptr(w_router),
+                                 _ptr(bias), _ptr(w_gu), _ptr(w_down), _ptr(h), _ptr(topk_idx),
+                                 _ptr(counts), _ptr(ab_saved), _ptr(ws),
+                                 ws.numel() if ws is not None else 0, _stream(stream)),
+           "moe_forward_save")
+
+
 def moe_route_affinities(desc, x, w_router, s_out, ws, stream=None) -> None:
     _need("moe_route_affinities", desc, x=x, w_router=w_router, s_out=s_out)
     _check(_lib.moe_route_affinities(ctypes.byref(desc), _ptr(x), _ptr(w_router), _ptr(s_out),
@@ -365,6 +386,27 @@ def moe_backward_bf16_grads(desc, x, w_router, bias, w_gu, w_down, dh, dx, dw_ro
                                         _ptr(dw_router), _ptr(dw_gu), _ptr(dw_down), _ptr(ws),
                                         ws.numel() if ws is not None else 0, _stream(stream)),
            "moe_backward_bf16_grads")
+
+
+def moe_backward_saved(desc, x, w_router, bias, w_gu, w_down, dh, ab_saved, dx, dw_router,
+                       dw_gu, dw_down, ws, bf16_grads: bool = False, stream=None) -> None:
+    """The backward from the pre-activations moe_forward_save kept."""
+    _need("moe_backward_saved", desc, x=x, w_router=w_router, bias=bias, w_gu=w_gu,
+          w_down=w_down, dh=dh, dx=dx, ab_saved=ab_saved)
+    sz = _sizes(desc)
+    esz = 2 if bf16_grads else 4
+    for name, t in (("dw_router", dw_router), ("dw_gu", dw_gu), ("dw_down", dw_down)):
+        if t is None:
+            continue
+        if not t.is_contiguous() or t.element_size() != esz or t.numel() * 4 < sz[name]:
+            raise MoeError(ERR_INVALID_ARG, f"moe_backward_saved: {name} must be a contiguous "
+                           f"{'bf16' if bf16_grads else 'fp32'} tensor of the gradient's shape")
+    _check(_lib.moe_backward_saved(ctypes.byref(desc), _ptr(x), _ptr(w_router), _ptr(bias),
+                                   _ptr(w_gu), _ptr(w_down), _ptr(dh), _ptr(ab_saved), _ptr(dx),
+                                   _ptr(dw_router), _ptr(dw_gu), _ptr(dw_down),
+                                   1 if bf16_grads else 0, _ptr(ws),
+                                   ws.numel() if ws is not None else 0, _stream(stream)),
+           "moe_backward_saved")
 
 
 def moe_backward_launch_count(desc) -> int:

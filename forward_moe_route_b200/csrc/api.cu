@@ -619,7 +619,7 @@ moe_status do_grouped(const Dims& D, const Layout& L, const void* x, const void*
                       const float* x_perm_scale, const int32_t* offsets, const int32_t* slot_of,
                       const float* topk_w, const void* w_gu, const float* w_gu_scale,
                       const void* w_down, const float* w_down_scale, void* y_slots, uint8_t* ws,
-                      int sms, cudaStream_t st) {
+                      int sms, cudaStream_t st, __nv_bfloat16* ab_save = nullptr) {
   if (D.T == 0) return MOE_OK;
   const int E = (int)D.E;
   int32_t* gtab = reinterpret_cast<int32_t*>(ws + L.gtab);
@@ -660,6 +660,7 @@ moe_status do_grouped(const Dims& D, const Layout& L, const void* x, const void*
     a.fmt = fmt;
     a.out_bf16 = D.f32 ? 0 : 1;
     a.h = hbuf;
+    a.ab = ab_save;
     rc = launch_gate_up(kind, w_gu, D.E, x, x_perm, esz, D.T, D.R, tok_tiles, a, st);
     if (rc != MOE_OK) return rc;
     if ((rc = trace(3, st)) != MOE_OK) return rc;
@@ -1030,7 +1031,7 @@ moe_status do_backward(const moe_layer_desc& s, const Dims& D, const Layout& L,
                        const BwdLayout& B, const void* x, const void* w_router,
                        const float* bias, const void* w_gu, const void* w_down, const void* dh,
                        void* dx, void* dw_router, void* dw_gu, void* dw_down, bool bf16_grads,
-                       uint8_t* ws, int sms, cudaStream_t st) {
+                       const void* ab_saved, uint8_t* ws, int sms, cudaStream_t st) {
   const int T = (int)D.T, d = (int)D.d, I = (int)D.I, N = (int)D.N, K = (int)D.K;
   const int Ks = (int)D.Ks, E = (int)D.E;
   int32_t* idx = reinterpret_cast<int32_t*>(ws + L.topk_idx);
@@ -1109,17 +1110,20 @@ moe_status do_backward(const moe_layer_desc& s, const Dims& D, const Layout& L,
   ga.K = K;
   ga.Ks = Ks;
   ga.inter = I;
-  // G1: a | b pre-activations of every (row, expert)
-  ga.tab = tab[0];
-  ga.c = ab;
-  ga.ldc = 2 * I;
-  rc = launch_gemm_bwd<false, gbwd::EPI_BF16>("backward GEMM ab = X W_gu^T", X, XP, WGU, WGU, ga,
-                                              mt_rows * nt(2 * I), st);
-  if (rc != MOE_OK) return rc;
+  // G1: a | b pre-activations of every (row, expert), unless the forward kept them
+  if (!ab_saved) {
+    ga.tab = tab[0];
+    ga.c = ab;
+    ga.ldc = 2 * I;
+    rc = launch_gemm_bwd<false, gbwd::EPI_BF16>("backward GEMM ab = X W_gu^T", X, XP, WGU, WGU,
+                                                ga, mt_rows * nt(2 * I), st);
+    if (rc != MOE_OK) return rc;
+  }
   // G2: dz' = dY W_down with the SwiGLU backward in the epilogue
   ga.tab = tab[1];
   ga.c = nullptr;
   ga.ab = ab;
+  ga.ab_saved = static_cast<const __nv_bfloat16*>(ab_saved);
   ga.zg = zg;
   ga.dab = dab;
   ga.dgp = dgp;
@@ -1331,11 +1335,12 @@ moe_status moe_combine(const moe_layer_desc* desc, const void* x_residual, const
   return do_combine(D, x_residual, y_slots, h, stream);
 }
 
-moe_status moe_forward(const moe_layer_desc* desc, const void* x, const void* x_residual,
-                       const void* w_router, const float* bias, const void* w_gu,
-                       const float* w_gu_scale, const void* w_down, const float* w_down_scale,
-                       void* h, int32_t* topk_idx, int32_t* counts, void* ws, size_t ws_bytes,
-                       cudaStream_t stream) {
+static moe_status forward_entry(const moe_layer_desc* desc, const void* x,
+                                const void* x_residual, const void* w_router, const float* bias,
+                                const void* w_gu, const float* w_gu_scale, const void* w_down,
+                                const float* w_down_scale, void* h, int32_t* topk_idx,
+                                int32_t* counts, void* ab_save, void* ws, size_t ws_bytes,
+                                cudaStream_t stream) {
   Dims D;
   moe_status rc = fill_dims(desc, &D);
   if (rc != MOE_OK) return rc;
@@ -1372,11 +1377,41 @@ moe_status moe_forward(const moe_layer_desc* desc, const void* x, const void* x_
                        perm_src, slot_of, x_perm, x_perm_scale, stream, cnt)) != MOE_OK)
     return rc;
   if ((rc = do_grouped(D, L, x, x_perm, x_perm_scale, offsets, slot_of, tw, w_gu, w_gu_scale,
-                       w_down, w_down_scale, y, w8, sms, stream)) != MOE_OK)
+                       w_down, w_down_scale, y, w8, sms, stream,
+                       static_cast<__nv_bfloat16*>(ab_save))) != MOE_OK)
     return rc;
   rc = do_combine(D, x_residual ? x_residual : x, y, h, stream);
   if (rc == MOE_OK) rc = trace(5, stream);
   return rc;
+}
+
+moe_status moe_forward(const moe_layer_desc* desc, const void* x, const void* x_residual,
+                       const void* w_router, const float* bias, const void* w_gu,
+                       const float* w_gu_scale, const void* w_down, const float* w_down_scale,
+                       void* h, int32_t* topk_idx, int32_t* counts, void* ws, size_t ws_bytes,
+                       cudaStream_t stream) {
+  return forward_entry(desc, x, x_residual, w_router, bias, w_gu, w_gu_scale, w_down,
+                       w_down_scale, h, topk_idx, counts, nullptr, ws, ws_bytes, stream);
+}
+
+size_t moe_saved_ab_bytes(const moe_layer_desc* desc) {
+  Dims D;
+  if (fill_dims(desc, &D) != MOE_OK) return 0;
+  if (D.act != MOE_DT_BF16 || D.w != MOE_DT_BF16) return 0;
+  return (size_t)(D.R + D.Ks * D.T) * 2 * D.I * 2;
+}
+
+moe_status moe_forward_save(const moe_layer_desc* desc, const void* x, const void* x_residual,
+                            const void* w_router, const float* bias, const void* w_gu,
+                            const void* w_down, void* h, int32_t* topk_idx, int32_t* counts,
+                            void* ab_saved, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  Dims D;
+  moe_status rc = fill_dims(desc, &D);
+  if (rc != MOE_OK) return rc;
+  if (D.act != MOE_DT_BF16 || D.w != MOE_DT_BF16) return MOE_ERR_UNSUPPORTED;
+  if (D.T > 0 && (!ab_saved || !aligned16(ab_saved))) return MOE_ERR_INVALID_ARG;
+  return forward_entry(desc, x, x_residual, w_router, bias, w_gu, nullptr, w_down, nullptr, h,
+                       topk_idx, counts, ab_saved, ws, ws_bytes, stream);
 }
 
 moe_status moe_route_affinities(const moe_layer_desc* desc, const void* x, const void* w_router,
@@ -1545,8 +1580,9 @@ size_t moe_backward_workspace_size(const moe_layer_desc* desc) {
 static moe_status backward_entry(const moe_layer_desc* desc, const void* x,
                                  const void* w_router, const float* bias, const void* w_gu,
                                  const void* w_down, const void* dh, void* dx, void* dw_router,
-                                 void* dw_gu, void* dw_down, bool bf16_grads, void* ws,
-                                 size_t ws_bytes, cudaStream_t stream) {
+                                 void* dw_gu, void* dw_down, bool bf16_grads,
+                                 const void* ab_saved, void* ws, size_t ws_bytes,
+                                 cudaStream_t stream) {
   Dims D;
   moe_status rc = fill_dims(desc, &D);
   if (rc != MOE_OK) return rc;
@@ -1557,7 +1593,7 @@ static moe_status backward_entry(const moe_layer_desc* desc, const void* x,
     if (!x || !w_router || !w_gu || !w_down || !dh || !dx || !dw_router || !dw_gu || !dw_down ||
         !aligned16(x) || !aligned16(w_router) || !aligned16(w_gu) || !aligned16(w_down) ||
         !aligned16(dh) || !aligned16(dx) || !aligned16(dw_router) || !aligned16(dw_gu) ||
-        !aligned16(dw_down) || (bias && !aligned16(bias)))
+        !aligned16(dw_down) || (bias && !aligned16(bias)) || (ab_saved && !aligned16(ab_saved)))
       return MOE_ERR_INVALID_ARG;
     if ((D.N * 2) % 16) return MOE_ERR_UNSUPPORTED;   // rows of dl must be 16-byte aligned
   }
@@ -1569,7 +1605,7 @@ static moe_status backward_entry(const moe_layer_desc* desc, const void* x,
   int sms;
   if ((rc = device_setup(&sms)) != MOE_OK) return rc;
   return do_backward(*desc, D, L, B, x, w_router, bias, w_gu, w_down, dh, dx, dw_router, dw_gu,
-                     dw_down, bf16_grads, static_cast<uint8_t*>(ws), sms, stream);
+                     dw_down, bf16_grads, ab_saved, static_cast<uint8_t*>(ws), sms, stream);
 }
 
 moe_status moe_backward(const moe_layer_desc* desc, const void* x, const void* w_router,
@@ -1577,7 +1613,7 @@ moe_status moe_backward(const moe_layer_desc* desc, const void* x, const void* w
                         void* dx, float* dw_router, float* dw_gu, float* dw_down, void* ws,
                         size_t ws_bytes, cudaStream_t stream) {
   return backward_entry(desc, x, w_router, bias, w_gu, w_down, dh, dx, dw_router, dw_gu, dw_down,
-                        false, ws, ws_bytes, stream);
+                        false, nullptr, ws, ws_bytes, stream);
 }
 
 moe_status moe_backward_bf16_grads(const moe_layer_desc* desc, const void* x,
@@ -1586,7 +1622,20 @@ moe_status moe_backward_bf16_grads(const moe_layer_desc* desc, const void* x,
                                    void* dw_gu, void* dw_down, void* ws, size_t ws_bytes,
                                    cudaStream_t stream) {
   return backward_entry(desc, x, w_router, bias, w_gu, w_down, dh, dx, dw_router, dw_gu, dw_down,
-                        true, ws, ws_bytes, stream);
+                        true, nullptr, ws, ws_bytes, stream);
+}
+
+moe_status moe_backward_saved(const moe_layer_desc* desc, const void* x, const void* w_router,
+                              const float* bias, const void* w_gu, const void* w_down,
+                              const void* dh, const void* ab_saved, void* dx, void* dw_router,
+                              void* dw_gu, void* dw_down, int32_t bf16_grads, void* ws,
+                              size_t ws_bytes, cudaStream_t stream) {
+  Dims D;
+  moe_status rc = fill_dims(desc, &D);
+  if (rc != MOE_OK) return rc;
+  if (D.T > 0 && !ab_saved) return MOE_ERR_INVALID_ARG;
+  return backward_entry(desc, x, w_router, bias, w_gu, w_down, dh, dx, dw_router, dw_gu, dw_down,
+                        bf16_grads != 0, ab_saved, ws, ws_bytes, stream);
 }
 
 int32_t moe_backward_launch_count(const moe_layer_desc* desc) {

@@ -97,6 +97,9 @@ __global__ void __launch_bounds__(1024) k_bwd_prep(const PrepArgs a) {
     const int am = routed ? 1 : 0, am0 = routed ? p0 : 0;
     put(a.tab_ab + e * F, rows, 2 * I, d, am, am0, 0, 0, we * 2 * I, 0, p0, padded, aux);
     put(a.tab_dz + e * F, rows, I, d, am, am0, 0, 0, 0, we * d, p0, padded, aux);
+    // the problem's first row among the forward's H rows (routed expert j:
+    // offsets[j]; shared expert s: R + s T), where saved pre-activations live
+    a.tab_dz[e * F + gbwd::F_SPARE] = routed ? a.offsets[e] : a.offsets[a.N] + (e - a.N) * T;
     put(a.tab_du + e * F, rows, d, 2 * I, 0, p0, 0, 0, 0, we * 2 * I, p0, padded, aux);
     // weight gradients contract over the expert's rows (zero rows pad them to 64)
     put(a.tab_dwd + e * F, d, I, routed ? padded : T, am, 0, routed ? p0 : 0, 0, 0, p0, we * d,

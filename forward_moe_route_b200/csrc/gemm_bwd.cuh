@@ -79,6 +79,9 @@ struct Args {
   long long ldc;           // elements per output row
   // EPI_SWIGLU_BWD
   const __nv_bfloat16* ab; // [rows, 2I] pre-activations a | b
+  // pre-activations saved by the forward ([H rows, 2I], the forward's row
+  // order; problem p's rows start at its F_SPARE field), read instead of ab
+  const __nv_bfloat16* ab_saved;
   __nv_bfloat16* zg;       // [rows, I]  g * SiLU(a) * b
   __nv_bfloat16* dab;      // [rows, 2I] da | db
   float* dgp;              // [rows, I / 256] partial <dz', z>
@@ -356,7 +359,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         //   da = dz b SiLU'(a),  db = dz SiLU(a),  dg partial = sum dz' z.
         const int I = a.inter;
         const float gw = (p[F_AUX] < 0 && valid) ? a.row_w[crow] : 1.0f;
-        const __nv_bfloat16* abr = a.ab + crow * 2 * I + col0;
+        const __nv_bfloat16* abr =
+            (a.ab_saved ? a.ab_saved + ((long long)p[F_SPARE] + row) * 2 * I : a.ab + crow * 2 * I) +
+            col0;
         __nv_bfloat16* zr = a.zg + crow * I + col0;
         __nv_bfloat16* dar = a.dab + crow * 2 * I + col0;
         float dgs = 0.f;

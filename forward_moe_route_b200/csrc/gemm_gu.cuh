@@ -22,6 +22,10 @@
 // tempty, every wait bounded, a cluster barrier before TMEM is freed), plus
 // xfull (the up warps' values are in the exchange buffer) and xempty (the
 // gate warps have read them) once per tile.
+//
+// With Args::ab set the gate warps also write the rounded pre-activations
+// a = X W_gate^T and the up warps b = X W_up^T of every row, so that a
+// backward can skip recomputing them.
 #pragma once
 
 #include "common.cuh"
@@ -53,6 +57,9 @@ struct Args {
   uint32_t fmt;            // UMMA operand format: 1 bf16, 2 tf32
   int out_bf16;
   void* h;                 // [rows, I]
+  // optional [rows, 2I] bf16 copy of the pre-activations a | b (gate values
+  // in columns 0..I-1, up values in I..2I-1), kept for the backward
+  __nv_bfloat16* ab;
 };
 
 __host__ inline size_t smem_bytes(int stages, int n_groups) {
@@ -247,12 +254,25 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (up_warp) {
         // the gate warps have read the previous tile's values
         if (!mbar_wait(xempty, ((uint32_t)tcount & 1u) ^ 1u, abort_flag)) break;
+        // this warp's up features are those of gate quadrant q - 2
+        const int f_up = ft * 2 * FM + (int)rank * FM + (q & 1) * 32 + lane;
+        __nv_bfloat16* bsave =
+            a.ab != nullptr && f_up < a.inter
+                ? a.ab + ((size_t)a.gt.c_row(g) + tok0) * 2 * a.inter + a.inter + f_up
+                : nullptr;
 #pragma unroll 1
         for (int c = par; c < nch; c += 2) {
           float v[16];
           tmem_ld16(tb + (uint32_t)(16 * c), v);
 #pragma unroll
           for (int j = 0; j < 16; ++j) xq[(16 * c + j) * 32 + lane] = v[j];
+          if (bsave != nullptr) {
+            // b of 16 tokens; each store writes 32 consecutive features of a row
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+              if (16 * c + j < ntok)
+                bsave[(size_t)(16 * c + j) * 2 * a.inter] = __float2bfloat16_rn(v[j]);
+          }
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(xfull);
@@ -271,6 +291,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               reinterpret_cast<__nv_bfloat16*>(xb)[j * 32 + lane] = __float2bfloat16_rn(h);
             else
               reinterpret_cast<float*>(xb)[j * 32 + lane] = h;
+          }
+          if (a.ab != nullptr && f_warp + lane < a.inter) {
+            // a of 16 tokens (the up warps write b); lane = feature, so each
+            // store writes 32 consecutive features of a row
+            __nv_bfloat16* asave = a.ab + (hrow0 + 16 * c) * 2 * a.inter + f_warp + lane;
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+              if (16 * c + j < ntok) asave[(size_t)j * 2 * a.inter] = __float2bfloat16_rn(v[j]);
           }
           __syncwarp();
           if (bf) {

@@ -195,6 +195,25 @@ moe_status moe_forward(const moe_layer_desc* desc, const void* x, const void* x_
                        void* h, int32_t* topk_idx, int32_t* counts, void* ws, size_t ws_bytes,
                        cudaStream_t stream);
 
+/* moe_forward that also keeps the expert pre-activations a = W_gate u and
+ * b = W_up u of every active (token, expert) row, rounded to bf16, for
+ * moe_backward_saved.  §3.6 of "DeepSeek Technical Report: MoE Architecture"
+ * caches the activations the linear layers' backward needs (in FP8 there);
+ * here they are kept in the layer's bf16.  bf16 layers only
+ * (MOE_ERR_UNSUPPORTED otherwise).
+ *   ab_saved [T*K + Ks*T, 2I] bf16 out, moe_saved_ab_bytes(desc) bytes, 16-byte
+ *     aligned: row r holds a in columns 0..I-1 and b in I..2I-1.  Rows
+ *     0..T*K-1 are the routed pairs in the permuted order of moe_permute
+ *     (expert-major, token order inside an expert), then T rows per shared
+ *     expert in token order.  The caller owns it; it is only valid together
+ *     with the same desc, x, w_router, bias and w_gu.
+ * Everything else as moe_forward. */
+size_t moe_saved_ab_bytes(const moe_layer_desc* desc);
+moe_status moe_forward_save(const moe_layer_desc* desc, const void* x, const void* x_residual,
+                            const void* w_router, const float* bias, const void* w_gu,
+                            const void* w_down, void* h, int32_t* topk_idx, int32_t* counts,
+                            void* ab_saved, void* ws, size_t ws_bytes, cudaStream_t stream);
+
 /* ---- Load balancing (training-time statistics and the bias update) -------
  * "DeepSeek Technical Report: MoE Architecture", §1.2 (L_ExpBal = alpha_1
  * sum_i f_i P_i with f_i the fraction of tokens that chose expert i and P_i
@@ -397,6 +416,21 @@ moe_status moe_backward_bf16_grads(const moe_layer_desc* desc, const void* x,
                                    const void* w_down, const void* dh, void* dx, void* dw_router,
                                    void* dw_gu, void* dw_down, void* ws, size_t ws_bytes,
                                    cudaStream_t stream);
+
+/* The backward from the pre-activations moe_forward_save kept, instead of
+ * recomputing them: the gate/up GEMM of the recomputation (a quarter of the
+ * backward's tensor-core work) is skipped; routing and the permutation are
+ * still rebuilt from x, which yields the same rows because both are
+ * deterministic.  ab_saved as written by moe_forward_save with the same desc,
+ * x, w_router, bias and w_gu (not checked); bf16_grads nonzero: dw_router,
+ * dw_gu and dw_down bf16 as in moe_backward_bf16_grads, else fp32 as in
+ * moe_backward.  Launches moe_backward_launch_count(desc) - 1 kernels.
+ * Everything else, workspace included, as moe_backward. */
+moe_status moe_backward_saved(const moe_layer_desc* desc, const void* x, const void* w_router,
+                              const float* bias, const void* w_gu, const void* w_down,
+                              const void* dh, const void* ab_saved, void* dx, void* dw_router,
+                              void* dw_gu, void* dw_down, int32_t bf16_grads, void* ws,
+                              size_t ws_bytes, cudaStream_t stream);
 
 /* Number of kernels moe_backward launches for `desc` (0 if invalid or T = 0). */
 int32_t moe_backward_launch_count(const moe_layer_desc* desc);

@@ -220,3 +220,39 @@ def test_expert_parallel_entry_points_reject_bad_arguments():
                                 ctypes.byref(off)) == moe.ERR_INVALID_ARG
     assert L.moe_ipc_open(None, None) == moe.ERR_INVALID_ARG
     assert L.moe_ipc_close(None) == moe.ERR_INVALID_ARG
+
+
+def test_saved_activation_entry_points_reject_bad_arguments():
+    """moe_forward_save / moe_backward_saved: bf16 layers only, a 16-byte
+    aligned ab_saved of moe_saved_ab_bytes bytes, checked before any CUDA call."""
+    L = moe.lib()
+    bf = v3(T=64)
+    T, K, Ks, I = bf.T, bf.top_k, bf.n_shared, bf.inter
+    assert moe.moe_saved_ab_bytes(bf) == (T * K + Ks * T) * 2 * I * 2
+    assert moe.moe_saved_ab_bytes(v3(dtype="e4m3")) == 0
+    assert moe.moe_saved_ab_bytes(v3(dtype="f32")) == 0
+    assert moe.moe_saved_ab_bytes(v3(top_k=300)) == 0
+    fwd = (16, None, 16, None, 16, 16, 16, None, None)
+    # no or misaligned ab_saved; FP8 and fp32 layers refused
+    assert L.moe_forward_save(ctypes.byref(bf), *fwd, None, 16, 1 << 30,
+                              None) == moe.ERR_INVALID_ARG
+    assert L.moe_forward_save(ctypes.byref(bf), *fwd, 24, 16, 1 << 30,
+                              None) == moe.ERR_INVALID_ARG
+    assert L.moe_forward_save(ctypes.byref(v3(dtype="e4m3")), *fwd, 16, 16, 1 << 30,
+                              None) == moe.ERR_UNSUPPORTED
+    assert L.moe_forward_save(ctypes.byref(v3(dtype="f32")), *fwd, 16, 16, 1 << 30,
+                              None) == moe.ERR_UNSUPPORTED
+    bwd = (16, 16, None, 16, 16, 16)
+    grads = (16, 16, 16, 16)
+    assert L.moe_backward_saved(ctypes.byref(bf), *bwd, None, *grads, 0, 16, 1 << 40,
+                                None) == moe.ERR_INVALID_ARG
+    assert L.moe_backward_saved(ctypes.byref(bf), *bwd, 40, *grads, 0, 16, 1 << 40,
+                                None) == moe.ERR_INVALID_ARG
+    assert L.moe_backward_saved(ctypes.byref(v3(dtype="f32")), *bwd, 16, *grads, 0, 16,
+                                1 << 40, None) == moe.ERR_UNSUPPORTED
+    # the binding refuses a short ab_saved
+    import torch
+    x = torch.zeros(T, bf.d, dtype=torch.bfloat16)
+    short = torch.zeros(T * K, 2 * I, dtype=torch.bfloat16)     # the shared rows missing
+    with pytest.raises(moe.MoeError, match="ab_saved holds"):
+        moe.moe_forward_save(bf, x, None, None, None, None, None, x, None, None, short, None)

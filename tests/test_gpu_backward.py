@@ -58,7 +58,21 @@ def upstream(cfg):
     return dh.cuda(), dh.double().numpy()
 
 
-def run_backward(cfg, inp, dh):
+def forward_save(cfg, inp):
+    """moe_forward_save of the layer: (h, ab_saved, status)."""
+    desc = moe.desc_from_config(cfg)
+    ws = moe.workspace(desc)
+    h = torch.empty(cfg.T, cfg.d, dtype=torch.bfloat16, device="cuda")
+    ab = torch.full((cfg.T * (cfg.top_k + cfg.n_shared), 2 * cfg.inter), float("nan"),
+                    dtype=torch.bfloat16, device="cuda")
+    assert ab.numel() * 2 == moe.moe_saved_ab_bytes(desc)
+    moe.moe_forward_save(desc, inp["x"], None, inp["w_r"], inp["bias"], inp["w_gu"],
+                         inp["w_down"], h, None, None, ab, ws)
+    return h, ab, moe.moe_last_device_status()
+
+
+def run_backward(cfg, inp, dh, ab_saved=None):
+    """moe_backward, or moe_backward_saved when the forward's a | b are given."""
     desc = moe.desc_from_config(cfg)
     ws = moe.backward_workspace(desc)
     E, I, d, N = cfg.n_experts, cfg.inter, cfg.d, cfg.n_routed
@@ -66,19 +80,30 @@ def run_backward(cfg, inp, dh):
     dwr = torch.full((N, d), float("nan"), dtype=torch.float32, device="cuda")
     dwgu = torch.full((E, 2 * I, d), float("nan"), dtype=torch.float32, device="cuda")
     dwd = torch.full((E, d, I), float("nan"), dtype=torch.float32, device="cuda")
-    moe.moe_backward(desc, inp["x"], inp["w_r"], inp["bias"], inp["w_gu"], inp["w_down"], dh, dx,
-                     dwr, dwgu, dwd, ws)
+    if ab_saved is None:
+        moe.moe_backward(desc, inp["x"], inp["w_r"], inp["bias"], inp["w_gu"], inp["w_down"], dh,
+                         dx, dwr, dwgu, dwd, ws)
+    else:
+        moe.moe_backward_saved(desc, inp["x"], inp["w_r"], inp["bias"], inp["w_gu"],
+                               inp["w_down"], dh, ab_saved, dx, dwr, dwgu, dwd, ws)
     st = moe.moe_last_device_status()
     return dx, dwr, dwgu, dwd, st
 
 
+@pytest.mark.parametrize("saved", [False, True], ids=["recompute", "saved"])
 @pytest.mark.parametrize("name", list(CASES))
-def test_backward_parity(name):
+def test_backward_parity(name, saved):
+    """Both backward forms against the oracle: recomputing a | b from x, and
+    reading the a | b that moe_forward_save kept."""
     cfg = CASES[name]
     moe.moe_last_device_status()
     inp = recipes.device_inputs(cfg)
     dh, dh64 = upstream(cfg)
-    dx, dwr, dwgu, dwd, st = run_backward(cfg, inp, dh)
+    ab = None
+    if saved:
+        _, ab, st = forward_save(cfg, inp)
+        assert st == moe.OK, moe.moe_status_string(st)
+    dx, dwr, dwgu, dwd, st = run_backward(cfg, inp, dh, ab)
     assert st == moe.OK, moe.moe_status_string(st)
     # the selection the backward used: the forward's routing of the same inputs
     desc = moe.desc_from_config(cfg)
@@ -162,3 +187,91 @@ def test_backward_bf16_weight_gradients(name):
     assert torch.equal(dx2, dx)
     for got, ref in ((dwr2, dwr), (dwgu2, dwgu), (dwd2, dwd)):
         assert torch.equal(got, ref.to(torch.bfloat16))
+
+
+@pytest.mark.parametrize("name", ["v3_small", "dsmoe16b_small", "v3_T1"])
+def test_forward_save(name):
+    """moe_forward_save: h is moe_forward's bit for bit, and ab_saved holds the
+    pre-activations a = u W_gate^T, b = u W_up^T of every routed pair in the
+    permuted row order (moe_permute's slot_of), then every shared expert's T
+    rows, within bf16 rounding of the fp64 oracle."""
+    cfg = CASES[name]
+    moe.moe_last_device_status()
+    inp = recipes.device_inputs(cfg)
+    h_save, ab, st = forward_save(cfg, inp)
+    assert st == moe.OK, moe.moe_status_string(st)
+    desc = moe.desc_from_config(cfg)
+    ws = moe.workspace(desc)
+    h = torch.empty_like(h_save)
+    moe.moe_forward(desc, inp["x"], None, inp["w_r"], inp["bias"], inp["w_gu"], None,
+                    inp["w_down"], None, h, None, None, ws)
+    assert moe.moe_last_device_status() == moe.OK
+    assert torch.equal(h, h_save)
+    # the row order: the permutation of the GPU's own routing
+    T, K, Ks, I = cfg.T, cfg.top_k, cfg.n_shared, cfg.inter
+    idx = torch.empty(T, K, dtype=torch.int32, device="cuda")
+    w = torch.empty(T, K, dtype=torch.float32, device="cuda")
+    counts = torch.empty(cfg.n_routed, dtype=torch.int32, device="cuda")
+    moe.moe_route(desc, inp["x"], inp["w_r"], inp["bias"], idx, w, counts, ws)
+    offsets = torch.empty(cfg.n_routed + 1, dtype=torch.int32, device="cuda")
+    perm_src = torch.empty(T * K, dtype=torch.int32, device="cuda")
+    slot_of = torch.empty(T * K, dtype=torch.int32, device="cuda")
+    x_perm = torch.empty(T * K, cfg.d, dtype=torch.bfloat16, device="cuda")
+    moe.moe_permute(desc, inp["x"], idx, counts, offsets, perm_src, slot_of, x_perm, None, ws)
+    assert moe.moe_last_device_status() == moe.OK
+    host = HostLayer(cfg)
+    g_idx = idx.cpu().numpy().astype(np.int64)
+    slots = slot_of.cpu().numpy().astype(np.int64)
+    got = f64(ab)
+    assert not np.isnan(got).any()
+    num = den = 0.0
+    flat = g_idx.reshape(-1)
+    for j in np.unique(flat):
+        pairs = np.nonzero(flat == j)[0]
+        wg, wu, _ = host.expert(Ks + int(j))
+        xt = host.x[pairs // K]
+        want = np.concatenate([xt @ wg.T, xt @ wu.T], axis=1)
+        num = max(num, float(np.max(np.abs(got[slots[pairs]] - want))))
+        den = max(den, float(np.max(np.abs(want))))
+    for s_ in range(Ks):
+        wg, wu, _ = host.expert(s_)
+        want = np.concatenate([host.x @ wg.T, host.x @ wu.T], axis=1)
+        rows = got[T * K + s_ * T: T * K + (s_ + 1) * T]
+        num = max(num, float(np.max(np.abs(rows - want))))
+        den = max(den, float(np.max(np.abs(want))))
+    assert num / den <= 1e-2, f"saved a | b: max-abs-rel {num / den:.3e}"
+
+
+@pytest.mark.parametrize("name", ["v3_small", "v3_T1"])
+def test_backward_saved_matches_recompute(name):
+    """moe_backward_saved against moe_backward on the same inputs: both read
+    bf16 pre-activations of the same products (kept by the forward or
+    recomputed), so the gradients agree to bf16 rounding; the bf16-gradient
+    form of the saved call rounds the same accumulators."""
+    cfg = CASES[name]
+    moe.moe_last_device_status()
+    inp = recipes.device_inputs(cfg)
+    dh, _ = upstream(cfg)
+    _, ab, st = forward_save(cfg, inp)
+    assert st == moe.OK
+    ref = run_backward(cfg, inp, dh)
+    got = run_backward(cfg, inp, dh, ab)
+    assert ref[4] == moe.OK and got[4] == moe.OK
+    for a, b in zip(got[:4], ref[:4]):
+        a64, b64 = f64(a), f64(b)
+        den = max(float(np.max(np.abs(b64))), 1e-30)
+        assert float(np.max(np.abs(a64 - b64))) / den <= 1e-2
+    desc = moe.desc_from_config(cfg)
+    ws = moe.backward_workspace(desc)
+    E, I, d, N = cfg.n_experts, cfg.inter, cfg.d, cfg.n_routed
+    bf = dict(dtype=torch.bfloat16, device="cuda")
+    dx2 = torch.full((cfg.T, d), float("nan"), **bf)
+    dwr2 = torch.full((N, d), float("nan"), **bf)
+    dwgu2 = torch.full((E, 2 * I, d), float("nan"), **bf)
+    dwd2 = torch.full((E, d, I), float("nan"), **bf)
+    moe.moe_backward_saved(desc, inp["x"], inp["w_r"], inp["bias"], inp["w_gu"], inp["w_down"],
+                           dh, ab, dx2, dwr2, dwgu2, dwd2, ws, bf16_grads=True)
+    assert moe.moe_last_device_status() == moe.OK
+    assert torch.equal(dx2, got[0])
+    for a, b in ((dwr2, got[1]), (dwgu2, got[2]), (dwd2, got[3])):
+        assert torch.equal(a, b.to(torch.bfloat16))

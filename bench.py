@@ -581,10 +581,12 @@ def run_backward(args, cfg):
                 moe.moe_forward(desc, inp["x"], None, inp["w_r"], inp["bias"], inp["w_gu"], None,
                                 inp["w_down"], None, h, None, None, fws, stream)
 
-        fwd_cost = {}
-        for save in (False, True, False, True):
-            for _ in range(3):
-                fwd(save)
+        # blocks of 5 forwards in the order A B B A A B B A after a warm-up,
+        # so that neither form gets the cooler GPU; medians of the blocks
+        for _ in range(6):
+            fwd(False)
+        blocks = {False: [], True: []}
+        for save in (False, True, True, False, False, True, True, False):
             f0 = torch.cuda.Event(enable_timing=True)
             f1 = torch.cuda.Event(enable_timing=True)
             f0.record(stream)
@@ -592,8 +594,10 @@ def run_backward(args, cfg):
                 fwd(save)
             f1.record(stream)
             torch.cuda.synchronize()
-            key = "forward_save_ms" if save else "forward_ms"
-            fwd_cost[key] = min(fwd_cost.get(key, 1e30), f0.elapsed_time(f1) / 5)
+            blocks[save].append(f0.elapsed_time(f1) / 5)
+        fwd_cost = {"forward_ms": statistics.median(blocks[False]),
+                    "forward_save_ms": statistics.median(blocks[True]),
+                    "blocks": "median of 4 blocks of 5 steps each, order ABBAABBA"}
         del fws
 
         def step():

@@ -106,6 +106,9 @@ _SIGS = {
                                           _P, ctypes.c_size_t, _P]),
     "moe_ipc_open": (ctypes.c_int, [_P, ctypes.POINTER(ctypes.c_void_p)]),
     "moe_ipc_close": (ctypes.c_int, [_P]),
+    "moe_backward_fp8_workspace_size": (ctypes.c_size_t, [_D]),
+    "moe_backward_fp8": (ctypes.c_int, [_D] + [_P] * 17 + [ctypes.c_size_t, _P]),
+    "moe_backward_fp8_launch_count": (ctypes.c_int32, [_D]),
     "moe_saved_ab_bytes": (ctypes.c_size_t, [_D]),
     "moe_forward_save": (ctypes.c_int, [_D, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                                         ctypes.c_size_t, _P]),
@@ -169,6 +172,9 @@ def _sizes(desc) -> dict:
         "y_slots": T * (K + Ks) * d * a, "s_out": T * N * 4,
         "dh": T * d * a, "dx": T * d * a, "dw_router": N * d * 4, "dw_gu": E * 2 * I * d * 4,
         "dw_down": E * d * I * 4, "ab_saved": (R + Ks * T) * 2 * I * 2,
+        "w_gu_t": E * d * 2 * I * w, "w_down_t": E * I * d * w,
+        "w_gu_t_scale": E * (d // 128) * (2 * I // 128) * 4 if fp8 else 0,
+        "w_down_t_scale": E * (I // 128) * (d // 128) * 4 if fp8 else 0,
     }
 
 
@@ -407,6 +413,47 @@ def moe_backward_saved(desc, x, w_router, bias, w_gu, w_down, dh, ab_saved, dx, 
                                    1 if bf16_grads else 0, _ptr(ws),
                                    ws.numel() if ws is not None else 0, _stream(stream)),
            "moe_backward_saved")
+
+
+def moe_backward_fp8_workspace_size(desc: MoeLayerDesc) -> int:
+    return int(_lib.moe_backward_fp8_workspace_size(ctypes.byref(desc)))
+
+
+def backward_fp8_workspace(desc: MoeLayerDesc, device="cuda"):
+    """A uint8 CUDA tensor of moe_backward_fp8_workspace_size(desc) bytes."""
+    import torch
+    n = moe_backward_fp8_workspace_size(desc)
+    if n == 0:
+        raise MoeError(ERR_UNSUPPORTED, "moe_backward_fp8_workspace_size")
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def moe_backward_fp8(desc, x, w_router, bias, w_gu, w_gu_scale, w_gu_t, w_gu_t_scale, w_down,
+                     w_down_scale, w_down_t, w_down_t_scale, dh, dx, dw_router, dw_gu, dw_down,
+                     ws, stream=None) -> None:
+    """The backward of an E4M3 layer with FP8 GEMMs; bf16 weight gradients."""
+    _need("moe_backward_fp8", desc, x=x, w_router=w_router, bias=bias, w_gu=w_gu,
+          w_gu_scale=w_gu_scale, w_gu_t=w_gu_t, w_gu_t_scale=w_gu_t_scale, w_down=w_down,
+          w_down_scale=w_down_scale, w_down_t=w_down_t, w_down_t_scale=w_down_t_scale, dh=dh,
+          dx=dx)
+    sz = _sizes(desc)
+    for name, t in (("dw_router", dw_router), ("dw_gu", dw_gu), ("dw_down", dw_down)):
+        if t is None:
+            continue
+        if not t.is_contiguous() or t.element_size() != 2 or t.numel() * 4 < sz[name]:
+            raise MoeError(ERR_INVALID_ARG, f"moe_backward_fp8: {name} must be a contiguous "
+                           "bf16 tensor of the gradient's shape")
+    _check(_lib.moe_backward_fp8(ctypes.byref(desc), _ptr(x), _ptr(w_router), _ptr(bias),
+                                 _ptr(w_gu), _ptr(w_gu_scale), _ptr(w_gu_t), _ptr(w_gu_t_scale),
+                                 _ptr(w_down), _ptr(w_down_scale), _ptr(w_down_t),
+                                 _ptr(w_down_t_scale), _ptr(dh), _ptr(dx), _ptr(dw_router),
+                                 _ptr(dw_gu), _ptr(dw_down), _ptr(ws),
+                                 ws.numel() if ws is not None else 0, _stream(stream)),
+           "moe_backward_fp8")
+
+
+def moe_backward_fp8_launch_count(desc) -> int:
+    return int(_lib.moe_backward_fp8_launch_count(ctypes.byref(desc)))
 
 
 def moe_backward_launch_count(desc) -> int:

@@ -18,6 +18,7 @@
 #include "permute.cuh"
 #include "route.cuh"
 #include "bwd.cuh"
+#include "bwd8.cuh"
 #include "gemm_bwd.cuh"
 
 using namespace moe;
@@ -167,16 +168,31 @@ moe_status device_setup(int* sms) {
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(gemm8::k_gemm_promoted<2, gemm8::EPI_SCATTER>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(gemm8::k_gemm_promoted<2, gemm8::EPI_BF16_OUT>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(gemm8::k_gemm_promoted<2, gemm8::EPI_SWIGLU_BWD>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(gemm8::k_gemm_promoted<2, gemm8::EPI_BF16_OUT, true>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute (dynamic shared memory)");
     // the promoted GEMMs re-split their registers with setmaxnreg; the split
     // adds up only if a thread starts with exactly LAUNCH_REGS registers
     {
-      cudaFuncAttributes fa[3];
+      cudaFuncAttributes fa[6];
       if (cudaFuncGetAttributes(&fa[0], gemm8::k_gemm_promoted<0, gemm8::EPI_F32_STORE>) !=
               cudaSuccess ||
           cudaFuncGetAttributes(&fa[1], gemm8::k_gemm_promoted<2, gemm8::EPI_SWIGLU_Q>) !=
               cudaSuccess ||
           cudaFuncGetAttributes(&fa[2], gemm8::k_gemm_promoted<2, gemm8::EPI_SCATTER>) !=
+              cudaSuccess ||
+          cudaFuncGetAttributes(&fa[3], gemm8::k_gemm_promoted<2, gemm8::EPI_BF16_OUT>) !=
+              cudaSuccess ||
+          cudaFuncGetAttributes(&fa[4], gemm8::k_gemm_promoted<2, gemm8::EPI_SWIGLU_BWD>) !=
+              cudaSuccess ||
+          cudaFuncGetAttributes(&fa[5], gemm8::k_gemm_promoted<2, gemm8::EPI_BF16_OUT, true>) !=
               cudaSuccess)
         return MOE_ERR_CUDA;
       for (const auto& f : fa)
@@ -1186,6 +1202,330 @@ moe_status do_backward(const moe_layer_desc& s, const Dims& D, const Layout& L,
                               (uint64_t)N, 1, ((N + 255) / 256) * nt(d), bf16_grads, st);
 }
 
+// ----------------------------------------------------------------------------- FP8 backward
+// Workspace of moe_backward_fp8: the forward's routing buffers, then the
+// 128-padded row space (routed segments, then one per shared expert) and the
+// FP8 operands of the backward GEMMs.
+struct Bwd8Layout {
+  int64_t rs;            // rows of the row space (a bound; a multiple of 128)
+  size_t poff, gtab, gtab_wd, gtab_wgu, kgroup, tabs, row_pair, row_w, row_tok;
+  size_t xq, xs, dhq, dhs, ab, zg, dab, dgp, dabq, dabs, dl, dxr, dslots;
+  size_t dhT, dhTs, zgT, zgTs, dabT, dabTs, xT, xTs, total;
+};
+
+Bwd8Layout bwd8_layout(const Dims& D, const Layout& L) {
+  Bwd8Layout B;
+  size_t o = align_up(L.gtab + (size_t)gemm::group_tab_ints((int)D.E) * 4, kAlign);
+  auto take = [&](size_t bytes) { size_t at = o; o = align_up(o + bytes, kAlign); return at; };
+  const int64_t rs = (D.R + 127 * D.N + 127) / 128 * 128 + D.Ks * (int64_t)bwd8::pad128((int)D.T);
+  const size_t d = D.d, I = D.I, R = (size_t)rs, E = D.E;
+  B.rs = rs;
+  B.poff = take((E + 1) * 4);
+  B.gtab = take((size_t)gemm::group_tab_ints((int)E) * 4);
+  B.gtab_wd = take((size_t)gemm::group_tab_ints((int)E) * 4);
+  B.gtab_wgu = take((size_t)gemm::group_tab_ints((int)E) * 4);
+  B.kgroup = take(2 * E * 4);
+  B.tabs = take(2 * gbwd::GB_FIELDS * 4);
+  B.row_pair = take(R * 4);
+  B.row_w = take(R * 4);
+  B.row_tok = take(R * 4);
+  B.xq = take(R * d);
+  B.xs = take(R * (d / 128) * 4);
+  B.dhq = take(R * d);
+  B.dhs = take(R * (d / 128) * 4);
+  B.ab = take(R * 2 * I * 2);
+  B.zg = take(R * I * 2);
+  B.dab = take(R * 2 * I * 2);
+  B.dgp = take(R * (I / 64) * 4);
+  B.dabq = take(R * 2 * I);
+  B.dabs = take(R * (2 * I / 128) * 4);
+  B.dl = take((size_t)D.T * D.N * 2);
+  B.dxr = take((size_t)D.T * d * 2);
+  B.dslots = take((size_t)D.T * (D.K + D.Ks) * d * 2);
+  B.dhT = take(d * R);
+  B.dhTs = take((R / 128) * d * 4);
+  B.zgT = take(I * R);
+  B.zgTs = take((R / 128) * I * 4);
+  B.dabT = take(2 * I * R);
+  B.dabTs = take((R / 128) * 2 * I * 4);
+  B.xT = take(d * R);
+  B.xTs = take((R / 128) * d * 4);
+  B.total = o;
+  return B;
+}
+
+struct Fp8Weights {
+  const void *gu, *gu_t, *down, *down_t;
+  const float *gu_s, *gu_t_s, *down_s, *down_t_s;
+};
+
+moe_status do_backward_fp8(const moe_layer_desc& s, const Dims& D, const Layout& L,
+                           const Bwd8Layout& B, const void* x, const void* w_router,
+                           const float* bias, const Fp8Weights& W, const void* dh, void* dx,
+                           void* dw_router, void* dw_gu, void* dw_down, uint8_t* ws, int sms,
+                           cudaStream_t st) {
+  const int T = (int)D.T, d = (int)D.d, I = (int)D.I, N = (int)D.N, K = (int)D.K;
+  const int Ks = (int)D.Ks, E = (int)D.E;
+  const int rs = (int)B.rs;
+  int32_t* idx = reinterpret_cast<int32_t*>(ws + L.topk_idx);
+  float* tw = reinterpret_cast<float*>(ws + L.topk_w);
+  int32_t* counts = reinterpret_cast<int32_t*>(ws + L.counts);
+  int32_t* hist = reinterpret_cast<int32_t*>(ws + L.hist);
+  int32_t* offsets = reinterpret_cast<int32_t*>(ws + L.offsets);
+  int32_t* perm_src = reinterpret_cast<int32_t*>(ws + L.perm_src);
+  int32_t* slot_of = reinterpret_cast<int32_t*>(ws + L.slot_of);
+  const float* logits = reinterpret_cast<const float*>(ws + L.logits);
+  int32_t* poff = reinterpret_cast<int32_t*>(ws + B.poff);
+  int32_t* gtab = reinterpret_cast<int32_t*>(ws + B.gtab);
+  int32_t* gtab_wd = reinterpret_cast<int32_t*>(ws + B.gtab_wd);
+  int32_t* gtab_wgu = reinterpret_cast<int32_t*>(ws + B.gtab_wgu);
+  int32_t* kgroup = reinterpret_cast<int32_t*>(ws + B.kgroup);
+  int32_t* tab_dxr = reinterpret_cast<int32_t*>(ws + B.tabs);
+  int32_t* tab_dwr = tab_dxr + gbwd::GB_FIELDS;
+  int32_t* row_pair = reinterpret_cast<int32_t*>(ws + B.row_pair);
+  float* row_w = reinterpret_cast<float*>(ws + B.row_w);
+  int32_t* row_tok = reinterpret_cast<int32_t*>(ws + B.row_tok);
+  uint8_t* xq = ws + B.xq;
+  float* xs = reinterpret_cast<float*>(ws + B.xs);
+  uint8_t* dhq = ws + B.dhq;
+  float* dhs = reinterpret_cast<float*>(ws + B.dhs);
+  auto* ab = reinterpret_cast<__nv_bfloat16*>(ws + B.ab);
+  auto* zg = reinterpret_cast<__nv_bfloat16*>(ws + B.zg);
+  auto* dab = reinterpret_cast<__nv_bfloat16*>(ws + B.dab);
+  float* dgp = reinterpret_cast<float*>(ws + B.dgp);
+  uint8_t* dabq = ws + B.dabq;
+  float* dabs = reinterpret_cast<float*>(ws + B.dabs);
+  auto* dl = reinterpret_cast<__nv_bfloat16*>(ws + B.dl);
+  auto* dxr = reinterpret_cast<__nv_bfloat16*>(ws + B.dxr);
+  auto* dslots = reinterpret_cast<__nv_bfloat16*>(ws + B.dslots);
+
+  // routing and the permutation maps, as in the forward
+  moe_status rc = do_route(s, D, L, x, w_router, bias, idx, tw, nullptr, ws, sms, st);
+  if (rc != MOE_OK) return rc;
+  rc = launch_chain("k_hist", perm::k_hist, dim3(D.n_chunks), dim3(256), N * 4, st,
+                    static_cast<const int32_t*>(idx), T, K, N, hist);
+  if (rc == MOE_OK)
+    rc = launch_scan(st, hist, (int)D.n_chunks, N, static_cast<const int32_t*>(nullptr), counts,
+                     offsets);
+  if (rc == MOE_OK)
+    rc = launch_chain("k_slots", perm::k_slots, dim3(D.n_chunks), dim3(perm::SLOT_WARPS * 32),
+                      perm::SLOT_WARPS * N * 4, st, static_cast<const int32_t*>(idx), T, K, N,
+                      static_cast<const int32_t*>(hist), slot_of, perm_src);
+  if (rc != MOE_OK) return rc;
+  bwd8::PrepArgs pa;
+  pa.offsets = offsets;
+  pa.T = T; pa.d = d; pa.I = I; pa.Ks = Ks; pa.N = N;
+  pa.poff = poff; pa.gtab = gtab; pa.gtab_wd = gtab_wd; pa.gtab_wgu = gtab_wgu;
+  pa.kgroup = kgroup; pa.tab_dxr = tab_dxr; pa.tab_dwr = tab_dwr;
+  rc = launch_chain("k_bwd8_prep", bwd8::k_bwd8_prep, dim3(1), dim3(1024), 0, st, pa);
+  if (rc == MOE_OK)
+    rc = launch_chain("k_bwd8_gather", bwd8::k_bwd8_gather, dim3((T + 7) / 8), dim3(256), 0, st,
+                      static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(dh),
+                      T, K, Ks, N, d, static_cast<const int32_t*>(idx),
+                      static_cast<const float*>(tw), static_cast<const int32_t*>(slot_of),
+                      static_cast<const int32_t*>(offsets), static_cast<const int32_t*>(poff), xq,
+                      xs, dhq, dhs, row_pair, row_w, row_tok);
+  if (rc == MOE_OK)
+    rc = launch_chain("k_bwd8_pads", bwd8::k_bwd8_pads, dim3(E + 1), dim3(128), 0, st,
+                      static_cast<const int32_t*>(offsets), N, T, rs,
+                      static_cast<const int32_t*>(poff), row_pair, row_w, row_tok);
+  if (rc != MOE_OK) return rc;
+
+  int stages = 0;
+  for (int sg = 6; sg >= 2 && !stages; --sg)
+    if (gemm8::smem_bytes(sg, E) <= (size_t)kMaxSmem) stages = sg;
+  if (!stages) return MOE_ERR_UNSUPPORTED;
+  const size_t smem = gemm8::smem_bytes(stages, E);
+  const int64_t mt_rows = rs / 128;                  // m-tiles of the row space (a bound)
+  auto grid_of = [&](int64_t tiles) { return (int)(tiles < sms ? tiles : sms); };
+  auto base_args = [&](const int32_t* gt, int n_tiles_n, int num_kb, int b_rows_per_expert) {
+    gemm8::Args a;
+    memset(&a, 0, sizeof(a));
+    a.gt.base = gt;
+    a.gt.n = E;
+    a.n_tiles_n = n_tiles_n;
+    a.num_kb = num_kb;
+    a.kb_elems = 128;
+    a.b_rows_per_expert = b_rows_per_expert;
+    a.stages = stages;
+    a.idesc = umma_idesc(0, gemm8::BM, gemm8::BN);
+    a.K = K;
+    a.Ks = Ks;
+    a.inter = I;
+    return a;
+  };
+  // G1: a | b = X W_gu^T, X rows in FP8
+  {
+    CUtensorMap ta, tb;
+    rc = make_tmap(&ta, xq, 1, d, rs, gemm8::BM);
+    if (rc == MOE_OK) rc = make_tmap(&tb, W.gu, 1, d, (uint64_t)E * 2 * I, gemm8::BN);
+    if (rc != MOE_OK) return rc;
+    gemm8::Args a = base_args(gtab, 2 * I / gemm8::BN, d / 128, 2 * I);
+    a.a_scale = xs;
+    a.a_rows = rs;
+    a.b_scale = W.gu_s;
+    a.out_bf16 = ab;
+    a.out_ld = 2 * I;
+    a.out_cols = 2 * I;
+    rc = launch_chain("FP8 backward GEMM ab = X W_gu^T",
+                      gemm8::k_gemm_promoted<2, gemm8::EPI_BF16_OUT>,
+                      dim3(grid_of(mt_rows * a.n_tiles_n)), dim3(gemm8::NUM_THREADS), smem, st,
+                      ta, tb, a);
+    if (rc != MOE_OK) return rc;
+  }
+  // G2: dz' = dY W_down with the SwiGLU backward in the epilogue (W_down^T rows)
+  {
+    CUtensorMap ta, tb;
+    rc = make_tmap(&ta, dhq, 1, d, rs, gemm8::BM);
+    if (rc == MOE_OK) rc = make_tmap(&tb, W.down_t, 1, d, (uint64_t)E * I, gemm8::BN);
+    if (rc != MOE_OK) return rc;
+    gemm8::Args a = base_args(gtab, (I + gemm8::BN - 1) / gemm8::BN, d / 128, I);
+    a.a_scale = dhs;
+    a.a_rows = rs;
+    a.b_scale = W.down_t_s;
+    a.ab = ab;
+    a.zg = zg;
+    a.dab = dab;
+    a.dgp = dgp;
+    a.row_w = row_w;
+    rc = launch_chain("FP8 backward GEMM dz = dY W_down",
+                      gemm8::k_gemm_promoted<2, gemm8::EPI_SWIGLU_BWD>,
+                      dim3(grid_of(mt_rows * a.n_tiles_n)), dim3(gemm8::NUM_THREADS), smem, st,
+                      ta, tb, a);
+    if (rc != MOE_OK) return rc;
+  }
+  // [da | db] rows to FP8
+  rc = launch_chain("k_quant_rows", perm::k_quant_rows, dim3((rs + 7) / 8), dim3(256), 0, st,
+                    static_cast<const __nv_bfloat16*>(dab), rs, 2 * I, dabq, dabs);
+  if (rc != MOE_OK) return rc;
+  // G3: du pieces = dAB W_gu (W_gu^T rows), scattered to the token-major slots
+  {
+    CUtensorMap ta, tb;
+    rc = make_tmap(&ta, dabq, 1, 2 * I, rs, gemm8::BM);
+    if (rc == MOE_OK) rc = make_tmap(&tb, W.gu_t, 1, 2 * I, (uint64_t)E * d, gemm8::BN);
+    if (rc != MOE_OK) return rc;
+    gemm8::Args a = base_args(gtab, d / gemm8::BN, 2 * I / 128, d);
+    a.a_scale = dabs;
+    a.a_rows = rs;
+    a.b_scale = W.gu_t_s;
+    a.y = dslots;
+    a.d = d;
+    a.pair_of = row_pair;
+    a.topk_w = nullptr;
+    rc = launch_chain("FP8 backward GEMM du = dAB W_gu",
+                      gemm8::k_gemm_promoted<2, gemm8::EPI_SCATTER>,
+                      dim3(grid_of(mt_rows * a.n_tiles_n)), dim3(gemm8::NUM_THREADS), smem, st,
+                      ta, tb, a);
+    if (rc != MOE_OK) return rc;
+  }
+  // gate-weight and affinity backward -> dl [T, N]
+  {
+    const route::Params p = route_params(s);
+    const int n_it = I / 64;
+    if (N <= 32) rc = launch_gate_bwd<1>(logits, p, idx, slot_of, offsets, poff, dgp, n_it, dl, st);
+    else if (N <= 64) rc = launch_gate_bwd<2>(logits, p, idx, slot_of, offsets, poff, dgp, n_it, dl, st);
+    else if (N <= 128) rc = launch_gate_bwd<4>(logits, p, idx, slot_of, offsets, poff, dgp, n_it, dl, st);
+    else if (N <= 256) rc = launch_gate_bwd<8>(logits, p, idx, slot_of, offsets, poff, dgp, n_it, dl, st);
+    else rc = launch_gate_bwd<16>(logits, p, idx, slot_of, offsets, poff, dgp, n_it, dl, st);
+    if (rc != MOE_OK) return rc;
+  }
+  // the router's part of dx in bf16 (gating stays BF16), then dx
+  auto nt = [](int64_t n) { return (n + gbwd::BN - 1) / gbwd::BN; };
+  const Operand X{x, (uint64_t)d, (uint64_t)T};
+  const Operand DL{dl, (uint64_t)N, (uint64_t)T}, WR{w_router, (uint64_t)d, (uint64_t)N};
+  gbwd::Args ga;
+  memset(&ga, 0, sizeof(ga));
+  ga.n_probs = 1;
+  ga.K = K;
+  ga.Ks = Ks;
+  ga.inter = I;
+  ga.tab = tab_dxr;
+  ga.c = dxr;
+  ga.ldc = d;
+  rc = launch_gemm_bwd<true, gbwd::EPI_BF16>("backward GEMM dx_router = dL W_r", DL, DL, WR, WR,
+                                             ga, nt(d) * ((T + 127) / 128), st);
+  if (rc != MOE_OK) return rc;
+  rc = do_combine(D, dxr, dslots, dx, st);
+  if (rc != MOE_OK) return rc;
+  // weight-gradient operands: 128-row x 1-column tiles, transposed
+  {
+    const dim3 blk(256);
+    rc = launch_chain("k_quant_cols dY", bwd8::k_quant_cols<true>, dim3(rs / 128, d / 64), blk, 0,
+                      st, static_cast<const __nv_bfloat16*>(dh),
+                      static_cast<const int32_t*>(row_tok), d, rs, ws + B.dhT,
+                      reinterpret_cast<float*>(ws + B.dhTs));
+    if (rc == MOE_OK)
+      rc = launch_chain("k_quant_cols gz", bwd8::k_quant_cols<false>, dim3(rs / 128, I / 64), blk,
+                        0, st, static_cast<const __nv_bfloat16*>(zg),
+                        static_cast<const int32_t*>(nullptr), I, rs, ws + B.zgT,
+                        reinterpret_cast<float*>(ws + B.zgTs));
+    if (rc == MOE_OK)
+      rc = launch_chain("k_quant_cols dAB", bwd8::k_quant_cols<false>,
+                        dim3(rs / 128, 2 * I / 64), blk, 0, st,
+                        static_cast<const __nv_bfloat16*>(dab),
+                        static_cast<const int32_t*>(nullptr), 2 * I, rs, ws + B.dabT,
+                        reinterpret_cast<float*>(ws + B.dabTs));
+    if (rc == MOE_OK)
+      rc = launch_chain("k_quant_cols X", bwd8::k_quant_cols<true>, dim3(rs / 128, d / 64), blk, 0,
+                        st, static_cast<const __nv_bfloat16*>(x),
+                        static_cast<const int32_t*>(row_tok), d, rs, ws + B.xT,
+                        reinterpret_cast<float*>(ws + B.xTs));
+    if (rc != MOE_OK) return rc;
+  }
+  // G4: dW_down = dY^T (g z) and G5: dW_gu = dAB^T X over each expert's rows,
+  // bf16 out
+  {
+    CUtensorMap ta, tb;
+    rc = make_tmap(&ta, ws + B.dhT, 1, rs, d, gemm8::BM);
+    if (rc == MOE_OK) rc = make_tmap(&tb, ws + B.zgT, 1, rs, I, gemm8::BN);
+    if (rc != MOE_OK) return rc;
+    gemm8::Args a = base_args(gtab_wd, (I + gemm8::BN - 1) / gemm8::BN, 0, 0);
+    a.kgroup = kgroup;
+    a.a_scale = reinterpret_cast<const float*>(ws + B.dhTs);
+    a.a_scale_ld = d;
+    a.a_rows = d;
+    a.b_scale = reinterpret_cast<const float*>(ws + B.zgTs);
+    a.b_scale_ld = I;
+    a.b_rows = I;
+    a.out_bf16 = static_cast<__nv_bfloat16*>(dw_down);
+    a.out_ld = I;
+    a.out_cols = I;
+    rc = launch_chain("FP8 backward GEMM dW_down = dY^T Z",
+                      gemm8::k_gemm_promoted<2, gemm8::EPI_BF16_OUT, true>,
+                      dim3(grid_of((int64_t)E * (d / 128) * a.n_tiles_n)),
+                      dim3(gemm8::NUM_THREADS), smem, st, ta, tb, a);
+    if (rc != MOE_OK) return rc;
+  }
+  {
+    CUtensorMap ta, tb;
+    rc = make_tmap(&ta, ws + B.dabT, 1, rs, 2 * I, gemm8::BM);
+    if (rc == MOE_OK) rc = make_tmap(&tb, ws + B.xT, 1, rs, d, gemm8::BN);
+    if (rc != MOE_OK) return rc;
+    gemm8::Args a = base_args(gtab_wgu, d / gemm8::BN, 0, 0);
+    a.kgroup = kgroup;
+    a.a_scale = reinterpret_cast<const float*>(ws + B.dabTs);
+    a.a_scale_ld = 2 * I;
+    a.a_rows = 2 * I;
+    a.b_scale = reinterpret_cast<const float*>(ws + B.xTs);
+    a.b_scale_ld = d;
+    a.b_rows = d;
+    a.out_bf16 = static_cast<__nv_bfloat16*>(dw_gu);
+    a.out_ld = d;
+    a.out_cols = d;
+    rc = launch_chain("FP8 backward GEMM dW_gu = dAB^T X",
+                      gemm8::k_gemm_promoted<2, gemm8::EPI_BF16_OUT, true>,
+                      dim3(grid_of((int64_t)E * (2 * I / 128) * a.n_tiles_n)),
+                      dim3(gemm8::NUM_THREADS), smem, st, ta, tb, a);
+    if (rc != MOE_OK) return rc;
+  }
+  // G6b: dW_r = dl^T X (bf16 gating GEMM), bf16 out
+  ga.tab = tab_dwr;
+  ga.c = dw_router;
+  ga.ldc = d;
+  return launch_gemm_bwd_pair("backward GEMM dW_r = dL^T X (CTA pairs)", DL, DL, X, X, ga,
+                              (uint64_t)N, 1, ((N + 255) / 256) * nt(d), true, st);
+}
+
 __global__ void k_selftest_wait(uint64_t limit_ns) {
   __shared__ uint64_t bar;
   if (threadIdx.x == 0) {
@@ -1636,6 +1976,58 @@ moe_status moe_backward_saved(const moe_layer_desc* desc, const void* x, const v
   if (D.T > 0 && !ab_saved) return MOE_ERR_INVALID_ARG;
   return backward_entry(desc, x, w_router, bias, w_gu, w_down, dh, dx, dw_router, dw_gu, dw_down,
                         bf16_grads != 0, ab_saved, ws, ws_bytes, stream);
+}
+
+size_t moe_backward_fp8_workspace_size(const moe_layer_desc* desc) {
+  Dims D;
+  if (fill_dims(desc, &D) != MOE_OK || !D.fp8) return 0;
+  return bwd8_layout(D, layout(D)).total;
+}
+
+moe_status moe_backward_fp8(const moe_layer_desc* desc, const void* x, const void* w_router,
+                            const float* bias, const void* w_gu, const float* w_gu_scale,
+                            const void* w_gu_t, const float* w_gu_t_scale, const void* w_down,
+                            const float* w_down_scale, const void* w_down_t,
+                            const float* w_down_t_scale, const void* dh, void* dx,
+                            void* dw_router, void* dw_gu, void* dw_down, void* ws,
+                            size_t ws_bytes, cudaStream_t stream) {
+  Dims D;
+  moe_status rc = fill_dims(desc, &D);
+  if (rc != MOE_OK) return rc;
+  if (!D.fp8) return MOE_ERR_UNSUPPORTED;
+  if (bias && desc->gate != MOE_GATE_SIGMOID) return MOE_ERR_INVALID_ARG;
+  if (D.E > 1024 || D.K + D.Ks > 32 || D.d % 256 || (D.N * 2) % 16) return MOE_ERR_UNSUPPORTED;
+  if (D.T > 0) {
+    const void* need[] = {x, w_router, w_gu, w_gu_t, w_down, w_down_t, dh, dx, dw_router, dw_gu,
+                          dw_down};
+    for (const void* p : need)
+      if (!p || !aligned16(p)) return MOE_ERR_INVALID_ARG;
+    const float* scales[] = {w_gu_scale, w_gu_t_scale, w_down_scale, w_down_t_scale};
+    for (const float* p : scales)
+      if (!p || ((uintptr_t)p & 3u)) return MOE_ERR_INVALID_ARG;
+    if (bias && !aligned16(bias)) return MOE_ERR_INVALID_ARG;
+  }
+  const Layout L = layout(D);
+  const Bwd8Layout B = bwd8_layout(D, L);
+  if (!ws || ws_bytes < B.total || !aligned16(ws)) return MOE_ERR_WORKSPACE;
+  if (B.rs >= ((int64_t)1 << 31) / 2) return MOE_ERR_INVALID_ARG;
+  if (D.T == 0) return MOE_OK;
+  int sms;
+  if ((rc = device_setup(&sms)) != MOE_OK) return rc;
+  const Fp8Weights W{w_gu, w_gu_t, w_down, w_down_t, w_gu_scale, w_gu_t_scale, w_down_scale,
+                     w_down_t_scale};
+  return do_backward_fp8(*desc, D, L, B, x, w_router, bias, W, dh, dx, dw_router, dw_gu, dw_down,
+                         static_cast<uint8_t*>(ws), sms, stream);
+}
+
+int32_t moe_backward_fp8_launch_count(const moe_layer_desc* desc) {
+  Dims D;
+  if (fill_dims(desc, &D) != MOE_OK || !D.fp8) return 0;
+  if (D.T == 0) return 0;
+  // route (2) + hist, scan, slots (3) + prep, gather, pads (3) + ab, dz, the dAB
+  // quantisation, du (4) + gate backward, dx_router, combine (3) + four
+  // column quantisations + dW_down, dW_gu, dW_r (7)
+  return 2 + 3 + 3 + 4 + 3 + 7;
 }
 
 int32_t moe_backward_launch_count(const moe_layer_desc* desc) {

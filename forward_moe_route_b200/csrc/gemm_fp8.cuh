@@ -56,7 +56,8 @@ static_assert(128 * CTRL_REGS + (NUM_THREADS - 128) * EPI_REGS == NUM_THREADS * 
 constexpr int NUM_EPI = NUM_THREADS - EPI_WARP0 * 32;   // 512
 constexpr int TMEM_COLS = 512;       // two 256-column partials
 
-enum Epi { EPI_F32_STORE = 0, EPI_SWIGLU_Q = 1, EPI_SCATTER = 2 };
+enum Epi { EPI_F32_STORE = 0, EPI_SWIGLU_Q = 1, EPI_SCATTER = 2, EPI_BF16_OUT = 3,
+           EPI_SWIGLU_BWD = 4 };
 
 struct Args {
   gemm::GroupTab gt;
@@ -93,11 +94,29 @@ struct Args {
   int plain;
   const float* row_w;
   const unsigned long long* group_base;
+  // BF16_OUT: out_bf16 [rows, out_ld] bf16, row c_row + i, columns < out_cols
+  __nv_bfloat16* out_bf16;
+  // SWIGLU_BWD (backward dz' = dh W_down; rows c_row + i, features < inter):
+  // a | b in, g z, [da | db] and per-64-feature partials of <dz', z> out;
+  // routed rows take their gate weight from row_w
+  const __nv_bfloat16* ab;   // [rows, 2I]
+  __nv_bfloat16* zg;         // [rows, I]
+  __nv_bfloat16* dab;        // [rows, 2I]
+  float* dgp;                // [rows, I / 64]
+  // weight-gradient mode (template WG): group g contracts over K elements
+  // kgroup[2g] .. + 128 kgroup[2g+1]; both operands carry one scale per row
+  // and 128-element k-block, stored k-block-major: a_scale[kb][a_scale_ld],
+  // b_scale[kb][b_scale_ld] (kb counted from K element 0); b_rows = rows of B
+  const int* kgroup;
+  int a_scale_ld, b_scale_ld, b_rows;
 };
+
+constexpr int SB_FLOATS = (NUM_EPI / 32) * 64;   // WG: per-warp column scales of a k-block
 
 __host__ inline size_t smem_bytes(int stages, int n_groups) {
   return 1024 + (size_t)stages * (BM * KB + BN * KB) + (size_t)(2 * stages + 6) * 8 + 16 +
-         2 * 4 * BM * sizeof(float) + (size_t)(n_groups + 1) * 4 + 64;
+         2 * 4 * BM * sizeof(float) + SB_FLOATS * sizeof(float) + (size_t)(n_groups + 1) * 4 +
+         64;
 }
 
 // ----------------------------------------------------------------------------- shared pieces
@@ -132,6 +151,103 @@ __device__ __forceinline__ void promote64(uint32_t tb, float (&acc)[64], float m
       acc[o + 1] = r.y;
     }
   }
+}
+
+// Promotion with a scale per accumulator column (weight-gradient mode):
+// acc[j] += (sa * sb[j]) * P[col0 + j], with sb the slice's 64 column scales
+// of this k-block in shared memory (every lane reads the same address).
+__device__ __forceinline__ void promote64_cols(uint32_t tb, float (&acc)[64], float sa,
+                                               const float* sb) {
+  const float2 a2 = make_float2(sa, sa);
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    uint32_t va[16], vb[16];
+    tmem_ld16_nowait(tb + (uint32_t)(32 * h), va);
+    tmem_ld16_nowait(tb + (uint32_t)(32 * h + 16), vb);
+    tmem_wait_ld2(va, vb);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int o = 32 * h + 2 * i;
+      const float2 m = __fmul2_rn(a2, *reinterpret_cast<const float2*>(sb + o));
+      const float2 r = __ffma2_rn(m, make_float2(__uint_as_float(va[2 * i]),
+                                                 __uint_as_float(va[2 * i + 1])),
+                                  make_float2(acc[o], acc[o + 1]));
+      acc[o] = r.x;
+      acc[o + 1] = r.y;
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int o = 32 * h + 16 + 2 * i;
+      const float2 m = __fmul2_rn(a2, *reinterpret_cast<const float2*>(sb + o));
+      const float2 r = __ffma2_rn(m, make_float2(__uint_as_float(vb[2 * i]),
+                                                 __uint_as_float(vb[2 * i + 1])),
+                                  make_float2(acc[o], acc[o + 1]));
+      acc[o] = r.x;
+      acc[o + 1] = r.y;
+    }
+  }
+}
+
+// 64 fp32 values as bf16 (round to nearest even) at dst, 16-byte stores.
+__device__ __forceinline__ void store_bf16x64(__nv_bfloat16* dst, const float (&v)[64]) {
+  uint4* o = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+    o[j] = make_uint4(gemm::pack_bf16x2(v[8 * j], v[8 * j + 1]),
+                      gemm::pack_bf16x2(v[8 * j + 2], v[8 * j + 3]),
+                      gemm::pack_bf16x2(v[8 * j + 4], v[8 * j + 5]),
+                      gemm::pack_bf16x2(v[8 * j + 6], v[8 * j + 7]));
+}
+
+// Backward epilogue of dz' = dh W_down for 64 features f0 .. f0+63 of row
+// crow (gate weight gw, 1 for a shared expert): with a, b the pre-activations,
+//   z = SiLU(a) b,  g z,  dz = g dz',  da = dz b SiLU'(a),  db = dz SiLU(a),
+// and the partial <dz', z> over these features.  A padding row (valid false)
+// gets zeros, so the weight-gradient quantisation may read it.
+__device__ __forceinline__ void epi_swiglu_bwd(const float (&acc)[64], const Args& a,
+                                               long long crow, int f0, float gw, bool valid) {
+  const int I = a.inter;
+  __nv_bfloat16* zr = a.zg + crow * I + f0;
+  __nv_bfloat16* dar = a.dab + crow * 2 * I + f0;
+  float dgs = 0.f;
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    uint32_t wz[4], wa[4], wb[4];
+    if (valid) {
+      const uint4 ra = *reinterpret_cast<const uint4*>(a.ab + crow * 2 * I + f0 + 8 * c);
+      const uint4 rb = *reinterpret_cast<const uint4*>(a.ab + crow * 2 * I + I + f0 + 8 * c);
+      const __nv_bfloat162* ha = reinterpret_cast<const __nv_bfloat162*>(&ra);
+      const __nv_bfloat162* hb = reinterpret_cast<const __nv_bfloat162*>(&rb);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        float zz[2], da2[2], db2[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const float av = h ? __high2float(ha[j]) : __low2float(ha[j]);
+          const float bv = h ? __high2float(hb[j]) : __low2float(hb[j]);
+          const float sg = 1.0f / (1.0f + __expf(-av));
+          const float si = av * sg;
+          const float z = si * bv;
+          const float dzp = acc[8 * c + 2 * j + h];
+          const float dz = gw * dzp;
+          dgs = fmaf(dzp, z, dgs);
+          zz[h] = gw * z;
+          da2[h] = dz * bv * (sg * (1.0f + av * (1.0f - sg)));
+          db2[h] = dz * si;
+        }
+        wz[j] = gemm::pack_bf16x2(zz[0], zz[1]);
+        wa[j] = gemm::pack_bf16x2(da2[0], da2[1]);
+        wb[j] = gemm::pack_bf16x2(db2[0], db2[1]);
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) wz[j] = wa[j] = wb[j] = 0u;
+    }
+    reinterpret_cast<uint4*>(zr)[c] = make_uint4(wz[0], wz[1], wz[2], wz[3]);
+    reinterpret_cast<uint4*>(dar)[c] = make_uint4(wa[0], wa[1], wa[2], wa[3]);
+    reinterpret_cast<uint4*>(dar + I)[c] = make_uint4(wb[0], wb[1], wb[2], wb[3]);
+  }
+  a.dgp[crow * (I / 64) + f0 / 64] = valid ? dgs : 0.f;
 }
 
 // GEMM1 epilogue of one row's 64-column slice cs (gate columns 0..31, the
@@ -192,7 +308,7 @@ __device__ __forceinline__ void epi_scatter(const float (&acc)[64], const Args& 
     const int pair = a.pair_of[a.gt.c_row(g) + grow];
     const int t = pair / a.K, k = pair - t * a.K;
     dst = (long long)t * (a.K + a.Ks) + k;
-    wgt = a.topk_w[pair];
+    wgt = a.topk_w ? a.topk_w[pair] : 1.0f;   // the backward's du pieces carry no weight
   } else {
     dst = (long long)grow * (a.K + a.Ks) + a.K + s_idx;
   }
@@ -205,7 +321,7 @@ __device__ __forceinline__ void epi_scatter(const float (&acc)[64], const Args& 
                       gemm::pack_bf16x2(acc[8 * j + 6] * wgt, acc[8 * j + 7] * wgt));
 }
 
-template <int KIND, int EPI>
+template <int KIND, int EPI, bool WG = false>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     k_gemm_promoted(const __grid_constant__ CUtensorMap tmA,
                        const __grid_constant__ CUtensorMap tmB, const Args a) {
@@ -226,7 +342,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* amax_buf = reinterpret_cast<float*>(tmem_slot + 4);   // [2][4][128]
-  int* s_prefix = reinterpret_cast<int*>(amax_buf + 2 * 4 * BM);
+  float* sb_buf = amax_buf + 2 * 4 * BM;                        // WG: [16 warps][64]
+  int* s_prefix = reinterpret_cast<int*>(sb_buf + SB_FLOATS);
 
   const int warp = warp_id(), lane = lane_id();
   const int n_groups = a.gt.count();
@@ -277,14 +394,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const int lm = mt - s_prefix[g];
           const int arow = (a.a_from_crow ? a.gt.c_row(g) : a.gt.a_row(g)) + lm * BM;
           const int ebase = a.gt.expert(g) * a.b_rows_per_expert;
-          for (int kb = 0; kb < a.num_kb; ++kb, ++it) {
+          const int k0 = WG ? a.kgroup[2 * g] : 0;
+          const int nkb = WG ? a.kgroup[2 * g + 1] : a.num_kb;
+          for (int kb = 0; kb < nkb; ++kb, ++it) {
             const int s = it % S;
             const uint32_t ph = (uint32_t)(it / S) & 1u;
             if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag)) { ok = false; break; }
             uint8_t* sa = smem + (size_t)s * stage_bytes;
             uint8_t* sb = sa + a_bytes;
             mbar_arrive_expect_tx(&full[s], stage_bytes);
-            const int kx = kb * a.kb_elems;
+            const int kx = k0 + kb * a.kb_elems;
             tma_load_2d(&tmA, &full[s], sa, kx, arow);
             if (EPI == EPI_SWIGLU_Q) {
               const int gr = ebase + nt * 128, ur = ebase + a.b_up_off + nt * 128;
@@ -311,7 +430,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         int it = 0, pu = 0;
         bool ok = true;
         for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
-          for (int kb = 0; kb < a.num_kb; ++kb, ++it, ++pu) {
+          int nkb = a.num_kb;
+          if (WG) {
+            const int g = gemm::find_group(s_prefix, n_groups, tile / a.n_tiles_n);
+            nkb = a.kgroup[2 * g + 1];
+          }
+          for (int kb = 0; kb < nkb; ++kb, ++it, ++pu) {
             const int s = it % S;
             const uint32_t ph = (uint32_t)(it / S) & 1u;
             const int p = pu & 1;
@@ -366,20 +490,47 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         sa_row = arow < a.a_rows ? a.a_scale + (size_t)arow * a.num_kb : nullptr;
         sb0 = a.b_scale + (eb + nt) * a.num_kb;                          // gate block
         sb1 = a.b_scale + (eb + a.b_up_off / 128 + nt) * a.num_kb;       // up block
-      } else {
+      } else if (!WG) {
         sa_row = arow < a.a_rows ? a.a_scale + (size_t)arow * a.num_kb : nullptr;
-        sb0 = a.b_scale + (eb + 2 * nt + cs / 2) * a.num_kb;
+        // a slice past the expert's last B row block (N not a multiple of 256)
+        // is never stored; its scale read stays inside the expert's blocks
+        sb0 = a.b_scale + (eb + min(2 * nt + cs / 2, kb_blocks_b - 1)) * a.num_kb;
         sb1 = sb0;
       }
       float acc[64];
 #pragma unroll
       for (int i = 0; i < 64; ++i) acc[i] = 0.f;
       const bool scaled = EPI != EPI_F32_STORE;
-      float na = scaled ? (sa_row ? sa_row[0] : 0.f) : 1.f;
-      float nb0 = scaled ? sb0[0] : 1.f, nb1 = scaled ? sb1[0] : 1.f;
-      for (int kb = 0; kb < a.num_kb; ++kb, ++pu) {
+      // weight-gradient mode: this group's K range, the row's and the slice's
+      // column scales of the next k-block (prefetched one k-block ahead)
+      const int nkb = WG ? a.kgroup[2 * g + 1] : a.num_kb;
+      const int kb0 = WG ? a.kgroup[2 * g] / 128 : 0;
+      const int ncol = nt * BN + col0;
+      float* sbw = sb_buf + ew * 64;
+      float wsa = 0.f, wsb0 = 0.f, wsb1 = 0.f;
+      if (WG && nkb > 0) {
+        wsa = arow < a.a_rows ? a.a_scale[(size_t)kb0 * a.a_scale_ld + arow] : 0.f;
+        wsb0 = ncol + lane < a.b_rows ? a.b_scale[(size_t)kb0 * a.b_scale_ld + ncol + lane] : 0.f;
+        wsb1 = ncol + 32 + lane < a.b_rows
+                   ? a.b_scale[(size_t)kb0 * a.b_scale_ld + ncol + 32 + lane] : 0.f;
+      }
+      float na = (scaled && !WG) ? (sa_row ? sa_row[0] : 0.f) : 1.f;
+      float nb0 = (scaled && !WG) ? sb0[0] : 1.f, nb1 = (scaled && !WG) ? sb1[0] : 1.f;
+      for (int kb = 0; kb < nkb; ++kb, ++pu) {
         const float m0 = na * nb0, m1 = na * nb1;
-        if (scaled && kb + 1 < a.num_kb) {
+        const float sa_k = wsa;
+        if (WG) {
+          sbw[lane] = wsb0;
+          sbw[32 + lane] = wsb1;
+          __syncwarp();
+          if (kb + 1 < nkb) {
+            const size_t kr = (size_t)(kb0 + kb + 1);
+            wsa = arow < a.a_rows ? a.a_scale[kr * a.a_scale_ld + arow] : 0.f;
+            wsb0 = ncol + lane < a.b_rows ? a.b_scale[kr * a.b_scale_ld + ncol + lane] : 0.f;
+            wsb1 = ncol + 32 + lane < a.b_rows ? a.b_scale[kr * a.b_scale_ld + ncol + 32 + lane]
+                                               : 0.f;
+          }
+        } else if (scaled && kb + 1 < nkb) {
           na = sa_row ? sa_row[kb + 1] : 0.f;
           nb0 = sb0[kb + 1];
           nb1 = sb1[kb + 1];
@@ -389,7 +540,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tc_fence_after();
         const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(p * BN + col0);
         // the router's unscaled promotion is a paired FMA with multiplier 1
-        promote64(tb, acc, m0, m1);
+        if (WG) promote64_cols(tb, acc, sa_k, sbw);
+        else promote64(tb, acc, m0, m1);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&pempty[p]);
@@ -415,6 +567,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                           (size_t)(a.gt.c_row(g) + grow), nt, abort_flag)) {
           ok = false;
           break;
+        }
+      } else if (EPI == EPI_BF16_OUT) {
+        if (valid && ncol + 64 <= a.out_cols)
+          store_bf16x64(a.out_bf16 + (size_t)(a.gt.c_row(g) + grow) * a.out_ld + ncol, acc);
+      } else if (EPI == EPI_SWIGLU_BWD) {
+        if (ncol + 64 <= a.inter) {
+          const long long crow = (long long)a.gt.c_row(g) + grow;
+          const float gw = (a.gt.aux(g) < 0 && valid) ? a.row_w[crow] : 1.0f;
+          epi_swiglu_bwd(acc, a, crow, ncol, gw, valid);
         }
       } else {
         if (valid) epi_scatter(acc, a, g, grow, nt * BN + col0);

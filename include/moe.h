@@ -432,6 +432,42 @@ moe_status moe_backward_saved(const moe_layer_desc* desc, const void* x, const v
                               void* dw_gu, void* dw_down, int32_t bf16_grads, void* ws,
                               size_t ws_bytes, cudaStream_t stream);
 
+/* ---- The backward with FP8 GEMMs (E4M3 layers) ----------------------------
+ * "DeepSeek Technical Report: MoE Architecture", §3.6: the activation-backward
+ * and weight-backward GEMMs in FP8 E4M3, activations per 1x128 tile, weights
+ * per 128x128 block, fp32 accumulation promoted every 128 elements; gating in
+ * BF16; weight gradients in BF16.  Same gradients as moe_backward.
+ * Tiles run along the dimension each GEMM contracts over: x and dh rows (over
+ * d) for a, b = W_gate u, W_up u and dz' = W_down^T dh; the [da | db] rows
+ * (over 2I) for du; and, for dW_down = sum dh (g z)^T and dW_gu = sum
+ * [da | db] u^T, which contract over an expert's rows, tiles of 128 rows x 1
+ * column, the expert's rows taken in token order and padded with zero rows to
+ * a multiple of 128 (a shared expert's rows are all T tokens).
+ * Weights: the forward's E4M3 codes and 128x128 block scales
+ * (moe_quantize_fp8_blockwise) and the same for the transposed matrices,
+ *   w_gu [E, 2I, d] + w_gu_scale [E, 2I/128, d/128],
+ *   w_gu_t [E, d, 2I] + w_gu_t_scale [E, d/128, 2I/128],
+ *   w_down [E, d, I] + w_down_scale [E, d/128, I/128],
+ *   w_down_t [E, I, d] + w_down_t_scale [E, I/128, d/128]
+ * (quantising a transposed bf16 matrix gives the transposed codes and scales,
+ * since a block's amax does not depend on its orientation).
+ *   x [T, d] bf16, w_router [N, d] bf16, bias [N] fp32 or NULL, dh [T, d] bf16
+ *   dx [T, d] bf16 out; dw_router [N, d], dw_gu [E, 2I, d], dw_down [E, d, I]
+ *     bf16 out (zeros for experts no token reaches)
+ *   ws: moe_backward_fp8_workspace_size(desc) bytes (0 for non-E4M3 layers).
+ * E4M3 layers only, with d a multiple of 256, K + Ks <= 32 and N*2 a multiple
+ * of 16 (MOE_ERR_UNSUPPORTED otherwise); tensors 16-byte aligned, scales
+ * 4-byte aligned.  Launches moe_backward_fp8_launch_count(desc) kernels. */
+size_t moe_backward_fp8_workspace_size(const moe_layer_desc* desc);
+moe_status moe_backward_fp8(const moe_layer_desc* desc, const void* x, const void* w_router,
+                            const float* bias, const void* w_gu, const float* w_gu_scale,
+                            const void* w_gu_t, const float* w_gu_t_scale, const void* w_down,
+                            const float* w_down_scale, const void* w_down_t,
+                            const float* w_down_t_scale, const void* dh, void* dx,
+                            void* dw_router, void* dw_gu, void* dw_down, void* ws,
+                            size_t ws_bytes, cudaStream_t stream);
+int32_t moe_backward_fp8_launch_count(const moe_layer_desc* desc);
+
 /* Number of kernels moe_backward launches for `desc` (0 if invalid or T = 0). */
 int32_t moe_backward_launch_count(const moe_layer_desc* desc);
 

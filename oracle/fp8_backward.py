@@ -26,8 +26,11 @@ Readings taken where the pages are silent:
     come out of FP8 GEMMs with fp32 accumulation and are not requantised.
   * dg (the gradient of a gate weight) is <dz', z> with dz' from that FP8
     GEMM, as the unquantised layer's <dh, W_down z> = <W_down^T dh, z>.
-  * Intermediates are held in fp32 before they are quantised (the GPU holds
-    a, b, g z and [da | db] in bf16; that rounding is inside the tolerance).
+  * Intermediates: by default a, b, g z and [da | db] are held in fp32 before
+    they are used or quantised.  With intermediates="bf16" they are rounded
+    to bfloat16 (nearest even, from fp32) first, as a GPU that stores them in
+    bf16 does; that form isolates the GEMMs' own error from this storage
+    choice.
   * The gating backward (gate weights, affinities, the router GEMMs) is exact
     here; on the GPU it runs in BF16 / fp32 as the forward's gating does.
 
@@ -75,6 +78,14 @@ def fp8_weight_grad(a_rows: np.ndarray, b_rows: np.ndarray) -> np.ndarray:
     return of8.dequant_act(qa, sa) @ of8.dequant_act(qb, sb).T
 
 
+def round_bf16(v: np.ndarray) -> np.ndarray:
+    """Nearest bfloat16 values (ties to even) of v rounded to fp32 first, as float64."""
+    f = np.ascontiguousarray(np.asarray(v, np.float64).astype(np.float32))
+    u = f.view(np.uint32).astype(np.uint64)
+    u = ((u + 0x7FFF + ((u >> 16) & 1)) >> 16) << 16
+    return u.astype(np.uint32).view(np.float32).astype(np.float64)
+
+
 def fp8_act(rows: np.ndarray) -> np.ndarray:
     """Rows quantised per 1x128 tile along their columns, dequantised."""
     q, s = of8.quantize_act_1x128(np.asarray(rows, np.float64).astype(F32))
@@ -82,7 +93,7 @@ def fp8_act(rows: np.ndarray) -> np.ndarray:
 
 
 def expert_backward_fp8(u: np.ndarray, dh: np.ndarray, g: np.ndarray, w_gate: np.ndarray,
-                        w_up: np.ndarray, w_down: np.ndarray):
+                        w_up: np.ndarray, w_down: np.ndarray, intermediates: str = "fp32"):
     """One expert's backward with FP8 GEMMs.
 
     u [M, d] and dh [M, d] are the expert's input rows and the upstream
@@ -93,33 +104,36 @@ def expert_backward_fp8(u: np.ndarray, dh: np.ndarray, g: np.ndarray, w_gate: np
     dh = np.asarray(dh, np.float64)
     g = np.asarray(g, np.float64)
     I = w_gate.shape[0]
+    keep = round_bf16 if intermediates == "bf16" else (lambda v: v)
     # the pre-activations, recomputed by the FP8 forward GEMM
     uh = fp8_act(u)
-    a = uh @ w_gate.T
-    b = uh @ w_up.T
+    a = keep(uh @ w_gate.T)
+    b = keep(uh @ w_up.T)
     # activation backward through W_down: dz' = dh W_down, dh rows in FP8
     dzp = fp8_act(dh) @ w_down
     z = mo.silu(a) * b
     dg = np.sum(dzp * z, axis=1)
     dz = g[:, None] * dzp
-    da = dz * b * mb.silu_grad(a)
-    db = dz * mo.silu(a)
+    da = keep(dz * b * mb.silu_grad(a))
+    db = keep(dz * mo.silu(a))
     dab = np.concatenate([da, db], axis=1)
     # activation backward through W_gate, W_up: [da | db] rows in FP8
     du = fp8_act(dab) @ np.concatenate([w_gate, w_up], axis=0)
     # weight backward: contract over the expert's rows, 128-row tiles
-    dw_down = fp8_weight_grad(dh, g[:, None] * z)
+    dw_down = fp8_weight_grad(dh, keep(g[:, None] * z))
     dw_gu = fp8_weight_grad(dab, u)
     return du, dg, dw_gu[:I], dw_gu[I:], dw_down
 
 
 def moe_backward_fp8(x, w_r, bias, expert: ExpertFn, dh, *, n_shared: int, gate: str,
                      top_k: int, n_group: int = 1, topk_group: int = 1, renorm: bool = False,
-                     route_scale: float = 1.0, idx_override: Optional[np.ndarray] = None) -> Dict:
+                     route_scale: float = 1.0, idx_override: Optional[np.ndarray] = None,
+                     intermediates: str = "fp32") -> Dict:
     """Gradients of the FP8 layer (u = x, separate residual), in the format of
     oracle.moe_backward.moe_backward: dx, dx_res, dw_r, experts {e: [dW_gate,
     dW_up, dW_down]} (experts no token reaches are absent), idx, g, dl.
-    expert(e) returns the dequantised E4M3 weights (w_gate, w_up, w_down)."""
+    expert(e) returns the dequantised E4M3 weights (w_gate, w_up, w_down);
+    intermediates "fp32" or "bf16" (see the module docstring)."""
     x = np.asarray(x, np.float64)
     dh = np.asarray(dh, np.float64)
     T, d = x.shape
@@ -139,7 +153,7 @@ def moe_backward_fp8(x, w_r, bias, expert: ExpertFn, dh, *, n_shared: int, gate:
     def run(e, rows, g_rows):
         w_gate, w_up, w_down = (np.asarray(w, np.float64) for w in expert(e))
         du, dg_rows, dwg, dwu, dwd = expert_backward_fp8(x[rows], dh[rows], g_rows, w_gate,
-                                                         w_up, w_down)
+                                                         w_up, w_down, intermediates)
         dx[rows] += du
         grads[e] = [dwg, dwu, dwd]
         return dg_rows

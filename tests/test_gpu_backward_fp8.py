@@ -1,0 +1,186 @@
+"""GPU parity of the FP8 backward (moe_backward_fp8) against the oracle's
+emulation of it (oracle/fp8_backward.py, pinned in
+tests/test_oracle_fp8_backward.py) and against the exact fp64 backward.
+
+Both sides use the same E4M3 weights: the GPU's moe_quantize_fp8_blockwise
+codes and scales equal the oracle's 128x128 quantisation bit for bit (checked
+in tests/test_gpu_fp8.py; the transposed matrices are checked here), and the
+GPU's selection (no gradient flows through the choice of experts).
+
+Bounds, every gradient as a whole tensor (max-abs-relative):
+  * 2e-2 (the bf16 layer's bound) of the emulation with bf16 intermediates,
+    which rounds a, b, g z and [da | db] to bf16 as the GPU stores them, so
+    both sides quantise the same values (measured 1.6e-3 .. 5.2e-3);
+  * 6e-2 (the FP8 layer's bound) of the emulation with fp32 intermediates,
+    where E4M3 codes of the intermediates near a rounding boundary differ
+    (measured 3e-3 .. 2.9e-2);
+  * 2^-3 (twice E4M3's relative step) of the exact fp64 backward (measured
+    2.5e-2 .. 6.6e-2).
+"""
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+import forward_moe_route_b200 as moe
+import synth
+from oracle import fp8 as of8
+from oracle import fp8_backward as fb
+from oracle import moe_backward as mb
+from oracle import moe_oracle as mo
+from synth import recipes
+
+from gpu_layer import HostLayer, f64
+
+pytestmark = pytest.mark.gpu
+
+TOL = 6e-2
+BF_TOL = 2e-2
+PLAIN_TOL = 2.0 ** -3
+TID_DH = 6
+
+C = recipes.CONFIGS
+CASES = {
+    # V3-like FP8 layer: sigmoid + bias, 4 groups / top-2, renorm x 2.5, ragged T
+    "v3_fp8_small": dataclasses.replace(
+        recipes.small_variant(C["v3_fp8"], T=300, d=512, inter=256, n_routed=32),
+        n_group=4, topk_group=2),
+    # I not a multiple of 256 (a half column tile in dz' and dW_down); about
+    # 150 rows per routed expert: segments of two 128-row blocks
+    "v3_fp8_ragged": dataclasses.replace(
+        recipes.small_variant(C["v3_fp8"], T=300, d=768, inter=384, n_routed=16),
+        n_group=4, topk_group=2),
+    # the V3 feature sizes d = 7168, I = 2048 with 16 routed experts
+    "v3_fp8_reduced": dataclasses.replace(
+        recipes.small_variant(C["v3_fp8"], T=384, d=7168, inter=2048, n_routed=16),
+        n_group=8, topk_group=4),
+    # one token: most experts get no row and zero weight gradients
+    "v3_fp8_T1": dataclasses.replace(
+        recipes.small_variant(C["v3_fp8"], T=1, d=256, inter=128, n_routed=32),
+        n_group=4, topk_group=2),
+}
+
+
+class Fp8Host(HostLayer):
+    """Host layer whose experts are the oracle's own 128x128 quantisation."""
+
+    def expert(self, e):
+        if e not in self._experts:
+            wg, wu, wd = recipes.host_expert(self.cfg, e)
+            gu = np.concatenate([wg, wu]).astype(np.float32)
+            qg, sg = of8.quantize_weight_128x128(gu)
+            qd, sd = of8.quantize_weight_128x128(wd.astype(np.float32))
+            guh = of8.dequant_weight(qg, sg)
+            I = self.cfg.inter
+            self._experts[e] = (guh[:I], guh[I:], of8.dequant_weight(qd, sd))
+        return self._experts[e]
+
+
+def quantize(w, rows, cols, E):
+    q = torch.empty(E, rows, cols, dtype=torch.uint8, device="cuda")
+    s = torch.empty(E, rows // 128, cols // 128, dtype=torch.float32, device="cuda")
+    moe.moe_quantize_fp8_blockwise(w.contiguous(), rows, cols, E, q, s)
+    return q, s
+
+
+def fp8_weights(cfg, inp):
+    E, I, d = cfg.n_experts, cfg.inter, cfg.d
+    gq, gs = quantize(inp["w_gu"], 2 * I, d, E)
+    gtq, gts = quantize(inp["w_gu"].transpose(1, 2), d, 2 * I, E)
+    dq, ds = quantize(inp["w_down"], d, I, E)
+    dtq, dts = quantize(inp["w_down"].transpose(1, 2), I, d, E)
+    return gq, gs, gtq, gts, dq, ds, dtq, dts
+
+
+def upstream(cfg):
+    v = synth.host_normal(cfg.T * cfg.d, 1.0, cfg.seed, TID_DH).reshape(cfg.T, cfg.d)
+    dh = torch.from_numpy(v).to(torch.bfloat16)
+    return dh.cuda(), dh.double().numpy()
+
+
+def run(cfg, inp, W, dh):
+    desc = moe.desc_from_config(cfg)
+    ws = moe.backward_fp8_workspace(desc)
+    E, I, d, N = cfg.n_experts, cfg.inter, cfg.d, cfg.n_routed
+    bf = dict(dtype=torch.bfloat16, device="cuda")
+    dx = torch.full((cfg.T, d), float("nan"), **bf)
+    dwr = torch.full((N, d), float("nan"), **bf)
+    dwgu = torch.full((E, 2 * I, d), float("nan"), **bf)
+    dwd = torch.full((E, d, I), float("nan"), **bf)
+    gq, gs, gtq, gts, dq, ds, dtq, dts = W
+    moe.moe_backward_fp8(desc, inp["x"], inp["w_r"], inp["bias"], gq, gs, gtq, gts, dq, ds, dtq,
+                         dts, dh, dx, dwr, dwgu, dwd, ws)
+    return dx, dwr, dwgu, dwd, moe.moe_last_device_status()
+
+
+def gpu_selection(cfg, inp):
+    desc = moe.desc_from_config(cfg)
+    ws = moe.workspace(desc)
+    idx = torch.empty(cfg.T, cfg.top_k, dtype=torch.int32, device="cuda")
+    w = torch.empty(cfg.T, cfg.top_k, dtype=torch.float32, device="cuda")
+    counts = torch.empty(cfg.n_routed, dtype=torch.int32, device="cuda")
+    moe.moe_route(desc, inp["x"], inp["w_r"], inp["bias"], idx, w, counts, ws)
+    return idx.cpu().numpy().astype(np.int64)
+
+
+def whole_err(cfg, got_of, ref_of, ref_experts):
+    num = den = 0.0
+    for e in range(cfg.n_experts):
+        got = f64(got_of(e))
+        want = ref_of(e) if e in ref_experts else np.zeros_like(got)
+        num = max(num, float(np.max(np.abs(got - want))))
+        den = max(den, float(np.max(np.abs(want))))
+    return num / den
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_fp8_backward_parity(name):
+    cfg = CASES[name]
+    moe.moe_last_device_status()
+    inp = recipes.device_inputs(cfg)
+    W = fp8_weights(cfg, inp)
+    # the transposed quantisation is the transpose of the codes and scales
+    assert torch.equal(W[2][0], W[0][0].t()) and torch.equal(W[3][0], W[1][0].t())
+    assert torch.equal(W[6][-1], W[4][-1].t()) and torch.equal(W[7][-1], W[5][-1].t())
+    dh, dh64 = upstream(cfg)
+    dx, dwr, dwgu, dwd, st = run(cfg, inp, W, dh)
+    assert st == moe.OK, moe.moe_status_string(st)
+    g_idx = gpu_selection(cfg, inp)
+    host = Fp8Host(cfg)
+    kw = dict(n_shared=cfg.n_shared, gate=cfg.gate, top_k=cfg.top_k, n_group=cfg.n_group,
+              topk_group=cfg.topk_group, renorm=cfg.renorm, route_scale=cfg.route_scale,
+              idx_override=g_idx)
+    emu = fb.moe_backward_fp8(host.x, host.w_r, host.bias, host.expert, dh64, **kw)
+    emu_bf = fb.moe_backward_fp8(host.x, host.w_r, host.bias, host.expert, dh64,
+                                 intermediates="bf16", **kw)
+    exact = mb.moe_backward(host.x, host.w_r, host.bias, host.expert, dh64, **kw)
+    for ref, tol, label in ((emu_bf, BF_TOL, "emulation with bf16 intermediates"),
+                            (emu, TOL, "emulation"), (exact, PLAIN_TOL, "exact")):
+        errs = {
+            "dx": mo.max_abs_rel(f64(dx), ref["dx"]),
+            "dw_router": mo.max_abs_rel(f64(dwr), ref["dw_r"]),
+            "dw_gu": whole_err(cfg, lambda e: dwgu[e],
+                               lambda e: np.concatenate(ref["experts"][e][:2]), ref["experts"]),
+            "dw_down": whole_err(cfg, lambda e: dwd[e], lambda e: ref["experts"][e][2],
+                                 ref["experts"]),
+        }
+        print(f"{name} vs {label}: " + ", ".join(f"{k} {v:.2e}" for k, v in errs.items()))
+        for k, v in errs.items():
+            assert v <= tol, f"{k} vs {label}: max-abs-rel {v:.3e} above {tol}"
+    untouched = [cfg.n_shared + j for j in range(cfg.n_routed) if not np.any(g_idx == j)]
+    if untouched:
+        assert torch.count_nonzero(dwgu[untouched]) == 0
+        assert torch.count_nonzero(dwd[untouched]) == 0
+
+
+def test_fp8_backward_is_deterministic():
+    cfg = CASES["v3_fp8_small"]
+    inp = recipes.device_inputs(cfg)
+    W = fp8_weights(cfg, inp)
+    dh, _ = upstream(cfg)
+    a = run(cfg, inp, W, dh)
+    b = run(cfg, inp, W, dh)
+    assert a[4] == moe.OK and b[4] == moe.OK
+    for x, y in zip(a[:4], b[:4]):
+        assert torch.equal(x, y)

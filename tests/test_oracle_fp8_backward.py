@@ -148,3 +148,23 @@ def test_fp8_backward_is_near_the_exact_backward(gate):
     assert errs[worst] <= bound, f"{worst}: {errs[worst]:.3e}"
     # and FP8 is not the exact backward: the quantisation shows
     assert errs["dx"] > 1e-4
+
+
+def test_round_bf16_matches_the_library_cast():
+    import torch
+    rng = np.random.default_rng(5)
+    v = np.concatenate([rng.normal(size=4000) * 10.0 ** rng.integers(-6, 6, 4000),
+                        [0.0, -0.0, 1.0, 1.00390625, 1.01171875, -3.0e38, 65504.0]])
+    want = torch.from_numpy(v.astype(np.float32)).to(torch.bfloat16).double().numpy()
+    assert np.array_equal(fb.round_bf16(v), want)
+
+
+def test_bf16_intermediates_stay_near_fp32_ones():
+    L = SmallLayer("sigmoid", T=150, seed=2)
+    a = L.fp8()
+    b = fb.moe_backward_fp8(L.x, L.w_r, L.bias, L.w.__getitem__, L.dh,
+                            intermediates="bf16", **L.kw())
+    assert not np.array_equal(a["dx"], b["dx"])
+    assert mo.max_abs_rel(b["dx"], a["dx"]) < 3e-2
+    for e in a["experts"]:
+        assert mo.max_abs_rel(b["experts"][e][2], a["experts"][e][2]) < 5e-2

@@ -542,15 +542,19 @@ def run_backward(args, cfg):
     recomputed pre-activations, dz with the SwiGLU backward, du, the gate and
     affinity backward, dW_down, dW_gu, dW_r), inputs resident in HBM.  With
     --saved the step is moe_backward_saved, which reads the pre-activations
-    moe_forward_save kept instead of recomputing them."""
+    moe_forward_save kept instead of recomputing them; for an E4M3 layer
+    (--config v3_fp8) it is moe_backward_fp8, the backward with FP8 GEMMs."""
     import torch
 
     import forward_moe_route_b200 as moe
     import synth
     from synth import recipes
     torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
-    if cfg.dtype != "bf16":
-        raise SystemExit("the backward is built for bf16 layers")
+    fp8 = cfg.dtype == "e4m3"
+    if cfg.dtype not in ("bf16", "e4m3"):
+        raise SystemExit("the backward is built for bf16 and E4M3 layers")
+    if fp8 and args.saved:
+        raise SystemExit("--saved is for bf16 layers")
     desc = moe.desc_from_config(cfg)
     inp = recipes.device_inputs(cfg, "cuda", load_zipf(cfg))
     dh32 = torch.empty(cfg.T, cfg.d, dtype=torch.float32, device="cuda")
@@ -559,14 +563,31 @@ def run_backward(args, cfg):
     del dh32
     E, I, d, N = cfg.n_experts, cfg.inter, cfg.d, cfg.n_routed
     dx = torch.empty(cfg.T, d, dtype=torch.bfloat16, device="cuda")
-    gdt = torch.bfloat16 if args.bf16_grads else torch.float32
+    gdt = torch.bfloat16 if (args.bf16_grads or fp8) else torch.float32
     dwr = torch.empty(N, d, dtype=gdt, device="cuda")
     dwgu = torch.empty(E, 2 * I, d, dtype=gdt, device="cuda")
     dwd = torch.empty(E, d, I, dtype=gdt, device="cuda")
-    ws = moe.backward_workspace(desc)
+    ws = moe.backward_fp8_workspace(desc) if fp8 else moe.backward_workspace(desc)
     stream = torch.cuda.current_stream()
     fwd_cost = None
-    if args.saved:
+    if fp8:
+        # E4M3 codes and 128x128 block scales of the weights and of their
+        # transposes (offline, like the forward's weight quantisation)
+        def quant(w, rows, cols):
+            q = torch.empty(E, rows, cols, dtype=torch.uint8, device="cuda")
+            sc = torch.empty(E, rows // 128, cols // 128, dtype=torch.float32, device="cuda")
+            moe.moe_quantize_fp8_blockwise(w.contiguous(), rows, cols, E, q, sc)
+            return q, sc
+
+        W8 = (quant(inp["w_gu"], 2 * I, d) + quant(inp["w_gu"].transpose(1, 2), d, 2 * I)
+              + quant(inp["w_down"], d, I) + quant(inp["w_down"].transpose(1, 2), I, d))
+        del inp["w_gu"], inp["w_down"]
+        torch.cuda.empty_cache()
+
+        def step():
+            moe.moe_backward_fp8(desc, inp["x"], inp["w_r"], inp["bias"], *W8, dh, dx, dwr, dwgu,
+                                 dwd, ws, stream)
+    elif args.saved:
         # the forward keeps a | b (moe_forward_save, outside the timed region);
         # its cost over the plain forward is timed alongside
         ab = torch.empty(moe.moe_saved_ab_bytes(desc) // 2, dtype=torch.bfloat16, device="cuda")
@@ -604,7 +625,7 @@ def run_backward(args, cfg):
             moe.moe_backward_saved(desc, inp["x"], inp["w_r"], inp["bias"], inp["w_gu"],
                                    inp["w_down"], dh, ab, dx, dwr, dwgu, dwd, ws,
                                    bf16_grads=args.bf16_grads, stream=stream)
-    else:
+    if not fp8 and not args.saved:
         call = moe.moe_backward_bf16_grads if args.bf16_grads else moe.moe_backward
 
         def step():
@@ -635,20 +656,24 @@ def run_backward(args, cfg):
     pk = peaks()
     done = fl["algorithmic"] + (0.0 if args.saved else fl["recompute"]) + fl["router"]
     tflops = done / (ms * 1e-3) / 1e12
+    # FP8 GEMMs against twice the measured bf16 rate (the sheet's FP8 : bf16 ratio)
+    peak = pk["bf16_tflops_sustained"] * (2.0 if fp8 else 1.0)
     return {"metric": "MoE-layer backward tokens/s", "value": cfg.T / (ms * 1e-3),
             "unit": "tokens/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": cfg.dtype, "data": "synthetic", "config": config_dict(cfg, 1),
-            "weight_gradients": "bf16" if args.bf16_grads else "fp32",
+            "weight_gradients": "bf16" if (args.bf16_grads or fp8) else "fp32",
+            "gemm_precision": "FP8 E4M3 (gating GEMMs bf16)" if fp8 else "bf16",
             "pre_activations": "saved by the forward" if args.saved else "recomputed",
             "forward_cost": fwd_cost,
             "backward_gemm_tflops": tflops,
             "backward_gemm_frac_of_peak": {
-                "measured_sustained": tflops / pk["bf16_tflops_sustained"],
-                "spec_dense": tflops / 2250.0},
+                ("measured_sustained_x2_fp8" if fp8 else "measured_sustained"): tflops / peak,
+                "spec_dense": tflops / (4500.0 if fp8 else 2250.0)},
             "backward_flops": fl,
             "algorithmic_tflops": (fl["algorithmic"] + fl["router"]) / (ms * 1e-3) / 1e12,
-            "gpu_launches": (moe.moe_backward_launch_count(desc) - (1 if args.saved else 0))
+            "gpu_launches": (moe.moe_backward_fp8_launch_count(desc) if fp8 else
+                             moe.moe_backward_launch_count(desc) - (1 if args.saved else 0))
             * args.steps,
             "clocks": clk}
 

@@ -1331,11 +1331,14 @@ moe_status do_backward_fp8(const moe_layer_desc& s, const Dims& D, const Layout&
                       static_cast<const int32_t*>(poff), row_pair, row_w, row_tok);
   if (rc != MOE_OK) return rc;
 
-  int stages = 0;
+  int stages = 0, wg_stages = 0;
   for (int sg = 6; sg >= 2 && !stages; --sg)
     if (gemm8::smem_bytes(sg, E) <= (size_t)kMaxSmem) stages = sg;
-  if (!stages) return MOE_ERR_UNSUPPORTED;
+  for (int sg = 6; sg >= 2 && !wg_stages; --sg)
+    if (gemm8::smem_bytes(sg, E, true) <= (size_t)kMaxSmem) wg_stages = sg;
+  if (!stages || !wg_stages) return MOE_ERR_UNSUPPORTED;
   const size_t smem = gemm8::smem_bytes(stages, E);
+  const size_t wg_smem = gemm8::smem_bytes(wg_stages, E, true);
   const int64_t mt_rows = rs / 128;                  // m-tiles of the row space (a bound)
   auto grid_of = [&](int64_t tiles) { return (int)(tiles < sms ? tiles : sms); };
   auto base_args = [&](const int32_t* gt, int n_tiles_n, int num_kb, int b_rows_per_expert) {
@@ -1477,9 +1480,11 @@ moe_status do_backward_fp8(const moe_layer_desc& s, const Dims& D, const Layout&
   {
     CUtensorMap ta, tb;
     rc = make_tmap(&ta, ws + B.dhT, 1, rs, d, gemm8::BM);
-    if (rc == MOE_OK) rc = make_tmap(&tb, ws + B.zgT, 1, rs, I, gemm8::BN);
+    if (rc == MOE_OK) rc = make_tmap(&tb, ws + B.zgT, 1, rs, I, gemm8::WG_BN);
     if (rc != MOE_OK) return rc;
-    gemm8::Args a = base_args(gtab_wd, (I + gemm8::BN - 1) / gemm8::BN, 0, 0);
+    gemm8::Args a = base_args(gtab_wd, (I + gemm8::WG_BN - 1) / gemm8::WG_BN, 0, 0);
+    a.stages = wg_stages;
+    a.idesc = umma_idesc(0, gemm8::BM, gemm8::WG_BN);
     a.kgroup = kgroup;
     a.a_scale = reinterpret_cast<const float*>(ws + B.dhTs);
     a.a_scale_ld = d;
@@ -1493,15 +1498,17 @@ moe_status do_backward_fp8(const moe_layer_desc& s, const Dims& D, const Layout&
     rc = launch_chain("FP8 backward GEMM dW_down = dY^T Z",
                       gemm8::k_gemm_promoted<2, gemm8::EPI_BF16_OUT, true>,
                       dim3(grid_of((int64_t)E * (d / 128) * a.n_tiles_n)),
-                      dim3(gemm8::NUM_THREADS), smem, st, ta, tb, a);
+                      dim3(gemm8::NUM_THREADS), wg_smem, st, ta, tb, a);
     if (rc != MOE_OK) return rc;
   }
   {
     CUtensorMap ta, tb;
     rc = make_tmap(&ta, ws + B.dabT, 1, rs, 2 * I, gemm8::BM);
-    if (rc == MOE_OK) rc = make_tmap(&tb, ws + B.xT, 1, rs, d, gemm8::BN);
+    if (rc == MOE_OK) rc = make_tmap(&tb, ws + B.xT, 1, rs, d, gemm8::WG_BN);
     if (rc != MOE_OK) return rc;
-    gemm8::Args a = base_args(gtab_wgu, d / gemm8::BN, 0, 0);
+    gemm8::Args a = base_args(gtab_wgu, d / gemm8::WG_BN, 0, 0);
+    a.stages = wg_stages;
+    a.idesc = umma_idesc(0, gemm8::BM, gemm8::WG_BN);
     a.kgroup = kgroup;
     a.a_scale = reinterpret_cast<const float*>(ws + B.dabTs);
     a.a_scale_ld = 2 * I;
@@ -1515,7 +1522,7 @@ moe_status do_backward_fp8(const moe_layer_desc& s, const Dims& D, const Layout&
     rc = launch_chain("FP8 backward GEMM dW_gu = dAB^T X",
                       gemm8::k_gemm_promoted<2, gemm8::EPI_BF16_OUT, true>,
                       dim3(grid_of((int64_t)E * (2 * I / 128) * a.n_tiles_n)),
-                      dim3(gemm8::NUM_THREADS), smem, st, ta, tb, a);
+                      dim3(gemm8::NUM_THREADS), wg_smem, st, ta, tb, a);
     if (rc != MOE_OK) return rc;
   }
   // G6b: dW_r = dl^T X (bf16 gating GEMM), bf16 out

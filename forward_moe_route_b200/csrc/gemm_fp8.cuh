@@ -112,10 +112,17 @@ struct Args {
 };
 
 constexpr int SB_FLOATS = (NUM_EPI / 32) * 64;   // WG: per-warp column scales of a k-block
+// Weight-gradient mode (WG) tiles are 128 x 128: each epilogue warp holds 32
+// accumulator columns, which leaves it registers to spare, and stages its
+// 32 rows x 64 bytes of bf16 output in shared memory.
+constexpr int WG_BN = BN / 2;
+constexpr int XOUT_BYTES = (NUM_EPI / 32) * 32 * (WG_BN / 4) * 2;
 
-__host__ inline size_t smem_bytes(int stages, int n_groups) {
-  return 1024 + (size_t)stages * (BM * KB + BN * KB) + (size_t)(2 * stages + 6) * 8 + 16 +
-         2 * 4 * BM * sizeof(float) + SB_FLOATS * sizeof(float) + (size_t)(n_groups + 1) * 4 +
+__host__ inline size_t smem_bytes(int stages, int n_groups, bool wg = false) {
+  return 1024 + (size_t)stages * (BM * KB + (wg ? WG_BN : BN) * KB) +
+         (wg ? (size_t)XOUT_BYTES : 0) +
+         (size_t)(2 * stages + 6) * 8 + 16 + 2 * 4 * BM * sizeof(float) +
+         SB_FLOATS * sizeof(float) + (size_t)(n_groups + 1) * 4 + (wg ? (size_t)n_groups * 16 : 0) +
          64;
 }
 
@@ -154,33 +161,21 @@ __device__ __forceinline__ void promote64(uint32_t tb, float (&acc)[64], float m
 }
 
 // Promotion with a scale per accumulator column (weight-gradient mode):
-// acc[j] += (sa * sb[j]) * P[col0 + j], with sb the slice's 64 column scales
+// acc[j] += (sa * sb[j]) * P[col0 + j], with sb the slice's NC column scales
 // of this k-block in shared memory (every lane reads the same address).
-__device__ __forceinline__ void promote64_cols(uint32_t tb, float (&acc)[64], float sa,
-                                               const float* sb) {
+template <int NC>
+__device__ __forceinline__ void promote_cols(uint32_t tb, float (&acc)[NC], float sa,
+                                             const float* sb) {
   const float2 a2 = make_float2(sa, sa);
 #pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    uint32_t va[16], vb[16];
-    tmem_ld16_nowait(tb + (uint32_t)(32 * h), va);
-    tmem_ld16_nowait(tb + (uint32_t)(32 * h + 16), vb);
-    tmem_wait_ld2(va, vb);
+  for (int h = 0; h < NC / 16; ++h) {
+    float v[16];
+    tmem_ld16(tb + (uint32_t)(16 * h), v);
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      const int o = 32 * h + 2 * i;
+      const int o = 16 * h + 2 * i;
       const float2 m = __fmul2_rn(a2, *reinterpret_cast<const float2*>(sb + o));
-      const float2 r = __ffma2_rn(m, make_float2(__uint_as_float(va[2 * i]),
-                                                 __uint_as_float(va[2 * i + 1])),
-                                  make_float2(acc[o], acc[o + 1]));
-      acc[o] = r.x;
-      acc[o + 1] = r.y;
-    }
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int o = 32 * h + 16 + 2 * i;
-      const float2 m = __fmul2_rn(a2, *reinterpret_cast<const float2*>(sb + o));
-      const float2 r = __ffma2_rn(m, make_float2(__uint_as_float(vb[2 * i]),
-                                                 __uint_as_float(vb[2 * i + 1])),
+      const float2 r = __ffma2_rn(m, make_float2(v[2 * i], v[2 * i + 1]),
                                   make_float2(acc[o], acc[o + 1]));
       acc[o] = r.x;
       acc[o + 1] = r.y;
@@ -329,11 +324,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
+  constexpr int TBN = WG ? WG_BN : BN;     // accumulator columns of a tile
+  constexpr int WC = TBN / 4;              // columns of one epilogue warp
   constexpr uint32_t a_bytes = BM * KB;
-  constexpr uint32_t b_bytes = BN * KB;
+  constexpr uint32_t b_bytes = TBN * KB;
   constexpr uint32_t stage_bytes = a_bytes + b_bytes;
   const int S = a.stages;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)S * stage_bytes);
+  uint8_t* xout = smem + (size_t)S * stage_bytes;        // WG: 16 warps x 32 rows x 128 B
+  uint64_t* full = reinterpret_cast<uint64_t*>(xout + (WG ? XOUT_BYTES : 0));
   uint64_t* empty = full + S;
   uint64_t* pfull = empty + S;
   uint64_t* pempty = pfull + 2;
@@ -344,6 +342,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   float* amax_buf = reinterpret_cast<float*>(tmem_slot + 4);   // [2][4][128]
   float* sb_buf = amax_buf + 2 * 4 * BM;                        // WG: [16 warps][64]
   int* s_prefix = reinterpret_cast<int*>(sb_buf + SB_FLOATS);
+  int* s_kgroup = s_prefix + a.gt.count() + 1;                  // WG: the groups' K ranges
 
   const int warp = warp_id(), lane = lane_id();
   const int n_groups = a.gt.count();
@@ -352,6 +351,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       a.zero_ptr[i] = 0;
   }
   for (int i = threadIdx.x; i <= n_groups; i += NUM_THREADS) s_prefix[i] = a.gt.prefix(i);
+  if (WG)
+    for (int i = threadIdx.x; i < n_groups; i += NUM_THREADS) {
+      s_kgroup[4 * i] = a.kgroup[2 * i];
+      s_kgroup[4 * i + 1] = a.kgroup[2 * i + 1];
+      s_kgroup[4 * i + 2] = a.gt.c_row(i);
+      s_kgroup[4 * i + 3] = a.gt.rows(i);
+    }
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(&full[s], 1);
@@ -394,8 +400,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const int lm = mt - s_prefix[g];
           const int arow = (a.a_from_crow ? a.gt.c_row(g) : a.gt.a_row(g)) + lm * BM;
           const int ebase = a.gt.expert(g) * a.b_rows_per_expert;
-          const int k0 = WG ? a.kgroup[2 * g] : 0;
-          const int nkb = WG ? a.kgroup[2 * g + 1] : a.num_kb;
+          const int k0 = WG ? s_kgroup[4 * g] : 0;
+          const int nkb = WG ? s_kgroup[4 * g + 1] : a.num_kb;
           for (int kb = 0; kb < nkb; ++kb, ++it) {
             const int s = it % S;
             const uint32_t ph = (uint32_t)(it / S) & 1u;
@@ -413,7 +419,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 tma_load_2d(&tmB, &full[s], sb + (size_t)(2 * c + 1) * 32 * KB, kx, ur + 32 * c);
               }
             } else {
-              tma_load_2d(&tmB, &full[s], sb, kx, ebase + nt * BN);
+              tma_load_2d(&tmB, &full[s], sb, kx, ebase + nt * TBN);
             }
           }
         }
@@ -433,7 +439,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           int nkb = a.num_kb;
           if (WG) {
             const int g = gemm::find_group(s_prefix, n_groups, tile / a.n_tiles_n);
-            nkb = a.kgroup[2 * g + 1];
+            nkb = s_kgroup[4 * g + 1];
           }
           for (int kb = 0; kb < nkb; ++kb, ++it, ++pu) {
             const int s = it % S;
@@ -446,7 +452,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             const uint32_t sa = smem_u32(smem + (size_t)s * stage_bytes);
             const uint64_t ad = umma_desc_sw128(sa);
             const uint64_t bd = umma_desc_sw128(sa + a_bytes);
-            const uint32_t d_tmem = tmem_base + (uint32_t)(p * BN);
+            const uint32_t d_tmem = tmem_base + (uint32_t)(p * TBN);
   #pragma unroll
             for (int k = 0; k < KB / 32; ++k)
               umma<KIND>(d_tmem, ad + (uint64_t)(k * 2), bd + (uint64_t)(k * 2), a.idesc,
@@ -467,12 +473,74 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // ------------------------------------------------------------------ promotion + epilogue
     const int ew = warp - EPI_WARP0;
     const int q = warp & 3;
-    const int cs = ew >> 2;                 // 64-column slice 0..3
+    const int cs = ew >> 2;                 // column slice 0..3 of WC columns
     const int r = q * 32 + lane;
-    const int col0 = cs * 64;
+    const int col0 = cs * WC;
     const int kb_blocks_b = a.b_rows_per_expert / 128;
     int pu = 0, tcount = 0;
     bool ok = true;
+    if constexpr (WG) {
+      // Weight gradients: short K ranges (an expert's rows), 128 x 128 tiles;
+      // group data comes from shared memory.
+      float* sbw = sb_buf + ew * 64;
+      for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x, ++tcount) {
+        const int mt = tile / a.n_tiles_n, nt = tile - mt * a.n_tiles_n;
+        const int g = gemm::find_group(s_prefix, n_groups, mt);
+        const int lm = mt - s_prefix[g];
+        const int* kg = s_kgroup + 4 * g;           // k0, k-blocks, c_row, rows
+        const int nkb = kg[1];
+        const int ncol = nt * TBN + col0;
+        const int arow = lm * BM + r;
+        float acc[WC];
+#pragma unroll
+        for (int i = 0; i < WC; ++i) acc[i] = 0.f;
+        for (int kb = 0; kb < nkb; ++kb, ++pu) {
+          // this k-block's row scale and the slice's column scales, loaded
+          // while the tensor cores compute the partial
+          const size_t kr = (size_t)(kg[0] / 128 + kb);
+          const float sa_k = arow < a.a_rows ? a.a_scale[kr * a.a_scale_ld + arow] : 0.f;
+          sbw[lane] = ncol + lane < a.b_rows ? a.b_scale[kr * a.b_scale_ld + ncol + lane] : 0.f;
+          __syncwarp();
+          const int p = pu & 1;
+          if (!mbar_wait(&pfull[p], (uint32_t)(pu >> 1) & 1u, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          promote_cols<WC>(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(p * TBN + col0),
+                           acc, sa_k, sbw);
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&pempty[p]);
+        }
+        if (!ok) break;
+        if constexpr (EPI == EPI_BF16_OUT) {
+          // stage the warp's 32 rows x 64 bytes (16-byte chunks XOR-swizzled
+          // by row pair, no bank conflicts either way) and write them back 8
+          // rows per instruction, 4 lanes a row
+          static_assert(WC == 32, "staging layout assumes 32 columns a warp");
+          uint8_t* xw = xout + (size_t)ew * 32 * 64;
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+            *reinterpret_cast<uint4*>(xw + lane * 64 + ((c ^ ((lane >> 1) & 3)) << 4)) =
+                make_uint4(gemm::pack_bf16x2(acc[8 * c], acc[8 * c + 1]),
+                           gemm::pack_bf16x2(acc[8 * c + 2], acc[8 * c + 3]),
+                           gemm::pack_bf16x2(acc[8 * c + 4], acc[8 * c + 5]),
+                           gemm::pack_bf16x2(acc[8 * c + 6], acc[8 * c + 7]));
+          __syncwarp();
+          const int wrow0 = lm * BM + q * 32;       // the warp's first row in the group
+          if (ncol + WC <= a.out_cols) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const int rr = 8 * k + (lane >> 2), c = lane & 3;
+              const uint4 v =
+                  *reinterpret_cast<const uint4*>(xw + rr * 64 + ((c ^ ((rr >> 1) & 3)) << 4));
+              if (wrow0 + rr < kg[3])
+                *reinterpret_cast<uint4*>(a.out_bf16 + (size_t)(kg[2] + wrow0 + rr) * a.out_ld +
+                                          ncol + c * 8) = v;
+            }
+          }
+          __syncwarp();
+        }
+      }
+    } else
     for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x, ++tcount) {
       const int mt = tile / a.n_tiles_n, nt = tile - mt * a.n_tiles_n;
       const int g = gemm::find_group(s_prefix, n_groups, mt);
@@ -490,47 +558,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         sa_row = arow < a.a_rows ? a.a_scale + (size_t)arow * a.num_kb : nullptr;
         sb0 = a.b_scale + (eb + nt) * a.num_kb;                          // gate block
         sb1 = a.b_scale + (eb + a.b_up_off / 128 + nt) * a.num_kb;       // up block
-      } else if (!WG) {
+      } else {
         sa_row = arow < a.a_rows ? a.a_scale + (size_t)arow * a.num_kb : nullptr;
         // a slice past the expert's last B row block (N not a multiple of 256)
         // is never stored; its scale read stays inside the expert's blocks
         sb0 = a.b_scale + (eb + min(2 * nt + cs / 2, kb_blocks_b - 1)) * a.num_kb;
         sb1 = sb0;
       }
-      float acc[64];
+      float acc[WC];
 #pragma unroll
-      for (int i = 0; i < 64; ++i) acc[i] = 0.f;
+      for (int i = 0; i < WC; ++i) acc[i] = 0.f;
       const bool scaled = EPI != EPI_F32_STORE;
-      // weight-gradient mode: this group's K range, the row's and the slice's
-      // column scales of the next k-block (prefetched one k-block ahead)
-      const int nkb = WG ? a.kgroup[2 * g + 1] : a.num_kb;
-      const int kb0 = WG ? a.kgroup[2 * g] / 128 : 0;
-      const int ncol = nt * BN + col0;
-      float* sbw = sb_buf + ew * 64;
-      float wsa = 0.f, wsb0 = 0.f, wsb1 = 0.f;
-      if (WG && nkb > 0) {
-        wsa = arow < a.a_rows ? a.a_scale[(size_t)kb0 * a.a_scale_ld + arow] : 0.f;
-        wsb0 = ncol + lane < a.b_rows ? a.b_scale[(size_t)kb0 * a.b_scale_ld + ncol + lane] : 0.f;
-        wsb1 = ncol + 32 + lane < a.b_rows
-                   ? a.b_scale[(size_t)kb0 * a.b_scale_ld + ncol + 32 + lane] : 0.f;
-      }
-      float na = (scaled && !WG) ? (sa_row ? sa_row[0] : 0.f) : 1.f;
-      float nb0 = (scaled && !WG) ? sb0[0] : 1.f, nb1 = (scaled && !WG) ? sb1[0] : 1.f;
+      const int nkb = a.num_kb;
+      const int ncol = nt * TBN + col0;
+      float na = scaled ? (sa_row ? sa_row[0] : 0.f) : 1.f;
+      float nb0 = scaled ? sb0[0] : 1.f, nb1 = scaled ? sb1[0] : 1.f;
       for (int kb = 0; kb < nkb; ++kb, ++pu) {
         const float m0 = na * nb0, m1 = na * nb1;
-        const float sa_k = wsa;
-        if (WG) {
-          sbw[lane] = wsb0;
-          sbw[32 + lane] = wsb1;
-          __syncwarp();
-          if (kb + 1 < nkb) {
-            const size_t kr = (size_t)(kb0 + kb + 1);
-            wsa = arow < a.a_rows ? a.a_scale[kr * a.a_scale_ld + arow] : 0.f;
-            wsb0 = ncol + lane < a.b_rows ? a.b_scale[kr * a.b_scale_ld + ncol + lane] : 0.f;
-            wsb1 = ncol + 32 + lane < a.b_rows ? a.b_scale[kr * a.b_scale_ld + ncol + 32 + lane]
-                                               : 0.f;
-          }
-        } else if (scaled && kb + 1 < nkb) {
+        if (scaled && kb + 1 < nkb) {
           na = sa_row ? sa_row[kb + 1] : 0.f;
           nb0 = sb0[kb + 1];
           nb1 = sb1[kb + 1];
@@ -538,19 +583,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int p = pu & 1;
         if (!mbar_wait(&pfull[p], (uint32_t)(pu >> 1) & 1u, abort_flag)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(p * BN + col0);
+        const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(p * TBN + col0);
         // the router's unscaled promotion is a paired FMA with multiplier 1
-        if (WG) promote64_cols(tb, acc, sa_k, sbw);
-        else promote64(tb, acc, m0, m1);
+        promote64(tb, acc, m0, m1);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&pempty[p]);
       }
       if (!ok) break;
-      if (EPI == EPI_F32_STORE) {
+      if constexpr (EPI == EPI_F32_STORE) {
         if (valid) {
-          float* orow = a.out + (size_t)(a.gt.c_row(g) + grow) * a.out_ld + nt * BN + col0;
-          const int c0 = nt * BN + col0;
+          float* orow = a.out + (size_t)(a.gt.c_row(g) + grow) * a.out_ld + nt * TBN + col0;
+          const int c0 = nt * TBN + col0;
           if (c0 + 64 <= a.out_cols) {
 #pragma unroll
             for (int j = 0; j < 16; ++j)
@@ -562,23 +606,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               if (c0 + j < a.out_cols) orow[j] = acc[j];
           }
         }
-      } else if (EPI == EPI_SWIGLU_Q) {
+      } else if constexpr (EPI == EPI_SWIGLU_Q) {
         if (!epi_swiglu_q(acc, a, amax_buf, xbar, tcount, cs, r, valid,
                           (size_t)(a.gt.c_row(g) + grow), nt, abort_flag)) {
           ok = false;
           break;
         }
-      } else if (EPI == EPI_BF16_OUT) {
+      } else if constexpr (EPI == EPI_BF16_OUT) {
         if (valid && ncol + 64 <= a.out_cols)
           store_bf16x64(a.out_bf16 + (size_t)(a.gt.c_row(g) + grow) * a.out_ld + ncol, acc);
-      } else if (EPI == EPI_SWIGLU_BWD) {
+      } else if constexpr (EPI == EPI_SWIGLU_BWD) {
         if (ncol + 64 <= a.inter) {
           const long long crow = (long long)a.gt.c_row(g) + grow;
           const float gw = (a.gt.aux(g) < 0 && valid) ? a.row_w[crow] : 1.0f;
           epi_swiglu_bwd(acc, a, crow, ncol, gw, valid);
         }
       } else {
-        if (valid) epi_scatter(acc, a, g, grow, nt * BN + col0);
+        if (valid) epi_scatter(acc, a, g, grow, nt * TBN + col0);
       }
     }
   }

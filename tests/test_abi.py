@@ -256,3 +256,32 @@ def test_saved_activation_entry_points_reject_bad_arguments():
     short = torch.zeros(T * K, 2 * I, dtype=torch.bfloat16)     # the shared rows missing
     with pytest.raises(moe.MoeError, match="ab_saved holds"):
         moe.moe_forward_save(bf, x, None, None, None, None, None, x, None, None, short, None)
+
+
+def test_fp8_backward_entry_point_rejects_bad_arguments():
+    """moe_backward_fp8: E4M3 layers only, d a multiple of 256, every pointer
+    present and aligned, checked before any CUDA call."""
+    L = moe.lib()
+    f8 = v3(T=64, dtype="e4m3")
+    assert moe.moe_backward_fp8_workspace_size(f8) > 0
+    assert moe.moe_backward_fp8_workspace_size(v3(T=64)) == 0
+    assert moe.moe_backward_fp8_launch_count(f8) == 22
+    assert moe.moe_backward_fp8_launch_count(v3(T=0, dtype="e4m3")) == 0
+    ptrs = [16] * 16          # x, w_router, bias, 8 weight pointers, dh, dx, 3 gradients
+    ptrs[2] = None            # bias
+    assert L.moe_backward_fp8(ctypes.byref(v3(T=64)), *ptrs, 16, 1 << 40,
+                              None) == moe.ERR_UNSUPPORTED
+    assert L.moe_backward_fp8(ctypes.byref(v3(T=64, d=7168 + 128, dtype="e4m3")), *ptrs, 16,
+                              1 << 40, None) == moe.ERR_UNSUPPORTED
+    for i in (0, 3, 5, 11, 15):           # a missing tensor or scale
+        bad = list(ptrs)
+        bad[i] = None
+        assert L.moe_backward_fp8(ctypes.byref(f8), *bad, 16, 1 << 40,
+                                  None) == moe.ERR_INVALID_ARG
+    bad = list(ptrs)
+    bad[5] = 24                           # a misaligned transposed weight (w_gu_t)
+    assert L.moe_backward_fp8(ctypes.byref(f8), *bad, 16, 1 << 40, None) == moe.ERR_INVALID_ARG
+    bad = list(ptrs)
+    bad[4] = 18                           # a scale (w_gu_scale) not 4-byte aligned
+    assert L.moe_backward_fp8(ctypes.byref(f8), *bad, 16, 1 << 40, None) == moe.ERR_INVALID_ARG
+    assert L.moe_backward_fp8(ctypes.byref(f8), *ptrs, 16, 1024, None) == moe.ERR_WORKSPACE

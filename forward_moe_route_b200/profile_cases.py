@@ -18,6 +18,8 @@ whole run ends in minutes:
             addresses): peer dispatch, expert GEMMs with per-group output
             addresses, the FP8 dispatch and row quantisation
   backward_bf16  the backward case with bf16 weight gradients
+  backward_saved the backward case reading the pre-activations the forward kept
+  backward_fp8   the backward case's shape as an E4M3 layer, FP8 GEMMs
 Inputs come from the seeded synthetic generator (synth/).
 """
 import argparse
@@ -207,8 +209,65 @@ def case_backward_bf16():
     torch.cuda.synchronize()
 
 
+def _backward_case(dtype):
+    import synth
+    cfg = dataclasses.replace(
+        recipes.small_variant(C["v3_fp8" if dtype == "e4m3" else "v3_bf16"], T=2048, d=7168,
+                              inter=2048, n_routed=8),
+        n_group=4, topk_group=2, top_k=4)
+    inp = recipes.device_inputs(cfg)
+    dh32 = torch.empty(cfg.T, cfg.d, dtype=torch.float32, device="cuda")
+    synth.dev_fill_normal(dh32, 1.0, cfg.seed, 6)
+    return cfg, inp, dh32.to(torch.bfloat16)
+
+
+def case_backward_saved():
+    cfg, inp, dh = _backward_case("bf16")
+    desc = moe.desc_from_config(cfg)
+    E, I, d, N = cfg.n_experts, cfg.inter, cfg.d, cfg.n_routed
+    ab = torch.empty(moe.moe_saved_ab_bytes(desc) // 2, dtype=torch.bfloat16, device="cuda")
+    h = torch.empty_like(dh)
+    moe.moe_forward_save(desc, inp["x"], None, inp["w_r"], inp["bias"], inp["w_gu"],
+                         inp["w_down"], h, None, None, ab, moe.workspace(desc))
+    ws = moe.backward_workspace(desc)
+    dx = torch.empty_like(dh)
+    dwr = torch.empty(N, d, dtype=torch.float32, device="cuda")
+    dwgu = torch.empty(E, 2 * I, d, dtype=torch.float32, device="cuda")
+    dwd = torch.empty(E, d, I, dtype=torch.float32, device="cuda")
+    for _ in range(2):
+        moe.moe_backward_saved(desc, inp["x"], inp["w_r"], inp["bias"], inp["w_gu"],
+                               inp["w_down"], dh, ab, dx, dwr, dwgu, dwd, ws)
+    torch.cuda.synchronize()
+
+
+def case_backward_fp8():
+    cfg, inp, dh = _backward_case("e4m3")
+    desc = moe.desc_from_config(cfg)
+    E, I, d, N = cfg.n_experts, cfg.inter, cfg.d, cfg.n_routed
+
+    def quant(w, r, c):
+        q = torch.empty(E, r, c, dtype=torch.uint8, device="cuda")
+        sc = torch.empty(E, r // 128, c // 128, dtype=torch.float32, device="cuda")
+        moe.moe_quantize_fp8_blockwise(w.contiguous(), r, c, E, q, sc)
+        return q, sc
+
+    W = (quant(inp["w_gu"], 2 * I, d) + quant(inp["w_gu"].transpose(1, 2), d, 2 * I)
+         + quant(inp["w_down"], d, I) + quant(inp["w_down"].transpose(1, 2), I, d))
+    ws = moe.backward_fp8_workspace(desc)
+    bf = dict(dtype=torch.bfloat16, device="cuda")
+    dx = torch.empty_like(dh)
+    dwr = torch.empty(N, d, **bf)
+    dwgu = torch.empty(E, 2 * I, d, **bf)
+    dwd = torch.empty(E, d, I, **bf)
+    for _ in range(2):
+        moe.moe_backward_fp8(desc, inp["x"], inp["w_r"], inp["bias"], *W, dh, dx, dwr, dwgu,
+                             dwd, ws)
+    torch.cuda.synchronize()
+
+
 CASES = {"route": case_route, "v3": case_v3, "fp8": case_fp8, "tiny": case_tiny,
-         "backward": case_backward, "ep": case_ep, "backward_bf16": case_backward_bf16}
+         "backward": case_backward, "ep": case_ep, "backward_bf16": case_backward_bf16,
+         "backward_saved": case_backward_saved, "backward_fp8": case_backward_fp8}
 
 
 def main():

@@ -34,7 +34,16 @@
 //     row), exchanges the per-slice amax through shared memory, and writes E4M3
 //     codes plus the fp32 tile scale.
 //   GEMM2 (SCATTER): 256 output columns, times the gate weight, bf16 rows
-//     scattered to the token-major slots.
+//     scattered to the token-major slots (weight 1 without topk_w: the
+//     backward's du pieces).
+//   Backward (same pipeline): BF16_OUT stores the tile as bf16 rows (the
+//     recomputed a | b); SWIGLU_BWD turns dz' = dY W_down into g z, [da | db]
+//     and per-64-feature partials of <dz', z>.
+//   Weight-gradient mode (template WG, dW = sum over an expert's rows): each
+//     group contracts over its own K range, both operands carry a scale per
+//     row and k-block, so the promotion multiplies every accumulator column
+//     by its own scale; tiles are 128 x 128 (32 columns a warp) and each warp
+//     writes its rows through a shared-memory staging buffer.
 #pragma once
 
 #include "common.cuh"

@@ -549,89 +549,90 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           __syncwarp();
         }
       }
-    } else
-    for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x, ++tcount) {
-      const int mt = tile / a.n_tiles_n, nt = tile - mt * a.n_tiles_n;
-      const int g = gemm::find_group(s_prefix, n_groups, mt);
-      const int lm = mt - s_prefix[g];
-      const int grow = lm * BM + r;
-      const bool valid = grow < a.gt.rows(g);
-      const int arow = (a.a_from_crow ? a.gt.c_row(g) : a.gt.a_row(g)) + grow;
-      const size_t eb = (size_t)a.gt.expert(g) * kb_blocks_b;
-      const float* sa_row = nullptr;
-      const float* sb0 = nullptr;
-      const float* sb1 = nullptr;
-      if (EPI == EPI_F32_STORE) {
-        // unscaled: plain fp32 accumulation of the k-block partials
-      } else if (EPI == EPI_SWIGLU_Q) {
-        sa_row = arow < a.a_rows ? a.a_scale + (size_t)arow * a.num_kb : nullptr;
-        sb0 = a.b_scale + (eb + nt) * a.num_kb;                          // gate block
-        sb1 = a.b_scale + (eb + a.b_up_off / 128 + nt) * a.num_kb;       // up block
-      } else {
-        sa_row = arow < a.a_rows ? a.a_scale + (size_t)arow * a.num_kb : nullptr;
-        // a slice past the expert's last B row block (N not a multiple of 256)
-        // is never stored; its scale read stays inside the expert's blocks
-        sb0 = a.b_scale + (eb + min(2 * nt + cs / 2, kb_blocks_b - 1)) * a.num_kb;
-        sb1 = sb0;
-      }
-      float acc[WC];
-#pragma unroll
-      for (int i = 0; i < WC; ++i) acc[i] = 0.f;
-      const bool scaled = EPI != EPI_F32_STORE;
-      const int nkb = a.num_kb;
-      const int ncol = nt * TBN + col0;
-      float na = scaled ? (sa_row ? sa_row[0] : 0.f) : 1.f;
-      float nb0 = scaled ? sb0[0] : 1.f, nb1 = scaled ? sb1[0] : 1.f;
-      for (int kb = 0; kb < nkb; ++kb, ++pu) {
-        const float m0 = na * nb0, m1 = na * nb1;
-        if (scaled && kb + 1 < nkb) {
-          na = sa_row ? sa_row[kb + 1] : 0.f;
-          nb0 = sb0[kb + 1];
-          nb1 = sb1[kb + 1];
+    } else {
+      for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x, ++tcount) {
+        const int mt = tile / a.n_tiles_n, nt = tile - mt * a.n_tiles_n;
+        const int g = gemm::find_group(s_prefix, n_groups, mt);
+        const int lm = mt - s_prefix[g];
+        const int grow = lm * BM + r;
+        const bool valid = grow < a.gt.rows(g);
+        const int arow = (a.a_from_crow ? a.gt.c_row(g) : a.gt.a_row(g)) + grow;
+        const size_t eb = (size_t)a.gt.expert(g) * kb_blocks_b;
+        const float* sa_row = nullptr;
+        const float* sb0 = nullptr;
+        const float* sb1 = nullptr;
+        if (EPI == EPI_F32_STORE) {
+          // unscaled: plain fp32 accumulation of the k-block partials
+        } else if (EPI == EPI_SWIGLU_Q) {
+          sa_row = arow < a.a_rows ? a.a_scale + (size_t)arow * a.num_kb : nullptr;
+          sb0 = a.b_scale + (eb + nt) * a.num_kb;                          // gate block
+          sb1 = a.b_scale + (eb + a.b_up_off / 128 + nt) * a.num_kb;       // up block
+        } else {
+          sa_row = arow < a.a_rows ? a.a_scale + (size_t)arow * a.num_kb : nullptr;
+          // a slice past the expert's last B row block (N not a multiple of 256)
+          // is never stored; its scale read stays inside the expert's blocks
+          sb0 = a.b_scale + (eb + min(2 * nt + cs / 2, kb_blocks_b - 1)) * a.num_kb;
+          sb1 = sb0;
         }
-        const int p = pu & 1;
-        if (!mbar_wait(&pfull[p], (uint32_t)(pu >> 1) & 1u, abort_flag)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(p * TBN + col0);
-        // the router's unscaled promotion is a paired FMA with multiplier 1
-        promote64(tb, acc, m0, m1);
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&pempty[p]);
-      }
-      if (!ok) break;
-      if constexpr (EPI == EPI_F32_STORE) {
-        if (valid) {
-          float* orow = a.out + (size_t)(a.gt.c_row(g) + grow) * a.out_ld + nt * TBN + col0;
-          const int c0 = nt * TBN + col0;
-          if (c0 + 64 <= a.out_cols) {
-#pragma unroll
-            for (int j = 0; j < 16; ++j)
-              reinterpret_cast<float4*>(orow)[j] =
-                  make_float4(acc[4 * j], acc[4 * j + 1], acc[4 * j + 2], acc[4 * j + 3]);
-          } else {
-#pragma unroll
-            for (int j = 0; j < 64; ++j)
-              if (c0 + j < a.out_cols) orow[j] = acc[j];
+        float acc[WC];
+  #pragma unroll
+        for (int i = 0; i < WC; ++i) acc[i] = 0.f;
+        const bool scaled = EPI != EPI_F32_STORE;
+        const int nkb = a.num_kb;
+        const int ncol = nt * TBN + col0;
+        float na = scaled ? (sa_row ? sa_row[0] : 0.f) : 1.f;
+        float nb0 = scaled ? sb0[0] : 1.f, nb1 = scaled ? sb1[0] : 1.f;
+        for (int kb = 0; kb < nkb; ++kb, ++pu) {
+          const float m0 = na * nb0, m1 = na * nb1;
+          if (scaled && kb + 1 < nkb) {
+            na = sa_row ? sa_row[kb + 1] : 0.f;
+            nb0 = sb0[kb + 1];
+            nb1 = sb1[kb + 1];
           }
+          const int p = pu & 1;
+          if (!mbar_wait(&pfull[p], (uint32_t)(pu >> 1) & 1u, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(p * TBN + col0);
+          // the router's unscaled promotion is a paired FMA with multiplier 1
+          promote64(tb, acc, m0, m1);
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&pempty[p]);
         }
-      } else if constexpr (EPI == EPI_SWIGLU_Q) {
-        if (!epi_swiglu_q(acc, a, amax_buf, xbar, tcount, cs, r, valid,
-                          (size_t)(a.gt.c_row(g) + grow), nt, abort_flag)) {
-          ok = false;
-          break;
+        if (!ok) break;
+        if constexpr (EPI == EPI_F32_STORE) {
+          if (valid) {
+            float* orow = a.out + (size_t)(a.gt.c_row(g) + grow) * a.out_ld + nt * TBN + col0;
+            const int c0 = nt * TBN + col0;
+            if (c0 + 64 <= a.out_cols) {
+  #pragma unroll
+              for (int j = 0; j < 16; ++j)
+                reinterpret_cast<float4*>(orow)[j] =
+                    make_float4(acc[4 * j], acc[4 * j + 1], acc[4 * j + 2], acc[4 * j + 3]);
+            } else {
+  #pragma unroll
+              for (int j = 0; j < 64; ++j)
+                if (c0 + j < a.out_cols) orow[j] = acc[j];
+            }
+          }
+        } else if constexpr (EPI == EPI_SWIGLU_Q) {
+          if (!epi_swiglu_q(acc, a, amax_buf, xbar, tcount, cs, r, valid,
+                            (size_t)(a.gt.c_row(g) + grow), nt, abort_flag)) {
+            ok = false;
+            break;
+          }
+        } else if constexpr (EPI == EPI_BF16_OUT) {
+          if (valid && ncol + 64 <= a.out_cols)
+            store_bf16x64(a.out_bf16 + (size_t)(a.gt.c_row(g) + grow) * a.out_ld + ncol, acc);
+        } else if constexpr (EPI == EPI_SWIGLU_BWD) {
+          if (ncol + 64 <= a.inter) {
+            const long long crow = (long long)a.gt.c_row(g) + grow;
+            const float gw = (a.gt.aux(g) < 0 && valid) ? a.row_w[crow] : 1.0f;
+            epi_swiglu_bwd(acc, a, crow, ncol, gw, valid);
+          }
+        } else {
+          if (valid) epi_scatter(acc, a, g, grow, nt * TBN + col0);
         }
-      } else if constexpr (EPI == EPI_BF16_OUT) {
-        if (valid && ncol + 64 <= a.out_cols)
-          store_bf16x64(a.out_bf16 + (size_t)(a.gt.c_row(g) + grow) * a.out_ld + ncol, acc);
-      } else if constexpr (EPI == EPI_SWIGLU_BWD) {
-        if (ncol + 64 <= a.inter) {
-          const long long crow = (long long)a.gt.c_row(g) + grow;
-          const float gw = (a.gt.aux(g) < 0 && valid) ? a.row_w[crow] : 1.0f;
-          epi_swiglu_bwd(acc, a, crow, ncol, gw, valid);
-        }
-      } else {
-        if (valid) epi_scatter(acc, a, g, grow, nt * TBN + col0);
       }
     }
   }

@@ -573,14 +573,7 @@ def run_backward(args, cfg):
     if fp8:
         # E4M3 codes and 128x128 block scales of the weights and of their
         # transposes (offline, like the forward's weight quantisation)
-        def quant(w, rows, cols):
-            q = torch.empty(E, rows, cols, dtype=torch.uint8, device="cuda")
-            sc = torch.empty(E, rows // 128, cols // 128, dtype=torch.float32, device="cuda")
-            moe.moe_quantize_fp8_blockwise(w.contiguous(), rows, cols, E, q, sc)
-            return q, sc
-
-        W8 = (quant(inp["w_gu"], 2 * I, d) + quant(inp["w_gu"].transpose(1, 2), d, 2 * I)
-              + quant(inp["w_down"], d, I) + quant(inp["w_down"].transpose(1, 2), I, d))
+        W8 = moe.fp8_backward_weights(inp["w_gu"], inp["w_down"])
         del inp["w_gu"], inp["w_down"]
         torch.cuda.empty_cache()
 

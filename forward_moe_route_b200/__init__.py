@@ -76,6 +76,8 @@ _SIGS = {
     "moe_bias_update": (ctypes.c_int, [_D, _P, _P, ctypes.c_float, _P]),
     "moe_quantize_fp8_blockwise": (ctypes.c_int, [_P, ctypes.c_int32, ctypes.c_int32,
                                                   ctypes.c_int32, _P, _P, _P]),
+    "moe_quantize_fp8_blockwise_t": (ctypes.c_int, [_P, ctypes.c_int32, ctypes.c_int32,
+                                                    ctypes.c_int32, _P, _P, _P]),
     "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "moe_last_device_status": (ctypes.c_int, [_P]),
     "moe_forward_launch_count": (ctypes.c_int32, [_D]),
@@ -322,6 +324,32 @@ def moe_quantize_fp8_blockwise(w_bf16, rows: int, cols: int, batch: int, w_e4m3,
     _check(_lib.moe_quantize_fp8_blockwise(_ptr(w_bf16), rows, cols, batch, _ptr(w_e4m3),
                                            _ptr(scale), _stream(stream)),
            "moe_quantize_fp8_blockwise")
+
+
+def moe_quantize_fp8_blockwise_t(w_bf16, rows: int, cols: int, batch: int, w_e4m3_t, scale_t,
+                                 stream=None) -> None:
+    _check(_lib.moe_quantize_fp8_blockwise_t(_ptr(w_bf16), rows, cols, batch, _ptr(w_e4m3_t),
+                                             _ptr(scale_t), _stream(stream)),
+           "moe_quantize_fp8_blockwise_t")
+
+
+def fp8_backward_weights(w_gu, w_down, stream=None):
+    """E4M3 codes and 128x128 block scales of a layer's bf16 expert weights
+    w_gu [E, 2I, d] and w_down [E, d, I] and of their transposes, in the
+    argument order of moe_backward_fp8: (w_gu, w_gu_scale, w_gu_t,
+    w_gu_t_scale, w_down, w_down_scale, w_down_t, w_down_t_scale)."""
+    import torch
+    E, two_i, d = w_gu.shape
+    I = w_down.shape[2]
+    out = []
+    for w, rows, cols in ((w_gu, two_i, d), (w_down, d, I)):
+        for quant, (r, c) in ((moe_quantize_fp8_blockwise, (rows, cols)),
+                              (moe_quantize_fp8_blockwise_t, (cols, rows))):
+            q = torch.empty(E, r, c, dtype=torch.uint8, device=w.device)
+            sc = torch.empty(E, r // 128, c // 128, dtype=torch.float32, device=w.device)
+            quant(w, rows, cols, E, q, sc, stream)
+            out += [q, sc]
+    return tuple(out)
 
 
 def moe_last_device_status(stream=None) -> int:

@@ -1830,10 +1830,23 @@ moe_status moe_quantize_fp8_blockwise(const void* w_bf16, int32_t rows, int32_t 
     return MOE_ERR_INVALID_ARG;
   const int64_t blocks = (int64_t)batch * (rows / 128) * (cols / 128);
   if (blocks >= ((int64_t)1 << 31)) return MOE_ERR_INVALID_ARG;
-  perm::k_quant_w<<<(unsigned)blocks, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(w_bf16),
-                                                         rows, cols,
-                                                         static_cast<uint8_t*>(w_e4m3), scale);
+  perm::k_quant_w<false><<<(unsigned)blocks, 256, 0, stream>>>(
+      static_cast<const __nv_bfloat16*>(w_bf16), rows, cols, static_cast<uint8_t*>(w_e4m3), scale);
   return launched("k_quant_w");
+}
+
+moe_status moe_quantize_fp8_blockwise_t(const void* w_bf16, int32_t rows, int32_t cols,
+                                        int32_t batch, void* w_e4m3_t, float* scale_t,
+                                        cudaStream_t stream) {
+  if (rows <= 0 || cols <= 0 || batch <= 0 || rows % 128 || cols % 128) return MOE_ERR_INVALID_ARG;
+  if (!w_bf16 || !w_e4m3_t || !scale_t || !aligned16(w_bf16) || !aligned16(w_e4m3_t))
+    return MOE_ERR_INVALID_ARG;
+  const int64_t blocks = (int64_t)batch * (rows / 128) * (cols / 128);
+  if (blocks >= ((int64_t)1 << 31)) return MOE_ERR_INVALID_ARG;
+  perm::k_quant_w<true><<<(unsigned)blocks, 256, 0, stream>>>(
+      static_cast<const __nv_bfloat16*>(w_bf16), rows, cols, static_cast<uint8_t*>(w_e4m3_t),
+      scale_t);
+  return launched("k_quant_w (transposed)");
 }
 
 const char* moe_status_string(moe_status status) {

@@ -701,10 +701,15 @@ __global__ void __launch_bounds__(256) k_combine_rows(const void* __restrict__ x
 
 // 128x128 block quantisation of bf16 weights to E4M3 (same rule as the
 // activation tiles).  One block of 256 threads per weight block.
+// TRANSPOSE: the codes and scales of the transposed matrix, [cols, rows] and
+// [cols / 128, rows / 128] (a block's amax does not depend on its
+// orientation, so these are the transposed matrix's own codes and scales).
+template <bool TRANSPOSE>
 __global__ void __launch_bounds__(256) k_quant_w(const __nv_bfloat16* __restrict__ w, int rows,
                                                  int cols, uint8_t* __restrict__ q,
                                                  float* __restrict__ scale) {
   __shared__ float red[8];
+  __shared__ __align__(16) uint8_t tile[TRANSPOSE ? 128 : 1][TRANSPOSE ? 128 + 16 : 1];
   const int bc = cols / 128, br = rows / 128;
   const int b = blockIdx.x;  // over batch * br * bc
   const int mat = b / (br * bc), rem = b - mat * br * bc;
@@ -736,7 +741,7 @@ __global__ void __launch_bounds__(256) k_quant_w(const __nv_bfloat16* __restrict
   for (int i = 1; i < 8; ++i) amax = fmaxf(amax, red[i]);
   const float sc = amax > 0.f ? __fdiv_rn(amax, 448.0f) : 0.f;
   const float inv = amax > 0.f ? __fdiv_rn(448.0f, amax) : 0.f;
-  uint8_t* dp = dst + (size_t)r * cols + half * 64;
+  uint8_t* dp = TRANSPOSE ? &tile[r][half * 64] : dst + (size_t)r * cols + half * 64;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     uint32_t wds[4];
@@ -750,7 +755,28 @@ __global__ void __launch_bounds__(256) k_quant_w(const __nv_bfloat16* __restrict
     }
     *reinterpret_cast<uint4*>(dp + i * 16) = make_uint4(wds[0], wds[1], wds[2], wds[3]);
   }
-  if (threadIdx.x == 0) scale[(size_t)mat * br * bc + bi * bc + bj] = sc;
+  if (TRANSPOSE) {
+    // block (bi, bj) of the codes becomes block (bj, bi) of the transpose:
+    // thread (c, half) writes 64 bytes of output row c, read down a column
+    __syncthreads();
+    const int c = threadIdx.x >> 1;
+    uint8_t* tp = q + (size_t)mat * rows * cols + ((size_t)bj * 128 + c) * rows + bi * 128 +
+                  half * 64;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      uint32_t wds[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int r0 = half * 64 + i * 16 + j * 4;
+        wds[j] = (uint32_t)tile[r0][c] | ((uint32_t)tile[r0 + 1][c] << 8) |
+                 ((uint32_t)tile[r0 + 2][c] << 16) | ((uint32_t)tile[r0 + 3][c] << 24);
+      }
+      *reinterpret_cast<uint4*>(tp + i * 16) = make_uint4(wds[0], wds[1], wds[2], wds[3]);
+    }
+    if (threadIdx.x == 0) scale[(size_t)mat * br * bc + bj * br + bi] = sc;
+  } else {
+    if (threadIdx.x == 0) scale[(size_t)mat * br * bc + bi * bc + bj] = sc;
+  }
 }
 
 }  // namespace perm

@@ -245,14 +245,7 @@ def case_backward_fp8():
     desc = moe.desc_from_config(cfg)
     E, I, d, N = cfg.n_experts, cfg.inter, cfg.d, cfg.n_routed
 
-    def quant(w, r, c):
-        q = torch.empty(E, r, c, dtype=torch.uint8, device="cuda")
-        sc = torch.empty(E, r // 128, c // 128, dtype=torch.float32, device="cuda")
-        moe.moe_quantize_fp8_blockwise(w.contiguous(), r, c, E, q, sc)
-        return q, sc
-
-    W = (quant(inp["w_gu"], 2 * I, d) + quant(inp["w_gu"].transpose(1, 2), d, 2 * I)
-         + quant(inp["w_down"], d, I) + quant(inp["w_down"].transpose(1, 2), I, d))
+    W = moe.fp8_backward_weights(inp["w_gu"], inp["w_down"])
     ws = moe.backward_fp8_workspace(desc)
     bf = dict(dtype=torch.bfloat16, device="cuda")
     dx = torch.empty_like(dh)

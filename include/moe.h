@@ -444,7 +444,8 @@ moe_status moe_backward_saved(const moe_layer_desc* desc, const void* x, const v
  * column, the expert's rows taken in token order and padded with zero rows to
  * a multiple of 128 (a shared expert's rows are all T tokens).
  * Weights: the forward's E4M3 codes and 128x128 block scales
- * (moe_quantize_fp8_blockwise) and the same for the transposed matrices,
+ * (moe_quantize_fp8_blockwise) and the same for the transposed matrices
+ * (moe_quantize_fp8_blockwise_t),
  *   w_gu [E, 2I, d] + w_gu_scale [E, 2I/128, d/128],
  *   w_gu_t [E, d, 2I] + w_gu_t_scale [E, d/128, 2I/128],
  *   w_down [E, d, I] + w_down_scale [E, d/128, I/128],
@@ -479,6 +480,15 @@ int32_t moe_backward_launch_count(const moe_layer_desc* desc);
 moe_status moe_quantize_fp8_blockwise(const void* w_bf16, int32_t rows, int32_t cols,
                                       int32_t batch, void* w_e4m3, float* scale,
                                       cudaStream_t stream);
+
+/* moe_quantize_fp8_blockwise of the transposed matrices, without forming
+ * them: w_e4m3_t [batch, cols, rows] codes and scale_t [batch, cols/128,
+ * rows/128] (the transposed layout of the same codes and scales, a 128x128
+ * block's amax being the same either way).  The transposed weights of
+ * moe_backward_fp8.  Same arguments and errors otherwise. */
+moe_status moe_quantize_fp8_blockwise_t(const void* w_bf16, int32_t rows, int32_t cols,
+                                        int32_t batch, void* w_e4m3_t, float* scale_t,
+                                        cudaStream_t stream);
 
 /* Human-readable name of a status. */
 const char* moe_status_string(moe_status status);

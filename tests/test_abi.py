@@ -285,3 +285,11 @@ def test_fp8_backward_entry_point_rejects_bad_arguments():
     bad[4] = 18                           # a scale (w_gu_scale) not 4-byte aligned
     assert L.moe_backward_fp8(ctypes.byref(f8), *bad, 16, 1 << 40, None) == moe.ERR_INVALID_ARG
     assert L.moe_backward_fp8(ctypes.byref(f8), *ptrs, 16, 1024, None) == moe.ERR_WORKSPACE
+
+
+def test_transposed_weight_quantisation_rejects_bad_arguments():
+    L = moe.lib()
+    assert L.moe_quantize_fp8_blockwise_t(16, 100, 128, 1, 16, 16, None) == moe.ERR_INVALID_ARG
+    assert L.moe_quantize_fp8_blockwise_t(16, 128, 128, 0, 16, 16, None) == moe.ERR_INVALID_ARG
+    assert L.moe_quantize_fp8_blockwise_t(16, 128, 128, 1, 24, 16, None) == moe.ERR_INVALID_ARG
+    assert L.moe_quantize_fp8_blockwise_t(None, 128, 128, 1, 16, 16, None) == moe.ERR_INVALID_ARG

@@ -4,8 +4,9 @@ tests/test_oracle_fp8_backward.py) and against the exact fp64 backward.
 
 Both sides use the same E4M3 weights: the GPU's moe_quantize_fp8_blockwise
 codes and scales equal the oracle's 128x128 quantisation bit for bit (checked
-in tests/test_gpu_fp8.py; the transposed matrices are checked here), and the
-GPU's selection (no gradient flows through the choice of experts).
+in tests/test_gpu_fp8.py; moe_quantize_fp8_blockwise_t's transposed codes and
+scales are checked here against the transposes of those), and the GPU's
+selection (no gradient flows through the choice of experts).
 
 Bounds, every gradient as a whole tensor (max-abs-relative):
   * 2e-2 (the bf16 layer's bound) of the emulation with bf16 intermediates,
@@ -77,20 +78,8 @@ class Fp8Host(HostLayer):
         return self._experts[e]
 
 
-def quantize(w, rows, cols, E):
-    q = torch.empty(E, rows, cols, dtype=torch.uint8, device="cuda")
-    s = torch.empty(E, rows // 128, cols // 128, dtype=torch.float32, device="cuda")
-    moe.moe_quantize_fp8_blockwise(w.contiguous(), rows, cols, E, q, s)
-    return q, s
-
-
 def fp8_weights(cfg, inp):
-    E, I, d = cfg.n_experts, cfg.inter, cfg.d
-    gq, gs = quantize(inp["w_gu"], 2 * I, d, E)
-    gtq, gts = quantize(inp["w_gu"].transpose(1, 2), d, 2 * I, E)
-    dq, ds = quantize(inp["w_down"], d, I, E)
-    dtq, dts = quantize(inp["w_down"].transpose(1, 2), I, d, E)
-    return gq, gs, gtq, gts, dq, ds, dtq, dts
+    return moe.fp8_backward_weights(inp["w_gu"], inp["w_down"])
 
 
 def upstream(cfg):
@@ -140,9 +129,10 @@ def test_fp8_backward_parity(name):
     moe.moe_last_device_status()
     inp = recipes.device_inputs(cfg)
     W = fp8_weights(cfg, inp)
-    # the transposed quantisation is the transpose of the codes and scales
-    assert torch.equal(W[2][0], W[0][0].t()) and torch.equal(W[3][0], W[1][0].t())
-    assert torch.equal(W[6][-1], W[4][-1].t()) and torch.equal(W[7][-1], W[5][-1].t())
+    # moe_quantize_fp8_blockwise_t gives the transposes of the codes and scales
+    for e in (0, cfg.n_experts - 1):
+        assert torch.equal(W[2][e], W[0][e].t()) and torch.equal(W[3][e], W[1][e].t())
+        assert torch.equal(W[6][e], W[4][e].t()) and torch.equal(W[7][e], W[5][e].t())
     dh, dh64 = upstream(cfg)
     dx, dwr, dwgu, dwd, st = run(cfg, inp, W, dh)
     assert st == moe.OK, moe.moe_status_string(st)

@@ -130,7 +130,7 @@ constexpr int XOUT_BYTES = (NUM_EPI / 32) * 32 * (WG_BN / 4) * 2;
 __host__ inline size_t smem_bytes(int stages, int n_groups, bool wg = false) {
   return 1024 + (size_t)stages * (BM * KB + (wg ? WG_BN : BN) * KB) +
          (wg ? (size_t)XOUT_BYTES : 0) +
-         (size_t)(2 * stages + 6) * 8 + 16 + 2 * 4 * BM * sizeof(float) +
+         (size_t)(2 * stages + 10) * 8 + 16 + 2 * 4 * BM * sizeof(float) +
          SB_FLOATS * sizeof(float) + (size_t)(n_groups + 1) * 4 + (wg ? (size_t)n_groups * 16 : 0) +
          64;
 }
@@ -334,6 +334,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   constexpr int TBN = WG ? WG_BN : BN;     // accumulator columns of a tile
+  // TMEM partials in flight: two of 256 columns, or four of 128 in the
+  // weight-gradient mode, so its MMA runs further ahead of the promotion
+  constexpr int NP = TMEM_COLS / TBN;
   constexpr int WC = TBN / 4;              // columns of one epilogue warp
   constexpr uint32_t a_bytes = BM * KB;
   constexpr uint32_t b_bytes = TBN * KB;
@@ -343,8 +346,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint64_t* full = reinterpret_cast<uint64_t*>(xout + (WG ? XOUT_BYTES : 0));
   uint64_t* empty = full + S;
   uint64_t* pfull = empty + S;
-  uint64_t* pempty = pfull + 2;
-  uint64_t* xbar = pempty + 2;       // amax exchange between the epilogue warps
+  uint64_t* pempty = pfull + NP;
+  uint64_t* xbar = pempty + NP;      // amax exchange between the epilogue warps
   uint64_t* drain = xbar + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -372,7 +375,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    for (int j = 0; j < 2; ++j) {
+    for (int j = 0; j < NP; ++j) {
       mbar_init(&pfull[j], 1);
       mbar_init(&pempty[j], NUM_EPI / 32);
     }
@@ -453,8 +456,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           for (int kb = 0; kb < nkb; ++kb, ++it, ++pu) {
             const int s = it % S;
             const uint32_t ph = (uint32_t)(it / S) & 1u;
-            const int p = pu & 1;
-            const uint32_t pph = (uint32_t)(pu >> 1) & 1u;
+            const int p = pu % NP;
+            const uint32_t pph = (uint32_t)(pu / NP) & 1u;
             if (!mbar_wait(&full[s], ph, abort_flag)) { ok = false; break; }
             if (!mbar_wait(&pempty[p], pph ^ 1u, abort_flag)) { ok = false; break; }
             tc_fence_after();
@@ -510,8 +513,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const float sa_k = arow < a.a_rows ? a.a_scale[kr * a.a_scale_ld + arow] : 0.f;
           sbw[lane] = ncol + lane < a.b_rows ? a.b_scale[kr * a.b_scale_ld + ncol + lane] : 0.f;
           __syncwarp();
-          const int p = pu & 1;
-          if (!mbar_wait(&pfull[p], (uint32_t)(pu >> 1) & 1u, abort_flag)) { ok = false; break; }
+          const int p = pu % NP;
+          if (!mbar_wait(&pfull[p], (uint32_t)(pu / NP) & 1u, abort_flag)) { ok = false; break; }
           tc_fence_after();
           promote_cols<WC>(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(p * TBN + col0),
                            acc, sa_k, sbw);
@@ -589,8 +592,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             nb0 = sb0[kb + 1];
             nb1 = sb1[kb + 1];
           }
-          const int p = pu & 1;
-          if (!mbar_wait(&pfull[p], (uint32_t)(pu >> 1) & 1u, abort_flag)) { ok = false; break; }
+          const int p = pu % NP;
+          if (!mbar_wait(&pfull[p], (uint32_t)(pu / NP) & 1u, abort_flag)) { ok = false; break; }
           tc_fence_after();
           const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(p * TBN + col0);
           // the router's unscaled promotion is a paired FMA with multiplier 1

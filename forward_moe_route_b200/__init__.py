@@ -109,7 +109,7 @@ _SIGS = {
     "moe_ipc_open": (ctypes.c_int, [_P, ctypes.POINTER(ctypes.c_void_p)]),
     "moe_ipc_close": (ctypes.c_int, [_P]),
     "moe_backward_fp8_workspace_size": (ctypes.c_size_t, [_D]),
-    "moe_backward_fp8": (ctypes.c_int, [_D] + [_P] * 17 + [ctypes.c_size_t, _P]),
+    "moe_backward_fp8": (ctypes.c_int, [_D] + [_P] * 15 + [ctypes.c_size_t, _P]),
     "moe_backward_fp8_launch_count": (ctypes.c_int32, [_D]),
     "moe_saved_ab_bytes": (ctypes.c_size_t, [_D]),
     "moe_forward_save": (ctypes.c_int, [_D, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
@@ -334,21 +334,21 @@ def moe_quantize_fp8_blockwise_t(w_bf16, rows: int, cols: int, batch: int, w_e4m
 
 
 def fp8_backward_weights(w_gu, w_down, stream=None):
-    """E4M3 codes and 128x128 block scales of a layer's bf16 expert weights
-    w_gu [E, 2I, d] and w_down [E, d, I] and of their transposes, in the
-    argument order of moe_backward_fp8: (w_gu, w_gu_scale, w_gu_t,
-    w_gu_t_scale, w_down, w_down_scale, w_down_t, w_down_t_scale)."""
+    """The E4M3 weights moe_backward_fp8 takes, from a layer's bf16 expert
+    weights w_gu [E, 2I, d] and w_down [E, d, I], in its argument order:
+    (w_gu, w_gu_scale, w_gu_t, w_gu_t_scale, w_down_t, w_down_t_scale)."""
     import torch
     E, two_i, d = w_gu.shape
     I = w_down.shape[2]
     out = []
-    for w, rows, cols in ((w_gu, two_i, d), (w_down, d, I)):
-        for quant, (r, c) in ((moe_quantize_fp8_blockwise, (rows, cols)),
-                              (moe_quantize_fp8_blockwise_t, (cols, rows))):
-            q = torch.empty(E, r, c, dtype=torch.uint8, device=w.device)
-            sc = torch.empty(E, r // 128, c // 128, dtype=torch.float32, device=w.device)
-            quant(w, rows, cols, E, q, sc, stream)
-            out += [q, sc]
+    for quant, w, rows, cols in ((moe_quantize_fp8_blockwise, w_gu, two_i, d),
+                                 (moe_quantize_fp8_blockwise_t, w_gu, two_i, d),
+                                 (moe_quantize_fp8_blockwise_t, w_down, d, I)):
+        r, c = (rows, cols) if quant is moe_quantize_fp8_blockwise else (cols, rows)
+        q = torch.empty(E, r, c, dtype=torch.uint8, device=w.device)
+        sc = torch.empty(E, r // 128, c // 128, dtype=torch.float32, device=w.device)
+        quant(w, rows, cols, E, q, sc, stream)
+        out += [q, sc]
     return tuple(out)
 
 
@@ -456,14 +456,12 @@ def backward_fp8_workspace(desc: MoeLayerDesc, device="cuda"):
     return torch.empty(n, dtype=torch.uint8, device=device)
 
 
-def moe_backward_fp8(desc, x, w_router, bias, w_gu, w_gu_scale, w_gu_t, w_gu_t_scale, w_down,
-                     w_down_scale, w_down_t, w_down_t_scale, dh, dx, dw_router, dw_gu, dw_down,
-                     ws, stream=None) -> None:
+def moe_backward_fp8(desc, x, w_router, bias, w_gu, w_gu_scale, w_gu_t, w_gu_t_scale, w_down_t,
+                     w_down_t_scale, dh, dx, dw_router, dw_gu, dw_down, ws, stream=None) -> None:
     """The backward of an E4M3 layer with FP8 GEMMs; bf16 weight gradients."""
     _need("moe_backward_fp8", desc, x=x, w_router=w_router, bias=bias, w_gu=w_gu,
-          w_gu_scale=w_gu_scale, w_gu_t=w_gu_t, w_gu_t_scale=w_gu_t_scale, w_down=w_down,
-          w_down_scale=w_down_scale, w_down_t=w_down_t, w_down_t_scale=w_down_t_scale, dh=dh,
-          dx=dx)
+          w_gu_scale=w_gu_scale, w_gu_t=w_gu_t, w_gu_t_scale=w_gu_t_scale, w_down_t=w_down_t,
+          w_down_t_scale=w_down_t_scale, dh=dh, dx=dx)
     sz = _sizes(desc)
     for name, t in (("dw_router", dw_router), ("dw_gu", dw_gu), ("dw_down", dw_down)):
         if t is None:
@@ -473,8 +471,8 @@ def moe_backward_fp8(desc, x, w_router, bias, w_gu, w_gu_scale, w_gu_t, w_gu_t_s
                            "bf16 tensor of the gradient's shape")
     _check(_lib.moe_backward_fp8(ctypes.byref(desc), _ptr(x), _ptr(w_router), _ptr(bias),
                                  _ptr(w_gu), _ptr(w_gu_scale), _ptr(w_gu_t), _ptr(w_gu_t_scale),
-                                 _ptr(w_down), _ptr(w_down_scale), _ptr(w_down_t),
-                                 _ptr(w_down_t_scale), _ptr(dh), _ptr(dx), _ptr(dw_router),
+                                 _ptr(w_down_t), _ptr(w_down_t_scale), _ptr(dh), _ptr(dx),
+                                 _ptr(dw_router),
                                  _ptr(dw_gu), _ptr(dw_down), _ptr(ws),
                                  ws.numel() if ws is not None else 0, _stream(stream)),
            "moe_backward_fp8")

@@ -1255,8 +1255,8 @@ Bwd8Layout bwd8_layout(const Dims& D, const Layout& L) {
 }
 
 struct Fp8Weights {
-  const void *gu, *gu_t, *down, *down_t;
-  const float *gu_s, *gu_t_s, *down_s, *down_t_s;
+  const void *gu, *gu_t, *down_t;
+  const float *gu_s, *gu_t_s, *down_t_s;
 };
 
 moe_status do_backward_fp8(const moe_layer_desc& s, const Dims& D, const Layout& L,
@@ -2006,8 +2006,7 @@ size_t moe_backward_fp8_workspace_size(const moe_layer_desc* desc) {
 
 moe_status moe_backward_fp8(const moe_layer_desc* desc, const void* x, const void* w_router,
                             const float* bias, const void* w_gu, const float* w_gu_scale,
-                            const void* w_gu_t, const float* w_gu_t_scale, const void* w_down,
-                            const float* w_down_scale, const void* w_down_t,
+                            const void* w_gu_t, const float* w_gu_t_scale, const void* w_down_t,
                             const float* w_down_t_scale, const void* dh, void* dx,
                             void* dw_router, void* dw_gu, void* dw_down, void* ws,
                             size_t ws_bytes, cudaStream_t stream) {
@@ -2018,11 +2017,10 @@ moe_status moe_backward_fp8(const moe_layer_desc* desc, const void* x, const voi
   if (bias && desc->gate != MOE_GATE_SIGMOID) return MOE_ERR_INVALID_ARG;
   if (D.E > 1024 || D.K + D.Ks > 32 || D.d % 256 || (D.N * 2) % 16) return MOE_ERR_UNSUPPORTED;
   if (D.T > 0) {
-    const void* need[] = {x, w_router, w_gu, w_gu_t, w_down, w_down_t, dh, dx, dw_router, dw_gu,
-                          dw_down};
+    const void* need[] = {x, w_router, w_gu, w_gu_t, w_down_t, dh, dx, dw_router, dw_gu, dw_down};
     for (const void* p : need)
       if (!p || !aligned16(p)) return MOE_ERR_INVALID_ARG;
-    const float* scales[] = {w_gu_scale, w_gu_t_scale, w_down_scale, w_down_t_scale};
+    const float* scales[] = {w_gu_scale, w_gu_t_scale, w_down_t_scale};
     for (const float* p : scales)
       if (!p || ((uintptr_t)p & 3u)) return MOE_ERR_INVALID_ARG;
     if (bias && !aligned16(bias)) return MOE_ERR_INVALID_ARG;
@@ -2034,8 +2032,7 @@ moe_status moe_backward_fp8(const moe_layer_desc* desc, const void* x, const voi
   if (D.T == 0) return MOE_OK;
   int sms;
   if ((rc = device_setup(&sms)) != MOE_OK) return rc;
-  const Fp8Weights W{w_gu, w_gu_t, w_down, w_down_t, w_gu_scale, w_gu_t_scale, w_down_scale,
-                     w_down_t_scale};
+  const Fp8Weights W{w_gu, w_gu_t, w_down_t, w_gu_scale, w_gu_t_scale, w_down_t_scale};
   return do_backward_fp8(*desc, D, L, B, x, w_router, bias, W, dh, dx, dw_router, dw_gu, dw_down,
                          static_cast<uint8_t*>(ws), sms, stream);
 }

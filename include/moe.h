@@ -443,15 +443,16 @@ moe_status moe_backward_saved(const moe_layer_desc* desc, const void* x, const v
  * [da | db] u^T, which contract over an expert's rows, tiles of 128 rows x 1
  * column, the expert's rows taken in token order and padded with zero rows to
  * a multiple of 128 (a shared expert's rows are all T tokens).
- * Weights: the forward's E4M3 codes and 128x128 block scales
- * (moe_quantize_fp8_blockwise) and the same for the transposed matrices
- * (moe_quantize_fp8_blockwise_t),
+ * Weights: E4M3 codes and 128x128 block scales as the forward's
+ * (moe_quantize_fp8_blockwise), and of the transposed matrices
+ * (moe_quantize_fp8_blockwise_t): every GEMM reads its weight K-major, so
+ * W_gate/W_up serve the recomputed a, b as they are and du transposed, and
+ * W_down serves dz' = W_down^T dh transposed only,
  *   w_gu [E, 2I, d] + w_gu_scale [E, 2I/128, d/128],
  *   w_gu_t [E, d, 2I] + w_gu_t_scale [E, d/128, 2I/128],
- *   w_down [E, d, I] + w_down_scale [E, d/128, I/128],
  *   w_down_t [E, I, d] + w_down_t_scale [E, I/128, d/128]
- * (quantising a transposed bf16 matrix gives the transposed codes and scales,
- * since a block's amax does not depend on its orientation).
+ * (the transposed codes and scales of the forward's, since a block's amax
+ * does not depend on its orientation).
  *   x [T, d] bf16, w_router [N, d] bf16, bias [N] fp32 or NULL, dh [T, d] bf16
  *   dx [T, d] bf16 out; dw_router [N, d], dw_gu [E, 2I, d], dw_down [E, d, I]
  *     bf16 out (zeros for experts no token reaches)
@@ -462,8 +463,7 @@ moe_status moe_backward_saved(const moe_layer_desc* desc, const void* x, const v
 size_t moe_backward_fp8_workspace_size(const moe_layer_desc* desc);
 moe_status moe_backward_fp8(const moe_layer_desc* desc, const void* x, const void* w_router,
                             const float* bias, const void* w_gu, const float* w_gu_scale,
-                            const void* w_gu_t, const float* w_gu_t_scale, const void* w_down,
-                            const float* w_down_scale, const void* w_down_t,
+                            const void* w_gu_t, const float* w_gu_t_scale, const void* w_down_t,
                             const float* w_down_t_scale, const void* dh, void* dx,
                             void* dw_router, void* dw_gu, void* dw_down, void* ws,
                             size_t ws_bytes, cudaStream_t stream);

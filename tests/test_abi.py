@@ -267,13 +267,13 @@ def test_fp8_backward_entry_point_rejects_bad_arguments():
     assert moe.moe_backward_fp8_workspace_size(v3(T=64)) == 0
     assert moe.moe_backward_fp8_launch_count(f8) == 22
     assert moe.moe_backward_fp8_launch_count(v3(T=0, dtype="e4m3")) == 0
-    ptrs = [16] * 16          # x, w_router, bias, 8 weight pointers, dh, dx, 3 gradients
+    ptrs = [16] * 14          # x, w_router, bias, 6 weight pointers, dh, dx, 3 gradients
     ptrs[2] = None            # bias
     assert L.moe_backward_fp8(ctypes.byref(v3(T=64)), *ptrs, 16, 1 << 40,
                               None) == moe.ERR_UNSUPPORTED
     assert L.moe_backward_fp8(ctypes.byref(v3(T=64, d=7168 + 128, dtype="e4m3")), *ptrs, 16,
                               1 << 40, None) == moe.ERR_UNSUPPORTED
-    for i in (0, 3, 5, 11, 15):           # a missing tensor or scale
+    for i in (0, 3, 5, 8, 9, 13):         # a missing tensor or scale
         bad = list(ptrs)
         bad[i] = None
         assert L.moe_backward_fp8(ctypes.byref(f8), *bad, 16, 1 << 40,

@@ -97,9 +97,7 @@ def run(cfg, inp, W, dh):
     dwr = torch.full((N, d), float("nan"), **bf)
     dwgu = torch.full((E, 2 * I, d), float("nan"), **bf)
     dwd = torch.full((E, d, I), float("nan"), **bf)
-    gq, gs, gtq, gts, dq, ds, dtq, dts = W
-    moe.moe_backward_fp8(desc, inp["x"], inp["w_r"], inp["bias"], gq, gs, gtq, gts, dq, ds, dtq,
-                         dts, dh, dx, dwr, dwgu, dwd, ws)
+    moe.moe_backward_fp8(desc, inp["x"], inp["w_r"], inp["bias"], *W, dh, dx, dwr, dwgu, dwd, ws)
     return dx, dwr, dwgu, dwd, moe.moe_last_device_status()
 
 
@@ -130,9 +128,13 @@ def test_fp8_backward_parity(name):
     inp = recipes.device_inputs(cfg)
     W = fp8_weights(cfg, inp)
     # moe_quantize_fp8_blockwise_t gives the transposes of the codes and scales
+    E, I, d = cfg.n_experts, cfg.inter, cfg.d
+    dq = torch.empty(E, d, I, dtype=torch.uint8, device="cuda")
+    ds = torch.empty(E, d // 128, I // 128, dtype=torch.float32, device="cuda")
+    moe.moe_quantize_fp8_blockwise(inp["w_down"], d, I, E, dq, ds)
     for e in (0, cfg.n_experts - 1):
         assert torch.equal(W[2][e], W[0][e].t()) and torch.equal(W[3][e], W[1][e].t())
-        assert torch.equal(W[6][e], W[4][e].t()) and torch.equal(W[7][e], W[5][e].t())
+        assert torch.equal(W[4][e], dq[e].t()) and torch.equal(W[5][e], ds[e].t())
     dh, dh64 = upstream(cfg)
     dx, dwr, dwgu, dwd, st = run(cfg, inp, W, dh)
     assert st == moe.OK, moe.moe_status_string(st)

@@ -130,7 +130,7 @@ constexpr int XOUT_BYTES = (NUM_EPI / 32) * 32 * (WG_BN / 4) * 2;
 __host__ inline size_t smem_bytes(int stages, int n_groups, bool wg = false) {
   return 1024 + (size_t)stages * (BM * KB + (wg ? WG_BN : BN) * KB) +
          (wg ? (size_t)XOUT_BYTES : 0) +
-         (size_t)(2 * stages + 10) * 8 + 16 + 2 * 4 * BM * sizeof(float) +
+         (size_t)(2 * stages + 14) * 8 + 16 + 2 * 4 * BM * sizeof(float) +
          SB_FLOATS * sizeof(float) + (size_t)(n_groups + 1) * 4 + (wg ? (size_t)n_groups * 16 : 0) +
          64;
 }
@@ -347,12 +347,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint64_t* empty = full + S;
   uint64_t* pfull = empty + S;
   uint64_t* pempty = pfull + NP;
-  uint64_t* xbar = pempty + NP;      // amax exchange between the epilogue warps
+  uint64_t* sfull = pempty + NP;     // WG: a partial slot's scales are in shared memory
+  uint64_t* xbar = sfull + NP;       // amax exchange between the epilogue warps
   uint64_t* drain = xbar + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* amax_buf = reinterpret_cast<float*>(tmem_slot + 4);   // [2][4][128]
-  float* sb_buf = amax_buf + 2 * 4 * BM;                        // WG: [16 warps][64]
+  float* sb_buf = amax_buf + 2 * 4 * BM;   // WG: NP slots of BM row + TBN column scales
   int* s_prefix = reinterpret_cast<int*>(sb_buf + SB_FLOATS);
   int* s_kgroup = s_prefix + a.gt.count() + 1;                  // WG: the groups' K ranges
 
@@ -378,6 +379,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     for (int j = 0; j < NP; ++j) {
       mbar_init(&pfull[j], 1);
       mbar_init(&pempty[j], NUM_EPI / 32);
+      mbar_init(&sfull[j], 1);
     }
     mbar_init(xbar, NUM_EPI);
     mbar_init(drain, 1);
@@ -479,6 +481,45 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         mbar_wait(drain, 0, &no_abort);
       }
       __syncwarp();
+    } else if (WG && warp == 2) {
+      // ------------------------------------------------------------------ scale loader (WG)
+      // the row and column scales of every (tile, k-block) into the shared
+      // slot of its TMEM partial, up to NP k-blocks ahead of the promotion
+      // (a slot is refilled once the promotion of its partial has released it)
+      int pu = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
+        const int mt = tile / a.n_tiles_n, nt = tile - mt * a.n_tiles_n;
+        const int g = gemm::find_group(s_prefix, n_groups, mt);
+        const int* kg = s_kgroup + 4 * g;
+        const int m0 = (mt - s_prefix[g]) * BM, n0 = nt * TBN;
+        for (int kb = 0; kb < kg[1]; ++kb, ++pu) {
+          const int p = pu % NP;
+          if (!mbar_wait(&pempty[p], ((uint32_t)(pu / NP) & 1u) ^ 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          const size_t kr = (size_t)(kg[0] / 128 + kb);
+          float* slot = sb_buf + p * (BM + TBN);
+          // all eight loads in flight before the first store
+          float v[(BM + TBN) / 32];
+#pragma unroll
+          for (int j = 0; j < BM / 32; ++j) {
+            const int i = 32 * j + lane;
+            v[j] = m0 + i < a.a_rows ? a.a_scale[kr * a.a_scale_ld + m0 + i] : 0.f;
+          }
+#pragma unroll
+          for (int j = 0; j < TBN / 32; ++j) {
+            const int i = 32 * j + lane;
+            v[BM / 32 + j] = n0 + i < a.b_rows ? a.b_scale[kr * a.b_scale_ld + n0 + i] : 0.f;
+          }
+#pragma unroll
+          for (int j = 0; j < (BM + TBN) / 32; ++j) slot[32 * j + lane] = v[j];
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sfull[p]);
+        }
+      }
+      __syncwarp();
     }
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(EPI_REGS));
@@ -493,8 +534,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     bool ok = true;
     if constexpr (WG) {
       // Weight gradients: short K ranges (an expert's rows), 128 x 128 tiles;
-      // group data comes from shared memory.
-      float* sbw = sb_buf + ew * 64;
+      // group data and the scales (staged by the scale-loader warp) come from
+      // shared memory.
       for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x, ++tcount) {
         const int mt = tile / a.n_tiles_n, nt = tile - mt * a.n_tiles_n;
         const int g = gemm::find_group(s_prefix, n_groups, mt);
@@ -502,22 +543,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int* kg = s_kgroup + 4 * g;           // k0, k-blocks, c_row, rows
         const int nkb = kg[1];
         const int ncol = nt * TBN + col0;
-        const int arow = lm * BM + r;
         float acc[WC];
 #pragma unroll
         for (int i = 0; i < WC; ++i) acc[i] = 0.f;
         for (int kb = 0; kb < nkb; ++kb, ++pu) {
-          // this k-block's row scale and the slice's column scales, loaded
-          // while the tensor cores compute the partial
-          const size_t kr = (size_t)(kg[0] / 128 + kb);
-          const float sa_k = arow < a.a_rows ? a.a_scale[kr * a.a_scale_ld + arow] : 0.f;
-          sbw[lane] = ncol + lane < a.b_rows ? a.b_scale[kr * a.b_scale_ld + ncol + lane] : 0.f;
-          __syncwarp();
           const int p = pu % NP;
-          if (!mbar_wait(&pfull[p], (uint32_t)(pu / NP) & 1u, abort_flag)) { ok = false; break; }
+          const uint32_t par = (uint32_t)(pu / NP) & 1u;
+          if (!mbar_wait(&sfull[p], par, abort_flag)) { ok = false; break; }
+          const float* slot = sb_buf + p * (BM + TBN);
+          const float sa_k = slot[r];
+          if (!mbar_wait(&pfull[p], par, abort_flag)) { ok = false; break; }
           tc_fence_after();
           promote_cols<WC>(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(p * TBN + col0),
-                           acc, sa_k, sbw);
+                           acc, sa_k, slot + BM + col0);
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&pempty[p]);
